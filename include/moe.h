@@ -1,0 +1,176 @@
+/*
+ * moe.h -- C ABI of libmoe.so: one sparse-MoE layer with GPU-resident expert
+ * routing and affine 4-bit experts, on one NVIDIA B200 (sm_100a).
+ *
+ * The layer is the Qwen3.6-35B-A3B MoE block that the Lily write-ups single
+ * out ("Perplexity's Lily: A Breakthrough Local Inference Engine Tailored
+ * Exclusively for Apple Silicon", section "The Model: Qwen3.6-35B-A3B in
+ * Focus"; "Perplexity Open Sources Apple Chip Inference Engine Lily",
+ * paragraphs 3 and 5): a router scores E experts and keeps k of them per
+ * token, one always-on shared expert sees every token, and every expert
+ * weight is MLX affine 4-bit with one bf16 scale and one bf16 bias per group
+ * of 64 weights along the input dimension.  The same write-ups ("How It
+ * Works: Prefill and Decode Strategies") keep the routing histogram, prefix
+ * scan and scatter on the GPU with no CPU synchronisation, and rebuild the
+ * 4-bit weights tile by tile inside the grouped expert GEMM.
+ *
+ * What one call computes, for tokens t = 0..T-1 (x, out: bf16 [T, H]):
+ *   l[t,e]   = x_t . W_r[e] (+ router_bias[e])                    (FP32)
+ *   idx[t,:] = the k experts with the largest l[t,e]; equal logits go to
+ *              the lower expert index; slot order = (logit desc, index asc)
+ *   w[t,j]   = exp(l[t,idx_j] - l[t,idx_0]) / sum_j' exp(...)    (softmax
+ *              over all experts renormalised over the k chosen ones)
+ *   expert e on row x:  h = bf16(silu(x W_g[e]^T) * (x W_u[e]^T)),
+ *                       y = h W_d[e]^T,  silu(z) = z / (1 + exp(-z))
+ *   sigma_t  = 1 / (1 + exp(-x_t . w_sg))
+ *   out_t    = bf16( sum_{j=0..k-1} w[t,j] * y_{t,idx_j}  +  sigma_t * ys_t )
+ *              summed in FP32 in exactly that order (ys = shared expert).
+ * Weights are used as w = scale * q + bias per group of 64 (q in 0..15).
+ *
+ * Storage.
+ *   bf16 values are passed as their 16-bit patterns (moe_bf16).
+ *   A q-matrix [R, C] is three row-major device arrays:
+ *     q      uint32 [R, C/8]  -- code i of a word = element 8w+i, bits 4i..4i+3
+ *     scales bf16   [R, C/64]
+ *     biases bf16   [R, C/64]
+ *   Stacked expert matrices add a leading [E] dimension, contiguous.
+ *   All pointers in moe_layer_desc, moe_routing and the x/out/workspace
+ *   arguments of moe_route/moe_forward/moe_decode are DEVICE pointers; only
+ *   moe_forward_host takes host x/out.
+ *
+ * Ownership.  The caller owns every buffer (weights, x, out, routing,
+ * workspace).  The library allocates no device memory and keeps no state
+ * between calls except cached kernel attributes.  Two calls must not share a
+ * workspace concurrently.
+ *
+ * Asynchrony.  moe_route, moe_forward, moe_decode and moe_rmsnorm enqueue
+ * work on `stream` (a cudaStream_t; NULL = the legacy default stream) and
+ * return without waiting for the device.  Their outputs are valid once the
+ * stream reaches that point.  No call reads device data back on the host
+ * except moe_get_status and moe_forward_host.
+ *
+ * Errors.  Every entry point returns a moe_status.  Arguments are validated on
+ * the host before anything is enqueued: a rejected call enqueues nothing.  A
+ * failed kernel launch returns MOE_ERR_CUDA.  Bounded device-side waits that
+ * give up record MOE_ERR_DEVICE_TIMEOUT in the workspace's status word, which
+ * moe_get_status returns.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t moe_bf16;   /* bf16 bit pattern */
+typedef void* moe_stream;    /* a cudaStream_t */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = -1,     /* NULL pointer, T out of range, misaligned pointer */
+  MOE_ERR_UNSUPPORTED = -2,     /* layout other than affine 4-bit / group 64, sizes not supported */
+  MOE_ERR_WORKSPACE = -3,       /* workspace NULL, too small, or misaligned */
+  MOE_ERR_CUDA = -4,            /* a CUDA runtime call or kernel launch failed */
+  MOE_ERR_DEVICE_TIMEOUT = -5   /* a bounded device-side wait gave up */
+} moe_status;
+
+/* One affine 4-bit matrix (or a stack of E of them); see "Storage" above. */
+typedef struct {
+  const uint32_t* q;
+  const moe_bf16* scales;
+  const moe_bf16* biases;
+} moe_qmat;
+
+/* One MoE layer.  Accepted layout (anything else is MOE_ERR_UNSUPPORTED, as
+ * the Lily loader refuses every layout but the one it was built for --
+ * "Perplexity Open Sources Apple Chip Inference Engine Lily", paragraph 3):
+ *   bits == 4, group_size == 64, renorm == 1,
+ *   1 <= k <= 8, k <= E <= 256,
+ *   H a multiple of 128 and <= 8192; I and I_shared multiples of 128 and <= 2048. */
+typedef struct {
+  int H;            /* hidden size */
+  int I;            /* routed expert intermediate size */
+  int I_shared;     /* shared expert intermediate size */
+  int E;            /* number of routed experts */
+  int k;            /* experts chosen per token */
+  int group_size;   /* must be 64 */
+  int bits;         /* must be 4 */
+  int renorm;       /* must be 1: weights renormalised over the chosen experts */
+  const moe_bf16* w_router;       /* [E, H] */
+  const float*    router_bias;    /* [E] or NULL; added to the logits before selection */
+  moe_qmat gate;                  /* [E, I, H] */
+  moe_qmat up;                    /* [E, I, H] */
+  moe_qmat down;                  /* [E, H, I] */
+  moe_qmat sh_gate;               /* [I_shared, H] */
+  moe_qmat sh_up;                 /* [I_shared, H] */
+  moe_qmat sh_down;               /* [H, I_shared] */
+  const moe_bf16* w_shared_gate;  /* [H]; sigma_t = sigmoid(x_t . w_shared_gate) */
+} moe_layer_desc;
+
+/* Routing results (device buffers owned by the caller).
+ *   topk_idx[t*k + j], topk_w[t*k + j]: chosen expert and weight of slot j;
+ *   counts[e]: rows routed to expert e;  offsets[0..E]: exclusive prefix sum;
+ *   perm[pos] = t*k + j, grouped by expert ascending, tokens ascending within
+ *   an expert (stable counting sort);  inv_perm[t*k + j] = pos;
+ *   sigma[t]: shared-expert gate (may be NULL). */
+typedef struct {
+  int32_t* topk_idx;   /* [T*k] */
+  float*   topk_w;     /* [T*k] */
+  int32_t* counts;     /* [E] */
+  int32_t* offsets;    /* [E+1] */
+  int32_t* perm;       /* [T*k] */
+  int32_t* inv_perm;   /* [T*k] */
+  float*   sigma;      /* [T] or NULL */
+} moe_routing;
+
+/* Bytes of device workspace that moe_route / moe_forward / moe_decode /
+ * moe_forward_host need for any T <= T_max.  Returns MOE_ERR_UNSUPPORTED or
+ * MOE_ERR_INVALID_ARG for a layer or T_max the other calls would reject. */
+int moe_workspace_size(const moe_layer_desc* layer, int T_max, size_t* bytes);
+
+/* Router logits, softmax top-k with renormalisation, shared gate, and the
+ * on-device expert histogram, prefix sum and permutation ("Perplexity's
+ * Lily: ...", section "How It Works: Prefill and Decode Strategies").
+ * x: device bf16 [T, H], 16-byte aligned.  r: required.  1 <= T <= 65536. */
+int moe_route(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_routing* r,
+              void* workspace, size_t workspace_bytes, moe_stream stream);
+
+/* The whole layer: routing, fused-dequant gate/up grouped GEMM with the
+ * SwiGLU epilogue, down-projection grouped GEMM, shared expert, and the
+ * fixed-order gather-combine.  x, out: device bf16 [T, H], 16-byte aligned,
+ * not overlapping.  r: optional (NULL = keep routing in the workspace).
+ * 1 <= T <= 65536; T <= 64 runs the decode kernels of moe_decode. */
+int moe_forward(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_bf16* out,
+                moe_routing* r, void* workspace, size_t workspace_bytes, moe_stream stream);
+
+/* The same function for 1 <= T <= 64 through the bandwidth-bound decode
+ * kernels (batch-1 decoding streams the active experts' weights: "How It
+ * Works: Prefill and Decode Strategies").  T > 64 is MOE_ERR_INVALID_ARG. */
+int moe_decode(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_bf16* out,
+               moe_routing* r, void* workspace, size_t workspace_bytes, moe_stream stream);
+
+/* moe_forward with x and out in HOST memory (page-locked for full speed):
+ * copies x to the workspace, runs the layer, copies the result back and waits
+ * for `stream`.  Weights stay device pointers. */
+int moe_forward_host(const moe_layer_desc* layer, const moe_bf16* x_host, int T, moe_bf16* out_host,
+                     void* workspace, size_t workspace_bytes, moe_stream stream);
+
+/* y_out[t] = bf16(y[t] / sqrt(mean(y[t]^2) + eps)) over H columns, weight 1,
+ * no residual: the input of the next layer in a stack of MoE layers.
+ * y, y_out: device bf16 [T, H], 16-byte aligned (may alias). */
+int moe_rmsnorm(const moe_bf16* y, moe_bf16* y_out, int T, int H, float eps, moe_stream stream);
+
+/* Waits for `stream`, returns the status word kept in `workspace` (MOE_OK or
+ * MOE_ERR_DEVICE_TIMEOUT) and clears it.  MOE_ERR_CUDA if the wait fails. */
+int moe_get_status(void* workspace, moe_stream stream);
+
+/* Static description of a status code. */
+const char* moe_strerror(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H_ */
