@@ -1,0 +1,323 @@
+// C ABI of libmoe.so: argument validation, workspace carving and the launch
+// sequence of one MoE layer on the caller's stream.  No host synchronisation
+// except in moe_get_status and moe_forward_host.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/moe.h"
+#include "kernels.h"
+
+namespace {
+
+using namespace moe;
+
+constexpr int kDecodeMaxT = 64;
+constexpr int kMaxT = 65536;
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Byte offsets of every workspace buffer for a call with T tokens.
+struct WsLayout {
+  size_t status, topk_idx, topk_w, counts, offsets, perm, inv_perm, sigma, seg, chunks, n_chunks, active,
+      n_active, h, h_s, Y, x_stage, out_stage, total;
+  int max_chunks;
+};
+
+WsLayout ws_layout(const moe_layer_desc* d, int T) {
+  WsLayout w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align_up(bytes);
+    return o;
+  };
+  const size_t n = static_cast<size_t>(T) * d->k;
+  const int cr = gemm_chunk_rows();
+  w.max_chunks = static_cast<int>(n / cr + T / cr + d->E + 2);
+  w.status = take(sizeof(int));
+  w.topk_idx = take(n * 4);
+  w.topk_w = take(n * 4);
+  w.counts = take(static_cast<size_t>(d->E) * 4);
+  w.offsets = take(static_cast<size_t>(d->E + 1) * 4);
+  w.perm = take(n * 4);
+  w.inv_perm = take(n * 4);
+  w.sigma = take(static_cast<size_t>(T) * 4);
+  w.seg = take(static_cast<size_t>(num_segments(static_cast<int>(n))) * d->E * 4);
+  w.chunks = take(static_cast<size_t>(w.max_chunks) * sizeof(Chunk));
+  w.n_chunks = take(4);
+  w.active = take(static_cast<size_t>(d->E + 1) * 4);
+  w.n_active = take(4);
+  w.h = take(n * d->I * 2);
+  w.h_s = take(static_cast<size_t>(T) * d->I_shared * 2);
+  w.Y = take((n + T) * d->H * 4);
+  w.x_stage = take(static_cast<size_t>(T) * d->H * 2);
+  w.out_stage = take(static_cast<size_t>(T) * d->H * 2);
+  w.total = off;
+  return w;
+}
+
+bool qmat_ok(const moe_qmat& m) {
+  return m.q && m.scales && m.biases && aligned16(m.q) && (reinterpret_cast<uintptr_t>(m.scales) & 1u) == 0 &&
+         (reinterpret_cast<uintptr_t>(m.biases) & 1u) == 0;
+}
+
+int validate_layer(const moe_layer_desc* d) {
+  if (!d) return MOE_ERR_INVALID_ARG;
+  if (d->bits != 4 || d->group_size != 64 || d->renorm != 1) return MOE_ERR_UNSUPPORTED;
+  if (d->k < 1 || d->k > kMaxK || d->E < d->k || d->E > kMaxE) return MOE_ERR_UNSUPPORTED;
+  if (d->H < 128 || d->H % 128 || d->H > 8192) return MOE_ERR_UNSUPPORTED;
+  if (d->I < 128 || d->I % 128 || d->I > 2048) return MOE_ERR_UNSUPPORTED;
+  if (d->I_shared < 128 || d->I_shared % 128 || d->I_shared > 2048) return MOE_ERR_UNSUPPORTED;
+  if (!d->w_router || !aligned16(d->w_router)) return MOE_ERR_INVALID_ARG;
+  if (d->router_bias && (reinterpret_cast<uintptr_t>(d->router_bias) & 3u)) return MOE_ERR_INVALID_ARG;
+  if (!qmat_ok(d->gate) || !qmat_ok(d->up) || !qmat_ok(d->down)) return MOE_ERR_INVALID_ARG;
+  if (!qmat_ok(d->sh_gate) || !qmat_ok(d->sh_up) || !qmat_ok(d->sh_down)) return MOE_ERR_INVALID_ARG;
+  if (!d->w_shared_gate || !aligned16(d->w_shared_gate)) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+int validate_ws(const moe_layer_desc* d, int T, void* ws, size_t ws_bytes) {
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1))) return MOE_ERR_WORKSPACE;
+  if (ws_layout(d, T).total > ws_bytes) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+int validate_routing(const moe_routing* r) {
+  if (!r) return MOE_OK;
+  if (!r->topk_idx || !r->topk_w || !r->counts || !r->offsets || !r->perm || !r->inv_perm)
+    return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+LayerPtr layer_ptrs(const moe_layer_desc* d) {
+  auto qp = [](const moe_qmat& m) { return QMatPtr{m.q, m.scales, m.biases}; };
+  return LayerPtr{d->w_router, d->router_bias, qp(d->gate), qp(d->up), qp(d->down),
+                  qp(d->sh_gate), qp(d->sh_up), qp(d->sh_down), d->w_shared_gate};
+}
+
+// Resolved device buffers of one call.
+struct Bufs {
+  char* base;
+  WsLayout w;
+  int32_t* topk_idx;
+  float* topk_w;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* perm;
+  int32_t* inv_perm;
+  float* sigma;
+  template <class P>
+  P* at(size_t off) const { return reinterpret_cast<P*>(base + off); }
+};
+
+Bufs resolve(const moe_layer_desc* d, int T, void* ws, const moe_routing* r) {
+  Bufs b;
+  b.base = static_cast<char*>(ws);
+  b.w = ws_layout(d, T);
+  b.topk_idx = r ? r->topk_idx : b.at<int32_t>(b.w.topk_idx);
+  b.topk_w = r ? r->topk_w : b.at<float>(b.w.topk_w);
+  b.counts = r ? r->counts : b.at<int32_t>(b.w.counts);
+  b.offsets = r ? r->offsets : b.at<int32_t>(b.w.offsets);
+  b.perm = r ? r->perm : b.at<int32_t>(b.w.perm);
+  b.inv_perm = r ? r->inv_perm : b.at<int32_t>(b.w.inv_perm);
+  b.sigma = (r && r->sigma) ? r->sigma : b.at<float>(b.w.sigma);
+  return b;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// Optional stage tracer: records ev[0] before the first stage and ev[i+1]
+// after stage i on the call's stream.
+struct Tracer {
+  cudaEvent_t ev[8];
+  int n = 0;
+  void mark(cudaStream_t s) {
+    if (n < 8) cudaEventRecord(ev[n++], s);
+  }
+};
+
+inline void mark(Tracer* tr, cudaStream_t s) {
+  if (tr) tr->mark(s);
+}
+
+int enqueue_route(const moe_layer_desc* d, const uint16_t* x, int T, const Bufs& b, cudaStream_t s,
+                  Tracer* tr = nullptr) {
+  mark(tr, s);
+  cudaError_t e = launch_router(x, d->w_router, d->router_bias, d->w_shared_gate, T, d->H, d->E, d->k,
+                                b.topk_idx, b.topk_w, b.sigma, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  mark(tr, s);
+  e = launch_group(b.topk_idx, T, d->k, d->E, gemm_chunk_rows(), b.at<int32_t>(b.w.seg), b.counts, b.offsets,
+                   b.perm, b.inv_perm, b.at<Chunk>(b.w.chunks), b.at<int32_t>(b.w.n_chunks),
+                   b.at<int32_t>(b.w.active), b.at<int32_t>(b.w.n_active), s);
+  mark(tr, s);
+  return cuda_status(e);
+}
+
+int enqueue_decode(const moe_layer_desc* d, const uint16_t* x, int T, uint16_t* out, const Bufs& b,
+                   cudaStream_t s, Tracer* tr = nullptr) {
+  int st = enqueue_route(d, x, T, b, s, tr);
+  if (st != MOE_OK) return st;
+  const Geometry g{T, d->H, d->I, d->I_shared, d->E, d->k};
+  const LayerPtr L = layer_ptrs(d);
+  uint16_t* h = b.at<uint16_t>(b.w.h);
+  uint16_t* h_s = b.at<uint16_t>(b.w.h_s);
+  cudaError_t e = launch_decode_gateup(g, L, x, b.offsets, b.perm, b.at<int32_t>(b.w.active),
+                                       b.at<int32_t>(b.w.n_active), h, h_s, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  mark(tr, s);
+  e = launch_decode_down_combine(g, L, h, h_s, b.topk_idx, b.topk_w, b.inv_perm, b.sigma, out, s);
+  mark(tr, s);
+  return cuda_status(e);
+}
+
+int enqueue_prefill(const moe_layer_desc* d, const uint16_t* x, int T, uint16_t* out, const Bufs& b,
+                    cudaStream_t s, Tracer* tr = nullptr) {
+  int st = enqueue_route(d, x, T, b, s, tr);
+  if (st != MOE_OK) return st;
+  const Geometry g{T, d->H, d->I, d->I_shared, d->E, d->k};
+  const LayerPtr L = layer_ptrs(d);
+  uint16_t* h = b.at<uint16_t>(b.w.h);
+  uint16_t* h_s = b.at<uint16_t>(b.w.h_s);
+  float* Y = b.at<float>(b.w.Y);
+  int* status = b.at<int>(b.w.status);
+  const Chunk* chunks = b.at<Chunk>(b.w.chunks);
+  const int32_t* n_chunks = b.at<int32_t>(b.w.n_chunks);
+  cudaError_t e = launch_gateup(g, L, x, b.perm, chunks, n_chunks, b.w.max_chunks, h, h_s, status, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  mark(tr, s);
+  e = launch_down(g, L, h, h_s, chunks, n_chunks, b.w.max_chunks, Y, status, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  mark(tr, s);
+  e = launch_combine(Y, b.inv_perm, b.topk_w, b.sigma, T, d->k, d->H, out, s);
+  mark(tr, s);
+  return cuda_status(e);
+}
+
+int check_call(const moe_layer_desc* d, const void* x, int T, int T_limit, const void* out, const moe_routing* r,
+               void* ws, size_t ws_bytes, bool need_out) {
+  int st = validate_layer(d);
+  if (st != MOE_OK) return st;
+  if (T < 1 || T > T_limit) return MOE_ERR_INVALID_ARG;
+  if (!x || !aligned16(x)) return MOE_ERR_INVALID_ARG;
+  if (need_out && (!out || !aligned16(out))) return MOE_ERR_INVALID_ARG;
+  st = validate_routing(r);
+  if (st != MOE_OK) return st;
+  return validate_ws(d, T, ws, ws_bytes);
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_workspace_size(const moe_layer_desc* layer, int T_max, size_t* bytes) {
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  const int st = validate_layer(layer);
+  if (st != MOE_OK) return st;
+  if (T_max < 1 || T_max > kMaxT) return MOE_ERR_INVALID_ARG;
+  *bytes = ws_layout(layer, T_max).total;
+  return MOE_OK;
+}
+
+int moe_route(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_routing* r, void* ws, size_t ws_bytes,
+              moe_stream stream) {
+  if (!r) return MOE_ERR_INVALID_ARG;
+  const int st = check_call(layer, x, T, kMaxT, nullptr, r, ws, ws_bytes, false);
+  if (st != MOE_OK) return st;
+  return enqueue_route(layer, x, T, resolve(layer, T, ws, r), static_cast<cudaStream_t>(stream));
+}
+
+int moe_forward(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_bf16* out, moe_routing* r, void* ws,
+                size_t ws_bytes, moe_stream stream) {
+  const int st = check_call(layer, x, T, kMaxT, out, r, ws, ws_bytes, true);
+  if (st != MOE_OK) return st;
+  const Bufs b = resolve(layer, T, ws, r);
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (T <= kDecodeMaxT) return enqueue_decode(layer, x, T, out, b, s);
+  return enqueue_prefill(layer, x, T, out, b, s);
+}
+
+int moe_decode(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_bf16* out, moe_routing* r, void* ws,
+               size_t ws_bytes, moe_stream stream) {
+  const int st = check_call(layer, x, T, kDecodeMaxT, out, r, ws, ws_bytes, true);
+  if (st != MOE_OK) return st;
+  return enqueue_decode(layer, x, T, out, resolve(layer, T, ws, r), static_cast<cudaStream_t>(stream));
+}
+
+int moe_forward_host(const moe_layer_desc* layer, const moe_bf16* x_host, int T, moe_bf16* out_host, void* ws,
+                     size_t ws_bytes, moe_stream stream) {
+  int st = validate_layer(layer);
+  if (st != MOE_OK) return st;
+  if (T < 1 || T > kMaxT || !x_host || !out_host) return MOE_ERR_INVALID_ARG;
+  st = validate_ws(layer, T, ws, ws_bytes);
+  if (st != MOE_OK) return st;
+  const Bufs b = resolve(layer, T, ws, nullptr);
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint16_t* xd = b.at<uint16_t>(b.w.x_stage);
+  uint16_t* od = b.at<uint16_t>(b.w.out_stage);
+  const size_t bytes = static_cast<size_t>(T) * layer->H * sizeof(uint16_t);
+  if (cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return MOE_ERR_CUDA;
+  st = (T <= kDecodeMaxT) ? enqueue_decode(layer, xd, T, od, b, s) : enqueue_prefill(layer, xd, T, od, b, s);
+  if (st != MOE_OK) return st;
+  if (cudaMemcpyAsync(out_host, od, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ERR_CUDA;
+  return cuda_status(cudaStreamSynchronize(s));
+}
+
+int moe_rmsnorm(const moe_bf16* y, moe_bf16* y_out, int T, int H, float eps, moe_stream stream) {
+  if (!y || !y_out || !aligned16(y) || !aligned16(y_out)) return MOE_ERR_INVALID_ARG;
+  if (T < 1 || T > kMaxT || H < 8 || H % 8 || H > 65536 || !(eps >= 0.f)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_rmsnorm(y, y_out, T, H, eps, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_forward_profiled(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_bf16* out, void* ws,
+                         size_t ws_bytes, moe_stream stream, float* stage_ms, int* n_stages) {
+  if (!stage_ms || !n_stages) return MOE_ERR_INVALID_ARG;
+  int st = check_call(layer, x, T, kMaxT, out, nullptr, ws, ws_bytes, true);
+  if (st != MOE_OK) return st;
+  const Bufs b = resolve(layer, T, ws, nullptr);
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Tracer tr;
+  for (int i = 0; i < 8; ++i)
+    if (cudaEventCreate(&tr.ev[i]) != cudaSuccess) {
+      for (int j = 0; j < i; ++j) cudaEventDestroy(tr.ev[j]);
+      return MOE_ERR_CUDA;
+    }
+  st = (T <= kDecodeMaxT) ? enqueue_decode(layer, x, T, out, b, s, &tr) : enqueue_prefill(layer, x, T, out, b, s, &tr);
+  if (st == MOE_OK && cudaEventSynchronize(tr.ev[tr.n - 1]) != cudaSuccess) st = MOE_ERR_CUDA;
+  *n_stages = 0;
+  if (st == MOE_OK) {
+    for (int i = 0; i + 1 < tr.n; ++i) cudaEventElapsedTime(&stage_ms[i], tr.ev[i], tr.ev[i + 1]);
+    *n_stages = tr.n - 1;
+  }
+  for (int i = 0; i < 8; ++i) cudaEventDestroy(tr.ev[i]);
+  return st;
+}
+
+int moe_get_status(void* ws, moe_stream stream) {
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1))) return MOE_ERR_WORKSPACE;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int host = 0;
+  if (cudaMemcpyAsync(&host, ws, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemsetAsync(ws, 0, sizeof(int), s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  return host;
+}
+
+const char* moe_strerror(int status) {
+  switch (status) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument (NULL or misaligned pointer, or T out of range)";
+    case MOE_ERR_UNSUPPORTED: return "unsupported layer (needs affine 4-bit, group 64, renorm, supported sizes)";
+    case MOE_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case MOE_ERR_CUDA: return "CUDA runtime error or kernel launch failure";
+    case MOE_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait gave up";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,96 @@
+// Deterministic gather-combine and the RMSNorm that links stacked layers.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+// out_t = bf16( sum_{j=0..k-1} w[t,j] * Y[inv_perm[t*k+j]]  +  sigma_t * Y[T*k + t] )
+// in FP32, in exactly that order, with no atomics: every token's sum is formed
+// by one thread per 8 columns, so the result is bitwise reproducible.
+__global__ void __launch_bounds__(256) combine_kernel(
+    const float* __restrict__ Y, const int32_t* __restrict__ inv_perm, const float* __restrict__ topk_w,
+    const float* __restrict__ sigma, int T, int k, int H, uint16_t* __restrict__ out) {
+  const int t = blockIdx.x;
+  int pos[kMaxK];
+  float w[kMaxK];
+#pragma unroll
+  for (int j = 0; j < kMaxK; ++j) {
+    pos[j] = j < k ? inv_perm[static_cast<size_t>(t) * k + j] : 0;
+    w[j] = j < k ? topk_w[static_cast<size_t>(t) * k + j] : 0.f;
+  }
+  const float sg = sigma[t];
+  const size_t shared_row = static_cast<size_t>(T) * k + t;
+  for (int c = threadIdx.x * 8; c < H; c += blockDim.x * 8) {
+    float acc[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+      if (j < k) {
+        const float4* y = reinterpret_cast<const float4*>(Y + static_cast<size_t>(pos[j]) * H + c);
+        const float4 a = y[0], b = y[1];
+        acc[0] = fmaf(w[j], a.x, acc[0]); acc[1] = fmaf(w[j], a.y, acc[1]);
+        acc[2] = fmaf(w[j], a.z, acc[2]); acc[3] = fmaf(w[j], a.w, acc[3]);
+        acc[4] = fmaf(w[j], b.x, acc[4]); acc[5] = fmaf(w[j], b.y, acc[5]);
+        acc[6] = fmaf(w[j], b.z, acc[6]); acc[7] = fmaf(w[j], b.w, acc[7]);
+      }
+    }
+    const float4* ys = reinterpret_cast<const float4*>(Y + shared_row * H + c);
+    const float4 a = ys[0], b = ys[1];
+    acc[0] = fmaf(sg, a.x, acc[0]); acc[1] = fmaf(sg, a.y, acc[1]);
+    acc[2] = fmaf(sg, a.z, acc[2]); acc[3] = fmaf(sg, a.w, acc[3]);
+    acc[4] = fmaf(sg, b.x, acc[4]); acc[5] = fmaf(sg, b.y, acc[5]);
+    acc[6] = fmaf(sg, b.z, acc[6]); acc[7] = fmaf(sg, b.w, acc[7]);
+    uint4 o;
+    o.x = pack_bf16x2(acc[0], acc[1]); o.y = pack_bf16x2(acc[2], acc[3]);
+    o.z = pack_bf16x2(acc[4], acc[5]); o.w = pack_bf16x2(acc[6], acc[7]);
+    *reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * H + c) = o;
+  }
+}
+
+// y_out = bf16(y / sqrt(mean(y^2) + eps)), one CTA per row, fixed reduction tree.
+__global__ void __launch_bounds__(256) rmsnorm_kernel(const uint16_t* __restrict__ y, uint16_t* __restrict__ out,
+                                                      int H, float eps) {
+  __shared__ float part[8];
+  const size_t row = blockIdx.x;
+  const uint4* src = reinterpret_cast<const uint4*>(y + row * H);
+  float ss = 0.f;
+  for (int c = threadIdx.x; c < H / 8; c += blockDim.x) {
+    const uint4 v = src[c];
+    const float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                        bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+#pragma unroll
+    for (int q = 0; q < 8; ++q) ss = fmaf(f[q], f[q], ss);
+  }
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  float tot = 0.f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) tot += part[w];
+  const float inv = 1.0f / sqrtf(tot / static_cast<float>(H) + eps);
+  uint4* dst = reinterpret_cast<uint4*>(out + row * H);
+  __syncthreads();   // y and out may alias: every read of the row is done
+  for (int c = threadIdx.x; c < H / 8; c += blockDim.x) {
+    const uint4 v = src[c];
+    uint4 o;
+    o.x = pack_bf16x2(bf16_lo(v.x) * inv, bf16_hi(v.x) * inv);
+    o.y = pack_bf16x2(bf16_lo(v.y) * inv, bf16_hi(v.y) * inv);
+    o.z = pack_bf16x2(bf16_lo(v.z) * inv, bf16_hi(v.z) * inv);
+    o.w = pack_bf16x2(bf16_lo(v.w) * inv, bf16_hi(v.w) * inv);
+    dst[c] = o;
+  }
+}
+
+cudaError_t launch_combine(const float* Y, const int32_t* inv_perm, const float* topk_w, const float* sigma,
+                           int T, int k, int H, uint16_t* out, cudaStream_t s) {
+  combine_kernel<<<T, 256, 0, s>>>(Y, inv_perm, topk_w, sigma, T, k, H, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rmsnorm(const uint16_t* y, uint16_t* out, int T, int H, float eps, cudaStream_t s) {
+  rmsnorm_kernel<<<T, 256, 0, s>>>(y, out, H, eps);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,63 @@
+// Host-side launchers of the MoE kernels (internal to libmoe.so).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+// Per-call geometry shared by the launchers.
+struct Geometry {
+  int T, H, I, Is, E, k;
+};
+
+// Device pointers of one layer (mirrors moe_layer_desc).
+struct QMatPtr {
+  const uint32_t* q;
+  const uint16_t* s;
+  const uint16_t* b;
+};
+struct LayerPtr {
+  const uint16_t* w_router;
+  const float* router_bias;
+  QMatPtr gate, up, down, sh_gate, sh_up, sh_down;
+  const uint16_t* w_sg;
+};
+
+// route.cu
+cudaError_t launch_router(const uint16_t* x, const uint16_t* w_router, const float* router_bias,
+                          const uint16_t* w_sg, int T, int H, int E, int k,
+                          int32_t* topk_idx, float* topk_w, float* sigma, cudaStream_t s);
+int num_segments(int n_entries);
+cudaError_t launch_group(const int32_t* topk_idx, int T, int k, int E, int chunk_rows,
+                         int32_t* seg_scratch, int32_t* counts, int32_t* offsets,
+                         int32_t* perm, int32_t* inv_perm, Chunk* chunks, int32_t* n_chunks,
+                         int32_t* active, int32_t* n_active, cudaStream_t s);
+
+// gemm.cu: grouped expert GEMMs over the device chunk list.
+int gemm_chunk_rows();
+cudaError_t launch_gateup(const Geometry& g, const LayerPtr& L, const uint16_t* x, const int32_t* perm,
+                          const Chunk* chunks, const int32_t* n_chunks, int max_chunks,
+                          uint16_t* h, uint16_t* h_s, int* status, cudaStream_t s);
+cudaError_t launch_down(const Geometry& g, const LayerPtr& L, const uint16_t* h, const uint16_t* h_s,
+                        const Chunk* chunks, const int32_t* n_chunks, int max_chunks,
+                        float* Y, int* status, cudaStream_t s);
+
+// combine.cu
+cudaError_t launch_combine(const float* Y, const int32_t* inv_perm, const float* topk_w, const float* sigma,
+                           int T, int k, int H, uint16_t* out, cudaStream_t s);
+cudaError_t launch_rmsnorm(const uint16_t* y, uint16_t* out, int T, int H, float eps, cudaStream_t s);
+
+// decode.cu: T <= 64
+cudaError_t launch_decode_gateup(const Geometry& g, const LayerPtr& L, const uint16_t* x,
+                                 const int32_t* offsets, const int32_t* perm,
+                                 const int32_t* active, const int32_t* n_active,
+                                 uint16_t* h, uint16_t* h_s, cudaStream_t s);
+cudaError_t launch_decode_down_combine(const Geometry& g, const LayerPtr& L, const uint16_t* h,
+                                       const uint16_t* h_s, const int32_t* topk_idx, const float* topk_w,
+                                       const int32_t* inv_perm, const float* sigma, uint16_t* out,
+                                       cudaStream_t s);
+
+}  // namespace moe

@@ -61,6 +61,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -129,13 +135,13 @@ typedef struct {
 /* Bytes of device workspace that moe_route / moe_forward / moe_decode /
  * moe_forward_host need for any T <= T_max.  Returns MOE_ERR_UNSUPPORTED or
  * MOE_ERR_INVALID_ARG for a layer or T_max the other calls would reject. */
-int moe_workspace_size(const moe_layer_desc* layer, int T_max, size_t* bytes);
+MOE_API int moe_workspace_size(const moe_layer_desc* layer, int T_max, size_t* bytes);
 
 /* Router logits, softmax top-k with renormalisation, shared gate, and the
  * on-device expert histogram, prefix sum and permutation ("Perplexity's
  * Lily: ...", section "How It Works: Prefill and Decode Strategies").
  * x: device bf16 [T, H], 16-byte aligned.  r: required.  1 <= T <= 65536. */
-int moe_route(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_routing* r,
+MOE_API int moe_route(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_routing* r,
               void* workspace, size_t workspace_bytes, moe_stream stream);
 
 /* The whole layer: routing, fused-dequant gate/up grouped GEMM with the
@@ -143,32 +149,43 @@ int moe_route(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_routing
  * fixed-order gather-combine.  x, out: device bf16 [T, H], 16-byte aligned,
  * not overlapping.  r: optional (NULL = keep routing in the workspace).
  * 1 <= T <= 65536; T <= 64 runs the decode kernels of moe_decode. */
-int moe_forward(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_bf16* out,
+MOE_API int moe_forward(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_bf16* out,
                 moe_routing* r, void* workspace, size_t workspace_bytes, moe_stream stream);
 
 /* The same function for 1 <= T <= 64 through the bandwidth-bound decode
  * kernels (batch-1 decoding streams the active experts' weights: "How It
  * Works: Prefill and Decode Strategies").  T > 64 is MOE_ERR_INVALID_ARG. */
-int moe_decode(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_bf16* out,
+MOE_API int moe_decode(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_bf16* out,
                moe_routing* r, void* workspace, size_t workspace_bytes, moe_stream stream);
 
 /* moe_forward with x and out in HOST memory (page-locked for full speed):
  * copies x to the workspace, runs the layer, copies the result back and waits
  * for `stream`.  Weights stay device pointers. */
-int moe_forward_host(const moe_layer_desc* layer, const moe_bf16* x_host, int T, moe_bf16* out_host,
+MOE_API int moe_forward_host(const moe_layer_desc* layer, const moe_bf16* x_host, int T, moe_bf16* out_host,
                      void* workspace, size_t workspace_bytes, moe_stream stream);
 
 /* y_out[t] = bf16(y[t] / sqrt(mean(y[t]^2) + eps)) over H columns, weight 1,
  * no residual: the input of the next layer in a stack of MoE layers.
  * y, y_out: device bf16 [T, H], 16-byte aligned (may alias). */
-int moe_rmsnorm(const moe_bf16* y, moe_bf16* y_out, int T, int H, float eps, moe_stream stream);
+MOE_API int moe_rmsnorm(const moe_bf16* y, moe_bf16* y_out, int T, int H, float eps, moe_stream stream);
+
+/* Stage timing (tracing).  Same as moe_forward, but records a CUDA event on
+ * `stream` before the first and after every stage, waits for the stream, and
+ * writes each stage's device time in milliseconds to stage_ms[0..n-1]:
+ *   T > 64:  router, group (histogram+scan+scatter), gate/up GEMM, down GEMM, combine
+ *   T <= 64: router, group, gate/up GEMV, down GEMV + combine, (unused)
+ * stage_ms: host array of at least 5 floats; *n_stages receives the count.
+ * The events are created and destroyed inside the call. */
+MOE_API int moe_forward_profiled(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_bf16* out,
+                                 void* workspace, size_t workspace_bytes, moe_stream stream,
+                                 float* stage_ms, int* n_stages);
 
 /* Waits for `stream`, returns the status word kept in `workspace` (MOE_OK or
  * MOE_ERR_DEVICE_TIMEOUT) and clears it.  MOE_ERR_CUDA if the wait fails. */
-int moe_get_status(void* workspace, moe_stream stream);
+MOE_API int moe_get_status(void* workspace, moe_stream stream);
 
 /* Static description of a status code. */
-const char* moe_strerror(int status);
+MOE_API const char* moe_strerror(int status);
 
 #ifdef __cplusplus
 }

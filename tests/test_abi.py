@@ -1,0 +1,129 @@
+"""The C-ABI library loads, exports every declared entry point, sizes its
+workspace, and rejects bad arguments on the host before touching a GPU."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from bit_quantized_expert_route_b200 import build as moe_build
+from bit_quantized_expert_route_b200 import moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    moe_build.build()
+    return moe.library()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "moe.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:MOE_API\s+)?(?:int|const char\*)\s+(moe_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert set(names) == set(moe.EXPORTS), names
+    for n in names:
+        assert hasattr(lib, n)
+
+
+def test_strerror(lib):
+    for code in (0, -1, -2, -3, -4, -5):
+        assert moe.strerror(code)
+    assert "unknown" in moe.strerror(42)
+
+
+FAKE = 0x10000   # a 16-byte-aligned non-NULL address; never dereferenced on these paths
+
+
+def fake_layer(**over):
+    qm = moe.QMatC(FAKE, FAKE, FAKE)
+    fields = dict(H=2048, I=512, I_shared=512, E=256, k=8, group_size=64, bits=4, renorm=1)
+    fields.update(over)
+    return moe.LayerC(fields["H"], fields["I"], fields["I_shared"], fields["E"], fields["k"], fields["group_size"],
+                      fields["bits"], fields["renorm"], FAKE, None, qm, qm, qm, qm, qm, qm, FAKE)
+
+
+def ws_size(lib, layer, T):
+    n = ctypes.c_size_t(0)
+    st = lib.moe_workspace_size(ctypes.byref(layer), T, ctypes.byref(n))
+    return st, n.value
+
+
+def test_workspace_size_monotone(lib):
+    L = fake_layer()
+    sizes = []
+    for T in (1, 8, 64, 512, 4096, 16384):
+        st, n = ws_size(lib, L, T)
+        assert st == 0
+        sizes.append(n)
+    assert sizes == sorted(sizes)
+    # Y (FP32, (T*k + T) x H) dominates at T=4096
+    assert sizes[4] >= 9 * 4096 * 2048 * 4
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(bits=8), moe.MOE_ERR_UNSUPPORTED),
+    (dict(group_size=128), moe.MOE_ERR_UNSUPPORTED),
+    (dict(renorm=0), moe.MOE_ERR_UNSUPPORTED),
+    (dict(k=9), moe.MOE_ERR_UNSUPPORTED),
+    (dict(k=0), moe.MOE_ERR_UNSUPPORTED),
+    (dict(E=300), moe.MOE_ERR_UNSUPPORTED),
+    (dict(E=4, k=8), moe.MOE_ERR_UNSUPPORTED),
+    (dict(H=200), moe.MOE_ERR_UNSUPPORTED),
+    (dict(I=96), moe.MOE_ERR_UNSUPPORTED),
+    (dict(I_shared=4096), moe.MOE_ERR_UNSUPPORTED),
+])
+def test_layer_validation(lib, over, code):
+    st, _ = ws_size(lib, fake_layer(**over), 16)
+    assert st == code
+
+
+def test_null_and_misaligned_pointers(lib):
+    L = fake_layer()
+    L.gate = moe.QMatC(FAKE, None, FAKE)
+    assert ws_size(lib, L, 4)[0] == moe.MOE_ERR_INVALID_ARG
+    L = fake_layer()
+    L.w_router = FAKE + 2
+    assert ws_size(lib, L, 4)[0] == moe.MOE_ERR_INVALID_ARG
+    L = fake_layer()
+    assert ws_size(lib, L, 0)[0] == moe.MOE_ERR_INVALID_ARG
+    assert ws_size(lib, L, 70000)[0] == moe.MOE_ERR_INVALID_ARG
+
+
+def test_calls_reject_before_launch(lib):
+    L = fake_layer()
+    st, need = ws_size(lib, L, 16)
+    out = FAKE
+    # workspace too small / misaligned / missing
+    assert lib.moe_forward(ctypes.byref(L), FAKE, 16, out, None, FAKE, need - 1, None) == moe.MOE_ERR_WORKSPACE
+    assert lib.moe_forward(ctypes.byref(L), FAKE, 16, out, None, FAKE + 16, need, None) == moe.MOE_ERR_WORKSPACE
+    assert lib.moe_forward(ctypes.byref(L), FAKE, 16, out, None, None, need, None) == moe.MOE_ERR_WORKSPACE
+    # bad T, x, out
+    assert lib.moe_forward(ctypes.byref(L), FAKE, 0, out, None, FAKE, need, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_forward(ctypes.byref(L), FAKE + 8, 16, out, None, FAKE, need, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_forward(ctypes.byref(L), FAKE, 16, None, None, FAKE, need, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_decode(ctypes.byref(L), FAKE, 65, out, None, FAKE, 1 << 40, None) == moe.MOE_ERR_INVALID_ARG
+    # moe_route needs a routing struct, and a complete one
+    assert lib.moe_route(ctypes.byref(L), FAKE, 16, None, FAKE, need, None) == moe.MOE_ERR_INVALID_ARG
+    r = moe.RoutingC(FAKE, FAKE, FAKE, None, FAKE, FAKE, None)
+    assert lib.moe_route(ctypes.byref(L), FAKE, 16, ctypes.byref(r), FAKE, need, None) == moe.MOE_ERR_INVALID_ARG
+    # unsupported layout wins over everything else
+    L8 = fake_layer(bits=8)
+    assert lib.moe_forward(ctypes.byref(L8), FAKE, 16, out, None, FAKE, need, None) == moe.MOE_ERR_UNSUPPORTED
+    assert lib.moe_forward_host(ctypes.byref(L), None, 16, out, FAKE, need, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_rmsnorm(FAKE, FAKE, 0, 2048, ctypes.c_float(1e-6), None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_rmsnorm(FAKE, FAKE + 4, 4, 2048, ctypes.c_float(1e-6), None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_get_status(None, None) == moe.MOE_ERR_WORKSPACE
+
+
+def test_library_is_built_for_sm100a():
+    moe_build.build()
+    assert "arch=compute_100a,code=sm_100a" in " ".join(moe_build.NVCC_FLAGS)
+    assert os.path.exists(moe_build.LIB)

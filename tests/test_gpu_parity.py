@@ -1,0 +1,175 @@
+"""GPU path vs the CPU oracle, through the C ABI.
+
+Routing (indices, histogram, offsets, permutation) must be bit-exact on
+screened inputs; the layer output must be within relative L2 5e-3 and
+max |err| 2e-2 * max |ref| of the float64 oracle.
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+from bit_quantized_expert_route_b200 import moe, synth
+from oracle import moe_ref
+from tests.gpu_util import assert_output_close, assert_routing_exact, bits_of, require_cuda, run_layer, to_dev_bits
+from tests.workloads import FULL, TINY, workload
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    require_cuda()
+
+
+# ------------------------------------------------------------- tiny layer --
+
+@pytest.mark.parametrize("T", [1, 3, 16, 17, 64, 65, 200, 700])
+@pytest.mark.parametrize("zipf", [False, True])
+def test_tiny_layer_all_tokens(T, zipf):
+    lay, x, _ = workload(0 if not zipf else 1, T, TINY, zipf=zipf)
+    ref = moe_ref.moe_layer(x, lay, TINY.k)
+    gpu = run_layer(lay, x)
+    assert gpu["status"] == 0
+    assert_routing_exact(gpu, ref)
+    assert_output_close(gpu["out"], ref["out"])
+
+
+@pytest.mark.parametrize("T", [5, 300])
+def test_route_only(T):
+    lay, x, _ = workload(2, T, TINY)
+    ref = moe_ref.route(x, lay, TINY.k)
+    gpu = run_layer(lay, x, entry="route")
+    assert_routing_exact(gpu, ref)
+
+
+@pytest.mark.parametrize("T", [4, 100])
+def test_zero_input_gives_exact_zero(T):
+    lay = synth.make_layer(0, 0, TINY)
+    x = np.zeros((T, TINY.H), dtype=np.uint16)
+    gpu = run_layer(lay, x)
+    np.testing.assert_array_equal(gpu["topk_idx"], np.tile(np.arange(TINY.k), (T, 1)))
+    np.testing.assert_array_equal(gpu["topk_w"], np.full((T, TINY.k), 1.0 / TINY.k))
+    assert np.all(moe_ref.bf16_to_f64(gpu["out"]) == 0.0)
+
+
+@pytest.mark.parametrize("T", [7, 300])
+def test_token_permutation(T):
+    lay, x, _ = workload(3, T, TINY)
+    p = np.random.default_rng(1).permutation(T)
+    a = run_layer(lay, x)
+    b = run_layer(lay, x[p])
+    np.testing.assert_array_equal(b["counts"], a["counts"])
+    np.testing.assert_array_equal(b["topk_idx"], a["topk_idx"][p])
+    np.testing.assert_array_equal(b["out"], a["out"][p])        # rows are computed independently
+
+
+@pytest.mark.parametrize("T", [6, 250])
+def test_doubling_down_projection_doubles_output(T):
+    lay, x, _ = workload(4, T, TINY)
+    a = run_layer(lay, x)
+    for qm in (lay.down, lay.sh_down):
+        qm.scales[...] = synth.to_bf16_bits(2 * moe_ref.bf16_to_f64(qm.scales))
+        qm.biases[...] = synth.to_bf16_bits(2 * moe_ref.bf16_to_f64(qm.biases))
+    b = run_layer(lay, x)
+    np.testing.assert_array_equal(moe_ref.bf16_to_f64(b["out"]), 2 * moe_ref.bf16_to_f64(a["out"]))
+
+
+@pytest.mark.parametrize("T", [8, 129])
+def test_run_to_run_bitwise(T):
+    lay, x, _ = workload(5, T, TINY)
+    a = run_layer(lay, x)
+    b = run_layer(lay, x)
+    for key in ("out", "topk_idx", "perm", "inv_perm", "counts"):
+        np.testing.assert_array_equal(a[key], b[key])
+    np.testing.assert_array_equal(a["topk_w"], b["topk_w"])
+
+
+@pytest.mark.parametrize("T", [8, 333])
+def test_forward_host_equals_device(T):
+    lay, x, _ = workload(6, T, TINY)
+    L = moe.MoELayer.from_synth(lay)
+    dev = run_layer(lay, x, dev_layer=L)
+    ws = moe.alloc_workspace(L, T)
+    xh = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
+    oh = torch.empty_like(xh).pin_memory()
+    moe.moe_forward_host(L, xh, oh, ws)
+    np.testing.assert_array_equal(oh.view(torch.int16).numpy().view(np.uint16), dev["out"])
+
+
+def test_decode_entry_rejects_large_T():
+    lay, x, _ = workload(7, 65, TINY)
+    with pytest.raises(moe.MoEError) as e:
+        run_layer(lay, x, entry="decode")
+    assert e.value.code == moe.MOE_ERR_INVALID_ARG
+
+
+def test_decode_entry_equals_forward():
+    lay, x, _ = workload(8, 40, TINY)
+    L = moe.MoELayer.from_synth(lay)
+    a = run_layer(lay, x, entry="decode", dev_layer=L)
+    b = run_layer(lay, x, entry="forward", dev_layer=L)
+    np.testing.assert_array_equal(a["out"], b["out"])
+
+
+def test_rmsnorm_matches_oracle():
+    rng = np.random.default_rng(9)
+    y_bits = synth.to_bf16_bits(rng.normal(0, 0.05, size=(37, 2048)))
+    y = to_dev_bits(y_bits)
+    out = torch.empty_like(y)
+    moe.moe_rmsnorm(y, out, 1e-6)
+    got = moe_ref.bf16_to_f64(bits_of(out))
+    want = moe_ref.rmsnorm_bf16(moe_ref.bf16_to_f64(y_bits))
+    diff = got != want
+    # FP32 reciprocal square root vs float64 division: at most one bf16 step apart, rarely
+    ulp = np.abs(want) * 2.0 ** -7
+    assert np.all(np.abs(got - want) <= ulp + 1e-30)
+    assert diff.mean() < 1e-3
+    moe.moe_rmsnorm(y, y, 1e-6)            # in place
+    np.testing.assert_array_equal(bits_of(y), bits_of(out))
+
+
+# ------------------------------------------------------------- full layer --
+
+@pytest.mark.parametrize("T", [1, 8, 64])
+def test_full_decode(T):
+    lay, x, _ = workload(10 + T, T, FULL)
+    ref = moe_ref.moe_layer(x, lay, FULL.k)
+    gpu = run_layer(lay, x)
+    assert gpu["status"] == 0
+    assert_routing_exact(gpu, ref)
+    assert_output_close(gpu["out"], ref["out"])
+
+
+@pytest.fixture(scope="module", params=["uniform", "zipf"])
+def full_prefill(request):
+    zipf = request.param == "zipf"
+    lay, x, red = workload(20 if not zipf else 21, 4096, FULL, zipf=zipf)
+    L = moe.MoELayer.from_synth(lay)
+    gpu = run_layer(lay, x, dev_layer=L)
+    return lay, x, L, gpu
+
+
+def test_full_prefill_routing_all_tokens(full_prefill):
+    lay, x, L, gpu = full_prefill
+    ref = moe_ref.route(x, lay, FULL.k)
+    assert_routing_exact(gpu, ref)
+    assert gpu["status"] == 0
+
+
+def test_full_prefill_sampled_outputs(full_prefill):
+    lay, x, L, gpu = full_prefill
+    sample = np.sort(np.random.default_rng(0).choice(4096, size=192, replace=False))
+    sample = np.unique(np.concatenate([sample, [0, 4095]]))
+    ref = moe_ref.moe_layer(x, lay, FULL.k, tokens=sample)
+    assert_output_close(gpu["out"][sample], ref["out"])
+
+
+def test_full_prefill_bitwise_repeatable(full_prefill):
+    lay, x, L, gpu = full_prefill
+    again = run_layer(lay, x, dev_layer=L)
+    np.testing.assert_array_equal(again["out"], gpu["out"])
+    np.testing.assert_array_equal(again["perm"], gpu["perm"])
