@@ -37,9 +37,9 @@ T_PREFILL = 4096
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PREFILL_LAUNCHES_PER_STEP = 7     # router, hist, scan, scatter, gate/up, down, combine
 DECODE_LAUNCHES_PER_STEP = 6      # router, hist, scan, scatter, gate/up GEMV, down GEMV+combine
-COMPUTE_DTYPE = "f32"             # arithmetic type of the grouped GEMMs
-DOMINANT_KERNEL_SRC = "bit_quantized_expert_route_b200/csrc/gemm_simt.cu"
-DOMINANT_KERNEL = "gateup_simt_kernel"
+COMPUTE_DTYPE = "bf16"            # grouped GEMM operands (FP32 accumulation in tensor memory)
+DOMINANT_KERNEL_SRC = "bit_quantized_expert_route_b200/csrc/gemm_tc.cu"
+DOMINANT_KERNEL = "grouped_gemm_tc_kernel<true>"
 DECODE_KERNEL_SRC = "bit_quantized_expert_route_b200/csrc/decode.cu"
 DECODE_KERNEL = "decode_gateup_kernel"
 

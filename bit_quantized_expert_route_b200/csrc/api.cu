@@ -62,8 +62,8 @@ WsLayout ws_layout(const moe_layer_desc* d, int T) {
 }
 
 bool qmat_ok(const moe_qmat& m) {
-  return m.q && m.scales && m.biases && aligned16(m.q) && (reinterpret_cast<uintptr_t>(m.scales) & 1u) == 0 &&
-         (reinterpret_cast<uintptr_t>(m.biases) & 1u) == 0;
+  return m.q && m.scales && m.biases && aligned16(m.q) && (reinterpret_cast<uintptr_t>(m.scales) & 3u) == 0 &&
+         (reinterpret_cast<uintptr_t>(m.biases) & 3u) == 0;
 }
 
 int validate_layer(const moe_layer_desc* d) {

@@ -36,7 +36,7 @@ cudaError_t launch_group(const int32_t* topk_idx, int T, int k, int E, int chunk
                          int32_t* perm, int32_t* inv_perm, Chunk* chunks, int32_t* n_chunks,
                          int32_t* active, int32_t* n_active, cudaStream_t s);
 
-// gemm.cu: grouped expert GEMMs over the device chunk list.
+// gemm_tc.cu: tcgen05 grouped expert GEMMs over the device chunk list.
 int gemm_chunk_rows();
 cudaError_t launch_gateup(const Geometry& g, const LayerPtr& L, const uint16_t* x, const int32_t* perm,
                           const Chunk* chunks, const int32_t* n_chunks, int max_chunks,
