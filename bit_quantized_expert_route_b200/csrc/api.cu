@@ -5,6 +5,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/moe.h"
 #include "kernels.h"
@@ -213,6 +214,36 @@ int check_call(const moe_layer_desc* d, const void* x, int T, int T_limit, const
 
 }  // namespace
 
+// Scratch of moe_route_static: one static device array per GPU that loads
+// the library (a CUDA __device__ variable exists on every device of the
+// context), so callers that cannot allocate need not pass a workspace.
+constexpr size_t kRouteStaticBytes = 512u * 1024u;
+static __device__ __align__(256) unsigned char g_route_static_scratch[kRouteStaticBytes];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_route_static_mu;
+void* g_route_static_ptr[kMaxDevices] = {};
+
+// Device address of the static scratch on the current device; looked up once
+// per device (host code cannot use the symbol itself as a device address).
+int route_static_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_route_static_mu);
+  if (!g_route_static_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_route_static_scratch) != cudaSuccess || !p) return MOE_ERR_CUDA;
+    g_route_static_ptr[dev] = p;
+  }
+  *out = g_route_static_ptr[dev];
+  return MOE_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 int moe_workspace_size(const moe_layer_desc* layer, int T_max, size_t* bytes) {
@@ -247,6 +278,46 @@ int moe_decode(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_bf16* 
   const int st = check_call(layer, x, T, kDecodeMaxT, out, r, ws, ws_bytes, true);
   if (st != MOE_OK) return st;
   return enqueue_decode(layer, x, T, out, resolve(layer, T, ws, r), static_cast<cudaStream_t>(stream));
+}
+
+int moe_route_static(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_routing* r, moe_stream stream) {
+  if (!r) return MOE_ERR_INVALID_ARG;
+  int st = validate_layer(layer);
+  if (st != MOE_OK) return st;
+  if (T < 1 || T > kMaxT || !x || !aligned16(x)) return MOE_ERR_INVALID_ARG;
+  st = validate_routing(r);
+  if (st != MOE_OK) return st;
+  // carve the static scratch: segment counts, chunk list, counters, active list, sigma
+  const size_t n = static_cast<size_t>(T) * layer->k;
+  const int cr = gemm_chunk_rows();
+  const int max_chunks = static_cast<int>(n / cr + T / cr + layer->E + 2);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align_up(bytes);
+    return o;
+  };
+  const size_t o_seg = take(static_cast<size_t>(num_segments(static_cast<int>(n))) * layer->E * 4);
+  const size_t o_chunks = take(static_cast<size_t>(max_chunks) * sizeof(Chunk));
+  const size_t o_nchunks = take(4);
+  const size_t o_active = take(static_cast<size_t>(layer->E + 1) * 4);
+  const size_t o_nactive = take(4);
+  const size_t o_sigma = r->sigma ? 0 : take(static_cast<size_t>(T) * 4);
+  if (off > kRouteStaticBytes) return MOE_ERR_WORKSPACE;
+  void* base = nullptr;
+  st = route_static_scratch(&base);
+  if (st != MOE_OK) return st;
+  char* b = static_cast<char*>(base);
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* sigma = r->sigma ? r->sigma : reinterpret_cast<float*>(b + o_sigma);
+  cudaError_t e = launch_router(x, layer->w_router, layer->router_bias, layer->w_shared_gate, T, layer->H,
+                                layer->E, layer->k, r->topk_idx, r->topk_w, sigma, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  e = launch_group(r->topk_idx, T, layer->k, layer->E, cr, reinterpret_cast<int32_t*>(b + o_seg), r->counts,
+                   r->offsets, r->perm, r->inv_perm, reinterpret_cast<Chunk*>(b + o_chunks),
+                   reinterpret_cast<int32_t*>(b + o_nchunks), reinterpret_cast<int32_t*>(b + o_active),
+                   reinterpret_cast<int32_t*>(b + o_nactive), s);
+  return cuda_status(e);
 }
 
 int moe_forward_host(const moe_layer_desc* layer, const moe_bf16* x_host, int T, moe_bf16* out_host, void* ws,

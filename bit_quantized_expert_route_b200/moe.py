@@ -25,7 +25,7 @@ MOE_ERR_DEVICE_TIMEOUT = -5
 
 # Every entry point declared in include/moe.h.
 EXPORTS = ("moe_workspace_size", "moe_route", "moe_forward", "moe_decode", "moe_forward_host",
-           "moe_rmsnorm", "moe_forward_profiled", "moe_get_status", "moe_strerror")
+           "moe_rmsnorm", "moe_forward_profiled", "moe_route_static", "moe_get_status", "moe_strerror")
 
 
 class QMatC(ctypes.Structure):
@@ -75,6 +75,7 @@ def library() -> ctypes.CDLL:
     lib.moe_rmsnorm.argtypes = [P, P, I, I, ctypes.c_float, P]
     lib.moe_forward_profiled.argtypes = [LP, P, I, P, P, S, P, ctypes.POINTER(ctypes.c_float),
                                          ctypes.POINTER(ctypes.c_int)]
+    lib.moe_route_static.argtypes = [LP, P, I, RP, P]
     lib.moe_get_status.argtypes = [P, P]
     lib.moe_strerror.argtypes = [I]
     lib.moe_strerror.restype = ctypes.c_char_p
@@ -194,6 +195,13 @@ def moe_route(layer: MoELayer, x: torch.Tensor, routing: Routing, workspace: tor
     T = x.shape[0]
     _check(library().moe_route(ctypes.byref(layer.desc), x.data_ptr(), T, ctypes.byref(routing.c),
                                workspace.data_ptr(), workspace.numel(), _stream(stream)), "moe_route")
+
+
+def moe_route_static(layer: MoELayer, x: torch.Tensor, routing: Routing, stream=None) -> None:
+    """moe_route without a workspace (scratch in a static device array of libmoe.so)."""
+    T = x.shape[0]
+    _check(library().moe_route_static(ctypes.byref(layer.desc), x.data_ptr(), T, ctypes.byref(routing.c),
+                                      _stream(stream)), "moe_route_static")
 
 
 def moe_forward(layer: MoELayer, x: torch.Tensor, out: torch.Tensor, workspace: torch.Tensor,

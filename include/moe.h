@@ -158,6 +158,33 @@ MOE_API int moe_forward(const moe_layer_desc* layer, const moe_bf16* x, int T, m
 MOE_API int moe_decode(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_bf16* out,
                moe_routing* r, void* workspace, size_t workspace_bytes, moe_stream stream);
 
+/* moe_route for callers that cannot allocate device memory.  The pages have
+ * no counterpart to this entry point; it exists for hosts that hand the
+ * library only the tensors it reads and writes -- a plug-in inside another
+ * runtime that exposes no allocator, or a serving loop with a fixed memory
+ * plan where a cudaMalloc (which may also synchronise the device) is not
+ * allowed.  It computes exactly what moe_route computes, with the same
+ * kernels, but takes no workspace: its scratch (per-segment expert counts,
+ * the chunk list, the active-expert list, and sigma when r->sigma is NULL)
+ * lives in one static device array of 512 KiB inside libmoe.so, which every
+ * GPU that loads the library holds until the process exits.
+ *   Limit: the call needs ceil(T*k/1024)*E*4 bytes of counts, plus
+ *   (T*k/128 + T/128 + E + 2)*16 bytes of chunk list, plus (E+1)*4 + 2*4
+ *   bytes, plus T*4 bytes if r->sigma is NULL, each rounded up to 256 bytes;
+ *   a call whose need exceeds 512 KiB returns MOE_ERR_WORKSPACE and enqueues
+ *   nothing (for E=256, k=8 this admits T <= 56704 when r->sigma is given,
+ *   T <= 39424 when it is NULL).
+ *   Set-up: the first call on each device looks up the array's device
+ *   address with cudaGetSymbolAddress while that device is current, so make
+ *   that first call before any stream capture on that device.
+ *   Sharing: all calls in the process use the same array and nothing in it
+ *   needs to start at zero (every call rewrites what it reads); two calls
+ *   whose GPU work overlaps (different streams, or host threads) race on it.
+ * Allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ * Arguments as for moe_route, minus the workspace; r is required. */
+MOE_API int moe_route_static(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_routing* r,
+                             moe_stream stream);
+
 /* moe_forward with x and out in HOST memory (page-locked for full speed):
  * copies x to the workspace, runs the layer, copies the result back and waits
  * for `stream`.  Weights stay device pointers. */
