@@ -35,8 +35,8 @@ sys.path.insert(0, ROOT)
 
 T_PREFILL = 4096
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-PREFILL_LAUNCHES_PER_STEP = 7     # router, hist, scan, scatter, gate/up, down, combine
-DECODE_LAUNCHES_PER_STEP = 6      # router, hist, scan, scatter, gate/up GEMV, down GEMV+combine
+PREFILL_LAUNCHES_PER_STEP = 6     # router (+ segment counts), scan, scatter, gate/up, down, combine
+DECODE_LAUNCHES_PER_STEP = 3      # routing (router+top-k+sort), gate/up GEMV, down GEMV+combine
 COMPUTE_DTYPE = "bf16"            # grouped GEMM operands (FP32 accumulation in tensor memory)
 DOMINANT_KERNEL_SRC = "bit_quantized_expert_route_b200/csrc/gemm_tc.cu"
 DOMINANT_KERNEL = "grouped_gemm_tc_kernel<true>"
@@ -54,6 +54,11 @@ def parse_args(argv=None):
     ap.add_argument("--decode-steps", type=int, default=400)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-only", action="store_true", help="only the decode measurement (profiling)")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass (profiling)")
+    ap.add_argument("--no-stages", action="store_true", help="skip the per-stage traced pass (profiling)")
+    ap.add_argument("--layers", type=int, default=4, help="prefill layers cycled")
+    ap.add_argument("--decode-layers", type=int, default=40, help="decode layers cycled")
     return ap.parse_args(argv)
 
 
@@ -193,18 +198,11 @@ def timed_loop(fn, steps, world):
 
 # --------------------------------------------------------------- our arm ---
 
-def run_ours(a):
+def prefill_phase(a, world, rank, dev, dims, zipf, peaks, peak_src):
+    """K timed steps of the whole layer at T=4096, then per-stage times and e2e."""
     import torch
     from bit_quantized_expert_route_b200 import moe, synth
-
-    world, rank, local = dist_setup(a.gpus)
-    dev = torch.device("cuda", torch.cuda.current_device())
-    dims = synth.Dims()
-    zipf = a.workload == "zipf"
-    peaks, peak_src = load_peaks()
-
-    # ---- prefill: 4 layers + 4 activation sets cycled (1.9 GB > L2) ----
-    NL = 4
+    NL = a.layers
     layers = [moe.MoELayer.from_tensors(dims, synth.make_layer_on_device(1000 * rank + 1 + i, i, dims, dev, zipf))
               for i in range(NL)]
     xs = [synth.make_x_on_device(1000 * rank + 11 + i, T_PREFILL, dims.H, dev) for i in range(NL)]
@@ -216,89 +214,129 @@ def run_ours(a):
 
     for i in range(a.warmup):
         step(i)
-    with ClockSampler(torch.cuda.current_device()) as clk:
-        total_ms = timed_loop(step, a.steps, world)
-    clocks = clk.summary()
-    ms_per_step = total_ms / a.steps
-    value = world * T_PREFILL * a.steps / (total_ms / 1e3)
+    total_ms = timed_loop(step, a.steps, world)
+    res = {"ms_per_step": total_ms / a.steps, "value": world * T_PREFILL * a.steps / (total_ms / 1e3)}
 
-    # per-stage device times over the same workload (events between stages)
-    stages = {}
-    for i in range(a.steps):
-        st = moe.moe_forward_profiled(layers[i % NL], xs[i % NL], out, ws)
-        for k_, v in st.items():
-            stages.setdefault(k_, []).append(v)
-    stage_ms = {k_: statistics.mean(v) for k_, v in stages.items()}
+    if not a.no_stages:
+        # per-stage device times over the same workload (events between stages)
+        stages = {}
+        for i in range(a.steps):
+            for k_, v in moe.moe_forward_profiled(layers[i % NL], xs[i % NL], out, ws).items():
+                stages.setdefault(k_, []).append(v)
+        stage_ms = {k_: statistics.mean(v) for k_, v in stages.items()}
+        rows = T_PREFILL * dims.k + T_PREFILL
+        flop_gateup = rows * 2 * 2 * dims.H * dims.I
+        flop_layer = T_PREFILL * (dims.k + 1) * 6 * dims.H * dims.I + 2 * T_PREFILL * dims.H * dims.E
+        achieved = flop_gateup / (stage_ms["gateup"] / 1e3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        tr = committed_traffic(DOMINANT_KERNEL, DOMINANT_KERNEL_SRC)
+        res["roofline"] = {"kernel": DOMINANT_KERNEL, "bound": "tensor", "achieved": round(achieved, 2),
+                           "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                           "peak_source": f"{peak_src} bf16 sustained",
+                           "algorithmic_per_launch": flop_gateup,
+                           "traffic": tr[0] if tr else None,
+                           "layer_frac": round(flop_layer / (res["ms_per_step"] / 1e3) / 1e12 / peak, 4)}
+        res["stage_ms"] = {k_: round(v, 4) for k_, v in stage_ms.items()}
     assert moe.moe_get_status(ws) == 0
 
-    rows = T_PREFILL * dims.k + T_PREFILL
-    flop_gateup = rows * 2 * 2 * dims.H * dims.I
-    flop_layer = T_PREFILL * (dims.k + 1) * 6 * dims.H * dims.I + 2 * T_PREFILL * dims.H * dims.E
-    achieved = flop_gateup / (stage_ms["gateup"] / 1e3) / 1e12
-    peak = peaks["bf16_tflops_sustained"]
-    tr = committed_traffic(DOMINANT_KERNEL, DOMINANT_KERNEL_SRC)
-    roofline = {"kernel": DOMINANT_KERNEL, "bound": "tensor", "achieved": round(achieved, 2),
-                "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                "peak_source": f"{peak_src} bf16 sustained",
-                "algorithmic_per_launch": flop_gateup,
-                "traffic": tr[0] if tr else None,
-                "layer_frac": round(flop_layer / (ms_per_step / 1e3) / 1e12 / peak, 4)}
+    if not a.no_e2e:
+        # the same call with host (pinned) buffers, copies inside the timed region
+        xh = [xs[i].cpu().pin_memory() for i in range(NL)]
+        oh = torch.empty_like(xh[0]).pin_memory()
 
-    # ---- e2e: the same call with host (pinned) buffers, copies inside ----
-    xh = [xs[i].cpu().pin_memory() for i in range(NL)]
-    oh = torch.empty_like(xh[0]).pin_memory()
-    ws_h = ws
+        def step_host(i):
+            moe.moe_forward_host(layers[i % NL], xh[i % NL], oh, ws)
 
-    def step_host(i):
-        moe.moe_forward_host(layers[i % NL], xh[i % NL], oh, ws_h)
+        for i in range(2):
+            step_host(i)
+        e2e_ms = timed_loop(step_host, a.steps, world)
+        res["e2e"] = {"value": round(world * T_PREFILL * a.steps / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+                      "h2d_bytes_per_step": T_PREFILL * dims.H * 2, "d2h_bytes_per_step": T_PREFILL * dims.H * 2}
+    del layers, xs
+    torch.cuda.empty_cache()
+    return res
 
-    for i in range(2):
-        step_host(i)
-    e2e_ms = timed_loop(step_host, a.steps, world)
-    e2e = {"value": round(world * T_PREFILL * a.steps / (e2e_ms / 1e3), 1), "unit": "tokens/s",
-           "h2d_bytes_per_step": T_PREFILL * dims.H * 2, "d2h_bytes_per_step": T_PREFILL * dims.H * 2}
 
-    # ---- decode T=1: 40 resident layers cycled ----
-    decode = None
-    if not a.no_decode:
-        del layers, xs
-        torch.cuda.empty_cache()
-        NLD = 40
-        dl = [moe.MoELayer.from_tensors(dims, synth.make_layer_on_device(5000 * rank + l, l, dims, dev, False))
-              for l in range(NLD)]
-        dx = synth.make_x_on_device(7000 + rank, 64, dims.H, dev)
-        dout = torch.empty((1, dims.H), dtype=torch.bfloat16, device=dev)
-        dws = moe.alloc_workspace(dl[0], 1, dev)
+def decode_phase(a, world, rank, dev, dims, peaks, peak_src):
+    """Decode T=1 through `decode_layers` resident layers, cycled (stream-launched and as a CUDA graph)."""
+    import torch
+    from bit_quantized_expert_route_b200 import moe, synth
+    NLD = a.decode_layers
+    dl = [moe.MoELayer.from_tensors(dims, synth.make_layer_on_device(5000 * rank + l, l, dims, dev, False))
+          for l in range(NLD)]
+    dx = synth.make_x_on_device(7000 + rank, 64, dims.H, dev)
+    dout = torch.empty((1, dims.H), dtype=torch.bfloat16, device=dev)
+    dws = moe.alloc_workspace(dl[0], 1, dev)
 
-        def dstep(i):
-            moe.moe_forward(dl[i % NLD], dx[i % 64:i % 64 + 1], dout, dws)
+    def dstep(i):
+        moe.moe_forward(dl[i % NLD], dx[i % 64:i % 64 + 1], dout, dws)
 
-        for i in range(max(a.warmup, 40)):
-            dstep(i)
-        d_ms = timed_loop(dstep, a.decode_steps, world)
-        us_tok = d_ms * 1e3 / a.decode_steps
+    for i in range(max(a.warmup, NLD)):
+        dstep(i)
+    d_ms = timed_loop(dstep, a.decode_steps, world)
+    us_tok_stream = d_ms * 1e3 / a.decode_steps
+    # the same layer calls captured once as a CUDA graph and replayed
+    gstream = torch.cuda.Stream()
+    graph = torch.cuda.CUDAGraph()
+    gstream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(gstream):
+        for l in range(NLD):
+            dstep(l)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(graph, stream=gstream):
+            for l in range(NLD):
+                dstep(l)
+    torch.cuda.synchronize()
+    reps = max(1, a.decode_steps // NLD)
+    for _ in range(2):
+        graph.replay()
+    g_ms = timed_loop(lambda i: graph.replay(), reps, world)
+    us_tok = g_ms * 1e3 / (reps * NLD)
+    del graph
+    expert_bytes = dims.I * dims.H // 2 + dims.I * (dims.H // 64) * 4          # one q-matrix [I,H]
+    gateup_bytes = (dims.k + 1) * 2 * expert_bytes
+    active_bytes = (dims.k + 1) * 3 * expert_bytes
+    res = {"workload": f"decode T=1, {NLD} resident layers cycled ({NLD * 0.456:.1f} GB)",
+           "us_per_token": round(us_tok, 3), "us_per_token_stream_launched": round(us_tok_stream, 3),
+           "timing": "us_per_token: the layer sequence as one CUDA graph, replayed; "
+                     "stream-launched: one moe_forward call per layer",
+           "active_expert_bytes": active_bytes,
+           "active_bytes_GBps": round(active_bytes / (us_tok / 1e6) / 1e9, 1),
+           "hbm_frac_active_bytes": round(active_bytes / (us_tok / 1e6) / 1e9 / peaks["hbm_gbs"], 4),
+           "gpu_launches": DECODE_LAUNCHES_PER_STEP * reps * NLD}
+    if not a.no_stages:
         dst = {}
         for i in range(min(a.decode_steps, 200)):
-            st = moe.moe_forward_profiled(dl[i % NLD], dx[i % 64:i % 64 + 1], dout, dws)
-            for k_, v in st.items():
+            for k_, v in moe.moe_forward_profiled(dl[i % NLD], dx[i % 64:i % 64 + 1], dout, dws).items():
                 dst.setdefault(k_, []).append(v)
         dstage = {k_: statistics.median(v) for k_, v in dst.items()}
-        expert_bytes = dims.I * dims.H // 2 + dims.I * (dims.H // 64) * 4          # one q-matrix [I,H]
-        gateup_bytes = (dims.k + 1) * 2 * expert_bytes
-        active_bytes = (dims.k + 1) * 3 * expert_bytes
         ach = gateup_bytes / (dstage["gateup"] / 1e3) / 1e9
         trd = committed_traffic(DECODE_KERNEL, DECODE_KERNEL_SRC)
-        decode = {"workload": "decode T=1, 40 resident layers cycled (18.2 GB)", "us_per_token": round(us_tok, 3),
-                  "active_expert_bytes": active_bytes,
-                  "active_bytes_GBps": round(active_bytes / (us_tok / 1e6) / 1e9, 1),
-                  "hbm_frac_active_bytes": round(active_bytes / (us_tok / 1e6) / 1e9 / peaks["hbm_gbs"], 4),
-                  "stage_us": {k_: round(v * 1e3, 2) for k_, v in dstage.items()},
-                  "roofline": {"kernel": DECODE_KERNEL, "bound": "hbm", "achieved": round(ach, 1),
-                               "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4),
-                               "peak_source": f"{peak_src} HBM copy", "algorithmic_per_launch": gateup_bytes,
-                               "traffic": trd[0] if trd else None},
-                  "gpu_launches": DECODE_LAUNCHES_PER_STEP * a.decode_steps}
-        del dl
+        res["stage_us"] = {k_: round(v * 1e3, 2) for k_, v in dstage.items()}
+        res["roofline"] = {"kernel": DECODE_KERNEL, "bound": "hbm", "achieved": round(ach, 1),
+                           "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4),
+                           "peak_source": f"{peak_src} HBM copy", "algorithmic_per_launch": gateup_bytes,
+                           "traffic": trd[0] if trd else None}
+    del dl
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_ours(a):
+    import torch
+    from bit_quantized_expert_route_b200 import synth
+
+    world, rank, local = dist_setup(a.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    dims = synth.Dims()
+    zipf = a.workload == "zipf"
+    peaks, peak_src = load_peaks()
+
+    clk = ClockSampler(torch.cuda.current_device()).__enter__()   # sampled across every timed phase
+    pre = {} if a.decode_only else prefill_phase(a, world, rank, dev, dims, zipf, peaks, peak_src)
+    decode = None if a.no_decode else decode_phase(a, world, rank, dev, dims, peaks, peak_src)
+    clk.__exit__(None, None, None)
+    clocks = clk.summary()
 
     # ---- CPU baseline: the oracle on a bounded sample, rank 0 at N=1 ----
     cpu = None
@@ -308,19 +346,21 @@ def run_ours(a):
     if rank == 0:
         line = {
             "metric": "MoE-layer tokens/s (prefill T=4096)",
-            "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
-            "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": COMPUTE_DTYPE, "data": "synthetic",
+            "value": round(pre["value"], 1) if pre else None, "unit": "tokens/s", "n_gpus": world,
+            "steps": a.steps, "warmup": a.warmup,
+            "ms_per_step": round(pre["ms_per_step"], 4) if pre else None, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": COMPUTE_DTYPE, "data": "synthetic",
             "config": {"workload": f"prefill T=4096 {'zipf(1.2) router bias' if zipf else 'uniform routing'}",
                        "T": T_PREFILL, "H": dims.H, "E": dims.E, "k": dims.k, "I": dims.I, "I_shared": dims.I_s,
                        "quant": "affine 4-bit, group 64, bf16 scale/bias",
-                       "l2": "4 layers + 4 activation sets cycled (1.9 GB read per cycle) > 126 MB L2",
+                       "l2": f"{a.layers} layers + {a.layers} activation sets cycled "
+                             f"({a.layers * 0.47:.1f} GB read per cycle) > 126 MB L2",
                        "parallelism": "replicas" if world > 1 else "single GPU"},
-            "roofline": roofline,
-            "stage_ms": {k_: round(v, 4) for k_, v in stage_ms.items()},
+            "roofline": pre.get("roofline"),
+            "stage_ms": pre.get("stage_ms"),
             "cpu_baseline": cpu,
-            "e2e": e2e,
-            "gpu_launches": PREFILL_LAUNCHES_PER_STEP * a.steps,
+            "e2e": pre.get("e2e"),
+            "gpu_launches": PREFILL_LAUNCHES_PER_STEP * a.steps if pre else 0,
             "clocks": clocks,
             "decode": decode,
         }

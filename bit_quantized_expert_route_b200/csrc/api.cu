@@ -7,8 +7,48 @@
 #include <cstring>
 #include <mutex>
 
-#include "../../include/moe.h"
+#include "moe.h"
 #include "kernels.h"
+
+namespace moe {
+
+cudaError_t ensure_smem(const void* func, int bytes) {
+  struct Entry {
+    const void* func;
+    int dev;
+    int bytes;
+  };
+  static std::mutex mu;
+  static Entry table[128];
+  static int n = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < n; ++i)
+    if (table[i].func == func && table[i].dev == dev) {
+      if (table[i].bytes >= bytes) return cudaSuccess;
+      e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+      if (e == cudaSuccess) table[i].bytes = bytes;
+      return e;
+    }
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && n < 128) table[n++] = Entry{func, dev, bytes};
+  return e;
+}
+
+// Keeps the device busy for `ns` nanoseconds (bounded by construction), so
+// that every launch a traced call enqueues is already queued when its first
+// stage starts: stage times then measure kernels, not host launch gaps.
+__global__ void busy_wait_kernel(unsigned long long ns) {
+  unsigned long long t0, t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+  do {
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  } while (t - t0 < ns);
+}
+
+}  // namespace moe
 
 namespace {
 
@@ -24,8 +64,8 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 // Byte offsets of every workspace buffer for a call with T tokens.
 struct WsLayout {
-  size_t status, topk_idx, topk_w, counts, offsets, perm, inv_perm, sigma, seg, chunks, n_chunks, active,
-      n_active, h, h_s, Y, x_stage, out_stage, total;
+  size_t status, counter, topk_idx, topk_w, counts, offsets, perm, inv_perm, sigma, seg, chunks, n_chunks,
+      active, n_active, logits, h, h_s, Y, x_stage, out_stage, total;
   int max_chunks;
 };
 
@@ -40,7 +80,8 @@ WsLayout ws_layout(const moe_layer_desc* d, int T) {
   const size_t n = static_cast<size_t>(T) * d->k;
   const int cr = gemm_chunk_rows();
   w.max_chunks = static_cast<int>(n / cr + T / cr + d->E + 2);
-  w.status = take(sizeof(int));
+  w.status = take(256);          // control block: status word, then the small-T routing counter
+  w.counter = w.status + 4;
   w.topk_idx = take(n * 4);
   w.topk_w = take(n * 4);
   w.counts = take(static_cast<size_t>(d->E) * 4);
@@ -48,14 +89,15 @@ WsLayout ws_layout(const moe_layer_desc* d, int T) {
   w.perm = take(n * 4);
   w.inv_perm = take(n * 4);
   w.sigma = take(static_cast<size_t>(T) * 4);
-  w.seg = take(static_cast<size_t>(num_segments(static_cast<int>(n))) * d->E * 4);
+  w.seg = take(static_cast<size_t>(num_segments(T)) * d->E * 4);
   w.chunks = take(static_cast<size_t>(w.max_chunks) * sizeof(Chunk));
   w.n_chunks = take(4);
   w.active = take(static_cast<size_t>(d->E + 1) * 4);
   w.n_active = take(4);
+  w.logits = take(static_cast<size_t>(T <= kDecodeMaxT ? T : 0) * (d->E + 1) * 4);
   w.h = take(n * d->I * 2);
   w.h_s = take(static_cast<size_t>(T) * d->I_shared * 2);
-  w.Y = take((n + T) * d->H * 4);
+  w.Y = take((n + T) * d->H * 2);
   w.x_stage = take(static_cast<size_t>(T) * d->H * 2);
   w.out_stage = take(static_cast<size_t>(T) * d->H * 2);
   w.total = off;
@@ -149,8 +191,16 @@ inline void mark(Tracer* tr, cudaStream_t s) {
 int enqueue_route(const moe_layer_desc* d, const uint16_t* x, int T, const Bufs& b, cudaStream_t s,
                   Tracer* tr = nullptr) {
   mark(tr, s);
+  if (T <= kDecodeMaxT) {
+    const RoutingPtrs rp{b.topk_idx, b.topk_w, b.sigma, b.counts, b.offsets, b.perm, b.inv_perm};
+    const cudaError_t e = launch_route_small(x, layer_ptrs(d), T, d->H, d->I, d->I_shared, d->E, d->k,
+                                             b.at<float>(b.w.logits), b.at<unsigned>(b.w.counter), rp,
+                                             b.at<int32_t>(b.w.active), b.at<int32_t>(b.w.n_active), s);
+    mark(tr, s);
+    return cuda_status(e);
+  }
   cudaError_t e = launch_router(x, d->w_router, d->router_bias, d->w_shared_gate, T, d->H, d->E, d->k,
-                                b.topk_idx, b.topk_w, b.sigma, s);
+                                b.topk_idx, b.topk_w, b.sigma, b.at<int32_t>(b.w.seg), b.at<int>(b.w.status), s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   mark(tr, s);
   e = launch_group(b.topk_idx, T, d->k, d->E, gemm_chunk_rows(), b.at<int32_t>(b.w.seg), b.counts, b.offsets,
@@ -185,7 +235,7 @@ int enqueue_prefill(const moe_layer_desc* d, const uint16_t* x, int T, uint16_t*
   const LayerPtr L = layer_ptrs(d);
   uint16_t* h = b.at<uint16_t>(b.w.h);
   uint16_t* h_s = b.at<uint16_t>(b.w.h_s);
-  float* Y = b.at<float>(b.w.Y);
+  uint16_t* Y = b.at<uint16_t>(b.w.Y);
   int* status = b.at<int>(b.w.status);
   const Chunk* chunks = b.at<Chunk>(b.w.chunks);
   const int32_t* n_chunks = b.at<int32_t>(b.w.n_chunks);
@@ -297,7 +347,7 @@ int moe_route_static(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_
     off += align_up(bytes);
     return o;
   };
-  const size_t o_seg = take(static_cast<size_t>(num_segments(static_cast<int>(n))) * layer->E * 4);
+  const size_t o_seg = take(static_cast<size_t>(num_segments(T)) * layer->E * 4);
   const size_t o_chunks = take(static_cast<size_t>(max_chunks) * sizeof(Chunk));
   const size_t o_nchunks = take(4);
   const size_t o_active = take(static_cast<size_t>(layer->E + 1) * 4);
@@ -311,7 +361,8 @@ int moe_route_static(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   float* sigma = r->sigma ? r->sigma : reinterpret_cast<float*>(b + o_sigma);
   cudaError_t e = launch_router(x, layer->w_router, layer->router_bias, layer->w_shared_gate, T, layer->H,
-                                layer->E, layer->k, r->topk_idx, r->topk_w, sigma, s);
+                                layer->E, layer->k, r->topk_idx, r->topk_w, sigma, reinterpret_cast<int32_t*>(b + o_seg),
+                                nullptr, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   e = launch_group(r->topk_idx, T, layer->k, layer->E, cr, reinterpret_cast<int32_t*>(b + o_seg), r->counts,
                    r->offsets, r->perm, r->inv_perm, reinterpret_cast<Chunk*>(b + o_chunks),
@@ -352,6 +403,8 @@ int moe_forward_profiled(const moe_layer_desc* layer, const moe_bf16* x, int T, 
   if (st != MOE_OK) return st;
   const Bufs b = resolve(layer, T, ws, nullptr);
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  busy_wait_kernel<<<1, 32, 0, s>>>(300000ull);     // 0.3 ms: the host enqueues the stages meanwhile
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   Tracer tr;
   for (int i = 0; i < 8; ++i)
     if (cudaEventCreate(&tr.ev[i]) != cudaSuccess) {

@@ -6,9 +6,10 @@ namespace moe {
 
 // out_t = bf16( sum_{j=0..k-1} w[t,j] * Y[inv_perm[t*k+j]]  +  sigma_t * Y[T*k + t] )
 // in FP32, in exactly that order, with no atomics: every token's sum is formed
-// by one thread per 8 columns, so the result is bitwise reproducible.
+// by one thread per 8 columns, so the result is bitwise reproducible.  Y (the
+// experts' down-projection rows) is stored as bf16.
 __global__ void __launch_bounds__(256) combine_kernel(
-    const float* __restrict__ Y, const int32_t* __restrict__ inv_perm, const float* __restrict__ topk_w,
+    const uint16_t* __restrict__ Y, const int32_t* __restrict__ inv_perm, const float* __restrict__ topk_w,
     const float* __restrict__ sigma, int T, int k, int H, uint16_t* __restrict__ out) {
   const int t = blockIdx.x;
   int pos[kMaxK];
@@ -27,20 +28,18 @@ __global__ void __launch_bounds__(256) combine_kernel(
 #pragma unroll
     for (int j = 0; j < kMaxK; ++j) {
       if (j < k) {
-        const float4* y = reinterpret_cast<const float4*>(Y + static_cast<size_t>(pos[j]) * H + c);
-        const float4 a = y[0], b = y[1];
-        acc[0] = fmaf(w[j], a.x, acc[0]); acc[1] = fmaf(w[j], a.y, acc[1]);
-        acc[2] = fmaf(w[j], a.z, acc[2]); acc[3] = fmaf(w[j], a.w, acc[3]);
-        acc[4] = fmaf(w[j], b.x, acc[4]); acc[5] = fmaf(w[j], b.y, acc[5]);
-        acc[6] = fmaf(w[j], b.z, acc[6]); acc[7] = fmaf(w[j], b.w, acc[7]);
+        const uint4 y = *reinterpret_cast<const uint4*>(Y + static_cast<size_t>(pos[j]) * H + c);
+        acc[0] = fmaf(w[j], bf16_lo(y.x), acc[0]); acc[1] = fmaf(w[j], bf16_hi(y.x), acc[1]);
+        acc[2] = fmaf(w[j], bf16_lo(y.y), acc[2]); acc[3] = fmaf(w[j], bf16_hi(y.y), acc[3]);
+        acc[4] = fmaf(w[j], bf16_lo(y.z), acc[4]); acc[5] = fmaf(w[j], bf16_hi(y.z), acc[5]);
+        acc[6] = fmaf(w[j], bf16_lo(y.w), acc[6]); acc[7] = fmaf(w[j], bf16_hi(y.w), acc[7]);
       }
     }
-    const float4* ys = reinterpret_cast<const float4*>(Y + shared_row * H + c);
-    const float4 a = ys[0], b = ys[1];
-    acc[0] = fmaf(sg, a.x, acc[0]); acc[1] = fmaf(sg, a.y, acc[1]);
-    acc[2] = fmaf(sg, a.z, acc[2]); acc[3] = fmaf(sg, a.w, acc[3]);
-    acc[4] = fmaf(sg, b.x, acc[4]); acc[5] = fmaf(sg, b.y, acc[5]);
-    acc[6] = fmaf(sg, b.z, acc[6]); acc[7] = fmaf(sg, b.w, acc[7]);
+    const uint4 ys = *reinterpret_cast<const uint4*>(Y + shared_row * H + c);
+    acc[0] = fmaf(sg, bf16_lo(ys.x), acc[0]); acc[1] = fmaf(sg, bf16_hi(ys.x), acc[1]);
+    acc[2] = fmaf(sg, bf16_lo(ys.y), acc[2]); acc[3] = fmaf(sg, bf16_hi(ys.y), acc[3]);
+    acc[4] = fmaf(sg, bf16_lo(ys.z), acc[4]); acc[5] = fmaf(sg, bf16_hi(ys.z), acc[5]);
+    acc[6] = fmaf(sg, bf16_lo(ys.w), acc[6]); acc[7] = fmaf(sg, bf16_hi(ys.w), acc[7]);
     uint4 o;
     o.x = pack_bf16x2(acc[0], acc[1]); o.y = pack_bf16x2(acc[2], acc[3]);
     o.z = pack_bf16x2(acc[4], acc[5]); o.w = pack_bf16x2(acc[6], acc[7]);
@@ -82,7 +81,7 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const uint16_t* __restrict
   }
 }
 
-cudaError_t launch_combine(const float* Y, const int32_t* inv_perm, const float* topk_w, const float* sigma,
+cudaError_t launch_combine(const uint16_t* Y, const int32_t* inv_perm, const float* topk_w, const float* sigma,
                            int T, int k, int H, uint16_t* out, cudaStream_t s) {
   combine_kernel<<<T, 256, 0, s>>>(Y, inv_perm, topk_w, sigma, T, k, H, out);
   return cudaGetLastError();

@@ -1,27 +1,41 @@
 // Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05, sm_100a)
-// with the affine 4-bit weights rebuilt tile by tile in shared memory.
+// with the affine 4-bit weights rebuilt tile by tile on chip.
 //
 // The write-ups this layer follows ("Perplexity's Lily: ...", sections "The
 // Model" and "How It Works: Prefill and Decode Strategies") reconstruct the
 // 4-bit weights one tile at a time inside the grouped expert GEMM, multiply in
-// bf16 and accumulate in FP32, never writing dense weights to memory.  Here a
-// tile is 128 weight rows x 64 inputs (exactly one quantisation group), the
-// FP32 accumulators live in tensor memory, and the expert's tokens form the
-// MMA's N dimension ("weights as M, tokens as N"), so a small expert group
-// wastes little work.
+// bf16 and accumulate in FP32, never writing dense weights to memory.  Here:
 //
-// One persistent CTA per SM walks the device-built unit list:
-//   unit = (chunk of <= 128 rows of one expert) x (block of 128 weight rows)
-// Warp roles (288 threads):
-//   warps 0-3  dequantise the packed tile of each stage into bf16 (128-byte
-//              swizzled K-major layout) and, after a unit's last stage, run
-//              the epilogue from tensor memory (lane quadrant = warp index);
-//   warps 4-7  loaders: cp.async gathers of the unit's token rows (B operand),
-//              the packed 4-bit words and the group scales / biases;
-//   warp 8     allocates tensor memory; one lane issues tcgen05.mma.
-// kGateUp = true: A = {W_gate, W_up} rows, two accumulators, epilogue
-//   h = bf16(silu(g) * u).  kGateUp = false: A = W_down rows, one
-//   accumulator, epilogue Y = acc (FP32).
+// * A tile is 128 weight rows x 64 inputs (exactly one quantisation group).
+//   The packed words of each tile (128 rows x 32 B) arrive by TMA into a deep
+//   shared-memory ring, the group scales / biases 8 groups at a time; dequant
+//   warps rebuild bf16(scale * q + bias) and store the tile into tensor
+//   memory, where the MMA reads it as its A operand.  The dense tile never
+//   touches shared memory.
+// * The expert's tokens are the MMA's N dimension (16..128 per chunk), staged
+//   in shared memory in the 128-byte swizzled K-major layout: gathered with
+//   cp.async (gate/up: rows of x picked by the permutation) or loaded by TMA
+//   (down: the chunk's rows of h are contiguous).
+// * FP32 accumulators live in tensor memory.  Epilogue warps read them, apply
+//   the epilogue (gate/up: h = bf16(silu(g) * u); down: Y = bf16(acc)), stage
+//   the tile in shared memory, release the accumulator, and only then write
+//   the tile out with coalesced 16-byte stores, overlapping the next unit.
+//
+// One persistent CTA per SM walks the device-built unit list
+//   unit = (chunk of <= 128 rows of one expert) x (block of 128 weight rows).
+// Warp roles (480 threads):
+//   warps 0-7   dequantisers (gate/up: warps 0-3 gate rows, 4-7 up rows;
+//               down: warps 0-3 even stages, 4-7 odd stages); TMEM lane
+//               quadrant = warp % 4 = row / 32
+//   warps 8-11  epilogue (lane quadrant = warp % 4)
+//   warp 12     token tiles (cp.async gathers, or one lane issuing TMA)
+//   warp 13     one lane issues the TMA loads of packed tiles and scales
+//   warp 14     tensor-memory allocation; one lane issues tcgen05.mma
+// Tensor memory (512 columns): gate/up = one accumulator pair (gate, up:
+// 2 x 128 columns) + 4 A stages of 64 columns; down = two accumulators of 128
+// columns (double-buffered) + 8 A stages of 32 columns.
+#include <cuda.h>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
@@ -29,52 +43,65 @@
 namespace moe {
 namespace {
 
-constexpr int BM = 128;    // weight rows per tile (MMA M)
-constexpr int BN = 128;    // rows (tokens) per chunk: MMA N <= 128
-constexpr int BK = 64;     // inputs per stage: one quantisation group, one 128-B swizzle row
-constexpr int kThreads = 288;
-constexpr int kMmaWarp = 8;
-constexpr uint32_t kTmemCols = 256;
+constexpr int BM = 128;          // weight rows per tile = TMEM lanes (MMA M)
+constexpr int BN = 128;          // rows (tokens) per chunk: MMA N <= 128
+constexpr int BK = 64;           // inputs per stage: one quantisation group
+constexpr int kBStages = 6;      // token-tile ring
+constexpr int kBLag = 3;         // gather cp.async groups in flight before signalling
+constexpr int kPStages = 8;      // packed-tile ring
+constexpr int kSBlock = 8;       // quantisation groups per scale block (16 B per row)
+constexpr int kThreads = 480;
+constexpr int kEpiWarp0 = 8;
+constexpr int kLoadWarp = 12;
+constexpr int kTmaWarp = 13;
+constexpr int kMmaWarp = 14;
+constexpr uint32_t kTmemCols = 512;
 
 template <bool kGateUp>
 struct Cfg {
-  static constexpr int NA = kGateUp ? 2 : 1;              // weight matrices per stage
-  static constexpr int STAGES = kGateUp ? 3 : 4;
-  static constexpr int LAG = STAGES - 1;                   // loader cp.async groups in flight
-  static constexpr int A_BYTES = BM * BK * 2;              // 16 KB bf16 tile
-  static constexpr int B_BYTES = BN * BK * 2;              // 16 KB bf16 tile
-  static constexpr int P_BYTES = BM * BK / 2;              // 4 KB packed words
-  static constexpr int S_BYTES = BM * 4;                   // 2 groups of scale (or bias) per row
-  static constexpr int STAGE_BYTES = NA * (A_BYTES + P_BYTES + 2 * S_BYTES) + B_BYTES;
-  static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
-  static constexpr int SMEM = BAR_OFF + 256 + 1024;        // barriers + alignment slack
-  // offsets inside a stage
-  static constexpr int OFF_A = 0;                          // NA x A_BYTES
-  static constexpr int OFF_B = NA * A_BYTES;
-  static constexpr int OFF_P = OFF_B + B_BYTES;            // NA x P_BYTES
-  static constexpr int OFF_S = OFF_P + NA * P_BYTES;       // NA x (scales, biases)
+  static constexpr int NA = kGateUp ? 2 : 1;                 // weight matrices per stage
+  static constexpr int ACC_COLS = NA * BN;                    // one accumulator set
+  static constexpr int ACC_BUFS = kGateUp ? 1 : 2;
+  static constexpr int A_COLS = NA * BK / 2;                  // TMEM columns per A stage
+  static constexpr int A_BASE = ACC_BUFS * ACC_COLS;
+  static constexpr int A_STAGES = (static_cast<int>(kTmemCols) - A_BASE) / A_COLS;
+  static constexpr int B_BYTES = BN * BK * 2;                 // 16 KB swizzled token tile
+  static constexpr int P_BYTES = BM * 32;                     // 4 KB packed tile of one matrix
+  static constexpr int S_BYTES = BM * kSBlock * 2;            // 2 KB: 8 groups of scales (or biases)
+  static constexpr int S_SLOT = NA * 2 * S_BYTES;             // scales + biases of every matrix
+  static constexpr int OUT_BYTES = BN * BM * 2;               // epilogue staging tile (bf16)
+  static constexpr int OFF_B = 0;
+  static constexpr int OFF_P = OFF_B + kBStages * B_BYTES;
+  static constexpr int OFF_S = OFF_P + kPStages * NA * P_BYTES;
+  static constexpr int OFF_OUT = OFF_S + 2 * S_SLOT;
+  static constexpr int BAR_OFF = OFF_OUT + OUT_BYTES;
+  static constexpr int SMEM = BAR_OFF + 512 + 1024;           // barriers + alignment slack
+  static constexpr int DQ_PER_STAGE = kGateUp ? 256 : 128;    // dequant threads consuming one stage
 };
 
-struct TcArgs {
+struct alignas(64) TcArgs {
+  CUtensorMap tm_q[2][2];  // packed words: [routed, shared][matrix]
+  CUtensorMap tm_s[2][2];  // scales:       [routed, shared][matrix] (valid when scales_tma)
+  CUtensorMap tm_b[2][2];  // biases
+  CUtensorMap tm_h[2];     // down: token tiles of h [routed, shared]
   Geometry g;
   QMatPtr W0, W1;          // routed stacks: {gate, up} or {down, -}
   QMatPtr S0, S1;          // shared expert: {sh_gate, sh_up} or {sh_down, -}
   const uint16_t* x;       // gate/up: token rows [T, H]
   const int32_t* perm;
-  const uint16_t* h;       // down: routed rows [T*k, I]
-  const uint16_t* h_s;     // down: shared rows [T, Is]
   uint16_t* h_out;         // gate/up output, routed [T*k, I]
   uint16_t* hs_out;        // gate/up output, shared [T, Is]
-  float* Y;                // down output [(T*k + T), H]
+  uint16_t* Y;             // down output, bf16 [(T*k + T), H]
   const Chunk* chunks;
   const int32_t* n_chunks;
   int* status;
+  int scales_tma;          // scale rows are 16-B strided (K % 512 == 0): scales arrive by TMA
 };
 
 struct UnitInfo {
   bool skip;
   bool shared;
-  int e, row0, rows, f0, K, nks;
+  int e, row0, rows, f0, K, nks, wrow;   // wrow: first weight row of the tile in its matrix stack
 };
 
 template <bool kGateUp>
@@ -91,55 +118,91 @@ __device__ __forceinline__ UnitInfo unit_info(const TcArgs& a, int u, int nfb) {
   ui.skip = ui.f0 >= R || ui.rows <= 0;
   ui.K = kGateUp ? a.g.H : Ie;
   ui.nks = ui.K / BK;
+  ui.wrow = (ui.shared ? 0 : ui.e * (kGateUp ? a.g.I : a.g.H)) + ui.f0;
   return ui;
 }
 
-// Row pointer bases (packed words, scales, biases) of weight row `row` of
-// matrix m of the unit.
-struct RowPtr {
-  const uint32_t* q;
-  const uint16_t* s;
-  const uint16_t* b;
+// Walks this CTA's stages in order: (unit, k-step) with global stage and
+// scale-block counts (a scale block starts at every k-step multiple of 8).
+template <bool kGateUp>
+struct StageCursor {
+  int u, ks;
+  uint32_t it, blk;
+  bool done;
+  UnitInfo ui;
+
+  __device__ __forceinline__ void seek_unit(const TcArgs& a, int from, int n_units, int nfb) {
+    for (u = from; u < n_units; u += gridDim.x) {
+      ui = unit_info<kGateUp>(a, u, nfb);
+      if (!ui.skip) {
+        ks = 0;
+        done = false;
+        return;
+      }
+    }
+    done = true;
+  }
+  __device__ __forceinline__ void begin(const TcArgs& a, int n_units, int nfb) {
+    it = 0;
+    blk = 0;
+    seek_unit(a, blockIdx.x, n_units, nfb);
+  }
+  __device__ __forceinline__ void next(const TcArgs& a, int n_units, int nfb) {
+    ++it;
+    if (++ks == ui.nks) seek_unit(a, u + gridDim.x, n_units, nfb);
+    if (!done && ks % kSBlock == 0) ++blk;
+  }
 };
 
 template <bool kGateUp>
-__device__ __forceinline__ RowPtr weight_row(const TcArgs& a, const UnitInfo& ui, int m, int row) {
-  const QMatPtr& W = ui.shared ? (m == 0 ? a.S0 : a.S1) : (m == 0 ? a.W0 : a.W1);
-  const int Ie = ui.shared ? a.g.Is : a.g.I;
-  const size_t rows_per_expert = kGateUp ? static_cast<size_t>(a.g.I) : static_cast<size_t>(a.g.H);
-  const size_t r = (ui.shared ? 0 : static_cast<size_t>(ui.e) * rows_per_expert) + row;
-  (void)Ie;
-  return RowPtr{W.q + r * (ui.K / 8), W.s + r * (ui.K / kGroup), W.b + r * (ui.K / kGroup)};
-}
-
-template <bool kGateUp>
-__global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const TcArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __grid_constant__ TcArgs a) {
   using C = Cfg<kGateUp>;
   extern __shared__ uint8_t smem_raw[];
-  // 1024-B aligned base (the swizzle atoms must start on 1024 B)
   const uint32_t raw_u32 = tc::smem_u32(smem_raw);
-  uint8_t* smem = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
+  uint8_t* smem = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);   // 1024-B aligned swizzle atoms
   const uint32_t sbase = tc::smem_u32(smem);
 
-  uint64_t* full_ld = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);   // [STAGES]
-  uint64_t* full_a = full_ld + C::STAGES;                                 // [STAGES]
-  uint64_t* empty = full_a + C::STAGES;                                   // [STAGES]
-  uint64_t* acc_full = empty + C::STAGES;
-  uint64_t* acc_empty = acc_full + 1;
-  uint64_t* drain = acc_empty + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* full_b = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);   // [kBStages]
+  uint64_t* empty_b = full_b + kBStages;                                // [kBStages]
+  uint64_t* full_p = empty_b + kBStages;                                // [kPStages]
+  uint64_t* empty_p = full_p + kPStages;                                // [kPStages]
+  uint64_t* full_s = empty_p + kPStages;                                // [2]
+  uint64_t* empty_s = full_s + 2;                                       // [2]
+  uint64_t* full_a = empty_s + 2;                                       // [A_STAGES]
+  uint64_t* empty_a = full_a + C::A_STAGES;                             // [A_STAGES]
+  uint64_t* acc_full = empty_a + C::A_STAGES;                           // [ACC_BUFS]
+  uint64_t* acc_empty = acc_full + C::ACC_BUFS;                         // [ACC_BUFS]
+  uint64_t* drain = acc_empty + C::ACC_BUFS;
+  uint64_t* epi_sync = drain + 1;                                       // [2] staging written / copied out
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epi_sync + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool b_by_tma = !kGateUp;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::STAGES; ++s) {
-      tc::mbar_init(&full_ld[s], 128);
-      tc::mbar_init(&full_a[s], 128);
-      tc::mbar_init(&empty[s], 1);
+    for (int s = 0; s < kBStages; ++s) {
+      tc::mbar_init(&full_b[s], b_by_tma ? 1 : 32);
+      tc::mbar_init(&empty_b[s], 1);
     }
-    tc::mbar_init(acc_full, 1);
-    tc::mbar_init(acc_empty, 128);
+    for (int s = 0; s < kPStages; ++s) {
+      tc::mbar_init(&full_p[s], 1);
+      tc::mbar_init(&empty_p[s], C::DQ_PER_STAGE);
+    }
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(&full_s[s], 1);
+      tc::mbar_init(&empty_s[s], 256);
+    }
+    for (int s = 0; s < C::A_STAGES; ++s) {
+      tc::mbar_init(&full_a[s], C::DQ_PER_STAGE);
+      tc::mbar_init(&empty_a[s], 1);
+    }
+    for (int b = 0; b < C::ACC_BUFS; ++b) {
+      tc::mbar_init(&acc_full[b], 1);
+      tc::mbar_init(&acc_empty[b], 128);
+    }
     tc::mbar_init(drain, 1);
+    tc::mbar_init(&epi_sync[0], 128);
+    tc::mbar_init(&epi_sync[1], 128);
     *abort_flag = 0;
     tc::fence_barrier_init();
   }
@@ -153,139 +216,248 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const TcAr
   const int n_units = *a.n_chunks * nfb;
   const int Tk = a.g.T * a.g.k;
 
-  if (warp >= 4 && warp < 8) {
-    // ------------------------------------------------------------ loaders
-    const int r = threadIdx.x - 128;         // tile row owned by this thread
+  if (warp < kEpiWarp0) {
+    // ------------------------------------------------------- dequantisers
+    const int r = threadIdx.x & 127;                 // weight row of the tile == TMEM lane
+    const int set = warp >> 2;                       // gate/up: matrix; down: stage parity
+    const int m = kGateUp ? set : 0;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const int psw = (r >> 2) & 1;                    // 32-byte swizzle of the packed tile rows
+    auto mine = [&](uint32_t it) { return kGateUp || static_cast<int>(it & 1u) == set; };
+    StageCursor<kGateUp> cur;
+    cur.begin(a, n_units, nfb);
+    while (!cur.done && !mine(cur.it)) cur.next(a, n_units, nfb);
+    bool ok = true;
+    uint32_t held_blk = 0xffffffffu;                 // scale block this thread still holds
+    while (!cur.done && ok) {
+      const uint32_t it = cur.it;
+      const int ks = cur.ks;
+      // scales of this stage: from the TMA'd block, or straight from global
+      uint32_t sv, bv;
+      if (a.scales_tma) {
+        if (cur.blk != held_blk) {
+          if (held_blk != 0xffffffffu) {
+            tc::fence_proxy_async_smem();            // generic reads of the block before its TMA refill
+            tc::mbar_arrive(&empty_s[held_blk & 1u]);
+          }
+          held_blk = cur.blk;
+          if (!tc::mbar_wait(&full_s[held_blk & 1u], (held_blk >> 1) & 1u, abort_flag, a.status)) {
+            ok = false;
+            break;
+          }
+        }
+        const uint16_t* sb = reinterpret_cast<const uint16_t*>(smem + C::OFF_S + (held_blk & 1u) * C::S_SLOT +
+                                                               m * 2 * C::S_BYTES + r * 16);
+        sv = sb[ks % kSBlock];
+        bv = sb[C::S_BYTES / 2 + ks % kSBlock];
+      } else {
+        const QMatPtr& W = cur.ui.shared ? (m == 0 ? a.S0 : a.S1) : (m == 0 ? a.W0 : a.W1);
+        const size_t row = static_cast<size_t>(cur.ui.wrow + r);
+        sv = __ldg(W.s + row * (cur.ui.K / kGroup) + ks);
+        bv = __ldg(W.b + row * (cur.ui.K / kGroup) + ks);
+      }
+      // packed words of this stage's tile row
+      const int sp = static_cast<int>(it % kPStages);
+      if (!tc::mbar_wait(&full_p[sp], (it / kPStages) & 1u, abort_flag, a.status)) {
+        ok = false;
+        break;
+      }
+      const uint8_t* prow = smem + C::OFF_P + (sp * C::NA + m) * C::P_BYTES + r * 32;
+      const uint4 q0 = *reinterpret_cast<const uint4*>(prow + (psw << 4));
+      const uint4 q1 = *reinterpret_cast<const uint4*>(prow + ((psw ^ 1) << 4));
+      __nv_bfloat162 s2, b2;
+      *reinterpret_cast<uint32_t*>(&s2) = sv | (sv << 16);
+      *reinterpret_cast<uint32_t*>(&b2) = bv | (bv << 16);
+      const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+      uint32_t cols[32];
+#pragma unroll
+      for (int wd = 0; wd < 8; ++wd) {
+        const uint4 d = tc::dequant8(words[wd], s2, b2);
+        cols[4 * wd + 0] = d.x;
+        cols[4 * wd + 1] = d.y;
+        cols[4 * wd + 2] = d.z;
+        cols[4 * wd + 3] = d.w;
+      }
+      // Hand the slot back only once its words are consumed.  The next TMA
+      // write into it is an async-proxy access following these generic-proxy
+      // reads: the proxy fence orders the two (the mbarrier alone does not).
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(&empty_p[sp]);
+      const int sa = static_cast<int>(it % C::A_STAGES);
+      if (!tc::mbar_wait(&empty_a[sa], ((it / C::A_STAGES) & 1u) ^ 1u, abort_flag, a.status)) {
+        ok = false;
+        break;
+      }
+      tc::tc_fence_after();
+      tc::tmem_st32(lane_base + C::A_BASE + sa * C::A_COLS + m * 32, cols);
+      tc::tmem_wait_st();
+      tc::tc_fence_before();
+      tc::mbar_arrive(&full_a[sa]);
+      cur.next(a, n_units, nfb);
+      while (!cur.done && !mine(cur.it)) cur.next(a, n_units, nfb);
+    }
+    if (ok && a.scales_tma && held_blk != 0xffffffffu) {
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(&empty_s[held_blk & 1u]);
+    }
+  } else if (warp < kLoadWarp) {
+    // ----------------------------------------------------------- epilogue
+    const int q = warp & 3;
+    const int r = q * 32 + lane;                     // weight row == TMEM lane == output feature in tile
+    const int et = threadIdx.x - kEpiWarp0 * 32;     // 0..127
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    uint16_t* stage = reinterpret_cast<uint16_t*>(smem + C::OFF_OUT);   // [BN tokens][BM features]
+    uint32_t tt = 0;
+    for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+      const UnitInfo ui = unit_info<kGateUp>(a, u, nfb);
+      if (ui.skip) continue;
+      const int buf = static_cast<int>(tt % C::ACC_BUFS);
+      if (!tc::mbar_wait(&acc_full[buf], (tt / C::ACC_BUFS) & 1u, abort_flag, a.status)) break;
+      tc::tc_fence_after();
+      const uint32_t acc = lane_base + buf * C::ACC_COLS;
+      for (int n0 = 0; n0 < ui.rows; n0 += 16) {
+        float v0[16];
+        tc::tmem_ld16(acc + n0, v0);
+        if (kGateUp) {
+          float v1[16];
+          tc::tmem_ld16(acc + BN + n0, v1);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float g = v0[j];
+            stage[(n0 + j) * BM + r] = float_to_bf16_bits(__fdividef(g * v1[j], 1.0f + __expf(-g)));
+          }
+        } else {
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) stage[(n0 + j) * BM + r] = float_to_bf16_bits(v0[j]);
+        }
+      }
+      // accumulator drained: hand it back to the MMA before writing the tile out
+      tc::tc_fence_before();
+      tc::mbar_arrive(&acc_empty[buf]);
+      tc::mbar_arrive(&epi_sync[0]);
+      if (!tc::mbar_wait(&epi_sync[0], tt & 1u, abort_flag, a.status)) break;
+      // coalesced copy-out: each token row of the tile is BM contiguous outputs (256 B)
+      const int chunks = ui.rows * (BM / 8);
+      for (int i = et; i < chunks; i += 128) {
+        const int n = i / (BM / 8), c = i % (BM / 8);
+        const int R = ui.row0 + n;
+        uint16_t* dst;
+        if (kGateUp)
+          dst = ui.shared ? a.hs_out + static_cast<size_t>(R - Tk) * a.g.Is : a.h_out + static_cast<size_t>(R) * a.g.I;
+        else
+          dst = a.Y + static_cast<size_t>(R) * a.g.H;
+        *reinterpret_cast<uint4*>(dst + ui.f0 + c * 8) = *reinterpret_cast<const uint4*>(stage + n * BM + c * 8);
+      }
+      tc::mbar_arrive(&epi_sync[1]);                     // the staging tile is free again
+      if (!tc::mbar_wait(&epi_sync[1], tt & 1u, abort_flag, a.status)) break;
+      ++tt;
+    }
+  } else if (warp == kLoadWarp) {
+    // ------------------------------------------------------- token tiles
     uint32_t it = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const UnitInfo ui = unit_info<kGateUp>(a, u, nfb);
       if (ui.skip) continue;
-      // B row source
-      const uint16_t* brow = nullptr;
-      if (r < ui.rows) {
-        const int R = ui.row0 + r;
-        if (kGateUp) {
+      if (b_by_tma) {
+        if (lane == 0) {
+          const void* tm = &a.tm_h[ui.shared ? 1 : 0];
+          const int y = ui.shared ? ui.row0 - Tk : ui.row0;
+          for (int ks = 0; ks < ui.nks; ++ks, ++it) {
+            const int s = static_cast<int>(it % kBStages);
+            if (!tc::mbar_wait(&empty_b[s], ((it / kBStages) & 1u) ^ 1u, abort_flag, a.status)) {
+              ok = false;
+              break;
+            }
+            tc::mbar_arrive_expect_tx(&full_b[s], C::B_BYTES);
+            tc::tma_load_2d(sbase + C::OFF_B + s * C::B_BYTES, tm, ks * BK, y, &full_b[s]);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        it = __shfl_sync(0xffffffffu, it, 0);
+        continue;
+      }
+      const uint16_t* brow[BN / 32];
+#pragma unroll
+      for (int i = 0; i < BN / 32; ++i) {
+        const int rr = lane + i * 32;
+        brow[i] = nullptr;
+        if (rr < ui.rows) {
+          const int R = ui.row0 + rr;
           const int tok = ui.shared ? (R - Tk) : (a.perm[R] / a.g.k);
-          brow = a.x + static_cast<size_t>(tok) * a.g.H;
-        } else {
-          brow = ui.shared ? a.h_s + static_cast<size_t>(R - Tk) * a.g.Is : a.h + static_cast<size_t>(R) * a.g.I;
+          brow[i] = a.x + static_cast<size_t>(tok) * a.g.H;
         }
       }
-      RowPtr wr[2];
-#pragma unroll
-      for (int m = 0; m < C::NA; ++m) wr[m] = weight_row<kGateUp>(a, ui, m, ui.f0 + r);
       for (int ks = 0; ks < ui.nks; ++ks, ++it) {
-        const int s = it % C::STAGES;
-        if (!tc::mbar_wait(&empty[s], ((it / C::STAGES) & 1u) ^ 1u, abort_flag, a.status)) {
+        const int s = static_cast<int>(it % kBStages);
+        if (!tc::mbar_wait(&empty_b[s], ((it / kBStages) & 1u) ^ 1u, abort_flag, a.status)) {
           ok = false;
           break;
         }
-        const uint32_t st = sbase + s * C::STAGE_BYTES;
-        if (brow) {
-          const uint32_t dst = st + C::OFF_B + r * 128;
+        const uint32_t st = sbase + C::OFF_B + s * C::B_BYTES;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) tc::cp_async16(dst + ((c ^ (r & 7)) << 4), brow + ks * BK + c * 8);
-        }
+        for (int i = 0; i < BN / 32; ++i) {
+          if (brow[i]) {
+            const int rr = lane + i * 32;
+            const uint32_t dst = st + rr * 128;
 #pragma unroll
-        for (int m = 0; m < C::NA; ++m) {
-          const uint32_t pd = st + C::OFF_P + m * C::P_BYTES + r * 32;
-          tc::cp_async16(pd, wr[m].q + ks * 8);
-          tc::cp_async16(pd + 16, wr[m].q + ks * 8 + 4);
-          const uint32_t sd = st + C::OFF_S + m * 2 * C::S_BYTES + r * 4;
-          const int gpair = ks & ~1;
-          asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(sd), "l"(wr[m].s + gpair) : "memory");
-          asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(sd + C::S_BYTES), "l"(wr[m].b + gpair)
-                       : "memory");
+            for (int c = 0; c < 8; ++c)
+              tc::cp_async16(dst + ((c ^ (rr & 7)) << 4), brow[i] + ks * BK + c * 8);
+          }
         }
         tc::cp_async_commit();
-        if (it >= static_cast<uint32_t>(C::LAG)) {
-          tc::cp_async_wait<C::LAG>();
+        if (it >= static_cast<uint32_t>(kBLag)) {
+          tc::cp_async_wait<kBLag>();
           tc::fence_proxy_async_smem();
-          tc::mbar_arrive(&full_ld[(it - C::LAG) % C::STAGES]);
+          tc::mbar_arrive(&full_b[(it - kBLag) % kBStages]);
         }
       }
     }
-    tc::cp_async_wait_all();
-    tc::fence_proxy_async_smem();
-    if (ok) {
-      const uint32_t first = it > static_cast<uint32_t>(C::LAG) ? it - C::LAG : 0u;
-      for (uint32_t j = first; j < it; ++j) tc::mbar_arrive(&full_ld[j % C::STAGES]);
+    if (!b_by_tma) {
+      tc::cp_async_wait_all();
+      tc::fence_proxy_async_smem();
+      if (ok) {
+        const uint32_t first = it > static_cast<uint32_t>(kBLag) ? it - kBLag : 0u;
+        for (uint32_t j = first; j < it; ++j) tc::mbar_arrive(&full_b[j % kBStages]);
+      }
     }
-  } else if (warp < 4) {
-    // ------------------------------------------------- dequant + epilogue
-    const int r = threadIdx.x;               // tile row == TMEM lane
-    uint32_t it = 0, tt = 0;
-    bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const UnitInfo ui = unit_info<kGateUp>(a, u, nfb);
-      if (ui.skip) continue;
-      for (int ks = 0; ks < ui.nks; ++ks, ++it) {
-        const int s = it % C::STAGES;
-        if (!tc::mbar_wait(&full_ld[s], (it / C::STAGES) & 1u, abort_flag, a.status)) {
-          ok = false;
-          break;
-        }
-        uint8_t* st = smem + s * C::STAGE_BYTES;
+  } else if (warp == kTmaWarp) {
+    // ----------------------------------------- packed tiles and scales (TMA)
+    if (lane == 0) {
+      StageCursor<kGateUp> cur;
+      cur.begin(a, n_units, nfb);
+      uint32_t last_blk = 0xffffffffu;
+      while (!cur.done) {
+        const int side = cur.ui.shared ? 1 : 0;
+        if (a.scales_tma && cur.blk != last_blk) {
+          last_blk = cur.blk;
+          const int ss = static_cast<int>(cur.blk & 1u);
+          if (!tc::mbar_wait(&empty_s[ss], ((cur.blk >> 1) & 1u) ^ 1u, abort_flag, a.status)) break;
+          tc::fence_proxy_async_smem();
+          tc::mbar_arrive_expect_tx(&full_s[ss], C::S_SLOT);
+          const uint32_t sdst = sbase + C::OFF_S + ss * C::S_SLOT;
 #pragma unroll
-        for (int m = 0; m < C::NA; ++m) {
-          const uint4* pk = reinterpret_cast<const uint4*>(st + C::OFF_P + m * C::P_BYTES + r * 32);
-          const uint4 w0 = pk[0], w1 = pk[1];
-          const uint16_t* sb = reinterpret_cast<const uint16_t*>(st + C::OFF_S + m * 2 * C::S_BYTES + r * 4);
-          const uint16_t sv = sb[ks & 1];
-          const uint16_t bv = sb[C::S_BYTES / 2 + (ks & 1)];
-          __nv_bfloat162 s2, b2;
-          *reinterpret_cast<uint32_t*>(&s2) = static_cast<uint32_t>(sv) | (static_cast<uint32_t>(sv) << 16);
-          *reinterpret_cast<uint32_t*>(&b2) = static_cast<uint32_t>(bv) | (static_cast<uint32_t>(bv) << 16);
-          const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-          uint8_t* arow = st + C::OFF_A + m * C::A_BYTES + r * 128;
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(arow + ((c ^ (r & 7)) << 4)) = tc::dequant8(words[c], s2, b2);
-        }
-        tc::fence_proxy_async_smem();
-        tc::mbar_arrive(&full_a[s]);
-      }
-      if (!ok) break;
-      // epilogue: accumulators of this unit
-      if (!tc::mbar_wait(acc_full, tt & 1u, abort_flag, a.status)) {
-        ok = false;
-        break;
-      }
-      tc::tc_fence_after();
-      const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-      const int feat = ui.f0 + r;
-      for (int n0 = 0; n0 < ui.rows; n0 += 16) {
-        float v0[16];
-        tc::tmem_ld16(lane_base + n0, v0);
-        if (kGateUp) {
-          float v1[16];
-          tc::tmem_ld16(lane_base + BN + n0, v1);
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int n = n0 + j;
-            if (n < ui.rows) {
-              const int R = ui.row0 + n;
-              uint16_t* dst = ui.shared ? a.hs_out + static_cast<size_t>(R - Tk) * a.g.Is
-                                        : a.h_out + static_cast<size_t>(R) * a.g.I;
-              dst[feat] = float_to_bf16_bits(silu(v0[j]) * v1[j]);
-            }
-          }
-        } else {
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int n = n0 + j;
-            if (n < ui.rows) a.Y[static_cast<size_t>(ui.row0 + n) * a.g.H + feat] = v0[j];
+          for (int mm = 0; mm < C::NA; ++mm) {
+            tc::tma_load_2d(sdst + mm * 2 * C::S_BYTES, &a.tm_s[side][mm], cur.ks, cur.ui.wrow, &full_s[ss]);
+            tc::tma_load_2d(sdst + mm * 2 * C::S_BYTES + C::S_BYTES, &a.tm_b[side][mm], cur.ks, cur.ui.wrow,
+                            &full_s[ss]);
           }
         }
+        const int sp = static_cast<int>(cur.it % kPStages);
+        if (!tc::mbar_wait(&empty_p[sp], ((cur.it / kPStages) & 1u) ^ 1u, abort_flag, a.status)) break;
+        tc::fence_proxy_async_smem();   // consumers' generic reads of the slot precede this async-proxy refill
+        tc::mbar_arrive_expect_tx(&full_p[sp], C::NA * C::P_BYTES);
+#pragma unroll
+        for (int mm = 0; mm < C::NA; ++mm)
+          tc::tma_load_2d(sbase + C::OFF_P + (sp * C::NA + mm) * C::P_BYTES, &a.tm_q[side][mm], cur.ks * 8,
+                          cur.ui.wrow, &full_p[sp]);
+        cur.next(a, n_units, nfb);
       }
-      tc::tc_fence_before();
-      tc::mbar_arrive(acc_empty);
-      ++tt;
     }
-  } else if (warp == kMmaWarp) {
+    __syncwarp();
+  } else {
     // ---------------------------------------------------------------- MMA
     if (lane == 0) {
       uint32_t it = 0, tt = 0;
@@ -295,35 +467,34 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const TcAr
         if (ui.skip) continue;
         const int n_mma = max(16, (ui.rows + 15) & ~15);
         const uint32_t idesc = tc::idesc_bf16(BM, n_mma);
-        if (!tc::mbar_wait(acc_empty, (tt & 1u) ^ 1u, abort_flag, a.status)) {
-          ok = false;
-          break;
-        }
+        const int buf = static_cast<int>(tt % C::ACC_BUFS);
+        if (!tc::mbar_wait(&acc_empty[buf], ((tt / C::ACC_BUFS) & 1u) ^ 1u, abort_flag, a.status)) break;
         tc::tc_fence_after();
+        const uint32_t acc = tmem + buf * C::ACC_COLS;
         for (int ks = 0; ks < ui.nks; ++ks, ++it) {
-          const int s = it % C::STAGES;
-          const uint32_t par = (it / C::STAGES) & 1u;
-          if (!tc::mbar_wait(&full_ld[s], par, abort_flag, a.status) ||
-              !tc::mbar_wait(&full_a[s], par, abort_flag, a.status)) {
+          const int sb = static_cast<int>(it % kBStages);
+          const int sa = static_cast<int>(it % C::A_STAGES);
+          if (!tc::mbar_wait(&full_b[sb], (it / kBStages) & 1u, abort_flag, a.status) ||
+              !tc::mbar_wait(&full_a[sa], (it / C::A_STAGES) & 1u, abort_flag, a.status)) {
             ok = false;
             break;
           }
           tc::tc_fence_after();
-          const uint32_t st = sbase + s * C::STAGE_BYTES;
+          const uint32_t bst = sbase + C::OFF_B + sb * C::B_BYTES;
+          const uint32_t ast = tmem + C::A_BASE + sa * C::A_COLS;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t bdesc = tc::sdesc_sw128(st + C::OFF_B + kk * 32);
-            const uint32_t acc = (ks > 0 || kk > 0) ? 1u : 0u;
+            const uint64_t bdesc = tc::sdesc_sw128(bst + kk * 32);
+            const uint32_t accum = (ks > 0 || kk > 0) ? 1u : 0u;
 #pragma unroll
-            for (int m = 0; m < C::NA; ++m) {
-              const uint64_t adesc = tc::sdesc_sw128(st + C::OFF_A + m * C::A_BYTES + kk * 32);
-              tc::mma_bf16_ss(tmem + m * BN, adesc, bdesc, idesc, acc);
-            }
+            for (int mm = 0; mm < C::NA; ++mm)
+              tc::mma_bf16_ts(acc + mm * BN, ast + mm * 32 + kk * 8, bdesc, idesc, accum);
           }
-          tc::mma_commit(&empty[s]);
+          tc::mma_commit(&empty_a[sa]);
+          tc::mma_commit(&empty_b[sb]);
         }
         if (!ok) break;
-        tc::mma_commit(acc_full);
+        tc::mma_commit(&acc_full[buf]);
         ++tt;
       }
       // every issued MMA has finished before tensor memory is released
@@ -338,6 +509,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const TcAr
   if (warp == kMmaWarp) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
+// ----------------------------------------------------------------- host ---
+
 int num_sms() {
   static int n = 0;
   if (n == 0) {
@@ -347,6 +520,53 @@ int num_sms() {
     if (n <= 0) n = 148;
   }
   return n;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D map over a row-major [rows, cols] array of `esize`-byte elements, box
+// [box_rows, box_cols].
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* base, uint64_t cols, uint64_t rows,
+              uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * static_cast<uint64_t>(esize)};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Maps of one affine 4-bit matrix stack [rows, K]: packed words (box 128 rows
+// x 8 words, 32-B swizzle) and, when the scale rows are 16-B strided, scales
+// and biases (box 128 rows x 8 groups).
+bool make_qmat_maps(TcArgs& a, int side, int m, const QMatPtr& W, int rows, int K) {
+  if (!make_map(&a.tm_q[side][m], CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, W.q, K / 8, rows, 8, BM,
+                CU_TENSOR_MAP_SWIZZLE_32B))
+    return false;
+  if (a.scales_tma) {
+    if (!make_map(&a.tm_s[side][m], CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, W.s, K / kGroup, rows, kSBlock, BM,
+                  CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map(&a.tm_b[side][m], CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, W.b, K / kGroup, rows, kSBlock, BM,
+                  CU_TENSOR_MAP_SWIZZLE_NONE))
+      return false;
+  }
+  return true;
 }
 
 }  // namespace
@@ -369,9 +589,12 @@ cudaError_t launch_gateup(const Geometry& g, const LayerPtr& L, const uint16_t* 
   a.chunks = chunks;
   a.n_chunks = n_chunks;
   a.status = status;
+  a.scales_tma = (g.H % (kGroup * kSBlock)) == 0;
+  if (!make_qmat_maps(a, 0, 0, L.gate, g.E * g.I, g.H) || !make_qmat_maps(a, 0, 1, L.up, g.E * g.I, g.H) ||
+      !make_qmat_maps(a, 1, 0, L.sh_gate, g.Is, g.H) || !make_qmat_maps(a, 1, 1, L.sh_up, g.Is, g.H))
+    return cudaErrorInvalidValue;
   using C = Cfg<true>;
-  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       C::SMEM);
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(grouped_gemm_tc_kernel<true>), C::SMEM);
   if (e != cudaSuccess) return e;
   const int nfb = max(g.I, g.Is) / BM;
   const int grid = max(1, min(max_chunks * nfb, num_sms()));
@@ -381,22 +604,25 @@ cudaError_t launch_gateup(const Geometry& g, const LayerPtr& L, const uint16_t* 
 
 cudaError_t launch_down(const Geometry& g, const LayerPtr& L, const uint16_t* h, const uint16_t* h_s,
                         const Chunk* chunks, const int32_t* n_chunks, int max_chunks,
-                        float* Y, int* status, cudaStream_t s) {
+                        uint16_t* Y, int* status, cudaStream_t s) {
   TcArgs a{};
   a.g = g;
   a.W0 = L.down;
   a.W1 = L.down;
   a.S0 = L.sh_down;
   a.S1 = L.sh_down;
-  a.h = h;
-  a.h_s = h_s;
   a.Y = Y;
   a.chunks = chunks;
   a.n_chunks = n_chunks;
   a.status = status;
+  a.scales_tma = (g.I % (kGroup * kSBlock)) == 0 && (g.Is % (kGroup * kSBlock)) == 0;
+  if (!make_qmat_maps(a, 0, 0, L.down, g.E * g.H, g.I) || !make_qmat_maps(a, 1, 0, L.sh_down, g.H, g.Is) ||
+      !make_map(&a.tm_h[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, g.I, static_cast<uint64_t>(g.T) * g.k, BK, BN,
+                CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&a.tm_h[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h_s, g.Is, g.T, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
   using C = Cfg<false>;
-  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       C::SMEM);
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(grouped_gemm_tc_kernel<false>), C::SMEM);
   if (e != cudaSuccess) return e;
   const int nfb = g.H / BM;
   const int grid = max(1, min(max_chunks * nfb, num_sms()));

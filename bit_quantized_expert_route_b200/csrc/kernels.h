@@ -26,11 +26,40 @@ struct LayerPtr {
   const uint16_t* w_sg;
 };
 
-// route.cu
+// Routing outputs of one call.
+struct RoutingPtrs {
+  int32_t* topk_idx;
+  float* topk_w;
+  float* sigma;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* perm;
+  int32_t* inv_perm;
+};
+
+// api.cu: raise a kernel's dynamic shared-memory limit once per device (and
+// again only if a launch needs more), keeping the attribute call off the
+// per-launch path.
+cudaError_t ensure_smem(const void* func, int bytes);
+
+// route_tc.cu: tensor-core router + top-k + shared gate (any T >= 1); also
+// writes seg_counts[ceil(T/128)][E], the expert counts of each 128-token
+// segment of the (token, slot) entries.
+constexpr int kRouteSegTokens = 128;
 cudaError_t launch_router(const uint16_t* x, const uint16_t* w_router, const float* router_bias,
                           const uint16_t* w_sg, int T, int H, int E, int k,
-                          int32_t* topk_idx, float* topk_w, float* sigma, cudaStream_t s);
-int num_segments(int n_entries);
+                          int32_t* topk_idx, float* topk_w, float* sigma, int32_t* seg_counts, int* status,
+                          cudaStream_t s);
+
+// route.cu
+int num_segments(int T);   // 128-token segments of the counting sort
+// T <= 64: router + top-k + shared gate + counting sort + active list in one launch.
+// logits: workspace [T, E+1] FP32; counter: workspace word that must be zero.
+cudaError_t launch_route_small(const uint16_t* x, const LayerPtr& L, int T, int H, int I, int Is, int E, int k,
+                               float* logits, unsigned* counter, const RoutingPtrs& r, int32_t* active,
+                               int32_t* n_active, cudaStream_t s);
+// Second and third pass of the counting sort (seg_scratch holds the router's
+// per-segment counts and is turned into per-segment bases in place).
 cudaError_t launch_group(const int32_t* topk_idx, int T, int k, int E, int chunk_rows,
                          int32_t* seg_scratch, int32_t* counts, int32_t* offsets,
                          int32_t* perm, int32_t* inv_perm, Chunk* chunks, int32_t* n_chunks,
@@ -43,10 +72,10 @@ cudaError_t launch_gateup(const Geometry& g, const LayerPtr& L, const uint16_t* 
                           uint16_t* h, uint16_t* h_s, int* status, cudaStream_t s);
 cudaError_t launch_down(const Geometry& g, const LayerPtr& L, const uint16_t* h, const uint16_t* h_s,
                         const Chunk* chunks, const int32_t* n_chunks, int max_chunks,
-                        float* Y, int* status, cudaStream_t s);
+                        uint16_t* Y, int* status, cudaStream_t s);
 
 // combine.cu
-cudaError_t launch_combine(const float* Y, const int32_t* inv_perm, const float* topk_w, const float* sigma,
+cudaError_t launch_combine(const uint16_t* Y, const int32_t* inv_perm, const float* topk_w, const float* sigma,
                            int T, int k, int H, uint16_t* out, cudaStream_t s);
 cudaError_t launch_rmsnorm(const uint16_t* y, uint16_t* out, int T, int H, float eps, cudaStream_t s);
 

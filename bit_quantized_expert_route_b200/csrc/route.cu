@@ -1,6 +1,6 @@
-// GPU-resident expert routing: router logits, top-k with renormalised softmax
-// weights, the shared-expert gate, and the token-to-expert histogram, prefix
-// sum and stable permutation.  Nothing here synchronises with the host: the
+// GPU-resident expert routing: the token-to-expert histogram, prefix sum and
+// stable permutation, and (for T <= 64) a one-launch router + top-k + sort.
+// The tensor-core router for larger T is in route_tc.cu.  Nothing here synchronises with the host: the
 // group sizes stay on the device and later kernels read them from there
 // ("Perplexity's Lily: ...", section "How It Works: Prefill and Decode
 // Strategies": histogram, prefix scan, scatter and block maps live in one GPU
@@ -11,112 +11,15 @@
 namespace moe {
 
 // ---------------------------------------------------------------------------
-// Router + top-k (SIMT).  One CTA scores TB tokens against all E experts.
-//   l[t,e]   = x_t . W_r[e] + b_e                        (FP32 accumulation)
-//   idx[t,:] = k best by (logit desc, expert index asc)
-//   w[t,j]   = exp(l_j - l_0) / sum_j' exp(l_j' - l_0)
-//   sigma_t  = sigmoid(x_t . w_sg)
-// ---------------------------------------------------------------------------
-template <int TB>
-__global__ void __launch_bounds__(256) router_topk_kernel(
-    const uint16_t* __restrict__ x, const uint16_t* __restrict__ w_router,
-    const float* __restrict__ router_bias, const uint16_t* __restrict__ w_sg,
-    int T, int H, int E, int k,
-    int32_t* __restrict__ topk_idx, float* __restrict__ topk_w, float* __restrict__ sigma) {
-  extern __shared__ uint4 smem_u4[];
-  const int vec = H / 8;                                   // uint4 (8 bf16) per row
-  uint4* xs = smem_u4;                                      // [TB][vec]
-  float* lg = reinterpret_cast<float*>(xs + TB * vec);      // [TB][E]
-  const int t0 = blockIdx.x * TB;
-  const int nt = min(TB, T - t0);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
-
-  for (int i = threadIdx.x; i < TB * vec; i += blockDim.x) {
-    const int r = i / vec, c = i - r * vec;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (r < nt) v = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t0 + r) * H)[c];
-    xs[i] = v;
-  }
-  __syncthreads();
-
-  for (int e = warp; e < E; e += nwarps) {
-    float acc[TB];
-#pragma unroll
-    for (int r = 0; r < TB; ++r) acc[r] = 0.f;
-    const uint4* wr = reinterpret_cast<const uint4*>(w_router + static_cast<size_t>(e) * H);
-    for (int c = lane; c < vec; c += 32) {
-      const uint4 wv = __ldg(wr + c);
-      const float w0 = bf16_lo(wv.x), w1 = bf16_hi(wv.x), w2 = bf16_lo(wv.y), w3 = bf16_hi(wv.y);
-      const float w4 = bf16_lo(wv.z), w5 = bf16_hi(wv.z), w6 = bf16_lo(wv.w), w7 = bf16_hi(wv.w);
-#pragma unroll
-      for (int r = 0; r < TB; ++r) {
-        const uint4 xv = xs[r * vec + c];
-        float a = acc[r];
-        a = fmaf(bf16_lo(xv.x), w0, a); a = fmaf(bf16_hi(xv.x), w1, a);
-        a = fmaf(bf16_lo(xv.y), w2, a); a = fmaf(bf16_hi(xv.y), w3, a);
-        a = fmaf(bf16_lo(xv.z), w4, a); a = fmaf(bf16_hi(xv.z), w5, a);
-        a = fmaf(bf16_lo(xv.w), w6, a); a = fmaf(bf16_hi(xv.w), w7, a);
-        acc[r] = a;
-      }
-    }
-    const float b = router_bias ? router_bias[e] : 0.f;
-#pragma unroll
-    for (int r = 0; r < TB; ++r) {
-      const float s = warp_sum(acc[r]);
-      if (lane == 0) lg[r * E + e] = s + b;
-    }
-  }
-  __syncthreads();
-
-  for (int r = warp; r < nt; r += nwarps) {
-    const int t = t0 + r;
-    select_topk_warp(lg + r * E, E, k, lane, topk_idx + static_cast<size_t>(t) * k,
-                     topk_w + static_cast<size_t>(t) * k);
-    float a = 0.f;
-    const uint4* ws = reinterpret_cast<const uint4*>(w_sg);
-    for (int c = lane; c < vec; c += 32) {
-      const uint4 wv = __ldg(ws + c);
-      const uint4 xv = xs[r * vec + c];
-      a = fmaf(bf16_lo(xv.x), bf16_lo(wv.x), a); a = fmaf(bf16_hi(xv.x), bf16_hi(wv.x), a);
-      a = fmaf(bf16_lo(xv.y), bf16_lo(wv.y), a); a = fmaf(bf16_hi(xv.y), bf16_hi(wv.y), a);
-      a = fmaf(bf16_lo(xv.z), bf16_lo(wv.z), a); a = fmaf(bf16_hi(xv.z), bf16_hi(wv.z), a);
-      a = fmaf(bf16_lo(xv.w), bf16_lo(wv.w), a); a = fmaf(bf16_hi(xv.w), bf16_hi(wv.w), a);
-    }
-    a = warp_sum(a);
-    if (lane == 0) sigma[t] = sigmoid(a);
-  }
-}
-
-// ---------------------------------------------------------------------------
 // Stable counting sort of the T*k (token, slot) entries by expert.
-// Entries are cut into segments of kSeg; one warp owns one segment.
-//   pass 1 (hist):    per-segment expert counts
+// Segment s = the entries of tokens [128 s, 128 s + 128), i.e. of one router
+// CTA, which already counted them per expert (pass 1).
 //   pass 2 (scan):    counts, offsets, per-segment bases, chunk list
 //   pass 3 (scatter): perm / inv_perm, ranks taken in entry order
 // Integer atomics only count (order-independent); every position comes from
 // the scan and an in-order rank, so the permutation is deterministic.
 // ---------------------------------------------------------------------------
-constexpr int kSeg = 1024;
 constexpr int kSegWarps = 4;
-
-__global__ void __launch_bounds__(32 * kSegWarps) hist_kernel(
-    const int32_t* __restrict__ topk_idx, int n, int E, int32_t* __restrict__ seg_counts) {
-  extern __shared__ int sh_hist[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int seg = blockIdx.x * kSegWarps + warp;
-  int* h = sh_hist + warp * E;
-  for (int e = lane; e < E; e += 32) h[e] = 0;
-  __syncwarp();
-  const int nseg = (n + kSeg - 1) / kSeg;
-  if (seg >= nseg) return;
-  const int b = seg * kSeg, end = min(b + kSeg, n);
-  for (int i = b + lane; i < end; i += 32) {
-    const int e = topk_idx[i];
-    if (e >= 0 && e < E) atomicAdd(&h[e], 1);
-  }
-  __syncwarp();
-  for (int e = lane; e < E; e += 32) seg_counts[static_cast<size_t>(seg) * E + e] = h[e];
-}
 
 // Block-wide exclusive scan over blockDim.x (<= 1024) ints; returns the total.
 __device__ int block_exclusive_scan(int v, int* scratch /*[32]*/, int* out_excl) {
@@ -161,18 +64,29 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(
   const int e = threadIdx.x;
   int c = 0;
   if (e < E)
-    for (int s = 0; s < nseg; ++s) c += seg_counts[static_cast<size_t>(s) * E + e];
+    for (int s0 = 0; s0 < nseg; s0 += 8) {
+      int v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = (s0 + j < nseg) ? seg_counts[static_cast<size_t>(s0 + j) * E + e] : 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) c += v[j];
+    }
   int off = 0;
   const int total = block_exclusive_scan(e < E ? c : 0, scratch, &off);
   if (e < E) {
     counts[e] = c;
     offsets[e] = off;
     int run = off;
-    for (int s = 0; s < nseg; ++s) {
-      const size_t i = static_cast<size_t>(s) * E + e;
-      const int v = seg_counts[i];
-      seg_counts[i] = run;     // becomes this segment's first position for expert e
-      run += v;
+    for (int s0 = 0; s0 < nseg; s0 += 8) {
+      int v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = (s0 + j < nseg) ? seg_counts[static_cast<size_t>(s0 + j) * E + e] : 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (s0 + j < nseg) {
+          seg_counts[static_cast<size_t>(s0 + j) * E + e] = run;   // this segment's first position for expert e
+          run += v[j];
+        }
     }
   }
   if (e == 0) offsets[E] = total;
@@ -205,22 +119,30 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(
 }
 
 __global__ void __launch_bounds__(32 * kSegWarps) scatter_kernel(
-    const int32_t* __restrict__ topk_idx, int n, int E, const int32_t* __restrict__ seg_base,
+    const int32_t* __restrict__ topk_idx, int n, int seg_len, int E, const int32_t* __restrict__ seg_base,
     int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm) {
   extern __shared__ int sh_cnt[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int seg = blockIdx.x * kSegWarps + warp;
-  const int nseg = (n + kSeg - 1) / kSeg;
+  const int nseg = (n + seg_len - 1) / seg_len;
   if (seg >= nseg) return;
   int* cnt = sh_cnt + warp * E;
   for (int e = lane; e < E; e += 32) cnt[e] = seg_base[static_cast<size_t>(seg) * E + e];
+  const int b = seg * seg_len, end = min(b + seg_len, n);
+  constexpr int kRounds = kRouteSegTokens * kMaxK / 32;   // 32 rounds of 32 entries at most
+  int ex[kRounds];
+#pragma unroll
+  for (int j = 0; j < kRounds; ++j) {
+    const int i = b + j * 32 + lane;
+    ex[j] = (i < end) ? topk_idx[i] : -1;                   // every load issued before the first round
+  }
   __syncwarp();
-  const int b = seg * kSeg, end = min(b + kSeg, n);
-  for (int base = b; base < end; base += 32) {
-    const int i = base + lane;
-    const bool valid = i < end;
-    int e = valid ? topk_idx[i] : -1;
-    if (valid && (e < 0 || e >= E)) e = -1;
+#pragma unroll
+  for (int j = 0; j < kRounds; ++j) {
+    if (b + j * 32 >= end) break;
+    const int i = b + j * 32 + lane;
+    int e = ex[j];
+    if (e >= E) e = -1;
     const unsigned peers = __match_any_sync(0xffffffffu, e);
     const int rank = __popc(peers & lanemask_lt());
     const int start = (e >= 0) ? cnt[e] : 0;
@@ -236,43 +158,171 @@ __global__ void __launch_bounds__(32 * kSegWarps) scatter_kernel(
 }
 
 // ---------------------------------------------------------------------------
+// Small-T routing (T <= 64): one launch does the router GEMV, top-k, shared
+// gate and the whole counting sort.  Warp w of CTA b scores row e = 8b + w
+// (e == E: the shared-gate vector) for every token, so the 1 MB router matrix
+// is streamed by ~33 CTAs at once.  The last CTA to finish (a counter in the
+// workspace, reset by that CTA) selects the experts, sorts the T*k entries
+// stably by expert and builds the active-expert list.
+// ---------------------------------------------------------------------------
+constexpr int kSmallWarps = 8;
+
+template <int TB>
+__global__ void __launch_bounds__(256) router_small_kernel(
+    const uint16_t* __restrict__ x, LayerPtr L, int T, int H, int I, int Is, int E, int k,
+    float* __restrict__ logits, unsigned* __restrict__ counter,
+    int32_t* __restrict__ topk_idx, float* __restrict__ topk_w, float* __restrict__ sigma,
+    int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
+    int32_t* __restrict__ inv_perm, int32_t* __restrict__ active, int32_t* __restrict__ n_active) {
+  extern __shared__ uint4 smem_u4[];
+  __shared__ int s_last;
+  __shared__ int s_scan[33];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int vec = H / 8;
+  const int E1 = E + 1;
+  const int e = blockIdx.x * kSmallWarps + warp;
+  const bool live = e <= E;
+  const uint4* wrow = reinterpret_cast<const uint4*>(e < E ? L.w_router + static_cast<size_t>(e) * H : L.w_sg);
+
+  uint4* xs = smem_u4;   // [TB][vec]
+  for (int t0 = 0; t0 < T; t0 += TB) {
+    const int nt = min(TB, T - t0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < TB * vec; i += blockDim.x) {
+      const int r = i / vec, c = i - r * vec;
+      xs[i] = r < nt ? reinterpret_cast<const uint4*>(x + static_cast<size_t>(t0 + r) * H)[c]
+                     : make_uint4(0u, 0u, 0u, 0u);
+    }
+    __syncthreads();
+    if (!live) continue;
+    float acc[TB];
+#pragma unroll
+    for (int r = 0; r < TB; ++r) acc[r] = 0.f;
+    for (int c = lane; c < vec; c += 32) {
+      const uint4 wv = __ldg(wrow + c);
+      const float w0 = bf16_lo(wv.x), w1 = bf16_hi(wv.x), w2 = bf16_lo(wv.y), w3 = bf16_hi(wv.y);
+      const float w4 = bf16_lo(wv.z), w5 = bf16_hi(wv.z), w6 = bf16_lo(wv.w), w7 = bf16_hi(wv.w);
+#pragma unroll
+      for (int r = 0; r < TB; ++r) {
+        const uint4 xv = xs[r * vec + c];
+        float a = acc[r];
+        a = fmaf(bf16_lo(xv.x), w0, a); a = fmaf(bf16_hi(xv.x), w1, a);
+        a = fmaf(bf16_lo(xv.y), w2, a); a = fmaf(bf16_hi(xv.y), w3, a);
+        a = fmaf(bf16_lo(xv.z), w4, a); a = fmaf(bf16_hi(xv.z), w5, a);
+        a = fmaf(bf16_lo(xv.w), w6, a); a = fmaf(bf16_hi(xv.w), w7, a);
+        acc[r] = a;
+      }
+    }
+    const float b = (e < E && L.router_bias) ? L.router_bias[e] : 0.f;
+#pragma unroll
+    for (int r = 0; r < TB; ++r) {
+      const float sum = warp_sum(acc[r]);
+      if (lane == 0 && r < nt) logits[static_cast<size_t>(t0 + r) * E1 + e] = sum + b;
+    }
+  }
+
+  // ---- the last CTA to finish does selection and grouping ----
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = (atomicAdd(counter, 1u) == gridDim.x - 1) ? 1 : 0;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  if (threadIdx.x == 0) *counter = 0u;
+
+  float* lg = reinterpret_cast<float*>(smem_u4);   // [T][E1], reuses the x tile
+  for (int i = threadIdx.x; i < T * E1; i += blockDim.x) lg[i] = __ldcg(logits + i);
+  __syncthreads();
+  for (int t = warp; t < T; t += kSmallWarps) {
+    select_topk_warp(lg + t * E1, E, k, lane, topk_idx + t * k, topk_w + t * k);
+    if (lane == 0) sigma[t] = sigmoid(lg[t * E1 + E]);
+  }
+  __syncthreads();
+
+  // histogram, exclusive scan and stable scatter of the n = T*k entries
+  int* hist = reinterpret_cast<int*>(smem_u4);       // [256] (logits no longer needed)
+  int* cursor = hist + 256;                          // [256]
+  const int n = T * k;
+  hist[threadIdx.x] = 0;
+  __syncthreads();
+  for (int i = threadIdx.x; i < n; i += blockDim.x) atomicAdd(&hist[topk_idx[i]], 1);
+  __syncthreads();
+  const int c = threadIdx.x < E ? hist[threadIdx.x] : 0;
+  int off = 0;
+  const int total = block_exclusive_scan(c, s_scan, &off);
+  if (threadIdx.x < E) {
+    counts[threadIdx.x] = c;
+    offsets[threadIdx.x] = off;
+    cursor[threadIdx.x] = off;
+  }
+  if (threadIdx.x == 0) offsets[E] = total;
+  int apos = 0;
+  const int nact = block_exclusive_scan((threadIdx.x < E && c > 0) ? 1 : 0, s_scan, &apos);
+  if (threadIdx.x < E && c > 0) active[apos] = threadIdx.x;
+  if (threadIdx.x == 0) {
+    active[nact] = E;
+    *n_active = nact + 1;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    for (int base = 0; base < n; base += 32) {
+      const int i = base + lane;
+      const int ex = i < n ? topk_idx[i] : -1;
+      const unsigned peers = __match_any_sync(0xffffffffu, ex);
+      const int rank = __popc(peers & lanemask_lt());
+      const int start = ex >= 0 ? cursor[ex] : 0;
+      __syncwarp();
+      if (ex >= 0) {
+        perm[start + rank] = i;
+        inv_perm[i] = start + rank;
+        if ((peers >> lane) == 1u) cursor[ex] = start + __popc(peers);
+      }
+      __syncwarp();
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Host launchers
 // ---------------------------------------------------------------------------
-int router_smem_bytes(int tb, int H, int E) { return tb * H * 2 + tb * E * 4; }
+int num_segments(int T) { return (T + kRouteSegTokens - 1) / kRouteSegTokens; }
 
-cudaError_t launch_router(const uint16_t* x, const uint16_t* w_router, const float* router_bias,
-                          const uint16_t* w_sg, int T, int H, int E, int k,
-                          int32_t* topk_idx, float* topk_w, float* sigma, cudaStream_t s) {
-  if (H <= 4096) {
-    constexpr int TB = 16;
-    const int smem = router_smem_bytes(TB, H, E);
-    cudaFuncSetAttribute(router_topk_kernel<TB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    router_topk_kernel<TB><<<(T + TB - 1) / TB, 256, smem, s>>>(x, w_router, router_bias, w_sg, T, H, E, k,
-                                                                 topk_idx, topk_w, sigma);
-  } else {
-    constexpr int TB = 8;
-    const int smem = router_smem_bytes(TB, H, E);
-    cudaFuncSetAttribute(router_topk_kernel<TB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    router_topk_kernel<TB><<<(T + TB - 1) / TB, 256, smem, s>>>(x, w_router, router_bias, w_sg, T, H, E, k,
-                                                                 topk_idx, topk_w, sigma);
-  }
+template <int TB>
+static cudaError_t launch_small_tb(const uint16_t* x, const LayerPtr& L, int T, int H, int I, int Is, int E, int k,
+                                   float* logits, unsigned* counter, const RoutingPtrs& r, int32_t* active,
+                                   int32_t* n_active, cudaStream_t s) {
+  const int grid = (E + 1 + kSmallWarps - 1) / kSmallWarps;
+  const int smem = max(TB * H * 2, max(T * (E + 1) * 4, 2048));
+  const cudaError_t e = ensure_smem(reinterpret_cast<const void*>(router_small_kernel<TB>), smem);
+  if (e != cudaSuccess) return e;
+  router_small_kernel<TB><<<grid, 256, smem, s>>>(x, L, T, H, I, Is, E, k, logits, counter, r.topk_idx, r.topk_w,
+                                                  r.sigma, r.counts, r.offsets, r.perm, r.inv_perm, active,
+                                                  n_active);
   return cudaGetLastError();
 }
 
-int num_segments(int n_entries) { return (n_entries + kSeg - 1) / kSeg; }
+cudaError_t launch_route_small(const uint16_t* x, const LayerPtr& L, int T, int H, int I, int Is, int E, int k,
+                               float* logits, unsigned* counter, const RoutingPtrs& r, int32_t* active,
+                               int32_t* n_active, cudaStream_t s) {
+  // tokens per pass over the router matrix: x tile of TB rows (bf16) in smem
+  if (T == 1) return launch_small_tb<1>(x, L, T, H, I, Is, E, k, logits, counter, r, active, n_active, s);
+  if (T <= 2) return launch_small_tb<2>(x, L, T, H, I, Is, E, k, logits, counter, r, active, n_active, s);
+  if (T <= 4 || H > 4096) return launch_small_tb<4>(x, L, T, H, I, Is, E, k, logits, counter, r, active, n_active, s);
+  return launch_small_tb<8>(x, L, T, H, I, Is, E, k, logits, counter, r, active, n_active, s);
+}
 
 cudaError_t launch_group(const int32_t* topk_idx, int T, int k, int E, int chunk_rows,
                          int32_t* seg_scratch, int32_t* counts, int32_t* offsets,
                          int32_t* perm, int32_t* inv_perm, Chunk* chunks, int32_t* n_chunks,
                          int32_t* active, int32_t* n_active, cudaStream_t s) {
   const int n = T * k;
-  const int nseg = num_segments(n);
+  const int nseg = num_segments(T);
   const int grid = (nseg + kSegWarps - 1) / kSegWarps;
   const int smem = kSegWarps * E * static_cast<int>(sizeof(int));
-  hist_kernel<<<grid, 32 * kSegWarps, smem, s>>>(topk_idx, n, E, seg_scratch);
   scan_kernel<<<1, kScanThreads, 0, s>>>(seg_scratch, nseg, E, T, k, chunk_rows, counts, offsets,
                                          chunks, n_chunks, active, n_active);
-  scatter_kernel<<<grid, 32 * kSegWarps, smem, s>>>(topk_idx, n, E, seg_scratch, perm, inv_perm);
+  scatter_kernel<<<grid, 32 * kSegWarps, smem, s>>>(topk_idx, n, kRouteSegTokens * k, E, seg_scratch, perm,
+                                                    inv_perm);
   return cudaGetLastError();
 }
 

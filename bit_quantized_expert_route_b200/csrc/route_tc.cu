@@ -1,0 +1,233 @@
+// Router for T > 64 on the tensor cores: logits, top-k with renormalised
+// softmax weights, and the shared-expert gate in one kernel.
+//
+// One CTA scores 128 tokens: D[128 tokens x E experts] = x W_r^T accumulates
+// in tensor memory (tcgen05.mma, bf16 operands in shared memory, FP32
+// accumulators), and a second 16-column MMA against [w_sg; 0 ... 0] yields
+// x . w_sg in column 256.  Each epilogue thread owns one token (its TMEM
+// lane), reads its E logits and keeps the k best in registers by insertion
+// in expert order, which realises the order (logit desc, expert index asc).
+// The CTA also counts its 128*k (token, slot) entries per expert: that is
+// the first pass of the counting sort (one segment per CTA).
+// ("Perplexity's Lily: ...", section "The Model": the router scores 256
+// experts and keeps 8, plus one shared expert for every token.)
+#include "common.cuh"
+#include "kernels.h"
+#include "tc.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kRM = 128;                  // tokens per CTA (TMEM lanes)
+constexpr int kRBK = 64;                  // inputs per stage
+constexpr int kRStages = 4;
+constexpr int kRLag = 2;
+constexpr int kRThreads = 160;            // warps 0-3: loaders then epilogue; warp 4: TMEM + MMA
+constexpr int kRMmaWarp = 4;
+constexpr int kA_BYTES = kRM * kRBK * 2;                  // 16 KB
+constexpr int kB_BYTES = kMaxE * kRBK * 2;                // 32 KB (up to 256 experts)
+constexpr int kG_BYTES = 16 * kRBK * 2;                   // 2 KB: w_sg row + 15 zero rows
+constexpr int kSTAGE = kA_BYTES + kB_BYTES + kG_BYTES;    // 50 KB (multiple of 1024)
+constexpr int kBAR_OFF = kRStages * kSTAGE;
+constexpr int kRSMEM = kBAR_OFF + 128 + kMaxE * 4 + 1024;   // barriers, histogram, alignment slack
+constexpr uint32_t kRTmemCols = 512;
+constexpr int kGateCol = 256;             // accumulator column of x . w_sg
+
+__global__ void __launch_bounds__(kRThreads, 1) router_tc_kernel(
+    const uint16_t* __restrict__ x, const uint16_t* __restrict__ w_router, const float* __restrict__ router_bias,
+    const uint16_t* __restrict__ w_sg, int T, int H, int E, int k, int32_t* __restrict__ topk_idx,
+    float* __restrict__ topk_w, float* __restrict__ sigma, int32_t* __restrict__ seg_counts, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_u32 = tc::smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
+  const uint32_t sbase = tc::smem_u32(smem);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBAR_OFF);
+  uint64_t* empty = full + kRStages;
+  uint64_t* acc_full = empty + kRStages;
+  uint64_t* drain = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* hist = reinterpret_cast<int*>(smem + kBAR_OFF + 128);       // [kMaxE] this CTA's expert counts
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t0 = blockIdx.x * kRM;
+  const int nks = H / kRBK;
+  const int n_mma = max(16, (E + 15) & ~15);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kRStages; ++s) {
+      tc::mbar_init(&full[s], 128);
+      tc::mbar_init(&empty[s], 1);
+    }
+    tc::mbar_init(acc_full, 1);
+    tc::mbar_init(drain, 1);
+    *abort_flag = 0;
+    tc::fence_barrier_init();
+  }
+  // zero rows 1..15 of every stage's gate tile once (row 0 is reloaded per stage)
+  if (warp < 4) {
+    for (int i = threadIdx.x; i < kMaxE; i += 128) hist[i] = 0;
+    for (int i = threadIdx.x; i < kRStages * 15 * 8; i += 128) {
+      const int s = i / 120, rr = 1 + (i % 120) / 8, c = i % 8;
+      *reinterpret_cast<uint4*>(smem + s * kSTAGE + kA_BYTES + kB_BYTES + rr * 128 + c * 16) =
+          make_uint4(0u, 0u, 0u, 0u);
+    }
+    tc::fence_proxy_async_smem();
+  }
+  if (warp == kRMmaWarp) tc::tmem_alloc(tmem_slot, kRTmemCols);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp < 4) {
+    // ---------------------------------------------------------- loaders
+    const int r = threadIdx.x;                                 // x row, and expert rows r, r + 128
+    const uint16_t* xrow = (t0 + r < T) ? x + static_cast<size_t>(t0 + r) * H : nullptr;
+    const uint16_t* wr0 = r < E ? w_router + static_cast<size_t>(r) * H : nullptr;
+    const uint16_t* wr1 = r + 128 < E ? w_router + static_cast<size_t>(r + 128) * H : nullptr;
+    bool ok = true;
+    int ks = 0;
+    for (; ks < nks; ++ks) {
+      const int s = ks % kRStages;
+      if (!tc::mbar_wait(&empty[s], ((ks / kRStages) & 1) ^ 1, abort_flag, status)) {
+        ok = false;
+        break;
+      }
+      const uint32_t st = sbase + s * kSTAGE;
+      const int sw = r & 7;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint32_t off = static_cast<uint32_t>(((c ^ sw) << 4));
+        if (xrow) tc::cp_async16(st + r * 128 + off, xrow + ks * kRBK + c * 8);
+        if (wr0) tc::cp_async16(st + kA_BYTES + r * 128 + off, wr0 + ks * kRBK + c * 8);
+        if (wr1) tc::cp_async16(st + kA_BYTES + (r + 128) * 128 + off, wr1 + ks * kRBK + c * 8);
+      }
+      if (r < 8) tc::cp_async16(st + kA_BYTES + kB_BYTES + (r << 4), w_sg + ks * kRBK + r * 8);   // row 0, no swizzle
+      tc::cp_async_commit();
+      if (ks >= kRLag) {
+        tc::cp_async_wait<kRLag>();
+        tc::fence_proxy_async_smem();
+        tc::mbar_arrive(&full[(ks - kRLag) % kRStages]);
+      }
+    }
+    tc::cp_async_wait_all();
+    tc::fence_proxy_async_smem();
+    if (ok)
+      for (int j = max(0, ks - kRLag); j < ks; ++j) tc::mbar_arrive(&full[j % kRStages]);
+
+    // --------------------------------------------------------- epilogue
+    if (ok && tc::mbar_wait(acc_full, 0, abort_flag, status)) {
+      tc::tc_fence_after();
+      const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+      float bv[kMaxK];
+      int bi[kMaxK];
+#pragma unroll
+      for (int j = 0; j < kMaxK; ++j) {
+        bv[j] = -INFINITY;
+        bi[j] = 0x7fffffff;
+      }
+      for (int c0 = 0; c0 < n_mma; c0 += 16) {
+        float v[16];
+        tc::tmem_ld16(lane_base + c0, v);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int e = c0 + i;
+          if (e < E) {
+            const float l = v[i] + (router_bias ? __ldg(router_bias + e) : 0.f);
+            if (l > bv[k - 1]) {
+              // insert after every kept logit >= l (equal logits keep the lower index first)
+              float cv = l;
+              int ci = e;
+#pragma unroll
+              for (int j = 0; j < kMaxK; ++j) {
+                if (j < k && cv > bv[j]) {
+                  const float tv = bv[j];
+                  const int ti = bi[j];
+                  bv[j] = cv;
+                  bi[j] = ci;
+                  cv = tv;
+                  ci = ti;
+                }
+              }
+            }
+          }
+        }
+      }
+      float g[16];
+      tc::tmem_ld16(lane_base + kGateCol, g);
+      tc::tmem_wait_ld();
+      const int t = t0 + r;
+      if (t < T) {
+        float z[kMaxK];
+        float sum = 0.f;
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j)
+          if (j < k) {
+            z[j] = expf(bv[j] - bv[0]);
+            sum += z[j];
+          }
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j)
+          if (j < k) {
+            topk_idx[static_cast<size_t>(t) * k + j] = bi[j];
+            topk_w[static_cast<size_t>(t) * k + j] = z[j] / sum;
+            atomicAdd(&hist[bi[j]], 1);      // counting is order-independent
+          }
+        sigma[t] = sigmoid(g[0]);
+      }
+    }
+    // this CTA's segment of the (token, slot) entries: expert counts for the sort
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    for (int e = threadIdx.x; e < E; e += 128) seg_counts[static_cast<size_t>(blockIdx.x) * E + e] = hist[e];
+  } else if (warp == kRMmaWarp) {
+    // -------------------------------------------------------------- MMA
+    if (lane == 0) {
+      const uint32_t idesc = tc::idesc_bf16(kRM, n_mma);
+      const uint32_t idesc_g = tc::idesc_bf16(kRM, 16);
+      bool ok = true;
+      for (int ks = 0; ks < nks; ++ks) {
+        const int s = ks % kRStages;
+        if (!tc::mbar_wait(&full[s], (ks / kRStages) & 1, abort_flag, status)) {
+          ok = false;
+          break;
+        }
+        tc::tc_fence_after();
+        const uint32_t st = sbase + s * kSTAGE;
+#pragma unroll
+        for (int kk = 0; kk < kRBK / 16; ++kk) {
+          const uint64_t adesc = tc::sdesc_sw128(st + kk * 32);
+          const uint32_t accum = (ks > 0 || kk > 0) ? 1u : 0u;
+          tc::mma_bf16_ss(tmem, adesc, tc::sdesc_sw128(st + kA_BYTES + kk * 32), idesc, accum);
+          tc::mma_bf16_ss(tmem + kGateCol, adesc, tc::sdesc_sw128(st + kA_BYTES + kB_BYTES + kk * 32), idesc_g,
+                          accum);
+        }
+        tc::mma_commit(&empty[s]);
+      }
+      if (ok) tc::mma_commit(acc_full);
+      tc::mma_commit(drain);
+      tc::mbar_wait_drain(drain, 0, status);
+    }
+    __syncwarp();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  if (warp == kRMmaWarp) tc::tmem_dealloc(tmem, kRTmemCols);
+}
+
+}  // namespace
+
+cudaError_t launch_router(const uint16_t* x, const uint16_t* w_router, const float* router_bias,
+                          const uint16_t* w_sg, int T, int H, int E, int k,
+                          int32_t* topk_idx, float* topk_w, float* sigma, int32_t* seg_counts, int* status,
+                          cudaStream_t s) {
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(router_tc_kernel), kRSMEM);
+  if (e != cudaSuccess) return e;
+  router_tc_kernel<<<(T + kRM - 1) / kRM, kRThreads, kRSMEM, s>>>(x, w_router, router_bias, w_sg, T, H, E, k,
+                                                                   topk_idx, topk_w, sigma, seg_counts, status);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

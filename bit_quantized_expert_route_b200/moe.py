@@ -187,7 +187,7 @@ def moe_workspace_size(layer: MoELayer, T_max: int) -> int:
 
 
 def alloc_workspace(layer: MoELayer, T_max: int, device="cuda") -> torch.Tensor:
-    """A device workspace for calls with T <= T_max (torch allocations are 256-byte aligned)."""
+    """A zero-filled device workspace for calls with T <= T_max (torch allocations are 256-byte aligned)."""
     return torch.zeros(moe_workspace_size(layer, T_max), dtype=torch.uint8, device=device)
 
 
@@ -233,7 +233,7 @@ def moe_rmsnorm(y: torch.Tensor, y_out: torch.Tensor, eps: float = 1e-6, stream=
 
 
 PREFILL_STAGES = ("router", "group", "gateup", "down", "combine")
-DECODE_STAGES = ("router", "group", "gateup", "down_combine")
+DECODE_STAGES = ("route", "gateup", "down_combine")
 
 
 def moe_forward_profiled(layer: MoELayer, x: torch.Tensor, out: torch.Tensor, workspace: torch.Tensor,

@@ -41,7 +41,10 @@
  * Ownership.  The caller owns every buffer (weights, x, out, routing,
  * workspace).  The library allocates no device memory and keeps no state
  * between calls except cached kernel attributes.  Two calls must not share a
- * workspace concurrently.
+ * workspace concurrently.  The first 256 bytes of a workspace are a control
+ * block (status word, a CTA counter) that must be zero before the workspace
+ * is first used (e.g. cudaMemset); the library leaves them zero after every
+ * call except for a recorded error status, which moe_get_status clears.
  *
  * Asynchrony.  moe_route, moe_forward, moe_decode and moe_rmsnorm enqueue
  * work on `stream` (a cudaStream_t; NULL = the legacy default stream) and
@@ -168,7 +171,7 @@ MOE_API int moe_decode(const moe_layer_desc* layer, const moe_bf16* x, int T, mo
  * the chunk list, the active-expert list, and sigma when r->sigma is NULL)
  * lives in one static device array of 512 KiB inside libmoe.so, which every
  * GPU that loads the library holds until the process exits.
- *   Limit: the call needs ceil(T*k/1024)*E*4 bytes of counts, plus
+ *   Limit: the call needs ceil(T/128)*E*4 bytes of counts, plus
  *   (T*k/128 + T/128 + E + 2)*16 bytes of chunk list, plus (E+1)*4 + 2*4
  *   bytes, plus T*4 bytes if r->sigma is NULL, each rounded up to 256 bytes;
  *   a call whose need exceeds 512 KiB returns MOE_ERR_WORKSPACE and enqueues
@@ -200,7 +203,7 @@ MOE_API int moe_rmsnorm(const moe_bf16* y, moe_bf16* y_out, int T, int H, float 
  * `stream` before the first and after every stage, waits for the stream, and
  * writes each stage's device time in milliseconds to stage_ms[0..n-1]:
  *   T > 64:  router, group (histogram+scan+scatter), gate/up GEMM, down GEMM, combine
- *   T <= 64: router, group, gate/up GEMV, down GEMV + combine, (unused)
+ *   T <= 64: routing (one kernel), gate/up GEMV, down GEMV + combine
  * stage_ms: host array of at least 5 floats; *n_stages receives the count.
  * The events are created and destroyed inside the call. */
 MOE_API int moe_forward_profiled(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_bf16* out,
