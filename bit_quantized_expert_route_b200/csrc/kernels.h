@@ -1,6 +1,7 @@
 // Host-side launchers of the MoE kernels (internal to libmoe.so).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -36,6 +37,11 @@ struct RoutingPtrs {
   int32_t* perm;
   int32_t* inv_perm;
 };
+
+// tmap.cu: 2-D TMA tensor map over a row-major [rows, cols] array of
+// `esize`-byte elements with box [box_rows, box_cols]; false on failure.
+bool make_tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* base, uint64_t cols, uint64_t rows,
+                  uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw);
 
 // api.cu: raise a kernel's dynamic shared-memory limit once per device (and
 // again only if a launch needs more), keeping the attribute call off the

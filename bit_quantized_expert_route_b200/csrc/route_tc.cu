@@ -21,7 +21,6 @@ namespace {
 constexpr int kRM = 128;                  // tokens per CTA (TMEM lanes)
 constexpr int kRBK = 64;                  // inputs per stage
 constexpr int kRStages = 4;
-constexpr int kRLag = 2;
 constexpr int kRThreads = 160;            // warps 0-3: loaders then epilogue; warp 4: TMEM + MMA
 constexpr int kRMmaWarp = 4;
 constexpr int kA_BYTES = kRM * kRBK * 2;                  // 16 KB
@@ -33,10 +32,78 @@ constexpr int kRSMEM = kBAR_OFF + 128 + kMaxE * 4 + 1024;   // barriers, histogr
 constexpr uint32_t kRTmemCols = 512;
 constexpr int kGateCol = 256;             // accumulator column of x . w_sg
 
+// One token's epilogue (this thread's TMEM lane): the E logits (+ bias) scanned
+// in expert order, the K largest kept by insertion (a later expert replaces a
+// kept one only if strictly larger, so equal logits keep the lower index
+// first), then renormalised softmax weights, the shared gate, and the token's
+// contribution to the CTA's expert histogram.
+template <int K>
+__device__ __forceinline__ void router_epilogue(uint32_t lane_base, int n_mma, int E, const float* __restrict__ bias,
+                                                int t, int T, int32_t* __restrict__ topk_idx,
+                                                float* __restrict__ topk_w, float* __restrict__ sigma, int* hist) {
+  float bv[K];
+  int bi[K];
+#pragma unroll
+  for (int j = 0; j < K; ++j) {
+    bv[j] = -INFINITY;
+    bi[j] = 0x7fffffff;
+  }
+  for (int c0 = 0; c0 < n_mma; c0 += 16) {
+    float v[16];
+    tc::tmem_ld16(lane_base + c0, v);
+    tc::tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int e = c0 + i;
+      if (e < E) {
+        float cv = v[i] + (bias ? __ldg(bias + e) : 0.f);
+        if (cv > bv[K - 1]) {
+          int ci = e;
+#pragma unroll
+          for (int j = 0; j < K; ++j) {
+            const bool take = cv > bv[j];
+            const float tv = bv[j];
+            const int ti = bi[j];
+            bv[j] = take ? cv : tv;
+            bi[j] = take ? ci : ti;
+            cv = take ? tv : cv;
+            ci = take ? ti : ci;
+          }
+        }
+      }
+    }
+  }
+  float g[16];
+  tc::tmem_ld16(lane_base + kGateCol, g);
+  tc::tmem_wait_ld();
+  if (t < T) {
+    float z[K];
+    float sum = 0.f;
+#pragma unroll
+    for (int j = 0; j < K; ++j) {
+      z[j] = expf(bv[j] - bv[0]);
+      sum += z[j];
+    }
+#pragma unroll
+    for (int j = 0; j < K; ++j) {
+      topk_idx[static_cast<size_t>(t) * K + j] = bi[j];
+      topk_w[static_cast<size_t>(t) * K + j] = z[j] / sum;
+      atomicAdd(&hist[bi[j]], 1);      // counting is order-independent
+    }
+    sigma[t] = sigmoid(g[0]);
+  }
+}
+
+struct alignas(64) RouterMaps {
+  CUtensorMap x;     // x [T, H], box 128 rows x 64 inputs, 128-B swizzle
+  CUtensorMap w;     // W_r [E, H], box n_mma rows x 64 inputs, 128-B swizzle
+  CUtensorMap g;     // w_sg [1, H], box 1 row x 64 inputs
+};
+
 __global__ void __launch_bounds__(kRThreads, 1) router_tc_kernel(
-    const uint16_t* __restrict__ x, const uint16_t* __restrict__ w_router, const float* __restrict__ router_bias,
-    const uint16_t* __restrict__ w_sg, int T, int H, int E, int k, int32_t* __restrict__ topk_idx,
-    float* __restrict__ topk_w, float* __restrict__ sigma, int32_t* __restrict__ seg_counts, int* status) {
+    const __grid_constant__ RouterMaps maps, const float* __restrict__ router_bias, int T, int H, int E, int k,
+    int32_t* __restrict__ topk_idx, float* __restrict__ topk_w, float* __restrict__ sigma,
+    int32_t* __restrict__ seg_counts, int* status) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = tc::smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
@@ -56,7 +123,7 @@ __global__ void __launch_bounds__(kRThreads, 1) router_tc_kernel(
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kRStages; ++s) {
-      tc::mbar_init(&full[s], 128);
+      tc::mbar_init(&full[s], 1);
       tc::mbar_init(&empty[s], 1);
     }
     tc::mbar_init(acc_full, 1);
@@ -81,101 +148,39 @@ __global__ void __launch_bounds__(kRThreads, 1) router_tc_kernel(
   const uint32_t tmem = *tmem_slot;
 
   if (warp < 4) {
-    // ---------------------------------------------------------- loaders
-    const int r = threadIdx.x;                                 // x row, and expert rows r, r + 128
-    const uint16_t* xrow = (t0 + r < T) ? x + static_cast<size_t>(t0 + r) * H : nullptr;
-    const uint16_t* wr0 = r < E ? w_router + static_cast<size_t>(r) * H : nullptr;
-    const uint16_t* wr1 = r + 128 < E ? w_router + static_cast<size_t>(r + 128) * H : nullptr;
+    // ---------------------------------------------------------- loader
+    // one thread streams the stages: x tile, router rows and the gate row
+    const int r = threadIdx.x;
     bool ok = true;
-    int ks = 0;
-    for (; ks < nks; ++ks) {
-      const int s = ks % kRStages;
-      if (!tc::mbar_wait(&empty[s], ((ks / kRStages) & 1) ^ 1, abort_flag, status)) {
-        ok = false;
-        break;
-      }
-      const uint32_t st = sbase + s * kSTAGE;
-      const int sw = r & 7;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint32_t off = static_cast<uint32_t>(((c ^ sw) << 4));
-        if (xrow) tc::cp_async16(st + r * 128 + off, xrow + ks * kRBK + c * 8);
-        if (wr0) tc::cp_async16(st + kA_BYTES + r * 128 + off, wr0 + ks * kRBK + c * 8);
-        if (wr1) tc::cp_async16(st + kA_BYTES + (r + 128) * 128 + off, wr1 + ks * kRBK + c * 8);
-      }
-      if (r < 8) tc::cp_async16(st + kA_BYTES + kB_BYTES + (r << 4), w_sg + ks * kRBK + r * 8);   // row 0, no swizzle
-      tc::cp_async_commit();
-      if (ks >= kRLag) {
-        tc::cp_async_wait<kRLag>();
-        tc::fence_proxy_async_smem();
-        tc::mbar_arrive(&full[(ks - kRLag) % kRStages]);
+    if (threadIdx.x == 0) {
+      const uint32_t tx = static_cast<uint32_t>(kA_BYTES + n_mma * kRBK * 2 + kRBK * 2);
+      for (int ks = 0; ks < nks; ++ks) {
+        const int s = ks % kRStages;
+        if (!tc::mbar_wait(&empty[s], ((ks / kRStages) & 1) ^ 1, abort_flag, status)) {
+          ok = false;
+          break;
+        }
+        const uint32_t st = sbase + s * kSTAGE;
+        tc::mbar_arrive_expect_tx(&full[s], tx);
+        tc::tma_load_2d(st, &maps.x, ks * kRBK, t0, &full[s]);
+        tc::tma_load_2d(st + kA_BYTES, &maps.w, ks * kRBK, 0, &full[s]);
+        tc::tma_load_2d(st + kA_BYTES + kB_BYTES, &maps.g, ks * kRBK, 0, &full[s]);
       }
     }
-    tc::cp_async_wait_all();
-    tc::fence_proxy_async_smem();
-    if (ok)
-      for (int j = max(0, ks - kRLag); j < ks; ++j) tc::mbar_arrive(&full[j % kRStages]);
 
     // --------------------------------------------------------- epilogue
     if (ok && tc::mbar_wait(acc_full, 0, abort_flag, status)) {
       tc::tc_fence_after();
       const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-      float bv[kMaxK];
-      int bi[kMaxK];
-#pragma unroll
-      for (int j = 0; j < kMaxK; ++j) {
-        bv[j] = -INFINITY;
-        bi[j] = 0x7fffffff;
-      }
-      for (int c0 = 0; c0 < n_mma; c0 += 16) {
-        float v[16];
-        tc::tmem_ld16(lane_base + c0, v);
-        tc::tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int e = c0 + i;
-          if (e < E) {
-            const float l = v[i] + (router_bias ? __ldg(router_bias + e) : 0.f);
-            if (l > bv[k - 1]) {
-              // insert after every kept logit >= l (equal logits keep the lower index first)
-              float cv = l;
-              int ci = e;
-#pragma unroll
-              for (int j = 0; j < kMaxK; ++j) {
-                if (j < k && cv > bv[j]) {
-                  const float tv = bv[j];
-                  const int ti = bi[j];
-                  bv[j] = cv;
-                  bi[j] = ci;
-                  cv = tv;
-                  ci = ti;
-                }
-              }
-            }
-          }
-        }
-      }
-      float g[16];
-      tc::tmem_ld16(lane_base + kGateCol, g);
-      tc::tmem_wait_ld();
-      const int t = t0 + r;
-      if (t < T) {
-        float z[kMaxK];
-        float sum = 0.f;
-#pragma unroll
-        for (int j = 0; j < kMaxK; ++j)
-          if (j < k) {
-            z[j] = expf(bv[j] - bv[0]);
-            sum += z[j];
-          }
-#pragma unroll
-        for (int j = 0; j < kMaxK; ++j)
-          if (j < k) {
-            topk_idx[static_cast<size_t>(t) * k + j] = bi[j];
-            topk_w[static_cast<size_t>(t) * k + j] = z[j] / sum;
-            atomicAdd(&hist[bi[j]], 1);      // counting is order-independent
-          }
-        sigma[t] = sigmoid(g[0]);
+      switch (k) {   // k fixed at compile time: the candidate list stays in registers
+        case 1: router_epilogue<1>(lane_base, n_mma, E, router_bias, t0 + r, T, topk_idx, topk_w, sigma, hist); break;
+        case 2: router_epilogue<2>(lane_base, n_mma, E, router_bias, t0 + r, T, topk_idx, topk_w, sigma, hist); break;
+        case 3: router_epilogue<3>(lane_base, n_mma, E, router_bias, t0 + r, T, topk_idx, topk_w, sigma, hist); break;
+        case 4: router_epilogue<4>(lane_base, n_mma, E, router_bias, t0 + r, T, topk_idx, topk_w, sigma, hist); break;
+        case 5: router_epilogue<5>(lane_base, n_mma, E, router_bias, t0 + r, T, topk_idx, topk_w, sigma, hist); break;
+        case 6: router_epilogue<6>(lane_base, n_mma, E, router_bias, t0 + r, T, topk_idx, topk_w, sigma, hist); break;
+        case 7: router_epilogue<7>(lane_base, n_mma, E, router_bias, t0 + r, T, topk_idx, topk_w, sigma, hist); break;
+        default: router_epilogue<8>(lane_base, n_mma, E, router_bias, t0 + r, T, topk_idx, topk_w, sigma, hist); break;
       }
     }
     // this CTA's segment of the (token, slot) entries: expert counts for the sort
@@ -223,10 +228,17 @@ cudaError_t launch_router(const uint16_t* x, const uint16_t* w_router, const flo
                           const uint16_t* w_sg, int T, int H, int E, int k,
                           int32_t* topk_idx, float* topk_w, float* sigma, int32_t* seg_counts, int* status,
                           cudaStream_t s) {
+  RouterMaps maps;
+  const uint32_t n_mma = static_cast<uint32_t>(max(16, (E + 15) & ~15));
+  if (!make_tmap_2d(&maps.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, H, T, kRBK, kRM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&maps.w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w_router, H, E, kRBK, n_mma,
+                    CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&maps.g, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w_sg, H, 1, kRBK, 1, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(router_tc_kernel), kRSMEM);
   if (e != cudaSuccess) return e;
-  router_tc_kernel<<<(T + kRM - 1) / kRM, kRThreads, kRSMEM, s>>>(x, w_router, router_bias, w_sg, T, H, E, k,
-                                                                   topk_idx, topk_w, sigma, seg_counts, status);
+  router_tc_kernel<<<(T + kRM - 1) / kRM, kRThreads, kRSMEM, s>>>(maps, router_bias, T, H, E, k, topk_idx, topk_w,
+                                                                   sigma, seg_counts, status);
   return cudaGetLastError();
 }
 
