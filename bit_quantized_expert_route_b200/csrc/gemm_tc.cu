@@ -459,45 +459,58 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- MMA
-    if (lane == 0) {
-      uint32_t it = 0, tt = 0;
-      bool ok = true;
-      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-        const UnitInfo ui = unit_info<kGateUp>(a, u, nfb);
-        if (ui.skip) continue;
-        const int n_mma = max(16, (ui.rows + 15) & ~15);
-        const uint32_t idesc = tc::idesc_bf16(BM, n_mma);
-        const int buf = static_cast<int>(tt % C::ACC_BUFS);
-        if (!tc::mbar_wait(&acc_empty[buf], ((tt / C::ACC_BUFS) & 1u) ^ 1u, abort_flag, a.status)) break;
+    // The whole warp walks the schedule and waits on the barriers; one elected
+    // lane issues.  Operand descriptors are formed once and advanced by adds
+    // (the shared-memory address field counts 16-byte units).
+    const bool leader = tc::elect_one_sync();
+    const uint64_t bdesc0 = tc::sdesc_sw128(sbase + C::OFF_B);
+    uint32_t it = 0, tt = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const UnitInfo ui = unit_info<kGateUp>(a, u, nfb);
+      if (ui.skip) continue;
+      const int n_mma = max(16, (ui.rows + 15) & ~15);
+      const uint32_t idesc = tc::idesc_bf16(BM, n_mma);
+      const int buf = static_cast<int>(tt % C::ACC_BUFS);
+      // (every wait's outcome is made warp-uniform so the lanes leave together)
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(&acc_empty[buf], ((tt / C::ACC_BUFS) & 1u) ^ 1u, abort_flag,
+                                                 a.status)))
+        break;
+      tc::tc_fence_after();
+      const uint32_t acc = tmem + buf * C::ACC_COLS;
+      for (int ks = 0; ks < ui.nks; ++ks, ++it) {
+        const int sb = static_cast<int>(it % kBStages);
+        const int sa = static_cast<int>(it % C::A_STAGES);
+        const bool got = tc::mbar_wait(&full_b[sb], (it / kBStages) & 1u, abort_flag, a.status) &&
+                         tc::mbar_wait(&full_a[sa], (it / C::A_STAGES) & 1u, abort_flag, a.status);
+        if (!__all_sync(0xffffffffu, got)) {
+          ok = false;
+          break;
+        }
         tc::tc_fence_after();
-        const uint32_t acc = tmem + buf * C::ACC_COLS;
-        for (int ks = 0; ks < ui.nks; ++ks, ++it) {
-          const int sb = static_cast<int>(it % kBStages);
-          const int sa = static_cast<int>(it % C::A_STAGES);
-          if (!tc::mbar_wait(&full_b[sb], (it / kBStages) & 1u, abort_flag, a.status) ||
-              !tc::mbar_wait(&full_a[sa], (it / C::A_STAGES) & 1u, abort_flag, a.status)) {
-            ok = false;
-            break;
-          }
-          tc::tc_fence_after();
-          const uint32_t bst = sbase + C::OFF_B + sb * C::B_BYTES;
+        if (leader) {
+          const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(sb * (C::B_BYTES >> 4));
           const uint32_t ast = tmem + C::A_BASE + sa * C::A_COLS;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t bdesc = tc::sdesc_sw128(bst + kk * 32);
             const uint32_t accum = (ks > 0 || kk > 0) ? 1u : 0u;
 #pragma unroll
             for (int mm = 0; mm < C::NA; ++mm)
-              tc::mma_bf16_ts(acc + mm * BN, ast + mm * 32 + kk * 8, bdesc, idesc, accum);
+              tc::mma_bf16_ts(acc + mm * BN, ast + mm * 32 + kk * 8, bdesc + static_cast<uint64_t>(kk * 2), idesc,
+                              accum);
           }
           tc::mma_commit(&empty_a[sa]);
           tc::mma_commit(&empty_b[sb]);
         }
-        if (!ok) break;
-        tc::mma_commit(&acc_full[buf]);
-        ++tt;
+        __syncwarp();
       }
-      // every issued MMA has finished before tensor memory is released
+      if (!ok) break;
+      if (leader) tc::mma_commit(&acc_full[buf]);
+      __syncwarp();
+      ++tt;
+    }
+    // every issued MMA has finished before tensor memory is released
+    if (leader) {
       tc::mma_commit(drain);
       tc::mbar_wait_drain(drain, 0, a.status);
     }
