@@ -36,12 +36,15 @@ sys.path.insert(0, ROOT)
 T_PREFILL = 4096
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PREFILL_LAUNCHES_PER_STEP = 6     # router (+ segment counts), scan, scatter, gate/up, down, combine
-DECODE_LAUNCHES_PER_STEP = 3      # routing (router+top-k+sort), gate/up GEMV, down GEMV+combine
+DECODE_LAUNCHES_PER_STEP = 3      # unfused: routing (router+top-k+sort), gate/up GEMV, down GEMV+combine
+FUSED_DECODE_LAUNCHES_PER_STEP = 1   # T <= 2: the whole layer in one cooperative launch
 COMPUTE_DTYPE = "bf16"            # grouped GEMM operands (FP32 accumulation in tensor memory)
 DOMINANT_KERNEL_SRC = "bit_quantized_expert_route_b200/csrc/gemm_tc.cu"
 DOMINANT_KERNEL = "grouped_gemm_tc_kernel<true>"
 DECODE_KERNEL_SRC = "bit_quantized_expert_route_b200/csrc/decode.cu"
 DECODE_KERNEL = "decode_gateup_kernel"
+FUSED_DECODE_KERNEL_SRC = "bit_quantized_expert_route_b200/csrc/decode_fused.cu"
+FUSED_DECODE_KERNEL = "decode_fused_kernel<1>"
 
 
 def parse_args(argv=None):
@@ -148,36 +151,53 @@ class ClockSampler:
 
 # --------------------------------------------------------------- helpers ---
 
-def dist_setup(n_gpus):
+def dist_setup(n_gpus, backend: str = "nccl"):
+    """One process per GPU: rank/world from the launcher's environment; the process group only
+    carries the barriers and the max-over-ranks timing (replicas exchange no data)."""
     import torch
     import torch.distributed as dist
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=60))
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return world, rank, local
 
 
-def barrier_sync(world):
+def barrier_sync(world, cuda: bool = True):
     import torch
     import torch.distributed as dist
-    torch.cuda.synchronize()
+    if cuda:
+        torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    torch.cuda.synchronize()
+    if cuda:
+        torch.cuda.synchronize()
 
 
-def max_over_ranks(v: float, world: int) -> float:
+def replica_seeds(rank: int, n_layers: int):
+    """Each replica draws its own layers and inputs: (layer seeds, activation seeds)."""
+    return [1000 * rank + 1 + i for i in range(n_layers)], [1000 * rank + 11 + i for i in range(n_layers)]
+
+
+def whole_job_rate(units_per_rank: float, world: int, ms_max: float) -> float:
+    """Units all ranks processed divided by the slowest rank's time."""
+    return units_per_rank * world / (ms_max / 1e3)
+
+
+def max_over_ranks(v: float, world: int, device: str = "cuda") -> float:
     if world == 1:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -203,9 +223,10 @@ def prefill_phase(a, world, rank, dev, dims, zipf, peaks, peak_src):
     import torch
     from bit_quantized_expert_route_b200 import moe, synth
     NL = a.layers
-    layers = [moe.MoELayer.from_tensors(dims, synth.make_layer_on_device(1000 * rank + 1 + i, i, dims, dev, zipf))
+    lseeds, xseeds = replica_seeds(rank, NL)
+    layers = [moe.MoELayer.from_tensors(dims, synth.make_layer_on_device(lseeds[i], i, dims, dev, zipf))
               for i in range(NL)]
-    xs = [synth.make_x_on_device(1000 * rank + 11 + i, T_PREFILL, dims.H, dev) for i in range(NL)]
+    xs = [synth.make_x_on_device(xseeds[i], T_PREFILL, dims.H, dev) for i in range(NL)]
     out = torch.empty_like(xs[0])
     ws = moe.alloc_workspace(layers[0], T_PREFILL, dev)
 
@@ -215,7 +236,7 @@ def prefill_phase(a, world, rank, dev, dims, zipf, peaks, peak_src):
     for i in range(a.warmup):
         step(i)
     total_ms = timed_loop(step, a.steps, world)
-    res = {"ms_per_step": total_ms / a.steps, "value": world * T_PREFILL * a.steps / (total_ms / 1e3)}
+    res = {"ms_per_step": total_ms / a.steps, "value": whole_job_rate(T_PREFILL * a.steps, world, total_ms)}
 
     if not a.no_stages:
         # per-stage device times over the same workload (events between stages)
@@ -250,7 +271,7 @@ def prefill_phase(a, world, rank, dev, dims, zipf, peaks, peak_src):
         for i in range(2):
             step_host(i)
         e2e_ms = timed_loop(step_host, a.steps, world)
-        res["e2e"] = {"value": round(world * T_PREFILL * a.steps / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+        res["e2e"] = {"value": round(whole_job_rate(T_PREFILL * a.steps, world, e2e_ms), 1), "unit": "tokens/s",
                       "h2d_bytes_per_step": T_PREFILL * dims.H * 2, "d2h_bytes_per_step": T_PREFILL * dims.H * 2}
     del layers, xs
     torch.cuda.empty_cache()
@@ -273,6 +294,9 @@ def decode_phase(a, world, rank, dev, dims, peaks, peak_src):
 
     for i in range(max(a.warmup, NLD)):
         dstep(i)
+    # one traced call tells which decode path runs (one fused launch or three)
+    fused = len(moe.moe_forward_profiled(dl[0], dx[0:1], dout, dws)) == 1
+    per_step = FUSED_DECODE_LAUNCHES_PER_STEP if fused else DECODE_LAUNCHES_PER_STEP
     d_ms = timed_loop(dstep, a.decode_steps, world)
     us_tok_stream = d_ms * 1e3 / a.decode_steps
     # the same layer calls captured once as a CUDA graph and replayed
@@ -303,19 +327,24 @@ def decode_phase(a, world, rank, dev, dims, peaks, peak_src):
            "active_expert_bytes": active_bytes,
            "active_bytes_GBps": round(active_bytes / (us_tok / 1e6) / 1e9, 1),
            "hbm_frac_active_bytes": round(active_bytes / (us_tok / 1e6) / 1e9 / peaks["hbm_gbs"], 4),
-           "gpu_launches": DECODE_LAUNCHES_PER_STEP * reps * NLD}
+           "gpu_launches": per_step * reps * NLD}
     if not a.no_stages:
         dst = {}
         for i in range(min(a.decode_steps, 200)):
             for k_, v in moe.moe_forward_profiled(dl[i % NLD], dx[i % 64:i % 64 + 1], dout, dws).items():
                 dst.setdefault(k_, []).append(v)
         dstage = {k_: statistics.median(v) for k_, v in dst.items()}
-        ach = gateup_bytes / (dstage["gateup"] / 1e3) / 1e9
-        trd = committed_traffic(DECODE_KERNEL, DECODE_KERNEL_SRC)
+        if fused:
+            # the one launch moves the active experts' weights (and the router matrix)
+            kern, src, alg, t_ms = FUSED_DECODE_KERNEL, FUSED_DECODE_KERNEL_SRC, active_bytes, dstage["decode_fused"]
+        else:
+            kern, src, alg, t_ms = DECODE_KERNEL, DECODE_KERNEL_SRC, gateup_bytes, dstage["gateup"]
+        ach = alg / (t_ms / 1e3) / 1e9
+        trd = committed_traffic(kern, src)
         res["stage_us"] = {k_: round(v * 1e3, 2) for k_, v in dstage.items()}
-        res["roofline"] = {"kernel": DECODE_KERNEL, "bound": "hbm", "achieved": round(ach, 1),
+        res["roofline"] = {"kernel": kern, "bound": "hbm", "achieved": round(ach, 1),
                            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4),
-                           "peak_source": f"{peak_src} HBM copy", "algorithmic_per_launch": gateup_bytes,
+                           "peak_source": f"{peak_src} HBM copy", "algorithmic_per_launch": alg,
                            "traffic": trd[0] if trd else None}
     del dl
     torch.cuda.empty_cache()

@@ -64,7 +64,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 // Byte offsets of every workspace buffer for a call with T tokens.
 struct WsLayout {
-  size_t status, counter, topk_idx, topk_w, counts, offsets, perm, inv_perm, sigma, seg, chunks, n_chunks,
+  size_t status, counter, grid_bar, topk_idx, topk_w, counts, offsets, perm, inv_perm, sigma, seg, chunks, n_chunks,
       active, n_active, logits, h, h_s, Y, x_stage, out_stage, total;
   int max_chunks;
 };
@@ -80,8 +80,9 @@ WsLayout ws_layout(const moe_layer_desc* d, int T) {
   const size_t n = static_cast<size_t>(T) * d->k;
   const int cr = gemm_chunk_rows();
   w.max_chunks = static_cast<int>(n / cr + T / cr + d->E + 2);
-  w.status = take(256);          // control block: status word, then the small-T routing counter
+  w.status = take(256);          // control block: status word, small-T routing counter, grid barrier
   w.counter = w.status + 4;
+  w.grid_bar = w.status + 8;     // [arrivals, generation] of the fused decode kernel's grid barrier
   w.topk_idx = take(n * 4);
   w.topk_w = take(n * 4);
   w.counts = take(static_cast<size_t>(d->E) * 4);
@@ -210,8 +211,29 @@ int enqueue_route(const moe_layer_desc* d, const uint16_t* x, int T, const Bufs&
   return cuda_status(e);
 }
 
+// Bulk copies of whole scale/bias tile rows need 16-byte aligned stacks.
+bool fused_decode_ok(const moe_layer_desc* d, const Geometry& g) {
+  const moe_qmat* m[6] = {&d->gate, &d->up, &d->down, &d->sh_gate, &d->sh_up, &d->sh_down};
+  for (const moe_qmat* q : m)
+    if (!aligned16(q->scales) || !aligned16(q->biases)) return false;
+  return decode_fused_supported(g);
+}
+
 int enqueue_decode(const moe_layer_desc* d, const uint16_t* x, int T, uint16_t* out, const Bufs& b,
                    cudaStream_t s, Tracer* tr = nullptr) {
+  {
+    const Geometry g{T, d->H, d->I, d->I_shared, d->E, d->k};
+    if (fused_decode_ok(d, g)) {
+      mark(tr, s);
+      const RoutingPtrs rp{b.topk_idx, b.topk_w, b.sigma, b.counts, b.offsets, b.perm, b.inv_perm};
+      const cudaError_t e = launch_decode_fused(
+          g, layer_ptrs(d), x, out, rp, b.at<int32_t>(b.w.active), b.at<int32_t>(b.w.n_active),
+          b.at<float>(b.w.logits), b.at<uint16_t>(b.w.h), b.at<uint16_t>(b.w.h_s), b.at<unsigned>(b.w.grid_bar),
+          b.at<int>(b.w.status), s);
+      mark(tr, s);
+      return cuda_status(e);
+    }
+  }
   int st = enqueue_route(d, x, T, b, s, tr);
   if (st != MOE_OK) return st;
   const Geometry g{T, d->H, d->I, d->I_shared, d->E, d->k};
@@ -427,7 +449,9 @@ int moe_get_status(void* ws, moe_stream stream) {
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   int host = 0;
   if (cudaMemcpyAsync(&host, ws, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ERR_CUDA;
-  if (cudaMemsetAsync(ws, 0, sizeof(int), s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  // a device timeout can leave the control block's counters mid-count: clear it whole
+  if (host != MOE_OK && cudaMemsetAsync(ws, 0, 16, s) != cudaSuccess) return MOE_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
   return host;
 }

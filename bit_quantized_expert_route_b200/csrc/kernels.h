@@ -95,4 +95,12 @@ cudaError_t launch_decode_down_combine(const Geometry& g, const LayerPtr& L, con
                                        const int32_t* inv_perm, const float* sigma, uint16_t* out,
                                        cudaStream_t s);
 
+// decode_fused.cu: the whole decode layer in one cooperative launch (T <= 2,
+// H a multiple of 1024 up to 2048).  bar: two zeroed workspace words (grid
+// barrier arrivals and generation); logits: workspace [T, E+1] FP32.
+bool decode_fused_supported(const Geometry& g);
+cudaError_t launch_decode_fused(const Geometry& g, const LayerPtr& L, const uint16_t* x, uint16_t* out,
+                                const RoutingPtrs& r, int32_t* active, int32_t* n_active, float* logits,
+                                uint16_t* h, uint16_t* h_s, unsigned* bar, int* status, cudaStream_t s);
+
 }  // namespace moe

@@ -234,6 +234,7 @@ def moe_rmsnorm(y: torch.Tensor, y_out: torch.Tensor, eps: float = 1e-6, stream=
 
 PREFILL_STAGES = ("router", "group", "gateup", "down", "combine")
 DECODE_STAGES = ("route", "gateup", "down_combine")
+FUSED_DECODE_STAGES = ("decode_fused",)
 
 
 def moe_forward_profiled(layer: MoELayer, x: torch.Tensor, out: torch.Tensor, workspace: torch.Tensor,
@@ -245,7 +246,7 @@ def moe_forward_profiled(layer: MoELayer, x: torch.Tensor, out: torch.Tensor, wo
     _check(library().moe_forward_profiled(ctypes.byref(layer.desc), x.data_ptr(), T, out.data_ptr(),
                                           workspace.data_ptr(), workspace.numel(), _stream(stream), ms,
                                           ctypes.byref(n)), "moe_forward_profiled")
-    names = PREFILL_STAGES if T > 64 else DECODE_STAGES
+    names = PREFILL_STAGES if T > 64 else (FUSED_DECODE_STAGES if n.value == 1 else DECODE_STAGES)
     return {names[i]: float(ms[i]) for i in range(n.value)}
 
 

@@ -157,7 +157,10 @@ MOE_API int moe_forward(const moe_layer_desc* layer, const moe_bf16* x, int T, m
 
 /* The same function for 1 <= T <= 64 through the bandwidth-bound decode
  * kernels (batch-1 decoding streams the active experts' weights: "How It
- * Works: Prefill and Decode Strategies").  T > 64 is MOE_ERR_INVALID_ARG. */
+ * Works: Prefill and Decode Strategies").  T > 64 is MOE_ERR_INVALID_ARG.
+ * For T <= 2 with H = 1024 or 2048 and 16-byte aligned scale and bias stacks
+ * the whole layer is ONE cooperative launch of one CTA per SM (grid-wide
+ * barriers in the workspace control block); otherwise three launches. */
 MOE_API int moe_decode(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_bf16* out,
                moe_routing* r, void* workspace, size_t workspace_bytes, moe_stream stream);
 
@@ -203,7 +206,9 @@ MOE_API int moe_rmsnorm(const moe_bf16* y, moe_bf16* y_out, int T, int H, float 
  * `stream` before the first and after every stage, waits for the stream, and
  * writes each stage's device time in milliseconds to stage_ms[0..n-1]:
  *   T > 64:  router, group (histogram+scan+scatter), gate/up GEMM, down GEMM, combine
- *   T <= 64: routing (one kernel), gate/up GEMV, down GEMV + combine
+ *   T <= 64: routing (one kernel), gate/up GEMV, down GEMV + combine, or a
+ *            single stage when the fused decode kernel runs (T <= 2,
+ *            H = 1024 or 2048, 16-byte aligned scale and bias stacks)
  * stage_ms: host array of at least 5 floats; *n_stages receives the count.
  * The events are created and destroyed inside the call. */
 MOE_API int moe_forward_profiled(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_bf16* out,

@@ -134,14 +134,46 @@ def test_rmsnorm_matches_oracle():
 
 # ------------------------------------------------------------- full layer --
 
-@pytest.mark.parametrize("T", [1, 8, 64])
+@pytest.mark.parametrize("T", [1, 2, 3, 8, 64])
 def test_full_decode(T):
+    # T <= 2 runs the single-launch fused decode kernel, larger T the unfused kernels
     lay, x, _ = workload(10 + T, T, FULL)
     ref = moe_ref.moe_layer(x, lay, FULL.k)
     gpu = run_layer(lay, x)
     assert gpu["status"] == 0
     assert_routing_exact(gpu, ref)
     assert_output_close(gpu["out"], ref["out"])
+
+
+@pytest.mark.parametrize("T", [1, 2])
+def test_full_decode_zipf(T):
+    lay, x, _ = workload(30 + T, T, FULL, zipf=True)
+    ref = moe_ref.moe_layer(x, lay, FULL.k)
+    gpu = run_layer(lay, x, entry="decode")
+    assert gpu["status"] == 0
+    assert_routing_exact(gpu, ref)
+    assert_output_close(gpu["out"], ref["out"])
+
+
+def test_full_decode_repeated_calls_one_workspace():
+    # the fused kernel's grid barrier state lives in the workspace control
+    # block: many calls in a row must keep giving the same bits
+    lay, x_bits, _ = workload(41, 1, FULL)
+    L = moe.MoELayer.from_synth(lay)
+    x = to_dev_bits(x_bits)
+    ws = moe.alloc_workspace(L, 1)
+    outs = []
+    for _ in range(5):
+        out = torch.empty_like(x)
+        moe.moe_decode(L, x, out, ws)
+        outs.append(out)
+    torch.cuda.synchronize()
+    assert moe.moe_get_status(ws) == 0
+    first = bits_of(outs[0])
+    for o in outs[1:]:
+        np.testing.assert_array_equal(bits_of(o), first)
+    ref = moe_ref.moe_layer(x_bits, lay, FULL.k)
+    assert_output_close(first, ref["out"])
 
 
 @pytest.fixture(scope="module", params=["uniform", "zipf"])
