@@ -68,16 +68,18 @@ struct FusedArgs {
   int off_bar, off_xs, off_xsum, off_hs, off_hsum, off_lg, off_rt, off_y;
 };
 
-// Routing state every CTA rebuilds in shared memory.
+// Routing state every CTA rebuilds in shared memory.  Expert slots in down
+// order: slot 0 is the shared expert (its rows are h rows T*k .. T*k+T-1),
+// slots 1..n_act the routed active experts ascending (rows off .. off+cnt-1).
 struct RouteSmem {
   int32_t idx[kFMaxT * kMaxK];
   float w[kFMaxT * kMaxK];
   float sigma[kFMaxT];
   int32_t perm[kFMaxT * kMaxK];
   int32_t inv_perm[kFMaxT * kMaxK];
-  int32_t counts[kMaxE];
-  int32_t offsets[kMaxE + 1];
-  int32_t active[kMaxE + 1];   // routed active experts ascending
+  int32_t slot_e[kFMaxT * kMaxK + 1];
+  int32_t slot_cnt[kFMaxT * kMaxK + 1];
+  int32_t slot_off[kFMaxT * kMaxK + 1];
   int32_t n_act;               // routed active experts
   int32_t abort;
 };
@@ -97,32 +99,13 @@ __device__ __forceinline__ void codes_f(uint32_t w, float (&f)[8]) {
   f[7] = __uint_as_float(((w >> 12) & M) | ONE);
 }
 
-// sum_i (1 + q_i/128) * v_i over the 32 codes of `qv`; v from an interleaved
-// staging row: float4 j of this lane's segment at vl[j * lanes].
-__device__ __forceinline__ float dot32f(const uint4& qv, const float4* __restrict__ vl, int lanes) {
-  const uint32_t words[4] = {qv.x, qv.y, qv.z, qv.w};
-  float a = 0.f;
-#pragma unroll
-  for (int wd = 0; wd < 4; ++wd) {
-    float f[8];
-    codes_f(words[wd], f);
-    const float4 v0 = vl[(2 * wd) * lanes];
-    const float4 v1 = vl[(2 * wd + 1) * lanes];
-    a = fmaf(f[0], v0.x, a); a = fmaf(f[1], v0.y, a); a = fmaf(f[2], v0.z, a); a = fmaf(f[3], v0.w, a);
-    a = fmaf(f[4], v1.x, a); a = fmaf(f[5], v1.y, a); a = fmaf(f[6], v1.z, a); a = fmaf(f[7], v1.w, a);
-  }
-  return a;
-}
-
 // Stage one bf16 row of n elements as FP32 in the `lanes`-interleaved layout
 // (element 32c + i at float4 ((c/lanes)*8 + i/4)*lanes + c%lanes).  Called by
-// `nthr` threads with index `tid`; l2_only reads through L2 (rows written by
-// other CTAs of this launch).
-__device__ __forceinline__ void stage_row_f(const uint16_t* src, int n, int lanes, float* dst, int tid, int nthr,
-                                            bool l2_only) {
+// `nthr` threads with index `tid`.
+__device__ __forceinline__ void stage_row_f(const uint16_t* src, int n, int lanes, float* dst, int tid, int nthr) {
   float4* d4 = reinterpret_cast<float4*>(dst);
   for (int u = tid; u < n / 8; u += nthr) {
-    const uint4 v = l2_only ? __ldcg(reinterpret_cast<const uint4*>(src) + u) : reinterpret_cast<const uint4*>(src)[u];
+    const uint4 v = reinterpret_cast<const uint4*>(src)[u];
     const int e0 = u * 8, c = e0 >> 5, ii = e0 & 31;
     const int win = c / lanes, ln = c - win * lanes;
     d4[(win * 8 + (ii >> 2)) * lanes + ln] = make_float4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y));
@@ -130,18 +113,79 @@ __device__ __forceinline__ void stage_row_f(const uint16_t* src, int n, int lane
   }
 }
 
+// Order-preserving 32-bit key of a float (larger float -> larger key; every
+// non-NaN float maps above 0).
+__device__ __forceinline__ uint32_t order_key(float f) {
+  const uint32_t u = f == 0.f ? 0u : __float_as_uint(f);   // -0 and +0 are one value
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Warp top-k over E <= 256 logits in shared memory with the same order as
+// the other routing kernels (larger logit first, equal logits -> lower expert
+// index): each pick is a lane-local scan of 8 keys and two warp reductions
+// (redux.sync max of the key, then min of the expert index among the lanes
+// holding that key).  Lane 0 writes the experts and exp(l_j - l_0) / sum.
+__device__ __forceinline__ void topk_redux(const float* lg, int E, int k, int lane, int32_t* idx_out,
+                                           float* w_out) {
+  uint32_t key[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int e = lane + 32 * i;
+    key[i] = e < E ? order_key(lg[e]) : 0u;
+  }
+  int sel[kMaxK];
+#pragma unroll
+  for (int j = 0; j < kMaxK; ++j) {
+    if (j < k) {
+      uint32_t best = 0u;
+      int bi = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (key[i] > best) {        // strictly greater: the lowest index among equal keys
+          best = key[i];
+          bi = i;
+        }
+      const uint32_t m = __reduce_max_sync(0xffffffffu, best);
+      const uint32_t cand = (best == m && m != 0u) ? static_cast<uint32_t>(lane + 32 * bi) : 0xffffffffu;
+      const uint32_t win = __reduce_min_sync(0xffffffffu, cand);
+      if (static_cast<int>(win & 31u) == lane) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (i == static_cast<int>(win >> 5)) key[i] = 0u;
+      }
+      sel[j] = static_cast<int>(win);
+    }
+  }
+  if (lane == 0) {
+    float z[kMaxK];
+    float sum = 0.f;
+    const float l0 = lg[sel[0]];
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j)
+      if (j < k) {
+        z[j] = expf(lg[sel[j]] - l0);
+        sum += z[j];
+      }
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j)
+      if (j < k) {
+        idx_out[j] = sel[j];
+        w_out[j] = z[j] / sum;
+      }
+  }
+}
+
 __device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kFWarps * 32) : "memory"); }
 
-// Grid-wide barrier, called by one thread per CTA (all CTAs co-resident).
-// bar[0] counts arrivals and is reset by the last arriver, which then bumps
-// the generation bar[1] with release semantics; the others wait (bounded)
-// for the generation to move.
+// Grid-wide barrier, called by one thread per CTA after a CTA barrier (all
+// CTAs co-resident).  bar[0] counts arrivals with acquire-release adds (each
+// arrival publishes its CTA's writes; the last arriver acquires them all),
+// the last arriver resets it and bumps the generation bar[1] with a release
+// store; the others spin (bounded) on an acquire load of the generation.
 __device__ bool grid_barrier(unsigned* bar, unsigned nblocks, int* status) {
   const unsigned gen = tc::ld_acquire_gpu(bar + 1);
-  __threadfence();
-  if (atomicAdd(bar, 1u) == nblocks - 1) {
+  if (tc::atom_add_acq_rel_gpu(bar, 1u) == nblocks - 1) {
     atomicExch(bar, 0u);
-    __threadfence();
     tc::st_release_gpu(bar + 1, gen + 1);
     return true;
   }
@@ -151,19 +195,21 @@ __device__ bool grid_barrier(unsigned* bar, unsigned nblocks, int* status) {
       if (status) atomicExch(status, kStatusTimeout);
       return false;
     }
-    __nanosleep(64);
   }
   return true;
 }
 
 // Unit schedule of one CTA: its gate/up units u = c, c+G, ... over the
-// global list [shared-expert units | routed units], then its down units.
+// global list [shared-expert units | routed units], then its down units
+// (dim blocks c, c+G, ..., each split into parts of at most spd_max slots,
+// balanced).
 struct Sched {
   int n_gu_units;      // global gate/up units
   int n_sh_units;      // of which shared-expert units (first)
   int units_per_exp;   // I / 16
   int n_slots;         // down slots: shared + routed active
   int n_down_parts;    // down units per dim block
+  int spd;             // slots per down unit (the last may have fewer)
   int n_blocks;        // dim blocks (H / 16)
   int my_gu, my_blocks;
 };
@@ -175,6 +221,7 @@ __device__ __forceinline__ Sched make_sched(const FusedArgs& a, int n_act) {
   s.n_gu_units = s.n_sh_units + n_act * s.units_per_exp;
   s.n_slots = n_act + 1;
   s.n_down_parts = (s.n_slots + a.spd - 1) / a.spd;
+  s.spd = (s.n_slots + s.n_down_parts - 1) / s.n_down_parts;
   s.n_blocks = a.g.H / kFDims;
   const int G = gridDim.x, c = blockIdx.x;
   s.my_gu = s.n_gu_units > c ? (s.n_gu_units - c + G - 1) / G : 0;
@@ -182,20 +229,24 @@ __device__ __forceinline__ Sched make_sched(const FusedArgs& a, int n_act) {
   return s;
 }
 
-// Expert of down slot j: slot 0 is the shared expert (index E), then the
-// routed active experts in ascending order.
-__device__ __forceinline__ int slot_expert(const RouteSmem& rt, int E, int j) { return j == 0 ? E : rt.active[j - 1]; }
+// Gate/up unit u: expert slot (0 = shared) and first feature.
+__device__ __forceinline__ void gu_unit(const Sched& s, int u, int& slot, int& f0) {
+  const bool sh = u < s.n_sh_units;
+  slot = sh ? 0 : 1 + (u - s.n_sh_units) / s.units_per_exp;
+  f0 = (sh ? u : (u - s.n_sh_units) % s.units_per_exp) * kFFeat;
+}
 
 // Issue the bulk copies of unit i of this CTA into ring slot `dst`.
+// gate/up layout: [q gate 16 rows][q up 16 rows][s gate][b gate][s up][b up];
+// down layout: per expert slot jj at jj * 9 Kmax: [q 16 rows][s][b].
 __device__ void issue_unit(const FusedArgs& a, const RouteSmem& rt, const Sched& s, int i, uint32_t dst,
                            uint64_t* full) {
   const Geometry& g = a.g;
   if (i < s.my_gu) {
-    const int u = blockIdx.x + i * gridDim.x;
-    const bool sh = u < s.n_sh_units;
-    const int e = sh ? g.E : rt.active[(u - s.n_sh_units) / s.units_per_exp];
-    const int f0 = (sh ? u : (u - s.n_sh_units) % s.units_per_exp) * kFFeat;
-    const size_t row0 = static_cast<size_t>(sh ? 0 : e * g.I) + f0;
+    int slot, f0;
+    gu_unit(s, blockIdx.x + i * gridDim.x, slot, f0);
+    const bool sh = slot == 0;
+    const size_t row0 = static_cast<size_t>(sh ? 0 : rt.slot_e[slot] * g.I) + f0;
     const QMatPtr Wg = sh ? a.L.sh_gate : a.L.gate;
     const QMatPtr Wu = sh ? a.L.sh_up : a.L.up;
     const uint32_t qb = kFFeat * g.H / 2, sb = kFFeat * g.H / 32;
@@ -210,27 +261,84 @@ __device__ void issue_unit(const FusedArgs& a, const RouteSmem& rt, const Sched&
   }
   const int di = i - s.my_gu;
   const int blk = blockIdx.x + (di / s.n_down_parts) * gridDim.x;
-  const int part = di % s.n_down_parts;
-  const int j0 = part * a.spd, nj = min(a.spd, s.n_slots - j0);
+  const int j0 = (di % s.n_down_parts) * s.spd, nj = min(s.spd, s.n_slots - j0);
   const int Kmax = max(g.I, g.Is);
   uint32_t bytes = 0;
   for (int jj = 0; jj < nj; ++jj) {
-    const bool sh = j0 + jj == 0;
-    const int K = sh ? g.Is : g.I;
+    const int K = j0 + jj == 0 ? g.Is : g.I;
     bytes += kFDims * K / 2 + 2 * (kFDims * K / 32);
   }
   tc::mbar_arrive_expect_tx(full, bytes);
   for (int jj = 0; jj < nj; ++jj) {
-    const int e = slot_expert(rt, g.E, j0 + jj);
-    const bool sh = e == g.E;
+    const bool sh = j0 + jj == 0;
     const int K = sh ? g.Is : g.I;
     const QMatPtr W = sh ? a.L.sh_down : a.L.down;
-    const size_t row0 = static_cast<size_t>(sh ? 0 : e * g.H) + blk * kFDims;
+    const size_t row0 = static_cast<size_t>(sh ? 0 : rt.slot_e[j0 + jj] * g.H) + blk * kFDims;
     const uint32_t base = dst + jj * (9 * Kmax);
     const uint32_t qb = kFDims * K / 2, sb = kFDims * K / 32;
     tc::bulk_load(base, W.q + row0 * (K / 8), qb, full);
     tc::bulk_load(base + 8 * Kmax, W.s + row0 * (K / kGroup), sb, full);
     tc::bulk_load(base + 8 * Kmax + Kmax / 2, W.b + row0 * (K / kGroup), sb, full);
+  }
+}
+
+// Sum over the warp of v[r(lane)] with r(lane) = 4*bit4 + 2*bit3 + bit2 of
+// the lane: a transposing butterfly (9 shuffles for 8 values).
+__device__ __forceinline__ float warp_reduce8(const float (&v)[8], int lane) {
+  const bool h16 = lane & 16, h8 = lane & 8, h4 = lane & 4;
+  float a4[4], a2[2];
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    a4[j] = (h16 ? v[j + 4] : v[j]) + __shfl_xor_sync(0xffffffffu, h16 ? v[j] : v[j + 4], 16);
+#pragma unroll
+  for (int j = 0; j < 2; ++j)
+    a2[j] = (h8 ? a4[j + 2] : a4[j]) + __shfl_xor_sync(0xffffffffu, h8 ? a4[j] : a4[j + 2], 8);
+  float r = (h4 ? a2[1] : a2[0]) + __shfl_xor_sync(0xffffffffu, h4 ? a2[0] : a2[1], 4);
+  r += __shfl_xor_sync(0xffffffffu, r, 2);
+  r += __shfl_xor_sync(0xffffffffu, r, 1);
+  return r;
+}
+
+// Sum over each half-warp of v[r(lane)] with r(lane) = 2*bit3 + bit2.
+__device__ __forceinline__ float halfwarp_reduce4(const float (&v)[4], int lane) {
+  const bool h8 = lane & 8, h4 = lane & 4;
+  float a2[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j)
+    a2[j] = (h8 ? v[j + 2] : v[j]) + __shfl_xor_sync(0xffffffffu, h8 ? v[j] : v[j + 2], 8);
+  float r = (h4 ? a2[1] : a2[0]) + __shfl_xor_sync(0xffffffffu, h4 ? a2[0] : a2[1], 4);
+  r += __shfl_xor_sync(0xffffffffu, r, 2);
+  r += __shfl_xor_sync(0xffffffffu, r, 1);
+  return r;
+}
+
+// sum_i (1 + q_i/128) * v_i for the 32 codes of qv against 32 staged values
+// held in registers (v[0..31]), four partial sums.
+__device__ __forceinline__ float dot32r(const uint4& qv, const float (&v)[32]) {
+  const uint32_t words[4] = {qv.x, qv.y, qv.z, qv.w};
+  float p[4];
+#pragma unroll
+  for (int wd = 0; wd < 4; ++wd) {
+    float f[8];
+    codes_f(words[wd], f);
+    float acc = f[0] * v[8 * wd];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) acc = fmaf(f[i], v[8 * wd + i], acc);
+    p[wd] = acc;
+  }
+  return (p[0] + p[1]) + (p[2] + p[3]);
+}
+
+// Load one 32-element segment of a staged row (interleave `lanes`) into registers.
+__device__ __forceinline__ void load_seg(const float* row, int c, int lanes, float (&v)[32]) {
+  const float4* r4 = reinterpret_cast<const float4*>(row) + ((c / lanes) * 8) * lanes + (c % lanes);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float4 q = r4[j * lanes];
+    v[4 * j] = q.x;
+    v[4 * j + 1] = q.y;
+    v[4 * j + 2] = q.z;
+    v[4 * j + 3] = q.w;
   }
 }
 
@@ -280,7 +388,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
   }
   if (!producer) {
     const int tid = threadIdx.x, nthr = kFWarps * 32;
-    for (int t = 0; t < T; ++t) stage_row_f(a.x + static_cast<size_t>(t) * g.H, g.H, 32, xs + t * xst, tid, nthr, false);
+    for (int t = 0; t < T; ++t) stage_row_f(a.x + static_cast<size_t>(t) * g.H, g.H, 32, xs + t * xst, tid, nthr);
     // router rows r = c, c + G, ...: warp w sums the K slice [w H/16, (w+1) H/16)
     const int nrows = (E1 - static_cast<int>(blockIdx.x) + gridDim.x - 1) / gridDim.x;
     const int kslice = g.H / kFWarps;
@@ -345,77 +453,50 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
   }
 
   // ---------------------------------------------------------------- phase B
+  // Every CTA rebuilds the routing from the logits (top-k by warp reductions,
+  // then a one-warp counting sort of the n = T*k <= 16 entries), so no
+  // further barrier is needed before the expert weights can be requested.
   for (int i = threadIdx.x; i < T * E1; i += blockDim.x) lg[i] = __ldcg(a.logits + i);
   __syncthreads();
   if (warp < T) {
-    select_topk_warp(lg + warp * E1, E, k, lane, rt.idx + warp * k, rt.w + warp * k);
+    topk_redux(lg + warp * E1, E, k, lane, rt.idx + warp * k, rt.w + warp * k);
     if (lane == 0) rt.sigma[warp] = sigmoid(lg[warp * E1 + E]);
   }
-  for (int e = threadIdx.x; e < E; e += blockDim.x) rt.counts[e] = 0;
   __syncthreads();
   const int n = T * k;
+  const int Tk = n;
   if (warp == 0) {
-    // counting sort of the n <= 16 entries: counts, offsets, stable ranks
-    for (int i = lane; i < n; i += 32) atomicAdd(&rt.counts[rt.idx[i]], 1);
-    __syncwarp();
-    int run = 0, nact = 0;
-    for (int e0 = 0; e0 < E; e0 += 32) {
-      const int e = e0 + lane;
-      const int c = e < E ? rt.counts[e] : 0;
-      int incl = c, act = c > 0 ? 1 : 0;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, o);
-        const int va = __shfl_up_sync(0xffffffffu, act, o);
-        if (lane >= o) {
-          incl += v;
-          act += va;
-        }
+    const bool live = lane < n;
+    const int e_i = live ? rt.idx[lane] : -1 - lane;          // distinct dummies for idle lanes
+    const unsigned peers = __match_any_sync(0xffffffffu, e_i);
+    const int rank = __popc(peers & lanemask_lt());           // same expert, earlier (token, slot)
+    const bool first = live && rank == 0;
+    const unsigned firsts = __ballot_sync(0xffffffffu, first);
+    int below = 0, abelow = 0;                                // entries / active experts with a smaller expert
+    for (int j = 0; j < n; ++j) {
+      const int ej = __shfl_sync(0xffffffffu, e_i, j);
+      below += ej < e_i ? 1 : 0;
+      abelow += (((firsts >> j) & 1u) && ej < e_i) ? 1 : 0;
+    }
+    if (live) {
+      const int pos = below + rank;
+      rt.perm[pos] = lane;
+      rt.inv_perm[lane] = pos;
+      if (first) {
+        rt.slot_e[1 + abelow] = e_i;
+        rt.slot_cnt[1 + abelow] = __popc(peers);
+        rt.slot_off[1 + abelow] = below;
       }
-      if (e < E) {
-        rt.offsets[e] = run + incl - c;
-        if (c > 0) rt.active[nact + act - 1] = e;
-      }
-      run += __shfl_sync(0xffffffffu, incl, 31);
-      nact += __shfl_sync(0xffffffffu, act, 31);
     }
     if (lane == 0) {
-      rt.offsets[E] = run;
-      rt.n_act = nact;
-    }
-    __syncwarp();
-    if (lane == 0) {
-      // stable scatter (entries in (token, slot) order)
-      int cur[kFMaxT * kMaxK];
-      for (int i = 0; i < n; ++i) {
-        int r = 0;
-        for (int j = 0; j < i; ++j) r += rt.idx[j] == rt.idx[i] ? 1 : 0;
-        cur[i] = rt.offsets[rt.idx[i]] + r;
-      }
-      for (int i = 0; i < n; ++i) {
-        rt.perm[cur[i]] = i;
-        rt.inv_perm[i] = cur[i];
-      }
+      rt.n_act = __popc(firsts);
+      rt.slot_e[0] = E;
+      rt.slot_cnt[0] = T;
+      rt.slot_off[0] = Tk;
     }
   }
   __syncthreads();
   const Sched s = make_sched(a, rt.n_act);
-  if (blockIdx.x == 0) {
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-      a.r.topk_idx[i] = rt.idx[i];
-      a.r.topk_w[i] = rt.w[i];
-      a.r.perm[i] = rt.perm[i];
-      a.r.inv_perm[i] = rt.inv_perm[i];
-    }
-    for (int e = threadIdx.x; e < E; e += blockDim.x) a.r.counts[e] = rt.counts[e];
-    for (int e = threadIdx.x; e <= E; e += blockDim.x) a.r.offsets[e] = rt.offsets[e];
-    for (int j = threadIdx.x; j < rt.n_act; j += blockDim.x) a.active[j] = rt.active[j];
-    if (threadIdx.x < T) a.r.sigma[threadIdx.x] = rt.sigma[threadIdx.x];
-    if (threadIdx.x == 0) {
-      a.active[rt.n_act] = E;
-      *a.n_active = rt.n_act + 1;
-    }
-  }
   const int n_units = s.my_gu + s.my_blocks * s.n_down_parts;
 
   if (producer) {
@@ -440,63 +521,101 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
   }
 
   // ------------------------------------------------------ consumer warps
+  // gate/up, two units at a time: warp pair p = warp / 2 owns 8 of the 64
+  // rows (2 units x 16 features x {gate, up}); thread (p, c) keeps segment c
+  // of every token's staged x in registers and runs 8 independent dot
+  // products against it.
   bool ok = true;
-  const int Tk = T * k;
-  for (int i = 0; i < s.my_gu && ok; ++i) {
-    const int sl = i % a.ring;
-    if (!tc::mbar_wait(&full[sl], (i / a.ring) & 1u, abort_flag, a.status)) {
-      ok = false;
-      break;
+  float* red = lg;   // [8 pairs][2 halves][8 rows][NT] partial sums (logits are no longer needed)
+  const int pr = warp >> 1, half = warp & 1;
+  const int nch = g.H / 32;
+  const uint32_t qb = kFFeat * g.H / 2, sb = kFFeat * g.H / 32;
+  for (int i0 = 0; i0 < s.my_gu && ok; i0 += 2) {
+    const int nu = min(2, s.my_gu - i0);
+    for (int ui = 0; ui < nu && ok; ++ui) {
+      const int i = i0 + ui;
+      if (!tc::mbar_wait(&full[i % a.ring], (i / a.ring) & 1u, abort_flag, a.status)) ok = false;
     }
-    const int u = blockIdx.x + i * gridDim.x;
-    const bool sh = u < s.n_sh_units;
-    const int e = sh ? E : rt.active[(u - s.n_sh_units) / s.units_per_exp];
-    const int f = (sh ? u : (u - s.n_sh_units) % s.units_per_exp) * kFFeat + warp;
-    const int nt = sh ? T : rt.counts[e];
-    const int pos0 = sh ? 0 : rt.offsets[e];
-    const uint8_t* slot = fsm + sl * a.slot_bytes;
-    const uint32_t qb = kFFeat * g.H / 2, sb = kFFeat * g.H / 32;
-    const uint4* qg = reinterpret_cast<const uint4*>(slot + warp * (g.H / 2));
-    const uint4* qu = reinterpret_cast<const uint4*>(slot + qb + warp * (g.H / 2));
-    const uint16_t* sg = reinterpret_cast<const uint16_t*>(slot + 2 * qb) + warp * (g.H / kGroup);
-    const uint16_t* bg = reinterpret_cast<const uint16_t*>(slot + 2 * qb + sb) + warp * (g.H / kGroup);
-    const uint16_t* su = reinterpret_cast<const uint16_t*>(slot + 2 * qb + 2 * sb) + warp * (g.H / kGroup);
-    const uint16_t* bu = reinterpret_cast<const uint16_t*>(slot + 2 * qb + 3 * sb) + warp * (g.H / kGroup);
-    int tok[NT];
+    if (!ok) break;
+    // this pair's rows: r = 8 pr + rr; unit r / 32, matrix (r / 16) & 1, feature r & 15
+    const int ur = (8 * pr) >> 5;
+    const bool rows_live = ur < nu;
+    int slot = 0, f0 = 0;
+    if (rows_live) gu_unit(s, blockIdx.x + (i0 + ur) * gridDim.x, slot, f0);
+    const int m = ((8 * pr) >> 4) & 1, fb = (8 * pr) & 15;     // rows rr = 0..7: features fb .. fb+7
+    const uint8_t* base = fsm + ((i0 + ur) % a.ring) * a.slot_bytes;
+    const uint8_t* qrow0 = base + m * qb + fb * (g.H / 2);
+    const uint16_t* srow0 = reinterpret_cast<const uint16_t*>(base + 2 * qb + m * 2 * sb) + fb * (g.H / kGroup);
+    const uint16_t* brow0 = reinterpret_cast<const uint16_t*>(base + 2 * qb + m * 2 * sb + sb) + fb * (g.H / kGroup);
+    // tokens of this unit's expert: routed slot -> its rows' tokens; shared -> 0..T-1
+    unsigned tmask = 0;
+    if (rows_live) {
+      if (slot == 0)
+        tmask = (1u << T) - 1u;
+      else
+        for (int r = 0; r < rt.slot_cnt[slot]; ++r) tmask |= 1u << (rt.perm[rt.slot_off[slot] + r] / k);
+    }
+    float acc[8][NT];
 #pragma unroll
-    for (int t = 0; t < NT; ++t) tok[t] = t < nt ? (sh ? t : rt.perm[pos0 + t] / k) : 0;
-    float ag[NT], au[NT];
+    for (int rr = 0; rr < 8; ++rr)
 #pragma unroll
-    for (int t = 0; t < NT; ++t) ag[t] = au[t] = 0.f;
-    for (int c = lane; c < g.H / 32; c += 32) {
-      const uint4 vg = qg[c], vu = qu[c];
-      const float s_g = 128.f * bf16_bits_to_float(sg[c >> 1]), b_g = bf16_bits_to_float(bg[c >> 1]);
-      const float s_u = 128.f * bf16_bits_to_float(su[c >> 1]), b_u = bf16_bits_to_float(bu[c >> 1]);
+      for (int t = 0; t < NT; ++t) acc[rr][t] = 0.f;
+    if (rows_live) {
+      for (int c = half * 32 + lane; c < nch; c += 64) {
 #pragma unroll
-      for (int t = 0; t < NT; ++t) {
-        if (t < nt) {
-          const float4* xl = reinterpret_cast<const float4*>(xs + tok[t] * xst) + ((c >> 5) * 8) * 32 + (c & 31);
-          const float X = xsum[tok[t] * (xst / 32) + c];
-          ag[t] = fmaf(s_g, dot32f(vg, xl, 32), fmaf(b_g - s_g, X, ag[t]));
-          au[t] = fmaf(s_u, dot32f(vu, xl, 32), fmaf(b_u - s_u, X, au[t]));
+        for (int t = 0; t < NT; ++t) {
+          if ((tmask >> t) & 1u) {
+            float xv[32];
+            load_seg(xs + t * xst, c, 32, xv);
+            const float X = xsum[t * (xst / 32) + c];
+#pragma unroll
+            for (int rr = 0; rr < 8; ++rr) {
+              const uint4 qv = reinterpret_cast<const uint4*>(qrow0 + rr * (g.H / 2))[c];
+              const float s128 = 128.f * bf16_bits_to_float(srow0[rr * (g.H / kGroup) + (c >> 1)]);
+              const float bb = bf16_bits_to_float(brow0[rr * (g.H / kGroup) + (c >> 1)]);
+              acc[rr][t] = fmaf(s128, dot32r(qv, xv), fmaf(bb - s128, X, acc[rr][t]));
+            }
+          }
         }
       }
     }
-    // the slot's words are consumed: release it (generic reads before the async refill)
+    // every read of the pair's slots is done: release them
     tc::fence_proxy_async_smem();
     __syncwarp();
-    if (lane == 0) tc::mbar_arrive(&empty[sl]);
+    if (lane == 0)
+      for (int ui = 0; ui < nu; ++ui) tc::mbar_arrive(&empty[(i0 + ui) % a.ring]);
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
-      const float gs = warp_sum(ag[t]), us = warp_sum(au[t]);
-      if (lane == 0 && t < nt) {
-        const uint16_t hv = float_to_bf16_bits(silu(gs) * us);
-        if (sh)
-          a.h_s[static_cast<size_t>(t) * g.Is + f] = hv;
-        else
-          a.h[static_cast<size_t>(pos0 + t) * g.I + f] = hv;
-      }
+      float v[8];
+#pragma unroll
+      for (int rr = 0; rr < 8; ++rr) v[rr] = acc[rr][t];
+      const float r = warp_reduce8(v, lane);
+      if ((lane & 3) == 0) red[((pr * 2 + half) * 8 + (lane >> 2)) * NT + t] = r;
     }
+    consumers_sync();
+    // h = bf16(silu(g) * u) for (unit, feature, token)
+    for (int q = threadIdx.x; q < nu * kFFeat * T; q += kFWarps * 32) {
+      const int ui = q / (kFFeat * T), f = (q / T) % kFFeat, t = q % T;
+      int uslot, uf0;
+      gu_unit(s, blockIdx.x + (i0 + ui) * gridDim.x, uslot, uf0);
+      bool member = uslot == 0;
+      int pos = t;
+      for (int r = 0; r < (uslot == 0 ? 0 : rt.slot_cnt[uslot]); ++r)
+        if (rt.perm[rt.slot_off[uslot] + r] / k == t) {
+          member = true;
+          pos = rt.slot_off[uslot] + r;
+        }
+      if (!member) continue;
+      const int rg = ui * 32 + f, ru = ui * 32 + 16 + f;      // gate and up rows of the pair
+      const float gs = red[(((rg >> 3) * 2 + 0) * 8 + (rg & 7)) * NT + t] + red[(((rg >> 3) * 2 + 1) * 8 + (rg & 7)) * NT + t];
+      const float us = red[(((ru >> 3) * 2 + 0) * 8 + (ru & 7)) * NT + t] + red[(((ru >> 3) * 2 + 1) * 8 + (ru & 7)) * NT + t];
+      const uint16_t hv = float_to_bf16_bits(silu(gs) * us);
+      if (uslot == 0)
+        a.h_s[static_cast<size_t>(t) * g.Is + uf0 + f] = hv;
+      else
+        a.h[static_cast<size_t>(pos) * g.I + uf0 + f] = hv;
+    }
+    consumers_sync();   // red is reused by the next pair
   }
   // Every h row is written: grid barrier (consumer thread 0 of each CTA).
   consumers_sync();
@@ -507,10 +626,18 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
   if (s.my_blocks > 0) {
     // stage every h row (routed rows I wide, shared rows Is wide; stride hst)
     const int tid = threadIdx.x, nthr = kFWarps * 32;
-    for (int r = 0; r < Tk + T; ++r) {
+    const int vmax = Kmax / 8;
+    for (int i = tid; i < (Tk + T) * vmax; i += nthr) {
+      const int r = i / vmax, u = i - r * vmax;
       const bool shr = r >= Tk;
+      if (u * 8 >= (shr ? g.Is : g.I)) continue;
       const uint16_t* src = shr ? a.h_s + static_cast<size_t>(r - Tk) * g.Is : a.h + static_cast<size_t>(r) * g.I;
-      stage_row_f(src, shr ? g.Is : g.I, 16, hs + r * hst, tid, nthr, true);
+      const uint4 v = __ldcg(reinterpret_cast<const uint4*>(src) + u);
+      const int c = u >> 2, ii = (u & 3) * 8;
+      float4* d4 = reinterpret_cast<float4*>(hs + r * hst);
+      const int win = c >> 4, ln = c & 15;
+      d4[(win * 8 + (ii >> 2)) * 16 + ln] = make_float4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y));
+      d4[(win * 8 + (ii >> 2) + 1) * 16 + ln] = make_float4(bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w));
     }
     consumers_sync();
     for (int i = tid; i < (Tk + T) * (hst / 32); i += nthr) {
@@ -530,7 +657,11 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
     }
     consumers_sync();
   }
-  const int hl = lane & 15, hh = lane >> 4;
+  // down units: half-warp hw = 2 warp + (lane >> 4) owns (slot jj = hw / 4,
+  // dims 4 (hw % 4) .. +3) of the unit; lane hl = lane & 15 walks segments
+  // c = hl, hl + 16, ... with the slot's staged h rows in registers.
+  const int hl = lane & 15, hw = warp * 2 + (lane >> 4);
+  const int jj = hw >> 2, dg = hw & 3;
   for (int di = 0; di < s.my_blocks * s.n_down_parts && ok; ++di) {
     const int i = s.my_gu + di;
     const int sl = i % a.ring;
@@ -539,50 +670,53 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
       break;
     }
     const int bl = di / s.n_down_parts;
-    const int j0 = (di % s.n_down_parts) * a.spd, nj = min(a.spd, s.n_slots - j0);
-    const uint8_t* slot = fsm + sl * a.slot_bytes;
-    // warp = output dim of the block; half-warps take the unit's slots in pairs
-    for (int jj0 = 0; jj0 < nj; jj0 += 2) {
-      const int jj = jj0 + hh;
-      const bool live = jj < nj;
-      const int e = live ? slot_expert(rt, E, j0 + jj) : E;
-      const bool sh = e == E;
-      const int K = sh ? g.Is : g.I;
-      const int nt = live ? (sh ? T : rt.counts[e]) : 0;
-      const int pos0 = sh ? Tk : (live ? rt.offsets[e] : 0);
-      const uint8_t* base = slot + jj * (9 * Kmax);
-      const uint4* qrow = reinterpret_cast<const uint4*>(base + warp * (K / 2));
-      const uint16_t* srow = reinterpret_cast<const uint16_t*>(base + 8 * Kmax) + warp * (K / kGroup);
-      const uint16_t* brow = reinterpret_cast<const uint16_t*>(base + 8 * Kmax + Kmax / 2) + warp * (K / kGroup);
-      float p[NT];
+    const int j0 = (di % s.n_down_parts) * s.spd, nj = min(s.spd, s.n_slots - j0);
+    const bool live = jj < nj;
+    const int j = j0 + jj;
+    const bool sh = j == 0;
+    const int K = sh ? g.Is : g.I;
+    const int nt = live ? rt.slot_cnt[j] : 0;
+    const int pos0 = live ? rt.slot_off[j] : 0;
+    const uint8_t* base = fsm + sl * a.slot_bytes + jj * (9 * Kmax);
+    const uint8_t* qrow0 = base + (dg * 4) * (K / 2);
+    const uint16_t* srow0 = reinterpret_cast<const uint16_t*>(base + 8 * Kmax) + (dg * 4) * (K / kGroup);
+    const uint16_t* brow0 = reinterpret_cast<const uint16_t*>(base + 8 * Kmax + Kmax / 2) + (dg * 4) * (K / kGroup);
+    float p[4][NT];
 #pragma unroll
-      for (int t = 0; t < NT; ++t) p[t] = 0.f;
-      if (live) {
-        for (int c = hl; c < K / 32; c += 16) {
-          const uint4 qv = qrow[c];
-          const float s128 = 128.f * bf16_bits_to_float(srow[c >> 1]), bb = bf16_bits_to_float(brow[c >> 1]);
+    for (int d = 0; d < 4; ++d)
 #pragma unroll
-          for (int t = 0; t < NT; ++t) {
-            if (t < nt) {
-              const int r = pos0 + t;
-              const float4* hl4 = reinterpret_cast<const float4*>(hs + r * hst) + ((c >> 4) * 8) * 16 + (c & 15);
-              const float X = hsum[r * (hst / 32) + c];
-              p[t] = fmaf(s128, dot32f(qv, hl4, 16), fmaf(bb - s128, X, p[t]));
+      for (int t = 0; t < NT; ++t) p[d][t] = 0.f;
+    if (live) {
+      for (int c = hl; c < K / 32; c += 16) {
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          if (t < nt) {
+            const int r = pos0 + t;
+            float hv[32];
+            load_seg(hs + r * hst, c, 16, hv);
+            const float X = hsum[r * (hst / 32) + c];
+#pragma unroll
+            for (int d = 0; d < 4; ++d) {
+              const uint4 qv = reinterpret_cast<const uint4*>(qrow0 + d * (K / 2))[c];
+              const float s128 = 128.f * bf16_bits_to_float(srow0[d * (K / kGroup) + (c >> 1)]);
+              const float bb = bf16_bits_to_float(brow0[d * (K / kGroup) + (c >> 1)]);
+              p[d][t] = fmaf(s128, dot32r(qv, hv), fmaf(bb - s128, X, p[d][t]));
             }
           }
         }
-      }
-#pragma unroll
-      for (int t = 0; t < NT; ++t) {
-        float v = p[t];
-#pragma unroll
-        for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (hl == 0 && t < nt) ys[((pos0 + t) * s.my_blocks + bl) * kFDims + warp] = v;
       }
     }
     tc::fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) tc::mbar_arrive(&empty[sl]);
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      float v[4];
+#pragma unroll
+      for (int d = 0; d < 4; ++d) v[d] = p[d][t];
+      const float r = halfwarp_reduce4(v, lane);
+      if ((hl & 3) == 0 && t < nt) ys[((pos0 + t) * s.my_blocks + bl) * kFDims + dg * 4 + (hl >> 2)] = r;
+    }
   }
   consumers_sync();
   if (!ok) return;
@@ -596,6 +730,30 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
     acc = fmaf(rt.sigma[t], ys[((Tk + t) * s.my_blocks + bl) * kFDims + d], acc);
     const int blk = blockIdx.x + bl * gridDim.x;
     a.out[static_cast<size_t>(t) * g.H + blk * kFDims + d] = float_to_bf16_bits(acc);
+  }
+  if (blockIdx.x == 0) {
+    // routing outputs (off the other CTAs' critical path)
+    for (int i = threadIdx.x; i < n; i += kFWarps * 32) {
+      a.r.topk_idx[i] = rt.idx[i];
+      a.r.topk_w[i] = rt.w[i];
+      a.r.perm[i] = rt.perm[i];
+      a.r.inv_perm[i] = rt.inv_perm[i];
+    }
+    for (int e = threadIdx.x; e <= E; e += kFWarps * 32) {
+      int c = 0, below = 0;
+      for (int i = 0; i < n; ++i) {
+        c += rt.idx[i] == e ? 1 : 0;
+        below += rt.idx[i] < e ? 1 : 0;
+      }
+      if (e < E) a.r.counts[e] = c;
+      a.r.offsets[e] = below;
+    }
+    for (int jx = threadIdx.x; jx < rt.n_act; jx += kFWarps * 32) a.active[jx] = rt.slot_e[1 + jx];
+    if (threadIdx.x < T) a.r.sigma[threadIdx.x] = rt.sigma[threadIdx.x];
+    if (threadIdx.x == 0) {
+      a.active[rt.n_act] = E;
+      *a.n_active = rt.n_act + 1;
+    }
   }
 }
 

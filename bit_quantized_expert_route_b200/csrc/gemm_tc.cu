@@ -23,14 +23,14 @@
 //
 // One persistent CTA per SM walks the device-built unit list
 //   unit = (chunk of <= 128 rows of one expert) x (block of 128 weight rows).
-// Warp roles (480 threads):
-//   warps 0-7   dequantisers (gate/up: warps 0-3 gate rows, 4-7 up rows;
-//               down: warps 0-3 even stages, 4-7 odd stages); TMEM lane
-//               quadrant = warp % 4 = row / 32
-//   warps 8-11  epilogue (lane quadrant = warp % 4)
-//   warp 12     token tiles (cp.async gathers, or one lane issuing TMA)
-//   warp 13     one lane issues the TMA loads of packed tiles and scales
-//   warp 14     tensor-memory allocation; one lane issues tcgen05.mma
+// Warp roles (736 threads):
+//   warps 0-15  dequantisers in 4 sets of 4 (gate/up: set = stage parity x
+//               matrix; down: set = stage mod 4); TMEM lane quadrant =
+//               warp % 4 = row / 32
+//   warps 16-19 epilogue (lane quadrant = warp % 4)
+//   warp 20     token tiles (cp.async gathers, or one lane issuing TMA)
+//   warp 21     one lane issues the TMA loads of packed tiles and scales
+//   warp 22     tensor-memory allocation; one lane issues tcgen05.mma
 // Tensor memory (512 columns): gate/up = one accumulator pair (gate, up:
 // 2 x 128 columns) + 4 A stages of 64 columns; down = two accumulators of 128
 // columns (double-buffered) + 8 A stages of 32 columns.
@@ -50,11 +50,12 @@ constexpr int kBStages = 6;      // token-tile ring
 constexpr int kBLag = 3;         // gather cp.async groups in flight before signalling
 constexpr int kPStages = 8;      // packed-tile ring
 constexpr int kSBlock = 8;       // quantisation groups per scale block (16 B per row)
-constexpr int kThreads = 480;
-constexpr int kEpiWarp0 = 8;
-constexpr int kLoadWarp = 12;
-constexpr int kTmaWarp = 13;
-constexpr int kMmaWarp = 14;
+constexpr int kDqWarps = 16;     // dequantiser warps (4 sets of 4: one per TMEM lane quadrant)
+constexpr int kEpiWarp0 = kDqWarps;
+constexpr int kLoadWarp = kEpiWarp0 + 4;
+constexpr int kTmaWarp = kLoadWarp + 1;
+constexpr int kMmaWarp = kTmaWarp + 1;
+constexpr int kThreads = (kMmaWarp + 1) * 32;
 constexpr uint32_t kTmemCols = 512;
 
 template <bool kGateUp>
@@ -190,7 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
     }
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&full_s[s], 1);
-      tc::mbar_init(&empty_s[s], 256);
+      tc::mbar_init(&empty_s[s], kDqWarps * 32);   // every dequantiser releases every block once
     }
     for (int s = 0; s < C::A_STAGES; ++s) {
       tc::mbar_init(&full_a[s], C::DQ_PER_STAGE);
@@ -219,11 +220,18 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
   if (warp < kEpiWarp0) {
     // ------------------------------------------------------- dequantisers
     const int r = threadIdx.x & 127;                 // weight row of the tile == TMEM lane
-    const int set = warp >> 2;                       // gate/up: matrix; down: stage parity
-    const int m = kGateUp ? set : 0;
+    // 4 sets of 4 warps.  gate/up: set = (stage parity, matrix); down: set =
+    // stage index mod 4.  Each stage is rebuilt by 128 threads per matrix, and
+    // a warp works on every second (gate/up) or fourth (down) stage, so the
+    // latency of one stage's loads, dequantisation and TMEM store overlaps the
+    // other sets' work.
+    const int set = warp >> 2;
+    const int m = kGateUp ? (set & 1) : 0;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const int psw = (r >> 2) & 1;                    // 32-byte swizzle of the packed tile rows
-    auto mine = [&](uint32_t it) { return kGateUp || static_cast<int>(it & 1u) == set; };
+    auto mine = [&](uint32_t it) {
+      return kGateUp ? static_cast<int>(it & 1u) == (set >> 1) : static_cast<int>(it & 3u) == set;
+    };
     StageCursor<kGateUp> cur;
     cur.begin(a, n_units, nfb);
     while (!cur.done && !mine(cur.it)) cur.next(a, n_units, nfb);
