@@ -81,6 +81,28 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const uint16_t* __restrict
   }
 }
 
+// xp = x with every group of 8 elements in the order (0,4,1,5,2,6,3,7), the
+// K order of the grouped GEMMs' operands.  One thread per 16 bytes.
+__global__ void __launch_bounds__(256) interleave_k8_kernel(const uint4* __restrict__ x, uint4* __restrict__ xp,
+                                                           size_t n16) {
+  const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n16) return;
+  const uint4 v = x[i];                                   // (x0,x1) (x2,x3) (x4,x5) (x6,x7)
+  uint4 o;
+  o.x = __byte_perm(v.x, v.z, 0x5410);                    // (x0, x4)
+  o.y = __byte_perm(v.x, v.z, 0x7632);                    // (x1, x5)
+  o.z = __byte_perm(v.y, v.w, 0x5410);                    // (x2, x6)
+  o.w = __byte_perm(v.y, v.w, 0x7632);                    // (x3, x7)
+  xp[i] = o;
+}
+
+cudaError_t launch_interleave_k8(const uint16_t* x, uint16_t* xp, int T, int H, cudaStream_t s) {
+  const size_t n16 = static_cast<size_t>(T) * H / 8;
+  interleave_k8_kernel<<<static_cast<unsigned>((n16 + 255) / 256), 256, 0, s>>>(
+      reinterpret_cast<const uint4*>(x), reinterpret_cast<uint4*>(xp), n16);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_combine(const uint16_t* Y, const int32_t* inv_perm, const float* topk_w, const float* sigma,
                            int T, int k, int H, uint16_t* out, cudaStream_t s) {
   combine_kernel<<<T, 256, 0, s>>>(Y, inv_perm, topk_w, sigma, T, k, H, out);

@@ -16,6 +16,11 @@
 //   in shared memory in the 128-byte swizzled K-major layout: gathered with
 //   cp.async (gate/up: rows of x picked by the permutation) or loaded by TMA
 //   (down: the chunk's rows of h are contiguous).
+// * Inside every group of 8 inputs the K order of both operands is
+//   (0,4,1,5,2,6,3,7): the order in which one AND-OR pulls code pairs out of
+//   a packed word.  x arrives in that order from a small interleaving pass,
+//   and the gate/up epilogue writes h in it, so the dequantiser needs no byte
+//   permutes.  A dot product does not depend on the order of its terms.
 // * FP32 accumulators live in tensor memory.  Epilogue warps read them, apply
 //   the epilogue (gate/up: h = bf16(silu(g) * u); down: Y = bf16(acc)), stage
 //   the tile in shared memory, release the accumulator, and only then write
@@ -23,14 +28,15 @@
 //
 // One persistent CTA per SM walks the device-built unit list
 //   unit = (chunk of <= 128 rows of one expert) x (block of 128 weight rows).
-// Warp roles (736 threads):
+// Warp roles (832 threads):
 //   warps 0-15  dequantisers in 4 sets of 4 (gate/up: set = stage parity x
 //               matrix; down: set = stage mod 4); TMEM lane quadrant =
 //               warp % 4 = row / 32
 //   warps 16-19 epilogue (lane quadrant = warp % 4)
-//   warp 20     token tiles (cp.async gathers, or one lane issuing TMA)
-//   warp 21     one lane issues the TMA loads of packed tiles and scales
-//   warp 22     tensor-memory allocation; one lane issues tcgen05.mma
+//   warps 20-23 token tiles: gate/up, each lane gathers one row with cp.async;
+//               down, one lane issues a 2-D TMA per stage
+//   warp 24     one lane issues the TMA loads of packed tiles and scales
+//   warp 25     tensor-memory allocation; one lane issues tcgen05.mma
 // Tensor memory (512 columns): gate/up = one accumulator pair (gate, up:
 // 2 x 128 columns) + 4 A stages of 64 columns; down = two accumulators of 128
 // columns (double-buffered) + 8 A stages of 32 columns.
@@ -52,8 +58,9 @@ constexpr int kPStages = 8;      // packed-tile ring
 constexpr int kSBlock = 8;       // quantisation groups per scale block (16 B per row)
 constexpr int kDqWarps = 16;     // dequantiser warps (4 sets of 4: one per TMEM lane quadrant)
 constexpr int kEpiWarp0 = kDqWarps;
-constexpr int kLoadWarp = kEpiWarp0 + 4;
-constexpr int kTmaWarp = kLoadWarp + 1;
+constexpr int kLoadWarp = kEpiWarp0 + 4;   // first of kLoadWarps token-tile warps
+constexpr int kLoadWarps = 4;              // gate/up: one gathered row per lane
+constexpr int kTmaWarp = kLoadWarp + kLoadWarps;
 constexpr int kMmaWarp = kTmaWarp + 1;
 constexpr int kThreads = (kMmaWarp + 1) * 32;
 constexpr uint32_t kTmemCols = 512;
@@ -182,7 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
   const bool b_by_tma = !kGateUp;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kBStages; ++s) {
-      tc::mbar_init(&full_b[s], b_by_tma ? 1 : 32);
+      tc::mbar_init(&full_b[s], b_by_tma ? 1 : kLoadWarps * 32);
       tc::mbar_init(&empty_b[s], 1);
     }
     for (int s = 0; s < kPStages; ++s) {
@@ -312,6 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
     // ----------------------------------------------------------- epilogue
     const int q = warp & 3;
     const int r = q * 32 + lane;                     // weight row == TMEM lane == output feature in tile
+    const int rpos = kGateUp ? tc::k8_pos(r) : r;    // h is stored in the K order of the down GEMM
     const int et = threadIdx.x - kEpiWarp0 * 32;     // 0..127
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
     uint16_t* stage = reinterpret_cast<uint16_t*>(smem + C::OFF_OUT);   // [BN tokens][BM features]
@@ -333,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const float g = v0[j];
-            stage[(n0 + j) * BM + r] = float_to_bf16_bits(__fdividef(g * v1[j], 1.0f + __expf(-g)));
+            stage[(n0 + j) * BM + rpos] = float_to_bf16_bits(__fdividef(g * v1[j], 1.0f + __expf(-g)));
           }
         } else {
           tc::tmem_wait_ld();
@@ -362,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
       if (!tc::mbar_wait(&epi_sync[1], tt & 1u, abort_flag, a.status)) break;
       ++tt;
     }
-  } else if (warp == kLoadWarp) {
+  } else if (warp < kTmaWarp) {
     // ------------------------------------------------------- token tiles
     uint32_t it = 0;
     bool ok = true;
@@ -370,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
       const UnitInfo ui = unit_info<kGateUp>(a, u, nfb);
       if (ui.skip) continue;
       if (b_by_tma) {
-        if (lane == 0) {
+        if (warp == kLoadWarp && lane == 0) {
           const void* tm = &a.tm_h[ui.shared ? 1 : 0];
           const int y = ui.shared ? ui.row0 - Tk : ui.row0;
           for (int ks = 0; ks < ui.nks; ++ks, ++it) {
@@ -387,33 +395,26 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
         it = __shfl_sync(0xffffffffu, it, 0);
         continue;
       }
-      const uint16_t* brow[BN / 32];
-#pragma unroll
-      for (int i = 0; i < BN / 32; ++i) {
-        const int rr = lane + i * 32;
-        brow[i] = nullptr;
-        if (rr < ui.rows) {
-          const int R = ui.row0 + rr;
-          const int tok = ui.shared ? (R - Tk) : (a.perm[R] / a.g.k);
-          brow[i] = a.x + static_cast<size_t>(tok) * a.g.H;
-        }
+      // lane of loader warp lw gathers tile row rr = 32 lw + lane
+      const int rr = (warp - kLoadWarp) * 32 + lane;
+      const uint16_t* brow = nullptr;
+      if (rr < ui.rows) {
+        const int R = ui.row0 + rr;
+        const int tok = ui.shared ? (R - Tk) : (a.perm[R] / a.g.k);
+        brow = a.x + static_cast<size_t>(tok) * a.g.H;
       }
+      const uint32_t rsw = static_cast<uint32_t>(rr & 7);
       for (int ks = 0; ks < ui.nks; ++ks, ++it) {
         const int s = static_cast<int>(it % kBStages);
         if (!tc::mbar_wait(&empty_b[s], ((it / kBStages) & 1u) ^ 1u, abort_flag, a.status)) {
           ok = false;
           break;
         }
-        const uint32_t st = sbase + C::OFF_B + s * C::B_BYTES;
+        if (brow) {
+          const uint32_t dst = sbase + C::OFF_B + s * C::B_BYTES + rr * 128;
+          const uint16_t* src = brow + ks * BK;
 #pragma unroll
-        for (int i = 0; i < BN / 32; ++i) {
-          if (brow[i]) {
-            const int rr = lane + i * 32;
-            const uint32_t dst = st + rr * 128;
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-              tc::cp_async16(dst + ((c ^ (rr & 7)) << 4), brow[i] + ks * BK + c * 8);
-          }
+          for (int c = 0; c < 8; ++c) tc::cp_async16(dst + ((c ^ rsw) << 4), src + c * 8);
         }
         tc::cp_async_commit();
         if (it >= static_cast<uint32_t>(kBLag)) {

@@ -81,6 +81,9 @@ cudaError_t launch_down(const Geometry& g, const LayerPtr& L, const uint16_t* h,
                         uint16_t* Y, int* status, cudaStream_t s);
 
 // combine.cu
+// xp = x with each group of 8 elements reordered (0,4,1,5,2,6,3,7): the K
+// order of the grouped GEMMs' operands (x and xp: [T, H] bf16, 16-B aligned).
+cudaError_t launch_interleave_k8(const uint16_t* x, uint16_t* xp, int T, int H, cudaStream_t s);
 cudaError_t launch_combine(const uint16_t* Y, const int32_t* inv_perm, const float* topk_w, const float* sigma,
                            int T, int k, int H, uint16_t* out, cudaStream_t s);
 cudaError_t launch_rmsnorm(const uint16_t* y, uint16_t* out, int T, int H, float eps, cudaStream_t s);

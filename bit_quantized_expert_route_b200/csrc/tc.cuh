@@ -264,18 +264,19 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 }
 
 // Eight 4-bit codes of one packed word (code i in bits 4i..4i+3) to eight bf16
-// weights w_i = bf16(scale * q_i + bias), in code order, as four bf16x2 words.
-// Codes enter as bf16 values 128 + q (exponent of 128, q in the low mantissa
-// bits), minus 128 gives q exactly, and one fused multiply-add rounds
-// scale * q + bias to bf16 once.
+// weights w_i = bf16(scale * q_i + bias), as four bf16x2 words holding the
+// code pairs (q0,q4) (q1,q5) (q2,q6) (q3,q7): the order one AND-OR per pair
+// produces.  The tensor-core operands use the same order along K inside
+// every group of 8 (the activations are permuted to match), so no byte
+// permute is needed.  Codes enter as bf16 values 128 + q (exponent of 128, q
+// in the low mantissa bits), minus 128 gives q exactly, and one fused
+// multiply-add rounds scale * q + bias to bf16 once.
 __device__ __forceinline__ uint4 dequant8(uint32_t w, __nv_bfloat162 s2, __nv_bfloat162 b2) {
   const uint32_t kMask = 0x000F000Fu, kMagic = 0x43004300u;     // bf16 128.0 in both halves
-  const uint32_t a04 = lop3_and_or(w, kMask, kMagic);           // (q0, q4)
-  const uint32_t a15 = lop3_and_or(w >> 4, kMask, kMagic);      // (q1, q5)
-  const uint32_t a26 = lop3_and_or(w >> 8, kMask, kMagic);      // (q2, q6)
-  const uint32_t a37 = lop3_and_or(w >> 12, kMask, kMagic);     // (q3, q7)
-  uint32_t p[4] = {prmt(a04, a15, 0x5410u), prmt(a26, a37, 0x5410u), prmt(a04, a15, 0x7632u),
-                   prmt(a26, a37, 0x7632u)};                      // (q0,q1) (q2,q3) (q4,q5) (q6,q7)
+  uint32_t p[4] = {lop3_and_or(w, kMask, kMagic),               // (q0, q4)
+                   lop3_and_or(w >> 4, kMask, kMagic),          // (q1, q5)
+                   lop3_and_or(w >> 8, kMask, kMagic),          // (q2, q6)
+                   lop3_and_or(w >> 12, kMask, kMagic)};        // (q3, q7)
   const __nv_bfloat162 c128 = __floats2bfloat162_rn(128.f, 128.f);
   uint4 out;
   uint32_t* o = reinterpret_cast<uint32_t*>(&out);
@@ -286,6 +287,12 @@ __device__ __forceinline__ uint4 dequant8(uint32_t w, __nv_bfloat162 s2, __nv_bf
     o[i] = *reinterpret_cast<uint32_t*>(&r);
   }
   return out;
+}
+
+// Position of element i of an 8-group in that interleaved order
+// (0,4,1,5,2,6,3,7): element i < 4 sits at 2i, element 4 + i at 2i + 1.
+__host__ __device__ __forceinline__ int k8_pos(int i) {
+  return (i & ~7) | ((i & 3) << 1) | ((i >> 2) & 1);
 }
 
 }  // namespace tc
