@@ -65,7 +65,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // Byte offsets of every workspace buffer for a call with T tokens.
 struct WsLayout {
   size_t status, counter, grid_bar, topk_idx, topk_w, counts, offsets, perm, inv_perm, sigma, seg, chunks, n_chunks,
-      active, n_active, logits, h, h_s, Y, x_perm, x_stage, out_stage, total;
+      active, n_active, logits, h, h_s, Y, x_stage, out_stage, total;
   int max_chunks;
 };
 
@@ -98,8 +98,7 @@ WsLayout ws_layout(const moe_layer_desc* d, int T) {
   w.logits = take(static_cast<size_t>(T <= kDecodeMaxT ? T : 0) * (d->E + 1) * 4);
   w.h = take(n * d->I * 2);
   w.h_s = take(static_cast<size_t>(T) * d->I_shared * 2);
-  w.Y = take((n + T) * d->H * 2);
-  w.x_perm = take(static_cast<size_t>(T > kDecodeMaxT ? T : 0) * d->H * 2);   // x in the GEMMs' K order
+  w.Y = take((n + T) * d->H * 2);   // also holds the gate/up GEMM's grouped token rows before the down GEMM
   w.x_stage = take(static_cast<size_t>(T) * d->H * 2);
   w.out_stage = take(static_cast<size_t>(T) * d->H * 2);
   w.total = off;
@@ -262,10 +261,10 @@ int enqueue_prefill(const moe_layer_desc* d, const uint16_t* x, int T, uint16_t*
   int* status = b.at<int>(b.w.status);
   const Chunk* chunks = b.at<Chunk>(b.w.chunks);
   const int32_t* n_chunks = b.at<int32_t>(b.w.n_chunks);
-  uint16_t* xp = b.at<uint16_t>(b.w.x_perm);
-  cudaError_t e = launch_interleave_k8(x, xp, T, d->H, s);
+  // the grouped token rows live in Y's storage until the down GEMM overwrites it
+  cudaError_t e = launch_gather_k8(x, b.perm, T, d->k, d->H, Y, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
-  e = launch_gateup(g, L, xp, b.perm, chunks, n_chunks, b.w.max_chunks, h, h_s, status, s);
+  e = launch_gateup(g, L, Y, chunks, n_chunks, b.w.max_chunks, h, h_s, status, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   mark(tr, s);
   e = launch_down(g, L, h, h_s, chunks, n_chunks, b.w.max_chunks, Y, status, s);

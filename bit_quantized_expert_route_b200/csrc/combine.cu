@@ -81,25 +81,31 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const uint16_t* __restrict
   }
 }
 
-// xp = x with every group of 8 elements in the order (0,4,1,5,2,6,3,7), the
-// K order of the grouped GEMMs' operands.  One thread per 16 bytes.
-__global__ void __launch_bounds__(256) interleave_k8_kernel(const uint4* __restrict__ x, uint4* __restrict__ xp,
-                                                           size_t n16) {
+// xg[R] = x[perm[R] / k] (R < T*k) or x[R - T*k] (the shared expert's rows),
+// with every group of 8 elements in the order (0,4,1,5,2,6,3,7): the gate/up
+// GEMM's token rows, contiguous per expert group, in its K order.  One thread
+// per 16 bytes.
+__global__ void __launch_bounds__(256) gather_k8_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ perm,
+                                                       int Tk, int k, int h8, size_t n16, uint4* __restrict__ xg) {
   const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= n16) return;
-  const uint4 v = x[i];                                   // (x0,x1) (x2,x3) (x4,x5) (x6,x7)
+  const int row = static_cast<int>(i / h8), c = static_cast<int>(i % h8);
+  const int t = row < Tk ? __ldg(perm + row) / k : row - Tk;
+  const uint4 v = __ldg(x + static_cast<size_t>(t) * h8 + c);   // (x0,x1) (x2,x3) (x4,x5) (x6,x7)
   uint4 o;
-  o.x = __byte_perm(v.x, v.z, 0x5410);                    // (x0, x4)
-  o.y = __byte_perm(v.x, v.z, 0x7632);                    // (x1, x5)
-  o.z = __byte_perm(v.y, v.w, 0x5410);                    // (x2, x6)
-  o.w = __byte_perm(v.y, v.w, 0x7632);                    // (x3, x7)
-  xp[i] = o;
+  o.x = __byte_perm(v.x, v.z, 0x5410);                        // (x0, x4)
+  o.y = __byte_perm(v.x, v.z, 0x7632);                        // (x1, x5)
+  o.z = __byte_perm(v.y, v.w, 0x5410);                        // (x2, x6)
+  o.w = __byte_perm(v.y, v.w, 0x7632);                        // (x3, x7)
+  xg[i] = o;
 }
 
-cudaError_t launch_interleave_k8(const uint16_t* x, uint16_t* xp, int T, int H, cudaStream_t s) {
-  const size_t n16 = static_cast<size_t>(T) * H / 8;
-  interleave_k8_kernel<<<static_cast<unsigned>((n16 + 255) / 256), 256, 0, s>>>(
-      reinterpret_cast<const uint4*>(x), reinterpret_cast<uint4*>(xp), n16);
+cudaError_t launch_gather_k8(const uint16_t* x, const int32_t* perm, int T, int k, int H, uint16_t* xg,
+                             cudaStream_t s) {
+  const int h8 = H / 8;
+  const size_t n16 = (static_cast<size_t>(T) * k + T) * h8;
+  gather_k8_kernel<<<static_cast<unsigned>((n16 + 255) / 256), 256, 0, s>>>(
+      reinterpret_cast<const uint4*>(x), perm, T * k, k, h8, n16, reinterpret_cast<uint4*>(xg));
   return cudaGetLastError();
 }
 

@@ -13,14 +13,14 @@
 //   memory, where the MMA reads it as its A operand.  The dense tile never
 //   touches shared memory.
 // * The expert's tokens are the MMA's N dimension (16..128 per chunk), staged
-//   in shared memory in the 128-byte swizzled K-major layout: gathered with
-//   cp.async (gate/up: rows of x picked by the permutation) or loaded by TMA
-//   (down: the chunk's rows of h are contiguous).
+//   in shared memory in the 128-byte swizzled K-major layout by one 2-D TMA
+//   per stage: the chunk's rows are contiguous (gate/up: a gather pass has
+//   written x's rows in grouped order; down: h is produced in that order).
 // * Inside every group of 8 inputs the K order of both operands is
 //   (0,4,1,5,2,6,3,7): the order in which one AND-OR pulls code pairs out of
-//   a packed word.  x arrives in that order from a small interleaving pass,
-//   and the gate/up epilogue writes h in it, so the dequantiser needs no byte
-//   permutes.  A dot product does not depend on the order of its terms.
+//   a packed word.  The gather pass writes x in that order and the gate/up
+//   epilogue writes h in it, so the dequantiser needs no byte permutes.  A
+//   dot product does not depend on the order of its terms.
 // * FP32 accumulators live in tensor memory.  Epilogue warps read them, apply
 //   the epilogue (gate/up: h = bf16(silu(g) * u); down: Y = bf16(acc)), stage
 //   the tile in shared memory, release the accumulator, and only then write
@@ -28,15 +28,14 @@
 //
 // One persistent CTA per SM walks the device-built unit list
 //   unit = (chunk of <= 128 rows of one expert) x (block of 128 weight rows).
-// Warp roles (832 threads):
+// Warp roles (736 threads):
 //   warps 0-15  dequantisers in 4 sets of 4 (gate/up: set = stage parity x
 //               matrix; down: set = stage mod 4); TMEM lane quadrant =
 //               warp % 4 = row / 32
 //   warps 16-19 epilogue (lane quadrant = warp % 4)
-//   warps 20-23 token tiles: gate/up, each lane gathers one row with cp.async;
-//               down, one lane issues a 2-D TMA per stage
-//   warp 24     one lane issues the TMA loads of packed tiles and scales
-//   warp 25     tensor-memory allocation; one lane issues tcgen05.mma
+//   warp 20     token tiles: one lane issues a 2-D TMA per stage
+//   warp 21     one lane issues the TMA loads of packed tiles and scales
+//   warp 22     tensor-memory allocation; one lane issues tcgen05.mma
 // Tensor memory (512 columns): gate/up = one accumulator pair (gate, up:
 // 2 x 128 columns) + 4 A stages of 64 columns; down = two accumulators of 128
 // columns (double-buffered) + 8 A stages of 32 columns.
@@ -58,12 +57,12 @@ constexpr int kPStages = 8;      // packed-tile ring
 constexpr int kSBlock = 8;       // quantisation groups per scale block (16 B per row)
 constexpr int kDqWarps = 16;     // dequantiser warps (4 sets of 4: one per TMEM lane quadrant)
 constexpr int kEpiWarp0 = kDqWarps;
-constexpr int kLoadWarp = kEpiWarp0 + 4;   // first of kLoadWarps token-tile warps
-constexpr int kLoadWarps = 4;              // gate/up: one gathered row per lane
-constexpr int kTmaWarp = kLoadWarp + kLoadWarps;
+constexpr int kLoadWarp = kEpiWarp0 + 4;   // token tiles
+constexpr int kTmaWarp = kLoadWarp + 1;
 constexpr int kMmaWarp = kTmaWarp + 1;
 constexpr int kThreads = (kMmaWarp + 1) * 32;
 constexpr uint32_t kTmemCols = 512;
+constexpr int kMaxCtaUnits = 256;   // chunk descriptors cached in shared memory per CTA
 
 template <bool kGateUp>
 struct Cfg {
@@ -83,7 +82,8 @@ struct Cfg {
   static constexpr int OFF_S = OFF_P + kPStages * NA * P_BYTES;
   static constexpr int OFF_OUT = OFF_S + 2 * S_SLOT;
   static constexpr int BAR_OFF = OFF_OUT + OUT_BYTES;
-  static constexpr int SMEM = BAR_OFF + 512 + 1024;           // barriers + alignment slack
+  static constexpr int OFF_UNITS = BAR_OFF + 512;             // this CTA's chunk descriptors
+  static constexpr int SMEM = OFF_UNITS + kMaxCtaUnits * 16 + 1024;   // + alignment slack
   static constexpr int DQ_PER_STAGE = kGateUp ? 256 : 128;    // dequant threads consuming one stage
 };
 
@@ -91,12 +91,10 @@ struct alignas(64) TcArgs {
   CUtensorMap tm_q[2][2];  // packed words: [routed, shared][matrix]
   CUtensorMap tm_s[2][2];  // scales:       [routed, shared][matrix] (valid when scales_tma)
   CUtensorMap tm_b[2][2];  // biases
-  CUtensorMap tm_h[2];     // down: token tiles of h [routed, shared]
+  CUtensorMap tm_h[2];     // token tiles: gate/up [grouped x rows, -], down [routed h, shared h]
   Geometry g;
   QMatPtr W0, W1;          // routed stacks: {gate, up} or {down, -}
   QMatPtr S0, S1;          // shared expert: {sh_gate, sh_up} or {sh_down, -}
-  const uint16_t* x;       // gate/up: token rows [T, H]
-  const int32_t* perm;
   uint16_t* h_out;         // gate/up output, routed [T*k, I]
   uint16_t* hs_out;        // gate/up output, shared [T, Is]
   uint16_t* Y;             // down output, bf16 [(T*k + T), H]
@@ -113,8 +111,12 @@ struct UnitInfo {
 };
 
 template <bool kGateUp>
-__device__ __forceinline__ UnitInfo unit_info(const TcArgs& a, int u, int nfb) {
-  const Chunk ch = a.chunks[u / nfb];
+__device__ __forceinline__ UnitInfo unit_info(const TcArgs& a, int u, int nfb, const Chunk* cache) {
+  // this CTA's units are u = blockIdx.x + i * gridDim.x; their chunks were
+  // copied to shared memory at the start, so the per-stage bookkeeping of
+  // every role never waits on a global load
+  const int i = (u - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x);
+  const Chunk ch = i < kMaxCtaUnits ? cache[i] : a.chunks[u / nfb];
   UnitInfo ui;
   ui.shared = ch.e >= a.g.E;
   ui.e = ch.e;
@@ -139,9 +141,10 @@ struct StageCursor {
   bool done;
   UnitInfo ui;
 
+  const Chunk* cache;
   __device__ __forceinline__ void seek_unit(const TcArgs& a, int from, int n_units, int nfb) {
     for (u = from; u < n_units; u += gridDim.x) {
-      ui = unit_info<kGateUp>(a, u, nfb);
+      ui = unit_info<kGateUp>(a, u, nfb, cache);
       if (!ui.skip) {
         ks = 0;
         done = false;
@@ -150,7 +153,8 @@ struct StageCursor {
     }
     done = true;
   }
-  __device__ __forceinline__ void begin(const TcArgs& a, int n_units, int nfb) {
+  __device__ __forceinline__ void begin(const TcArgs& a, int n_units, int nfb, const Chunk* units) {
+    cache = units;
     it = 0;
     blk = 0;
     seek_unit(a, blockIdx.x, n_units, nfb);
@@ -186,10 +190,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool b_by_tma = !kGateUp;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kBStages; ++s) {
-      tc::mbar_init(&full_b[s], b_by_tma ? 1 : kLoadWarps * 32);
+      tc::mbar_init(&full_b[s], 1);
       tc::mbar_init(&empty_b[s], 1);
     }
     for (int s = 0; s < kPStages; ++s) {
@@ -214,15 +217,19 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
     *abort_flag = 0;
     tc::fence_barrier_init();
   }
+  const int nfb = (kGateUp ? max(a.g.I, a.g.Is) : a.g.H) / BM;
+  const int n_units = *a.n_chunks * nfb;
+  const int Tk = a.g.T * a.g.k;
+  Chunk* units = reinterpret_cast<Chunk*>(smem + C::OFF_UNITS);
+  for (int i = threadIdx.x; i < kMaxCtaUnits; i += blockDim.x) {
+    const int u = static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
+    if (u < n_units) units[i] = a.chunks[u / nfb];
+  }
   if (warp == kMmaWarp) tc::tmem_alloc(tmem_slot, kTmemCols);
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
-  const int nfb = (kGateUp ? max(a.g.I, a.g.Is) : a.g.H) / BM;
-  const int n_units = *a.n_chunks * nfb;
-  const int Tk = a.g.T * a.g.k;
 
   if (warp < kEpiWarp0) {
     // ------------------------------------------------------- dequantisers
@@ -240,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
       return kGateUp ? static_cast<int>(it & 1u) == (set >> 1) : static_cast<int>(it & 3u) == set;
     };
     StageCursor<kGateUp> cur;
-    cur.begin(a, n_units, nfb);
+    cur.begin(a, n_units, nfb, units);
     while (!cur.done && !mine(cur.it)) cur.next(a, n_units, nfb);
     bool ok = true;
     uint32_t held_blk = 0xffffffffu;                 // scale block this thread still holds
@@ -325,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
     uint16_t* stage = reinterpret_cast<uint16_t*>(smem + C::OFF_OUT);   // [BN tokens][BM features]
     uint32_t tt = 0;
     for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
-      const UnitInfo ui = unit_info<kGateUp>(a, u, nfb);
+      const UnitInfo ui = unit_info<kGateUp>(a, u, nfb, units);
       if (ui.skip) continue;
       const int buf = static_cast<int>(tt % C::ACC_BUFS);
       if (!tc::mbar_wait(&acc_full[buf], (tt / C::ACC_BUFS) & 1u, abort_flag, a.status)) break;
@@ -370,73 +377,35 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
       if (!tc::mbar_wait(&epi_sync[1], tt & 1u, abort_flag, a.status)) break;
       ++tt;
     }
-  } else if (warp < kTmaWarp) {
+  } else if (warp == kLoadWarp) {
     // ------------------------------------------------------- token tiles
-    uint32_t it = 0;
-    bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const UnitInfo ui = unit_info<kGateUp>(a, u, nfb);
-      if (ui.skip) continue;
-      if (b_by_tma) {
-        if (warp == kLoadWarp && lane == 0) {
-          const void* tm = &a.tm_h[ui.shared ? 1 : 0];
-          const int y = ui.shared ? ui.row0 - Tk : ui.row0;
-          for (int ks = 0; ks < ui.nks; ++ks, ++it) {
-            const int s = static_cast<int>(it % kBStages);
-            if (!tc::mbar_wait(&empty_b[s], ((it / kBStages) & 1u) ^ 1u, abort_flag, a.status)) {
-              ok = false;
-              break;
-            }
-            tc::mbar_arrive_expect_tx(&full_b[s], C::B_BYTES);
-            tc::tma_load_2d(sbase + C::OFF_B + s * C::B_BYTES, tm, ks * BK, y, &full_b[s]);
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        const UnitInfo ui = unit_info<kGateUp>(a, u, nfb, units);
+        if (ui.skip) continue;
+        // gate/up: rows of the grouped x (shared-expert rows follow the routed
+        // ones); down: routed h or shared h
+        const void* tm = &a.tm_h[(!kGateUp && ui.shared) ? 1 : 0];
+        const int y = (!kGateUp && ui.shared) ? ui.row0 - Tk : ui.row0;
+        for (int ks = 0; ks < ui.nks; ++ks, ++it) {
+          const int s = static_cast<int>(it % kBStages);
+          if (!tc::mbar_wait(&empty_b[s], ((it / kBStages) & 1u) ^ 1u, abort_flag, a.status)) {
+            ok = false;
+            break;
           }
-        }
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-        it = __shfl_sync(0xffffffffu, it, 0);
-        continue;
-      }
-      // lane of loader warp lw gathers tile row rr = 32 lw + lane
-      const int rr = (warp - kLoadWarp) * 32 + lane;
-      const uint16_t* brow = nullptr;
-      if (rr < ui.rows) {
-        const int R = ui.row0 + rr;
-        const int tok = ui.shared ? (R - Tk) : (a.perm[R] / a.g.k);
-        brow = a.x + static_cast<size_t>(tok) * a.g.H;
-      }
-      const uint32_t rsw = static_cast<uint32_t>(rr & 7);
-      for (int ks = 0; ks < ui.nks; ++ks, ++it) {
-        const int s = static_cast<int>(it % kBStages);
-        if (!tc::mbar_wait(&empty_b[s], ((it / kBStages) & 1u) ^ 1u, abort_flag, a.status)) {
-          ok = false;
-          break;
-        }
-        if (brow) {
-          const uint32_t dst = sbase + C::OFF_B + s * C::B_BYTES + rr * 128;
-          const uint16_t* src = brow + ks * BK;
-#pragma unroll
-          for (int c = 0; c < 8; ++c) tc::cp_async16(dst + ((c ^ rsw) << 4), src + c * 8);
-        }
-        tc::cp_async_commit();
-        if (it >= static_cast<uint32_t>(kBLag)) {
-          tc::cp_async_wait<kBLag>();
-          tc::fence_proxy_async_smem();
-          tc::mbar_arrive(&full_b[(it - kBLag) % kBStages]);
+          tc::mbar_arrive_expect_tx(&full_b[s], C::B_BYTES);
+          tc::tma_load_2d(sbase + C::OFF_B + s * C::B_BYTES, tm, ks * BK, y, &full_b[s]);
         }
       }
     }
-    if (!b_by_tma) {
-      tc::cp_async_wait_all();
-      tc::fence_proxy_async_smem();
-      if (ok) {
-        const uint32_t first = it > static_cast<uint32_t>(kBLag) ? it - kBLag : 0u;
-        for (uint32_t j = first; j < it; ++j) tc::mbar_arrive(&full_b[j % kBStages]);
-      }
-    }
+    __syncwarp();
   } else if (warp == kTmaWarp) {
     // ----------------------------------------- packed tiles and scales (TMA)
     if (lane == 0) {
       StageCursor<kGateUp> cur;
-      cur.begin(a, n_units, nfb);
+      cur.begin(a, n_units, nfb, units);
       uint32_t last_blk = 0xffffffffu;
       while (!cur.done) {
         const int side = cur.ui.shared ? 1 : 0;
@@ -476,7 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
     uint32_t it = 0, tt = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const UnitInfo ui = unit_info<kGateUp>(a, u, nfb);
+      const UnitInfo ui = unit_info<kGateUp>(a, u, nfb, units);
       if (ui.skip) continue;
       const int n_mma = max(16, (ui.rows + 15) & ~15);
       const uint32_t idesc = tc::idesc_bf16(BM, n_mma);
@@ -570,26 +539,27 @@ bool make_qmat_maps(TcArgs& a, int side, int m, const QMatPtr& W, int rows, int 
 
 int gemm_chunk_rows() { return BN; }
 
-cudaError_t launch_gateup(const Geometry& g, const LayerPtr& L, const uint16_t* x, const int32_t* perm,
-                          const Chunk* chunks, const int32_t* n_chunks, int max_chunks,
-                          uint16_t* h, uint16_t* h_s, int* status, cudaStream_t s) {
+cudaError_t launch_gateup(const Geometry& g, const LayerPtr& L, const uint16_t* xg, const Chunk* chunks,
+                          const int32_t* n_chunks, int max_chunks, uint16_t* h, uint16_t* h_s, int* status,
+                          cudaStream_t s) {
   TcArgs a{};
   a.g = g;
   a.W0 = L.gate;
   a.W1 = L.up;
   a.S0 = L.sh_gate;
   a.S1 = L.sh_up;
-  a.x = x;
-  a.perm = perm;
   a.h_out = h;
   a.hs_out = h_s;
   a.chunks = chunks;
   a.n_chunks = n_chunks;
   a.status = status;
   a.scales_tma = (g.H % (kGroup * kSBlock)) == 0;
+  const uint64_t rows = static_cast<uint64_t>(g.T) * g.k + g.T;
   if (!make_qmat_maps(a, 0, 0, L.gate, g.E * g.I, g.H) || !make_qmat_maps(a, 0, 1, L.up, g.E * g.I, g.H) ||
-      !make_qmat_maps(a, 1, 0, L.sh_gate, g.Is, g.H) || !make_qmat_maps(a, 1, 1, L.sh_up, g.Is, g.H))
+      !make_qmat_maps(a, 1, 0, L.sh_gate, g.Is, g.H) || !make_qmat_maps(a, 1, 1, L.sh_up, g.Is, g.H) ||
+      !make_map(&a.tm_h[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, xg, g.H, rows, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
+  a.tm_h[1] = a.tm_h[0];
   using C = Cfg<true>;
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(grouped_gemm_tc_kernel<true>), C::SMEM);
   if (e != cudaSuccess) return e;

@@ -73,17 +73,21 @@ cudaError_t launch_group(const int32_t* topk_idx, int T, int k, int E, int chunk
 
 // gemm_tc.cu: tcgen05 grouped expert GEMMs over the device chunk list.
 int gemm_chunk_rows();
-cudaError_t launch_gateup(const Geometry& g, const LayerPtr& L, const uint16_t* x, const int32_t* perm,
-                          const Chunk* chunks, const int32_t* n_chunks, int max_chunks,
-                          uint16_t* h, uint16_t* h_s, int* status, cudaStream_t s);
+// xg: the grouped token rows [T*k + T, H] (routed rows in expert order, then
+// the shared expert's T rows), each group of 8 in the interleaved K order.
+cudaError_t launch_gateup(const Geometry& g, const LayerPtr& L, const uint16_t* xg, const Chunk* chunks,
+                          const int32_t* n_chunks, int max_chunks, uint16_t* h, uint16_t* h_s, int* status,
+                          cudaStream_t s);
 cudaError_t launch_down(const Geometry& g, const LayerPtr& L, const uint16_t* h, const uint16_t* h_s,
                         const Chunk* chunks, const int32_t* n_chunks, int max_chunks,
                         uint16_t* Y, int* status, cudaStream_t s);
 
 // combine.cu
-// xp = x with each group of 8 elements reordered (0,4,1,5,2,6,3,7): the K
-// order of the grouped GEMMs' operands (x and xp: [T, H] bf16, 16-B aligned).
-cudaError_t launch_interleave_k8(const uint16_t* x, uint16_t* xp, int T, int H, cudaStream_t s);
+// xg[R] = row perm[R] / k of x for R < T*k, row R - T*k for the shared
+// expert's rows, each group of 8 elements reordered (0,4,1,5,2,6,3,7): the
+// B operand of the gate/up GEMM in its grouped order and K order.
+cudaError_t launch_gather_k8(const uint16_t* x, const int32_t* perm, int T, int k, int H, uint16_t* xg,
+                             cudaStream_t s);
 cudaError_t launch_combine(const uint16_t* Y, const int32_t* inv_perm, const float* topk_w, const float* sigma,
                            int T, int k, int H, uint16_t* out, cudaStream_t s);
 cudaError_t launch_rmsnorm(const uint16_t* y, uint16_t* out, int T, int H, float eps, cudaStream_t s);
