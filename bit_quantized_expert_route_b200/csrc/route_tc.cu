@@ -4,11 +4,13 @@
 // One CTA scores 128 tokens: D[128 tokens x E experts] = x W_r^T accumulates
 // in tensor memory (tcgen05.mma, bf16 operands in shared memory, FP32
 // accumulators), and a second 16-column MMA against [w_sg; 0 ... 0] yields
-// x . w_sg in column 256.  Each epilogue thread owns one token (its TMEM
-// lane), reads its E logits and keeps the k best in registers by insertion
-// in expert order, which realises the order (logit desc, expert index asc).
-// The CTA also counts its 128*k (token, slot) entries per expert: that is
-// the first pass of the counting sort (one segment per CTA).
+// x . w_sg in column 256.  The epilogue gives each token four threads (one
+// per quarter of the experts, all reading the token's TMEM lane): each keeps
+// the k best of its quarter in registers by insertion in expert order, then
+// the first thread merges the four sorted lists, which realises the order
+// (logit desc, expert index asc).  The CTA also counts its 128*k (token,
+// slot) entries per expert: the first pass of the counting sort (one segment
+// per CTA).
 // ("Perplexity's Lily: ...", section "The Model": the router scores 256
 // experts and keeps 8, plus one shared expert for every token.)
 #include "common.cuh"
@@ -21,25 +23,31 @@ namespace {
 constexpr int kRM = 128;                  // tokens per CTA (TMEM lanes)
 constexpr int kRBK = 64;                  // inputs per stage
 constexpr int kRStages = 4;
-constexpr int kRThreads = 160;            // warps 0-3: loaders then epilogue; warp 4: TMEM + MMA
-constexpr int kRMmaWarp = 4;
+constexpr int kREpiWarps = 16;            // 4 per TMEM lane quadrant: one expert quarter each
+constexpr int kRLoadWarp = kREpiWarps;    // one lane issues the TMA loads
+constexpr int kRMmaWarp = kREpiWarps + 1; // TMEM + MMA
+constexpr int kRThreads = (kRMmaWarp + 1) * 32;
 constexpr int kA_BYTES = kRM * kRBK * 2;                  // 16 KB
 constexpr int kB_BYTES = kMaxE * kRBK * 2;                // 32 KB (up to 256 experts)
 constexpr int kG_BYTES = 16 * kRBK * 2;                   // 2 KB: w_sg row + 15 zero rows
 constexpr int kSTAGE = kA_BYTES + kB_BYTES + kG_BYTES;    // 50 KB (multiple of 1024)
 constexpr int kBAR_OFF = kRStages * kSTAGE;
-constexpr int kRSMEM = kBAR_OFF + 128 + kMaxE * 4 + 1024;   // barriers, histogram, alignment slack
+constexpr int kPART_OFF = kBAR_OFF + 128 + kMaxE * 4;       // per-token partial lists [3][128][2 x kMaxK]
+constexpr int kRSMEM = kPART_OFF + 3 * kRM * 2 * kMaxK * 4 + 1024;   // + alignment slack
 constexpr uint32_t kRTmemCols = 512;
 constexpr int kGateCol = 256;             // accumulator column of x . w_sg
 
-// One token's epilogue (this thread's TMEM lane): the E logits (+ bias) scanned
-// in expert order, the K largest kept by insertion (a later expert replaces a
-// kept one only if strictly larger, so equal logits keep the lower index
-// first), then renormalised softmax weights, the shared gate, and the token's
-// contribution to the CTA's expert histogram.
+// One token's epilogue (this thread's TMEM lane), part `part` of 4: logits of
+// experts [c_lo, c_hi) (+ bias) scanned in expert order, the K largest kept by
+// insertion (a later expert replaces a kept one only if strictly larger, so
+// equal logits keep the lower index first).  Parts 1-3 publish their sorted
+// lists; part 0 merges them (ties go to the lower part, whose experts are
+// lower), then writes the renormalised softmax weights, the shared gate and
+// the token's contribution to the CTA's expert histogram.
 template <int K>
-__device__ __forceinline__ void router_epilogue(uint32_t lane_base, int n_mma, int E, const float* __restrict__ bias,
-                                                int t, int T, int32_t* __restrict__ topk_idx,
+__device__ __forceinline__ void router_epilogue(uint32_t lane_base, int part, int c_lo, int c_hi, int E,
+                                                const float* __restrict__ bias, int tl, int t, int T,
+                                                float* pv, int* pi, int32_t* __restrict__ topk_idx,
                                                 float* __restrict__ topk_w, float* __restrict__ sigma, int* hist) {
   float bv[K];
   int bi[K];
@@ -48,28 +56,54 @@ __device__ __forceinline__ void router_epilogue(uint32_t lane_base, int n_mma, i
     bv[j] = -INFINITY;
     bi[j] = 0x7fffffff;
   }
-  for (int c0 = 0; c0 < n_mma; c0 += 16) {
+  for (int c0 = c_lo; c0 < c_hi; c0 += 16) {
     float v[16];
     tc::tmem_ld16(lane_base + c0, v);
     tc::tmem_wait_ld();
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const int e = c0 + i;
-      if (e < E) {
-        float cv = v[i] + (bias ? __ldg(bias + e) : 0.f);
-        if (cv > bv[K - 1]) {
-          int ci = e;
+      // branch-free insertion (no divergence between the warp's tokens)
+      float cv = e < E ? v[i] + (bias ? __ldg(bias + e) : 0.f) : -INFINITY;
+      int ci = e;
 #pragma unroll
-          for (int j = 0; j < K; ++j) {
-            const bool take = cv > bv[j];
-            const float tv = bv[j];
-            const int ti = bi[j];
-            bv[j] = take ? cv : tv;
-            bi[j] = take ? ci : ti;
-            cv = take ? tv : cv;
-            ci = take ? ti : ci;
-          }
-        }
+      for (int j = 0; j < K; ++j) {
+        const bool take = cv > bv[j];
+        const float tv = bv[j];
+        const int ti = bi[j];
+        bv[j] = take ? cv : tv;
+        bi[j] = take ? ci : ti;
+        cv = take ? tv : cv;
+        ci = take ? ti : ci;
+      }
+    }
+  }
+  if (part > 0) {
+#pragma unroll
+    for (int j = 0; j < K; ++j) {
+      pv[((part - 1) * kRM + tl) * kMaxK + j] = bv[j];
+      pi[((part - 1) * kRM + tl) * kMaxK + j] = bi[j];
+    }
+  }
+  asm volatile("bar.sync 2, %0;" ::"n"(kREpiWarps * 32) : "memory");
+  if (part > 0) return;
+  // merge parts 1..3 into this thread's list; entries are inserted only if
+  // strictly larger, so on ties the earlier (lower-expert) entry stays first
+#pragma unroll 1
+  for (int q = 0; q < 3; ++q) {
+#pragma unroll
+    for (int jj = 0; jj < K; ++jj) {
+      float cv = pv[(q * kRM + tl) * kMaxK + jj];
+      int ci = pi[(q * kRM + tl) * kMaxK + jj];
+#pragma unroll
+      for (int j = 0; j < K; ++j) {
+        const bool take = cv > bv[j];
+        const float tv = bv[j];
+        const int ti = bi[j];
+        bv[j] = take ? cv : tv;
+        bi[j] = take ? ci : ti;
+        cv = take ? tv : cv;
+        ci = take ? ti : ci;
       }
     }
   }
@@ -132,9 +166,10 @@ __global__ void __launch_bounds__(kRThreads, 1) router_tc_kernel(
     tc::fence_barrier_init();
   }
   // zero rows 1..15 of every stage's gate tile once (row 0 is reloaded per stage)
-  if (warp < 4) {
-    for (int i = threadIdx.x; i < kMaxE; i += 128) hist[i] = 0;
-    for (int i = threadIdx.x; i < kRStages * 15 * 8; i += 128) {
+  constexpr int kEpiThreads = kREpiWarps * 32;
+  if (warp < kREpiWarps) {
+    for (int i = threadIdx.x; i < kMaxE; i += kEpiThreads) hist[i] = 0;
+    for (int i = threadIdx.x; i < kRStages * 15 * 8; i += kEpiThreads) {
       const int s = i / 120, rr = 1 + (i % 120) / 8, c = i % 8;
       *reinterpret_cast<uint4*>(smem + s * kSTAGE + kA_BYTES + kB_BYTES + rr * 128 + c * 16) =
           make_uint4(0u, 0u, 0u, 0u);
@@ -147,19 +182,14 @@ __global__ void __launch_bounds__(kRThreads, 1) router_tc_kernel(
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp < 4) {
+  if (warp == kRLoadWarp) {
     // ---------------------------------------------------------- loader
     // one thread streams the stages: x tile, router rows and the gate row
-    const int r = threadIdx.x;
-    bool ok = true;
-    if (threadIdx.x == 0) {
+    if (lane == 0) {
       const uint32_t tx = static_cast<uint32_t>(kA_BYTES + n_mma * kRBK * 2 + kRBK * 2);
       for (int ks = 0; ks < nks; ++ks) {
         const int s = ks % kRStages;
-        if (!tc::mbar_wait(&empty[s], ((ks / kRStages) & 1) ^ 1, abort_flag, status)) {
-          ok = false;
-          break;
-        }
+        if (!tc::mbar_wait(&empty[s], ((ks / kRStages) & 1) ^ 1, abort_flag, status)) break;
         const uint32_t st = sbase + s * kSTAGE;
         tc::mbar_arrive_expect_tx(&full[s], tx);
         tc::tma_load_2d(st, &maps.x, ks * kRBK, t0, &full[s]);
@@ -167,25 +197,44 @@ __global__ void __launch_bounds__(kRThreads, 1) router_tc_kernel(
         tc::tma_load_2d(st + kA_BYTES + kB_BYTES, &maps.g, ks * kRBK, 0, &full[s]);
       }
     }
-
+    __syncwarp();
+  } else if (warp < kREpiWarps) {
     // --------------------------------------------------------- epilogue
-    if (ok && tc::mbar_wait(acc_full, 0, abort_flag, status)) {
+    // warp w reads TMEM lane quadrant w % 4 (its 32 tokens) and the expert
+    // quarter w / 4 of their logits
+    const int q = warp & 3, part = warp >> 2, tl = q * 32 + lane;
+    const int quarter = ((n_mma / 4) + 15) & ~15;
+    const int c_lo = min(part * quarter, n_mma), c_hi = min(c_lo + quarter, n_mma);
+    const uint32_t got = tc::mbar_wait(acc_full, 0, abort_flag, status) ? 1u : 0u;
+    uint32_t all_got;   // the epilogue threads agree before any of them enters its barriers
+    asm volatile("{\n\t.reg .pred p, r;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred r, 3, %2, p;\n\t"
+                 "selp.u32 %0, 1, 0, r;\n\t}"
+                 : "=r"(all_got)
+                 : "r"(got), "n"(kEpiThreads)
+                 : "memory");
+    if (all_got) {
       tc::tc_fence_after();
-      const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-      switch (k) {   // k fixed at compile time: the candidate list stays in registers
-        case 1: router_epilogue<1>(lane_base, n_mma, E, router_bias, t0 + r, T, topk_idx, topk_w, sigma, hist); break;
-        case 2: router_epilogue<2>(lane_base, n_mma, E, router_bias, t0 + r, T, topk_idx, topk_w, sigma, hist); break;
-        case 3: router_epilogue<3>(lane_base, n_mma, E, router_bias, t0 + r, T, topk_idx, topk_w, sigma, hist); break;
-        case 4: router_epilogue<4>(lane_base, n_mma, E, router_bias, t0 + r, T, topk_idx, topk_w, sigma, hist); break;
-        case 5: router_epilogue<5>(lane_base, n_mma, E, router_bias, t0 + r, T, topk_idx, topk_w, sigma, hist); break;
-        case 6: router_epilogue<6>(lane_base, n_mma, E, router_bias, t0 + r, T, topk_idx, topk_w, sigma, hist); break;
-        case 7: router_epilogue<7>(lane_base, n_mma, E, router_bias, t0 + r, T, topk_idx, topk_w, sigma, hist); break;
-        default: router_epilogue<8>(lane_base, n_mma, E, router_bias, t0 + r, T, topk_idx, topk_w, sigma, hist); break;
+      const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      float* pv = reinterpret_cast<float*>(smem + kPART_OFF);
+      int* pi = reinterpret_cast<int*>(pv + 3 * kRM * kMaxK);
+      const int t = t0 + tl;
+#define ROUTER_EPI(K) router_epilogue<K>(lane_base, part, c_lo, c_hi, E, router_bias, tl, t, T, pv, pi, topk_idx, \
+                                         topk_w, sigma, hist)
+      switch (k) {   // k fixed at compile time: the candidate lists stay in registers
+        case 1: ROUTER_EPI(1); break;
+        case 2: ROUTER_EPI(2); break;
+        case 3: ROUTER_EPI(3); break;
+        case 4: ROUTER_EPI(4); break;
+        case 5: ROUTER_EPI(5); break;
+        case 6: ROUTER_EPI(6); break;
+        case 7: ROUTER_EPI(7); break;
+        default: ROUTER_EPI(8); break;
       }
+#undef ROUTER_EPI
     }
     // this CTA's segment of the (token, slot) entries: expert counts for the sort
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    for (int e = threadIdx.x; e < E; e += 128) seg_counts[static_cast<size_t>(blockIdx.x) * E + e] = hist[e];
+    asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
+    for (int e = threadIdx.x; e < E; e += kEpiThreads) seg_counts[static_cast<size_t>(blockIdx.x) * E + e] = hist[e];
   } else if (warp == kRMmaWarp) {
     // -------------------------------------------------------------- MMA
     if (lane == 0) {
