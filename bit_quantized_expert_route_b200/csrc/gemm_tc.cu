@@ -52,7 +52,6 @@ constexpr int BM = 128;          // weight rows per tile = TMEM lanes (MMA M)
 constexpr int BN = 128;          // rows (tokens) per chunk: MMA N <= 128
 constexpr int BK = 64;           // inputs per stage: one quantisation group
 constexpr int kBStages = 6;      // token-tile ring
-constexpr int kBLag = 3;         // gather cp.async groups in flight before signalling
 constexpr int kPStages = 8;      // packed-tile ring
 constexpr int kSBlock = 8;       // quantisation groups per scale block (16 B per row)
 constexpr int kDqWarps = 16;     // dequantiser warps (4 sets of 4: one per TMEM lane quadrant)
