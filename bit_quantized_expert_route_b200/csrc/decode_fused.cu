@@ -34,8 +34,15 @@
 // waits are bounded; a timeout records MOE_ERR_DEVICE_TIMEOUT in the status
 // word and the kernel returns.
 //
-// Dequantisation and dot products follow the decode kernels (decode.cu):
-//   sum_i (s q_i + b) x_i = 128 s * sum_i (1 + q_i/128) x_i + (b - 128 s) * sum_i x_i.
+// Dot products on the tensor cores (warp-level mma.sync, bf16 in, FP32
+// accumulation): per group of 64 inputs, with A = 128 + q as exact bf16 values
+// (one AND-OR per code pair, no scale applied) and B = the activations,
+//   sum_i (s q_i + b) x_i = s * (sum_i (128 + q_i) x_i - 128 X) + b X,  X = sum_i x_i,
+// applied per group after the MMAs.  Inside each group of 8 inputs both
+// operands use the order (0,4,1,5,2,6,3,7) in which the AND-OR yields code
+// pairs; the activations are staged in that order, so no permutes are
+// needed.  The integer work per code drops from ~2 (nibble to float) to ~1
+// instruction per code pair.
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
@@ -84,33 +91,46 @@ struct RouteSmem {
   int32_t abort;
 };
 
-__host__ __device__ __forceinline__ int fx_stride(int H) { return (H + 1023) / 1024 * 1024; }   // 32-lane windows
-__host__ __device__ __forceinline__ int fh_stride(int I) { return (I + 511) / 512 * 512; }      // 16-lane windows
 
-__device__ __forceinline__ void codes_f(uint32_t w, float (&f)[8]) {
-  const uint32_t M = 0x000F0000u, ONE = 0x3F800000u;
-  f[0] = __uint_as_float(((w << 16) & M) | ONE);
-  f[1] = __uint_as_float(((w << 12) & M) | ONE);
-  f[2] = __uint_as_float(((w << 8) & M) | ONE);
-  f[3] = __uint_as_float(((w << 4) & M) | ONE);
-  f[4] = __uint_as_float((w & M) | ONE);
-  f[5] = __uint_as_float(((w >> 4) & M) | ONE);
-  f[6] = __uint_as_float(((w >> 8) & M) | ONE);
-  f[7] = __uint_as_float(((w >> 12) & M) | ONE);
+// 8 bf16 values (x0,x1)(x2,x3)(x4,x5)(x6,x7) in the interleaved K order
+// (x0,x4)(x1,x5)(x2,x6)(x3,x7).
+__device__ __forceinline__ uint4 interleave8(const uint4& v) {   // (x0,x1)(x2,x3)(x4,x5)(x6,x7)
+  uint4 o;
+  o.x = __byte_perm(v.x, v.z, 0x5410);
+  o.y = __byte_perm(v.x, v.z, 0x7632);
+  o.z = __byte_perm(v.y, v.w, 0x5410);
+  o.w = __byte_perm(v.y, v.w, 0x7632);
+  return o;
 }
 
-// Stage one bf16 row of n elements as FP32 in the `lanes`-interleaved layout
-// (element 32c + i at float4 ((c/lanes)*8 + i/4)*lanes + c%lanes).  Called by
-// `nthr` threads with index `tid`.
-__device__ __forceinline__ void stage_row_f(const uint16_t* src, int n, int lanes, float* dst, int tid, int nthr) {
-  float4* d4 = reinterpret_cast<float4*>(dst);
-  for (int u = tid; u < n / 8; u += nthr) {
-    const uint4 v = reinterpret_cast<const uint4*>(src)[u];
-    const int e0 = u * 8, c = e0 >> 5, ii = e0 & 31;
-    const int win = c / lanes, ln = c - win * lanes;
-    d4[(win * 8 + (ii >> 2)) * lanes + ln] = make_float4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y));
-    d4[(win * 8 + (ii >> 2) + 1) * lanes + ln] = make_float4(bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w));
-  }
+// D (16 rows x 8 tokens, FP32) += A (16 x 16, bf16) B (16 x 8, bf16).
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t code_pair(uint32_t w, int shift) {   // bf16 pair (128 + q_i, 128 + q_{i+4})
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(w >> shift), "r"(0x000F000Fu), "r"(0x43004300u));
+  return d;
+}
+
+// One group of 64 inputs for rows g, g+8 of a 16-row weight tile (lane g =
+// lane/4, t = lane%4): lane reads words 2t, 2t+1 of the group in both rows
+// (qg, qg8: this lane's 8 bytes) and the 32 staged activations of token g at
+// 8-groups 2t, 2t+1 (xb0, xb1; zero for padding tokens).  d gets
+// sum (128 + q) x for (row g, tokens 2t, 2t+1) and (row g+8, same tokens).
+__device__ __forceinline__ void group_dot(float (&d)[4], const uint2& qg, const uint2& qg8, const uint4& xb0,
+                                          const uint4& xb1) {
+  d[0] = d[1] = d[2] = d[3] = 0.f;
+  mma16816(d, code_pair(qg.x, 0), code_pair(qg8.x, 0), code_pair(qg.x, 4), code_pair(qg8.x, 4), xb0.x, xb0.y);
+  mma16816(d, code_pair(qg.x, 8), code_pair(qg8.x, 8), code_pair(qg.x, 12), code_pair(qg8.x, 12), xb0.z, xb0.w);
+  mma16816(d, code_pair(qg.y, 0), code_pair(qg8.y, 0), code_pair(qg.y, 4), code_pair(qg8.y, 4), xb1.x, xb1.y);
+  mma16816(d, code_pair(qg.y, 8), code_pair(qg8.y, 8), code_pair(qg.y, 12), code_pair(qg8.y, 12), xb1.z, xb1.w);
 }
 
 // Order-preserving 32-bit key of a float (larger float -> larger key; every
@@ -282,66 +302,6 @@ __device__ void issue_unit(const FusedArgs& a, const RouteSmem& rt, const Sched&
   }
 }
 
-// Sum over the warp of v[r(lane)] with r(lane) = 4*bit4 + 2*bit3 + bit2 of
-// the lane: a transposing butterfly (9 shuffles for 8 values).
-__device__ __forceinline__ float warp_reduce8(const float (&v)[8], int lane) {
-  const bool h16 = lane & 16, h8 = lane & 8, h4 = lane & 4;
-  float a4[4], a2[2];
-#pragma unroll
-  for (int j = 0; j < 4; ++j)
-    a4[j] = (h16 ? v[j + 4] : v[j]) + __shfl_xor_sync(0xffffffffu, h16 ? v[j] : v[j + 4], 16);
-#pragma unroll
-  for (int j = 0; j < 2; ++j)
-    a2[j] = (h8 ? a4[j + 2] : a4[j]) + __shfl_xor_sync(0xffffffffu, h8 ? a4[j] : a4[j + 2], 8);
-  float r = (h4 ? a2[1] : a2[0]) + __shfl_xor_sync(0xffffffffu, h4 ? a2[0] : a2[1], 4);
-  r += __shfl_xor_sync(0xffffffffu, r, 2);
-  r += __shfl_xor_sync(0xffffffffu, r, 1);
-  return r;
-}
-
-// Sum over each half-warp of v[r(lane)] with r(lane) = 2*bit3 + bit2.
-__device__ __forceinline__ float halfwarp_reduce4(const float (&v)[4], int lane) {
-  const bool h8 = lane & 8, h4 = lane & 4;
-  float a2[2];
-#pragma unroll
-  for (int j = 0; j < 2; ++j)
-    a2[j] = (h8 ? v[j + 2] : v[j]) + __shfl_xor_sync(0xffffffffu, h8 ? v[j] : v[j + 2], 8);
-  float r = (h4 ? a2[1] : a2[0]) + __shfl_xor_sync(0xffffffffu, h4 ? a2[0] : a2[1], 4);
-  r += __shfl_xor_sync(0xffffffffu, r, 2);
-  r += __shfl_xor_sync(0xffffffffu, r, 1);
-  return r;
-}
-
-// sum_i (1 + q_i/128) * v_i for the 32 codes of qv against 32 staged values
-// held in registers (v[0..31]), four partial sums.
-__device__ __forceinline__ float dot32r(const uint4& qv, const float (&v)[32]) {
-  const uint32_t words[4] = {qv.x, qv.y, qv.z, qv.w};
-  float p[4];
-#pragma unroll
-  for (int wd = 0; wd < 4; ++wd) {
-    float f[8];
-    codes_f(words[wd], f);
-    float acc = f[0] * v[8 * wd];
-#pragma unroll
-    for (int i = 1; i < 8; ++i) acc = fmaf(f[i], v[8 * wd + i], acc);
-    p[wd] = acc;
-  }
-  return (p[0] + p[1]) + (p[2] + p[3]);
-}
-
-// Load one 32-element segment of a staged row (interleave `lanes`) into registers.
-__device__ __forceinline__ void load_seg(const float* row, int c, int lanes, float (&v)[32]) {
-  const float4* r4 = reinterpret_cast<const float4*>(row) + ((c / lanes) * 8) * lanes + (c % lanes);
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const float4 q = r4[j * lanes];
-    v[4 * j] = q.x;
-    v[4 * j + 1] = q.y;
-    v[4 * j + 2] = q.z;
-    v[4 * j + 3] = q.w;
-  }
-}
-
 template <int NT>
 __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid_constant__ FusedArgs a) {
   extern __shared__ __align__(128) uint8_t fsm[];
@@ -351,17 +311,15 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
   const uint32_t ring0 = tc::smem_u32(fsm);
   uint64_t* full = reinterpret_cast<uint64_t*>(fsm + a.off_bar);
   uint64_t* empty = full + kFRingMax;
-  float* xs = reinterpret_cast<float*>(fsm + a.off_xs);       // [T][fx_stride(H)]
-  float* xsum = reinterpret_cast<float*>(fsm + a.off_xsum);   // [T][fx_stride(H)/32]
-  float* hs = reinterpret_cast<float*>(fsm + a.off_hs);       // [rows][fh_stride(Kmax)]
-  float* hsum = reinterpret_cast<float*>(fsm + a.off_hsum);   // [rows][fh_stride(Kmax)/32]
+  uint16_t* xs = reinterpret_cast<uint16_t*>(fsm + a.off_xs);   // [T][H] bf16, interleaved K order
+  float* xsum = reinterpret_cast<float*>(fsm + a.off_xsum);      // [T][H/64] group sums
+  uint16_t* hs = reinterpret_cast<uint16_t*>(fsm + a.off_hs);   // [T*k + T][Kmax] bf16, interleaved K order
+  float* hsum = reinterpret_cast<float*>(fsm + a.off_hsum);      // [T*k + T][Kmax/64] group sums
   float* lg = reinterpret_cast<float*>(fsm + a.off_lg);       // [T][E1], also the router partials
   RouteSmem& rt = *reinterpret_cast<RouteSmem*>(fsm + a.off_rt);
   float* ys = reinterpret_cast<float*>(fsm + a.off_y);        // [T*k + T][my_blocks][16]
   volatile int* abort_flag = &rt.abort;
-  const int xst = fx_stride(g.H);
   const int Kmax = max(g.I, g.Is);
-  const int hst = fh_stride(Kmax);
   const bool producer = warp == kFWarps;
 
   if (threadIdx.x == 0) {
@@ -388,7 +346,8 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
   }
   if (!producer) {
     const int tid = threadIdx.x, nthr = kFWarps * 32;
-    for (int t = 0; t < T; ++t) stage_row_f(a.x + static_cast<size_t>(t) * g.H, g.H, 32, xs + t * xst, tid, nthr);
+    for (int i = tid; i < T * (g.H / 8); i += nthr)
+      reinterpret_cast<uint4*>(xs)[i] = interleave8(__ldg(reinterpret_cast<const uint4*>(a.x) + i));
     // router rows r = c, c + G, ...: warp w sums the K slice [w H/16, (w+1) H/16)
     const int nrows = (E1 - static_cast<int>(blockIdx.x) + gridDim.x - 1) / gridDim.x;
     const int kslice = g.H / kFWarps;
@@ -421,19 +380,16 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
       }
     }
     consumers_sync();
-    for (int i = tid; i < T * xst / 32; i += nthr) {
-      const int t = i / (xst / 32), c = i % (xst / 32);
-      if (c < g.H / 32) {
-        const float4* r4 = reinterpret_cast<const float4*>(xs + t * xst);
-        const int win = c >> 5, ln = c & 31;
-        float sum = 0.f;
+    for (int i = tid; i < T * (g.H / 64); i += nthr) {     // sums over groups of 64 (fixed order)
+      const uint4* r4 = reinterpret_cast<const uint4*>(xs) + i * 8;
+      float sum = 0.f;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float4 q = r4[(win * 8 + j) * 32 + ln];
-          sum += (q.x + q.y) + (q.z + q.w);
-        }
-        xsum[t * (xst / 32) + c] = sum;
+      for (int j = 0; j < 8; ++j) {
+        const uint4 v = r4[j];
+        sum += ((bf16_lo(v.x) + bf16_hi(v.x)) + (bf16_lo(v.y) + bf16_hi(v.y))) +
+               ((bf16_lo(v.z) + bf16_hi(v.z)) + (bf16_lo(v.w) + bf16_hi(v.w)));
       }
+      xsum[i] = sum;
     }
     if (tid < nrows * T) {
       const int rr = tid / T, t = tid % T;
@@ -521,101 +477,106 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
   }
 
   // ------------------------------------------------------ consumer warps
-  // gate/up, two units at a time: warp pair p = warp / 2 owns 8 of the 64
-  // rows (2 units x 16 features x {gate, up}); thread (p, c) keeps segment c
-  // of every token's staged x in registers and runs 8 independent dot
-  // products against it.
+  // gate/up, two units at a time: warp w owns the 16-row tile w % 4 (unit
+  // (w%4)/2, matrix (w%4)%2) for the K quarter w / 4; per group of 64 inputs
+  // four mma.sync on the tile, then the group's scale and bias.
   bool ok = true;
-  float* red = lg;   // [8 pairs][2 halves][8 rows][NT] partial sums (logits are no longer needed)
-  const int pr = warp >> 1, half = warp & 1;
-  const int nch = g.H / 32;
+  float* red = lg;   // [4 tiles][4 K quarters][16 rows][NT] partial sums (logits are no longer needed)
+  const int lg4 = lane >> 2, lt = lane & 3;
   const uint32_t qb = kFFeat * g.H / 2, sb = kFFeat * g.H / 32;
-  for (int i0 = 0; i0 < s.my_gu && ok; i0 += 2) {
-    const int nu = min(2, s.my_gu - i0);
-    for (int ui = 0; ui < nu && ok; ++ui) {
-      const int i = i0 + ui;
-      if (!tc::mbar_wait(&full[i % a.ring], (i / a.ring) & 1u, abort_flag, a.status)) ok = false;
-    }
-    if (!ok) break;
-    // this pair's rows: r = 8 pr + rr; unit r / 32, matrix (r / 16) & 1, feature r & 15
-    const int ur = (8 * pr) >> 5;
-    const bool rows_live = ur < nu;
-    int slot = 0, f0 = 0;
-    if (rows_live) gu_unit(s, blockIdx.x + (i0 + ur) * gridDim.x, slot, f0);
-    const int m = ((8 * pr) >> 4) & 1, fb = (8 * pr) & 15;     // rows rr = 0..7: features fb .. fb+7
-    const uint8_t* base = fsm + ((i0 + ur) % a.ring) * a.slot_bytes;
-    const uint8_t* qrow0 = base + m * qb + fb * (g.H / 2);
-    const uint16_t* srow0 = reinterpret_cast<const uint16_t*>(base + 2 * qb + m * 2 * sb) + fb * (g.H / kGroup);
-    const uint16_t* brow0 = reinterpret_cast<const uint16_t*>(base + 2 * qb + m * 2 * sb + sb) + fb * (g.H / kGroup);
-    // tokens of this unit's expert: routed slot -> its rows' tokens; shared -> 0..T-1
-    unsigned tmask = 0;
-    if (rows_live) {
-      if (slot == 0)
-        tmask = (1u << T) - 1u;
-      else
-        for (int r = 0; r < rt.slot_cnt[slot]; ++r) tmask |= 1u << (rt.perm[rt.slot_off[slot] + r] / k);
-    }
-    float acc[8][NT];
+  const int ngrp = g.H / kGroup;
+  {
+    const int tile = warp & 3, kq = warp >> 2;
+    const int gq = ngrp / 4;                       // groups per K quarter
+    for (int i0 = 0; i0 < s.my_gu && ok; i0 += 2) {
+      const int nu = min(2, s.my_gu - i0);
+      for (int ui = 0; ui < nu && ok; ++ui) {
+        const int i = i0 + ui;
+        if (!tc::mbar_wait(&full[i % a.ring], (i / a.ring) & 1u, abort_flag, a.status)) ok = false;
+      }
+      if (!ok) break;
+      const int ur = tile >> 1, m = tile & 1;
+      const bool live = ur < nu;
+      float y[2][NT];
 #pragma unroll
-    for (int rr = 0; rr < 8; ++rr)
+      for (int r = 0; r < 2; ++r)
 #pragma unroll
-      for (int t = 0; t < NT; ++t) acc[rr][t] = 0.f;
-    if (rows_live) {
-      for (int c = half * 32 + lane; c < nch; c += 64) {
+        for (int t = 0; t < NT; ++t) y[r][t] = 0.f;
+      if (live) {
+        int slot, f0;
+        gu_unit(s, blockIdx.x + (i0 + ur) * gridDim.x, slot, f0);
+        unsigned tmask = 0;                          // tokens of this unit's expert
+        if (slot == 0)
+          tmask = (1u << T) - 1u;
+        else
+          for (int r = 0; r < rt.slot_cnt[slot]; ++r) tmask |= 1u << (rt.perm[rt.slot_off[slot] + r] / k);
+        const uint8_t* base = fsm + ((i0 + ur) % a.ring) * a.slot_bytes;
+        const uint8_t* qrow = base + m * qb + lg4 * (g.H / 2) + lt * 8;       // rows lg4, lg4 + 8
+        const uint16_t* srow = reinterpret_cast<const uint16_t*>(base + 2 * qb + m * 2 * sb);
+        const uint16_t* brow = srow + sb / 2;
+        const bool tok_live = lg4 < T && ((tmask >> lg4) & 1u);
+        const uint4* xrow = reinterpret_cast<const uint4*>(xs + (tok_live ? lg4 : 0) * g.H) + lt * 2;
+        for (int G = kq * gq; G < (kq + 1) * gq; ++G) {
+          const uint2 qa = *reinterpret_cast<const uint2*>(qrow + G * 32);
+          const uint2 qc = *reinterpret_cast<const uint2*>(qrow + 8 * (g.H / 2) + G * 32);
+          const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+          const uint4 xb0 = tok_live ? xrow[G * 8] : z, xb1 = tok_live ? xrow[G * 8 + 1] : z;
+          float d[4];
+          group_dot(d, qa, qc, xb0, xb1);
+          if (lt == 0) {   // columns 0, 1 = tokens 0, 1
 #pragma unroll
-        for (int t = 0; t < NT; ++t) {
-          if ((tmask >> t) & 1u) {
-            float xv[32];
-            load_seg(xs + t * xst, c, 32, xv);
-            const float X = xsum[t * (xst / 32) + c];
+            for (int r = 0; r < 2; ++r) {
+              const int row = lg4 + 8 * r;
+              const float sc = bf16_bits_to_float(srow[row * ngrp + G]);
+              const float bi = bf16_bits_to_float(brow[row * ngrp + G]);
 #pragma unroll
-            for (int rr = 0; rr < 8; ++rr) {
-              const uint4 qv = reinterpret_cast<const uint4*>(qrow0 + rr * (g.H / 2))[c];
-              const float s128 = 128.f * bf16_bits_to_float(srow0[rr * (g.H / kGroup) + (c >> 1)]);
-              const float bb = bf16_bits_to_float(brow0[rr * (g.H / kGroup) + (c >> 1)]);
-              acc[rr][t] = fmaf(s128, dot32r(qv, xv), fmaf(bb - s128, X, acc[rr][t]));
+              for (int t = 0; t < NT; ++t)
+                if (t < T) {
+                  const float X = xsum[t * ngrp + G];
+                  y[r][t] = fmaf(sc, d[2 * r + t] - 128.f * X, fmaf(bi, X, y[r][t]));
+                }
             }
           }
         }
       }
-    }
-    // every read of the pair's slots is done: release them
-    tc::fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0)
-      for (int ui = 0; ui < nu; ++ui) tc::mbar_arrive(&empty[(i0 + ui) % a.ring]);
+      // every read of the pair's slots is done: release them
+      tc::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0)
+        for (int ui = 0; ui < nu; ++ui) tc::mbar_arrive(&empty[(i0 + ui) % a.ring]);
+      if (lt == 0)
 #pragma unroll
-    for (int t = 0; t < NT; ++t) {
-      float v[8];
+        for (int r = 0; r < 2; ++r)
 #pragma unroll
-      for (int rr = 0; rr < 8; ++rr) v[rr] = acc[rr][t];
-      const float r = warp_reduce8(v, lane);
-      if ((lane & 3) == 0) red[((pr * 2 + half) * 8 + (lane >> 2)) * NT + t] = r;
-    }
-    consumers_sync();
-    // h = bf16(silu(g) * u) for (unit, feature, token)
-    for (int q = threadIdx.x; q < nu * kFFeat * T; q += kFWarps * 32) {
-      const int ui = q / (kFFeat * T), f = (q / T) % kFFeat, t = q % T;
-      int uslot, uf0;
-      gu_unit(s, blockIdx.x + (i0 + ui) * gridDim.x, uslot, uf0);
-      bool member = uslot == 0;
-      int pos = t;
-      for (int r = 0; r < (uslot == 0 ? 0 : rt.slot_cnt[uslot]); ++r)
-        if (rt.perm[rt.slot_off[uslot] + r] / k == t) {
-          member = true;
-          pos = rt.slot_off[uslot] + r;
+          for (int t = 0; t < NT; ++t) red[((tile * 4 + kq) * 16 + lg4 + 8 * r) * NT + t] = y[r][t];
+      consumers_sync();
+      // h = bf16(silu(g) * u) for (unit, feature, token); K quarters summed in order
+      for (int q = threadIdx.x; q < nu * kFFeat * T; q += kFWarps * 32) {
+        const int ui = q / (kFFeat * T), f = (q / T) % kFFeat, t = q % T;
+        int uslot, uf0;
+        gu_unit(s, blockIdx.x + (i0 + ui) * gridDim.x, uslot, uf0);
+        bool member = uslot == 0;
+        int pos = t;
+        for (int r = 0; r < (uslot == 0 ? 0 : rt.slot_cnt[uslot]); ++r)
+          if (rt.perm[rt.slot_off[uslot] + r] / k == t) {
+            member = true;
+            pos = rt.slot_off[uslot] + r;
+          }
+        if (!member) continue;
+        float gs = 0.f, us = 0.f;
+#pragma unroll
+        for (int kq2 = 0; kq2 < 4; ++kq2) {
+          gs += red[(((ui * 2 + 0) * 4 + kq2) * 16 + f) * NT + t];
+          us += red[(((ui * 2 + 1) * 4 + kq2) * 16 + f) * NT + t];
         }
-      if (!member) continue;
-      const int rg = ui * 32 + f, ru = ui * 32 + 16 + f;      // gate and up rows of the pair
-      const float gs = red[(((rg >> 3) * 2 + 0) * 8 + (rg & 7)) * NT + t] + red[(((rg >> 3) * 2 + 1) * 8 + (rg & 7)) * NT + t];
-      const float us = red[(((ru >> 3) * 2 + 0) * 8 + (ru & 7)) * NT + t] + red[(((ru >> 3) * 2 + 1) * 8 + (ru & 7)) * NT + t];
-      const uint16_t hv = float_to_bf16_bits(silu(gs) * us);
-      if (uslot == 0)
-        a.h_s[static_cast<size_t>(t) * g.Is + uf0 + f] = hv;
-      else
-        a.h[static_cast<size_t>(pos) * g.I + uf0 + f] = hv;
+        const uint16_t hv = float_to_bf16_bits(silu(gs) * us);
+        if (uslot == 0)
+          a.h_s[static_cast<size_t>(t) * g.Is + uf0 + f] = hv;
+        else
+          a.h[static_cast<size_t>(pos) * g.I + uf0 + f] = hv;
+      }
+      consumers_sync();   // red is reused by the next pair
     }
-    consumers_sync();   // red is reused by the next pair
   }
   // Every h row is written: grid barrier (consumer thread 0 of each CTA).
   consumers_sync();
@@ -624,7 +585,8 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
   if (rt.abort) return;
 
   if (s.my_blocks > 0) {
-    // stage every h row (routed rows I wide, shared rows Is wide; stride hst)
+    // stage every h row (routed rows I wide, shared rows Is wide) in the
+    // interleaved K order, and its sums over groups of 64
     const int tid = threadIdx.x, nthr = kFWarps * 32;
     const int vmax = Kmax / 8;
     for (int i = tid; i < (Tk + T) * vmax; i += nthr) {
@@ -632,93 +594,105 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
       const bool shr = r >= Tk;
       if (u * 8 >= (shr ? g.Is : g.I)) continue;
       const uint16_t* src = shr ? a.h_s + static_cast<size_t>(r - Tk) * g.Is : a.h + static_cast<size_t>(r) * g.I;
-      const uint4 v = __ldcg(reinterpret_cast<const uint4*>(src) + u);
-      const int c = u >> 2, ii = (u & 3) * 8;
-      float4* d4 = reinterpret_cast<float4*>(hs + r * hst);
-      const int win = c >> 4, ln = c & 15;
-      d4[(win * 8 + (ii >> 2)) * 16 + ln] = make_float4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y));
-      d4[(win * 8 + (ii >> 2) + 1) * 16 + ln] = make_float4(bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w));
+      reinterpret_cast<uint4*>(hs + static_cast<size_t>(r) * Kmax)[u] =
+          interleave8(__ldcg(reinterpret_cast<const uint4*>(src) + u));
     }
     consumers_sync();
-    for (int i = tid; i < (Tk + T) * (hst / 32); i += nthr) {
-      const int r = i / (hst / 32), c = i % (hst / 32);
+    const int kg = Kmax / kGroup;
+    for (int i = tid; i < (Tk + T) * kg; i += nthr) {
+      const int r = i / kg, G = i % kg;
       const int K = r >= Tk ? g.Is : g.I;
-      if (c < K / 32) {
-        const float4* r4 = reinterpret_cast<const float4*>(hs + r * hst);
-        const int win = c >> 4, ln = c & 15;
+      if (G * kGroup < K) {
+        const uint4* r4 = reinterpret_cast<const uint4*>(hs + static_cast<size_t>(r) * Kmax) + G * 8;
         float sum = 0.f;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const float4 q = r4[(win * 8 + j) * 16 + ln];
-          sum += (q.x + q.y) + (q.z + q.w);
+          const uint4 v = r4[j];
+          sum += ((bf16_lo(v.x) + bf16_hi(v.x)) + (bf16_lo(v.y) + bf16_hi(v.y))) +
+                 ((bf16_lo(v.z) + bf16_hi(v.z)) + (bf16_lo(v.w) + bf16_hi(v.w)));
         }
-        hsum[r * (hst / 32) + c] = sum;
+        hsum[i] = sum;
       }
     }
     consumers_sync();
   }
-  // down units: half-warp hw = 2 warp + (lane >> 4) owns (slot jj = hw / 4,
-  // dims 4 (hw % 4) .. +3) of the unit; lane hl = lane & 15 walks segments
-  // c = hl, hl + 16, ... with the slot's staged h rows in registers.
-  const int hl = lane & 15, hw = warp * 2 + (lane >> 4);
-  const int jj = hw >> 2, dg = hw & 3;
-  for (int di = 0; di < s.my_blocks * s.n_down_parts && ok; ++di) {
-    const int i = s.my_gu + di;
-    const int sl = i % a.ring;
-    if (!tc::mbar_wait(&full[sl], (i / a.ring) & 1u, abort_flag, a.status)) {
-      ok = false;
-      break;
-    }
-    const int bl = di / s.n_down_parts;
-    const int j0 = (di % s.n_down_parts) * s.spd, nj = min(s.spd, s.n_slots - j0);
-    const bool live = jj < nj;
-    const int j = j0 + jj;
-    const bool sh = j == 0;
-    const int K = sh ? g.Is : g.I;
-    const int nt = live ? rt.slot_cnt[j] : 0;
-    const int pos0 = live ? rt.slot_off[j] : 0;
-    const uint8_t* base = fsm + sl * a.slot_bytes + jj * (9 * Kmax);
-    const uint8_t* qrow0 = base + (dg * 4) * (K / 2);
-    const uint16_t* srow0 = reinterpret_cast<const uint16_t*>(base + 8 * Kmax) + (dg * 4) * (K / kGroup);
-    const uint16_t* brow0 = reinterpret_cast<const uint16_t*>(base + 8 * Kmax + Kmax / 2) + (dg * 4) * (K / kGroup);
-    float p[4][NT];
+  // down units: warp w owns expert slot w % 8 of the unit (16 dims x K) for
+  // the K half w / 8; lanes hold rows (dims) lg4, lg4 + 8 and tokens 0, 1
+  {
+    const int jj = warp & 7, kh = warp >> 3;
+    const int kg = Kmax / kGroup;
+    float* redd = lg;   // [8 slots][2 K halves][16 dims][NT]
+    for (int di = 0; di < s.my_blocks * s.n_down_parts && ok; ++di) {
+      const int i = s.my_gu + di;
+      const int sl = i % a.ring;
+      if (!tc::mbar_wait(&full[sl], (i / a.ring) & 1u, abort_flag, a.status)) {
+        ok = false;
+        break;
+      }
+      const int bl = di / s.n_down_parts;
+      const int j0 = (di % s.n_down_parts) * s.spd, nj = min(s.spd, s.n_slots - j0);
+      const bool live = jj < nj;
+      const int j = j0 + jj;
+      const int K = j == 0 ? g.Is : g.I;
+      const int ng = K / kGroup, gh = ng / 2;       // groups, groups per K half
+      const int nt = live ? rt.slot_cnt[j] : 0;
+      const int pos0 = live ? rt.slot_off[j] : 0;
+      float y[2][NT];
 #pragma unroll
-    for (int d = 0; d < 4; ++d)
+      for (int r = 0; r < 2; ++r)
 #pragma unroll
-      for (int t = 0; t < NT; ++t) p[d][t] = 0.f;
-    if (live) {
-      for (int c = hl; c < K / 32; c += 16) {
+        for (int t = 0; t < NT; ++t) y[r][t] = 0.f;
+      if (live) {
+        const uint8_t* base = fsm + sl * a.slot_bytes + jj * (9 * Kmax);
+        const uint8_t* qrow = base + lg4 * (K / 2) + lt * 8;
+        const uint16_t* srow = reinterpret_cast<const uint16_t*>(base + 8 * Kmax);
+        const uint16_t* brow = reinterpret_cast<const uint16_t*>(base + 8 * Kmax + Kmax / 2);
+        const bool tok_live = lg4 < nt;
+        const int hr = pos0 + (tok_live ? lg4 : 0);
+        const uint4* hrow = reinterpret_cast<const uint4*>(hs + static_cast<size_t>(hr) * Kmax) + lt * 2;
+        for (int G = kh * gh; G < (kh + 1) * gh; ++G) {
+          const uint2 qa = *reinterpret_cast<const uint2*>(qrow + G * 32);
+          const uint2 qc = *reinterpret_cast<const uint2*>(qrow + 8 * (K / 2) + G * 32);
+          const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+          const uint4 hb0 = tok_live ? hrow[G * 8] : z, hb1 = tok_live ? hrow[G * 8 + 1] : z;
+          float d[4];
+          group_dot(d, qa, qc, hb0, hb1);
+          if (lt == 0) {
 #pragma unroll
-        for (int t = 0; t < NT; ++t) {
-          if (t < nt) {
-            const int r = pos0 + t;
-            float hv[32];
-            load_seg(hs + r * hst, c, 16, hv);
-            const float X = hsum[r * (hst / 32) + c];
+            for (int r = 0; r < 2; ++r) {
+              const int row = lg4 + 8 * r;
+              const float sc = bf16_bits_to_float(srow[row * ng + G]);
+              const float bi = bf16_bits_to_float(brow[row * ng + G]);
 #pragma unroll
-            for (int d = 0; d < 4; ++d) {
-              const uint4 qv = reinterpret_cast<const uint4*>(qrow0 + d * (K / 2))[c];
-              const float s128 = 128.f * bf16_bits_to_float(srow0[d * (K / kGroup) + (c >> 1)]);
-              const float bb = bf16_bits_to_float(brow0[d * (K / kGroup) + (c >> 1)]);
-              p[d][t] = fmaf(s128, dot32r(qv, hv), fmaf(bb - s128, X, p[d][t]));
+              for (int t = 0; t < NT; ++t)
+                if (t < nt) {
+                  const float X = hsum[(pos0 + t) * kg + G];
+                  y[r][t] = fmaf(sc, d[2 * r + t] - 128.f * X, fmaf(bi, X, y[r][t]));
+                }
             }
           }
         }
       }
-    }
-    tc::fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) tc::mbar_arrive(&empty[sl]);
+      tc::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&empty[sl]);
+      if (lt == 0)
 #pragma unroll
-    for (int t = 0; t < NT; ++t) {
-      float v[4];
+        for (int r = 0; r < 2; ++r)
 #pragma unroll
-      for (int d = 0; d < 4; ++d) v[d] = p[d][t];
-      const float r = halfwarp_reduce4(v, lane);
-      if ((hl & 3) == 0 && t < nt) ys[((pos0 + t) * s.my_blocks + bl) * kFDims + dg * 4 + (hl >> 2)] = r;
+          for (int t = 0; t < NT; ++t) redd[((jj * 2 + kh) * 16 + lg4 + 8 * r) * NT + t] = y[r][t];
+      consumers_sync();
+      // y rows of this unit's slots: both K halves summed in order
+      for (int q = threadIdx.x; q < nj * kFDims * NT; q += kFWarps * 32) {
+        const int js = q / (kFDims * NT), d = (q / NT) % kFDims, t = q % NT;
+        const int jx = j0 + js;
+        if (t < rt.slot_cnt[jx])
+          ys[((rt.slot_off[jx] + t) * s.my_blocks + bl) * kFDims + d] =
+              redd[((js * 2 + 0) * 16 + d) * NT + t] + redd[((js * 2 + 1) * 16 + d) * NT + t];
+      }
+      consumers_sync();
     }
   }
-  consumers_sync();
   if (!ok) return;
   // combine: out[t, d] = bf16( sum_j w[t,j] * y[inv_perm[t k + j]][d] + sigma_t * y[T k + t][d] )
   for (int i = threadIdx.x; i < T * s.my_blocks * kFDims; i += kFWarps * 32) {
@@ -798,7 +772,6 @@ cudaError_t launch_decode_fused(const Geometry& g, const LayerPtr& L, const uint
   a.slot_bytes = 18 * g.H;                                   // one gate/up unit
   a.spd = a.slot_bytes / (9 * Kmax);
   if (a.spd > kFMaxSpd) a.spd = kFMaxSpd;
-  const int xst = fx_stride(g.H), hst = fh_stride(Kmax);
   const int rows = g.T * g.k + g.T;
   const int blocks_per_cta = (g.H / kFDims + G - 1) / G;
   auto al = [](int v) { return (v + 127) / 128 * 128; };
@@ -808,9 +781,10 @@ cudaError_t launch_decode_fused(const Geometry& g, const LayerPtr& L, const uint
     off += al(bytes);
     return o;
   };
-  const int lg_floats = max(g.T * (g.E + 1), (g.E + 1 + G - 1) / G * kFWarps * kFMaxT);
-  const int fixed = al(2 * kFRingMax * 8) + al(g.T * xst * 4) + al(g.T * (xst / 32) * 4) + al(rows * hst * 4) +
-                    al(rows * (hst / 32) * 4) + al(lg_floats * 4) +
+  // lg: logits, then the router partials, then the dot-product reductions
+  const int lg_floats = max(max(g.T * (g.E + 1), (g.E + 1 + G - 1) / G * kFWarps * kFMaxT), 16 * 16 * kFMaxT);
+  const int fixed = al(2 * kFRingMax * 8) + al(g.T * g.H * 2) + al(g.T * (g.H / kGroup) * 4) + al(rows * Kmax * 2) +
+                    al(rows * (Kmax / kGroup) * 4) + al(lg_floats * 4) +
                     al(static_cast<int>(sizeof(RouteSmem))) + al(rows * blocks_per_cta * kFDims * 4);
   const int budget = 227 * 1024 - fixed;
   a.ring = budget / a.slot_bytes;
@@ -818,10 +792,10 @@ cudaError_t launch_decode_fused(const Geometry& g, const LayerPtr& L, const uint
   if (a.ring < 2 || a.spd < 1) return cudaErrorInvalidValue;
   take(a.ring * a.slot_bytes);
   a.off_bar = take(2 * kFRingMax * 8);
-  a.off_xs = take(g.T * xst * 4);
-  a.off_xsum = take(g.T * (xst / 32) * 4);
-  a.off_hs = take(rows * hst * 4);
-  a.off_hsum = take(rows * (hst / 32) * 4);
+  a.off_xs = take(g.T * g.H * 2);
+  a.off_xsum = take(g.T * (g.H / kGroup) * 4);
+  a.off_hs = take(rows * Kmax * 2);
+  a.off_hsum = take(rows * (Kmax / kGroup) * 4);
   a.off_lg = take(lg_floats * 4);
   a.off_rt = take(static_cast<int>(sizeof(RouteSmem)));
   a.off_y = take(rows * blocks_per_cta * kFDims * 4);
