@@ -477,105 +477,99 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
   }
 
   // ------------------------------------------------------ consumer warps
-  // gate/up, two units at a time: warp w owns the 16-row tile w % 4 (unit
-  // (w%4)/2, matrix (w%4)%2) for the K quarter w / 4; per group of 64 inputs
-  // four mma.sync on the tile, then the group's scale and bias.
+  // gate/up, one unit at a time (its compute overlaps the next unit's
+  // arrival): warp w owns the 16-row tile w % 2 (gate or up) for the K eighth
+  // w / 2; per group of 64 inputs four mma.sync, then the group's scale and
+  // bias.
   bool ok = true;
-  float* red = lg;   // [4 tiles][4 K quarters][16 rows][NT] partial sums (logits are no longer needed)
+  float* red = lg;   // [2 tiles][8 K eighths][16 rows][NT] partial sums (logits are no longer needed)
   const int lg4 = lane >> 2, lt = lane & 3;
   const uint32_t qb = kFFeat * g.H / 2, sb = kFFeat * g.H / 32;
   const int ngrp = g.H / kGroup;
   {
-    const int tile = warp & 3, kq = warp >> 2;
-    const int gq = ngrp / 4;                       // groups per K quarter
-    for (int i0 = 0; i0 < s.my_gu && ok; i0 += 2) {
-      const int nu = min(2, s.my_gu - i0);
-      for (int ui = 0; ui < nu && ok; ++ui) {
-        const int i = i0 + ui;
-        if (!tc::mbar_wait(&full[i % a.ring], (i / a.ring) & 1u, abort_flag, a.status)) ok = false;
+    const int m = warp & 1, ke = warp >> 1;
+    const int ge = ngrp / 8;                       // groups per K eighth
+    for (int i = 0; i < s.my_gu && ok; ++i) {
+      const int sl = i % a.ring;
+      if (!tc::mbar_wait(&full[sl], (i / a.ring) & 1u, abort_flag, a.status)) {
+        ok = false;
+        break;
       }
-      if (!ok) break;
-      const int ur = tile >> 1, m = tile & 1;
-      const bool live = ur < nu;
+      int slot, f0;
+      gu_unit(s, blockIdx.x + i * gridDim.x, slot, f0);
+      unsigned tmask = 0;                            // tokens of this unit's expert
+      if (slot == 0)
+        tmask = (1u << T) - 1u;
+      else
+        for (int r = 0; r < rt.slot_cnt[slot]; ++r) tmask |= 1u << (rt.perm[rt.slot_off[slot] + r] / k);
+      const uint8_t* base = fsm + sl * a.slot_bytes;
+      const uint8_t* qrow = base + m * qb + lg4 * (g.H / 2) + lt * 8;         // rows lg4, lg4 + 8
+      const uint16_t* srow = reinterpret_cast<const uint16_t*>(base + 2 * qb + m * 2 * sb);
+      const uint16_t* brow = srow + sb / 2;
+      const bool tok_live = lg4 < T && ((tmask >> lg4) & 1u);
+      const uint4* xrow = reinterpret_cast<const uint4*>(xs + (tok_live ? lg4 : 0) * g.H) + lt * 2;
       float y[2][NT];
 #pragma unroll
       for (int r = 0; r < 2; ++r)
 #pragma unroll
         for (int t = 0; t < NT; ++t) y[r][t] = 0.f;
-      if (live) {
-        int slot, f0;
-        gu_unit(s, blockIdx.x + (i0 + ur) * gridDim.x, slot, f0);
-        unsigned tmask = 0;                          // tokens of this unit's expert
-        if (slot == 0)
-          tmask = (1u << T) - 1u;
-        else
-          for (int r = 0; r < rt.slot_cnt[slot]; ++r) tmask |= 1u << (rt.perm[rt.slot_off[slot] + r] / k);
-        const uint8_t* base = fsm + ((i0 + ur) % a.ring) * a.slot_bytes;
-        const uint8_t* qrow = base + m * qb + lg4 * (g.H / 2) + lt * 8;       // rows lg4, lg4 + 8
-        const uint16_t* srow = reinterpret_cast<const uint16_t*>(base + 2 * qb + m * 2 * sb);
-        const uint16_t* brow = srow + sb / 2;
-        const bool tok_live = lg4 < T && ((tmask >> lg4) & 1u);
-        const uint4* xrow = reinterpret_cast<const uint4*>(xs + (tok_live ? lg4 : 0) * g.H) + lt * 2;
-        for (int G = kq * gq; G < (kq + 1) * gq; ++G) {
-          const uint2 qa = *reinterpret_cast<const uint2*>(qrow + G * 32);
-          const uint2 qc = *reinterpret_cast<const uint2*>(qrow + 8 * (g.H / 2) + G * 32);
-          const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-          const uint4 xb0 = tok_live ? xrow[G * 8] : z, xb1 = tok_live ? xrow[G * 8 + 1] : z;
-          float d[4];
-          group_dot(d, qa, qc, xb0, xb1);
-          if (lt == 0) {   // columns 0, 1 = tokens 0, 1
+      for (int G = ke * ge; G < (ke + 1) * ge; ++G) {
+        const uint2 qa = *reinterpret_cast<const uint2*>(qrow + G * 32);
+        const uint2 qc = *reinterpret_cast<const uint2*>(qrow + 8 * (g.H / 2) + G * 32);
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        const uint4 xb0 = tok_live ? xrow[G * 8] : z, xb1 = tok_live ? xrow[G * 8 + 1] : z;
+        float d[4];
+        group_dot(d, qa, qc, xb0, xb1);
+        if (lt == 0) {   // columns 0, 1 = tokens 0, 1
 #pragma unroll
-            for (int r = 0; r < 2; ++r) {
-              const int row = lg4 + 8 * r;
-              const float sc = bf16_bits_to_float(srow[row * ngrp + G]);
-              const float bi = bf16_bits_to_float(brow[row * ngrp + G]);
+          for (int r = 0; r < 2; ++r) {
+            const int row = lg4 + 8 * r;
+            const float sc = bf16_bits_to_float(srow[row * ngrp + G]);
+            const float bi = bf16_bits_to_float(brow[row * ngrp + G]);
 #pragma unroll
-              for (int t = 0; t < NT; ++t)
-                if (t < T) {
-                  const float X = xsum[t * ngrp + G];
-                  y[r][t] = fmaf(sc, d[2 * r + t] - 128.f * X, fmaf(bi, X, y[r][t]));
-                }
-            }
+            for (int t = 0; t < NT; ++t)
+              if (t < T) {
+                const float X = xsum[t * ngrp + G];
+                y[r][t] = fmaf(sc, d[2 * r + t] - 128.f * X, fmaf(bi, X, y[r][t]));
+              }
           }
         }
       }
-      // every read of the pair's slots is done: release them
+      // every read of the unit's slot is done: release it
       tc::fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0)
-        for (int ui = 0; ui < nu; ++ui) tc::mbar_arrive(&empty[(i0 + ui) % a.ring]);
+      if (lane == 0) tc::mbar_arrive(&empty[sl]);
       if (lt == 0)
 #pragma unroll
         for (int r = 0; r < 2; ++r)
 #pragma unroll
-          for (int t = 0; t < NT; ++t) red[((tile * 4 + kq) * 16 + lg4 + 8 * r) * NT + t] = y[r][t];
+          for (int t = 0; t < NT; ++t) red[((m * 8 + ke) * 16 + lg4 + 8 * r) * NT + t] = y[r][t];
       consumers_sync();
-      // h = bf16(silu(g) * u) for (unit, feature, token); K quarters summed in order
-      for (int q = threadIdx.x; q < nu * kFFeat * T; q += kFWarps * 32) {
-        const int ui = q / (kFFeat * T), f = (q / T) % kFFeat, t = q % T;
-        int uslot, uf0;
-        gu_unit(s, blockIdx.x + (i0 + ui) * gridDim.x, uslot, uf0);
-        bool member = uslot == 0;
+      // h = bf16(silu(g) * u) for (feature, token); K eighths summed in order
+      if (threadIdx.x < kFFeat * T) {
+        const int f = threadIdx.x / T, t = threadIdx.x % T;
+        bool member = slot == 0;
         int pos = t;
-        for (int r = 0; r < (uslot == 0 ? 0 : rt.slot_cnt[uslot]); ++r)
-          if (rt.perm[rt.slot_off[uslot] + r] / k == t) {
+        for (int r = 0; r < (slot == 0 ? 0 : rt.slot_cnt[slot]); ++r)
+          if (rt.perm[rt.slot_off[slot] + r] / k == t) {
             member = true;
-            pos = rt.slot_off[uslot] + r;
+            pos = rt.slot_off[slot] + r;
           }
-        if (!member) continue;
-        float gs = 0.f, us = 0.f;
+        if (member) {
+          float gs = 0.f, us = 0.f;
 #pragma unroll
-        for (int kq2 = 0; kq2 < 4; ++kq2) {
-          gs += red[(((ui * 2 + 0) * 4 + kq2) * 16 + f) * NT + t];
-          us += red[(((ui * 2 + 1) * 4 + kq2) * 16 + f) * NT + t];
+          for (int e8 = 0; e8 < 8; ++e8) {
+            gs += red[((0 * 8 + e8) * 16 + f) * NT + t];
+            us += red[((1 * 8 + e8) * 16 + f) * NT + t];
+          }
+          const uint16_t hv = float_to_bf16_bits(silu(gs) * us);
+          if (slot == 0)
+            a.h_s[static_cast<size_t>(t) * g.Is + f0 + f] = hv;
+          else
+            a.h[static_cast<size_t>(pos) * g.I + f0 + f] = hv;
         }
-        const uint16_t hv = float_to_bf16_bits(silu(gs) * us);
-        if (uslot == 0)
-          a.h_s[static_cast<size_t>(t) * g.Is + uf0 + f] = hv;
-        else
-          a.h[static_cast<size_t>(pos) * g.I + uf0 + f] = hv;
       }
-      consumers_sync();   // red is reused by the next pair
+      consumers_sync();   // red is reused by the next unit
     }
   }
   // Every h row is written: grid barrier (consumer thread 0 of each CTA).
