@@ -396,15 +396,14 @@ int moe_route_static(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_
   return cuda_status(e);
 }
 
-int moe_forward_host(const moe_layer_desc* layer, const moe_bf16* x_host, int T, moe_bf16* out_host, void* ws,
-                     size_t ws_bytes, moe_stream stream) {
+static int forward_host_enqueue(const moe_layer_desc* layer, const moe_bf16* x_host, int T, moe_bf16* out_host,
+                                void* ws, size_t ws_bytes, cudaStream_t s) {
   int st = validate_layer(layer);
   if (st != MOE_OK) return st;
   if (T < 1 || T > kMaxT || !x_host || !out_host) return MOE_ERR_INVALID_ARG;
   st = validate_ws(layer, T, ws, ws_bytes);
   if (st != MOE_OK) return st;
   const Bufs b = resolve(layer, T, ws, nullptr);
-  const cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint16_t* xd = b.at<uint16_t>(b.w.x_stage);
   uint16_t* od = b.at<uint16_t>(b.w.out_stage);
   const size_t bytes = static_cast<size_t>(T) * layer->H * sizeof(uint16_t);
@@ -412,8 +411,22 @@ int moe_forward_host(const moe_layer_desc* layer, const moe_bf16* x_host, int T,
   st = (T <= kDecodeMaxT) ? enqueue_decode(layer, xd, T, od, b, s) : enqueue_prefill(layer, xd, T, od, b, s);
   if (st != MOE_OK) return st;
   if (cudaMemcpyAsync(out_host, od, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ERR_CUDA;
-  return cuda_status(cudaStreamSynchronize(s));
+  return MOE_OK;
 }
+
+int moe_forward_host_async(const moe_layer_desc* layer, const moe_bf16* x_host, int T, moe_bf16* out_host,
+                           void* ws, size_t ws_bytes, moe_stream stream) {
+  return forward_host_enqueue(layer, x_host, T, out_host, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int moe_forward_host(const moe_layer_desc* layer, const moe_bf16* x_host, int T, moe_bf16* out_host, void* ws,
+                     size_t ws_bytes, moe_stream stream) {
+  const cudaStream_t s0 = static_cast<cudaStream_t>(stream);
+  const int st = forward_host_enqueue(layer, x_host, T, out_host, ws, ws_bytes, s0);
+  if (st != MOE_OK) return st;
+  return cuda_status(cudaStreamSynchronize(s0));
+}
+
 
 int moe_rmsnorm(const moe_bf16* y, moe_bf16* y_out, int T, int H, float eps, moe_stream stream) {
   if (!y || !y_out || !aligned16(y) || !aligned16(y_out)) return MOE_ERR_INVALID_ARG;

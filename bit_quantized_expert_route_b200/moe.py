@@ -24,7 +24,7 @@ MOE_ERR_CUDA = -4
 MOE_ERR_DEVICE_TIMEOUT = -5
 
 # Every entry point declared in include/moe.h.
-EXPORTS = ("moe_workspace_size", "moe_route", "moe_forward", "moe_decode", "moe_forward_host",
+EXPORTS = ("moe_workspace_size", "moe_route", "moe_forward", "moe_decode", "moe_forward_host", "moe_forward_host_async",
            "moe_rmsnorm", "moe_forward_profiled", "moe_route_static", "moe_get_status", "moe_strerror")
 
 
@@ -72,6 +72,7 @@ def library() -> ctypes.CDLL:
     lib.moe_forward.argtypes = [LP, P, I, P, RP, P, S, P]
     lib.moe_decode.argtypes = [LP, P, I, P, RP, P, S, P]
     lib.moe_forward_host.argtypes = [LP, P, I, P, P, S, P]
+    lib.moe_forward_host_async.argtypes = [LP, P, I, P, P, S, P]
     lib.moe_rmsnorm.argtypes = [P, P, I, I, ctypes.c_float, P]
     lib.moe_forward_profiled.argtypes = [LP, P, I, P, P, S, P, ctypes.POINTER(ctypes.c_float),
                                          ctypes.POINTER(ctypes.c_int)]
@@ -225,6 +226,15 @@ def moe_forward_host(layer: MoELayer, x_host: torch.Tensor, out_host: torch.Tens
     T = x_host.shape[0]
     _check(library().moe_forward_host(ctypes.byref(layer.desc), x_host.data_ptr(), T, out_host.data_ptr(),
                                       workspace.data_ptr(), workspace.numel(), _stream(stream)), "moe_forward_host")
+
+
+def moe_forward_host_async(layer: MoELayer, x_host: torch.Tensor, out_host: torch.Tensor, workspace: torch.Tensor,
+                           stream=None) -> None:
+    """moe_forward_host without the final wait (page-locked x_host/out_host for overlap)."""
+    T = x_host.shape[0]
+    _check(library().moe_forward_host_async(ctypes.byref(layer.desc), x_host.data_ptr(), T, out_host.data_ptr(),
+                                            workspace.data_ptr(), workspace.numel(), _stream(stream)),
+           "moe_forward_host_async")
 
 
 def moe_rmsnorm(y: torch.Tensor, y_out: torch.Tensor, eps: float = 1e-6, stream=None) -> None:

@@ -50,7 +50,7 @@
  * work on `stream` (a cudaStream_t; NULL = the legacy default stream) and
  * return without waiting for the device.  Their outputs are valid once the
  * stream reaches that point.  No call reads device data back on the host
- * except moe_get_status and moe_forward_host.
+ * except moe_get_status and moe_forward_host (moe_forward_host_async does not wait).
  *
  * Errors.  Every entry point returns a moe_status.  Arguments are validated on
  * the host before anything is enqueued: a rejected call enqueues nothing.  A
@@ -196,6 +196,15 @@ MOE_API int moe_route_static(const moe_layer_desc* layer, const moe_bf16* x, int
  * for `stream`.  Weights stay device pointers. */
 MOE_API int moe_forward_host(const moe_layer_desc* layer, const moe_bf16* x_host, int T, moe_bf16* out_host,
                      void* workspace, size_t workspace_bytes, moe_stream stream);
+
+/* moe_forward_host without the final wait: enqueues the copy of x to the
+ * workspace, the layer and the copy of the result to out_host on `stream` and
+ * returns.  out_host is valid once the stream reaches that point; x_host must
+ * stay unchanged until then.  With page-locked buffers the copies are
+ * asynchronous, so a caller that alternates two streams (each with its own
+ * workspace) overlaps one call's copies with another call's kernels. */
+MOE_API int moe_forward_host_async(const moe_layer_desc* layer, const moe_bf16* x_host, int T, moe_bf16* out_host,
+                                   void* workspace, size_t workspace_bytes, moe_stream stream);
 
 /* y_out[t] = bf16(y[t] / sqrt(mean(y[t]^2) + eps)) over H columns, weight 1,
  * no residual: the input of the next layer in a stack of MoE layers.

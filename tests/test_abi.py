@@ -118,6 +118,8 @@ def test_calls_reject_before_launch(lib):
     L8 = fake_layer(bits=8)
     assert lib.moe_forward(ctypes.byref(L8), FAKE, 16, out, None, FAKE, need, None) == moe.MOE_ERR_UNSUPPORTED
     assert lib.moe_forward_host(ctypes.byref(L), None, 16, out, FAKE, need, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_forward_host_async(ctypes.byref(L), None, 16, out, FAKE, need, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_forward_host_async(ctypes.byref(L), FAKE, 16, out, FAKE, 16, None) == moe.MOE_ERR_WORKSPACE
     assert lib.moe_rmsnorm(FAKE, FAKE, 0, 2048, ctypes.c_float(1e-6), None) == moe.MOE_ERR_INVALID_ARG
     assert lib.moe_rmsnorm(FAKE, FAKE + 4, 4, 2048, ctypes.c_float(1e-6), None) == moe.MOE_ERR_INVALID_ARG
     assert lib.moe_get_status(None, None) == moe.MOE_ERR_WORKSPACE

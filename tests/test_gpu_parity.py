@@ -100,6 +100,25 @@ def test_forward_host_equals_device(T):
     np.testing.assert_array_equal(oh.view(torch.int16).numpy().view(np.uint16), dev["out"])
 
 
+@pytest.mark.parametrize("T", [5, 200])
+def test_forward_host_async_two_streams(T):
+    # alternating streams and workspaces, as a streaming caller would do
+    lay, x_bits, _ = workload(60 + T, T, TINY)
+    L = moe.MoELayer.from_synth(lay)
+    x = to_dev_bits(x_bits)
+    ref = torch.empty_like(x)
+    moe.moe_forward(L, x, ref, moe.alloc_workspace(L, T))
+    xh = x.cpu().pin_memory()
+    outs = [torch.empty_like(xh).pin_memory() for _ in range(2)]
+    wss = [moe.alloc_workspace(L, T) for _ in range(2)]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    for i in range(4):
+        moe.moe_forward_host_async(L, xh, outs[i % 2], wss[i % 2], stream=streams[i % 2])
+    torch.cuda.synchronize()
+    for o in outs:
+        np.testing.assert_array_equal(o.view(torch.int16).numpy(), bits_of(ref).view(np.int16))
+
+
 def test_decode_entry_rejects_large_T():
     lay, x, _ = workload(7, 65, TINY)
     with pytest.raises(moe.MoEError) as e:
