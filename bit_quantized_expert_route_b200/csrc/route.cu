@@ -99,12 +99,16 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(
   const int nch = (rows + chunk_rows - 1) / chunk_rows;
   int first = 0;
   const int nchunks = block_exclusive_scan(nch, scratch, &first);
+  // piece q starts at row floor(rows q / nch) = q base + floor(q rem / nch)
+  // (rows = base nch + rem); q rem < nch^2 <= (T_max k / 128)^2 fits 32 bits
+  const int base = nch > 0 ? rows / nch : 0, rem = nch > 0 ? rows % nch : 0;
+  int r0 = 0;
   for (int q = 0; q < nch; ++q) {
-    const int r0 = static_cast<int>((static_cast<long long>(rows) * q) / nch);
-    const int r1 = static_cast<int>((static_cast<long long>(rows) * (q + 1)) / nch);
+    const int r1 = (q + 1) * base + ((q + 1) * rem) / nch;
     Chunk ch;
     ch.e = e; ch.row0 = base_row + r0; ch.rows = r1 - r0; ch.pad = 0;
     chunks[first + q] = ch;
+    r0 = r1;
   }
   if (e == 0) *n_chunks = nchunks;
 

@@ -46,6 +46,20 @@ def test_route_only(T):
     assert_routing_exact(gpu, ref)
 
 
+# One layer per expert split of the tensor-core router: clusters of 1, 2 or 4
+# CTAs, each CTA owning a block of 16..128 experts (the last block ragged when
+# E is not a multiple of it), lists of 1, 2, 4 or 8 candidates for k.
+@pytest.mark.parametrize("E,k,zipf", [(64, 4, False), (160, 6, True), (200, 3, False), (250, 1, True),
+                                      (256, 7, False), (256, 8, True)])
+def test_route_expert_splits(E, k, zipf):
+    dims = dataclasses.replace(TINY, E=E, k=k)
+    lay, x, _ = workload(40 + E + k, 300, dims, zipf=zipf)
+    ref = moe_ref.route(x, lay, k)
+    gpu = run_layer(lay, x, entry="route")
+    assert gpu["status"] == 0
+    assert_routing_exact(gpu, ref)
+
+
 @pytest.mark.parametrize("T", [4, 100])
 def test_zero_input_gives_exact_zero(T):
     lay = synth.make_layer(0, 0, TINY)
