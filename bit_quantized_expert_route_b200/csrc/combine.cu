@@ -22,6 +22,8 @@ __device__ __forceinline__ void fma_bf16x8(float (&acc)[8], float w, const uint4
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(
     const uint16_t* __restrict__ Y, const int32_t* __restrict__ inv_perm, const float* __restrict__ topk_w,
     const float* __restrict__ sigma, int T, int k, int H, uint16_t* __restrict__ out) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int t = blockIdx.x;
   int pos[kMaxK];
   float w[kMaxK];
@@ -70,6 +72,8 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(
 // y_out = bf16(y / sqrt(mean(y^2) + eps)), one CTA per row, fixed reduction tree.
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const uint16_t* __restrict__ y, uint16_t* __restrict__ out,
                                                       int H, float eps) {
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ float part[8];
   const size_t row = blockIdx.x;
   const uint4* src = reinterpret_cast<const uint4*>(y + row * H);
@@ -121,6 +125,8 @@ __global__ void __launch_bounds__(kGatherWarps * 32) gather_k8_kernel(const uint
                                                                     const int32_t* __restrict__ perm, int Tk,
                                                                     int k, int h8, int rows,
                                                                     uint4* __restrict__ xg) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * kGatherWarps + (threadIdx.x >> 5);
   if (row >= rows) return;
@@ -145,20 +151,17 @@ __global__ void __launch_bounds__(kGatherWarps * 32) gather_k8_kernel(const uint
 cudaError_t launch_gather_k8(const uint16_t* x, const int32_t* perm, int T, int k, int H, uint16_t* xg,
                              cudaStream_t s) {
   const int rows = T * k + T;
-  gather_k8_kernel<<<(rows + kGatherWarps - 1) / kGatherWarps, kGatherWarps * 32, 0, s>>>(
-      reinterpret_cast<const uint4*>(x), perm, T * k, k, H / 8, rows, reinterpret_cast<uint4*>(xg));
-  return cudaGetLastError();
+  return launch_pdl(gather_k8_kernel, dim3((rows + kGatherWarps - 1) / kGatherWarps), dim3(kGatherWarps * 32), 0,
+                    s, reinterpret_cast<const uint4*>(x), perm, T * k, k, H / 8, rows, reinterpret_cast<uint4*>(xg));
 }
 
 cudaError_t launch_combine(const uint16_t* Y, const int32_t* inv_perm, const float* topk_w, const float* sigma,
                            int T, int k, int H, uint16_t* out, cudaStream_t s) {
-  combine_kernel<<<T, kCombThreads, 0, s>>>(Y, inv_perm, topk_w, sigma, T, k, H, out);
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel, dim3(T), dim3(kCombThreads), 0, s, Y, inv_perm, topk_w, sigma, T, k, H, out);
 }
 
 cudaError_t launch_rmsnorm(const uint16_t* y, uint16_t* out, int T, int H, float eps, cudaStream_t s) {
-  rmsnorm_kernel<<<T, 256, 0, s>>>(y, out, H, eps);
-  return cudaGetLastError();
+  return launch_pdl(rmsnorm_kernel, dim3(T), dim3(256), 0, s, y, out, H, eps);
 }
 
 }  // namespace moe

@@ -42,6 +42,15 @@ __device__ __forceinline__ float warp_sum(float v) {
 __device__ __forceinline__ float silu(float z) { return z / (1.0f + expf(-z)); }
 __device__ __forceinline__ float sigmoid(float z) { return 1.0f / (1.0f + expf(-z)); }
 
+// Programmatic dependent launch (kernels.h, launch_pdl): pdl_wait() returns
+// once the previous grid of the stream has completed and its writes are
+// visible; pdl_launch_dependents() lets the next grid be scheduled (its CTAs
+// then run their prologue and wait in their own pdl_wait()).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ uint32_t lanemask_lt() {
   uint32_t m;
   asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));

@@ -216,6 +216,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
     *abort_flag = 0;
     tc::fence_barrier_init();
   }
+  // the barrier set-up above touched only shared memory
+  pdl_wait();
+  pdl_launch_dependents();
   const int nfb = (kGateUp ? max(a.g.I, a.g.Is) : a.g.H) / BM;
   const int n_units = *a.n_chunks * nfb;
   const int Tk = a.g.T * a.g.k;
@@ -564,8 +567,7 @@ cudaError_t launch_gateup(const Geometry& g, const LayerPtr& L, const uint16_t* 
   if (e != cudaSuccess) return e;
   const int nfb = max(g.I, g.Is) / BM;
   const int grid = max(1, min(max_chunks * nfb, num_sms()));
-  grouped_gemm_tc_kernel<true><<<grid, kThreads, C::SMEM, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(grouped_gemm_tc_kernel<true>, dim3(grid), dim3(kThreads), C::SMEM, s, a);
 }
 
 cudaError_t launch_down(const Geometry& g, const LayerPtr& L, const uint16_t* h, const uint16_t* h_s,
@@ -592,8 +594,7 @@ cudaError_t launch_down(const Geometry& g, const LayerPtr& L, const uint16_t* h,
   if (e != cudaSuccess) return e;
   const int nfb = g.H / BM;
   const int grid = max(1, min(max_chunks * nfb, num_sms()));
-  grouped_gemm_tc_kernel<false><<<grid, kThreads, C::SMEM, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(grouped_gemm_tc_kernel<false>, dim3(grid), dim3(kThreads), C::SMEM, s, a);
 }
 
 }  // namespace moe

@@ -43,6 +43,27 @@ struct RoutingPtrs {
 bool make_tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* base, uint64_t cols, uint64_t rows,
                   uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw);
 
+// Launch with programmatic dependent launch: the kernel may be scheduled
+// while the previous kernel of the stream still runs, so its launch and
+// prologue overlap that kernel's tail.  Every kernel launched this way calls
+// pdl_wait() before its first global-memory access (its prologue touches only
+// its own shared and tensor memory) and then pdl_launch_dependents().
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // api.cu: raise a kernel's dynamic shared-memory limit once per device (and
 // again only if a launch needs more), keeping the attribute call off the
 // per-launch path.

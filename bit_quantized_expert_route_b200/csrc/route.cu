@@ -60,6 +60,8 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(
     int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
     Chunk* __restrict__ chunks, int32_t* __restrict__ n_chunks,
     int32_t* __restrict__ active, int32_t* __restrict__ n_active) {
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ int scratch[33];
   const int e = threadIdx.x;
   int c = 0;
@@ -125,6 +127,8 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(
 __global__ void __launch_bounds__(32 * kSegWarps) scatter_kernel(
     const int32_t* __restrict__ topk_idx, int n, int seg_len, int E, const int32_t* __restrict__ seg_base,
     int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm) {
+  pdl_wait();
+  pdl_launch_dependents();
   extern __shared__ int sh_cnt[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int seg = blockIdx.x * kSegWarps + warp;
@@ -323,11 +327,11 @@ cudaError_t launch_group(const int32_t* topk_idx, int T, int k, int E, int chunk
   const int nseg = num_segments(T);
   const int grid = (nseg + kSegWarps - 1) / kSegWarps;
   const int smem = kSegWarps * E * static_cast<int>(sizeof(int));
-  scan_kernel<<<1, kScanThreads, 0, s>>>(seg_scratch, nseg, E, T, k, chunk_rows, counts, offsets,
-                                         chunks, n_chunks, active, n_active);
-  scatter_kernel<<<grid, 32 * kSegWarps, smem, s>>>(topk_idx, n, kRouteSegTokens * k, E, seg_scratch, perm,
-                                                    inv_perm);
-  return cudaGetLastError();
+  cudaError_t e = launch_pdl(scan_kernel, dim3(1), dim3(kScanThreads), 0, s, seg_scratch, nseg, E, T, k, chunk_rows,
+                             counts, offsets, chunks, n_chunks, active, n_active);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(scatter_kernel, dim3(grid), dim3(32 * kSegWarps), static_cast<size_t>(smem), s, topk_idx, n,
+                    kRouteSegTokens * k, E, static_cast<const int32_t*>(seg_scratch), perm, inv_perm);
 }
 
 }  // namespace moe

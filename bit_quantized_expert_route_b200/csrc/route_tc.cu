@@ -276,6 +276,9 @@ __global__ void __launch_bounds__(kRThreads, 1) router_tc_kernel(
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // the prologue touched only this CTA's shared and tensor memory
+  pdl_wait();
+  pdl_launch_dependents();
 
   if (warp == kRLoadWarp) {
     // ---------------------------------------------------------- loader
@@ -421,13 +424,15 @@ cudaError_t launch_router(const uint16_t* x, const uint16_t* w_router, const flo
   cfg.blockDim = dim3(kRThreads);
   cfg.dynamicSmemBytes = kRSMEM;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = static_cast<unsigned>(sp.S);
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // as launch_pdl
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, router_tc_kernel, maps, router_bias, T, H, E, k, sp.S, sp.C, topk_idx, topk_w,
                             sigma, seg_counts, status);
 }
