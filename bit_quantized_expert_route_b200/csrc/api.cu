@@ -264,6 +264,7 @@ int enqueue_prefill(const moe_layer_desc* d, const uint16_t* x, int T, uint16_t*
   // the grouped token rows live in Y's storage until the down GEMM overwrites it
   cudaError_t e = launch_gather_k8(x, b.perm, T, d->k, d->H, Y, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
+  mark(tr, s);
   e = launch_gateup(g, L, Y, chunks, n_chunks, b.w.max_chunks, h, h_s, status, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   mark(tr, s);

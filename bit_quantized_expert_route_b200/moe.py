@@ -242,7 +242,7 @@ def moe_rmsnorm(y: torch.Tensor, y_out: torch.Tensor, eps: float = 1e-6, stream=
     _check(library().moe_rmsnorm(y.data_ptr(), y_out.data_ptr(), T, H, float(eps), _stream(stream)), "moe_rmsnorm")
 
 
-PREFILL_STAGES = ("router", "group", "gateup", "down", "combine")
+PREFILL_STAGES = ("router", "group", "gather", "gateup", "down", "combine")
 DECODE_STAGES = ("route", "gateup", "down_combine")
 FUSED_DECODE_STAGES = ("decode_fused",)
 

@@ -214,11 +214,12 @@ MOE_API int moe_rmsnorm(const moe_bf16* y, moe_bf16* y_out, int T, int H, float 
 /* Stage timing (tracing).  Same as moe_forward, but records a CUDA event on
  * `stream` before the first and after every stage, waits for the stream, and
  * writes each stage's device time in milliseconds to stage_ms[0..n-1]:
- *   T > 64:  router, group (histogram+scan+scatter), gate/up GEMM, down GEMM, combine
+ *   T > 64:  router, group (histogram+scan+scatter), gather of the grouped
+ *            token rows, gate/up GEMM, down GEMM, combine
  *   T <= 64: routing (one kernel), gate/up GEMV, down GEMV + combine, or a
  *            single stage when the fused decode kernel runs (T <= 2,
  *            H = 1024 or 2048, 16-byte aligned scale and bias stacks)
- * stage_ms: host array of at least 5 floats; *n_stages receives the count.
+ * stage_ms: host array of at least 6 floats; *n_stages receives the count.
  * The events are created and destroyed inside the call. */
 MOE_API int moe_forward_profiled(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_bf16* out,
                                  void* workspace, size_t workspace_bytes, moe_stream stream,
