@@ -194,6 +194,20 @@ def test_zero_input_closed_form():
     np.testing.assert_array_equal(r["out"], np.zeros((5, TINY.H)))                     # silu(0)*0 = 0
 
 
+def test_zero_input_with_router_bias_closed_form():
+    """x = 0: the logits are the router bias itself, so the choice is the k largest
+    bias entries (brute force), the weights their softmax, and the output 0."""
+    lay = synth.make_layer(0, 0, TINY, zipf=True)
+    bias = np.asarray(lay.router_bias, dtype=np.float32).astype(np.float64)
+    x = np.zeros((3, TINY.H), dtype=np.uint16)
+    r = moe_ref.moe_layer(x, lay, TINY.k)
+    want_idx = _brute_force_topk(bias[None, :], TINY.k)[0]
+    np.testing.assert_array_equal(r["topk_idx"], np.tile(want_idx, (3, 1)))
+    want_w = scipy.special.softmax(bias[want_idx])
+    np.testing.assert_allclose(r["topk_w"], np.tile(want_w, (3, 1)), rtol=1e-13, atol=0)
+    np.testing.assert_array_equal(r["out"], np.zeros((3, TINY.H)))
+
+
 def test_one_hot_routing_equals_dense_mlp():
     d = dataclasses.replace(TINY, k=1)
     lay, x, _ = workload(11, 12, d)
