@@ -60,6 +60,30 @@ def test_route_expert_splits(E, k, zipf):
     assert_routing_exact(gpu, ref)
 
 
+# Degenerate layers: every token chooses every expert (E = k = 8), and a
+# single expert (E = k = 1); both on the decode path (T <= 64) and prefill.
+@pytest.mark.parametrize("E,k,T", [(8, 8, 5), (8, 8, 300), (1, 1, 3), (1, 1, 130)])
+def test_degenerate_expert_counts(E, k, T):
+    dims = dataclasses.replace(TINY, E=E, k=k)
+    lay, x, _ = workload(60 + E + T, T, dims)
+    ref = moe_ref.moe_layer(x, lay, k)
+    gpu = run_layer(lay, x)
+    assert gpu["status"] == 0
+    assert_routing_exact(gpu, ref)
+    assert_output_close(gpu["out"], ref["out"])
+
+
+# Token counts at the edges of the router's 128-token tiles (one cluster each).
+@pytest.mark.parametrize("T", [127, 128, 129, 256])
+def test_router_tile_boundaries(T):
+    lay, x, _ = workload(70 + T, T, TINY)
+    ref = moe_ref.moe_layer(x, lay, TINY.k)
+    gpu = run_layer(lay, x)
+    assert gpu["status"] == 0
+    assert_routing_exact(gpu, ref)
+    assert_output_close(gpu["out"], ref["out"])
+
+
 @pytest.mark.parametrize("T", [4, 100])
 def test_zero_input_gives_exact_zero(T):
     lay = synth.make_layer(0, 0, TINY)

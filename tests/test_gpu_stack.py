@@ -22,7 +22,8 @@ import torch
 
 from bit_quantized_expert_route_b200 import moe, synth
 from oracle import moe_ref
-from tests.gpu_util import assert_output_close, bits_of, require_cuda, run_layer, to_dev_bits
+from tests.gpu_util import (assert_output_close, assert_routing_up_to_near_ties, bits_of, require_cuda, run_layer,
+                            to_dev_bits)
 from tests.workloads import FULL, workload
 
 pytestmark = pytest.mark.gpu
@@ -83,6 +84,26 @@ def test_stack_16k_tokens_layer0_sampled():
     np.testing.assert_array_equal(gpu["perm"], r["perm"])
     sample = np.unique(np.concatenate([np.random.default_rng(1).choice(T, size=96, replace=False), [0, T - 1]]))
     ref = moe_ref.moe_layer(x_bits, lay, FULL.k, tokens=sample)
+    assert_output_close(gpu["out"][sample], ref["out"])
+
+
+def test_max_tokens_routing_and_sampled_outputs():
+    """The largest call the library accepts (T = 65536).  At this size a few tokens
+    have two of their best logits within FP32 rounding of each other, so the order
+    of those two may differ from float64's: routing is exact up to such near ties
+    (and bit-exact once the accepted order is fed back), outputs are checked on a
+    sample that includes the first and last token."""
+    T = 65536
+    lay, x_bits, _ = workload(107, T, FULL)
+    L = moe.MoELayer.from_synth(lay)
+    gpu = run_layer(lay, x_bits, dev_layer=L)
+    assert gpu["status"] == 0
+    r = moe_ref.route(x_bits, lay, FULL.k)
+    override = assert_routing_up_to_near_ties(gpu, r, FULL.k)
+    assert len(override) <= 16, len(override)
+    sample = np.unique(np.concatenate([np.random.default_rng(2).choice(T, size=64, replace=False), [0, T - 1],
+                                       np.array(sorted(override), dtype=np.int64)]))
+    ref = moe_ref.moe_layer(x_bits, lay, FULL.k, tokens=sample, idx_override=override)
     assert_output_close(gpu["out"][sample], ref["out"])
 
 
