@@ -1,5 +1,5 @@
-// Host-side construction of TMA tensor maps (the driver's encoder is looked
-// up once through the runtime, so the library needs no link to libcuda).
+// Host-side construction of TMA tensor maps (the CUDA driver API's encoder is
+// looked up once through the runtime, so the library needs no link to libcuda).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
