@@ -51,6 +51,11 @@
  * return without waiting for the device.  Their outputs are valid once the
  * stream reaches that point.  No call reads device data back on the host
  * except moe_get_status and moe_forward_host (moe_forward_host_async does not wait).
+ * The prefill kernels and moe_rmsnorm are launched with programmatic
+ * dependent launch: a kernel may be scheduled, and set up its own on-chip
+ * state, while the preceding work of the stream finishes, but it reads and
+ * writes no global memory before that work has completed, so stream order
+ * holds for every buffer as with ordinary launches.
  *
  * Errors.  Every entry point returns a moe_status.  Arguments are validated on
  * the host before anything is enqueued: a rejected call enqueues nothing.  A
