@@ -129,3 +129,22 @@ def test_library_is_built_for_sm100a():
     moe_build.build()
     assert "arch=compute_100a,code=sm_100a" in " ".join(moe_build.NVCC_FLAGS)
     assert os.path.exists(moe_build.LIB)
+
+
+def _static_route_need(T, E, k, sigma_given):
+    """Scratch bytes of moe_route_static as moe.h states them (each piece rounded to 256 B)."""
+    r = lambda b: (b + 255) // 256 * 256
+    n = r(-(-T // 128) * E * 4) + r((T * k // 128 + T // 128 + E + 2) * 16) + r(4) + r((E + 1) * 4) + r(4)
+    return n + (0 if sigma_given else r(T * 4))
+
+
+def test_static_route_limits(lib):
+    """moe_route_static admits T <= 56704 (sigma given) / 39424 (sigma NULL) for E=256, k=8,
+    and rejects the next T on the host with MOE_ERR_WORKSPACE before any CUDA call.
+    (Only the rejecting side is called: an accepted call would launch kernels.)"""
+    L = fake_layer()
+    for sigma, limit in ((FAKE, 56704), (None, 39424)):
+        assert _static_route_need(limit, 256, 8, sigma is not None) <= 512 * 1024
+        assert _static_route_need(limit + 1, 256, 8, sigma is not None) > 512 * 1024
+        r = moe.RoutingC(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, sigma)
+        assert lib.moe_route_static(ctypes.byref(L), FAKE, limit + 1, ctypes.byref(r), None) == moe.MOE_ERR_WORKSPACE
