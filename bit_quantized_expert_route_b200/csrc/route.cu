@@ -19,7 +19,7 @@ namespace moe {
 // Integer atomics only count (order-independent); every position comes from
 // the scan and an in-order rank, so the permutation is deterministic.
 // ---------------------------------------------------------------------------
-constexpr int kSegWarps = 4;
+constexpr int kSegWarps = 4;   // scatter warps per 128-token segment (32 tokens each)
 
 // Block-wide exclusive scan over blockDim.x (<= 1024) ints; returns the total.
 __device__ int block_exclusive_scan(int v, int* scratch /*[32]*/, int* out_excl) {
@@ -124,33 +124,49 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(
   }
 }
 
+// One CTA per segment; warp w ranks the entries of the segment's tokens
+// [32 w, 32 w + 32).  Each warp first counts its slice's experts, so warp w
+// starts expert e at the segment's base plus the counts of slices 0..w-1;
+// then it ranks its entries in order, 32 per round (at most k rounds).
 __global__ void __launch_bounds__(32 * kSegWarps) scatter_kernel(
     const int32_t* __restrict__ topk_idx, int n, int seg_len, int E, const int32_t* __restrict__ seg_base,
     int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm) {
   pdl_wait();
   pdl_launch_dependents();
-  extern __shared__ int sh_cnt[];
+  extern __shared__ int sh_cnt[];   // [kSegWarps][E]: slice counts, then each slice's first positions
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int seg = blockIdx.x * kSegWarps + warp;
-  const int nseg = (n + seg_len - 1) / seg_len;
-  if (seg >= nseg) return;
+  const int seg = blockIdx.x;
+  const int slice_len = seg_len / kSegWarps;
+  const int b = seg * seg_len + warp * slice_len, end = min(b + slice_len, n);
   int* cnt = sh_cnt + warp * E;
-  for (int e = lane; e < E; e += 32) cnt[e] = seg_base[static_cast<size_t>(seg) * E + e];
-  const int b = seg * seg_len, end = min(b + seg_len, n);
-  constexpr int kRounds = kRouteSegTokens * kMaxK / 32;   // 32 rounds of 32 entries at most
+  for (int e = lane; e < E; e += 32) cnt[e] = 0;
+  constexpr int kRounds = kRouteSegTokens * kMaxK / 32 / kSegWarps;   // 8 rounds of 32 entries at most
   int ex[kRounds];
 #pragma unroll
   for (int j = 0; j < kRounds; ++j) {
     const int i = b + j * 32 + lane;
-    ex[j] = (i < end) ? topk_idx[i] : -1;                   // every load issued before the first round
+    const int e = (i < end) ? topk_idx[i] : -1;                     // every load issued before the first use
+    ex[j] = (e >= 0 && e < E) ? e : -1;
   }
   __syncwarp();
+#pragma unroll
+  for (int j = 0; j < kRounds; ++j)
+    if (ex[j] >= 0) atomicAdd(&cnt[ex[j]], 1);                       // counting is order-independent
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = seg_base[static_cast<size_t>(seg) * E + e];
+    for (int w = 0; w < kSegWarps; ++w) {
+      const int c = sh_cnt[w * E + e];
+      sh_cnt[w * E + e] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
 #pragma unroll
   for (int j = 0; j < kRounds; ++j) {
     if (b + j * 32 >= end) break;
     const int i = b + j * 32 + lane;
-    int e = ex[j];
-    if (e >= E) e = -1;
+    const int e = ex[j];
     const unsigned peers = __match_any_sync(0xffffffffu, e);
     const int rank = __popc(peers & lanemask_lt());
     const int start = (e >= 0) ? cnt[e] : 0;
@@ -325,7 +341,7 @@ cudaError_t launch_group(const int32_t* topk_idx, int T, int k, int E, int chunk
                          int32_t* active, int32_t* n_active, cudaStream_t s) {
   const int n = T * k;
   const int nseg = num_segments(T);
-  const int grid = (nseg + kSegWarps - 1) / kSegWarps;
+  const int grid = nseg;
   const int smem = kSegWarps * E * static_cast<int>(sizeof(int));
   cudaError_t e = launch_pdl(scan_kernel, dim3(1), dim3(kScanThreads), 0, s, seg_scratch, nseg, E, T, k, chunk_rows,
                              counts, offsets, chunks, n_chunks, active, n_active);
