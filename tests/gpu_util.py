@@ -104,6 +104,7 @@ def assert_routing_up_to_near_ties(gpu: dict, ref: dict, k: int) -> dict:
     np.testing.assert_array_equal(gpu["perm"], perm)
     np.testing.assert_array_equal(gpu["inv_perm"], inv_perm)
     np.testing.assert_allclose(gpu["topk_w"], moe_ref.topk_weights(logits, idx), rtol=0, atol=2e-6)
+    assert np.all(np.abs(gpu["topk_w"].sum(axis=1) - 1.0) < 1e-6)
     np.testing.assert_allclose(gpu["sigma"], ref["sigma"], rtol=0, atol=2e-6)
     return override
 
