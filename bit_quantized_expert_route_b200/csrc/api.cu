@@ -3,12 +3,14 @@
 // except in moe_get_status and moe_forward_host.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
 
 #include "moe.h"
 #include "kernels.h"
+#include "tc.cuh"
 
 namespace moe {
 
@@ -37,6 +39,12 @@ cudaError_t ensure_smem(const void* func, int bytes) {
   return e;
 }
 
+namespace {
+std::atomic<long long> g_wait_limit{tc::kDefaultWaitLimit};
+}  // namespace
+
+long long wait_limit_cycles() { return g_wait_limit.load(std::memory_order_relaxed); }
+
 // Keeps the device busy for `ns` nanoseconds (bounded by construction), so
 // that every launch a traced call enqueues is already queued when its first
 // stage starts: stage times then measure kernels, not host launch gaps.
@@ -56,6 +64,7 @@ using namespace moe;
 
 constexpr int kDecodeMaxT = 64;
 constexpr int kMaxT = 65536;
+constexpr int kMaxStackLayers = 1024;
 constexpr size_t kAlign = 256;
 
 size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
@@ -249,8 +258,10 @@ int enqueue_decode(const moe_layer_desc* d, const uint16_t* x, int T, uint16_t* 
   return cuda_status(e);
 }
 
+// out: the layer output (may be NULL when norm_out is given); norm_out (may
+// be NULL): RMSNorm(out) with weight 1 and eps, fused into the combine.
 int enqueue_prefill(const moe_layer_desc* d, const uint16_t* x, int T, uint16_t* out, const Bufs& b,
-                    cudaStream_t s, Tracer* tr = nullptr) {
+                    cudaStream_t s, Tracer* tr = nullptr, uint16_t* norm_out = nullptr, float eps = 0.f) {
   int st = enqueue_route(d, x, T, b, s, tr);
   if (st != MOE_OK) return st;
   const Geometry g{T, d->H, d->I, d->I_shared, d->E, d->k};
@@ -262,7 +273,7 @@ int enqueue_prefill(const moe_layer_desc* d, const uint16_t* x, int T, uint16_t*
   const Chunk* chunks = b.at<Chunk>(b.w.chunks);
   const int32_t* n_chunks = b.at<int32_t>(b.w.n_chunks);
   // the grouped token rows live in Y's storage until the down GEMM overwrites it
-  cudaError_t e = launch_gather_k8(x, b.perm, T, d->k, d->H, Y, s);
+  cudaError_t e = launch_gather_k8(x, b.perm, T, d->k, d->H, Y, status, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   mark(tr, s);
   e = launch_gateup(g, L, Y, chunks, n_chunks, b.w.max_chunks, h, h_s, status, s);
@@ -271,9 +282,20 @@ int enqueue_prefill(const moe_layer_desc* d, const uint16_t* x, int T, uint16_t*
   e = launch_down(g, L, h, h_s, chunks, n_chunks, b.w.max_chunks, Y, status, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   mark(tr, s);
-  e = launch_combine(Y, b.inv_perm, b.topk_w, b.sigma, T, d->k, d->H, out, s);
+  e = launch_combine(Y, b.inv_perm, b.topk_w, b.sigma, T, d->k, d->H, out, norm_out, eps, status, s);
   mark(tr, s);
   return cuda_status(e);
+}
+
+// One layer of a stack: out (may be NULL) receives the layer output and
+// norm_out (may be NULL) its RMSNorm, the next layer's input.
+int enqueue_layer(const moe_layer_desc* d, const uint16_t* x, int T, uint16_t* out, uint16_t* norm_out, float eps,
+                  const Bufs& b, cudaStream_t s) {
+  if (T > kDecodeMaxT) return enqueue_prefill(d, x, T, out, b, s, nullptr, norm_out, eps);
+  uint16_t* y = out ? out : norm_out;
+  const int st = enqueue_decode(d, x, T, y, b, s);
+  if (st != MOE_OK || !norm_out) return st;
+  return cuda_status(launch_rmsnorm(y, norm_out, T, d->H, eps, s));   // in place when out is NULL
 }
 
 int check_call(const moe_layer_desc* d, const void* x, int T, int T_limit, const void* out, const moe_routing* r,
@@ -294,6 +316,9 @@ int check_call(const moe_layer_desc* d, const void* x, int T, int T_limit, const
 // the library (a CUDA __device__ variable exists on every device of the
 // context), so callers that cannot allocate need not pass a workspace.
 constexpr size_t kRouteStaticBytes = 512u * 1024u;
+// moe.h states the scratch limit with 128-token segments and 128-row chunks.
+static_assert(moe::kGemmChunkRows == 128 && moe::kRouteSegTokens == 128,
+              "update moe_route_static's documented limit");
 static __device__ __align__(256) unsigned char g_route_static_scratch[kRouteStaticBytes];
 
 namespace {
@@ -316,6 +341,41 @@ int route_static_scratch(void** out) {
   }
   *out = g_route_static_ptr[dev];
   return MOE_OK;
+}
+
+// Pieces of the static scratch for one moe_route_static call: the same
+// buffers a workspace provides to moe_route (control block first, which the
+// zero-initialised array and every call leave zero except for a recorded
+// error status), each rounded up to 256 bytes.
+struct RouteStaticLayout {
+  size_t status, counter, seg, chunks, n_chunks, active, n_active, logits, sigma, total;
+};
+
+RouteStaticLayout route_static_layout(const moe_layer_desc* d, int T, bool sigma_given) {
+  RouteStaticLayout l{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align_up(bytes);
+    return o;
+  };
+  l.status = take(256);   // status word, then the small-T routing counter
+  l.counter = l.status + 4;
+  if (T <= kDecodeMaxT) {
+    l.logits = take(static_cast<size_t>(T) * (d->E + 1) * 4);
+  } else {
+    const size_t n = static_cast<size_t>(T) * d->k;
+    const int cr = gemm_chunk_rows();
+    const size_t max_chunks = n / cr + T / cr + d->E + 2;
+    l.seg = take(static_cast<size_t>(num_segments(T)) * d->E * 4);
+    l.chunks = take(max_chunks * sizeof(Chunk));
+    l.n_chunks = take(4);
+  }
+  l.active = take(static_cast<size_t>(d->E + 1) * 4);
+  l.n_active = take(4);
+  l.sigma = sigma_given ? 0 : take(static_cast<size_t>(T) * 4);
+  l.total = off;
+  return l;
 }
 
 }  // namespace
@@ -356,6 +416,38 @@ int moe_decode(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_bf16* 
   return enqueue_decode(layer, x, T, out, resolve(layer, T, ws, r), static_cast<cudaStream_t>(stream));
 }
 
+int moe_forward_stack(const moe_layer_desc* layers, int n_layers, const moe_bf16* x, int T, moe_bf16* out,
+                      moe_bf16* trace, float eps, void* ws, size_t ws_bytes, moe_stream stream) {
+  if (!layers || n_layers < 1 || n_layers > kMaxStackLayers) return MOE_ERR_INVALID_ARG;
+  if (!(eps >= 0.f) || (trace && !aligned16(trace))) return MOE_ERR_INVALID_ARG;
+  for (int l = 0; l < n_layers; ++l) {
+    const moe_layer_desc& d = layers[l];
+    const int st = check_call(&d, x, T, kMaxT, out, nullptr, ws, ws_bytes, true);
+    if (st != MOE_OK) return st;
+    const moe_layer_desc& d0 = layers[0];
+    if (d.H != d0.H || d.I != d0.I || d.I_shared != d0.I_shared || d.E != d0.E || d.k != d0.k)
+      return MOE_ERR_UNSUPPORTED;
+  }
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t act = static_cast<size_t>(T) * layers[0].H;
+  const Bufs b0 = resolve(&layers[0], T, ws, nullptr);
+  uint16_t* pingpong[2] = {b0.at<uint16_t>(b0.w.x_stage), b0.at<uint16_t>(b0.w.out_stage)};
+  uint16_t* tr = reinterpret_cast<uint16_t*>(trace);
+  if (tr && cudaMemcpyAsync(tr, x, act * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess) return MOE_ERR_CUDA;
+  const uint16_t* xin = x;
+  for (int l = 0; l < n_layers; ++l) {
+    const bool last = l == n_layers - 1;
+    uint16_t* y = last ? out : (tr ? tr + (2 * l + 1) * act : nullptr);
+    uint16_t* next = last ? nullptr : (tr ? tr + (2 * l + 2) * act : pingpong[l & 1]);
+    const int st = enqueue_layer(&layers[l], xin, T, y, next, eps, resolve(&layers[l], T, ws, nullptr), s);
+    if (st != MOE_OK) return st;
+    xin = next;
+  }
+  if (tr && cudaMemcpyAsync(tr + (2 * n_layers - 1) * act, out, act * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
 int moe_route_static(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_routing* r, moe_stream stream) {
   if (!r) return MOE_ERR_INVALID_ARG;
   int st = validate_layer(layer);
@@ -363,38 +455,32 @@ int moe_route_static(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_
   if (T < 1 || T > kMaxT || !x || !aligned16(x)) return MOE_ERR_INVALID_ARG;
   st = validate_routing(r);
   if (st != MOE_OK) return st;
-  // carve the static scratch: segment counts, chunk list, counters, active list, sigma
-  const size_t n = static_cast<size_t>(T) * layer->k;
-  const int cr = gemm_chunk_rows();
-  const int max_chunks = static_cast<int>(n / cr + T / cr + layer->E + 2);
-  size_t off = 0;
-  auto take = [&](size_t bytes) {
-    const size_t o = off;
-    off += align_up(bytes);
-    return o;
-  };
-  const size_t o_seg = take(static_cast<size_t>(num_segments(T)) * layer->E * 4);
-  const size_t o_chunks = take(static_cast<size_t>(max_chunks) * sizeof(Chunk));
-  const size_t o_nchunks = take(4);
-  const size_t o_active = take(static_cast<size_t>(layer->E + 1) * 4);
-  const size_t o_nactive = take(4);
-  const size_t o_sigma = r->sigma ? 0 : take(static_cast<size_t>(T) * 4);
-  if (off > kRouteStaticBytes) return MOE_ERR_WORKSPACE;
+  // carve the static scratch exactly as a workspace is carved for moe_route
+  const RouteStaticLayout sl = route_static_layout(layer, T, r->sigma != nullptr);
+  if (sl.total > kRouteStaticBytes) return MOE_ERR_WORKSPACE;
   void* base = nullptr;
   st = route_static_scratch(&base);
   if (st != MOE_OK) return st;
   char* b = static_cast<char*>(base);
-  const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  float* sigma = r->sigma ? r->sigma : reinterpret_cast<float*>(b + o_sigma);
-  cudaError_t e = launch_router(x, layer->w_router, layer->router_bias, layer->w_shared_gate, T, layer->H,
-                                layer->E, layer->k, r->topk_idx, r->topk_w, sigma, reinterpret_cast<int32_t*>(b + o_seg),
-                                nullptr, s);
-  if (e != cudaSuccess) return MOE_ERR_CUDA;
-  e = launch_group(r->topk_idx, T, layer->k, layer->E, cr, reinterpret_cast<int32_t*>(b + o_seg), r->counts,
-                   r->offsets, r->perm, r->inv_perm, reinterpret_cast<Chunk*>(b + o_chunks),
-                   reinterpret_cast<int32_t*>(b + o_nchunks), reinterpret_cast<int32_t*>(b + o_active),
-                   reinterpret_cast<int32_t*>(b + o_nactive), s);
-  return cuda_status(e);
+  Bufs bufs;
+  bufs.base = b;
+  bufs.w = WsLayout{};
+  bufs.w.status = sl.status;
+  bufs.w.counter = sl.counter;
+  bufs.w.seg = sl.seg;
+  bufs.w.chunks = sl.chunks;
+  bufs.w.n_chunks = sl.n_chunks;
+  bufs.w.active = sl.active;
+  bufs.w.n_active = sl.n_active;
+  bufs.w.logits = sl.logits;
+  bufs.topk_idx = r->topk_idx;
+  bufs.topk_w = r->topk_w;
+  bufs.counts = r->counts;
+  bufs.offsets = r->offsets;
+  bufs.perm = r->perm;
+  bufs.inv_perm = r->inv_perm;
+  bufs.sigma = r->sigma ? r->sigma : reinterpret_cast<float*>(b + sl.sigma);
+  return enqueue_route(layer, x, T, bufs, static_cast<cudaStream_t>(stream));
 }
 
 static int forward_host_enqueue(const moe_layer_desc* layer, const moe_bf16* x_host, int T, moe_bf16* out_host,
@@ -462,7 +548,12 @@ int moe_forward_profiled(const moe_layer_desc* layer, const moe_bf16* x, int T, 
 }
 
 int moe_get_status(void* ws, moe_stream stream) {
-  if (!ws || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1))) return MOE_ERR_WORKSPACE;
+  if (!ws) {
+    // the status word of moe_route_static's scratch on the current device
+    const int st = route_static_scratch(&ws);
+    if (st != MOE_OK) return st;
+  }
+  if (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) return MOE_ERR_WORKSPACE;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   int host = 0;
   if (cudaMemcpyAsync(&host, ws, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ERR_CUDA;
@@ -471,6 +562,11 @@ int moe_get_status(void* ws, moe_stream stream) {
   if (host != MOE_OK && cudaMemsetAsync(ws, 0, 16, s) != cudaSuccess) return MOE_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
   return host;
+}
+
+int moe_set_wait_limit(long long cycles) {
+  g_wait_limit.store(cycles > 0 ? cycles : tc::kDefaultWaitLimit, std::memory_order_relaxed);
+  return MOE_OK;
 }
 
 const char* moe_strerror(int status) {

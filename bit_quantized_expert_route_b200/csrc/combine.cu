@@ -10,7 +10,15 @@ namespace moe {
 // experts' down-projection rows) is stored as bf16.  Each thread issues all
 // 2 (k + 1) of its 16-byte loads before the first FMA, so a CTA keeps many
 // DRAM requests in flight.
+//
+// In a stack of layers the next layer's input is RMSNorm(out_t) (weight 1, no
+// residual): with norm_out given, the CTA also sums the squares of the row's
+// bf16 outputs (per thread in column order, then the warps' sums in a fixed
+// tree) and writes norm_out_t = bf16(out_t / sqrt(mean(out_t^2) + eps)), the
+// value the stand-alone RMSNorm computes from out_t, without another pass
+// over the row.  out may be NULL when only the normalised row is wanted.
 constexpr int kCombThreads = 128;
+constexpr int kCombMaxIters = 4;    // 16-column pieces per thread: H <= 128 * 16 * 4 = 8192
 
 __device__ __forceinline__ void fma_bf16x8(float (&acc)[8], float w, const uint4& y) {
   acc[0] = fmaf(w, bf16_lo(y.x), acc[0]); acc[1] = fmaf(w, bf16_hi(y.x), acc[1]);
@@ -19,11 +27,39 @@ __device__ __forceinline__ void fma_bf16x8(float (&acc)[8], float w, const uint4
   acc[6] = fmaf(w, bf16_lo(y.w), acc[6]); acc[7] = fmaf(w, bf16_hi(y.w), acc[7]);
 }
 
+__device__ __forceinline__ uint4 pack8(const float (&a)[8]) {
+  uint4 o;
+  o.x = pack_bf16x2(a[0], a[1]); o.y = pack_bf16x2(a[2], a[3]);
+  o.z = pack_bf16x2(a[4], a[5]); o.w = pack_bf16x2(a[6], a[7]);
+  return o;
+}
+
+__device__ __forceinline__ float sumsq8(const uint4& v, float ss) {
+  ss = fmaf(bf16_lo(v.x), bf16_lo(v.x), ss); ss = fmaf(bf16_hi(v.x), bf16_hi(v.x), ss);
+  ss = fmaf(bf16_lo(v.y), bf16_lo(v.y), ss); ss = fmaf(bf16_hi(v.y), bf16_hi(v.y), ss);
+  ss = fmaf(bf16_lo(v.z), bf16_lo(v.z), ss); ss = fmaf(bf16_hi(v.z), bf16_hi(v.z), ss);
+  ss = fmaf(bf16_lo(v.w), bf16_lo(v.w), ss); ss = fmaf(bf16_hi(v.w), bf16_hi(v.w), ss);
+  return ss;
+}
+
+__device__ __forceinline__ uint4 scale8(const uint4& v, float s) {
+  uint4 o;
+  o.x = pack_bf16x2(bf16_lo(v.x) * s, bf16_hi(v.x) * s);
+  o.y = pack_bf16x2(bf16_lo(v.y) * s, bf16_hi(v.y) * s);
+  o.z = pack_bf16x2(bf16_lo(v.z) * s, bf16_hi(v.z) * s);
+  o.w = pack_bf16x2(bf16_lo(v.w) * s, bf16_hi(v.w) * s);
+  return o;
+}
+
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(
     const uint16_t* __restrict__ Y, const int32_t* __restrict__ inv_perm, const float* __restrict__ topk_w,
-    const float* __restrict__ sigma, int T, int k, int H, uint16_t* __restrict__ out) {
+    const float* __restrict__ sigma, int T, int k, int H, uint16_t* __restrict__ out,
+    uint16_t* __restrict__ norm_out, float eps, const int* status) {
   pdl_wait();
   pdl_launch_dependents();
+  // a recorded error means inv_perm may hold entries no kernel wrote: skip
+  if (*reinterpret_cast<volatile const int*>(status) != 0) return;
+  __shared__ float part[kCombThreads / 32];
   const int t = blockIdx.x;
   int pos[kMaxK];
   float w[kMaxK];
@@ -34,7 +70,12 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(
   }
   const float sg = __ldg(sigma + t);
   const size_t shared_row = static_cast<size_t>(T) * k + t;
-  for (int c = threadIdx.x * 16; c < H; c += kCombThreads * 16) {
+  uint4 keep[2 * kCombMaxIters];      // this thread's bf16 outputs, kept for the normalisation
+  float ss = 0.f;
+#pragma unroll
+  for (int it = 0; it < kCombMaxIters; ++it) {
+    const int c = (it * kCombThreads + threadIdx.x) * 16;
+    if (c >= H) break;
     uint4 ya[kMaxK], yb[kMaxK];
 #pragma unroll
     for (int j = 0; j < kMaxK; ++j) {
@@ -58,19 +99,38 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(
     }
     fma_bf16x8(a0, sg, sa);
     fma_bf16x8(a1, sg, sb);
-    uint4 o0, o1;
-    o0.x = pack_bf16x2(a0[0], a0[1]); o0.y = pack_bf16x2(a0[2], a0[3]);
-    o0.z = pack_bf16x2(a0[4], a0[5]); o0.w = pack_bf16x2(a0[6], a0[7]);
-    o1.x = pack_bf16x2(a1[0], a1[1]); o1.y = pack_bf16x2(a1[2], a1[3]);
-    o1.z = pack_bf16x2(a1[4], a1[5]); o1.w = pack_bf16x2(a1[6], a1[7]);
-    uint4* dst = reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * H + c);
-    dst[0] = o0;
-    dst[1] = o1;
+    const uint4 o0 = pack8(a0), o1 = pack8(a1);
+    if (out) {
+      uint4* dst = reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * H + c);
+      dst[0] = o0;
+      dst[1] = o1;
+    }
+    keep[2 * it] = o0;
+    keep[2 * it + 1] = o1;
+    ss = sumsq8(o1, sumsq8(o0, ss));
+  }
+  if (norm_out == nullptr) return;
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  float tot = 0.f;
+#pragma unroll
+  for (int w8 = 0; w8 < kCombThreads / 32; ++w8) tot += part[w8];
+  const float inv = 1.0f / sqrtf(tot / static_cast<float>(H) + eps);
+#pragma unroll
+  for (int it = 0; it < kCombMaxIters; ++it) {
+    const int c = (it * kCombThreads + threadIdx.x) * 16;
+    if (c >= H) break;
+    uint4* dst = reinterpret_cast<uint4*>(norm_out + static_cast<size_t>(t) * H + c);
+    dst[0] = scale8(keep[2 * it], inv);
+    dst[1] = scale8(keep[2 * it + 1], inv);
   }
 }
 
 // y_out = bf16(y / sqrt(mean(y^2) + eps)), one CTA per row, fixed reduction tree.
-__global__ void __launch_bounds__(256) rmsnorm_kernel(const uint16_t* __restrict__ y, uint16_t* __restrict__ out,
+// y and out may be the same buffer (no __restrict__): each thread reads its
+// columns of the row before any thread writes them back.
+__global__ void __launch_bounds__(256) rmsnorm_kernel(const uint16_t* y, uint16_t* out,
                                                       int H, float eps) {
   pdl_wait();
   pdl_launch_dependents();
@@ -124,9 +184,11 @@ __device__ __forceinline__ uint4 interleave_k8(const uint4& v) {   // (x0,x1)(x2
 __global__ void __launch_bounds__(kGatherWarps * 32) gather_k8_kernel(const uint4* __restrict__ x,
                                                                     const int32_t* __restrict__ perm, int Tk,
                                                                     int k, int h8, int rows,
-                                                                    uint4* __restrict__ xg) {
+                                                                    uint4* __restrict__ xg, const int* status) {
   pdl_wait();
   pdl_launch_dependents();
+  // a recorded error means perm may hold entries no kernel wrote: skip
+  if (*reinterpret_cast<volatile const int*>(status) != 0) return;
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * kGatherWarps + (threadIdx.x >> 5);
   if (row >= rows) return;
@@ -149,15 +211,19 @@ __global__ void __launch_bounds__(kGatherWarps * 32) gather_k8_kernel(const uint
 }
 
 cudaError_t launch_gather_k8(const uint16_t* x, const int32_t* perm, int T, int k, int H, uint16_t* xg,
-                             cudaStream_t s) {
+                             const int* status, cudaStream_t s) {
   const int rows = T * k + T;
   return launch_pdl(gather_k8_kernel, dim3((rows + kGatherWarps - 1) / kGatherWarps), dim3(kGatherWarps * 32), 0,
-                    s, reinterpret_cast<const uint4*>(x), perm, T * k, k, H / 8, rows, reinterpret_cast<uint4*>(xg));
+                    s, reinterpret_cast<const uint4*>(x), perm, T * k, k, H / 8, rows, reinterpret_cast<uint4*>(xg),
+                    status);
 }
 
 cudaError_t launch_combine(const uint16_t* Y, const int32_t* inv_perm, const float* topk_w, const float* sigma,
-                           int T, int k, int H, uint16_t* out, cudaStream_t s) {
-  return launch_pdl(combine_kernel, dim3(T), dim3(kCombThreads), 0, s, Y, inv_perm, topk_w, sigma, T, k, H, out);
+                           int T, int k, int H, uint16_t* out, uint16_t* norm_out, float eps, const int* status,
+                           cudaStream_t s) {
+  if (H % 16 || H > kCombThreads * 16 * kCombMaxIters) return cudaErrorInvalidValue;
+  return launch_pdl(combine_kernel, dim3(T), dim3(kCombThreads), 0, s, Y, inv_perm, topk_w, sigma, T, k, H, out,
+                    norm_out, eps, status);
 }
 
 cudaError_t launch_rmsnorm(const uint16_t* y, uint16_t* out, int T, int H, float eps, cudaStream_t s) {

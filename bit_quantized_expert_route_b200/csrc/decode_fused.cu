@@ -57,6 +57,7 @@ constexpr int kFDims = 16;                      // output dims per down block (o
 constexpr int kFMaxSpd = 8;                     // expert slots per down unit
 constexpr int kFRingMax = 8;
 constexpr int kFMaxT = 2;
+constexpr int kFRouterRows = 2;                 // router rows per CTA with loads in flight together
 
 struct FusedArgs {
   Geometry g;
@@ -72,6 +73,7 @@ struct FusedArgs {
   unsigned* bar;          // [0] arrivals, [1] generation
   int* status;
   int ring, slot_bytes, spd;
+  long long wait_limit;   // cycles before a bounded wait gives up
   int off_bar, off_xs, off_xsum, off_hs, off_hsum, off_lg, off_rt, off_y;
 };
 
@@ -197,26 +199,38 @@ __device__ __forceinline__ void topk_redux(const float* lg, int E, int k, int la
 
 __device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kFWarps * 32) : "memory"); }
 
-// Grid-wide barrier, called by one thread per CTA after a CTA barrier (all
-// CTAs co-resident).  bar[0] counts arrivals with acquire-release adds (each
-// arrival publishes its CTA's writes; the last arriver acquires them all),
-// the last arriver resets it and bumps the generation bar[1] with a release
-// store; the others spin (bounded) on an acquire load of the generation.
-__device__ bool grid_barrier(unsigned* bar, unsigned nblocks, int* status) {
-  const unsigned gen = tc::ld_acquire_gpu(bar + 1);
-  if (tc::atom_add_acq_rel_gpu(bar, 1u) == nblocks - 1) {
-    atomicExch(bar, 0u);
-    tc::st_release_gpu(bar + 1, gen + 1);
-    return true;
-  }
-  const long long deadline = clock64() + (1ll << 32);
-  while (tc::ld_acquire_gpu(bar + 1) == gen) {
+// Grid-wide barrier n (1, 2, ...) of one launch, called by one thread per
+// CTA after a CTA barrier (all CTAs are co-resident).  bar[0] counts arrivals
+// over the whole launch: each CTA adds 1 with release semantics (publishing
+// what its threads wrote before the CTA barrier) and polls, bounded, until
+// the count reaches n * nblocks, then acquires.  No arriver has to reset or
+// publish anything, so the barrier costs one release-add and the polls.
+// bar[0] starts every launch at zero: grid_exit resets it.
+__device__ bool grid_barrier(unsigned* bar, unsigned target, int* status, long long limit) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(bar) : "memory");
+  const long long deadline = clock64() + limit;
+  for (;;) {
+    unsigned v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
+    if (v >= target) break;
     if (clock64() > deadline) {
       if (status) atomicExch(status, kStatusTimeout);
       return false;
     }
   }
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
   return true;
+}
+
+// Called once per CTA by the thread that polls the barrier, after its last
+// grid_barrier (or after giving up on one): the last CTA to get here resets
+// both words for the next launch on the same workspace.  Every CTA has then
+// finished polling bar[0].
+__device__ void grid_exit(unsigned* bar, unsigned nblocks) {
+  if (atomicAdd(bar + 1, 1u) == nblocks - 1) {
+    bar[0] = 0u;
+    bar[1] = 0u;
+  }
 }
 
 // Unit schedule of one CTA: its gate/up units u = c, c+G, ... over the
@@ -346,37 +360,50 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
   }
   if (!producer) {
     const int tid = threadIdx.x, nthr = kFWarps * 32;
-    for (int i = tid; i < T * (g.H / 8); i += nthr)
-      reinterpret_cast<uint4*>(xs)[i] = interleave8(__ldg(reinterpret_cast<const uint4*>(a.x) + i));
-    // router rows r = c, c + G, ...: warp w sums the K slice [w H/16, (w+1) H/16)
+    // router rows r = c, c + G, ...: thread tid owns the inputs [4 tid, 4 tid + 4)
+    // of every row and token.  x and the first rows are requested before any
+    // of them is used, so they arrive in one memory round trip; x is then
+    // staged from the same registers.
     const int nrows = (E1 - static_cast<int>(blockIdx.x) + gridDim.x - 1) / gridDim.x;
-    const int kslice = g.H / kFWarps;
+    const int c = 4 * tid;
+    const bool live = c < g.H;
+    uint2 xv[NT];
+#pragma unroll
+    for (int t = 0; t < NT; ++t)
+      xv[t] = (live && t < T) ? __ldg(reinterpret_cast<const uint2*>(a.x + static_cast<size_t>(t) * g.H + c))
+                              : make_uint2(0u, 0u);
     float* part = lg;   // [nrows][kFWarps][NT] partials (lg is free until phase B)
-    for (int rr = 0; rr < nrows; ++rr) {
-      const int row = blockIdx.x + rr * gridDim.x;
-      const uint16_t* wrow = row < E ? a.L.w_router + static_cast<size_t>(row) * g.H : a.L.w_sg;
-      float acc[NT];
+    for (int r0 = 0; r0 < nrows; r0 += kFRouterRows) {
+      uint2 wv[kFRouterRows];
 #pragma unroll
-      for (int t = 0; t < NT; ++t) acc[t] = 0.f;
-      for (int c = warp * kslice + lane * 4; c < (warp + 1) * kslice; c += 128) {
-        const uint2 wv = __ldg(reinterpret_cast<const uint2*>(wrow + c));
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {
-          if (t < T) {
-            const uint2 xv = __ldg(reinterpret_cast<const uint2*>(a.x + static_cast<size_t>(t) * g.H + c));
-            float s = acc[t];
-            s = fmaf(bf16_lo(xv.x), bf16_lo(wv.x), s);
-            s = fmaf(bf16_hi(xv.x), bf16_hi(wv.x), s);
-            s = fmaf(bf16_lo(xv.y), bf16_lo(wv.y), s);
-            s = fmaf(bf16_hi(xv.y), bf16_hi(wv.y), s);
-            acc[t] = s;
-          }
-        }
+      for (int q = 0; q < kFRouterRows; ++q) {
+        const int row = blockIdx.x + (r0 + q) * gridDim.x;
+        const uint16_t* wrow = row < E ? a.L.w_router + static_cast<size_t>(row) * g.H : a.L.w_sg;
+        wv[q] = (live && r0 + q < nrows) ? __ldg(reinterpret_cast<const uint2*>(wrow + c)) : make_uint2(0u, 0u);
       }
 #pragma unroll
-      for (int t = 0; t < NT; ++t) {
-        const float v = warp_sum(acc[t]);
-        if (lane == 0) part[(rr * kFWarps + warp) * NT + t] = v;
+      for (int q = 0; q < kFRouterRows; ++q) {
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          float s = fmaf(bf16_lo(xv[t].x), bf16_lo(wv[q].x), 0.f);
+          s = fmaf(bf16_hi(xv[t].x), bf16_hi(wv[q].x), s);
+          s = fmaf(bf16_lo(xv[t].y), bf16_lo(wv[q].y), s);
+          s = fmaf(bf16_hi(xv[t].y), bf16_hi(wv[q].y), s);
+          s = warp_sum(s);
+          if (lane == 0 && r0 + q < nrows && t < T) part[((r0 + q) * kFWarps + warp) * NT + t] = s;
+        }
+      }
+    }
+    // x in the interleaved K order: threads 2i, 2i+1 hold the halves of 8-group i
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      uint2 p;
+      p.x = __shfl_xor_sync(0xffffffffu, xv[t].x, 1);
+      p.y = __shfl_xor_sync(0xffffffffu, xv[t].y, 1);
+      if (live && t < T) {
+        const uint32_t lo = (tid & 1) ? p.y : xv[t].x, hi = (tid & 1) ? xv[t].y : p.x;
+        reinterpret_cast<uint2*>(xs + static_cast<size_t>(t) * g.H)[tid] =
+            make_uint2(__byte_perm(lo, hi, 0x5410), __byte_perm(lo, hi, 0x7632));
       }
     }
     consumers_sync();
@@ -401,7 +428,10 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
     }
   }
   __syncthreads();
-  if (threadIdx.x == 0 && !grid_barrier(a.bar, gridDim.x, a.status)) rt.abort = 1;
+  if (threadIdx.x == 0 && !grid_barrier(a.bar, gridDim.x, a.status, a.wait_limit)) {
+    rt.abort = 1;
+    grid_exit(a.bar, gridDim.x);
+  }
   __syncthreads();
   if (rt.abort) {
     if (producer && lane == 0 && early) tc::mbar_wait_drain(&full[0], 0, a.status);
@@ -463,7 +493,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
       if (early) last[0] = 0;
       for (int i = early ? 1 : 0; i < n_units; ++i) {
         const int sl = i % a.ring;
-        if (!tc::mbar_wait(&empty[sl], ((i / a.ring) & 1u) ^ 1u, abort_flag, a.status)) break;
+        if (!tc::mbar_wait(&empty[sl], ((i / a.ring) & 1u) ^ 1u, abort_flag, a.status, a.wait_limit)) break;
         tc::fence_proxy_async_smem();   // consumers' generic reads of the slot precede the refill
         issue_unit(a, rt, s, i, ring0 + sl * a.slot_bytes, &full[sl]);
         last[sl] = i;
@@ -491,7 +521,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
     const int ge = ngrp / 8;                       // groups per K eighth
     for (int i = 0; i < s.my_gu && ok; ++i) {
       const int sl = i % a.ring;
-      if (!tc::mbar_wait(&full[sl], (i / a.ring) & 1u, abort_flag, a.status)) {
+      if (!tc::mbar_wait(&full[sl], (i / a.ring) & 1u, abort_flag, a.status, a.wait_limit)) {
         ok = false;
         break;
       }
@@ -574,7 +604,10 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
   }
   // Every h row is written: grid barrier (consumer thread 0 of each CTA).
   consumers_sync();
-  if (threadIdx.x == 0 && (!ok || !grid_barrier(a.bar, gridDim.x, a.status))) rt.abort = 1;
+  if (threadIdx.x == 0) {
+    if (!ok || !grid_barrier(a.bar, 2u * gridDim.x, a.status, a.wait_limit)) rt.abort = 1;
+    grid_exit(a.bar, gridDim.x);
+  }
   consumers_sync();
   if (rt.abort) return;
 
@@ -619,7 +652,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
     for (int di = 0; di < s.my_blocks * s.n_down_parts && ok; ++di) {
       const int i = s.my_gu + di;
       const int sl = i % a.ring;
-      if (!tc::mbar_wait(&full[sl], (i / a.ring) & 1u, abort_flag, a.status)) {
+      if (!tc::mbar_wait(&full[sl], (i / a.ring) & 1u, abort_flag, a.status, a.wait_limit)) {
         ok = false;
         break;
       }
@@ -761,6 +794,7 @@ cudaError_t launch_decode_fused(const Geometry& g, const LayerPtr& L, const uint
   a.h_s = h_s;
   a.bar = bar;
   a.status = status;
+  a.wait_limit = wait_limit_cycles();
   const int G = fused_grid();
   const int Kmax = g.I > g.Is ? g.I : g.Is;
   a.slot_bytes = 18 * g.H;                                   // one gate/up unit

@@ -101,6 +101,7 @@ struct alignas(64) TcArgs {
   const int32_t* n_chunks;
   int* status;
   int scales_tma;          // scale rows are 16-B strided (K % 512 == 0): scales arrive by TMA
+  long long wait_limit;    // cycles before a bounded wait gives up
 };
 
 struct UnitInfo {
@@ -219,6 +220,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
   // the barrier set-up above touched only shared memory
   pdl_wait();
   pdl_launch_dependents();
+  // an error recorded in the status word (a bounded wait of this call's
+  // router, or of an earlier call, gave up) means the chunk list may not
+  // describe this call's tokens: do nothing (uniform over the CTA)
+  if (*reinterpret_cast<volatile const int*>(a.status) != 0) return;
   const int nfb = (kGateUp ? max(a.g.I, a.g.Is) : a.g.H) / BM;
   const int n_units = *a.n_chunks * nfb;
   const int Tk = a.g.T * a.g.k;
@@ -265,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
             tc::mbar_arrive(&empty_s[held_blk & 1u]);
           }
           held_blk = cur.blk;
-          if (!tc::mbar_wait(&full_s[held_blk & 1u], (held_blk >> 1) & 1u, abort_flag, a.status)) {
+          if (!tc::mbar_wait(&full_s[held_blk & 1u], (held_blk >> 1) & 1u, abort_flag, a.status, a.wait_limit)) {
             ok = false;
             break;
           }
@@ -282,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
       }
       // packed words of this stage's tile row
       const int sp = static_cast<int>(it % kPStages);
-      if (!tc::mbar_wait(&full_p[sp], (it / kPStages) & 1u, abort_flag, a.status)) {
+      if (!tc::mbar_wait(&full_p[sp], (it / kPStages) & 1u, abort_flag, a.status, a.wait_limit)) {
         ok = false;
         break;
       }
@@ -308,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
       tc::fence_proxy_async_smem();
       tc::mbar_arrive(&empty_p[sp]);
       const int sa = static_cast<int>(it % C::A_STAGES);
-      if (!tc::mbar_wait(&empty_a[sa], ((it / C::A_STAGES) & 1u) ^ 1u, abort_flag, a.status)) {
+      if (!tc::mbar_wait(&empty_a[sa], ((it / C::A_STAGES) & 1u) ^ 1u, abort_flag, a.status, a.wait_limit)) {
         ok = false;
         break;
       }
@@ -337,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
       const UnitInfo ui = unit_info<kGateUp>(a, u, nfb, units);
       if (ui.skip) continue;
       const int buf = static_cast<int>(tt % C::ACC_BUFS);
-      if (!tc::mbar_wait(&acc_full[buf], (tt / C::ACC_BUFS) & 1u, abort_flag, a.status)) break;
+      if (!tc::mbar_wait(&acc_full[buf], (tt / C::ACC_BUFS) & 1u, abort_flag, a.status, a.wait_limit)) break;
       tc::tc_fence_after();
       const uint32_t acc = lane_base + buf * C::ACC_COLS;
       for (int n0 = 0; n0 < ui.rows; n0 += 16) {
@@ -362,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
       tc::tc_fence_before();
       tc::mbar_arrive(&acc_empty[buf]);
       tc::mbar_arrive(&epi_sync[0]);
-      if (!tc::mbar_wait(&epi_sync[0], tt & 1u, abort_flag, a.status)) break;
+      if (!tc::mbar_wait(&epi_sync[0], tt & 1u, abort_flag, a.status, a.wait_limit)) break;
       // coalesced copy-out: each token row of the tile is BM contiguous outputs (256 B)
       const int chunks = ui.rows * (BM / 8);
       for (int i = et; i < chunks; i += 128) {
@@ -376,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
         *reinterpret_cast<uint4*>(dst + ui.f0 + c * 8) = *reinterpret_cast<const uint4*>(stage + n * BM + c * 8);
       }
       tc::mbar_arrive(&epi_sync[1]);                     // the staging tile is free again
-      if (!tc::mbar_wait(&epi_sync[1], tt & 1u, abort_flag, a.status)) break;
+      if (!tc::mbar_wait(&epi_sync[1], tt & 1u, abort_flag, a.status, a.wait_limit)) break;
       ++tt;
     }
   } else if (warp == kLoadWarp) {
@@ -393,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
         const int y = (!kGateUp && ui.shared) ? ui.row0 - Tk : ui.row0;
         for (int ks = 0; ks < ui.nks; ++ks, ++it) {
           const int s = static_cast<int>(it % kBStages);
-          if (!tc::mbar_wait(&empty_b[s], ((it / kBStages) & 1u) ^ 1u, abort_flag, a.status)) {
+          if (!tc::mbar_wait(&empty_b[s], ((it / kBStages) & 1u) ^ 1u, abort_flag, a.status, a.wait_limit)) {
             ok = false;
             break;
           }
@@ -401,6 +406,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
           tc::tma_load_2d(sbase + C::OFF_B + s * C::B_BYTES, tm, ks * BK, y, &full_b[s]);
         }
       }
+      // every tile this thread requested has landed before the CTA may exit
+      tc::drain_ring(full_b, kBStages, it, a.status);
     }
     __syncwarp();
   } else if (warp == kTmaWarp) {
@@ -409,13 +416,15 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
       StageCursor<kGateUp> cur;
       cur.begin(a, n_units, nfb, units);
       uint32_t last_blk = 0xffffffffu;
+      uint32_t p_fills = 0, s_fills = 0;   // packed-tile and scale-block fills issued
       while (!cur.done) {
         const int side = cur.ui.shared ? 1 : 0;
         if (a.scales_tma && cur.blk != last_blk) {
           last_blk = cur.blk;
           const int ss = static_cast<int>(cur.blk & 1u);
-          if (!tc::mbar_wait(&empty_s[ss], ((cur.blk >> 1) & 1u) ^ 1u, abort_flag, a.status)) break;
+          if (!tc::mbar_wait(&empty_s[ss], ((cur.blk >> 1) & 1u) ^ 1u, abort_flag, a.status, a.wait_limit)) break;
           tc::fence_proxy_async_smem();
+          ++s_fills;
           tc::mbar_arrive_expect_tx(&full_s[ss], C::S_SLOT);
           const uint32_t sdst = sbase + C::OFF_S + ss * C::S_SLOT;
 #pragma unroll
@@ -426,8 +435,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
           }
         }
         const int sp = static_cast<int>(cur.it % kPStages);
-        if (!tc::mbar_wait(&empty_p[sp], ((cur.it / kPStages) & 1u) ^ 1u, abort_flag, a.status)) break;
+        if (!tc::mbar_wait(&empty_p[sp], ((cur.it / kPStages) & 1u) ^ 1u, abort_flag, a.status, a.wait_limit)) break;
         tc::fence_proxy_async_smem();   // consumers' generic reads of the slot precede this async-proxy refill
+        ++p_fills;
         tc::mbar_arrive_expect_tx(&full_p[sp], C::NA * C::P_BYTES);
 #pragma unroll
         for (int mm = 0; mm < C::NA; ++mm)
@@ -435,6 +445,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
                           cur.ui.wrow, &full_p[sp]);
         cur.next(a, n_units, nfb);
       }
+      // every copy this thread requested has landed before the CTA may exit
+      tc::drain_ring(full_p, kPStages, p_fills, a.status);
+      tc::drain_ring(full_s, 2, s_fills, a.status);
     }
     __syncwarp();
   } else {
@@ -454,15 +467,15 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
       const int buf = static_cast<int>(tt % C::ACC_BUFS);
       // (every wait's outcome is made warp-uniform so the lanes leave together)
       if (!__all_sync(0xffffffffu, tc::mbar_wait(&acc_empty[buf], ((tt / C::ACC_BUFS) & 1u) ^ 1u, abort_flag,
-                                                 a.status)))
+                                                 a.status, a.wait_limit)))
         break;
       tc::tc_fence_after();
       const uint32_t acc = tmem + buf * C::ACC_COLS;
       for (int ks = 0; ks < ui.nks; ++ks, ++it) {
         const int sb = static_cast<int>(it % kBStages);
         const int sa = static_cast<int>(it % C::A_STAGES);
-        const bool got = tc::mbar_wait(&full_b[sb], (it / kBStages) & 1u, abort_flag, a.status) &&
-                         tc::mbar_wait(&full_a[sa], (it / C::A_STAGES) & 1u, abort_flag, a.status);
+        const bool got = tc::mbar_wait(&full_b[sb], (it / kBStages) & 1u, abort_flag, a.status, a.wait_limit) &&
+                         tc::mbar_wait(&full_a[sa], (it / C::A_STAGES) & 1u, abort_flag, a.status, a.wait_limit);
         if (!__all_sync(0xffffffffu, got)) {
           ok = false;
           break;
@@ -539,6 +552,7 @@ bool make_qmat_maps(TcArgs& a, int side, int m, const QMatPtr& W, int rows, int 
 
 }  // namespace
 
+static_assert(BN == kGemmChunkRows, "the chunk list and the GEMM tile must agree");
 int gemm_chunk_rows() { return BN; }
 
 cudaError_t launch_gateup(const Geometry& g, const LayerPtr& L, const uint16_t* xg, const Chunk* chunks,
@@ -555,6 +569,7 @@ cudaError_t launch_gateup(const Geometry& g, const LayerPtr& L, const uint16_t* 
   a.chunks = chunks;
   a.n_chunks = n_chunks;
   a.status = status;
+  a.wait_limit = wait_limit_cycles();
   a.scales_tma = (g.H % (kGroup * kSBlock)) == 0;
   const uint64_t rows = static_cast<uint64_t>(g.T) * g.k + g.T;
   if (!make_qmat_maps(a, 0, 0, L.gate, g.E * g.I, g.H) || !make_qmat_maps(a, 0, 1, L.up, g.E * g.I, g.H) ||
@@ -583,6 +598,7 @@ cudaError_t launch_down(const Geometry& g, const LayerPtr& L, const uint16_t* h,
   a.chunks = chunks;
   a.n_chunks = n_chunks;
   a.status = status;
+  a.wait_limit = wait_limit_cycles();
   a.scales_tma = (g.I % (kGroup * kSBlock)) == 0 && (g.Is % (kGroup * kSBlock)) == 0;
   if (!make_qmat_maps(a, 0, 0, L.down, g.E * g.H, g.I) || !make_qmat_maps(a, 1, 0, L.sh_down, g.H, g.Is) ||
       !make_map(&a.tm_h[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, g.I, static_cast<uint64_t>(g.T) * g.k, BK, BN,

@@ -64,6 +64,10 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
+// api.cu: SM clock cycles after which the kernels' bounded device-side waits
+// give up (moe_set_wait_limit; default tc::kDefaultWaitLimit, ~2 s).
+long long wait_limit_cycles();
+
 // api.cu: raise a kernel's dynamic shared-memory limit once per device (and
 // again only if a launch needs more), keeping the attribute call off the
 // per-launch path.
@@ -93,6 +97,9 @@ cudaError_t launch_group(const int32_t* topk_idx, int T, int k, int E, int chunk
                          int32_t* active, int32_t* n_active, cudaStream_t s);
 
 // gemm_tc.cu: tcgen05 grouped expert GEMMs over the device chunk list.
+// Rows per chunk of the chunk list (the GEMM tile's token count); moe.h states
+// moe_route_static's scratch limit with this value.
+constexpr int kGemmChunkRows = 128;
 int gemm_chunk_rows();
 // xg: the grouped token rows [T*k + T, H] (routed rows in expert order, then
 // the shared expert's T rows), each group of 8 in the interleaved K order.
@@ -107,10 +114,15 @@ cudaError_t launch_down(const Geometry& g, const LayerPtr& L, const uint16_t* h,
 // xg[R] = row perm[R] / k of x for R < T*k, row R - T*k for the shared
 // expert's rows, each group of 8 elements reordered (0,4,1,5,2,6,3,7): the
 // B operand of the gate/up GEMM in its grouped order and K order.
+// status: the call's status word; gather, combine and the grouped GEMMs do
+// nothing while it holds an error (their index inputs may then be unwritten).
 cudaError_t launch_gather_k8(const uint16_t* x, const int32_t* perm, int T, int k, int H, uint16_t* xg,
-                             cudaStream_t s);
+                             const int* status, cudaStream_t s);
+// out (may be NULL) = the layer output; norm_out (may be NULL) = RMSNorm(out)
+// with weight 1 and `eps`, the next stacked layer's input.
 cudaError_t launch_combine(const uint16_t* Y, const int32_t* inv_perm, const float* topk_w, const float* sigma,
-                           int T, int k, int H, uint16_t* out, cudaStream_t s);
+                           int T, int k, int H, uint16_t* out, uint16_t* norm_out, float eps, const int* status,
+                           cudaStream_t s);
 cudaError_t launch_rmsnorm(const uint16_t* y, uint16_t* out, int T, int H, float eps, cudaStream_t s);
 
 // decode.cu: T <= 64

@@ -228,7 +228,7 @@ RouterSplit router_split(int E) {
 __global__ void __launch_bounds__(kRThreads, 1) router_tc_kernel(
     const __grid_constant__ RouterMaps maps, const float* __restrict__ router_bias, int T, int H, int E, int k,
     int S, int C, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w, float* __restrict__ sigma,
-    int32_t* __restrict__ seg_counts, int* status) {
+    int32_t* __restrict__ seg_counts, int* status, long long wait_limit) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = tc::smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
@@ -285,15 +285,18 @@ __global__ void __launch_bounds__(kRThreads, 1) router_tc_kernel(
     // one thread streams the stages: x tile, this CTA's router rows, the gate row
     if (lane == 0) {
       const uint32_t tx = static_cast<uint32_t>(kA_BYTES + C * kRBK * 2 + (with_gate ? kRBK * 2 : 0));
-      for (int ks = 0; ks < nks; ++ks) {
+      int ks = 0;
+      for (; ks < nks; ++ks) {
         const int s = ks % kRStages;
-        if (!tc::mbar_wait(&empty[s], ((ks / kRStages) & 1) ^ 1, abort_flag, status)) break;
+        if (!tc::mbar_wait(&empty[s], ((ks / kRStages) & 1) ^ 1, abort_flag, status, wait_limit)) break;
         const uint32_t st = sbase + s * kSTAGE;
         tc::mbar_arrive_expect_tx(&full[s], tx);
         tc::tma_load_2d(st, &maps.x, ks * kRBK, t0, &full[s]);
         tc::tma_load_2d(st + kA_BYTES, &maps.w, ks * kRBK, e0, &full[s]);
         if (with_gate) tc::tma_load_2d(st + kA_BYTES + kB_BYTES, &maps.g, ks * kRBK, 0, &full[s]);
       }
+      // every stage this thread requested has landed before the CTA may exit
+      tc::drain_ring(full, kRStages, static_cast<uint32_t>(ks), status);
     }
     __syncwarp();
   } else if (warp < kREpiWarps) {
@@ -303,7 +306,7 @@ __global__ void __launch_bounds__(kRThreads, 1) router_tc_kernel(
     const int q = warp & 3, part = warp >> 2, tl = q * 32 + lane;
     const int quarter = ((C / 4) + 15) & ~15;
     const int c_lo = min(part * quarter, C), c_hi = min(c_lo + quarter, C);
-    const uint32_t got = tc::mbar_wait(acc_full, 0, abort_flag, status) ? 1u : 0u;
+    const uint32_t got = tc::mbar_wait(acc_full, 0, abort_flag, status, wait_limit) ? 1u : 0u;
     uint32_t all_got;   // the epilogue threads agree before any of them enters its barriers
     asm volatile("{\n\t.reg .pred p, r;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred r, 3, %2, p;\n\t"
                  "selp.u32 %0, 1, 0, r;\n\t}"
@@ -337,7 +340,7 @@ __global__ void __launch_bounds__(kRThreads, 1) router_tc_kernel(
       bool ok = true;
       for (int ks = 0; ks < nks; ++ks) {
         const int s = ks % kRStages;
-        if (!tc::mbar_wait(&full[s], (ks / kRStages) & 1, abort_flag, status)) {
+        if (!tc::mbar_wait(&full[s], (ks / kRStages) & 1, abort_flag, status, wait_limit)) {
           ok = false;
           break;
         }
@@ -434,7 +437,7 @@ cudaError_t launch_router(const uint16_t* x, const uint16_t* w_router, const flo
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, router_tc_kernel, maps, router_bias, T, H, E, k, sp.S, sp.C, topk_idx, topk_w,
-                            sigma, seg_counts, status);
+                            sigma, seg_counts, status, wait_limit_cycles());
 }
 
 }  // namespace moe

@@ -42,16 +42,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Default limit of a bounded wait, in SM clock cycles (~2 s at 1.9 GHz).
+// Waits that drain copies or tensor-core work already issued always use it.
+constexpr long long kDefaultWaitLimit = 1ll << 32;
+
 // Bounded wait for the phase with the given parity to complete.  Gives up
-// after ~2 s of device clock or as soon as another thread of the CTA has
-// given up (*abort != 0); on giving up it records the timeout in the status
-// word and raises *abort.  Returns false when it gave up.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* status) {
+// after `limit` cycles of device clock or as soon as another thread of the CTA
+// has given up (*abort != 0); on giving up it records the timeout in the
+// status word and raises *abort.  Returns false when it gave up.  Short limits
+// (failure-injection runs) are checked on every poll, the default one every
+// 256 polls.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* status,
+                                          long long limit = kDefaultWaitLimit) {
   if (mbar_try_wait(bar, parity)) return true;
-  const long long deadline = clock64() + (1ll << 32);
+  const long long deadline = clock64() + limit;
+  const uint32_t check_mask = limit < (1ll << 24) ? 0u : 255u;
   for (uint32_t n = 1;; ++n) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((n & 255u) == 0) {
+    if ((n & check_mask) == 0) {
       if (*abort) return false;
       if (clock64() > deadline) {
         *abort = 1;
@@ -63,9 +71,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 // Bounded wait that ignores the abort flag: used to drain in-flight tensor-core
-// work before tensor memory is released.
+// work or copies before tensor or shared memory is released.
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, int* status) {
-  const long long deadline = clock64() + (1ll << 32);
+  const long long deadline = clock64() + kDefaultWaitLimit;
   for (uint32_t n = 0;; ++n) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((n & 255u) == 255u && clock64() > deadline) {
@@ -73,6 +81,15 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, 
       return false;
     }
   }
+}
+
+// A producer that has issued fills 0 .. n-1 of an S-slot ring (fill i into
+// slot i % S, completing phase i / S of full[i % S]) waits until the last S of
+// them have landed.  On the normal path they were all consumed already and
+// this returns at once; after an abort it keeps the CTA from exiting (and its
+// shared memory from being reused) while an async copy into it is in flight.
+__device__ __forceinline__ void drain_ring(uint64_t* full, uint32_t S, uint32_t n, int* status) {
+  for (uint32_t i = n > S ? n - S : 0u; i < n; ++i) mbar_wait_drain(&full[i % S], (i / S) & 1u, status);
 }
 
 // -------------------------------------------------------------- cp.async --

@@ -25,7 +25,8 @@ MOE_ERR_DEVICE_TIMEOUT = -5
 
 # Every entry point declared in include/moe.h.
 EXPORTS = ("moe_workspace_size", "moe_route", "moe_forward", "moe_decode", "moe_forward_host", "moe_forward_host_async",
-           "moe_rmsnorm", "moe_forward_profiled", "moe_route_static", "moe_get_status", "moe_strerror")
+           "moe_forward_stack", "moe_rmsnorm", "moe_forward_profiled", "moe_route_static", "moe_get_status",
+           "moe_set_wait_limit", "moe_strerror")
 
 
 class QMatC(ctypes.Structure):
@@ -74,10 +75,12 @@ def library() -> ctypes.CDLL:
     lib.moe_forward_host.argtypes = [LP, P, I, P, P, S, P]
     lib.moe_forward_host_async.argtypes = [LP, P, I, P, P, S, P]
     lib.moe_rmsnorm.argtypes = [P, P, I, I, ctypes.c_float, P]
+    lib.moe_forward_stack.argtypes = [LP, I, P, I, P, P, ctypes.c_float, P, S, P]
     lib.moe_forward_profiled.argtypes = [LP, P, I, P, P, S, P, ctypes.POINTER(ctypes.c_float),
                                          ctypes.POINTER(ctypes.c_int)]
     lib.moe_route_static.argtypes = [LP, P, I, RP, P]
     lib.moe_get_status.argtypes = [P, P]
+    lib.moe_set_wait_limit.argtypes = [ctypes.c_longlong]
     lib.moe_strerror.argtypes = [I]
     lib.moe_strerror.restype = ctypes.c_char_p
     for name in EXPORTS:
@@ -237,6 +240,23 @@ def moe_forward_host_async(layer: MoELayer, x_host: torch.Tensor, out_host: torc
            "moe_forward_host_async")
 
 
+class LayerStack:
+    """A host array of layer descriptors for moe_forward_stack (keeps the layers' tensors alive)."""
+
+    def __init__(self, layers):
+        self.layers = list(layers)
+        self.array = (LayerC * len(self.layers))(*(L.desc for L in self.layers))
+
+
+def moe_forward_stack(stack: LayerStack, x: torch.Tensor, out: torch.Tensor, workspace: torch.Tensor,
+                      trace: torch.Tensor | None = None, eps: float = 1e-6, stream=None) -> None:
+    """len(stack.layers) layers joined by RMSNorm in one enqueued sequence (see include/moe.h)."""
+    T = x.shape[0]
+    _check(library().moe_forward_stack(stack.array, len(stack.layers), x.data_ptr(), T, out.data_ptr(),
+                                       _ptr(trace), float(eps), workspace.data_ptr(), workspace.numel(),
+                                       _stream(stream)), "moe_forward_stack")
+
+
 def moe_rmsnorm(y: torch.Tensor, y_out: torch.Tensor, eps: float = 1e-6, stream=None) -> None:
     T, H = y.shape
     _check(library().moe_rmsnorm(y.data_ptr(), y_out.data_ptr(), T, H, float(eps), _stream(stream)), "moe_rmsnorm")
@@ -260,5 +280,11 @@ def moe_forward_profiled(layer: MoELayer, x: torch.Tensor, out: torch.Tensor, wo
     return {names[i]: float(ms[i]) for i in range(n.value)}
 
 
-def moe_get_status(workspace: torch.Tensor, stream=None) -> int:
-    return int(library().moe_get_status(workspace.data_ptr(), _stream(stream)))
+def moe_get_status(workspace: torch.Tensor | None, stream=None) -> int:
+    """Status word of a workspace (None: of moe_route_static's static scratch); cleared when not MOE_OK."""
+    return int(library().moe_get_status(_ptr(workspace), _stream(stream)))
+
+
+def moe_set_wait_limit(cycles: int) -> None:
+    """SM clock cycles before the kernels' bounded waits give up (<= 0: the default, about 2 s)."""
+    _check(library().moe_set_wait_limit(int(cycles)), "moe_set_wait_limit")

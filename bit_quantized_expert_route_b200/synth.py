@@ -156,7 +156,7 @@ def make_layer_on_device(seed: int, layer: int, dims: Dims, device, zipf: bool =
         "router_bias": None,
     }
     if zipf:
-        out["router_bias"] = torch.from_numpy(zipf_router_bias(_rng(_KEY_W, seed, layer), d.E)).to(device)
+        out["router_bias"] = zipf_bias_on_device(seed, layer, d, device)
     out["gate"] = _dev_qmat(g, (d.E,), d.I, d.H, d.group, device)
     out["up"] = _dev_qmat(g, (d.E,), d.I, d.H, d.group, device)
     out["down"] = _dev_qmat(g, (d.E,), d.H, d.I, d.group, device)
@@ -165,6 +165,13 @@ def make_layer_on_device(seed: int, layer: int, dims: Dims, device, zipf: bool =
     out["sh_down"] = _dev_qmat(g, (), d.H, d.I_s, d.group, device)
     out["w_shared_gate"] = (torch.randn((d.H,), generator=g, device=device) * 0.02).to(torch.bfloat16)
     return out
+
+
+def zipf_bias_on_device(seed: int, layer: int, dims: Dims, device) -> torch.Tensor:
+    """The skewed workload's router bias of layer (seed, layer) as a float32 device tensor: the
+    same bias make_layer_on_device(..., zipf=True) adds, so a uniform layer's tensors plus this
+    bias form the skewed layer."""
+    return torch.from_numpy(zipf_router_bias(_rng(_KEY_W, seed, layer), dims.E)).to(device)
 
 
 def make_x_on_device(seed: int, T: int, H: int, device) -> torch.Tensor:

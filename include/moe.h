@@ -103,7 +103,15 @@ typedef struct {
  * "Perplexity Open Sources Apple Chip Inference Engine Lily", paragraph 3):
  *   bits == 4, group_size == 64, renorm == 1,
  *   1 <= k <= 8, k <= E <= 256,
- *   H a multiple of 128 and <= 8192; I and I_shared multiples of 128 and <= 2048. */
+ *   H a multiple of 128 and <= 8192; I and I_shared multiples of 128 and <= 2048.
+ * The layer the write-ups describe ("Perplexity's Lily: ...", section "The
+ * Model: Qwen3.6-35B-A3B in Focus": 256 experts, 8 chosen per token) has
+ * k = 8, E = 256, H = 2048 and I = I_shared = 512, so these bounds admit it
+ * and every size of its family.  They are narrower than "any k <= E, any
+ * multiple of the group size" on purpose: every weight tile of the expert
+ * GEMMs is 128 rows (one tensor-memory lane per row) and stays full, and each
+ * token's k candidates stay in registers through the top-k merges.  A layer
+ * outside them is refused on the host before anything is enqueued. */
 typedef struct {
   int H;            /* hidden size */
   int I;            /* routed expert intermediate size */
@@ -141,8 +149,13 @@ typedef struct {
 } moe_routing;
 
 /* Bytes of device workspace that moe_route / moe_forward / moe_decode /
- * moe_forward_host need for any T <= T_max.  Returns MOE_ERR_UNSUPPORTED or
- * MOE_ERR_INVALID_ARG for a layer or T_max the other calls would reject. */
+ * moe_forward_host / moe_forward_stack need for any T <= T_max.  The
+ * workspace holds the routing buffers the GPU builds for itself (histogram,
+ * prefix sums, permutation and the tile list of the grouped GEMMs: "Perplexity's
+ * Lily: ...", section "How It Works: Prefill and Decode Strategies", which
+ * keeps them on the device with no CPU synchronisation) and the experts'
+ * intermediate rows.  Returns MOE_ERR_UNSUPPORTED or MOE_ERR_INVALID_ARG for
+ * a layer or T_max the other calls would reject. */
 MOE_API int moe_workspace_size(const moe_layer_desc* layer, int T_max, size_t* bytes);
 
 /* Router logits, softmax top-k with renormalisation, shared gate, and the
@@ -154,8 +167,13 @@ MOE_API int moe_route(const moe_layer_desc* layer, const moe_bf16* x, int T, moe
 
 /* The whole layer: routing, fused-dequant gate/up grouped GEMM with the
  * SwiGLU epilogue, down-projection grouped GEMM, shared expert, and the
- * fixed-order gather-combine.  x, out: device bf16 [T, H], 16-byte aligned,
- * not overlapping.  r: optional (NULL = keep routing in the workspace).
+ * fixed-order gather-combine.  The write-ups ("Perplexity's Lily: ...",
+ * sections "The Model: Qwen3.6-35B-A3B in Focus" and "How It Works: Prefill
+ * and Decode Strategies") describe this layer: routed experts chosen on the
+ * GPU, their 4-bit weights rebuilt tile by tile inside the grouped GEMM with
+ * bf16 products and FP32 accumulation, and one always-on shared expert.
+ * x, out: device bf16 [T, H], 16-byte aligned, not overlapping.
+ * r: optional (NULL = keep routing in the workspace).
  * 1 <= T <= 65536; T <= 64 runs the decode kernels of moe_decode. */
 MOE_API int moe_forward(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_bf16* out,
                 moe_routing* r, void* workspace, size_t workspace_bytes, moe_stream stream);
@@ -169,28 +187,59 @@ MOE_API int moe_forward(const moe_layer_desc* layer, const moe_bf16* x, int T, m
 MOE_API int moe_decode(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_bf16* out,
                moe_routing* r, void* workspace, size_t workspace_bytes, moe_stream stream);
 
+/* A stack of MoE layers joined by RMSNorm, enqueued on one stream with no
+ * host synchronisation between layers ("Perplexity's Lily: ...", section "How
+ * It Works: Prefill and Decode Strategies": the layers of a forward pass are
+ * recorded into one GPU submission with no CPU round trip), so the whole call
+ * can also be captured once as a CUDA graph and replayed:
+ *   a_0 = x;  y_l = layer_l(a_l);  a_{l+1} = bf16(y_l / sqrt(mean(y_l^2) + eps))
+ * (RMSNorm with weight 1 and no residual, over the bf16 values of y_l);
+ * out = y_{n_layers-1}.  For T > 64 the RMSNorm is computed inside the
+ * layer's combine kernel (the row's sum of squares is formed while its output
+ * is written); for T <= 64 it is a separate small kernel.
+ *   layers: host array of n_layers (1..1024) descriptors with equal H, I,
+ *           I_shared, E and k.
+ *   x, out: device bf16 [T, H], 16-byte aligned, not overlapping.
+ *   trace:  NULL, or device bf16 [n_layers][2][T][H] that receives a_l in
+ *           trace[l][0] and y_l in trace[l][1] (for debugging and tests).
+ *   workspace: as for moe_forward with the same T (moe_workspace_size); the
+ *           activations between layers live in it.
+ * Validation covers every layer before anything is enqueued. */
+MOE_API int moe_forward_stack(const moe_layer_desc* layers, int n_layers, const moe_bf16* x, int T, moe_bf16* out,
+                              moe_bf16* trace, float eps, void* workspace, size_t workspace_bytes,
+                              moe_stream stream);
+
 /* moe_route for callers that cannot allocate device memory.  The pages have
  * no counterpart to this entry point; it exists for hosts that hand the
  * library only the tensors it reads and writes -- a plug-in inside another
  * runtime that exposes no allocator, or a serving loop with a fixed memory
  * plan where a cudaMalloc (which may also synchronise the device) is not
- * allowed.  It computes exactly what moe_route computes, with the same
- * kernels, but takes no workspace: its scratch (per-segment expert counts,
- * the chunk list, the active-expert list, and sigma when r->sigma is NULL)
- * lives in one static device array of 512 KiB inside libmoe.so, which every
- * GPU that loads the library holds until the process exits.
- *   Limit: the call needs ceil(T/128)*E*4 bytes of counts, plus
- *   (T*k/128 + T/128 + E + 2)*16 bytes of chunk list, plus (E+1)*4 + 2*4
- *   bytes, plus T*4 bytes if r->sigma is NULL, each rounded up to 256 bytes;
- *   a call whose need exceeds 512 KiB returns MOE_ERR_WORKSPACE and enqueues
- *   nothing (for E=256, k=8 this admits T <= 56704 when r->sigma is given,
- *   T <= 39424 when it is NULL).
+ * allowed.  It runs the same kernels as moe_route for the same T (T <= 64:
+ * the one-launch small-T router; larger T: the tensor-core router and the
+ * counting-sort passes), so its outputs are those of moe_route, but it takes
+ * no workspace: its scratch (a 256-byte control block with a status word,
+ * then for T <= 64 the T x (E+1) logits, otherwise the per-segment expert
+ * counts and the chunk list; the active-expert list; and sigma when r->sigma
+ * is NULL) lives in one static device array of 512 KiB inside libmoe.so,
+ * which every GPU that loads the library holds until the process exits.
+ *   Limit: the call needs 256 bytes of control block, plus for T <= 64
+ *   T*(E+1)*4 bytes of logits, or for T > 64 ceil(T/128)*E*4 bytes of counts
+ *   and (T*k/128 + T/128 + E + 2)*16 + 4 bytes of chunk list, plus
+ *   (E+1)*4 + 4 bytes of active list, plus T*4 bytes if r->sigma is NULL,
+ *   each piece rounded up to 256 bytes; a call whose need exceeds 512 KiB
+ *   returns MOE_ERR_WORKSPACE and enqueues nothing (for E=256, k=8 this
+ *   admits T <= 56704 when r->sigma is given, T <= 39424 when it is NULL).
  *   Set-up: the first call on each device looks up the array's device
  *   address with cudaGetSymbolAddress while that device is current, so make
  *   that first call before any stream capture on that device.
- *   Sharing: all calls in the process use the same array and nothing in it
- *   needs to start at zero (every call rewrites what it reads); two calls
- *   whose GPU work overlaps (different streams, or host threads) race on it.
+ *   Sharing: all calls in the process use the same array.  Its control block
+ *   starts at zero (static storage) and every call leaves it zero except for
+ *   a recorded error status; nothing else in it needs to start at zero
+ *   (every call rewrites what it reads).  Two calls whose GPU work overlaps
+ *   (different streams, or host threads) race on it.
+ *   Errors: a bounded device-side wait that gives up records
+ *   MOE_ERR_DEVICE_TIMEOUT in the array's status word; moe_get_status(NULL,
+ *   stream) returns it (and clears the control block).
  * Allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
  * Arguments as for moe_route, minus the workspace; r is required. */
 MOE_API int moe_route_static(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_routing* r,
@@ -231,8 +280,23 @@ MOE_API int moe_forward_profiled(const moe_layer_desc* layer, const moe_bf16* x,
                                  float* stage_ms, int* n_stages);
 
 /* Waits for `stream`, returns the status word kept in `workspace` (MOE_OK or
- * MOE_ERR_DEVICE_TIMEOUT) and clears it.  MOE_ERR_CUDA if the wait fails. */
+ * MOE_ERR_DEVICE_TIMEOUT) and, when it is not MOE_OK, clears the control
+ * block.  workspace == NULL reads the status word of moe_route_static's
+ * static scratch on the current device instead.  MOE_ERR_CUDA if the wait
+ * fails; MOE_ERR_WORKSPACE if workspace is not 256-byte aligned. */
 MOE_API int moe_get_status(void* workspace, moe_stream stream);
+
+/* Failure detection control: the kernels' bounded device-side waits (on
+ * mbarriers and grid barriers) give up after `cycles` SM clock cycles and
+ * record MOE_ERR_DEVICE_TIMEOUT (cycles <= 0 restores the default, 2^32 cycles,
+ * about 2 s).  Process-wide; it applies to kernels enqueued after the call.
+ * Waits that drain copies or tensor-core work a kernel has already issued keep
+ * the default, so a kernel that gives up never exits with a copy into its
+ * shared memory in flight.  A short limit exists to test the error path: a
+ * call whose waits give up leaves its outputs unwritten (kernels that would
+ * read unwritten routing indices do nothing while the status word holds an
+ * error) and reports the timeout through moe_get_status. */
+MOE_API int moe_set_wait_limit(long long cycles);
 
 /* Static description of a status code. */
 MOE_API const char* moe_strerror(int status);

@@ -85,6 +85,21 @@ def test_layer_validation(lib, over, code):
     assert st == code
 
 
+# The documented edges of the accepted layout (include/moe.h, moe_layer_desc):
+# 1 <= k <= 8, k <= E <= 256, H a multiple of 128 up to 8192, I and I_shared
+# multiples of 128 up to 2048.  Multiples of the group size (64) that are not
+# multiples of 128 are refused on purpose (full 128-row weight tiles).
+@pytest.mark.parametrize("over,code", [
+    (dict(k=1, E=1), 0), (dict(k=8, E=8), 0), (dict(k=8, E=256), 0), (dict(E=257), moe.MOE_ERR_UNSUPPORTED),
+    (dict(H=128), 0), (dict(H=8192), 0), (dict(H=8320), moe.MOE_ERR_UNSUPPORTED),
+    (dict(H=192), moe.MOE_ERR_UNSUPPORTED), (dict(H=64), moe.MOE_ERR_UNSUPPORTED),
+    (dict(I=128), 0), (dict(I=2048), 0), (dict(I=2176), moe.MOE_ERR_UNSUPPORTED), (dict(I=192), moe.MOE_ERR_UNSUPPORTED),
+    (dict(I_shared=128), 0), (dict(I_shared=2048), 0), (dict(I_shared=320), moe.MOE_ERR_UNSUPPORTED),
+])
+def test_documented_layout_edges(lib, over, code):
+    assert ws_size(lib, fake_layer(**over), 16)[0] == code
+
+
 def test_null_and_misaligned_pointers(lib):
     L = fake_layer()
     L.gate = moe.QMatC(FAKE, None, FAKE)
@@ -122,7 +137,11 @@ def test_calls_reject_before_launch(lib):
     assert lib.moe_forward_host_async(ctypes.byref(L), FAKE, 16, out, FAKE, 16, None) == moe.MOE_ERR_WORKSPACE
     assert lib.moe_rmsnorm(FAKE, FAKE, 0, 2048, ctypes.c_float(1e-6), None) == moe.MOE_ERR_INVALID_ARG
     assert lib.moe_rmsnorm(FAKE, FAKE + 4, 4, 2048, ctypes.c_float(1e-6), None) == moe.MOE_ERR_INVALID_ARG
-    assert lib.moe_get_status(None, None) == moe.MOE_ERR_WORKSPACE
+    assert lib.moe_get_status(FAKE + 16, None) == moe.MOE_ERR_WORKSPACE
+    # NULL reads moe_route_static's status word: with no CUDA device the lookup itself fails
+    import torch
+    if not torch.cuda.is_available():
+        assert lib.moe_get_status(None, None) == moe.MOE_ERR_CUDA
 
 
 def test_library_is_built_for_sm100a():
@@ -131,10 +150,15 @@ def test_library_is_built_for_sm100a():
     assert os.path.exists(moe_build.LIB)
 
 
-def _static_route_need(T, E, k, sigma_given):
+def _static_route_need(T, E, k, sigma_given, chunk=128):
     """Scratch bytes of moe_route_static as moe.h states them (each piece rounded to 256 B)."""
     r = lambda b: (b + 255) // 256 * 256
-    n = r(-(-T // 128) * E * 4) + r((T * k // 128 + T // 128 + E + 2) * 16) + r(4) + r((E + 1) * 4) + r(4)
+    n = 256
+    if T <= 64:
+        n += r(T * (E + 1) * 4)
+    else:
+        n += r(-(-T // chunk) * E * 4) + r((T * k // chunk + T // chunk + E + 2) * 16) + r(4)
+    n += r((E + 1) * 4) + r(4)
     return n + (0 if sigma_given else r(T * 4))
 
 

@@ -134,3 +134,87 @@ def test_stack_40_layers_gpu_properties(T):
     assert np.all(np.isfinite(moe_ref.bf16_to_f64(a_bits)))
     # bf16 rounding of a unit-RMS row moves its RMS by well under 1%
     assert np.all(np.abs(a_rms - 1.0) < 1e-2), a_rms
+
+
+# ------------------------------------------------------- moe_forward_stack --
+
+def _rmsnorm_f64_bits(y_bits: np.ndarray, eps: float = 1e-6) -> np.ndarray:
+    """bf16(y / sqrt(mean(y^2) + eps)) of bf16 rows in float64 (torch), as bf16 bits: the
+    normalisation identity the stack's fused RMSNorm must satisfy on its own output."""
+    y = torch.from_numpy(moe_ref.bf16_to_f64(y_bits))
+    v = y / torch.sqrt((y * y).mean(dim=1, keepdim=True) + eps)
+    return v.to(torch.float32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def _ulp_distance(a: np.ndarray, b: np.ndarray) -> np.ndarray:
+    """Distance in bf16 units in the last place between two arrays of finite bf16 bit patterns."""
+    def ordered(u):
+        u = u.astype(np.int32)
+        return np.where(u & 0x8000, 0x8000 - (u & 0x7FFF), 0x8000 + u)
+    return np.abs(ordered(a) - ordered(b))
+
+
+@pytest.mark.parametrize("T,n_layers", [(1, 4), (8, 3), (64, 3), (65, 2), (512, 3)])
+def test_forward_stack_matches_single_layer_calls(T, n_layers):
+    """moe_forward_stack vs the per-layer entry points on the stack's own activations: every
+    layer's output is bit-identical to moe_forward on the same input (same kernels), and every
+    next input is the RMSNorm of that output (float64 identity within one bf16 ulp, and within
+    one ulp of the stand-alone moe_rmsnorm).  The per-layer path itself is held to the oracle by
+    test_stack_layer_by_layer."""
+    dev = torch.device("cuda", 0)
+    layers = [moe.MoELayer.from_tensors(FULL, synth.make_layer_on_device(300 + T, l, FULL, dev, l % 2 == 1))
+              for l in range(n_layers)]
+    stack = moe.LayerStack(layers)
+    x = synth.make_x_on_device(310 + T, T, FULL.H, dev)
+    out = torch.empty_like(x)
+    ws = moe.alloc_workspace(layers[0], T, dev)
+    trace = torch.empty((n_layers, 2, T, FULL.H), dtype=torch.bfloat16, device=dev)
+    moe.moe_forward_stack(stack, x, out, ws, trace=trace)
+    torch.cuda.synchronize()
+    assert moe.moe_get_status(ws) == 0
+    assert torch.equal(trace[0, 0], x)
+    assert torch.equal(trace[-1, 1], out)
+    ws1 = moe.alloc_workspace(layers[0], T, dev)
+    for l, L in enumerate(layers):
+        y = torch.empty_like(x)
+        moe.moe_forward(L, trace[l, 0].contiguous(), y, ws1)
+        torch.cuda.synchronize()
+        assert torch.equal(y, trace[l, 1]), f"layer {l}: stack output differs from moe_forward"
+        if l + 1 < n_layers:
+            got = bits_of(trace[l + 1, 0])
+            assert int(_ulp_distance(got, _rmsnorm_f64_bits(bits_of(trace[l, 1]))).max()) <= 1
+            ref = torch.empty_like(x)
+            moe.moe_rmsnorm(trace[l, 1].contiguous(), ref, 1e-6)
+            torch.cuda.synchronize()
+            assert int(_ulp_distance(got, bits_of(ref)).max()) <= 1
+    assert moe.moe_get_status(ws1) == 0
+
+
+@pytest.mark.parametrize("T", [1, 4096])
+def test_forward_stack_graph_replay_is_bitwise_repeatable(T):
+    """The whole stack captured once as a CUDA graph and replayed gives the stream-launched result."""
+    dev = torch.device("cuda", 0)
+    n_layers = 6
+    layers = [moe.MoELayer.from_tensors(FULL, synth.make_layer_on_device(400 + T, l, FULL, dev, False))
+              for l in range(n_layers)]
+    stack = moe.LayerStack(layers)
+    x = synth.make_x_on_device(410 + T, T, FULL.H, dev)
+    ws = moe.alloc_workspace(layers[0], T, dev)
+    want = torch.empty_like(x)
+    moe.moe_forward_stack(stack, x, want, ws)
+    torch.cuda.synchronize()
+    got = torch.empty_like(x)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            moe.moe_forward_stack(stack, x, got, ws, stream=s)
+    torch.cuda.synchronize()
+    for _ in range(2):
+        got.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(got, want)
+    del g
+    assert moe.moe_get_status(ws) == 0

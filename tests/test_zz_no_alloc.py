@@ -5,9 +5,12 @@ inside another runtime with no allocator to offer, a serving loop whose memory
 plan forbids a cudaMalloc and the device synchronisation it can cause).  For
 them moe_route_static keeps its scratch in a static device array inside
 libmoe.so instead of a caller workspace.  This file checks, through the C ABI,
-that two calls in a row give what moe_route gives, and that a call needing
-more than the array holds is refused before anything is enqueued.  It is named
-to run last so that a failure here cannot hide any other test's result.
+that two calls in a row give what moe_route gives, that its routing matches
+the CPU oracle on both sides of T = 64 (where moe_route, and so this entry
+point, switches from the one-launch small-T router to the tensor-core router),
+that its status word reads back as MOE_OK, and that a call needing more than
+the array holds is refused before anything is enqueued.  It is named to run
+last so that a failure here cannot hide any other test's result.
 """
 from __future__ import annotations
 
@@ -18,7 +21,8 @@ import pytest
 import torch
 
 from bit_quantized_expert_route_b200 import moe
-from tests.gpu_util import require_cuda, to_dev_bits
+from oracle import moe_ref
+from tests.gpu_util import assert_routing_exact, require_cuda, to_dev_bits
 from tests.workloads import FULL, TINY, workload
 
 pytestmark = pytest.mark.gpu
@@ -54,6 +58,25 @@ def test_static_route_matches_route_on_two_calls(dims, T, seeds):
             np.testing.assert_array_equal(got[f], want[f])
         np.testing.assert_allclose(got["topk_w"], want["topk_w"], rtol=0, atol=2e-6)
         np.testing.assert_allclose(got["sigma"], want["sigma"], rtol=0, atol=2e-6)
+
+
+@pytest.mark.parametrize("T", [1, 5, 64, 65, 300, 4096])
+def test_static_route_matches_oracle(T):
+    """Both routers behind the entry point (T <= 64 and T > 64) against the oracle, bit for bit."""
+    require_cuda()
+    lay, x, _ = workload(50 + T % 7, T, FULL)
+    L = moe.MoELayer.from_synth(lay)
+    got = _route(L, x, static=True)
+    assert moe.moe_get_status(None) == moe.MOE_OK
+    ref = moe_ref.route(x, lay, FULL.k)
+    gpu = {
+        "topk_idx": got["topk_idx"].reshape(T, FULL.k).astype(np.int64),
+        "topk_w": got["topk_w"].reshape(T, FULL.k).astype(np.float64),
+        "counts": got["counts"].astype(np.int64), "offsets": got["offsets"].astype(np.int64),
+        "perm": got["perm"].astype(np.int64), "inv_perm": got["inv_perm"].astype(np.int64),
+        "sigma": got["sigma"].astype(np.float64),
+    }
+    assert_routing_exact(gpu, ref)
 
 
 def test_static_route_without_sigma_output():
