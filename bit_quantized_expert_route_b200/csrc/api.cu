@@ -63,6 +63,7 @@ namespace {
 using namespace moe;
 
 constexpr int kDecodeMaxT = 64;
+constexpr int kFusedMaxT = 8;       // tokens the fused decode kernel takes
 constexpr int kMaxT = 65536;
 constexpr int kMaxStackLayers = 1024;
 constexpr size_t kAlign = 256;
@@ -74,7 +75,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // Byte offsets of every workspace buffer for a call with T tokens.
 struct WsLayout {
   size_t status, counter, grid_bar, topk_idx, topk_w, counts, offsets, perm, inv_perm, sigma, seg, chunks, n_chunks,
-      active, n_active, logits, h, h_s, Y, x_stage, out_stage, total;
+      active, n_active, logits, h, h_s, Y, x_stage, out_stage, dec_y, dec_sumsq, total;
   int max_chunks;
 };
 
@@ -110,6 +111,10 @@ WsLayout ws_layout(const moe_layer_desc* d, int T) {
   w.Y = take((n + T) * d->H * 2);   // also holds the gate/up GEMM's grouped token rows before the down GEMM
   w.x_stage = take(static_cast<size_t>(T) * d->H * 2);
   w.out_stage = take(static_cast<size_t>(T) * d->H * 2);
+  // the fused decode kernel's outputs between stacked layers and the CTAs'
+  // partial sums of their squares
+  w.dec_y = take(static_cast<size_t>(T <= kFusedMaxT ? T : 0) * d->H * 2);
+  w.dec_sumsq = take(static_cast<size_t>(T <= kFusedMaxT ? kFusedMaxGrid * 8 : 0) * 4);
   w.total = off;
   return w;
 }
@@ -198,10 +203,14 @@ inline void mark(Tracer* tr, cudaStream_t s) {
   if (tr) tr->mark(s);
 }
 
+// Routing of T tokens.  T <= 64 without `grouped`: one launch of the small-T
+// router (routing outputs and active list only).  Otherwise the tensor-core
+// router and the counting-sort passes, which also build the chunk list the
+// grouped GEMMs walk.
 int enqueue_route(const moe_layer_desc* d, const uint16_t* x, int T, const Bufs& b, cudaStream_t s,
-                  Tracer* tr = nullptr) {
+                  Tracer* tr = nullptr, bool grouped = false) {
   mark(tr, s);
-  if (T <= kDecodeMaxT) {
+  if (T <= kDecodeMaxT && !grouped) {
     const RoutingPtrs rp{b.topk_idx, b.topk_w, b.sigma, b.counts, b.offsets, b.perm, b.inv_perm};
     const cudaError_t e = launch_route_small(x, layer_ptrs(d), T, d->H, d->I, d->I_shared, d->E, d->k,
                                              b.at<float>(b.w.logits), b.at<unsigned>(b.w.counter), rp,
@@ -220,6 +229,20 @@ int enqueue_route(const moe_layer_desc* d, const uint16_t* x, int T, const Bufs&
   return cuda_status(e);
 }
 
+// n_layers (<= decode_fused_max_layers()) layers of one geometry through the
+// fused decode kernel; with_routing: the last layer's routing goes to b's
+// routing buffers.
+cudaError_t launch_fused_layers(const Geometry& g, const LayerPtr* layers, int n_layers, const uint16_t* x,
+                                uint16_t* out, uint16_t* trace, float eps, const Bufs& b, bool with_routing,
+                                cudaStream_t s) {
+  RoutingPtrs rp{b.topk_idx, b.topk_w, b.sigma, b.counts, b.offsets, b.perm, b.inv_perm};
+  if (!with_routing) rp = RoutingPtrs{};
+  return launch_decode_fused(g, layers, n_layers, x, out, b.at<uint16_t>(b.w.dec_y), b.at<float>(b.w.dec_sumsq),
+                             trace, eps, rp, b.at<int32_t>(b.w.active), b.at<int32_t>(b.w.n_active),
+                             b.at<float>(b.w.logits), b.at<uint16_t>(b.w.h), b.at<uint16_t>(b.w.h_s),
+                             b.at<unsigned>(b.w.grid_bar), b.at<int>(b.w.status), s);
+}
+
 // Bulk copies of whole scale/bias tile rows need 16-byte aligned stacks.
 bool fused_decode_ok(const moe_layer_desc* d, const Geometry& g) {
   const moe_qmat* m[6] = {&d->gate, &d->up, &d->down, &d->sh_gate, &d->sh_up, &d->sh_down};
@@ -228,17 +251,23 @@ bool fused_decode_ok(const moe_layer_desc* d, const Geometry& g) {
   return decode_fused_supported(g);
 }
 
+// moe_forward's choice for T tokens: the single-launch fused decode kernel
+// where it applies, else the tensor-core path.  (The GEMV kernels of
+// moe_decode do FP32 work per weight and token, which the tensor cores
+// outrun as soon as an expert sees more than a couple of tokens.)
+bool forward_uses_fused_decode(const moe_layer_desc* d, int T) {
+  const Geometry g{T, d->H, d->I, d->I_shared, d->E, d->k};
+  return T <= kFusedMaxT && fused_decode_ok(d, g);
+}
+
 int enqueue_decode(const moe_layer_desc* d, const uint16_t* x, int T, uint16_t* out, const Bufs& b,
                    cudaStream_t s, Tracer* tr = nullptr) {
   {
     const Geometry g{T, d->H, d->I, d->I_shared, d->E, d->k};
     if (fused_decode_ok(d, g)) {
       mark(tr, s);
-      const RoutingPtrs rp{b.topk_idx, b.topk_w, b.sigma, b.counts, b.offsets, b.perm, b.inv_perm};
-      const cudaError_t e = launch_decode_fused(
-          g, layer_ptrs(d), x, out, rp, b.at<int32_t>(b.w.active), b.at<int32_t>(b.w.n_active),
-          b.at<float>(b.w.logits), b.at<uint16_t>(b.w.h), b.at<uint16_t>(b.w.h_s), b.at<unsigned>(b.w.grid_bar),
-          b.at<int>(b.w.status), s);
+      const LayerPtr L = layer_ptrs(d);
+      const cudaError_t e = launch_fused_layers(g, &L, 1, x, out, nullptr, 0.f, b, true, s);
       mark(tr, s);
       return cuda_status(e);
     }
@@ -262,7 +291,7 @@ int enqueue_decode(const moe_layer_desc* d, const uint16_t* x, int T, uint16_t* 
 // be NULL): RMSNorm(out) with weight 1 and eps, fused into the combine.
 int enqueue_prefill(const moe_layer_desc* d, const uint16_t* x, int T, uint16_t* out, const Bufs& b,
                     cudaStream_t s, Tracer* tr = nullptr, uint16_t* norm_out = nullptr, float eps = 0.f) {
-  int st = enqueue_route(d, x, T, b, s, tr);
+  int st = enqueue_route(d, x, T, b, s, tr, /*grouped=*/true);
   if (st != MOE_OK) return st;
   const Geometry g{T, d->H, d->I, d->I_shared, d->E, d->k};
   const LayerPtr L = layer_ptrs(d);
@@ -291,7 +320,7 @@ int enqueue_prefill(const moe_layer_desc* d, const uint16_t* x, int T, uint16_t*
 // norm_out (may be NULL) its RMSNorm, the next layer's input.
 int enqueue_layer(const moe_layer_desc* d, const uint16_t* x, int T, uint16_t* out, uint16_t* norm_out, float eps,
                   const Bufs& b, cudaStream_t s) {
-  if (T > kDecodeMaxT) return enqueue_prefill(d, x, T, out, b, s, nullptr, norm_out, eps);
+  if (!forward_uses_fused_decode(d, T)) return enqueue_prefill(d, x, T, out, b, s, nullptr, norm_out, eps);
   uint16_t* y = out ? out : norm_out;
   const int st = enqueue_decode(d, x, T, y, b, s);
   if (st != MOE_OK || !norm_out) return st;
@@ -405,7 +434,7 @@ int moe_forward(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_bf16*
   if (st != MOE_OK) return st;
   const Bufs b = resolve(layer, T, ws, r);
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (T <= kDecodeMaxT) return enqueue_decode(layer, x, T, out, b, s);
+  if (forward_uses_fused_decode(layer, T)) return enqueue_decode(layer, x, T, out, b, s);
   return enqueue_prefill(layer, x, T, out, b, s);
 }
 
@@ -433,6 +462,29 @@ int moe_forward_stack(const moe_layer_desc* layers, int n_layers, const moe_bf16
   const Bufs b0 = resolve(&layers[0], T, ws, nullptr);
   uint16_t* pingpong[2] = {b0.at<uint16_t>(b0.w.x_stage), b0.at<uint16_t>(b0.w.out_stage)};
   uint16_t* tr = reinterpret_cast<uint16_t*>(trace);
+  bool fused = true;
+  for (int l = 0; l < n_layers; ++l) fused = fused && forward_uses_fused_decode(&layers[l], T);
+  if (fused) {
+    // whole chunks of layers per launch of the fused decode kernel, which
+    // applies the RMSNorm between its layers itself and writes the trace
+    const moe_layer_desc& d0 = layers[0];
+    const Geometry g{T, d0.H, d0.I, d0.I_shared, d0.E, d0.k};
+    const int chunk = decode_fused_max_layers();
+    LayerPtr lp[kMaxStackLayers];
+    for (int l = 0; l < n_layers; ++l) lp[l] = layer_ptrs(&layers[l]);
+    const uint16_t* xin = x;
+    for (int l0 = 0, c = 0; l0 < n_layers; l0 += chunk, ++c) {
+      const int nl = n_layers - l0 < chunk ? n_layers - l0 : chunk;
+      const bool last = l0 + nl == n_layers;
+      uint16_t* cout = last ? out : pingpong[c & 1];
+      if (launch_fused_layers(g, lp + l0, nl, xin, cout, tr ? tr + 2 * l0 * act : nullptr, eps, b0, false, s) !=
+          cudaSuccess)
+        return MOE_ERR_CUDA;
+      if (!last && launch_rmsnorm(cout, cout, T, d0.H, eps, s) != cudaSuccess) return MOE_ERR_CUDA;
+      xin = cout;
+    }
+    return MOE_OK;
+  }
   if (tr && cudaMemcpyAsync(tr, x, act * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess) return MOE_ERR_CUDA;
   const uint16_t* xin = x;
   for (int l = 0; l < n_layers; ++l) {
@@ -495,7 +547,7 @@ static int forward_host_enqueue(const moe_layer_desc* layer, const moe_bf16* x_h
   uint16_t* od = b.at<uint16_t>(b.w.out_stage);
   const size_t bytes = static_cast<size_t>(T) * layer->H * sizeof(uint16_t);
   if (cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return MOE_ERR_CUDA;
-  st = (T <= kDecodeMaxT) ? enqueue_decode(layer, xd, T, od, b, s) : enqueue_prefill(layer, xd, T, od, b, s);
+  st = forward_uses_fused_decode(layer, T) ? enqueue_decode(layer, xd, T, od, b, s) : enqueue_prefill(layer, xd, T, od, b, s);
   if (st != MOE_OK) return st;
   if (cudaMemcpyAsync(out_host, od, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
@@ -536,7 +588,7 @@ int moe_forward_profiled(const moe_layer_desc* layer, const moe_bf16* x, int T, 
       for (int j = 0; j < i; ++j) cudaEventDestroy(tr.ev[j]);
       return MOE_ERR_CUDA;
     }
-  st = (T <= kDecodeMaxT) ? enqueue_decode(layer, x, T, out, b, s, &tr) : enqueue_prefill(layer, x, T, out, b, s, &tr);
+  st = forward_uses_fused_decode(layer, T) ? enqueue_decode(layer, x, T, out, b, s, &tr) : enqueue_prefill(layer, x, T, out, b, s, &tr);
   if (st == MOE_OK && cudaEventSynchronize(tr.ev[tr.n - 1]) != cudaSuccess) st = MOE_ERR_CUDA;
   *n_stages = 0;
   if (st == MOE_OK) {

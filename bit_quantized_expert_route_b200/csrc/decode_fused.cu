@@ -1,48 +1,56 @@
-// Fused decode layer for T <= 2: router, top-k, grouping, gate/up + SwiGLU,
-// down projection and the fixed-order combine in ONE cooperative launch of
-// one CTA per SM ("Perplexity's Lily: ...", section "How It Works: Prefill
-// and Decode Strategies": batch-1 decode streams the active experts' packed
-// weights, so the layer is bound by how fast those bytes arrive).
+// Fused decode for T <= 8 tokens: router, top-k, grouping, gate/up + SwiGLU,
+// down projection and the fixed-order combine of a whole STACK of layers in
+// ONE cooperative launch of one CTA per SM ("Perplexity's Lily: ...", section
+// "How It Works: Prefill and Decode Strategies": decoding a few tokens streams
+// the active experts' packed weights, so a layer is bound by how fast those
+// bytes arrive, and the forward pass is one GPU submission with no CPU round
+// trip).  A single moe_forward call is a stack of one layer.
 //
-// Why one launch: at T = 1 the active weights are ~16 MB, about 2.5 us of HBM
-// time.  As separate launches the layer pays several launch latencies, and no
-// weight load can start before the routing kernel has finished.  Here the
-// phases are separated by two grid-wide barriers (all CTAs are co-resident:
-// cooperative launch), and every CTA issues ALL of its weight tiles as
-// asynchronous bulk copies the moment routing is known, so the memory system
-// sees the whole working set at once:
+// Why one launch for many layers: at T = 1 a layer's active weights are
+// ~16 MB, about 2.5 us of HBM time, so launch latency, cold instruction
+// caches and memory latency decide the layer time.  Inside one launch the
+// code stays warm from layer to layer, nothing is launched between layers,
+// and the producer warp fetches the next layer's router rows and first
+// shared-expert tile while the current layer still computes.
 //
-//   A  router logits: CTA c scores rows c, c+G, ... of [W_r; w_sg] for every
-//      token and stores them; CTAs that own a shared-expert unit already
-//      start that unit's copy (it does not depend on routing).
-//   -- grid barrier --
+// Each layer, with three grid-wide barriers (all CTAs are co-resident:
+// cooperative launch):
+//
+//   A  input: layer 0 reads x; layer l > 0 reads the previous layer's output
+//      y (bf16) and the CTAs' partial sums of its squares and applies
+//      RMSNorm (weight 1): x = bf16(y / sqrt(mean(y^2) + eps)).  Router
+//      logits: CTA c scores rows c, c+G, ... of [W_r; w_sg] (from shared
+//      memory, copied there by the producer ahead of time) for every token.
+//   -- grid barrier (logits) --
 //   B  every CTA reads the T x (E+1) logits and repeats the (tiny, exact and
 //      deterministic) top-k, shared gate and counting sort, so it knows the
-//      active experts without another barrier; CTA 0 also writes the routing
-//      outputs.
-//   C  gate/up units: (expert slot, 16 features) -> h = bf16(silu(g) * u),
-//      one feature per consumer warp.
-//   -- grid barrier (h complete) --  the producer warp keeps copying the down
+//      active experts without another barrier.
+//   C  gate/up units: (expert slot, 16 features) -> h = bf16(silu(g) * u).
+//   -- grid barrier (h complete) --  the producer keeps copying the down
 //      tiles meanwhile: they depend on the routing, not on h.
-//   D  down units: (16 output dims, up to 8 expert slots), one dim per
-//      consumer warp; then the combine of each token's k + 1 terms in slot
-//      order, then the shared term, exactly as the unfused decode kernels.
+//   D  down units: (16 output dims, up to 8 expert slots); then the combine
+//      of each token's k + 1 terms in slot order, then the shared term,
+//      exactly as the other kernels; the CTA writes its output dims and the
+//      partial sum of their squares.
+//   -- grid barrier (outputs complete; between layers only) --
 //
 // Weight tiles stream through a ring of shared-memory slots filled by one
 // producer thread (cp.async.bulk, completion on the slot's "full" mbarrier)
-// and released by the 16 consumer warps ("empty" mbarrier, count 16).  All
+// and released by the 16 consumer warps ("empty" mbarrier, one arrival per
+// warp).  The ring position runs on across layers, so the producer can start
+// the next layer's routing-independent tile as soon as a slot frees up.  All
 // waits are bounded; a timeout records MOE_ERR_DEVICE_TIMEOUT in the status
-// word and the kernel returns.
+// word and the kernel returns with every copy it issued landed.
 //
 // Dot products on the tensor cores (warp-level mma.sync, bf16 in, FP32
-// accumulation): per group of 64 inputs, with A = 128 + q as exact bf16 values
-// (one AND-OR per code pair, no scale applied) and B = the activations,
+// accumulation; the T <= 8 tokens are the 8 columns of the n8 tile): per group
+// of 64 inputs, with A = 128 + q as exact bf16 values (one AND-OR per code
+// pair, no scale applied) and B = the activations,
 //   sum_i (s q_i + b) x_i = s * (sum_i (128 + q_i) x_i - 128 X) + b X,  X = sum_i x_i,
 // applied per group after the MMAs.  Inside each group of 8 inputs both
 // operands use the order (0,4,1,5,2,6,3,7) in which the AND-OR yields code
 // pairs; the activations are staged in that order, so no permutes are
-// needed.  The integer work per code drops from ~2 (nibble to float) to ~1
-// instruction per code pair.
+// needed.
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
@@ -52,29 +60,37 @@ namespace {
 
 constexpr int kFWarps = 16;                     // consumer warps
 constexpr int kFThreads = (kFWarps + 1) * 32;   // + the producer warp
-constexpr int kFFeat = 16;                      // features per gate/up unit (one per consumer warp)
-constexpr int kFDims = 16;                      // output dims per down block (one per consumer warp)
-constexpr int kFMaxSpd = 8;                     // expert slots per down unit
+constexpr int kFFeat = 16;                      // features per gate/up unit
+constexpr int kFDims = 16;                      // output dims per down block
+constexpr int kFMaxSpd = 8;                     // expert slots per down unit (one per warp pair)
 constexpr int kFRingMax = 8;
-constexpr int kFMaxT = 2;
+constexpr int kFMaxT = 8;                       // tokens: the n8 column tile of mma.sync
 constexpr int kFRouterRows = 2;                 // router rows per CTA with loads in flight together
+constexpr int kFMaxRouterRows = 4;              // router rows per CTA held in shared memory
+constexpr int kFMaxLayers = 40;                 // layers per launch (kernel-parameter space)
+constexpr int kFMaxGrid = 160;                  // CTAs (SMs) the RMSNorm partial sums are read for in one pass
 
 struct FusedArgs {
   Geometry g;
-  LayerPtr L;
-  const uint16_t* x;
-  uint16_t* out;
-  RoutingPtrs r;
+  int n_layers;
+  float eps;              // RMSNorm between layers
+  const uint16_t* x;      // input of layer 0 [T, H]
+  uint16_t* out;          // output of the last layer [T, H]
+  uint16_t* y;            // outputs of the other layers [T, H] (workspace)
+  float* sumsq;           // [G][kFMaxT] partial sums of squares of y (workspace)
+  uint16_t* trace;        // NULL or [n_layers][2][T][H]: layer inputs and outputs
+  RoutingPtrs r;          // routing outputs of the last layer (topk_idx NULL: none)
   int32_t* active;
   int32_t* n_active;
   float* logits;          // [T, E+1]
   uint16_t* h;            // [T*k, I]
   uint16_t* h_s;          // [T, Is]
-  unsigned* bar;          // [0] arrivals, [1] generation
+  unsigned* bar;          // [0] arrivals, [1] exits
   int* status;
-  int ring, slot_bytes, spd;
+  int ring, slot_bytes, spd, rows_per_cta;
   long long wait_limit;   // cycles before a bounded wait gives up
-  int off_bar, off_xs, off_xsum, off_hs, off_hsum, off_lg, off_rt, off_y;
+  int off_bar, off_wr, off_xs, off_xsum, off_lg, off_rt, off_y, off_nrm;
+  LayerPtr layers[kFMaxLayers];
 };
 
 // Routing state every CTA rebuilds in shared memory.  Expert slots in down
@@ -93,18 +109,6 @@ struct RouteSmem {
   int32_t abort;
 };
 
-
-// 8 bf16 values (x0,x1)(x2,x3)(x4,x5)(x6,x7) in the interleaved K order
-// (x0,x4)(x1,x5)(x2,x6)(x3,x7).
-__device__ __forceinline__ uint4 interleave8(const uint4& v) {   // (x0,x1)(x2,x3)(x4,x5)(x6,x7)
-  uint4 o;
-  o.x = __byte_perm(v.x, v.z, 0x5410);
-  o.y = __byte_perm(v.x, v.z, 0x7632);
-  o.z = __byte_perm(v.y, v.w, 0x5410);
-  o.w = __byte_perm(v.y, v.w, 0x7632);
-  return o;
-}
-
 // D (16 rows x 8 tokens, FP32) += A (16 x 16, bf16) B (16 x 8, bf16).
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
@@ -121,10 +125,21 @@ __device__ __forceinline__ uint32_t code_pair(uint32_t w, int shift) {   // bf16
   return d;
 }
 
+// 8 bf16 values (x0,x1)(x2,x3)(x4,x5)(x6,x7) in the interleaved K order
+// (x0,x4)(x1,x5)(x2,x6)(x3,x7).
+__device__ __forceinline__ uint4 interleave8(const uint4& v) {
+  uint4 o;
+  o.x = __byte_perm(v.x, v.z, 0x5410);
+  o.y = __byte_perm(v.x, v.z, 0x7632);
+  o.z = __byte_perm(v.y, v.w, 0x5410);
+  o.w = __byte_perm(v.y, v.w, 0x7632);
+  return o;
+}
+
 // One group of 64 inputs for rows g, g+8 of a 16-row weight tile (lane g =
 // lane/4, t = lane%4): lane reads words 2t, 2t+1 of the group in both rows
 // (qg, qg8: this lane's 8 bytes) and the 32 staged activations of token g at
-// 8-groups 2t, 2t+1 (xb0, xb1; zero for padding tokens).  d gets
+// 8-groups 2t, 2t+1 (xb0, xb1; zero for tokens outside the unit).  d gets
 // sum (128 + q) x for (row g, tokens 2t, 2t+1) and (row g+8, same tokens).
 __device__ __forceinline__ void group_dot(float (&d)[4], const uint2& qg, const uint2& qg8, const uint4& xb0,
                                           const uint4& xb1) {
@@ -199,13 +214,14 @@ __device__ __forceinline__ void topk_redux(const float* lg, int E, int k, int la
 
 __device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kFWarps * 32) : "memory"); }
 
-// Grid-wide barrier n (1, 2, ...) of one launch, called by one thread per
-// CTA after a CTA barrier (all CTAs are co-resident).  bar[0] counts arrivals
-// over the whole launch: each CTA adds 1 with release semantics (publishing
-// what its threads wrote before the CTA barrier) and polls, bounded, until
-// the count reaches n * nblocks, then acquires.  No arriver has to reset or
-// publish anything, so the barrier costs one release-add and the polls.
-// bar[0] starts every launch at zero: grid_exit resets it.
+// Grid-wide barrier number n (target n * nblocks) of one launch, called by
+// one thread per CTA after a barrier of the CTA's consumers (all CTAs are
+// co-resident).  bar[0] counts arrivals over the whole launch: each CTA adds
+// 1 with release semantics (publishing what its threads wrote before the CTA
+// barrier) and polls, bounded, until the count reaches the target, then
+// acquires.  No arriver has to reset or publish anything, so the barrier
+// costs one release-add and the polls.  bar[0] starts every launch at zero:
+// grid_exit resets it.
 __device__ bool grid_barrier(unsigned* bar, unsigned target, int* status, long long limit) {
   asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(bar) : "memory");
   const long long deadline = clock64() + limit;
@@ -233,10 +249,10 @@ __device__ void grid_exit(unsigned* bar, unsigned nblocks) {
   }
 }
 
-// Unit schedule of one CTA: its gate/up units u = c, c+G, ... over the
-// global list [shared-expert units | routed units], then its down units
-// (dim blocks c, c+G, ..., each split into parts of at most spd_max slots,
-// balanced).
+// Unit schedule of one CTA in one layer: its gate/up units u = c, c+G, ...
+// over the global list [shared-expert units | routed units], then its down
+// units (dim blocks c, c+G, ..., each split into parts of at most spd_max
+// slots, balanced).
 struct Sched {
   int n_gu_units;      // global gate/up units
   int n_sh_units;      // of which shared-expert units (first)
@@ -245,7 +261,7 @@ struct Sched {
   int n_down_parts;    // down units per dim block
   int spd;             // slots per down unit (the last may have fewer)
   int n_blocks;        // dim blocks (H / 16)
-  int my_gu, my_blocks;
+  int my_gu, my_blocks, n_units;
 };
 
 __device__ __forceinline__ Sched make_sched(const FusedArgs& a, int n_act) {
@@ -260,6 +276,7 @@ __device__ __forceinline__ Sched make_sched(const FusedArgs& a, int n_act) {
   const int G = gridDim.x, c = blockIdx.x;
   s.my_gu = s.n_gu_units > c ? (s.n_gu_units - c + G - 1) / G : 0;
   s.my_blocks = s.n_blocks > c ? (s.n_blocks - c + G - 1) / G : 0;
+  s.n_units = s.my_gu + s.my_blocks * s.n_down_parts;
   return s;
 }
 
@@ -270,27 +287,32 @@ __device__ __forceinline__ void gu_unit(const Sched& s, int u, int& slot, int& f
   f0 = (sh ? u : (u - s.n_sh_units) % s.units_per_exp) * kFFeat;
 }
 
-// Issue the bulk copies of unit i of this CTA into ring slot `dst`.
-// gate/up layout: [q gate 16 rows][q up 16 rows][s gate][b gate][s up][b up];
+// Issue the bulk copies of the gate/up tile (expert e, features f0..f0+15)
+// of layer L into `dst`: [q gate 16 rows][q up 16 rows][s gate][b gate][s up][b up].
+__device__ void issue_gateup(const Geometry& g, const LayerPtr& L, int e, int f0, uint32_t dst, uint64_t* full) {
+  const bool sh = e >= g.E;
+  const size_t row0 = static_cast<size_t>(sh ? 0 : e * g.I) + f0;
+  const QMatPtr Wg = sh ? L.sh_gate : L.gate;
+  const QMatPtr Wu = sh ? L.sh_up : L.up;
+  const uint32_t qb = kFFeat * g.H / 2, sb = kFFeat * g.H / 32;
+  tc::mbar_arrive_expect_tx(full, 2 * qb + 4 * sb);
+  tc::bulk_load(dst, Wg.q + row0 * (g.H / 8), qb, full);
+  tc::bulk_load(dst + qb, Wu.q + row0 * (g.H / 8), qb, full);
+  tc::bulk_load(dst + 2 * qb, Wg.s + row0 * (g.H / kGroup), sb, full);
+  tc::bulk_load(dst + 2 * qb + sb, Wg.b + row0 * (g.H / kGroup), sb, full);
+  tc::bulk_load(dst + 2 * qb + 2 * sb, Wu.s + row0 * (g.H / kGroup), sb, full);
+  tc::bulk_load(dst + 2 * qb + 3 * sb, Wu.b + row0 * (g.H / kGroup), sb, full);
+}
+
+// Issue the bulk copies of unit i of this CTA (layer L) into ring slot `dst`.
 // down layout: per expert slot jj at jj * 9 Kmax: [q 16 rows][s][b].
-__device__ void issue_unit(const FusedArgs& a, const RouteSmem& rt, const Sched& s, int i, uint32_t dst,
-                           uint64_t* full) {
+__device__ void issue_unit(const FusedArgs& a, const LayerPtr& L, const RouteSmem& rt, const Sched& s, int i,
+                           uint32_t dst, uint64_t* full) {
   const Geometry& g = a.g;
   if (i < s.my_gu) {
     int slot, f0;
     gu_unit(s, blockIdx.x + i * gridDim.x, slot, f0);
-    const bool sh = slot == 0;
-    const size_t row0 = static_cast<size_t>(sh ? 0 : rt.slot_e[slot] * g.I) + f0;
-    const QMatPtr Wg = sh ? a.L.sh_gate : a.L.gate;
-    const QMatPtr Wu = sh ? a.L.sh_up : a.L.up;
-    const uint32_t qb = kFFeat * g.H / 2, sb = kFFeat * g.H / 32;
-    tc::mbar_arrive_expect_tx(full, 2 * qb + 4 * sb);
-    tc::bulk_load(dst, Wg.q + row0 * (g.H / 8), qb, full);
-    tc::bulk_load(dst + qb, Wu.q + row0 * (g.H / 8), qb, full);
-    tc::bulk_load(dst + 2 * qb, Wg.s + row0 * (g.H / kGroup), sb, full);
-    tc::bulk_load(dst + 2 * qb + sb, Wg.b + row0 * (g.H / kGroup), sb, full);
-    tc::bulk_load(dst + 2 * qb + 2 * sb, Wu.s + row0 * (g.H / kGroup), sb, full);
-    tc::bulk_load(dst + 2 * qb + 3 * sb, Wu.b + row0 * (g.H / kGroup), sb, full);
+    issue_gateup(g, L, rt.slot_e[slot], f0, dst, full);
     return;
   }
   const int di = i - s.my_gu;
@@ -306,7 +328,7 @@ __device__ void issue_unit(const FusedArgs& a, const RouteSmem& rt, const Sched&
   for (int jj = 0; jj < nj; ++jj) {
     const bool sh = j0 + jj == 0;
     const int K = sh ? g.Is : g.I;
-    const QMatPtr W = sh ? a.L.sh_down : a.L.down;
+    const QMatPtr W = sh ? L.sh_down : L.down;
     const size_t row0 = static_cast<size_t>(sh ? 0 : rt.slot_e[j0 + jj] * g.H) + blk * kFDims;
     const uint32_t base = dst + jj * (9 * Kmax);
     const uint32_t qb = kFDims * K / 2, sb = kFDims * K / 32;
@@ -316,81 +338,189 @@ __device__ void issue_unit(const FusedArgs& a, const RouteSmem& rt, const Sched&
   }
 }
 
+// This CTA's router rows of layer L (rows c, c+G, ... of [W_r; w_sg]) into
+// the shared-memory row buffer; completes on `full`.
+__device__ void issue_router_rows(const Geometry& g, const LayerPtr& L, int nrows, uint32_t dst, uint64_t* full) {
+  const uint32_t rb = static_cast<uint32_t>(g.H) * 2;
+  tc::mbar_arrive_expect_tx(full, nrows * rb);
+  for (int rr = 0; rr < nrows; ++rr) {
+    const int row = blockIdx.x + rr * gridDim.x;
+    const uint16_t* src = row < g.E ? L.w_router + static_cast<size_t>(row) * g.H : L.w_sg;
+    tc::bulk_load(dst + rr * rb, src, rb, full);
+  }
+}
+
 template <int NT>
 __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid_constant__ FusedArgs a) {
   extern __shared__ __align__(128) uint8_t fsm[];
   const Geometry& g = a.g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = g.T, k = g.k, E = g.E, E1 = g.E + 1;
+  const int G = static_cast<int>(gridDim.x);
   const uint32_t ring0 = tc::smem_u32(fsm);
   uint64_t* full = reinterpret_cast<uint64_t*>(fsm + a.off_bar);
   uint64_t* empty = full + kFRingMax;
+  uint64_t* rfull = empty + kFRingMax;    // router rows of the current layer have landed
+  uint64_t* rfree = rfull + 1;            // consumers are done with the router rows
+  uint64_t* ready = rfree + 1;            // the layer's routing is in shared memory
+  const uint16_t* wr = reinterpret_cast<const uint16_t*>(fsm + a.off_wr);   // [rows_per_cta][H]
+  // x (phases A, C) and h (phase D) share one staging area, as do their group sums
   uint16_t* xs = reinterpret_cast<uint16_t*>(fsm + a.off_xs);   // [T][H] bf16, interleaved K order
   float* xsum = reinterpret_cast<float*>(fsm + a.off_xsum);      // [T][H/64] group sums
-  uint16_t* hs = reinterpret_cast<uint16_t*>(fsm + a.off_hs);   // [T*k + T][Kmax] bf16, interleaved K order
-  float* hsum = reinterpret_cast<float*>(fsm + a.off_hsum);      // [T*k + T][Kmax/64] group sums
-  float* lg = reinterpret_cast<float*>(fsm + a.off_lg);       // [T][E1], also the router partials
+  uint16_t* hs = xs;                                             // [T*k + T][Kmax] bf16, interleaved K order
+  float* hsum = xsum;                                            // [T*k + T][Kmax/64] group sums
+  float* lg = reinterpret_cast<float*>(fsm + a.off_lg);          // logits; router partials; dot reductions
   RouteSmem& rt = *reinterpret_cast<RouteSmem*>(fsm + a.off_rt);
-  float* ys = reinterpret_cast<float*>(fsm + a.off_y);        // [T*k + T][my_blocks][16]
+  float* ys = reinterpret_cast<float*>(fsm + a.off_y);           // [T*k + T][my_blocks][16]
+  float* nrm = reinterpret_cast<float*>(fsm + a.off_nrm);        // [T] 1/rms of the layer input
   volatile int* abort_flag = &rt.abort;
   const int Kmax = max(g.I, g.Is);
+  const int n = T * k, Tk = n;
+  const int nrows = (E1 - static_cast<int>(blockIdx.x) + G - 1) / G;   // router rows of this CTA
   const bool producer = warp == kFWarps;
+  const bool early = static_cast<int>(blockIdx.x) < g.Is / kFFeat;      // first unit is a shared-expert unit
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < a.ring; ++s) {
       tc::mbar_init(&full[s], 1);
       tc::mbar_init(&empty[s], kFWarps);
     }
+    tc::mbar_init(rfull, 1);
+    tc::mbar_init(rfree, 1);
+    tc::mbar_init(ready, 1);
     rt.abort = 0;
     tc::fence_barrier_init();
   }
   __syncthreads();
 
-  // ---------------------------------------------------------------- phase A
-  // The first unit of a CTA whose first gate/up unit is a shared-expert unit
-  // does not depend on routing: start its copy now.
-  const bool early = static_cast<int>(blockIdx.x) < g.Is / kFFeat;
-  if (producer && lane == 0 && early) {
-    Sched s0{};
-    s0.n_sh_units = g.Is / kFFeat;
-    s0.units_per_exp = g.I / kFFeat;
-    s0.n_gu_units = s0.n_sh_units;
-    s0.my_gu = 1;
-    issue_unit(a, rt, s0, 0, ring0, &full[0]);
+  if (producer) {
+    // ------------------------------------------------------- producer warp
+    // Per layer: the routing-independent first unit (a shared-expert tile),
+    // then, once the layer's routing is known, the next layer's router rows
+    // and the rest of this layer's units.  Ring fills are numbered across
+    // layers in the order the consumers take them.
+    if (lane == 0) {
+      uint32_t fill = 0;             // ring fills issued
+      issue_router_rows(g, a.layers[0], nrows, tc::smem_u32(wr), rfull);
+      uint32_t rfills = 1;
+      bool ok = true;
+      for (int l = 0; l < a.n_layers && ok; ++l) {
+        const LayerPtr& L = a.layers[l];
+        const uint32_t base = fill;
+        if (early) {
+          const int sl = static_cast<int>(fill % a.ring);
+          if (!tc::mbar_wait(&empty[sl], ((fill / a.ring) & 1u) ^ 1u, abort_flag, a.status, a.wait_limit)) break;
+          tc::fence_proxy_async_smem();
+          issue_gateup(g, L, E, static_cast<int>(blockIdx.x) * kFFeat, ring0 + sl * a.slot_bytes, &full[sl]);
+          ++fill;
+        }
+        if (!tc::mbar_wait(ready, static_cast<uint32_t>(l) & 1u, abort_flag, a.status, a.wait_limit)) break;
+        const Sched s = make_sched(a, rt.n_act);
+        if (l + 1 < a.n_layers) {
+          // the consumers finished with this layer's router rows before its routing was ready
+          if (!tc::mbar_wait(rfree, static_cast<uint32_t>(l) & 1u, abort_flag, a.status, a.wait_limit)) break;
+          tc::fence_proxy_async_smem();
+          issue_router_rows(g, a.layers[l + 1], nrows, tc::smem_u32(wr), rfull);
+          ++rfills;
+        }
+        for (uint32_t i = fill - base; i < static_cast<uint32_t>(s.n_units); ++i) {
+          const int sl = static_cast<int>(fill % a.ring);
+          if (!tc::mbar_wait(&empty[sl], ((fill / a.ring) & 1u) ^ 1u, abort_flag, a.status, a.wait_limit)) {
+            ok = false;
+            break;
+          }
+          tc::fence_proxy_async_smem();   // consumers' generic reads of the slot precede the refill
+          issue_unit(a, L, rt, s, static_cast<int>(i), ring0 + sl * a.slot_bytes, &full[sl]);
+          ++fill;
+        }
+      }
+      // every copy this thread issued has landed before the CTA may exit
+      tc::drain_ring(full, static_cast<uint32_t>(a.ring), fill, a.status);
+      tc::drain_ring(rfull, 1u, rfills, a.status);
+    }
+    __syncwarp();
+    return;
   }
-  if (!producer) {
-    const int tid = threadIdx.x, nthr = kFWarps * 32;
-    // router rows r = c, c + G, ...: thread tid owns the inputs [4 tid, 4 tid + 4)
-    // of every row and token.  x and the first rows are requested before any
-    // of them is used, so they arrive in one memory round trip; x is then
-    // staged from the same registers.
-    const int nrows = (E1 - static_cast<int>(blockIdx.x) + gridDim.x - 1) / gridDim.x;
-    const int c = 4 * tid;
-    const bool live = c < g.H;
+
+  // ------------------------------------------------------ consumer warps
+  const int tid = threadIdx.x, nthr = kFWarps * 32;
+  const int lg4 = lane >> 2, lt = lane & 3;
+  const int ngrp = g.H / kGroup;
+  const uint32_t qb = kFFeat * g.H / 2, sb = kFFeat * g.H / 32;
+  const size_t act = static_cast<size_t>(T) * g.H;
+  uint32_t fill = 0;      // ring fills consumed
+  unsigned nbar = 0;      // grid barriers passed
+  // Abort handling: a wait that gives up raises rt.abort (and makes later
+  // waits give up at once).  No consumer warp leaves a loop on its own: every
+  // warp keeps taking the same CTA barriers, skipping the work, and the
+  // decision to stop is read from rt.abort right after a CTA barrier, where
+  // every thread sees the same value.
+  for (int l = 0; l < a.n_layers; ++l) {
+    const LayerPtr& L = a.layers[l];
+    const bool last = l + 1 == a.n_layers;
+    bool ok = true;
+
+    // -------------------------------------------------------------- phase A
+    // the layer input: x, or RMSNorm of the previous layer's output
+    if (l > 0) {
+      // warp t sums the CTAs' partials of token t: lane i takes CTAs i, i+32,
+      // ... (all loads in flight at once), then a fixed shuffle tree; the
+      // same order in every CTA
+      if (warp < T) {
+        float part[kFMaxGrid / 32];
+#pragma unroll
+        for (int j = 0; j < kFMaxGrid / 32; ++j) {
+          const int c = lane + 32 * j;
+          part[j] = c < G ? __ldcg(a.sumsq + c * kFMaxT + warp) : 0.f;
+        }
+        float ss = 0.f;
+#pragma unroll
+        for (int j = 0; j < kFMaxGrid / 32; ++j) ss += part[j];
+        ss = warp_sum(ss);
+        if (lane == 0) nrm[warp] = 1.0f / sqrtf(ss / static_cast<float>(g.H) + a.eps);
+      }
+      consumers_sync();
+    }
+    const uint16_t* src = l == 0 ? a.x : a.y;
+    const int c4 = 4 * tid;
+    const bool live = c4 < g.H;
     uint2 xv[NT];
 #pragma unroll
-    for (int t = 0; t < NT; ++t)
-      xv[t] = (live && t < T) ? __ldg(reinterpret_cast<const uint2*>(a.x + static_cast<size_t>(t) * g.H + c))
-                              : make_uint2(0u, 0u);
-    float* part = lg;   // [nrows][kFWarps][NT] partials (lg is free until phase B)
-    for (int r0 = 0; r0 < nrows; r0 += kFRouterRows) {
-      uint2 wv[kFRouterRows];
-#pragma unroll
-      for (int q = 0; q < kFRouterRows; ++q) {
-        const int row = blockIdx.x + (r0 + q) * gridDim.x;
-        const uint16_t* wrow = row < E ? a.L.w_router + static_cast<size_t>(row) * g.H : a.L.w_sg;
-        wv[q] = (live && r0 + q < nrows) ? __ldg(reinterpret_cast<const uint2*>(wrow + c)) : make_uint2(0u, 0u);
+    for (int t = 0; t < NT; ++t) {
+      xv[t] = make_uint2(0u, 0u);
+      if (live && t < T) {
+        xv[t] = __ldcg(reinterpret_cast<const uint2*>(src + static_cast<size_t>(t) * g.H + c4));
+        if (l > 0) {
+          const float s = nrm[t];
+          xv[t].x = pack_bf16x2(bf16_lo(xv[t].x) * s, bf16_hi(xv[t].x) * s);
+          xv[t].y = pack_bf16x2(bf16_lo(xv[t].y) * s, bf16_hi(xv[t].y) * s);
+        }
+        if (a.trace && blockIdx.x == 0)
+          *reinterpret_cast<uint2*>(a.trace + 2 * l * act + static_cast<size_t>(t) * g.H + c4) = xv[t];
       }
+    }
+    // router rows r = c, c + G, ... (staged by the producer): thread tid owns
+    // the inputs [4 tid, 4 tid + 4) of every row and token
+    // (wait outcomes are made warp-uniform: the work they guard uses warp-collective instructions)
+    ok = __all_sync(0xffffffffu, tc::mbar_wait(rfull, static_cast<uint32_t>(l) & 1u, abort_flag, a.status,
+                                               a.wait_limit));
+    float* part = lg;   // [nrows][kFWarps][NT] partials (lg is free until phase B)
+    if (ok) {
+      for (int r0 = 0; r0 < nrows; r0 += kFRouterRows) {
 #pragma unroll
-      for (int q = 0; q < kFRouterRows; ++q) {
+        for (int q = 0; q < kFRouterRows; ++q) {
+          const uint2 wv = (live && r0 + q < nrows)
+                               ? *reinterpret_cast<const uint2*>(wr + static_cast<size_t>(r0 + q) * g.H + c4)
+                               : make_uint2(0u, 0u);
 #pragma unroll
-        for (int t = 0; t < NT; ++t) {
-          float s = fmaf(bf16_lo(xv[t].x), bf16_lo(wv[q].x), 0.f);
-          s = fmaf(bf16_hi(xv[t].x), bf16_hi(wv[q].x), s);
-          s = fmaf(bf16_lo(xv[t].y), bf16_lo(wv[q].y), s);
-          s = fmaf(bf16_hi(xv[t].y), bf16_hi(wv[q].y), s);
-          s = warp_sum(s);
-          if (lane == 0 && r0 + q < nrows && t < T) part[((r0 + q) * kFWarps + warp) * NT + t] = s;
+          for (int t = 0; t < NT; ++t) {
+            float s = fmaf(bf16_lo(xv[t].x), bf16_lo(wv.x), 0.f);
+            s = fmaf(bf16_hi(xv[t].x), bf16_hi(wv.x), s);
+            s = fmaf(bf16_lo(xv[t].y), bf16_lo(wv.y), s);
+            s = fmaf(bf16_hi(xv[t].y), bf16_hi(wv.y), s);
+            s = warp_sum(s);
+            if (lane == 0 && r0 + q < nrows && t < T) part[((r0 + q) * kFWarps + warp) * NT + t] = s;
+          }
         }
       }
     }
@@ -407,7 +537,11 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
       }
     }
     consumers_sync();
-    for (int i = tid; i < T * (g.H / 64); i += nthr) {     // sums over groups of 64 (fixed order)
+    if (tid == 0) {
+      tc::fence_proxy_async_smem();      // the row buffer's generic reads precede its next TMA refill
+      tc::mbar_arrive(rfree);
+    }
+    for (int i = tid; i < T * ngrp; i += nthr) {     // sums over groups of 64 (fixed order)
       const uint4* r4 = reinterpret_cast<const uint4*>(xs) + i * 8;
       float sum = 0.f;
 #pragma unroll
@@ -418,344 +552,333 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
       }
       xsum[i] = sum;
     }
-    if (tid < nrows * T) {
+    if (ok && tid < nrows * T) {
       const int rr = tid / T, t = tid % T;
-      const int row = blockIdx.x + rr * gridDim.x;
+      const int row = blockIdx.x + rr * G;
       float v = 0.f;
       for (int w = 0; w < kFWarps; ++w) v += part[(rr * kFWarps + w) * NT + t];
-      if (row < E && a.L.router_bias) v += a.L.router_bias[row];
+      if (row < E && L.router_bias) v += L.router_bias[row];
       __stcg(a.logits + static_cast<size_t>(t) * E1 + row, v);
     }
-  }
-  __syncthreads();
-  if (threadIdx.x == 0 && !grid_barrier(a.bar, gridDim.x, a.status, a.wait_limit)) {
-    rt.abort = 1;
-    grid_exit(a.bar, gridDim.x);
-  }
-  __syncthreads();
-  if (rt.abort) {
-    if (producer && lane == 0 && early) tc::mbar_wait_drain(&full[0], 0, a.status);
-    return;
-  }
-
-  // ---------------------------------------------------------------- phase B
-  // Every CTA rebuilds the routing from the logits (top-k by warp reductions,
-  // then a one-warp counting sort of the n = T*k <= 16 entries), so no
-  // further barrier is needed before the expert weights can be requested.
-  for (int i = threadIdx.x; i < T * E1; i += blockDim.x) lg[i] = __ldcg(a.logits + i);
-  __syncthreads();
-  if (warp < T) {
-    topk_redux(lg + warp * E1, E, k, lane, rt.idx + warp * k, rt.w + warp * k);
-    if (lane == 0) rt.sigma[warp] = sigmoid(lg[warp * E1 + E]);
-  }
-  __syncthreads();
-  const int n = T * k;
-  const int Tk = n;
-  if (warp == 0) {
-    const bool live = lane < n;
-    const int e_i = live ? rt.idx[lane] : -1 - lane;          // distinct dummies for idle lanes
-    const unsigned peers = __match_any_sync(0xffffffffu, e_i);
-    const int rank = __popc(peers & lanemask_lt());           // same expert, earlier (token, slot)
-    const bool first = live && rank == 0;
-    const unsigned firsts = __ballot_sync(0xffffffffu, first);
-    int below = 0, abelow = 0;                                // entries / active experts with a smaller expert
-    for (int j = 0; j < n; ++j) {
-      const int ej = __shfl_sync(0xffffffffu, e_i, j);
-      below += ej < e_i ? 1 : 0;
-      abelow += (((firsts >> j) & 1u) && ej < e_i) ? 1 : 0;
+    consumers_sync();
+    if (tid == 0) {
+      if (rt.abort || !grid_barrier(a.bar, (++nbar) * G, a.status, a.wait_limit)) rt.abort = 1;
     }
-    if (live) {
+    consumers_sync();
+    if (rt.abort) break;
+
+    // -------------------------------------------------------------- phase B
+    // Every CTA rebuilds the routing from the logits (top-k by warp
+    // reductions, then a counting sort of the n = T*k <= 64 entries), so no
+    // further barrier is needed before the expert weights can be requested.
+    for (int i = tid; i < T * E1; i += nthr) lg[i] = __ldcg(a.logits + i);
+    consumers_sync();
+    if (warp < T) {
+      topk_redux(lg + warp * E1, E, k, lane, rt.idx + warp * k, rt.w + warp * k);
+      if (lane == 0) rt.sigma[warp] = sigmoid(lg[warp * E1 + E]);
+    }
+    consumers_sync();
+    if (tid < n) {
+      // stable rank: entries with a smaller expert, then earlier entries of
+      // the same expert; active experts below this one
+      const int e_i = rt.idx[tid];
+      int below = 0, rank = 0, abelow = 0, cnt = 0;
+      for (int j = 0; j < n; ++j) {
+        const int ej = rt.idx[j];
+        below += ej < e_i ? 1 : 0;
+        rank += (ej == e_i && j < tid) ? 1 : 0;
+        cnt += ej == e_i ? 1 : 0;
+        bool first_j = true;                              // entry j is its expert's first occurrence
+        for (int q = 0; q < j; ++q) first_j = first_j && rt.idx[q] != ej;
+        abelow += (first_j && ej < e_i) ? 1 : 0;
+      }
       const int pos = below + rank;
-      rt.perm[pos] = lane;
-      rt.inv_perm[lane] = pos;
-      if (first) {
+      rt.perm[pos] = tid;
+      rt.inv_perm[tid] = pos;
+      if (rank == 0) {
         rt.slot_e[1 + abelow] = e_i;
-        rt.slot_cnt[1 + abelow] = __popc(peers);
+        rt.slot_cnt[1 + abelow] = cnt;
         rt.slot_off[1 + abelow] = below;
       }
     }
-    if (lane == 0) {
-      rt.n_act = __popc(firsts);
+    if (tid == nthr - 1) {
+      int nact = 0;
+      for (int j = 0; j < n; ++j) {
+        bool first_j = true;
+        for (int q = 0; q < j; ++q) first_j = first_j && rt.idx[q] != rt.idx[j];
+        nact += first_j ? 1 : 0;
+      }
+      rt.n_act = nact;
       rt.slot_e[0] = E;
       rt.slot_cnt[0] = T;
       rt.slot_off[0] = Tk;
     }
-  }
-  __syncthreads();
-  const Sched s = make_sched(a, rt.n_act);
-  const int n_units = s.my_gu + s.my_blocks * s.n_down_parts;
-
-  if (producer) {
-    // ------------------------------------------------------- producer warp
-    if (lane == 0) {
-      int last[kFRingMax];
-      for (int sl = 0; sl < kFRingMax; ++sl) last[sl] = -1;
-      if (early) last[0] = 0;
-      for (int i = early ? 1 : 0; i < n_units; ++i) {
-        const int sl = i % a.ring;
-        if (!tc::mbar_wait(&empty[sl], ((i / a.ring) & 1u) ^ 1u, abort_flag, a.status, a.wait_limit)) break;
-        tc::fence_proxy_async_smem();   // consumers' generic reads of the slot precede the refill
-        issue_unit(a, rt, s, i, ring0 + sl * a.slot_bytes, &full[sl]);
-        last[sl] = i;
-      }
-      // every copy this thread issued has landed before the CTA may exit
-      for (int sl = 0; sl < a.ring; ++sl)
-        if (last[sl] >= 0) tc::mbar_wait_drain(&full[sl], (last[sl] / a.ring) & 1u, a.status);
-    }
-    __syncwarp();
-    return;
-  }
-
-  // ------------------------------------------------------ consumer warps
-  // gate/up, one unit at a time (its compute overlaps the next unit's
-  // arrival): warp w owns the 16-row tile w % 2 (gate or up) for the K eighth
-  // w / 2; per group of 64 inputs four mma.sync, then the group's scale and
-  // bias.
-  bool ok = true;
-  float* red = lg;   // [2 tiles][8 K eighths][16 rows][NT] partial sums (logits are no longer needed)
-  const int lg4 = lane >> 2, lt = lane & 3;
-  const uint32_t qb = kFFeat * g.H / 2, sb = kFFeat * g.H / 32;
-  const int ngrp = g.H / kGroup;
-  {
-    const int m = warp & 1, ke = warp >> 1;
-    const int ge = ngrp / 8;                       // groups per K eighth
-    for (int i = 0; i < s.my_gu && ok; ++i) {
-      const int sl = i % a.ring;
-      if (!tc::mbar_wait(&full[sl], (i / a.ring) & 1u, abort_flag, a.status, a.wait_limit)) {
-        ok = false;
-        break;
-      }
-      int slot, f0;
-      gu_unit(s, blockIdx.x + i * gridDim.x, slot, f0);
-      unsigned tmask = 0;                            // tokens of this unit's expert
-      if (slot == 0)
-        tmask = (1u << T) - 1u;
-      else
-        for (int r = 0; r < rt.slot_cnt[slot]; ++r) tmask |= 1u << (rt.perm[rt.slot_off[slot] + r] / k);
-      const uint8_t* base = fsm + sl * a.slot_bytes;
-      const uint8_t* qrow = base + m * qb + lg4 * (g.H / 2) + lt * 8;         // rows lg4, lg4 + 8
-      const uint16_t* srow = reinterpret_cast<const uint16_t*>(base + 2 * qb + m * 2 * sb);
-      const uint16_t* brow = srow + sb / 2;
-      const bool tok_live = lg4 < T && ((tmask >> lg4) & 1u);
-      const uint4* xrow = reinterpret_cast<const uint4*>(xs + (tok_live ? lg4 : 0) * g.H) + lt * 2;
-      float y[2][NT];
-#pragma unroll
-      for (int r = 0; r < 2; ++r)
-#pragma unroll
-        for (int t = 0; t < NT; ++t) y[r][t] = 0.f;
-      for (int G = ke * ge; G < (ke + 1) * ge; ++G) {
-        const uint2 qa = *reinterpret_cast<const uint2*>(qrow + G * 32);
-        const uint2 qc = *reinterpret_cast<const uint2*>(qrow + 8 * (g.H / 2) + G * 32);
-        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-        const uint4 xb0 = tok_live ? xrow[G * 8] : z, xb1 = tok_live ? xrow[G * 8 + 1] : z;
-        float d[4];
-        group_dot(d, qa, qc, xb0, xb1);
-        if (lt == 0) {   // columns 0, 1 = tokens 0, 1
-#pragma unroll
-          for (int r = 0; r < 2; ++r) {
-            const int row = lg4 + 8 * r;
-            const float sc = bf16_bits_to_float(srow[row * ngrp + G]);
-            const float bi = bf16_bits_to_float(brow[row * ngrp + G]);
-#pragma unroll
-            for (int t = 0; t < NT; ++t)
-              if (t < T) {
-                const float X = xsum[t * ngrp + G];
-                y[r][t] = fmaf(sc, d[2 * r + t] - 128.f * X, fmaf(bi, X, y[r][t]));
-              }
-          }
-        }
-      }
-      // every read of the unit's slot is done: release it
-      tc::fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&empty[sl]);
-      if (lt == 0)
-#pragma unroll
-        for (int r = 0; r < 2; ++r)
-#pragma unroll
-          for (int t = 0; t < NT; ++t) red[((m * 8 + ke) * 16 + lg4 + 8 * r) * NT + t] = y[r][t];
-      consumers_sync();
-      // h = bf16(silu(g) * u) for (feature, token); K eighths summed in order
-      if (threadIdx.x < kFFeat * T) {
-        const int f = threadIdx.x / T, t = threadIdx.x % T;
-        bool member = slot == 0;
-        int pos = t;
-        for (int r = 0; r < (slot == 0 ? 0 : rt.slot_cnt[slot]); ++r)
-          if (rt.perm[rt.slot_off[slot] + r] / k == t) {
-            member = true;
-            pos = rt.slot_off[slot] + r;
-          }
-        if (member) {
-          float gs = 0.f, us = 0.f;
-#pragma unroll
-          for (int e8 = 0; e8 < 8; ++e8) {
-            gs += red[((0 * 8 + e8) * 16 + f) * NT + t];
-            us += red[((1 * 8 + e8) * 16 + f) * NT + t];
-          }
-          const uint16_t hv = float_to_bf16_bits(silu(gs) * us);
-          if (slot == 0)
-            a.h_s[static_cast<size_t>(t) * g.Is + f0 + f] = hv;
-          else
-            a.h[static_cast<size_t>(pos) * g.I + f0 + f] = hv;
-        }
-      }
-      consumers_sync();   // red is reused by the next unit
-    }
-  }
-  // Every h row is written: grid barrier (consumer thread 0 of each CTA).
-  consumers_sync();
-  if (threadIdx.x == 0) {
-    if (!ok || !grid_barrier(a.bar, 2u * gridDim.x, a.status, a.wait_limit)) rt.abort = 1;
-    grid_exit(a.bar, gridDim.x);
-  }
-  consumers_sync();
-  if (rt.abort) return;
-
-  if (s.my_blocks > 0) {
-    // stage every h row (routed rows I wide, shared rows Is wide) in the
-    // interleaved K order, and its sums over groups of 64
-    const int tid = threadIdx.x, nthr = kFWarps * 32;
-    const int vmax = Kmax / 8;
-    for (int i = tid; i < (Tk + T) * vmax; i += nthr) {
-      const int r = i / vmax, u = i - r * vmax;
-      const bool shr = r >= Tk;
-      if (u * 8 >= (shr ? g.Is : g.I)) continue;
-      const uint16_t* src = shr ? a.h_s + static_cast<size_t>(r - Tk) * g.Is : a.h + static_cast<size_t>(r) * g.I;
-      reinterpret_cast<uint4*>(hs + static_cast<size_t>(r) * Kmax)[u] =
-          interleave8(__ldcg(reinterpret_cast<const uint4*>(src) + u));
-    }
     consumers_sync();
-    const int kg = Kmax / kGroup;
-    for (int i = tid; i < (Tk + T) * kg; i += nthr) {
-      const int r = i / kg, G = i % kg;
-      const int K = r >= Tk ? g.Is : g.I;
-      if (G * kGroup < K) {
-        const uint4* r4 = reinterpret_cast<const uint4*>(hs + static_cast<size_t>(r) * Kmax) + G * 8;
-        float sum = 0.f;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint4 v = r4[j];
-          sum += ((bf16_lo(v.x) + bf16_hi(v.x)) + (bf16_lo(v.y) + bf16_hi(v.y))) +
-                 ((bf16_lo(v.z) + bf16_hi(v.z)) + (bf16_lo(v.w) + bf16_hi(v.w)));
-        }
-        hsum[i] = sum;
-      }
-    }
-    consumers_sync();
-  }
-  // down units: warp w owns expert slot w % 8 of the unit (16 dims x K) for
-  // the K half w / 8; lanes hold rows (dims) lg4, lg4 + 8 and tokens 0, 1
-  {
-    const int jj = warp & 7, kh = warp >> 3;
-    const int kg = Kmax / kGroup;
-    float* redd = lg;   // [8 slots][2 K halves][16 dims][NT]
-    for (int di = 0; di < s.my_blocks * s.n_down_parts && ok; ++di) {
-      const int i = s.my_gu + di;
-      const int sl = i % a.ring;
-      if (!tc::mbar_wait(&full[sl], (i / a.ring) & 1u, abort_flag, a.status, a.wait_limit)) {
-        ok = false;
-        break;
-      }
-      const int bl = di / s.n_down_parts;
-      const int j0 = (di % s.n_down_parts) * s.spd, nj = min(s.spd, s.n_slots - j0);
-      const bool live = jj < nj;
-      const int j = j0 + jj;
-      const int K = j == 0 ? g.Is : g.I;
-      const int ng = K / kGroup, gh = ng / 2;       // groups, groups per K half
-      const int nt = live ? rt.slot_cnt[j] : 0;
-      const int pos0 = live ? rt.slot_off[j] : 0;
-      float y[2][NT];
-#pragma unroll
-      for (int r = 0; r < 2; ++r)
-#pragma unroll
-        for (int t = 0; t < NT; ++t) y[r][t] = 0.f;
-      if (live) {
-        const uint8_t* base = fsm + sl * a.slot_bytes + jj * (9 * Kmax);
-        const uint8_t* qrow = base + lg4 * (K / 2) + lt * 8;
-        const uint16_t* srow = reinterpret_cast<const uint16_t*>(base + 8 * Kmax);
-        const uint16_t* brow = reinterpret_cast<const uint16_t*>(base + 8 * Kmax + Kmax / 2);
-        const bool tok_live = lg4 < nt;
-        const int hr = pos0 + (tok_live ? lg4 : 0);
-        const uint4* hrow = reinterpret_cast<const uint4*>(hs + static_cast<size_t>(hr) * Kmax) + lt * 2;
-        for (int G = kh * gh; G < (kh + 1) * gh; ++G) {
-          const uint2 qa = *reinterpret_cast<const uint2*>(qrow + G * 32);
-          const uint2 qc = *reinterpret_cast<const uint2*>(qrow + 8 * (K / 2) + G * 32);
+    if (tid == 0) tc::mbar_arrive(ready);   // the producer may now schedule this layer's units
+    const Sched s = make_sched(a, rt.n_act);
+
+    // -------------------------------------------------------------- phase C
+    // gate/up, one unit at a time (its compute overlaps the next unit's
+    // arrival): warp w owns the 16-row tile w % 2 (gate or up) for the K
+    // eighth w / 2; per group of 64 inputs four mma.sync, then the group's
+    // scale and bias for the lane's two token columns.
+    float* red = lg;   // [2 tiles][8 K eighths][16 rows][NT] partial sums (logits are no longer needed)
+    {
+      const int m = warp & 1, ke = warp >> 1;
+      const int ge = ngrp / 8;                       // groups per K eighth
+      for (int i = 0; i < s.my_gu; ++i, ++fill) {
+        const int sl = static_cast<int>(fill % a.ring);
+        const bool got =
+            __all_sync(0xffffffffu, tc::mbar_wait(&full[sl], (fill / a.ring) & 1u, abort_flag, a.status, a.wait_limit));
+        int slot, f0;
+        gu_unit(s, blockIdx.x + i * G, slot, f0);
+        unsigned tmask = 0;                            // tokens of this unit's expert
+        if (slot == 0)
+          tmask = (1u << T) - 1u;
+        else
+          for (int r = 0; r < rt.slot_cnt[slot]; ++r) tmask |= 1u << (rt.perm[rt.slot_off[slot] + r] / k);
+        const uint8_t* ub = fsm + sl * a.slot_bytes;
+        const uint8_t* qrow = ub + m * qb + lg4 * (g.H / 2) + lt * 8;         // rows lg4, lg4 + 8
+        const uint16_t* srow = reinterpret_cast<const uint16_t*>(ub + 2 * qb + m * 2 * sb);
+        const uint16_t* brow = srow + sb / 2;
+        const bool tok_live = lg4 < T && ((tmask >> lg4) & 1u);
+        const uint4* xrow = reinterpret_cast<const uint4*>(xs + (tok_live ? lg4 : 0) * g.H) + lt * 2;
+        float y[2][2] = {{0.f, 0.f}, {0.f, 0.f}};     // [row lg4 / lg4 + 8][token 2 lt / 2 lt + 1]
+        for (int G8 = ke * ge; got && G8 < (ke + 1) * ge; ++G8) {
+          const uint2 qa = *reinterpret_cast<const uint2*>(qrow + G8 * 32);
+          const uint2 qc = *reinterpret_cast<const uint2*>(qrow + 8 * (g.H / 2) + G8 * 32);
           const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-          const uint4 hb0 = tok_live ? hrow[G * 8] : z, hb1 = tok_live ? hrow[G * 8 + 1] : z;
+          const uint4 xb0 = tok_live ? xrow[G8 * 8] : z, xb1 = tok_live ? xrow[G8 * 8 + 1] : z;
           float d[4];
-          group_dot(d, qa, qc, hb0, hb1);
-          if (lt == 0) {
+          group_dot(d, qa, qc, xb0, xb1);
 #pragma unroll
-            for (int r = 0; r < 2; ++r) {
-              const int row = lg4 + 8 * r;
-              const float sc = bf16_bits_to_float(srow[row * ng + G]);
-              const float bi = bf16_bits_to_float(brow[row * ng + G]);
+          for (int c = 0; c < 2; ++c) {
+            const int t = 2 * lt + c;
+            if (t < T) {
+              const float X = xsum[t * ngrp + G8];
 #pragma unroll
-              for (int t = 0; t < NT; ++t)
-                if (t < nt) {
-                  const float X = hsum[(pos0 + t) * kg + G];
-                  y[r][t] = fmaf(sc, d[2 * r + t] - 128.f * X, fmaf(bi, X, y[r][t]));
-                }
+              for (int r = 0; r < 2; ++r) {
+                const int row = lg4 + 8 * r;
+                const float sc = bf16_bits_to_float(srow[row * ngrp + G8]);
+                const float bi = bf16_bits_to_float(brow[row * ngrp + G8]);
+                y[r][c] = fmaf(sc, d[2 * r + c] - 128.f * X, fmaf(bi, X, y[r][c]));
+              }
             }
           }
         }
-      }
-      tc::fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&empty[sl]);
-      if (lt == 0)
+        // every read of the unit's slot is done: release it (a slot that never
+        // filled is not handed back: the producer is stopping as well)
+        tc::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && got) tc::mbar_arrive(&empty[sl]);
 #pragma unroll
-        for (int r = 0; r < 2; ++r)
+        for (int c = 0; c < 2; ++c)
+          if (2 * lt + c < T)
 #pragma unroll
-          for (int t = 0; t < NT; ++t) redd[((jj * 2 + kh) * 16 + lg4 + 8 * r) * NT + t] = y[r][t];
+            for (int r = 0; r < 2; ++r) red[((m * 8 + ke) * 16 + lg4 + 8 * r) * NT + 2 * lt + c] = y[r][c];
+        consumers_sync();
+        // h = bf16(silu(g) * u) for (feature, token); K eighths summed in order
+        if (tid < kFFeat * T && !rt.abort) {
+          const int f = tid / T, t = tid % T;
+          bool member = slot == 0;
+          int pos = t;
+          for (int r = 0; r < (slot == 0 ? 0 : rt.slot_cnt[slot]); ++r)
+            if (rt.perm[rt.slot_off[slot] + r] / k == t) {
+              member = true;
+              pos = rt.slot_off[slot] + r;
+            }
+          if (member) {
+            float gs = 0.f, us = 0.f;
+#pragma unroll
+            for (int e8 = 0; e8 < 8; ++e8) {
+              gs += red[((0 * 8 + e8) * 16 + f) * NT + t];
+              us += red[((1 * 8 + e8) * 16 + f) * NT + t];
+            }
+            const uint16_t hv = float_to_bf16_bits(silu(gs) * us);
+            if (slot == 0)
+              a.h_s[static_cast<size_t>(t) * g.Is + f0 + f] = hv;
+            else
+              a.h[static_cast<size_t>(pos) * g.I + f0 + f] = hv;
+          }
+        }
+        consumers_sync();   // red is reused by the next unit
+      }
+    }
+    // Every h row is written: grid barrier.
+    consumers_sync();
+    if (tid == 0) {
+      if (rt.abort || !grid_barrier(a.bar, (++nbar) * G, a.status, a.wait_limit)) rt.abort = 1;
+    }
+    consumers_sync();
+    if (rt.abort) break;
+
+    // -------------------------------------------------------------- phase D
+    if (s.my_blocks > 0) {
+      // stage every h row (routed rows I wide, shared rows Is wide) in the
+      // interleaved K order, and its sums over groups of 64
+      const int vmax = Kmax / 8;
+      for (int i = tid; i < (Tk + T) * vmax; i += nthr) {
+        const int r = i / vmax, u = i - r * vmax;
+        const bool shr = r >= Tk;
+        if (u * 8 >= (shr ? g.Is : g.I)) continue;
+        const uint16_t* hsrc =
+            shr ? a.h_s + static_cast<size_t>(r - Tk) * g.Is : a.h + static_cast<size_t>(r) * g.I;
+        reinterpret_cast<uint4*>(hs + static_cast<size_t>(r) * Kmax)[u] =
+            interleave8(__ldcg(reinterpret_cast<const uint4*>(hsrc) + u));
+      }
       consumers_sync();
-      // y rows of this unit's slots: both K halves summed in order
-      for (int q = threadIdx.x; q < nj * kFDims * NT; q += kFWarps * 32) {
-        const int js = q / (kFDims * NT), d = (q / NT) % kFDims, t = q % NT;
-        const int jx = j0 + js;
-        if (t < rt.slot_cnt[jx])
-          ys[((rt.slot_off[jx] + t) * s.my_blocks + bl) * kFDims + d] =
-              redd[((js * 2 + 0) * 16 + d) * NT + t] + redd[((js * 2 + 1) * 16 + d) * NT + t];
+      const int kg = Kmax / kGroup;
+      for (int i = tid; i < (Tk + T) * kg; i += nthr) {
+        const int r = i / kg, G8 = i % kg;
+        const int K = r >= Tk ? g.Is : g.I;
+        if (G8 * kGroup < K) {
+          const uint4* r4 = reinterpret_cast<const uint4*>(hs + static_cast<size_t>(r) * Kmax) + G8 * 8;
+          float sum = 0.f;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint4 v = r4[j];
+            sum += ((bf16_lo(v.x) + bf16_hi(v.x)) + (bf16_lo(v.y) + bf16_hi(v.y))) +
+                   ((bf16_lo(v.z) + bf16_hi(v.z)) + (bf16_lo(v.w) + bf16_hi(v.w)));
+          }
+          hsum[i] = sum;
+        }
       }
       consumers_sync();
     }
-  }
-  if (!ok) return;
-  // combine: out[t, d] = bf16( sum_j w[t,j] * y[inv_perm[t k + j]][d] + sigma_t * y[T k + t][d] )
-  for (int i = threadIdx.x; i < T * s.my_blocks * kFDims; i += kFWarps * 32) {
-    const int t = i / (s.my_blocks * kFDims), rem = i % (s.my_blocks * kFDims);
-    const int bl = rem / kFDims, d = rem % kFDims;
-    float acc = 0.f;
-    for (int j = 0; j < k; ++j)
-      acc = fmaf(rt.w[t * k + j], ys[(rt.inv_perm[t * k + j] * s.my_blocks + bl) * kFDims + d], acc);
-    acc = fmaf(rt.sigma[t], ys[((Tk + t) * s.my_blocks + bl) * kFDims + d], acc);
-    const int blk = blockIdx.x + bl * gridDim.x;
-    a.out[static_cast<size_t>(t) * g.H + blk * kFDims + d] = float_to_bf16_bits(acc);
-  }
-  if (blockIdx.x == 0) {
-    // routing outputs (off the other CTAs' critical path)
-    for (int i = threadIdx.x; i < n; i += kFWarps * 32) {
-      a.r.topk_idx[i] = rt.idx[i];
-      a.r.topk_w[i] = rt.w[i];
-      a.r.perm[i] = rt.perm[i];
-      a.r.inv_perm[i] = rt.inv_perm[i];
-    }
-    for (int e = threadIdx.x; e <= E; e += kFWarps * 32) {
-      int c = 0, below = 0;
-      for (int i = 0; i < n; ++i) {
-        c += rt.idx[i] == e ? 1 : 0;
-        below += rt.idx[i] < e ? 1 : 0;
+    // down units: warp w owns expert slot w % 8 of the unit (16 dims x K) for
+    // the K half w / 8; lanes hold rows (dims) lg4, lg4 + 8 and token columns
+    // 2 lt, 2 lt + 1
+    {
+      const int jj = warp & 7, kh = warp >> 3;
+      const int kg = Kmax / kGroup;
+      float* redd = lg;   // [8 slots][2 K halves][16 dims][NT]
+      for (int di = 0; di < s.my_blocks * s.n_down_parts; ++di, ++fill) {
+        const int sl = static_cast<int>(fill % a.ring);
+        const bool got =
+            __all_sync(0xffffffffu, tc::mbar_wait(&full[sl], (fill / a.ring) & 1u, abort_flag, a.status, a.wait_limit));
+        const int bl = di / s.n_down_parts;
+        const int j0 = (di % s.n_down_parts) * s.spd, nj = min(s.spd, s.n_slots - j0);
+        const bool jlive = got && jj < nj;
+        const int j = j0 + jj;
+        const int K = j == 0 ? g.Is : g.I;
+        const int ng = K / kGroup, gh = ng / 2;       // groups, groups per K half
+        const int nt = jlive ? rt.slot_cnt[j] : 0;
+        const int pos0 = jlive ? rt.slot_off[j] : 0;
+        float y[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+        if (jlive) {
+          const uint8_t* ub = fsm + sl * a.slot_bytes + jj * (9 * Kmax);
+          const uint8_t* qrow = ub + lg4 * (K / 2) + lt * 8;
+          const uint16_t* srow = reinterpret_cast<const uint16_t*>(ub + 8 * Kmax);
+          const uint16_t* brow = reinterpret_cast<const uint16_t*>(ub + 8 * Kmax + Kmax / 2);
+          const bool tok_live = lg4 < nt;
+          const int hr = pos0 + (tok_live ? lg4 : 0);
+          const uint4* hrow = reinterpret_cast<const uint4*>(hs + static_cast<size_t>(hr) * Kmax) + lt * 2;
+          for (int G8 = kh * gh; G8 < (kh + 1) * gh; ++G8) {
+            const uint2 qa = *reinterpret_cast<const uint2*>(qrow + G8 * 32);
+            const uint2 qc = *reinterpret_cast<const uint2*>(qrow + 8 * (K / 2) + G8 * 32);
+            const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+            const uint4 hb0 = tok_live ? hrow[G8 * 8] : z, hb1 = tok_live ? hrow[G8 * 8 + 1] : z;
+            float d[4];
+            group_dot(d, qa, qc, hb0, hb1);
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              const int t = 2 * lt + c;
+              if (t < nt) {
+                const float X = hsum[(pos0 + t) * kg + G8];
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                  const int row = lg4 + 8 * r;
+                  const float sc = bf16_bits_to_float(srow[row * ng + G8]);
+                  const float bi = bf16_bits_to_float(brow[row * ng + G8]);
+                  y[r][c] = fmaf(sc, d[2 * r + c] - 128.f * X, fmaf(bi, X, y[r][c]));
+                }
+              }
+            }
+          }
+        }
+        tc::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && got) tc::mbar_arrive(&empty[sl]);
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+          if (2 * lt + c < nt)
+#pragma unroll
+            for (int r = 0; r < 2; ++r) redd[((jj * 2 + kh) * 16 + lg4 + 8 * r) * NT + 2 * lt + c] = y[r][c];
+        consumers_sync();
+        // y rows of this unit's slots: both K halves summed in order
+        for (int q = tid; q < nj * kFDims * NT; q += nthr) {
+          const int js = q / (kFDims * NT), d = (q / NT) % kFDims, t = q % NT;
+          const int jx = j0 + js;
+          if (t < rt.slot_cnt[jx])
+            ys[((rt.slot_off[jx] + t) * s.my_blocks + bl) * kFDims + d] =
+                redd[((js * 2 + 0) * 16 + d) * NT + t] + redd[((js * 2 + 1) * 16 + d) * NT + t];
+        }
+        consumers_sync();
       }
-      if (e < E) a.r.counts[e] = c;
-      a.r.offsets[e] = below;
     }
-    for (int jx = threadIdx.x; jx < rt.n_act; jx += kFWarps * 32) a.active[jx] = rt.slot_e[1 + jx];
-    if (threadIdx.x < T) a.r.sigma[threadIdx.x] = rt.sigma[threadIdx.x];
-    if (threadIdx.x == 0) {
-      a.active[rt.n_act] = E;
-      *a.n_active = rt.n_act + 1;
+    consumers_sync();
+    if (rt.abort) break;
+    // combine: out[t, d] = bf16( sum_j w[t,j] * y[inv_perm[t k + j]][d] + sigma_t * y[T k + t][d] );
+    // between layers the CTA also sums the squares of its bf16 outputs per token
+    uint16_t* dst = last ? a.out : a.y;
+    for (int i = tid; i < T * s.my_blocks * kFDims; i += nthr) {
+      const int t = i / (s.my_blocks * kFDims), rem = i % (s.my_blocks * kFDims);
+      const int bl = rem / kFDims, d = rem % kFDims;
+      float acc = 0.f;
+      for (int j = 0; j < k; ++j)
+        acc = fmaf(rt.w[t * k + j], ys[(rt.inv_perm[t * k + j] * s.my_blocks + bl) * kFDims + d], acc);
+      acc = fmaf(rt.sigma[t], ys[((Tk + t) * s.my_blocks + bl) * kFDims + d], acc);
+      const int blk = blockIdx.x + bl * G;
+      const uint16_t ov = float_to_bf16_bits(acc);
+      const size_t o = static_cast<size_t>(t) * g.H + blk * kFDims + d;
+      dst[o] = ov;
+      if (a.trace) a.trace[(2 * l + 1) * act + o] = ov;
+      if (!last) lg[i] = bf16_bits_to_float(ov) * bf16_bits_to_float(ov);
+    }
+    if (!last) {
+      consumers_sync();
+      if (tid < T) {
+        float ss = 0.f;
+        for (int q = 0; q < s.my_blocks * kFDims; ++q) ss += lg[tid * s.my_blocks * kFDims + q];
+        __stcg(a.sumsq + blockIdx.x * kFMaxT + tid, ss);
+      }
+    } else if (blockIdx.x == 0 && a.r.topk_idx) {
+      // routing outputs of the last layer (off the other CTAs' critical path)
+      for (int i = tid; i < n; i += nthr) {
+        a.r.topk_idx[i] = rt.idx[i];
+        a.r.topk_w[i] = rt.w[i];
+        a.r.perm[i] = rt.perm[i];
+        a.r.inv_perm[i] = rt.inv_perm[i];
+      }
+      for (int e = tid; e <= E; e += nthr) {
+        int c = 0, below = 0;
+        for (int i = 0; i < n; ++i) {
+          c += rt.idx[i] == e ? 1 : 0;
+          below += rt.idx[i] < e ? 1 : 0;
+        }
+        if (e < E) a.r.counts[e] = c;
+        a.r.offsets[e] = below;
+      }
+      for (int jx = tid; jx < rt.n_act; jx += nthr) a.active[jx] = rt.slot_e[1 + jx];
+      if (tid < T) a.r.sigma[tid] = rt.sigma[tid];
+      if (tid == 0) {
+        a.active[rt.n_act] = E;
+        *a.n_active = rt.n_act + 1;
+      }
+    }
+    // the layer's outputs are complete once every CTA passes the next barrier
+    if (!last) {
+      consumers_sync();
+      if (tid == 0) {
+        if (rt.abort || !grid_barrier(a.bar, (++nbar) * G, a.status, a.wait_limit)) rt.abort = 1;
+      }
+      consumers_sync();
+      if (rt.abort) break;
     }
   }
+  // (after an abort, rt.abort also stops a producer still waiting for a
+  // layer that will not come)
+  if (tid == 0) grid_exit(a.bar, gridDim.x);
 }
 
 int fused_grid() {
@@ -768,6 +891,50 @@ int fused_grid() {
   return n;
 }
 
+// Shared-memory carve-up of one launch (identical for every layer).
+struct FusedLayout {
+  int ring, slot_bytes, spd, rows_per_cta;
+  int off_bar, off_wr, off_xs, off_xsum, off_lg, off_rt, off_y, off_nrm, total;
+};
+
+FusedLayout fused_layout(const Geometry& g, int G) {
+  FusedLayout f{};
+  const int Kmax = g.I > g.Is ? g.I : g.Is;
+  f.slot_bytes = 18 * g.H;                                   // one gate/up unit
+  f.spd = f.slot_bytes / (9 * Kmax);
+  if (f.spd > kFMaxSpd) f.spd = kFMaxSpd;
+  f.rows_per_cta = (g.E + 1 + G - 1) / G;
+  const int rows = g.T * g.k + g.T;
+  const int blocks_per_cta = (g.H / kFDims + G - 1) / G;
+  auto al = [](int v) { return (v + 127) / 128 * 128; };
+  const int lg_floats = max(max(g.T * (g.E + 1), f.rows_per_cta * kFWarps * kFMaxT),
+                            max(16 * 16 * kFMaxT, g.T * blocks_per_cta * kFDims));
+  const int stage_bytes = max(g.T * g.H * 2, rows * Kmax * 2);
+  const int sums_bytes = max(g.T * (g.H / kGroup) * 4, rows * (Kmax / kGroup) * 4);
+  const int fixed = al((2 * kFRingMax + 3) * 8) + al(f.rows_per_cta * g.H * 2) + al(stage_bytes) + al(sums_bytes) +
+                    al(lg_floats * 4) + al(static_cast<int>(sizeof(RouteSmem))) +
+                    al(rows * blocks_per_cta * kFDims * 4) + al(kFMaxT * 4);
+  f.ring = (227 * 1024 - fixed) / f.slot_bytes;
+  if (f.ring > kFRingMax) f.ring = kFRingMax;
+  int off = 0;
+  auto take = [&](int bytes) {
+    const int o = off;
+    off += al(bytes);
+    return o;
+  };
+  take(f.ring * f.slot_bytes);
+  f.off_bar = take((2 * kFRingMax + 3) * 8);
+  f.off_wr = take(f.rows_per_cta * g.H * 2);
+  f.off_xs = take(stage_bytes);
+  f.off_xsum = take(sums_bytes);
+  f.off_lg = take(lg_floats * 4);
+  f.off_rt = take(static_cast<int>(sizeof(RouteSmem)));
+  f.off_y = take(rows * blocks_per_cta * kFDims * 4);
+  f.off_nrm = take(kFMaxT * 4);
+  f.total = off;
+  return f;
+}
+
 }  // namespace
 
 bool decode_fused_supported(const Geometry& g) {
@@ -775,17 +942,30 @@ bool decode_fused_supported(const Geometry& g) {
   if (g.H % 1024 || g.H > 2048) return false;
   if (g.I % kFFeat || g.Is % kFFeat) return false;
   const int Kmax = g.I > g.Is ? g.I : g.Is;
-  return 9 * Kmax <= 18 * g.H;   // at least one expert slot per down unit
+  if (9 * Kmax > 18 * g.H) return false;                  // at least one expert slot per down unit
+  const int G = fused_grid();
+  if (G > kFMaxGrid || G > kFusedMaxGrid) return false;
+  if ((g.E + 1 + G - 1) / G > kFMaxRouterRows) return false;
+  const FusedLayout f = fused_layout(g, G);
+  return f.ring >= 2 && f.total <= 227 * 1024;
 }
 
-cudaError_t launch_decode_fused(const Geometry& g, const LayerPtr& L, const uint16_t* x, uint16_t* out,
-                                const RoutingPtrs& r, int32_t* active, int32_t* n_active, float* logits,
-                                uint16_t* h, uint16_t* h_s, unsigned* bar, int* status, cudaStream_t s) {
+int decode_fused_max_layers() { return kFMaxLayers; }
+
+cudaError_t launch_decode_fused(const Geometry& g, const LayerPtr* layers, int n_layers, const uint16_t* x,
+                                uint16_t* out, uint16_t* y, float* sumsq, uint16_t* trace, float eps,
+                                const RoutingPtrs& r, int32_t* active, int32_t* n_active, float* logits, uint16_t* h,
+                                uint16_t* h_s, unsigned* bar, int* status, cudaStream_t s) {
+  if (n_layers < 1 || n_layers > kFMaxLayers || !decode_fused_supported(g)) return cudaErrorInvalidValue;
   FusedArgs a{};
   a.g = g;
-  a.L = L;
+  a.n_layers = n_layers;
+  a.eps = eps;
   a.x = x;
   a.out = out;
+  a.y = y;
+  a.sumsq = sumsq;
+  a.trace = trace;
   a.r = r;
   a.active = active;
   a.n_active = n_active;
@@ -795,47 +975,31 @@ cudaError_t launch_decode_fused(const Geometry& g, const LayerPtr& L, const uint
   a.bar = bar;
   a.status = status;
   a.wait_limit = wait_limit_cycles();
+  for (int l = 0; l < n_layers; ++l) a.layers[l] = layers[l];
   const int G = fused_grid();
-  const int Kmax = g.I > g.Is ? g.I : g.Is;
-  a.slot_bytes = 18 * g.H;                                   // one gate/up unit
-  a.spd = a.slot_bytes / (9 * Kmax);
-  if (a.spd > kFMaxSpd) a.spd = kFMaxSpd;
-  const int rows = g.T * g.k + g.T;
-  const int blocks_per_cta = (g.H / kFDims + G - 1) / G;
-  auto al = [](int v) { return (v + 127) / 128 * 128; };
-  int off = 0;
-  auto take = [&](int bytes) {
-    const int o = off;
-    off += al(bytes);
-    return o;
-  };
-  // lg: logits, then the router partials, then the dot-product reductions
-  const int lg_floats = max(max(g.T * (g.E + 1), (g.E + 1 + G - 1) / G * kFWarps * kFMaxT), 16 * 16 * kFMaxT);
-  const int fixed = al(2 * kFRingMax * 8) + al(g.T * g.H * 2) + al(g.T * (g.H / kGroup) * 4) + al(rows * Kmax * 2) +
-                    al(rows * (Kmax / kGroup) * 4) + al(lg_floats * 4) +
-                    al(static_cast<int>(sizeof(RouteSmem))) + al(rows * blocks_per_cta * kFDims * 4);
-  const int budget = 227 * 1024 - fixed;
-  a.ring = budget / a.slot_bytes;
-  if (a.ring > kFRingMax) a.ring = kFRingMax;
-  if (a.ring < 2 || a.spd < 1) return cudaErrorInvalidValue;
-  take(a.ring * a.slot_bytes);
-  a.off_bar = take(2 * kFRingMax * 8);
-  a.off_xs = take(g.T * g.H * 2);
-  a.off_xsum = take(g.T * (g.H / kGroup) * 4);
-  a.off_hs = take(rows * Kmax * 2);
-  a.off_hsum = take(rows * (Kmax / kGroup) * 4);
-  a.off_lg = take(lg_floats * 4);
-  a.off_rt = take(static_cast<int>(sizeof(RouteSmem)));
-  a.off_y = take(rows * blocks_per_cta * kFDims * 4);
-  const int smem = off;
-  const void* fn = g.T == 1 ? reinterpret_cast<const void*>(decode_fused_kernel<1>)
-                            : reinterpret_cast<const void*>(decode_fused_kernel<2>);
-  cudaError_t e = ensure_smem(fn, smem);
+  const FusedLayout f = fused_layout(g, G);
+  a.ring = f.ring;
+  a.slot_bytes = f.slot_bytes;
+  a.spd = f.spd;
+  a.rows_per_cta = f.rows_per_cta;
+  a.off_bar = f.off_bar;
+  a.off_wr = f.off_wr;
+  a.off_xs = f.off_xs;
+  a.off_xsum = f.off_xsum;
+  a.off_lg = f.off_lg;
+  a.off_rt = f.off_rt;
+  a.off_y = f.off_y;
+  a.off_nrm = f.off_nrm;
+  const void* fn = g.T == 1   ? reinterpret_cast<const void*>(decode_fused_kernel<1>)
+                   : g.T == 2 ? reinterpret_cast<const void*>(decode_fused_kernel<2>)
+                   : g.T <= 4 ? reinterpret_cast<const void*>(decode_fused_kernel<4>)
+                              : reinterpret_cast<const void*>(decode_fused_kernel<8>);
+  cudaError_t e = ensure_smem(fn, f.total);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(G);
   cfg.blockDim = dim3(kFThreads);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = f.total;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;
@@ -843,7 +1007,9 @@ cudaError_t launch_decode_fused(const Geometry& g, const LayerPtr& L, const uint
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (g.T == 1) return cudaLaunchKernelEx(&cfg, decode_fused_kernel<1>, a);
-  return cudaLaunchKernelEx(&cfg, decode_fused_kernel<2>, a);
+  if (g.T == 2) return cudaLaunchKernelEx(&cfg, decode_fused_kernel<2>, a);
+  if (g.T <= 4) return cudaLaunchKernelEx(&cfg, decode_fused_kernel<4>, a);
+  return cudaLaunchKernelEx(&cfg, decode_fused_kernel<8>, a);
 }
 
 }  // namespace moe

@@ -135,12 +135,19 @@ cudaError_t launch_decode_down_combine(const Geometry& g, const LayerPtr& L, con
                                        const int32_t* inv_perm, const float* sigma, uint16_t* out,
                                        cudaStream_t s);
 
-// decode_fused.cu: the whole decode layer in one cooperative launch (T <= 2,
-// H a multiple of 1024 up to 2048).  bar: two zeroed workspace words (grid
-// barrier arrivals and generation); logits: workspace [T, E+1] FP32.
+// decode_fused.cu: a stack of 1..decode_fused_max_layers() decode layers
+// (T <= 8, H = 1024 or 2048) in one cooperative launch; layer l > 0 takes
+// RMSNorm(eps) of layer l-1's output.  y: workspace [T, H] bf16 (outputs
+// between layers); sumsq: workspace [kFusedMaxGrid][8] FP32; bar: two zeroed
+// workspace words (grid barrier arrivals and exits); logits: workspace
+// [T, E+1] FP32; trace: NULL or [n_layers][2][T][H]; r.topk_idx NULL: no
+// routing outputs (else those of the last layer).
+constexpr int kFusedMaxGrid = 1024;
 bool decode_fused_supported(const Geometry& g);
-cudaError_t launch_decode_fused(const Geometry& g, const LayerPtr& L, const uint16_t* x, uint16_t* out,
-                                const RoutingPtrs& r, int32_t* active, int32_t* n_active, float* logits,
-                                uint16_t* h, uint16_t* h_s, unsigned* bar, int* status, cudaStream_t s);
+int decode_fused_max_layers();
+cudaError_t launch_decode_fused(const Geometry& g, const LayerPtr* layers, int n_layers, const uint16_t* x,
+                                uint16_t* out, uint16_t* y, float* sumsq, uint16_t* trace, float eps,
+                                const RoutingPtrs& r, int32_t* active, int32_t* n_active, float* logits, uint16_t* h,
+                                uint16_t* h_s, unsigned* bar, int* status, cudaStream_t s);
 
 }  // namespace moe

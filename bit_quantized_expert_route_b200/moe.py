@@ -276,7 +276,7 @@ def moe_forward_profiled(layer: MoELayer, x: torch.Tensor, out: torch.Tensor, wo
     _check(library().moe_forward_profiled(ctypes.byref(layer.desc), x.data_ptr(), T, out.data_ptr(),
                                           workspace.data_ptr(), workspace.numel(), _stream(stream), ms,
                                           ctypes.byref(n)), "moe_forward_profiled")
-    names = PREFILL_STAGES if T > 64 else (FUSED_DECODE_STAGES if n.value == 1 else DECODE_STAGES)
+    names = {1: FUSED_DECODE_STAGES, len(DECODE_STAGES): DECODE_STAGES, len(PREFILL_STAGES): PREFILL_STAGES}[n.value]
     return {names[i]: float(ms[i]) for i in range(n.value)}
 
 

@@ -174,7 +174,11 @@ MOE_API int moe_route(const moe_layer_desc* layer, const moe_bf16* x, int T, moe
  * bf16 products and FP32 accumulation, and one always-on shared expert.
  * x, out: device bf16 [T, H], 16-byte aligned, not overlapping.
  * r: optional (NULL = keep routing in the workspace).
- * 1 <= T <= 65536; T <= 64 runs the decode kernels of moe_decode. */
+ * 1 <= T <= 65536.  For T <= 2 with H = 1024 or 2048 and 16-byte aligned
+ * scale and bias stacks it runs moe_decode's single-launch fused kernel; for
+ * every other T, the tensor-core kernels above (the GEMV kernels of
+ * moe_decode spend FP32 work on every weight for every token, which the
+ * tensor cores outrun as soon as an expert sees a few tokens). */
 MOE_API int moe_forward(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_bf16* out,
                 moe_routing* r, void* workspace, size_t workspace_bytes, moe_stream stream);
 
@@ -194,9 +198,10 @@ MOE_API int moe_decode(const moe_layer_desc* layer, const moe_bf16* x, int T, mo
  * can also be captured once as a CUDA graph and replayed:
  *   a_0 = x;  y_l = layer_l(a_l);  a_{l+1} = bf16(y_l / sqrt(mean(y_l^2) + eps))
  * (RMSNorm with weight 1 and no residual, over the bf16 values of y_l);
- * out = y_{n_layers-1}.  For T > 64 the RMSNorm is computed inside the
- * layer's combine kernel (the row's sum of squares is formed while its output
- * is written); for T <= 64 it is a separate small kernel.
+ * out = y_{n_layers-1}.  Each layer runs what moe_forward runs for T; on the
+ * tensor-core path the RMSNorm is computed inside the layer's combine kernel
+ * (the row's sum of squares is formed while its output is written), after
+ * the fused decode kernel it is a separate small kernel.
  *   layers: host array of n_layers (1..1024) descriptors with equal H, I,
  *           I_shared, E and k.
  *   x, out: device bf16 [T, H], 16-byte aligned, not overlapping.
@@ -268,11 +273,9 @@ MOE_API int moe_rmsnorm(const moe_bf16* y, moe_bf16* y_out, int T, int H, float 
 /* Stage timing (tracing).  Same as moe_forward, but records a CUDA event on
  * `stream` before the first and after every stage, waits for the stream, and
  * writes each stage's device time in milliseconds to stage_ms[0..n-1]:
- *   T > 64:  router, group (histogram+scan+scatter), gather of the grouped
- *            token rows, gate/up GEMM, down GEMM, combine
- *   T <= 64: routing (one kernel), gate/up GEMV, down GEMV + combine, or a
- *            single stage when the fused decode kernel runs (T <= 2,
- *            H = 1024 or 2048, 16-byte aligned scale and bias stacks)
+ *   tensor-core path: router, group (histogram+scan+scatter), gather of the
+ *            grouped token rows, gate/up GEMM, down GEMM, combine (6 stages)
+ *   fused decode kernel (when moe_forward uses it): one stage
  * stage_ms: host array of at least 6 floats; *n_stages receives the count.
  * The events are created and destroyed inside the call. */
 MOE_API int moe_forward_profiled(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_bf16* out,

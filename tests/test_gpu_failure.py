@@ -23,7 +23,7 @@ import torch
 from bit_quantized_expert_route_b200 import moe
 from oracle import moe_ref
 from tests.gpu_util import assert_output_close, bits_of, require_cuda, to_dev_bits
-from tests.workloads import TINY, workload
+from tests.workloads import FULL, TINY, workload
 
 pytestmark = pytest.mark.gpu
 
@@ -92,3 +92,29 @@ def test_router_wait_runs_out_and_the_next_call_is_correct():
     assert moe.moe_get_status(ws) == moe.MOE_ERR_DEVICE_TIMEOUT
     assert int(ws[:16].count_nonzero()) == 0
     _assert_next_call_correct(lay, x, L, xd, out, ws)
+
+
+@pytest.mark.parametrize("T", [1, 8])
+def test_fused_decode_waits_run_out_and_the_next_call_is_correct(T):
+    """The single-launch decode kernel's producer, consumers and grid barriers all give up
+    after one cycle; every CTA leaves (its copies landed), the grid-barrier words are reset
+    for the next launch, and the next call on the same workspace is correct."""
+    lay, x, _ = workload(82 + T, T, FULL)
+    L = moe.MoELayer.from_synth(lay)
+    xd = to_dev_bits(x)
+    out = torch.empty_like(xd)
+    ws = moe.alloc_workspace(L, T)
+    moe.moe_set_wait_limit(1)
+    try:
+        moe.moe_forward(L, xd, out, ws)
+        torch.cuda.synchronize()
+    finally:
+        moe.moe_set_wait_limit(0)
+    assert moe.moe_get_status(ws) == moe.MOE_ERR_DEVICE_TIMEOUT
+    assert int(ws[:16].count_nonzero()) == 0
+    for _ in range(2):
+        moe.moe_forward(L, xd, out, ws)
+        torch.cuda.synchronize()
+        assert moe.moe_get_status(ws) == moe.MOE_OK
+        m = moe_ref.compare(moe_ref.bf16_to_f64(bits_of(out)), moe_ref.moe_layer(x, lay, FULL.k)["out"])
+        assert m["rel_l2"] <= moe_ref.REL_L2_TOL and m["max_err_rel"] <= moe_ref.MAX_ERR_TOL, m

@@ -164,12 +164,17 @@ def test_decode_entry_rejects_large_T():
     assert e.value.code == moe.MOE_ERR_INVALID_ARG
 
 
-def test_decode_entry_equals_forward():
-    lay, x, _ = workload(8, 40, TINY)
+@pytest.mark.parametrize("dims,T", [(TINY, 40), (FULL, 12)])
+def test_decode_entry_and_forward_both_match_oracle(dims, T):
+    # moe_decode runs the GEMV kernels; moe_forward runs the tensor-core path at these T
+    lay, x, _ = workload(8, T, dims)
     L = moe.MoELayer.from_synth(lay)
-    a = run_layer(lay, x, entry="decode", dev_layer=L)
-    b = run_layer(lay, x, entry="forward", dev_layer=L)
-    np.testing.assert_array_equal(a["out"], b["out"])
+    ref = moe_ref.moe_layer(x, lay, dims.k)
+    for entry in ("decode", "forward"):
+        gpu = run_layer(lay, x, entry=entry, dev_layer=L)
+        assert gpu["status"] == 0
+        assert_routing_exact(gpu, ref)
+        assert_output_close(gpu["out"], ref["out"])
 
 
 def test_rmsnorm_matches_oracle():
@@ -191,18 +196,22 @@ def test_rmsnorm_matches_oracle():
 
 # ------------------------------------------------------------- full layer --
 
-@pytest.mark.parametrize("T", [1, 2, 3, 8, 64])
-def test_full_decode(T):
-    # T <= 2 runs the single-launch fused decode kernel, larger T the unfused kernels
+@pytest.mark.parametrize("T,entry", [(1, "forward"), (2, "forward"), (3, "forward"), (5, "forward"),
+                                     (8, "forward"), (9, "forward"), (64, "forward"),
+                                     (3, "decode"), (8, "decode"), (9, "decode"), (64, "decode")])
+def test_full_decode(T, entry):
+    # T <= 8 runs the single-launch fused decode kernel (both entries); larger
+    # T runs the tensor-core path through moe_forward and the GEMV kernels
+    # through moe_decode
     lay, x, _ = workload(10 + T, T, FULL)
     ref = moe_ref.moe_layer(x, lay, FULL.k)
-    gpu = run_layer(lay, x)
+    gpu = run_layer(lay, x, entry=entry)
     assert gpu["status"] == 0
     assert_routing_exact(gpu, ref)
     assert_output_close(gpu["out"], ref["out"])
 
 
-@pytest.mark.parametrize("T", [1, 2])
+@pytest.mark.parametrize("T", [1, 2, 8])
 def test_full_decode_zipf(T):
     lay, x, _ = workload(30 + T, T, FULL, zipf=True)
     ref = moe_ref.moe_layer(x, lay, FULL.k)

@@ -154,7 +154,10 @@ def _ulp_distance(a: np.ndarray, b: np.ndarray) -> np.ndarray:
     return np.abs(ordered(a) - ordered(b))
 
 
-@pytest.mark.parametrize("T,n_layers", [(1, 4), (8, 3), (64, 3), (65, 2), (512, 3)])
+# T <= 8: the fused decode kernel runs the stack in launches of up to 40
+# layers (42 layers: two launches and a stand-alone RMSNorm between them);
+# larger T: the tensor-core path with the RMSNorm fused into the combine.
+@pytest.mark.parametrize("T,n_layers", [(1, 4), (2, 42), (8, 3), (64, 3), (65, 2), (512, 3)])
 def test_forward_stack_matches_single_layer_calls(T, n_layers):
     """moe_forward_stack vs the per-layer entry points on the stack's own activations: every
     layer's output is bit-identical to moe_forward on the same input (same kernels), and every
