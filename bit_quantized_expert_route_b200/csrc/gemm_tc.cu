@@ -83,7 +83,7 @@ struct Cfg {
   static constexpr int BAR_OFF = OFF_OUT + OUT_BYTES;
   static constexpr int OFF_UNITS = BAR_OFF + 512;             // this CTA's chunk descriptors
   static constexpr int SMEM = OFF_UNITS + kMaxCtaUnits * 16 + 1024;   // + alignment slack
-  static constexpr int DQ_PER_STAGE = kGateUp ? 256 : 128;    // dequant threads consuming one stage (8 or 4 warps)
+  static constexpr int DQ_PER_STAGE = kGateUp ? 256 : 128;    // dequant threads consuming one stage
 };
 
 struct alignas(64) TcArgs {
@@ -110,24 +110,12 @@ struct UnitInfo {
   int e, row0, rows, f0, K, nks, wrow;   // wrow: first weight row of the tile in its matrix stack
 };
 
-// Unit of round r of this CTA.  The chunk list is sorted by size, largest
-// first, and the units are dealt in snake order (round r gives CTA b unit
-// r G + b for even r, r G + G - 1 - b for odd r): each CTA's rounds alternate
-// between larger and smaller units of the same size class, so the CTAs'
-// totals stay close and the kernel does not wait on one overloaded SM.
-// A CTA's units increase with r, so its walk ends at the first unit past the
-// list.
-__device__ __forceinline__ int snake_unit(int r) {
-  const int G = static_cast<int>(gridDim.x), b = static_cast<int>(blockIdx.x);
-  return r * G + ((r & 1) ? (G - 1 - b) : b);
-}
-
 template <bool kGateUp>
 __device__ __forceinline__ UnitInfo unit_info(const TcArgs& a, int u, int nfb, const Chunk* cache) {
-  // this CTA's units are u = snake_unit(i); their chunks were copied to
-  // shared memory at the start, so the per-stage bookkeeping of every role
-  // never waits on a global load
-  const int i = u / static_cast<int>(gridDim.x);
+  // this CTA's units are u = blockIdx.x + i * gridDim.x; their chunks were
+  // copied to shared memory at the start, so the per-stage bookkeeping of
+  // every role never waits on a global load
+  const int i = (u - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x);
   const Chunk ch = i < kMaxCtaUnits ? cache[i] : a.chunks[u / nfb];
   UnitInfo ui;
   ui.shared = ch.e >= a.g.E;
@@ -144,32 +132,18 @@ __device__ __forceinline__ UnitInfo unit_info(const TcArgs& a, int u, int nfb, c
   return ui;
 }
 
-// Barrier operations of a whole (converged) warp: one arrival stands for its
-// 32 threads (the barriers count warps), and a wait's outcome is the same in
-// every lane, so the lanes leave a role's loop together.  Each thread's own
-// memory (and tensor-memory) operations are ordered before the arrival by
-// the warp synchronisation and the arrival's release semantics.
-__device__ __forceinline__ void warp_arrive(uint64_t* bar, int lane) {
-  __syncwarp();
-  if (lane == 0) tc::mbar_arrive(bar);
-}
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* status,
-                                          long long limit) {
-  return __all_sync(0xffffffffu, tc::mbar_wait(bar, parity, abort, status, limit));
-}
-
 // Walks this CTA's stages in order: (unit, k-step) with global stage and
 // scale-block counts (a scale block starts at every k-step multiple of 8).
 template <bool kGateUp>
 struct StageCursor {
-  int r, u, ks;
+  int u, ks;
   uint32_t it, blk;
   bool done;
   UnitInfo ui;
 
   const Chunk* cache;
   __device__ __forceinline__ void seek_unit(const TcArgs& a, int from, int n_units, int nfb) {
-    for (r = from; (u = snake_unit(r)) < n_units; ++r) {
+    for (u = from; u < n_units; u += gridDim.x) {
       ui = unit_info<kGateUp>(a, u, nfb, cache);
       if (!ui.skip) {
         ks = 0;
@@ -183,11 +157,11 @@ struct StageCursor {
     cache = units;
     it = 0;
     blk = 0;
-    seek_unit(a, 0, n_units, nfb);
+    seek_unit(a, blockIdx.x, n_units, nfb);
   }
   __device__ __forceinline__ void next(const TcArgs& a, int n_units, int nfb) {
     ++it;
-    if (++ks == ui.nks) seek_unit(a, r + 1, n_units, nfb);
+    if (++ks == ui.nks) seek_unit(a, u + gridDim.x, n_units, nfb);
     if (!done && ks % kSBlock == 0) ++blk;
   }
 };
@@ -223,23 +197,23 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
     }
     for (int s = 0; s < kPStages; ++s) {
       tc::mbar_init(&full_p[s], 1);
-      tc::mbar_init(&empty_p[s], C::DQ_PER_STAGE / 32);
+      tc::mbar_init(&empty_p[s], C::DQ_PER_STAGE);
     }
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&full_s[s], 1);
-      tc::mbar_init(&empty_s[s], kDqWarps);        // every dequantiser warp releases every block once
+      tc::mbar_init(&empty_s[s], kDqWarps * 32);   // every dequantiser releases every block once
     }
     for (int s = 0; s < C::A_STAGES; ++s) {
-      tc::mbar_init(&full_a[s], C::DQ_PER_STAGE / 32);
+      tc::mbar_init(&full_a[s], C::DQ_PER_STAGE);
       tc::mbar_init(&empty_a[s], 1);
     }
     for (int b = 0; b < C::ACC_BUFS; ++b) {
       tc::mbar_init(&acc_full[b], 1);
-      tc::mbar_init(&acc_empty[b], 4);
+      tc::mbar_init(&acc_empty[b], 128);
     }
     tc::mbar_init(drain, 1);
-    tc::mbar_init(&epi_sync[0], 4);
-    tc::mbar_init(&epi_sync[1], 4);
+    tc::mbar_init(&epi_sync[0], 128);
+    tc::mbar_init(&epi_sync[1], 128);
     *abort_flag = 0;
     tc::fence_barrier_init();
   }
@@ -255,7 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
   const int Tk = a.g.T * a.g.k;
   Chunk* units = reinterpret_cast<Chunk*>(smem + C::OFF_UNITS);
   for (int i = threadIdx.x; i < kMaxCtaUnits; i += blockDim.x) {
-    const int u = snake_unit(i);
+    const int u = static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
     if (u < n_units) units[i] = a.chunks[u / nfb];
   }
   if (warp == kMmaWarp) tc::tmem_alloc(tmem_slot, kTmemCols);
@@ -293,10 +267,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
         if (cur.blk != held_blk) {
           if (held_blk != 0xffffffffu) {
             tc::fence_proxy_async_smem();            // generic reads of the block before its TMA refill
-            warp_arrive(&empty_s[held_blk & 1u], lane);
+            tc::mbar_arrive(&empty_s[held_blk & 1u]);
           }
           held_blk = cur.blk;
-          if (!warp_wait(&full_s[held_blk & 1u], (held_blk >> 1) & 1u, abort_flag, a.status, a.wait_limit)) {
+          if (!tc::mbar_wait(&full_s[held_blk & 1u], (held_blk >> 1) & 1u, abort_flag, a.status, a.wait_limit)) {
             ok = false;
             break;
           }
@@ -313,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
       }
       // packed words of this stage's tile row
       const int sp = static_cast<int>(it % kPStages);
-      if (!warp_wait(&full_p[sp], (it / kPStages) & 1u, abort_flag, a.status, a.wait_limit)) {
+      if (!tc::mbar_wait(&full_p[sp], (it / kPStages) & 1u, abort_flag, a.status, a.wait_limit)) {
         ok = false;
         break;
       }
@@ -337,9 +311,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
       // write into it is an async-proxy access following these generic-proxy
       // reads: the proxy fence orders the two (the mbarrier alone does not).
       tc::fence_proxy_async_smem();
-      warp_arrive(&empty_p[sp], lane);
+      tc::mbar_arrive(&empty_p[sp]);
       const int sa = static_cast<int>(it % C::A_STAGES);
-      if (!warp_wait(&empty_a[sa], ((it / C::A_STAGES) & 1u) ^ 1u, abort_flag, a.status, a.wait_limit)) {
+      if (!tc::mbar_wait(&empty_a[sa], ((it / C::A_STAGES) & 1u) ^ 1u, abort_flag, a.status, a.wait_limit)) {
         ok = false;
         break;
       }
@@ -347,13 +321,13 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
       tc::tmem_st32(lane_base + C::A_BASE + sa * C::A_COLS + m * 32, cols);
       tc::tmem_wait_st();
       tc::tc_fence_before();
-      warp_arrive(&full_a[sa], lane);
+      tc::mbar_arrive(&full_a[sa]);
       cur.next(a, n_units, nfb);
       while (!cur.done && !mine(cur.it)) cur.next(a, n_units, nfb);
     }
     if (ok && a.scales_tma && held_blk != 0xffffffffu) {
       tc::fence_proxy_async_smem();
-      warp_arrive(&empty_s[held_blk & 1u], lane);
+      tc::mbar_arrive(&empty_s[held_blk & 1u]);
     }
   } else if (warp < kLoadWarp) {
     // ----------------------------------------------------------- epilogue
@@ -364,11 +338,11 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
     uint16_t* stage = reinterpret_cast<uint16_t*>(smem + C::OFF_OUT);   // [BN tokens][BM features]
     uint32_t tt = 0;
-    for (int rd = 0, u; (u = snake_unit(rd)) < n_units; ++rd) {
+    for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
       const UnitInfo ui = unit_info<kGateUp>(a, u, nfb, units);
       if (ui.skip) continue;
       const int buf = static_cast<int>(tt % C::ACC_BUFS);
-      if (!warp_wait(&acc_full[buf], (tt / C::ACC_BUFS) & 1u, abort_flag, a.status, a.wait_limit)) break;
+      if (!tc::mbar_wait(&acc_full[buf], (tt / C::ACC_BUFS) & 1u, abort_flag, a.status, a.wait_limit)) break;
       tc::tc_fence_after();
       const uint32_t acc = lane_base + buf * C::ACC_COLS;
       for (int n0 = 0; n0 < ui.rows; n0 += 16) {
@@ -391,9 +365,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
       }
       // accumulator drained: hand it back to the MMA before writing the tile out
       tc::tc_fence_before();
-      warp_arrive(&acc_empty[buf], lane);
-      warp_arrive(&epi_sync[0], lane);
-      if (!warp_wait(&epi_sync[0], tt & 1u, abort_flag, a.status, a.wait_limit)) break;
+      tc::mbar_arrive(&acc_empty[buf]);
+      tc::mbar_arrive(&epi_sync[0]);
+      if (!tc::mbar_wait(&epi_sync[0], tt & 1u, abort_flag, a.status, a.wait_limit)) break;
       // coalesced copy-out: each token row of the tile is BM contiguous outputs (256 B)
       const int chunks = ui.rows * (BM / 8);
       for (int i = et; i < chunks; i += 128) {
@@ -406,8 +380,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
           dst = a.Y + static_cast<size_t>(R) * a.g.H;
         *reinterpret_cast<uint4*>(dst + ui.f0 + c * 8) = *reinterpret_cast<const uint4*>(stage + n * BM + c * 8);
       }
-      warp_arrive(&epi_sync[1], lane);                   // the staging tile is free again
-      if (!warp_wait(&epi_sync[1], tt & 1u, abort_flag, a.status, a.wait_limit)) break;
+      tc::mbar_arrive(&epi_sync[1]);                     // the staging tile is free again
+      if (!tc::mbar_wait(&epi_sync[1], tt & 1u, abort_flag, a.status, a.wait_limit)) break;
       ++tt;
     }
   } else if (warp == kLoadWarp) {
@@ -415,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
     if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
-      for (int rd = 0, u; ok && (u = snake_unit(rd)) < n_units; ++rd) {
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
         const UnitInfo ui = unit_info<kGateUp>(a, u, nfb, units);
         if (ui.skip) continue;
         // gate/up: rows of the grouped x (shared-expert rows follow the routed
@@ -485,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
     const uint64_t bdesc0 = tc::sdesc_sw128(sbase + C::OFF_B);
     uint32_t it = 0, tt = 0;
     bool ok = true;
-    for (int rd = 0, u; ok && (u = snake_unit(rd)) < n_units; ++rd) {
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const UnitInfo ui = unit_info<kGateUp>(a, u, nfb, units);
       if (ui.skip) continue;
       const int n_mma = max(16, (ui.rows + 15) & ~15);

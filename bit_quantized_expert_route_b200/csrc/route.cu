@@ -102,34 +102,16 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(
   int first = 0;
   const int nchunks = block_exclusive_scan(nch, scratch, &first);
   // piece q starts at row floor(rows q / nch) = q base + floor(q rem / nch)
-  // (rows = base nch + rem); q rem < nch^2 <= (T_max k / 128)^2 fits 32 bits.
-  // The list is ordered by size, largest first (a counting sort on the row
-  // count), so that the grouped GEMMs can deal their units longest first;
-  // the order of equal-size chunks is arbitrary, which changes which SM
-  // computes a tile but not what it computes.
-  __shared__ int s_bucket[kGemmChunkRows + 1];   // chunks per size, then fill positions
-  const int nb = chunk_rows + 1;
-  for (int i = threadIdx.x; i < nb; i += blockDim.x) s_bucket[i] = 0;
-  __syncthreads();
+  // (rows = base nch + rem); q rem < nch^2 <= (T_max k / 128)^2 fits 32 bits
   const int base = nch > 0 ? rows / nch : 0, rem = nch > 0 ? rows % nch : 0;
-  for (int q = 0, r0 = 0; q < nch; ++q) {
-    const int r1 = (q + 1) * base + ((q + 1) * rem) / nch;
-    atomicAdd(&s_bucket[chunk_rows - (r1 - r0)], 1);
-    r0 = r1;
-  }
-  __syncthreads();
-  int boff = 0;
-  block_exclusive_scan(threadIdx.x < nb ? s_bucket[threadIdx.x] : 0, scratch, &boff);
-  if (threadIdx.x < nb) s_bucket[threadIdx.x] = boff;
-  __syncthreads();
-  for (int q = 0, r0 = 0; q < nch; ++q) {
+  int r0 = 0;
+  for (int q = 0; q < nch; ++q) {
     const int r1 = (q + 1) * base + ((q + 1) * rem) / nch;
     Chunk ch;
     ch.e = e; ch.row0 = base_row + r0; ch.rows = r1 - r0; ch.pad = 0;
-    chunks[atomicAdd(&s_bucket[chunk_rows - ch.rows], 1)] = ch;
+    chunks[first + q] = ch;
     r0 = r1;
   }
-  (void)first;
   if (e == 0) *n_chunks = nchunks;
 
   // Active-expert list: routed experts with rows, ascending, then the shared one.

@@ -178,3 +178,43 @@ def make_x_on_device(seed: int, T: int, H: int, device) -> torch.Tensor:
     g = torch.Generator(device=device)
     g.manual_seed((seed * 2_000_029 + 5) & 0x7FFFFFFF)
     return torch.randn((T, H), generator=g, device=device).to(torch.bfloat16)
+
+
+# --------------------------------------------------------------------------
+# Decode attention over a fixed-block KV cache: seeded q, paged K/V and a
+# shuffled block table (no attention arithmetic here).
+# --------------------------------------------------------------------------
+_KEY_ATTN = 0x4154544E   # stream tag for an attention case
+
+
+@dataclasses.dataclass
+class AttnCase:
+    """One decode-attention step's inputs in storage form."""
+    q: np.ndarray             # uint16 (bf16) [B, Hq, D]
+    k_cache: np.ndarray       # uint16 (bf16) [n_blocks, Hkv, block, D]
+    v_cache: np.ndarray       # uint16 (bf16) [n_blocks, Hkv, block, D]
+    block_table: np.ndarray   # int32 [B, max_blocks]: physical block of each logical block
+    ctx_len: np.ndarray       # int32 [B]
+
+
+def make_attention_case(seed: int, ctx_lens, Hq: int = 16, Hkv: int = 2, D: int = 256, block: int = 64,
+                        spare_blocks: int = 3) -> AttnCase:
+    """q, k, v ~ N(0, 1) as bf16; every sequence's logical blocks are mapped to physical
+    blocks by one seeded permutation of all blocks (plus `spare_blocks` unused ones), so
+    the table is scattered as a paged cache's would be."""
+    rng = _rng(_KEY_ATTN, seed)
+    ctx = np.asarray(list(ctx_lens), dtype=np.int32)
+    B = len(ctx)
+    per_seq = [(int(n) + block - 1) // block for n in ctx]
+    max_blocks = max(per_seq)
+    n_blocks = sum(per_seq) + spare_blocks
+    phys = rng.permutation(n_blocks).astype(np.int32)
+    table = np.full((B, max_blocks), -1, dtype=np.int32)
+    pos = 0
+    for b, nb in enumerate(per_seq):
+        table[b, :nb] = phys[pos:pos + nb]
+        pos += nb
+    q = to_bf16_bits(rng.normal(0.0, 1.0, size=(B, Hq, D)))
+    k = to_bf16_bits(rng.normal(0.0, 1.0, size=(n_blocks, Hkv, block, D)))
+    v = to_bf16_bits(rng.normal(0.0, 1.0, size=(n_blocks, Hkv, block, D)))
+    return AttnCase(q, k, v, table, ctx)
