@@ -45,6 +45,7 @@ sys.path.insert(0, ROOT)
 
 T_PREFILL = 4096
 SWEEP_T = (1, 8, 64, 512, 4096, 16384)
+ATTN_L = (4096, 32768, 131072)    # decode-attention context lengths (one sequence, 16 Q heads, 2 KV heads, D=256)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PREFILL_LAUNCHES_PER_STEP = 7     # router (+ segment counts), scan, scatter, gather, gate/up, down, combine
 UNFUSED_DECODE_LAUNCHES = 3       # routing (router+top-k+sort), gate/up GEMV, down GEMV+combine
@@ -75,8 +76,12 @@ def parse_args(argv=None):
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-tiny", action="store_true")
+    ap.add_argument("--no-attn", action="store_true", help="skip the decode-attention workload")
+    ap.add_argument("--attn-L", type=str, default=",".join(str(n) for n in ATTN_L))
+    ap.add_argument("--attn-reps", type=int, default=30, help="timed launches per attention point")
     ap.add_argument("--no-zipf-prefill", action="store_true", help="skip the skewed prefill workload")
     ap.add_argument("--decode-only", action="store_true", help="only the decode measurement (profiling)")
+    ap.add_argument("--attn-only", action="store_true", help="only the decode-attention measurement (profiling)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass (profiling)")
     ap.add_argument("--no-stages", action="store_true", help="skip the per-stage traced pass (profiling)")
     ap.add_argument("--layers", type=int, default=4, help="prefill layers cycled")
@@ -536,6 +541,68 @@ def tiny_phase(a, world, dev):
             "bound": "launch latency (3 dependent launches of ~1 KB of work each)"}
 
 
+# --------------------------------------------------- decode attention ---
+
+def attention_phase(a, world, rank, dev, peaks, peak_src):
+    """One decode step of GQA attention over a fixed-block KV cache (attn_decode) for one sequence
+    of L positions: 16 query heads, 2 KV heads, D=256, blocks of 64 rows in a shuffled block table.
+    Each timed launch is bracketed by its own CUDA events with a 512 MB write between launches, so
+    the cache is read from HBM even where it fits in L2; the oracle is timed on the host."""
+    import torch
+    from bit_quantized_expert_route_b200 import attn, moe, synth
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    pts = {}
+    for L in [int(n) for n in a.attn_L.split(",") if n]:
+        c = synth.make_attention_case_on_device(900 + rank, [L], dev)
+        out = torch.empty_like(c.q)
+        mb = c.block_table.shape[1]
+        ws = attn.alloc_workspace(1, 2, 256, 64, mb, dev)
+        for _ in range(max(3, a.warmup)):
+            attn.attn_decode(c.q, c.k_cache, c.v_cache, c.block_table, c.ctx_len, out, ws)
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(a.attn_reps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            attn.attn_decode(c.q, c.k_cache, c.v_cache, c.block_table, c.ctx_len, out, ws)
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        ms = max_over_ranks(statistics.median(ts), world)
+        assert moe.moe_get_status(ws) == 0
+        n_split, cps = attn.plan(1, 2, 64, mb)
+        kv = L * 2 * 256 * 2 * 2                      # keys + values of both KV heads, bf16
+        overhead = (n_split * 2 * 8 * (256 + 2) * 4 * 2) if n_split > 1 else 0   # partials written + read
+        pts[str(L)] = {"us": round(ms * 1e3, 3), "steps_per_s": round(whole_job_rate(1, world, ms), 1),
+                       "kv_bytes": kv, "split_partial_bytes": overhead, "n_split": n_split, "chunks_per_split": cps,
+                       "launches_per_step": 2 if n_split > 1 else 1,
+                       "roofline": hbm_roofline("attn_decode_kernel<256>", kv, ms, peaks, peak_src)}
+        del c, out, ws
+        torch.cuda.empty_cache()
+    del flush
+    torch.cuda.empty_cache()
+    return {"workload": "decode attention, 1 sequence, 16 Q heads / 2 KV heads (GQA groups of 8), D=256, "
+                        "fixed blocks of 64 rows, shuffled block table, bf16 K/V ~ N(0,1)",
+            "timing": "median of per-launch CUDA-event times, L2 flushed (512 MB write) between launches",
+            "roofline_note": "algorithmic bytes = L x 2 KV heads x (K + V) x 256 x 2 B; the split partials "
+                             "(split_partial_bytes) are overhead on top",
+            "points": pts}
+
+
+def attention_oracle_times():
+    """The float64 attention oracle on this host for every context length of the workload."""
+    from bit_quantized_expert_route_b200 import synth
+    from oracle import attn_ref
+    res = {}
+    for L in ATTN_L:
+        c = synth.make_attention_case(900, [L])
+        t0 = time.perf_counter()
+        attn_ref.decode_attention(c.q, c.k_cache, c.v_cache, c.block_table, c.ctx_len)
+        res[str(L)] = {"seconds": round(time.perf_counter() - t0, 3)}
+    return res
+
+
 # ------------------------------------------------------------ CPU oracle ---
 
 def _oracle_time(fn, single_core: bool = False):
@@ -593,6 +660,8 @@ def oracle_phase(a):
         dt_ = _oracle_time(lambda: moe_ref.moe_layer(xs, lay, dims.k))
         sw[str(T)] = {"seconds": round(dt_, 3), "tokens_per_s": round(T / dt_, 2)}
     res["sweep_layer0"] = sw
+    if not a.no_attn:
+        res["attention"] = attention_oracle_times()
     cpu_baseline = {"value": res["prefill_uniform"]["tokens_per_s"], "unit": "tokens/s", "cores": cores,
                     "kind": "oracle", "sample": "the whole uniform prefill input (4096 tokens), one call, "
                                                 "NumPy float64, BLAS threads = cores",
@@ -615,6 +684,9 @@ def run_ours(a):
 
     clk = ClockSampler(torch.cuda.current_device()).__enter__()   # sampled across every timed phase
     pre = {}
+    if a.attn_only:
+        a.decode_only, a.no_decode = True, True
+        workloads["attention"] = attention_phase(a, world, rank, dev, peaks, peak_src)
     if not a.decode_only:
         pre = prefill_phase(a, world, rank, dev, dims, zipf, peaks, peak_src, e2e=True)
         if not a.no_zipf_prefill and not zipf:
@@ -630,6 +702,8 @@ def run_ours(a):
     torch.cuda.empty_cache()
     if not a.no_tiny and not a.decode_only:
         workloads["tiny"] = tiny_phase(a, world, dev)
+    if not a.no_attn and not a.decode_only:
+        workloads["attention"] = attention_phase(a, world, rank, dev, peaks, peak_src)
     clk.__exit__(None, None, None)
     clocks = clk.summary()
 

@@ -75,7 +75,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // Byte offsets of every workspace buffer for a call with T tokens.
 struct WsLayout {
   size_t status, counter, grid_bar, topk_idx, topk_w, counts, offsets, perm, inv_perm, sigma, seg, chunks, n_chunks,
-      active, n_active, logits, h, h_s, Y, x_stage, out_stage, dec_y, dec_sumsq, total;
+      active, n_active, logits, h, h_s, Y, x_stage, out_stage, xch[4], total;
   int max_chunks;
 };
 
@@ -92,7 +92,7 @@ WsLayout ws_layout(const moe_layer_desc* d, int T) {
   w.max_chunks = static_cast<int>(n / cr + T / cr + d->E + 2);
   w.status = take(256);          // control block: status word, small-T routing counter, grid barrier
   w.counter = w.status + 4;
-  w.grid_bar = w.status + 8;     // [arrivals, generation] of the fused decode kernel's grid barrier
+  w.grid_bar = w.status + 8;     // fused decode kernel: [unused, exit counter, epoch]
   w.topk_idx = take(n * 4);
   w.topk_w = take(n * 4);
   w.counts = take(static_cast<size_t>(d->E) * 4);
@@ -111,10 +111,10 @@ WsLayout ws_layout(const moe_layer_desc* d, int T) {
   w.Y = take((n + T) * d->H * 2);   // also holds the gate/up GEMM's grouped token rows before the down GEMM
   w.x_stage = take(static_cast<size_t>(T) * d->H * 2);
   w.out_stage = take(static_cast<size_t>(T) * d->H * 2);
-  // the fused decode kernel's outputs between stacked layers and the CTAs'
-  // partial sums of their squares
-  w.dec_y = take(static_cast<size_t>(T <= kFusedMaxT ? T : 0) * d->H * 2);
-  w.dec_sumsq = take(static_cast<size_t>(T <= kFusedMaxT ? kFusedMaxGrid * 8 : 0) * 4);
+  // the fused decode kernel's exchange words: logits, h, outputs between
+  // stacked layers and the CTAs' sums of squares of them
+  for (int i = 0; i < 4; ++i)
+    w.xch[i] = take(T <= kFusedMaxT ? fused_exchange_words(T, d->H, d->I, d->I_shared, d->E, d->k, i) * 8 : 0);
   w.total = off;
   return w;
 }
@@ -237,10 +237,11 @@ cudaError_t launch_fused_layers(const Geometry& g, const LayerPtr* layers, int n
                                 cudaStream_t s) {
   RoutingPtrs rp{b.topk_idx, b.topk_w, b.sigma, b.counts, b.offsets, b.perm, b.inv_perm};
   if (!with_routing) rp = RoutingPtrs{};
-  return launch_decode_fused(g, layers, n_layers, x, out, b.at<uint16_t>(b.w.dec_y), b.at<float>(b.w.dec_sumsq),
-                             trace, eps, rp, b.at<int32_t>(b.w.active), b.at<int32_t>(b.w.n_active),
-                             b.at<float>(b.w.logits), b.at<uint16_t>(b.w.h), b.at<uint16_t>(b.w.h_s),
-                             b.at<unsigned>(b.w.grid_bar), b.at<int>(b.w.status), s);
+  const FusedExchange xch{b.at<unsigned long long>(b.w.xch[0]), b.at<unsigned long long>(b.w.xch[1]),
+                          b.at<unsigned long long>(b.w.xch[2]), b.at<unsigned long long>(b.w.xch[3])};
+  return launch_decode_fused(g, layers, n_layers, x, out, trace, eps, rp, b.at<int32_t>(b.w.active),
+                             b.at<int32_t>(b.w.n_active), xch, b.at<unsigned>(b.w.grid_bar), b.at<int>(b.w.status),
+                             s);
 }
 
 // Bulk copies of whole scale/bias tile rows need 16-byte aligned stacks.
@@ -629,6 +630,7 @@ const char* moe_strerror(int status) {
     case MOE_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     case MOE_ERR_CUDA: return "CUDA runtime error or kernel launch failure";
     case MOE_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait gave up";
+    case MOE_ERR_DEVICE_INDEX: return "a device-side bounds check found an index out of range";
     default: return "unknown status";
   }
 }

@@ -14,6 +14,7 @@ constexpr int kMaxE = 256;          // largest supported expert count
 
 // Status codes written to the workspace status word (mirror moe_status).
 constexpr int kStatusTimeout = -5;
+constexpr int kStatusBadIndex = -6;
 
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
   return __uint_as_float(static_cast<uint32_t>(b) << 16);

@@ -13,26 +13,28 @@
 // and the producer warp fetches the next layer's router rows and first
 // shared-expert tile while the current layer still computes.
 //
-// Each layer, with three grid-wide barriers (all CTAs are co-resident:
-// cooperative launch):
+// Each layer has three all-to-all exchanges between the CTAs (all CTAs are
+// co-resident: cooperative launch).  None is a grid barrier: the values
+// travel in tagged 64-bit words that a reader polls until they are current
+// (see wait_word), so a CTA goes on the moment the data it needs is there.
 //
 //   A  input: layer 0 reads x; layer l > 0 reads the previous layer's output
 //      y (bf16) and the CTAs' partial sums of its squares and applies
 //      RMSNorm (weight 1): x = bf16(y / sqrt(mean(y^2) + eps)).  Router
 //      logits: CTA c scores rows c, c+G, ... of [W_r; w_sg] (from shared
-//      memory, copied there by the producer ahead of time) for every token.
-//   -- grid barrier (logits) --
+//      memory, copied there by the producer ahead of time) for every token
+//      and publishes them.                               -- exchange: logits
 //   B  every CTA reads the T x (E+1) logits and repeats the (tiny, exact and
 //      deterministic) top-k, shared gate and counting sort, so it knows the
-//      active experts without another barrier.
-//   C  gate/up units: (expert slot, 16 features) -> h = bf16(silu(g) * u).
-//   -- grid barrier (h complete) --  the producer keeps copying the down
-//      tiles meanwhile: they depend on the routing, not on h.
+//      active experts without another exchange.
+//   C  gate/up units: (expert slot, 16 features) -> h = bf16(silu(g) * u),
+//      published pair by pair.                           -- exchange: h
+//      The producer keeps copying the down tiles meanwhile: they depend on
+//      the routing, not on h.
 //   D  down units: (16 output dims, up to 8 expert slots); then the combine
 //      of each token's k + 1 terms in slot order, then the shared term,
-//      exactly as the other kernels; the CTA writes its output dims and the
-//      partial sum of their squares.
-//   -- grid barrier (outputs complete; between layers only) --
+//      exactly as the other kernels; between layers the CTA publishes its
+//      output dims and the partial sum of their squares.  -- exchange: y
 //
 // Weight tiles stream through a ring of shared-memory slots filled by one
 // producer thread (cp.async.bulk, completion on the slot's "full" mbarrier)
@@ -69,6 +71,7 @@ constexpr int kFRouterRows = 2;                 // router rows per CTA with load
 constexpr int kFMaxRouterRows = 4;              // router rows per CTA held in shared memory
 constexpr int kFMaxLayers = 40;                 // layers per launch (kernel-parameter space)
 constexpr int kFMaxGrid = 160;                  // CTAs (SMs) the RMSNorm partial sums are read for in one pass
+constexpr int kFRowPad = 32;                    // bytes after each staged row of codes (bank spread)
 
 struct FusedArgs {
   Geometry g;
@@ -76,18 +79,19 @@ struct FusedArgs {
   float eps;              // RMSNorm between layers
   const uint16_t* x;      // input of layer 0 [T, H]
   uint16_t* out;          // output of the last layer [T, H]
-  uint16_t* y;            // outputs of the other layers [T, H] (workspace)
-  float* sumsq;           // [G][kFMaxT] partial sums of squares of y (workspace)
   uint16_t* trace;        // NULL or [n_layers][2][T][H]: layer inputs and outputs
   RoutingPtrs r;          // routing outputs of the last layer (topk_idx NULL: none)
   int32_t* active;
   int32_t* n_active;
-  float* logits;          // [T, E+1]
-  uint16_t* h;            // [T*k, I]
-  uint16_t* h_s;          // [T, Is]
-  unsigned* bar;          // [0] arrivals, [1] exits
+  // tagged exchange words (workspace): payload in the low half
+  unsigned long long* lgx;     // [T][E+1] logits (FP32 bits)
+  unsigned long long* hx;      // [T*k + T][Kmax/2] h (two bf16), routed rows then shared rows
+  unsigned long long* yx;      // [T][H/2] outputs of the layers before the last (two bf16)
+  unsigned long long* ssx;     // [G][kFMaxT] each CTA's sum of squares of its outputs (FP32 bits)
+  unsigned* bar;          // [1] exit counter, [2] epoch
   int* status;
   int ring, slot_bytes, spd, rows_per_cta;
+  int rs_gu, rs_dn, dslot;   // staged row strides of gate/up and down codes; bytes per down expert slot
   long long wait_limit;   // cycles before a bounded wait gives up
   int off_bar, off_wr, off_xs, off_xsum, off_lg, off_rt, off_y, off_nrm;
   LayerPtr layers[kFMaxLayers];
@@ -105,8 +109,10 @@ struct RouteSmem {
   int32_t slot_e[kFMaxT * kMaxK + 1];
   int32_t slot_cnt[kFMaxT * kMaxK + 1];
   int32_t slot_off[kFMaxT * kMaxK + 1];
+  int32_t first[kFMaxT * kMaxK];   // entry i is its expert's first occurrence
   int32_t n_act;               // routed active experts
   int32_t abort;
+  uint32_t epoch;              // the launch's epoch (tags of layer l: (epoch + 1) * 64 + l)
 };
 
 // D (16 rows x 8 tokens, FP32) += A (16 x 16, bf16) B (16 x 8, bf16).
@@ -143,11 +149,59 @@ __device__ __forceinline__ uint4 interleave8(const uint4& v) {
 // sum (128 + q) x for (row g, tokens 2t, 2t+1) and (row g+8, same tokens).
 __device__ __forceinline__ void group_dot(float (&d)[4], const uint2& qg, const uint2& qg8, const uint4& xb0,
                                           const uint4& xb1) {
+  float e[4] = {0.f, 0.f, 0.f, 0.f};   // two accumulation chains, summed at the end
   d[0] = d[1] = d[2] = d[3] = 0.f;
   mma16816(d, code_pair(qg.x, 0), code_pair(qg8.x, 0), code_pair(qg.x, 4), code_pair(qg8.x, 4), xb0.x, xb0.y);
-  mma16816(d, code_pair(qg.x, 8), code_pair(qg8.x, 8), code_pair(qg.x, 12), code_pair(qg8.x, 12), xb0.z, xb0.w);
+  mma16816(e, code_pair(qg.x, 8), code_pair(qg8.x, 8), code_pair(qg.x, 12), code_pair(qg8.x, 12), xb0.z, xb0.w);
   mma16816(d, code_pair(qg.y, 0), code_pair(qg8.y, 0), code_pair(qg.y, 4), code_pair(qg8.y, 4), xb1.x, xb1.y);
-  mma16816(d, code_pair(qg.y, 8), code_pair(qg8.y, 8), code_pair(qg.y, 12), code_pair(qg8.y, 12), xb1.z, xb1.w);
+  mma16816(e, code_pair(qg.y, 8), code_pair(qg8.y, 8), code_pair(qg.y, 12), code_pair(qg8.y, 12), xb1.z, xb1.w);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) d[i] += e[i];
+}
+
+// One warp's share of a 16-row weight tile: groups g0 .. g0 + ng - 1 (ng <=
+// NG) of 64 inputs.  Lane (lg4, lt) holds rows lg4 and lg4 + 8 (codes at
+// qrow and qrow + 8 rs, already offset by the lane's 8 bytes) and token
+// columns 2 lt, 2 lt + 1 (valid below tn; activations at xrow, in uint4 units
+// already offset by the lane; group sums at xsum[t * xs + G]); scales and
+// biases are rows of ngr groups.  The scales and biases of all the warp's
+// groups are loaded up front, then each group adds
+// s (sum (128 + q) x - 128 X) + b X to y[row][column].
+template <int NG>
+__device__ __forceinline__ void tile_groups(float (&y)[2][2], const uint8_t* qrow, int rs, const uint16_t* srow,
+                                            const uint16_t* brow, int ngr, int g0, int ng, const uint4* xrow,
+                                            bool tok_live, const float* xsum, int xs, int tn, int lg4, int lt) {
+  float sv[2][NG], bv[2][NG];
+#pragma unroll
+  for (int q = 0; q < NG; ++q) {
+    const int G = g0 + (q < ng ? q : 0);
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      sv[r][q] = bf16_bits_to_float(srow[(lg4 + 8 * r) * ngr + G]);
+      bv[r][q] = bf16_bits_to_float(brow[(lg4 + 8 * r) * ngr + G]);
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < NG; ++q) {
+    if (q < ng) {
+      const int G = g0 + q;
+      const uint2 qa = *reinterpret_cast<const uint2*>(qrow + G * 32);
+      const uint2 qc = *reinterpret_cast<const uint2*>(qrow + 8 * rs + G * 32);
+      const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+      const uint4 xb0 = tok_live ? xrow[G * 8] : z, xb1 = tok_live ? xrow[G * 8 + 1] : z;
+      float d[4];
+      group_dot(d, qa, qc, xb0, xb1);
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int t = 2 * lt + c;
+        if (t < tn) {
+          const float X = xsum[t * xs + G];
+#pragma unroll
+          for (int r = 0; r < 2; ++r) y[r][c] = fmaf(sv[r][q], d[2 * r + c] - 128.f * X, fmaf(bv[r][q], X, y[r][c]));
+        }
+      }
+    }
+  }
 }
 
 // Order-preserving 32-bit key of a float (larger float -> larger key; every
@@ -159,93 +213,114 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 
 // Warp top-k over E <= 256 logits in shared memory with the same order as
 // the other routing kernels (larger logit first, equal logits -> lower expert
-// index): each pick is a lane-local scan of 8 keys and two warp reductions
-// (redux.sync max of the key, then min of the expert index among the lanes
-// holding that key).  Lane 0 writes the experts and exp(l_j - l_0) / sum.
+// index).  Lane i holds the keys of experts i, i + 32, ..., sorted once by a
+// 19-comparator network on (key, expert) pairs, so its best candidate is
+// always its head.  A pick is one redux.sync max over the heads and one min
+// over the experts of the lanes holding that key; the winning lane pops its
+// head.  Lanes j < k then form exp(l_j - l_0) in parallel and divide by their
+// sum (a fixed shuffle tree).
+__device__ __forceinline__ bool key_before(uint32_t ka, int ia, uint32_t kb, int ib) {
+  return ka > kb || (ka == kb && ia < ib);
+}
+__device__ __forceinline__ void cas(uint32_t (&key)[8], int (&ix)[8], int i, int j) {
+  const bool keep = key_before(key[i], ix[i], key[j], ix[j]);
+  const uint32_t ki = keep ? key[i] : key[j], kj = keep ? key[j] : key[i];
+  const int ii = keep ? ix[i] : ix[j], ij = keep ? ix[j] : ix[i];
+  key[i] = ki;
+  key[j] = kj;
+  ix[i] = ii;
+  ix[j] = ij;
+}
 __device__ __forceinline__ void topk_redux(const float* lg, int E, int k, int lane, int32_t* idx_out,
                                            float* w_out) {
   uint32_t key[8];
+  int ix[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const int e = lane + 32 * i;
-    key[i] = e < E ? order_key(lg[e]) : 0u;
+    ix[i] = lane + 32 * i;
+    key[i] = ix[i] < E ? order_key(lg[ix[i]]) : 0u;
   }
-  int sel[kMaxK];
+  cas(key, ix, 0, 1); cas(key, ix, 2, 3); cas(key, ix, 4, 5); cas(key, ix, 6, 7);
+  cas(key, ix, 0, 2); cas(key, ix, 1, 3); cas(key, ix, 4, 6); cas(key, ix, 5, 7);
+  cas(key, ix, 1, 2); cas(key, ix, 5, 6);
+  cas(key, ix, 0, 4); cas(key, ix, 1, 5); cas(key, ix, 2, 6); cas(key, ix, 3, 7);
+  cas(key, ix, 2, 4); cas(key, ix, 3, 5);
+  cas(key, ix, 1, 2); cas(key, ix, 3, 4); cas(key, ix, 5, 6);
+  int mine = 0, first = 0;
 #pragma unroll
   for (int j = 0; j < kMaxK; ++j) {
     if (j < k) {
-      uint32_t best = 0u;
-      int bi = 0;
+      const uint32_t m = __reduce_max_sync(0xffffffffu, key[0]);
+      const uint32_t win = __reduce_min_sync(0xffffffffu, key[0] == m ? static_cast<uint32_t>(ix[0]) : 0xffffffffu);
+      if (static_cast<uint32_t>(ix[0]) == win) {   // pop the head
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        if (key[i] > best) {        // strictly greater: the lowest index among equal keys
-          best = key[i];
-          bi = i;
+        for (int i = 0; i < 7; ++i) {
+          key[i] = key[i + 1];
+          ix[i] = ix[i + 1];
         }
-      const uint32_t m = __reduce_max_sync(0xffffffffu, best);
-      const uint32_t cand = (best == m && m != 0u) ? static_cast<uint32_t>(lane + 32 * bi) : 0xffffffffu;
-      const uint32_t win = __reduce_min_sync(0xffffffffu, cand);
-      if (static_cast<int>(win & 31u) == lane) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          if (i == static_cast<int>(win >> 5)) key[i] = 0u;
+        key[7] = 0u;
+        ix[7] = 0x7fffffff;
       }
-      sel[j] = static_cast<int>(win);
+      if (lane == j) mine = static_cast<int>(win);
+      if (j == 0) first = static_cast<int>(win);
     }
   }
-  if (lane == 0) {
-    float z[kMaxK];
-    float sum = 0.f;
-    const float l0 = lg[sel[0]];
-#pragma unroll
-    for (int j = 0; j < kMaxK; ++j)
-      if (j < k) {
-        z[j] = expf(lg[sel[j]] - l0);
-        sum += z[j];
-      }
-#pragma unroll
-    for (int j = 0; j < kMaxK; ++j)
-      if (j < k) {
-        idx_out[j] = sel[j];
-        w_out[j] = z[j] / sum;
-      }
+  const float z = lane < k ? expf(lg[mine] - lg[first]) : 0.f;
+  const float sum = warp_sum(z);
+  if (lane < k) {
+    idx_out[lane] = mine;
+    w_out[lane] = z / sum;
   }
 }
 
 __device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kFWarps * 32) : "memory"); }
 
-// Grid-wide barrier number n (target n * nblocks) of one launch, called by
-// one thread per CTA after a barrier of the CTA's consumers (all CTAs are
-// co-resident).  bar[0] counts arrivals over the whole launch: each CTA adds
-// 1 with release semantics (publishing what its threads wrote before the CTA
-// barrier) and polls, bounded, until the count reaches the target, then
-// acquires.  No arriver has to reset or publish anything, so the barrier
-// costs one release-add and the polls.  bar[0] starts every launch at zero:
-// grid_exit resets it.
-__device__ bool grid_barrier(unsigned* bar, unsigned target, int* status, long long limit) {
-  asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(bar) : "memory");
-  const long long deadline = clock64() + limit;
-  for (;;) {
-    unsigned v;
-    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
-    if (v >= target) break;
-    if (clock64() > deadline) {
-      if (status) atomicExch(status, kStatusTimeout);
-      return false;
-    }
-  }
-  asm volatile("fence.acq_rel.gpu;" ::: "memory");
-  return true;
+// Exchanges between CTAs carry their own readiness: every value travels in a
+// 64-bit word whose high half is a tag unique to (launch, layer), stored and
+// loaded whole (an aligned 8-byte access is single-copy atomic).  A reader
+// polls the words it needs until each carries the current tag -- one round
+// trip through L2, no fence and no separate counter.  A word left from an
+// earlier layer or launch carries another tag, so it is never taken for a
+// current one.  Tag of layer l: (epoch + 1) * 64 + l, with the epoch read
+// from the workspace at the start of a launch and advanced once by the last
+// CTA to leave (launch_exit); 2^32 / 64 launches before it wraps.
+__device__ __forceinline__ unsigned long long ld_word(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_word(unsigned long long* p, uint32_t tag, uint32_t payload) {
+  const unsigned long long v = (static_cast<unsigned long long>(tag) << 32) | payload;
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
-// Called once per CTA by the thread that polls the barrier, after its last
-// grid_barrier (or after giving up on one): the last CTA to get here resets
-// both words for the next launch on the same workspace.  Every CTA has then
-// finished polling bar[0].
-__device__ void grid_exit(unsigned* bar, unsigned nblocks) {
+// The payload of *p once it carries `tag`.  Bounded: gives up (ok = false,
+// status recorded, the CTA's abort flag raised) after the deadline or as
+// soon as another thread of the CTA has given up.
+__device__ __forceinline__ uint32_t wait_word(const unsigned long long* p, uint32_t tag, long long deadline,
+                                              volatile int* abort, int* status, bool& ok) {
+  unsigned long long v = ld_word(p);
+  for (uint32_t n = 0; ok && static_cast<uint32_t>(v >> 32) != tag; ++n) {
+    if ((n & 15u) == 15u && (*abort || clock64() > deadline)) {
+      ok = false;
+      if (!*abort) {
+        *abort = 1;
+        if (status) atomicExch(status, kStatusTimeout);
+      }
+      break;
+    }
+    v = ld_word(p);
+  }
+  return static_cast<uint32_t>(v);
+}
+
+// Called once per CTA at its end: the last CTA to leave advances the epoch
+// (bar[2]) for the next launch on the same workspace and resets its exit
+// counter (bar[1]).  Every CTA read the epoch at its start.
+__device__ void launch_exit(unsigned* bar, unsigned nblocks) {
   if (atomicAdd(bar + 1, 1u) == nblocks - 1) {
-    bar[0] = 0u;
     bar[1] = 0u;
+    bar[2] = bar[2] + 1u;
   }
 }
 
@@ -287,55 +362,82 @@ __device__ __forceinline__ void gu_unit(const Sched& s, int u, int& slot, int& f
   f0 = (sh ? u : (u - s.n_sh_units) % s.units_per_exp) * kFFeat;
 }
 
-// Issue the bulk copies of the gate/up tile (expert e, features f0..f0+15)
-// of layer L into `dst`: [q gate 16 rows][q up 16 rows][s gate][b gate][s up][b up].
-__device__ void issue_gateup(const Geometry& g, const LayerPtr& L, int e, int f0, uint32_t dst, uint64_t* full) {
+// Staged tiles.  Every row of 4-bit codes is copied to its own shared-memory
+// row of stride (row bytes + 32): the 8 rows that one mma fragment reads then
+// start in 8 different bank groups, so a warp's code load is conflict-free.
+// The producer warp's 32 lanes issue the row copies together (lane 0 first
+// raised the slot's transaction count; the caller's __syncwarp orders it).
+//
+// gate/up unit (expert e, features f0..f0+15):
+//   [16 gate rows][16 up rows] (stride rs_gu = H/2 + 32), then
+//   [s gate][b gate][s up][b up] (16 x H/64 bf16 each).
+__device__ __forceinline__ uint32_t gateup_bytes(const Geometry& g) {
+  return 2 * kFFeat * (g.H / 2) + 4 * (kFFeat * g.H / 32);
+}
+__device__ void issue_gateup(const FusedArgs& a, const LayerPtr& L, int e, int f0, uint32_t dst, uint64_t* full,
+                             int lane) {
+  const Geometry& g = a.g;
   const bool sh = e >= g.E;
   const size_t row0 = static_cast<size_t>(sh ? 0 : e * g.I) + f0;
-  const QMatPtr Wg = sh ? L.sh_gate : L.gate;
-  const QMatPtr Wu = sh ? L.sh_up : L.up;
-  const uint32_t qb = kFFeat * g.H / 2, sb = kFFeat * g.H / 32;
-  tc::mbar_arrive_expect_tx(full, 2 * qb + 4 * sb);
-  tc::bulk_load(dst, Wg.q + row0 * (g.H / 8), qb, full);
-  tc::bulk_load(dst + qb, Wu.q + row0 * (g.H / 8), qb, full);
-  tc::bulk_load(dst + 2 * qb, Wg.s + row0 * (g.H / kGroup), sb, full);
-  tc::bulk_load(dst + 2 * qb + sb, Wg.b + row0 * (g.H / kGroup), sb, full);
-  tc::bulk_load(dst + 2 * qb + 2 * sb, Wu.s + row0 * (g.H / kGroup), sb, full);
-  tc::bulk_load(dst + 2 * qb + 3 * sb, Wu.b + row0 * (g.H / kGroup), sb, full);
+  const QMatPtr& W = lane < 16 ? (sh ? L.sh_gate : L.gate) : (sh ? L.sh_up : L.up);
+  const int r = lane & 15;
+  tc::bulk_load(dst + (lane >> 4) * kFFeat * a.rs_gu + r * a.rs_gu, W.q + (row0 + r) * (g.H / 8), g.H / 2, full);
+  if (lane < 4) {
+    const QMatPtr& V = lane < 2 ? (sh ? L.sh_gate : L.gate) : (sh ? L.sh_up : L.up);
+    const uint32_t sb = kFFeat * g.H / 32;
+    tc::bulk_load(dst + 2 * kFFeat * a.rs_gu + lane * sb, ((lane & 1) ? V.b : V.s) + row0 * (g.H / kGroup), sb,
+                  full);
+  }
 }
 
-// Issue the bulk copies of unit i of this CTA (layer L) into ring slot `dst`.
-// down layout: per expert slot jj at jj * 9 Kmax: [q 16 rows][s][b].
-__device__ void issue_unit(const FusedArgs& a, const LayerPtr& L, const RouteSmem& rt, const Sched& s, int i,
-                           uint32_t dst, uint64_t* full) {
-  const Geometry& g = a.g;
-  if (i < s.my_gu) {
-    int slot, f0;
-    gu_unit(s, blockIdx.x + i * gridDim.x, slot, f0);
-    issue_gateup(g, L, rt.slot_e[slot], f0, dst, full);
-    return;
-  }
-  const int di = i - s.my_gu;
-  const int blk = blockIdx.x + (di / s.n_down_parts) * gridDim.x;
-  const int j0 = (di % s.n_down_parts) * s.spd, nj = min(s.spd, s.n_slots - j0);
-  const int Kmax = max(g.I, g.Is);
+// down unit (16 output dims of dim block blk, expert slots j0..j0+nj-1): per
+// slot jj at jj * dslot: [16 code rows, stride rs_dn = Kmax/2 + 32][s: 16 x
+// K/64][b at + Kmax/2].  Returns the bytes to expect.
+__device__ __forceinline__ uint32_t down_bytes(const Geometry& g, int j0, int nj) {
   uint32_t bytes = 0;
   for (int jj = 0; jj < nj; ++jj) {
     const int K = j0 + jj == 0 ? g.Is : g.I;
     bytes += kFDims * K / 2 + 2 * (kFDims * K / 32);
   }
-  tc::mbar_arrive_expect_tx(full, bytes);
-  for (int jj = 0; jj < nj; ++jj) {
+  return bytes;
+}
+__device__ void issue_down(const FusedArgs& a, const LayerPtr& L, const RouteSmem& rt, int blk, int j0, int nj,
+                           uint32_t dst, uint64_t* full, int lane) {
+  const Geometry& g = a.g;
+  const int Kmax = max(g.I, g.Is);
+  for (int c = lane; c < nj * (kFDims + 2); c += 32) {
+    const int jj = c / (kFDims + 2), r = c % (kFDims + 2);
     const bool sh = j0 + jj == 0;
     const int K = sh ? g.Is : g.I;
-    const QMatPtr W = sh ? L.sh_down : L.down;
+    const QMatPtr& W = sh ? L.sh_down : L.down;
     const size_t row0 = static_cast<size_t>(sh ? 0 : rt.slot_e[j0 + jj] * g.H) + blk * kFDims;
-    const uint32_t base = dst + jj * (9 * Kmax);
-    const uint32_t qb = kFDims * K / 2, sb = kFDims * K / 32;
-    tc::bulk_load(base, W.q + row0 * (K / 8), qb, full);
-    tc::bulk_load(base + 8 * Kmax, W.s + row0 * (K / kGroup), sb, full);
-    tc::bulk_load(base + 8 * Kmax + Kmax / 2, W.b + row0 * (K / kGroup), sb, full);
+    const uint32_t base = dst + jj * a.dslot;
+    if (r < kFDims)
+      tc::bulk_load(base + r * a.rs_dn, W.q + (row0 + r) * (K / 8), K / 2, full);
+    else
+      tc::bulk_load(base + kFDims * a.rs_dn + (r - kFDims) * (Kmax / 2), (r == kFDims ? W.s : W.b) +
+                    row0 * (K / kGroup), kFDims * K / 32, full);
   }
+}
+
+// Issue unit i of this CTA (layer L) into ring slot `dst` (whole producer warp).
+__device__ void issue_unit(const FusedArgs& a, const LayerPtr& L, const RouteSmem& rt, const Sched& s, int i,
+                           uint32_t dst, uint64_t* full, int lane) {
+  const Geometry& g = a.g;
+  if (i < s.my_gu) {
+    int slot, f0;
+    gu_unit(s, blockIdx.x + i * gridDim.x, slot, f0);
+    if (lane == 0) tc::mbar_arrive_expect_tx(full, gateup_bytes(g));
+    __syncwarp();
+    issue_gateup(a, L, rt.slot_e[slot], f0, dst, full, lane);
+    return;
+  }
+  const int di = i - s.my_gu;
+  const int blk = blockIdx.x + (di / s.n_down_parts) * gridDim.x;
+  const int j0 = (di % s.n_down_parts) * s.spd, nj = min(s.spd, s.n_slots - j0);
+  if (lane == 0) tc::mbar_arrive_expect_tx(full, down_bytes(g, j0, nj));
+  __syncwarp();
+  issue_down(a, L, rt, blk, j0, nj, dst, full, lane);
 }
 
 // This CTA's router rows of layer L (rows c, c+G, ... of [W_r; w_sg]) into
@@ -389,6 +491,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
     tc::mbar_init(rfree, 1);
     tc::mbar_init(ready, 1);
     rt.abort = 0;
+    rt.epoch = *reinterpret_cast<volatile const unsigned*>(a.bar + 2);
     tc::fence_barrier_init();
   }
   __syncthreads();
@@ -398,43 +501,50 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
     // Per layer: the routing-independent first unit (a shared-expert tile),
     // then, once the layer's routing is known, the next layer's router rows
     // and the rest of this layer's units.  Ring fills are numbered across
-    // layers in the order the consumers take them.
-    if (lane == 0) {
-      uint32_t fill = 0;             // ring fills issued
-      issue_router_rows(g, a.layers[0], nrows, tc::smem_u32(wr), rfull);
-      uint32_t rfills = 1;
-      bool ok = true;
-      for (int l = 0; l < a.n_layers && ok; ++l) {
-        const LayerPtr& L = a.layers[l];
-        const uint32_t base = fill;
-        if (early) {
-          const int sl = static_cast<int>(fill % a.ring);
-          if (!tc::mbar_wait(&empty[sl], ((fill / a.ring) & 1u) ^ 1u, abort_flag, a.status, a.wait_limit)) break;
-          tc::fence_proxy_async_smem();
-          issue_gateup(g, L, E, static_cast<int>(blockIdx.x) * kFFeat, ring0 + sl * a.slot_bytes, &full[sl]);
-          ++fill;
-        }
-        if (!tc::mbar_wait(ready, static_cast<uint32_t>(l) & 1u, abort_flag, a.status, a.wait_limit)) break;
-        const Sched s = make_sched(a, rt.n_act);
-        if (l + 1 < a.n_layers) {
-          // the consumers finished with this layer's router rows before its routing was ready
-          if (!tc::mbar_wait(rfree, static_cast<uint32_t>(l) & 1u, abort_flag, a.status, a.wait_limit)) break;
-          tc::fence_proxy_async_smem();
-          issue_router_rows(g, a.layers[l + 1], nrows, tc::smem_u32(wr), rfull);
-          ++rfills;
-        }
-        for (uint32_t i = fill - base; i < static_cast<uint32_t>(s.n_units); ++i) {
-          const int sl = static_cast<int>(fill % a.ring);
-          if (!tc::mbar_wait(&empty[sl], ((fill / a.ring) & 1u) ^ 1u, abort_flag, a.status, a.wait_limit)) {
-            ok = false;
-            break;
-          }
-          tc::fence_proxy_async_smem();   // consumers' generic reads of the slot precede the refill
-          issue_unit(a, L, rt, s, static_cast<int>(i), ring0 + sl * a.slot_bytes, &full[sl]);
-          ++fill;
-        }
+    // layers in the order the consumers take them.  The whole warp runs the
+    // loop (its waits are made warp-uniform) and issues each tile's row
+    // copies together.
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, tc::mbar_wait(bar, parity, abort_flag, a.status, a.wait_limit));
+    };
+    uint32_t fill = 0;             // ring fills issued
+    if (lane == 0) issue_router_rows(g, a.layers[0], nrows, tc::smem_u32(wr), rfull);
+    uint32_t rfills = 1;
+    bool ok = true;
+    for (int l = 0; l < a.n_layers && ok; ++l) {
+      const LayerPtr& L = a.layers[l];
+      const uint32_t base = fill;
+      if (early) {
+        const int sl = static_cast<int>(fill % a.ring);
+        if (!wait_all(&empty[sl], ((fill / a.ring) & 1u) ^ 1u)) break;
+        tc::fence_proxy_async_smem();
+        if (lane == 0) tc::mbar_arrive_expect_tx(&full[sl], gateup_bytes(g));
+        __syncwarp();
+        issue_gateup(a, L, E, static_cast<int>(blockIdx.x) * kFFeat, ring0 + sl * a.slot_bytes, &full[sl], lane);
+        ++fill;
       }
-      // every copy this thread issued has landed before the CTA may exit
+      if (!wait_all(ready, static_cast<uint32_t>(l) & 1u)) break;
+      const Sched s = make_sched(a, rt.n_act);
+      if (l + 1 < a.n_layers) {
+        // the consumers finished with this layer's router rows before its routing was ready
+        if (!wait_all(rfree, static_cast<uint32_t>(l) & 1u)) break;
+        tc::fence_proxy_async_smem();
+        if (lane == 0) issue_router_rows(g, a.layers[l + 1], nrows, tc::smem_u32(wr), rfull);
+        ++rfills;
+      }
+      for (uint32_t i = fill - base; i < static_cast<uint32_t>(s.n_units); ++i) {
+        const int sl = static_cast<int>(fill % a.ring);
+        if (!wait_all(&empty[sl], ((fill / a.ring) & 1u) ^ 1u)) {
+          ok = false;
+          break;
+        }
+        tc::fence_proxy_async_smem();   // consumers' generic reads of the slot precede the refill
+        issue_unit(a, L, rt, s, static_cast<int>(i), ring0 + sl * a.slot_bytes, &full[sl], lane);
+        ++fill;
+      }
+    }
+    // every copy this warp issued has landed before the CTA may exit
+    if (lane == 0) {
       tc::drain_ring(full, static_cast<uint32_t>(a.ring), fill, a.status);
       tc::drain_ring(rfull, 1u, rfills, a.status);
     }
@@ -446,10 +556,9 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
   const int tid = threadIdx.x, nthr = kFWarps * 32;
   const int lg4 = lane >> 2, lt = lane & 3;
   const int ngrp = g.H / kGroup;
-  const uint32_t qb = kFFeat * g.H / 2, sb = kFFeat * g.H / 32;
+  const uint32_t sb = kFFeat * g.H / 32;   // bytes of one scale (or bias) block of a gate/up tile
   const size_t act = static_cast<size_t>(T) * g.H;
   uint32_t fill = 0;      // ring fills consumed
-  unsigned nbar = 0;      // grid barriers passed
   // Abort handling: a wait that gives up raises rt.abort (and makes later
   // waits give up at once).  No consumer warp leaves a loop on its own: every
   // warp keeps taking the same CTA barriers, skipping the work, and the
@@ -461,17 +570,39 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
     bool ok = true;
 
     // -------------------------------------------------------------- phase A
-    // the layer input: x, or RMSNorm of the previous layer's output
-    if (l > 0) {
-      // warp t sums the CTAs' partials of token t: lane i takes CTAs i, i+32,
-      // ... (all loads in flight at once), then a fixed shuffle tree; the
-      // same order in every CTA
+    // the layer input: x, or RMSNorm of the previous layer's output, read
+    // from the exchange words as soon as every CTA has published its part
+    const uint32_t tag = (rt.epoch + 1u) * 64u + static_cast<uint32_t>(l);
+    const int c4 = 4 * tid;
+    const bool live = c4 < g.H;
+    uint2 xv[NT];
+    if (l == 0) {
+#pragma unroll
+      for (int t = 0; t < NT; ++t)
+        xv[t] = (live && t < T) ? __ldcg(reinterpret_cast<const uint2*>(a.x + static_cast<size_t>(t) * g.H + c4))
+                                : make_uint2(0u, 0u);
+    } else {
+      const long long deadline = clock64() + a.wait_limit;
+      const unsigned long long* yrow = a.yx + tid * 2;
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        xv[t] = make_uint2(0u, 0u);
+        if (live && t < T) {
+          xv[t].x = wait_word(yrow + t * (g.H / 2), tag - 1u, deadline, abort_flag, a.status, ok);
+          xv[t].y = wait_word(yrow + t * (g.H / 2) + 1, tag - 1u, deadline, abort_flag, a.status, ok);
+        }
+      }
+      // warp t sums the CTAs' partial sums of squares of token t: lane i
+      // takes CTAs i, i+32, ..., then a fixed shuffle tree; the same order in
+      // every CTA
       if (warp < T) {
         float part[kFMaxGrid / 32];
 #pragma unroll
         for (int j = 0; j < kFMaxGrid / 32; ++j) {
           const int c = lane + 32 * j;
-          part[j] = c < G ? __ldcg(a.sumsq + c * kFMaxT + warp) : 0.f;
+          part[j] = c < G ? __uint_as_float(wait_word(a.ssx + c * kFMaxT + warp, tag - 1u, deadline, abort_flag,
+                                                      a.status, ok))
+                          : 0.f;
         }
         float ss = 0.f;
 #pragma unroll
@@ -480,30 +611,25 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
         if (lane == 0) nrm[warp] = 1.0f / sqrtf(ss / static_cast<float>(g.H) + a.eps);
       }
       consumers_sync();
-    }
-    const uint16_t* src = l == 0 ? a.x : a.y;
-    const int c4 = 4 * tid;
-    const bool live = c4 < g.H;
-    uint2 xv[NT];
 #pragma unroll
-    for (int t = 0; t < NT; ++t) {
-      xv[t] = make_uint2(0u, 0u);
-      if (live && t < T) {
-        xv[t] = __ldcg(reinterpret_cast<const uint2*>(src + static_cast<size_t>(t) * g.H + c4));
-        if (l > 0) {
+      for (int t = 0; t < NT; ++t) {
+        if (live && t < T) {
           const float s = nrm[t];
           xv[t].x = pack_bf16x2(bf16_lo(xv[t].x) * s, bf16_hi(xv[t].x) * s);
           xv[t].y = pack_bf16x2(bf16_lo(xv[t].y) * s, bf16_hi(xv[t].y) * s);
         }
-        if (a.trace && blockIdx.x == 0)
-          *reinterpret_cast<uint2*>(a.trace + 2 * l * act + static_cast<size_t>(t) * g.H + c4) = xv[t];
       }
     }
+    if (a.trace && blockIdx.x == 0)
+#pragma unroll
+      for (int t = 0; t < NT; ++t)
+        if (live && t < T)
+          *reinterpret_cast<uint2*>(a.trace + 2 * l * act + static_cast<size_t>(t) * g.H + c4) = xv[t];
     // router rows r = c, c + G, ... (staged by the producer): thread tid owns
     // the inputs [4 tid, 4 tid + 4) of every row and token
     // (wait outcomes are made warp-uniform: the work they guard uses warp-collective instructions)
-    ok = __all_sync(0xffffffffu, tc::mbar_wait(rfull, static_cast<uint32_t>(l) & 1u, abort_flag, a.status,
-                                               a.wait_limit));
+    ok = __all_sync(0xffffffffu, ok && tc::mbar_wait(rfull, static_cast<uint32_t>(l) & 1u, abort_flag, a.status,
+                                                     a.wait_limit));
     float* part = lg;   // [nrows][kFWarps][NT] partials (lg is free until phase B)
     if (ok) {
       for (int r0 = 0; r0 < nrows; r0 += kFRouterRows) {
@@ -541,6 +667,14 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
       tc::fence_proxy_async_smem();      // the row buffer's generic reads precede its next TMA refill
       tc::mbar_arrive(rfree);
     }
+    if (ok && tid < nrows * T) {      // this CTA's logits go out first: every CTA waits for them
+      const int rr = tid / T, t = tid % T;
+      const int row = blockIdx.x + rr * G;
+      float v = 0.f;
+      for (int w = 0; w < kFWarps; ++w) v += part[(rr * kFWarps + w) * NT + t];
+      if (row < E && L.router_bias) v += L.router_bias[row];
+      st_word(a.lgx + static_cast<size_t>(t) * E1 + row, tag, __float_as_uint(v));
+    }
     for (int i = tid; i < T * ngrp; i += nthr) {     // sums over groups of 64 (fixed order)
       const uint4* r4 = reinterpret_cast<const uint4*>(xs) + i * 8;
       float sum = 0.f;
@@ -552,66 +686,63 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
       }
       xsum[i] = sum;
     }
-    if (ok && tid < nrows * T) {
-      const int rr = tid / T, t = tid % T;
-      const int row = blockIdx.x + rr * G;
-      float v = 0.f;
-      for (int w = 0; w < kFWarps; ++w) v += part[(rr * kFWarps + w) * NT + t];
-      if (row < E && L.router_bias) v += L.router_bias[row];
-      __stcg(a.logits + static_cast<size_t>(t) * E1 + row, v);
-    }
-    consumers_sync();
-    if (tid == 0) {
-      if (rt.abort || !grid_barrier(a.bar, (++nbar) * G, a.status, a.wait_limit)) rt.abort = 1;
+    consumers_sync();   // the partials in lg are consumed before phase B reuses it
+
+    // -------------------------------------------------------------- phase B
+    // Every CTA rebuilds the routing from all CTAs' logits (top-k by warp
+    // reductions, then a counting sort of the n = T*k <= 64 entries), so no
+    // further exchange is needed before the expert weights can be requested.
+    {
+      const long long deadline = clock64() + a.wait_limit;
+      for (int i = tid; i < T * E1; i += nthr)
+        lg[i] = __uint_as_float(wait_word(a.lgx + i, tag, deadline, abort_flag, a.status, ok));
     }
     consumers_sync();
     if (rt.abort) break;
-
-    // -------------------------------------------------------------- phase B
-    // Every CTA rebuilds the routing from the logits (top-k by warp
-    // reductions, then a counting sort of the n = T*k <= 64 entries), so no
-    // further barrier is needed before the expert weights can be requested.
-    for (int i = tid; i < T * E1; i += nthr) lg[i] = __ldcg(a.logits + i);
-    consumers_sync();
     if (warp < T) {
       topk_redux(lg + warp * E1, E, k, lane, rt.idx + warp * k, rt.w + warp * k);
       if (lane == 0) rt.sigma[warp] = sigmoid(lg[warp * E1 + E]);
     }
     consumers_sync();
-    if (tid < n) {
-      // stable rank: entries with a smaller expert, then earlier entries of
-      // the same expert; active experts below this one
-      const int e_i = rt.idx[tid];
-      int below = 0, rank = 0, abelow = 0, cnt = 0;
-      for (int j = 0; j < n; ++j) {
-        const int ej = rt.idx[j];
-        below += ej < e_i ? 1 : 0;
-        rank += (ej == e_i && j < tid) ? 1 : 0;
-        cnt += ej == e_i ? 1 : 0;
-        bool first_j = true;                              // entry j is its expert's first occurrence
-        for (int q = 0; q < j; ++q) first_j = first_j && rt.idx[q] != ej;
-        abelow += (first_j && ej < e_i) ? 1 : 0;
+    if (warp == 0) {
+      // grouping by one warp, O(n) per entry: first occurrences, then each
+      // entry's stable rank (entries with a smaller expert, then earlier
+      // entries of the same expert) and the active experts below its own
+      for (int i = lane; i < n; i += 32) {
+        const int e = rt.idx[i];
+        int f = 1;
+        for (int j = 0; j < i; ++j) f &= rt.idx[j] != e ? 1 : 0;
+        rt.first[i] = f;
       }
-      const int pos = below + rank;
-      rt.perm[pos] = tid;
-      rt.inv_perm[tid] = pos;
-      if (rank == 0) {
-        rt.slot_e[1 + abelow] = e_i;
-        rt.slot_cnt[1 + abelow] = cnt;
-        rt.slot_off[1 + abelow] = below;
-      }
-    }
-    if (tid == nthr - 1) {
+      __syncwarp();
       int nact = 0;
-      for (int j = 0; j < n; ++j) {
-        bool first_j = true;
-        for (int q = 0; q < j; ++q) first_j = first_j && rt.idx[q] != rt.idx[j];
-        nact += first_j ? 1 : 0;
+      for (int i = lane; i < n; i += 32) {
+        const int e_i = rt.idx[i];
+        int below = 0, rank = 0, abelow = 0, cnt = 0;
+        for (int j = 0; j < n; ++j) {
+          const int ej = rt.idx[j];
+          below += ej < e_i ? 1 : 0;
+          rank += (ej == e_i && j < i) ? 1 : 0;
+          cnt += ej == e_i ? 1 : 0;
+          abelow += (rt.first[j] && ej < e_i) ? 1 : 0;
+        }
+        const int pos = below + rank;
+        rt.perm[pos] = i;
+        rt.inv_perm[i] = pos;
+        if (rt.first[i]) {
+          rt.slot_e[1 + abelow] = e_i;
+          rt.slot_cnt[1 + abelow] = cnt;
+          rt.slot_off[1 + abelow] = below;
+          ++nact;
+        }
       }
-      rt.n_act = nact;
-      rt.slot_e[0] = E;
-      rt.slot_cnt[0] = T;
-      rt.slot_off[0] = Tk;
+      nact = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(nact)));
+      if (lane == 0) {
+        rt.n_act = nact;
+        rt.slot_e[0] = E;
+        rt.slot_cnt[0] = T;
+        rt.slot_off[0] = Tk;
+      }
     }
     consumers_sync();
     if (tid == 0) tc::mbar_arrive(ready);   // the producer may now schedule this layer's units
@@ -638,34 +769,14 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
         else
           for (int r = 0; r < rt.slot_cnt[slot]; ++r) tmask |= 1u << (rt.perm[rt.slot_off[slot] + r] / k);
         const uint8_t* ub = fsm + sl * a.slot_bytes;
-        const uint8_t* qrow = ub + m * qb + lg4 * (g.H / 2) + lt * 8;         // rows lg4, lg4 + 8
-        const uint16_t* srow = reinterpret_cast<const uint16_t*>(ub + 2 * qb + m * 2 * sb);
+        const uint8_t* qrow = ub + (m * kFFeat + lg4) * a.rs_gu + lt * 8;     // rows lg4, lg4 + 8
+        const uint16_t* srow = reinterpret_cast<const uint16_t*>(ub + 2 * kFFeat * a.rs_gu + m * 2 * sb);
         const uint16_t* brow = srow + sb / 2;
         const bool tok_live = lg4 < T && ((tmask >> lg4) & 1u);
         const uint4* xrow = reinterpret_cast<const uint4*>(xs + (tok_live ? lg4 : 0) * g.H) + lt * 2;
         float y[2][2] = {{0.f, 0.f}, {0.f, 0.f}};     // [row lg4 / lg4 + 8][token 2 lt / 2 lt + 1]
-        for (int G8 = ke * ge; got && G8 < (ke + 1) * ge; ++G8) {
-          const uint2 qa = *reinterpret_cast<const uint2*>(qrow + G8 * 32);
-          const uint2 qc = *reinterpret_cast<const uint2*>(qrow + 8 * (g.H / 2) + G8 * 32);
-          const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-          const uint4 xb0 = tok_live ? xrow[G8 * 8] : z, xb1 = tok_live ? xrow[G8 * 8 + 1] : z;
-          float d[4];
-          group_dot(d, qa, qc, xb0, xb1);
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const int t = 2 * lt + c;
-            if (t < T) {
-              const float X = xsum[t * ngrp + G8];
-#pragma unroll
-              for (int r = 0; r < 2; ++r) {
-                const int row = lg4 + 8 * r;
-                const float sc = bf16_bits_to_float(srow[row * ngrp + G8]);
-                const float bi = bf16_bits_to_float(brow[row * ngrp + G8]);
-                y[r][c] = fmaf(sc, d[2 * r + c] - 128.f * X, fmaf(bi, X, y[r][c]));
-              }
-            }
-          }
-        }
+        tile_groups<4>(y, qrow, a.rs_gu, srow, brow, ngrp, ke * ge, got ? ge : 0, xrow, tok_live, xsum, ngrp, T, lg4,
+                       lt);
         // every read of the unit's slot is done: release it (a slot that never
         // filled is not handed back: the producer is stopping as well)
         tc::fence_proxy_async_smem();
@@ -677,37 +788,36 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
 #pragma unroll
             for (int r = 0; r < 2; ++r) red[((m * 8 + ke) * 16 + lg4 + 8 * r) * NT + 2 * lt + c] = y[r][c];
         consumers_sync();
-        // h = bf16(silu(g) * u) for (feature, token); K eighths summed in order
-        if (tid < kFFeat * T && !rt.abort) {
-          const int f = tid / T, t = tid % T;
+        // h = bf16(silu(g) * u) for (feature pair, token); K eighths summed in
+        // order; each pair goes out as one exchange word of h row `pos`
+        // (routed rows in expert order, then the shared expert's rows)
+        if (tid < (kFFeat / 2) * T && !rt.abort) {
+          const int fp = tid / T, t = tid % T;
           bool member = slot == 0;
-          int pos = t;
+          int pos = Tk + t;
           for (int r = 0; r < (slot == 0 ? 0 : rt.slot_cnt[slot]); ++r)
             if (rt.perm[rt.slot_off[slot] + r] / k == t) {
               member = true;
               pos = rt.slot_off[slot] + r;
             }
           if (member) {
-            float gs = 0.f, us = 0.f;
+            uint32_t hv[2];
 #pragma unroll
-            for (int e8 = 0; e8 < 8; ++e8) {
-              gs += red[((0 * 8 + e8) * 16 + f) * NT + t];
-              us += red[((1 * 8 + e8) * 16 + f) * NT + t];
+            for (int q = 0; q < 2; ++q) {
+              const int f = 2 * fp + q;
+              float gs = 0.f, us = 0.f;
+#pragma unroll
+              for (int e8 = 0; e8 < 8; ++e8) {
+                gs += red[((0 * 8 + e8) * 16 + f) * NT + t];
+                us += red[((1 * 8 + e8) * 16 + f) * NT + t];
+              }
+              hv[q] = float_to_bf16_bits(silu(gs) * us);
             }
-            const uint16_t hv = float_to_bf16_bits(silu(gs) * us);
-            if (slot == 0)
-              a.h_s[static_cast<size_t>(t) * g.Is + f0 + f] = hv;
-            else
-              a.h[static_cast<size_t>(pos) * g.I + f0 + f] = hv;
+            st_word(a.hx + static_cast<size_t>(pos) * (Kmax / 2) + (f0 / 2 + fp), tag, hv[0] | (hv[1] << 16));
           }
         }
         consumers_sync();   // red is reused by the next unit
       }
-    }
-    // Every h row is written: grid barrier.
-    consumers_sync();
-    if (tid == 0) {
-      if (rt.abort || !grid_barrier(a.bar, (++nbar) * G, a.status, a.wait_limit)) rt.abort = 1;
     }
     consumers_sync();
     if (rt.abort) break;
@@ -715,16 +825,21 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
     // -------------------------------------------------------------- phase D
     if (s.my_blocks > 0) {
       // stage every h row (routed rows I wide, shared rows Is wide) in the
-      // interleaved K order, and its sums over groups of 64
+      // interleaved K order, as each CTA's gate/up units publish it, and its
+      // sums over groups of 64
+      const long long deadline = clock64() + a.wait_limit;
       const int vmax = Kmax / 8;
       for (int i = tid; i < (Tk + T) * vmax; i += nthr) {
         const int r = i / vmax, u = i - r * vmax;
         const bool shr = r >= Tk;
         if (u * 8 >= (shr ? g.Is : g.I)) continue;
-        const uint16_t* hsrc =
-            shr ? a.h_s + static_cast<size_t>(r - Tk) * g.Is : a.h + static_cast<size_t>(r) * g.I;
-        reinterpret_cast<uint4*>(hs + static_cast<size_t>(r) * Kmax)[u] =
-            interleave8(__ldcg(reinterpret_cast<const uint4*>(hsrc) + u));
+        const unsigned long long* w4 = a.hx + static_cast<size_t>(r) * (Kmax / 2) + u * 4;
+        uint4 v;
+        v.x = wait_word(w4, tag, deadline, abort_flag, a.status, ok);
+        v.y = wait_word(w4 + 1, tag, deadline, abort_flag, a.status, ok);
+        v.z = wait_word(w4 + 2, tag, deadline, abort_flag, a.status, ok);
+        v.w = wait_word(w4 + 3, tag, deadline, abort_flag, a.status, ok);
+        reinterpret_cast<uint4*>(hs + static_cast<size_t>(r) * Kmax)[u] = interleave8(v);
       }
       consumers_sync();
       const int kg = Kmax / kGroup;
@@ -766,35 +881,16 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
         const int pos0 = jlive ? rt.slot_off[j] : 0;
         float y[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
         if (jlive) {
-          const uint8_t* ub = fsm + sl * a.slot_bytes + jj * (9 * Kmax);
-          const uint8_t* qrow = ub + lg4 * (K / 2) + lt * 8;
-          const uint16_t* srow = reinterpret_cast<const uint16_t*>(ub + 8 * Kmax);
-          const uint16_t* brow = reinterpret_cast<const uint16_t*>(ub + 8 * Kmax + Kmax / 2);
+          const uint8_t* ub = fsm + sl * a.slot_bytes + jj * a.dslot;
+          const uint8_t* qrow = ub + lg4 * a.rs_dn + lt * 8;
+          const uint16_t* srow = reinterpret_cast<const uint16_t*>(ub + kFDims * a.rs_dn);
+          const uint16_t* brow = reinterpret_cast<const uint16_t*>(ub + kFDims * a.rs_dn + Kmax / 2);
           const bool tok_live = lg4 < nt;
           const int hr = pos0 + (tok_live ? lg4 : 0);
           const uint4* hrow = reinterpret_cast<const uint4*>(hs + static_cast<size_t>(hr) * Kmax) + lt * 2;
-          for (int G8 = kh * gh; G8 < (kh + 1) * gh; ++G8) {
-            const uint2 qa = *reinterpret_cast<const uint2*>(qrow + G8 * 32);
-            const uint2 qc = *reinterpret_cast<const uint2*>(qrow + 8 * (K / 2) + G8 * 32);
-            const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-            const uint4 hb0 = tok_live ? hrow[G8 * 8] : z, hb1 = tok_live ? hrow[G8 * 8 + 1] : z;
-            float d[4];
-            group_dot(d, qa, qc, hb0, hb1);
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-              const int t = 2 * lt + c;
-              if (t < nt) {
-                const float X = hsum[(pos0 + t) * kg + G8];
-#pragma unroll
-                for (int r = 0; r < 2; ++r) {
-                  const int row = lg4 + 8 * r;
-                  const float sc = bf16_bits_to_float(srow[row * ng + G8]);
-                  const float bi = bf16_bits_to_float(brow[row * ng + G8]);
-                  y[r][c] = fmaf(sc, d[2 * r + c] - 128.f * X, fmaf(bi, X, y[r][c]));
-                }
-              }
-            }
-          }
+          for (int gb = 0; gb < gh; gb += 4)
+            tile_groups<4>(y, qrow, a.rs_dn, srow, brow, ng, kh * gh + gb, min(4, gh - gb), hrow, tok_live,
+                           hsum + pos0 * kg, kg, nt, lg4, lt);
         }
         tc::fence_proxy_async_smem();
         __syncwarp();
@@ -818,29 +914,40 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
     }
     consumers_sync();
     if (rt.abort) break;
-    // combine: out[t, d] = bf16( sum_j w[t,j] * y[inv_perm[t k + j]][d] + sigma_t * y[T k + t][d] );
-    // between layers the CTA also sums the squares of its bf16 outputs per token
-    uint16_t* dst = last ? a.out : a.y;
-    for (int i = tid; i < T * s.my_blocks * kFDims; i += nthr) {
-      const int t = i / (s.my_blocks * kFDims), rem = i % (s.my_blocks * kFDims);
-      const int bl = rem / kFDims, d = rem % kFDims;
-      float acc = 0.f;
-      for (int j = 0; j < k; ++j)
-        acc = fmaf(rt.w[t * k + j], ys[(rt.inv_perm[t * k + j] * s.my_blocks + bl) * kFDims + d], acc);
-      acc = fmaf(rt.sigma[t], ys[((Tk + t) * s.my_blocks + bl) * kFDims + d], acc);
+    // combine: out[t, d] = bf16( sum_j w[t,j] * y[inv_perm[t k + j]][d] + sigma_t * y[T k + t][d] ),
+    // two adjacent dims per thread; between layers the outputs go out as
+    // exchange words and the CTA also sums the squares of its bf16 outputs
+    // per token (dim pairs in order)
+    for (int i = tid; i < T * s.my_blocks * (kFDims / 2); i += nthr) {
+      const int t = i / (s.my_blocks * (kFDims / 2)), rem = i % (s.my_blocks * (kFDims / 2));
+      const int bl = rem / (kFDims / 2), d = 2 * (rem % (kFDims / 2));
+      uint32_t ov[2];
+      float sq = 0.f;
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        float acc = 0.f;
+        for (int j = 0; j < k; ++j)
+          acc = fmaf(rt.w[t * k + j], ys[(rt.inv_perm[t * k + j] * s.my_blocks + bl) * kFDims + d + q], acc);
+        acc = fmaf(rt.sigma[t], ys[((Tk + t) * s.my_blocks + bl) * kFDims + d + q], acc);
+        ov[q] = float_to_bf16_bits(acc);
+        sq = fmaf(bf16_bits_to_float(ov[q]), bf16_bits_to_float(ov[q]), sq);
+      }
       const int blk = blockIdx.x + bl * G;
-      const uint16_t ov = float_to_bf16_bits(acc);
       const size_t o = static_cast<size_t>(t) * g.H + blk * kFDims + d;
-      dst[o] = ov;
-      if (a.trace) a.trace[(2 * l + 1) * act + o] = ov;
-      if (!last) lg[i] = bf16_bits_to_float(ov) * bf16_bits_to_float(ov);
+      const uint32_t pair = ov[0] | (ov[1] << 16);
+      if (last)
+        *reinterpret_cast<uint32_t*>(a.out + o) = pair;
+      else
+        st_word(a.yx + o / 2, tag, pair);
+      if (a.trace) *reinterpret_cast<uint32_t*>(a.trace + (2 * l + 1) * act + o) = pair;
+      lg[i] = sq;
     }
     if (!last) {
       consumers_sync();
       if (tid < T) {
         float ss = 0.f;
-        for (int q = 0; q < s.my_blocks * kFDims; ++q) ss += lg[tid * s.my_blocks * kFDims + q];
-        __stcg(a.sumsq + blockIdx.x * kFMaxT + tid, ss);
+        for (int q = 0; q < s.my_blocks * (kFDims / 2); ++q) ss += lg[tid * s.my_blocks * (kFDims / 2) + q];
+        st_word(a.ssx + blockIdx.x * kFMaxT + tid, tag, __float_as_uint(ss));
       }
     } else if (blockIdx.x == 0 && a.r.topk_idx) {
       // routing outputs of the last layer (off the other CTAs' critical path)
@@ -866,19 +973,13 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
         *a.n_active = rt.n_act + 1;
       }
     }
-    // the layer's outputs are complete once every CTA passes the next barrier
-    if (!last) {
-      consumers_sync();
-      if (tid == 0) {
-        if (rt.abort || !grid_barrier(a.bar, (++nbar) * G, a.status, a.wait_limit)) rt.abort = 1;
-      }
-      consumers_sync();
-      if (rt.abort) break;
-    }
+    // the next layer reads the outputs from the exchange words; its phase A
+    // reuses shared memory the combine still reads
+    consumers_sync();
   }
   // (after an abort, rt.abort also stops a producer still waiting for a
   // layer that will not come)
-  if (tid == 0) grid_exit(a.bar, gridDim.x);
+  if (tid == 0) launch_exit(a.bar, gridDim.x);
 }
 
 int fused_grid() {
@@ -893,15 +994,18 @@ int fused_grid() {
 
 // Shared-memory carve-up of one launch (identical for every layer).
 struct FusedLayout {
-  int ring, slot_bytes, spd, rows_per_cta;
+  int ring, slot_bytes, spd, rows_per_cta, rs_gu, rs_dn, dslot;
   int off_bar, off_wr, off_xs, off_xsum, off_lg, off_rt, off_y, off_nrm, total;
 };
 
 FusedLayout fused_layout(const Geometry& g, int G) {
   FusedLayout f{};
   const int Kmax = g.I > g.Is ? g.I : g.Is;
-  f.slot_bytes = 18 * g.H;                                   // one gate/up unit
-  f.spd = f.slot_bytes / (9 * Kmax);
+  f.rs_gu = g.H / 2 + kFRowPad;
+  f.rs_dn = Kmax / 2 + kFRowPad;
+  f.dslot = kFDims * f.rs_dn + Kmax;                        // codes, then scales and biases
+  f.slot_bytes = 2 * kFFeat * f.rs_gu + 4 * (kFFeat * g.H / 32);   // one gate/up unit
+  f.spd = f.slot_bytes / f.dslot;
   if (f.spd > kFMaxSpd) f.spd = kFMaxSpd;
   f.rows_per_cta = (g.E + 1 + G - 1) / G;
   const int rows = g.T * g.k + g.T;
@@ -940,22 +1044,25 @@ FusedLayout fused_layout(const Geometry& g, int G) {
 bool decode_fused_supported(const Geometry& g) {
   if (g.T < 1 || g.T > kFMaxT) return false;
   if (g.H % 1024 || g.H > 2048) return false;
-  if (g.I % kFFeat || g.Is % kFFeat) return false;
-  const int Kmax = g.I > g.Is ? g.I : g.Is;
-  if (9 * Kmax > 18 * g.H) return false;                  // at least one expert slot per down unit
+  if (g.I % kGroup || g.Is % kGroup) return false;      // whole groups: every staged row is 16-byte sized
   const int G = fused_grid();
   if (G > kFMaxGrid || G > kFusedMaxGrid) return false;
+  // Every CTA must own a router row: a CTA's logits of layer l + 1 are
+  // published only after it has read everything of layer l, and every
+  // reader of layer l + 1's data first waits for all CTAs' logits, which is
+  // what makes reusing the exchange words from layer to layer safe.
+  if (G > g.E + 1) return false;
   if ((g.E + 1 + G - 1) / G > kFMaxRouterRows) return false;
   const FusedLayout f = fused_layout(g, G);
-  return f.ring >= 2 && f.total <= 227 * 1024;
+  return f.spd >= 1 && f.ring >= 2 && f.total <= 227 * 1024;   // spd: at least one expert slot per down unit
 }
 
 int decode_fused_max_layers() { return kFMaxLayers; }
 
 cudaError_t launch_decode_fused(const Geometry& g, const LayerPtr* layers, int n_layers, const uint16_t* x,
-                                uint16_t* out, uint16_t* y, float* sumsq, uint16_t* trace, float eps,
-                                const RoutingPtrs& r, int32_t* active, int32_t* n_active, float* logits, uint16_t* h,
-                                uint16_t* h_s, unsigned* bar, int* status, cudaStream_t s) {
+                                uint16_t* out, uint16_t* trace, float eps, const RoutingPtrs& r, int32_t* active,
+                                int32_t* n_active, const FusedExchange& xch, unsigned* bar, int* status,
+                                cudaStream_t s) {
   if (n_layers < 1 || n_layers > kFMaxLayers || !decode_fused_supported(g)) return cudaErrorInvalidValue;
   FusedArgs a{};
   a.g = g;
@@ -963,15 +1070,14 @@ cudaError_t launch_decode_fused(const Geometry& g, const LayerPtr* layers, int n
   a.eps = eps;
   a.x = x;
   a.out = out;
-  a.y = y;
-  a.sumsq = sumsq;
   a.trace = trace;
   a.r = r;
   a.active = active;
   a.n_active = n_active;
-  a.logits = logits;
-  a.h = h;
-  a.h_s = h_s;
+  a.lgx = xch.logits;
+  a.hx = xch.h;
+  a.yx = xch.y;
+  a.ssx = xch.sumsq;
   a.bar = bar;
   a.status = status;
   a.wait_limit = wait_limit_cycles();
@@ -982,6 +1088,9 @@ cudaError_t launch_decode_fused(const Geometry& g, const LayerPtr* layers, int n
   a.slot_bytes = f.slot_bytes;
   a.spd = f.spd;
   a.rows_per_cta = f.rows_per_cta;
+  a.rs_gu = f.rs_gu;
+  a.rs_dn = f.rs_dn;
+  a.dslot = f.dslot;
   a.off_bar = f.off_bar;
   a.off_wr = f.off_wr;
   a.off_xs = f.off_xs;

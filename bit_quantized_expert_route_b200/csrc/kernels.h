@@ -137,17 +137,33 @@ cudaError_t launch_decode_down_combine(const Geometry& g, const LayerPtr& L, con
 
 // decode_fused.cu: a stack of 1..decode_fused_max_layers() decode layers
 // (T <= 8, H = 1024 or 2048) in one cooperative launch; layer l > 0 takes
-// RMSNorm(eps) of layer l-1's output.  y: workspace [T, H] bf16 (outputs
-// between layers); sumsq: workspace [kFusedMaxGrid][8] FP32; bar: two zeroed
-// workspace words (grid barrier arrivals and exits); logits: workspace
-// [T, E+1] FP32; trace: NULL or [n_layers][2][T][H]; r.topk_idx NULL: no
-// routing outputs (else those of the last layer).
+// RMSNorm(eps) of layer l-1's output.  The CTAs exchange logits, h and the
+// layer outputs through tagged 64-bit words in the workspace (FusedExchange,
+// sizes from fused_exchange_words).  bar: workspace words [1] exit counter
+// and [2] epoch (zero in a new workspace); trace: NULL or
+// [n_layers][2][T][H]; r.topk_idx NULL: no routing outputs (else those of
+// the last layer).
 constexpr int kFusedMaxGrid = 1024;
+struct FusedExchange {
+  unsigned long long* logits;   // [T][E+1]
+  unsigned long long* h;        // [T*k + T][max(I, Is)/2]
+  unsigned long long* y;        // [T][H/2]
+  unsigned long long* sumsq;    // [kFusedMaxGrid][8]
+};
+inline size_t fused_exchange_words(int T, int H, int I, int Is, int E, int k, int which) {
+  const int Kmax = I > Is ? I : Is;
+  switch (which) {
+    case 0: return static_cast<size_t>(T) * (E + 1);
+    case 1: return static_cast<size_t>(T * k + T) * (Kmax / 2);
+    case 2: return static_cast<size_t>(T) * (H / 2);
+    default: return static_cast<size_t>(kFusedMaxGrid) * 8;
+  }
+}
 bool decode_fused_supported(const Geometry& g);
 int decode_fused_max_layers();
 cudaError_t launch_decode_fused(const Geometry& g, const LayerPtr* layers, int n_layers, const uint16_t* x,
-                                uint16_t* out, uint16_t* y, float* sumsq, uint16_t* trace, float eps,
-                                const RoutingPtrs& r, int32_t* active, int32_t* n_active, float* logits, uint16_t* h,
-                                uint16_t* h_s, unsigned* bar, int* status, cudaStream_t s);
+                                uint16_t* out, uint16_t* trace, float eps, const RoutingPtrs& r, int32_t* active,
+                                int32_t* n_active, const FusedExchange& xch, unsigned* bar, int* status,
+                                cudaStream_t s);
 
 }  // namespace moe

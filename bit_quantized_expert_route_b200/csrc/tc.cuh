@@ -42,6 +42,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Default limit of a bounded wait, in SM clock cycles (~2 s at 1.9 GHz).
 // Waits that drain copies or tensor-core work already issued always use it.
 constexpr long long kDefaultWaitLimit = 1ll << 32;
@@ -50,15 +63,18 @@ constexpr long long kDefaultWaitLimit = 1ll << 32;
 // after `limit` cycles of device clock or as soon as another thread of the CTA
 // has given up (*abort != 0); on giving up it records the timeout in the
 // status word and raises *abort.  Returns false when it gave up.  Short limits
-// (failure-injection runs) are checked on every poll, the default one every
+// (failure-injection runs) are checked on every poll and poll with the
+// non-blocking test_wait (try_wait may itself wait for a while inside the
+// hardware, longer than such a limit); the default limit is checked every
 // 256 polls.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* status,
                                           long long limit = kDefaultWaitLimit) {
-  if (mbar_try_wait(bar, parity)) return true;
+  const bool short_limit = limit < (1ll << 24);
+  if (short_limit ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
   const long long deadline = clock64() + limit;
-  const uint32_t check_mask = limit < (1ll << 24) ? 0u : 255u;
+  const uint32_t check_mask = short_limit ? 0u : 255u;
   for (uint32_t n = 1;; ++n) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (short_limit ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
     if ((n & check_mask) == 0) {
       if (*abort) return false;
       if (clock64() > deadline) {

@@ -22,6 +22,7 @@ MOE_ERR_UNSUPPORTED = -2
 MOE_ERR_WORKSPACE = -3
 MOE_ERR_CUDA = -4
 MOE_ERR_DEVICE_TIMEOUT = -5
+MOE_ERR_DEVICE_INDEX = -6
 
 # Every entry point declared in include/moe.h.
 EXPORTS = ("moe_workspace_size", "moe_route", "moe_forward", "moe_decode", "moe_forward_host", "moe_forward_host_async",

@@ -218,3 +218,42 @@ def make_attention_case(seed: int, ctx_lens, Hq: int = 16, Hkv: int = 2, D: int 
     k = to_bf16_bits(rng.normal(0.0, 1.0, size=(n_blocks, Hkv, block, D)))
     v = to_bf16_bits(rng.normal(0.0, 1.0, size=(n_blocks, Hkv, block, D)))
     return AttnCase(q, k, v, table, ctx)
+
+
+@dataclasses.dataclass
+class AttnDeviceCase:
+    """An attention case generated on the device (full-size inputs): torch tensors."""
+    q: torch.Tensor             # bf16 [B, Hq, D]
+    k_cache: torch.Tensor       # bf16 [n_blocks, Hkv, block, D]
+    v_cache: torch.Tensor
+    block_table: torch.Tensor   # int32 [B, max_blocks]
+    ctx_len: torch.Tensor       # int32 [B]
+
+
+def make_attention_case_on_device(seed: int, ctx_lens, device, Hq: int = 16, Hkv: int = 2, D: int = 256,
+                                  block: int = 64, spare_blocks: int = 3) -> AttnDeviceCase:
+    """The recipe of make_attention_case drawn by torch's generator on `device` (a different
+    stream of numbers): q, k, v ~ N(0, 1) bf16, one seeded permutation of the physical blocks."""
+    g = torch.Generator(device=device)
+    g.manual_seed((seed * 3_000_017 + _KEY_ATTN) & 0x7FFFFFFF)
+    ctx = [int(n) for n in ctx_lens]
+    per_seq = [(n + block - 1) // block for n in ctx]
+    n_blocks = sum(per_seq) + spare_blocks
+    phys = torch.randperm(n_blocks, generator=g, device=device).to(torch.int32)
+    table = torch.full((len(ctx), max(per_seq)), -1, dtype=torch.int32, device=device)
+    pos = 0
+    for b, nb in enumerate(per_seq):
+        table[b, :nb] = phys[pos:pos + nb]
+        pos += nb
+    q = torch.randn((len(ctx), Hq, D), generator=g, device=device).to(torch.bfloat16)
+    k = torch.randn((n_blocks, Hkv, block, D), generator=g, device=device).to(torch.bfloat16)
+    v = torch.randn((n_blocks, Hkv, block, D), generator=g, device=device).to(torch.bfloat16)
+    return AttnDeviceCase(q, k, v, table, torch.tensor(ctx, dtype=torch.int32, device=device))
+
+
+def attention_case_to_host(c: AttnDeviceCase) -> AttnCase:
+    """The same inputs in the storage form of make_attention_case (bf16 bit patterns)."""
+    def bits(t):
+        return t.detach().cpu().view(torch.int16).numpy().view(np.uint16).copy()
+    return AttnCase(bits(c.q), bits(c.k_cache), bits(c.v_cache), c.block_table.cpu().numpy().copy(),
+                    c.ctx_len.cpu().numpy().copy())

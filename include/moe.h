@@ -88,7 +88,8 @@ typedef enum {
   MOE_ERR_UNSUPPORTED = -2,     /* layout other than affine 4-bit / group 64, sizes not supported */
   MOE_ERR_WORKSPACE = -3,       /* workspace NULL, too small, or misaligned */
   MOE_ERR_CUDA = -4,            /* a CUDA runtime call or kernel launch failed */
-  MOE_ERR_DEVICE_TIMEOUT = -5   /* a bounded device-side wait gave up */
+  MOE_ERR_DEVICE_TIMEOUT = -5,  /* a bounded device-side wait gave up */
+  MOE_ERR_DEVICE_INDEX = -6     /* a device-side bounds check found an index out of range (attn.h) */
 } moe_status;
 
 /* One affine 4-bit matrix (or a stack of E of them); see "Storage" above. */
