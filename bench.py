@@ -46,6 +46,7 @@ sys.path.insert(0, ROOT)
 T_PREFILL = 4096
 SWEEP_T = (1, 8, 64, 512, 4096, 16384)
 ATTN_L = (4096, 32768, 131072)    # decode-attention context lengths (one sequence, 16 Q heads, 2 KV heads, D=256)
+GDN_B = (1, 8, 64)                # recurrence batch sizes (16 key heads, 32 value heads, 128 x 128 FP32 state)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PREFILL_LAUNCHES_PER_STEP = 7     # router (+ segment counts), scan, scatter, gather, gate/up, down, combine
 UNFUSED_DECODE_LAUNCHES = 3       # routing (router+top-k+sort), gate/up GEMV, down GEMV+combine
@@ -82,6 +83,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-zipf-prefill", action="store_true", help="skip the skewed prefill workload")
     ap.add_argument("--decode-only", action="store_true", help="only the decode measurement (profiling)")
     ap.add_argument("--attn-only", action="store_true", help="only the decode-attention measurement (profiling)")
+    ap.add_argument("--no-gdn", action="store_true", help="skip the Gated DeltaNet recurrence workload")
+    ap.add_argument("--gdn-only", action="store_true", help="only the recurrence measurement (profiling)")
+    ap.add_argument("--gdn-B", type=str, default=",".join(str(n) for n in GDN_B))
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass (profiling)")
     ap.add_argument("--no-stages", action="store_true", help="skip the per-stage traced pass (profiling)")
     ap.add_argument("--layers", type=int, default=4, help="prefill layers cycled")
@@ -590,6 +594,67 @@ def attention_phase(a, world, rank, dev, peaks, peak_src):
             "points": pts}
 
 
+def gdn_phase(a, world, rank, dev, peaks, peak_src):
+    """One Gated DeltaNet decode step (gdn_decode_step) for B sequences: 16 key heads, 32 value heads,
+    128 x 128 FP32 state per value head, updated in place.  Per-launch CUDA events with a 512 MB
+    write between launches (the state is read from HBM even where it fits in L2)."""
+    import torch
+    from bit_quantized_expert_route_b200 import deltanet, moe, synth
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    Hk, Hv, dk, dv = 16, 32, 128, 128
+    pts = {}
+    for B in [int(n) for n in a.gdn_B.split(",") if n]:
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(910 + 31 * rank + B)
+        q = torch.randn((B, Hk, dk), generator=gen, device=dev).to(torch.bfloat16)
+        k = torch.randn((B, Hk, dk), generator=gen, device=dev).to(torch.bfloat16)
+        v = torch.randn((B, Hv, dv), generator=gen, device=dev).to(torch.bfloat16)
+        g = torch.log(torch.rand((B, Hv), generator=gen, device=dev) * 0.149 + 0.85)
+        beta = torch.rand((B, Hv), generator=gen, device=dev) * 0.9 + 0.05
+        state = torch.randn((B, Hv, dv, dk), generator=gen, device=dev) * 0.05
+        out = torch.empty_like(v)
+        for _ in range(max(3, a.warmup)):
+            deltanet.gdn_decode_step(q, k, v, g, beta, state, out)
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(a.attn_reps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            deltanet.gdn_decode_step(q, k, v, g, beta, state, out)
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        ms = max_over_ranks(statistics.median(ts), world)
+        nb = B * Hv * dv * dk * 4 * 2 + B * (2 * Hk * dk + 2 * Hv * dv) * 2 + B * Hv * 8
+        pts[str(B)] = {"us": round(ms * 1e3, 3), "tokens_per_s": round(whole_job_rate(B, world, ms), 1),
+                       "bytes": nb, "launches_per_step": 1,
+                       "roofline": hbm_roofline("gdn_step_kernel<128>", nb, ms, peaks, peak_src)}
+        del q, k, v, g, beta, state, out
+        torch.cuda.empty_cache()
+    del flush
+    torch.cuda.empty_cache()
+    return {"workload": "Gated DeltaNet decode step, 16 key heads / 32 value heads, 128 x 128 FP32 state per value "
+                        "head, q, k, v ~ N(0,1) bf16, alpha ~ U(0.85, 0.999), beta ~ U(0.05, 0.95)",
+            "timing": "median of per-launch CUDA-event times, L2 flushed (512 MB write) between launches",
+            "roofline_note": "algorithmic bytes = the state read and written (B x 32 x 128 x 128 x 4 B x 2) "
+                             "+ q, k, v, out, g, beta",
+            "points": pts}
+
+
+def gdn_oracle_times():
+    """The float64 recurrence oracle on this host for every batch size of the workload."""
+    from bit_quantized_expert_route_b200 import synth
+    from oracle import deltanet_ref
+    res = {}
+    for B in GDN_B:
+        c = synth.make_deltanet_case(910, B)
+        t0 = time.perf_counter()
+        deltanet_ref.recurrent_step(c.q, c.k, c.v, c.g, c.beta, c.state)
+        res[str(B)] = {"seconds": round(time.perf_counter() - t0, 3)}
+    return res
+
+
 def attention_oracle_times():
     """The float64 attention oracle on this host for every context length of the workload."""
     from bit_quantized_expert_route_b200 import synth
@@ -662,6 +727,8 @@ def oracle_phase(a):
     res["sweep_layer0"] = sw
     if not a.no_attn:
         res["attention"] = attention_oracle_times()
+    if not a.no_gdn:
+        res["gated_deltanet"] = gdn_oracle_times()
     cpu_baseline = {"value": res["prefill_uniform"]["tokens_per_s"], "unit": "tokens/s", "cores": cores,
                     "kind": "oracle", "sample": "the whole uniform prefill input (4096 tokens), one call, "
                                                 "NumPy float64, BLAS threads = cores",
@@ -684,9 +751,12 @@ def run_ours(a):
 
     clk = ClockSampler(torch.cuda.current_device()).__enter__()   # sampled across every timed phase
     pre = {}
-    if a.attn_only:
+    if a.attn_only or a.gdn_only:
         a.decode_only, a.no_decode = True, True
-        workloads["attention"] = attention_phase(a, world, rank, dev, peaks, peak_src)
+        if a.attn_only:
+            workloads["attention"] = attention_phase(a, world, rank, dev, peaks, peak_src)
+        if a.gdn_only:
+            workloads["gated_deltanet"] = gdn_phase(a, world, rank, dev, peaks, peak_src)
     if not a.decode_only:
         pre = prefill_phase(a, world, rank, dev, dims, zipf, peaks, peak_src, e2e=True)
         if not a.no_zipf_prefill and not zipf:
@@ -704,6 +774,8 @@ def run_ours(a):
         workloads["tiny"] = tiny_phase(a, world, dev)
     if not a.no_attn and not a.decode_only:
         workloads["attention"] = attention_phase(a, world, rank, dev, peaks, peak_src)
+    if not a.no_gdn and not a.decode_only:
+        workloads["gated_deltanet"] = gdn_phase(a, world, rank, dev, peaks, peak_src)
     clk.__exit__(None, None, None)
     clocks = clk.summary()
 

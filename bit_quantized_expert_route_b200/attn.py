@@ -44,7 +44,7 @@ def alloc_workspace(B: int, Hkv: int, D: int, block: int, max_blocks: int, devic
 
 
 def plan(B: int, Hkv: int, block: int, max_blocks: int) -> tuple[int, int]:
-    """(ranges per sequence and key/value head, 32-position chunks per range)."""
+    """(ranges per sequence and key/value head, 16-position chunks per range)."""
     ns, cps = ctypes.c_int(0), ctypes.c_int(0)
     moe._check(library().attn_decode_plan(B, Hkv, block, max_blocks, ctypes.byref(ns), ctypes.byref(cps)),
                "attn_decode_plan")

@@ -13,13 +13,15 @@
 //
 // Design.
 //   * Grid (n_split, Hkv, B): CTA (s, g, b) takes a contiguous range of
-//     32-position chunks of sequence b's key/value head g.  One producer
+//     16-position chunks of sequence b's key/value head g.  One producer
 //     thread streams each chunk's keys and values with TMA tiled copies
-//     (D / 64 boxes of 32 rows x 128 B per cache, 128-byte swizzle) into a
-//     ring of shared-memory stages; four consumer warps take the chunks in
-//     turn, each keeping its own running maximum, weight sum and output.
-//   * Per chunk a warp computes S^T = K Q^T on mma.sync m16n8k16 with the 32
-//     positions as M (two tiles) and the group's heads as the 8 columns, so
+//     (D / 64 boxes of 16 rows x 128 B per cache, 128-byte swizzle) into a
+//     ring of shared-memory stages (12 for D = 256: three per consumer warp,
+//     so a warp computes on one chunk while its next two are in flight);
+//     four consumer warps take the chunks in turn, each keeping its own
+//     running maximum, weight sum and output.
+//   * Per chunk a warp computes S^T = K Q^T on mma.sync m16n8k16 with the 16
+//     positions as M and the group's heads as the 8 columns, so
 //     no tensor-core row is padding; the keys come from shared memory by
 //     ldmatrix (the swizzle makes the 8 rows of a matrix hit 8 different
 //     bank groups).  The weights P^T (bf16) become the B operand of
@@ -45,19 +47,20 @@
 namespace moe {
 namespace {
 
-constexpr int kAChunk = 32;                     // positions per pipeline stage
+constexpr int kAChunk = 16;                     // positions per pipeline stage (one m16 tile)
+constexpr int kAMT = kAChunk / 16;              // m16 tiles per stage
 constexpr int kABoxCols = 64;                   // elements per swizzled box row (128 B)
-constexpr int kABoxBytes = kAChunk * 128;       // one box: 32 rows x 128 B
+constexpr int kABoxBytes = kAChunk * 128;       // one box: 16 rows x 128 B
 constexpr int kAWarps = 4;                      // consumer warps
 constexpr int kAThreads = (kAWarps + 1) * 32;   // + the producer warp
 constexpr int kAMaxGroup = 8;                   // query heads per key/value head: the n8 columns
-constexpr int kARingMax = 8;
+constexpr int kARingMax = 24;
 constexpr int kACombThreads = 256;              // combine CTA: 32 dims x 8 warps over the ranges
 constexpr int kAMaxSplit = 1024;                // ranges per (sequence, KV head) the combine takes
 constexpr int kATabCache = 512;                 // block-table entries a CTA fetches up front
 
 struct alignas(64) AttnArgs {
-  CUtensorMap tk, tv;          // caches as [n_blocks * Hkv * block rows][D], box 32 rows x 64 cols, 128B swizzle
+  CUtensorMap tk, tv;          // caches as [n_blocks * Hkv * block rows][D], box 16 rows x 64 cols, 128B swizzle
   const uint16_t* q;           // [B][Hq][D]
   const int32_t* table;        // [B][max_blocks]
   const int32_t* ctx;          // [B]
@@ -254,9 +257,9 @@ __global__ void __launch_bounds__(kAThreads, 1) attn_decode_kernel(const __grid_
       }
       const uint32_t kb = sbase + sl * STAGE, vb = kb + HALF;
       // S^T = K Q^T for the two 16-row tiles
-      float s[2][4], s2[2][4];   // even and odd k-steps accumulate apart (two dependency chains)
+      float s[kAMT][4], s2[kAMT][4];   // even and odd k-steps accumulate apart (two dependency chains)
 #pragma unroll
-      for (int mt = 0; mt < 2; ++mt) {
+      for (int mt = 0; mt < kAMT; ++mt) {
         s[mt][0] = s[mt][1] = s[mt][2] = s[mt][3] = 0.f;
         s2[mt][0] = s2[mt][1] = s2[mt][2] = s2[mt][3] = 0.f;
         const int row = mt * 16 + mr + 8 * (mi & 1);
@@ -272,7 +275,7 @@ __global__ void __launch_bounds__(kAThreads, 1) attn_decode_kernel(const __grid_
       // scale, mask, running maximum per head column
       float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-      for (int mt = 0; mt < 2; ++mt)
+      for (int mt = 0; mt < kAMT; ++mt)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const bool live = mt * 16 + r8 + 8 * h < nv;
@@ -289,7 +292,7 @@ __global__ void __launch_bounds__(kAThreads, 1) attn_decode_kernel(const __grid_
       m1 = n1;
       float ps0 = 0.f, ps1 = 0.f;
 #pragma unroll
-      for (int mt = 0; mt < 2; ++mt)
+      for (int mt = 0; mt < kAMT; ++mt)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           s[mt][2 * h] = exp2f(s[mt][2 * h] - n0);
@@ -308,7 +311,7 @@ __global__ void __launch_bounds__(kAThreads, 1) attn_decode_kernel(const __grid_
       }
       // O^T += V^T P^T, one 16-position k-step per score tile
 #pragma unroll
-      for (int mt = 0; mt < 2; ++mt) {
+      for (int mt = 0; mt < kAMT; ++mt) {
         const uint32_t b0 = movmatrix_t(pack_bf16x2(s[mt][0], s[mt][1]));
         const uint32_t b1 = movmatrix_t(pack_bf16x2(s[mt][2], s[mt][3]));
         const int row = mt * 16 + mr + 8 * (mi >> 1);

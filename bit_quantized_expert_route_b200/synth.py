@@ -257,3 +257,36 @@ def attention_case_to_host(c: AttnDeviceCase) -> AttnCase:
         return t.detach().cpu().view(torch.int16).numpy().view(np.uint16).copy()
     return AttnCase(bits(c.q), bits(c.k_cache), bits(c.v_cache), c.block_table.cpu().numpy().copy(),
                     c.ctx_len.cpu().numpy().copy())
+
+
+# --------------------------------------------------------------------------
+# Gated DeltaNet decode step: seeded q, k, v (bf16), per-head log-decay and
+# write strength, and an FP32 state (no recurrence arithmetic here).
+# --------------------------------------------------------------------------
+_KEY_DELTA = 0x474E4554   # stream tag for a recurrence case
+
+
+@dataclasses.dataclass
+class DeltaCase:
+    """One recurrence step's inputs in storage form."""
+    q: np.ndarray       # uint16 (bf16) [B, H_k, d_k]
+    k: np.ndarray       # uint16 (bf16) [B, H_k, d_k]
+    v: np.ndarray       # uint16 (bf16) [B, H_v, d_v]
+    g: np.ndarray       # float32 [B, H_v]: log-decay, alpha = exp(g)
+    beta: np.ndarray    # float32 [B, H_v]
+    state: np.ndarray   # float32 [B, H_v, d_v, d_k]
+
+
+def make_deltanet_case(seed: int, B: int, Hk: int = 16, Hv: int = 32, dk: int = 128, dv: int = 128,
+                       step: int = 0) -> DeltaCase:
+    """q, k, v ~ N(0, 1) as bf16; alpha ~ U(0.85, 0.999) (g = ln alpha); beta ~ U(0.05, 0.95);
+    state ~ N(0, 0.05^2) FP32 (a state after many steps of unit-norm keys).  `step` draws a
+    further token's inputs from the same case stream (the state is then ignored)."""
+    rng = _rng(_KEY_DELTA, seed * 1000 + step)
+    q = to_bf16_bits(rng.normal(0.0, 1.0, size=(B, Hk, dk)))
+    k = to_bf16_bits(rng.normal(0.0, 1.0, size=(B, Hk, dk)))
+    v = to_bf16_bits(rng.normal(0.0, 1.0, size=(B, Hv, dv)))
+    g = np.log(rng.uniform(0.85, 0.999, size=(B, Hv))).astype(np.float32)
+    beta = rng.uniform(0.05, 0.95, size=(B, Hv)).astype(np.float32)
+    state = rng.normal(0.0, 0.05, size=(B, Hv, dv, dk)).astype(np.float32)
+    return DeltaCase(q, k, v, g, beta, state)

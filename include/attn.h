@@ -33,7 +33,7 @@
  * bf16.  The weights use a running maximum per head, so no score overflows.
  *
  * Limits (else MOE_ERR_UNSUPPORTED): D = 128 or 256; Hq a multiple of Hkv
- * with Hq / Hkv <= 8; block a multiple of 32; n_blocks * Hkv * block < 2^31.
+ * with Hq / Hkv <= 8; block a multiple of 16; n_blocks * Hkv * block < 2^31.
  * B <= 65535.  Alignment (else MOE_ERR_INVALID_ARG): the caches 16 bytes, q,
  * block_table and ctx_len 4 bytes, out 2 bytes.
  *
@@ -67,7 +67,7 @@ MOE_API size_t attn_decode_workspace_size(int B, int Hkv, int D, int block, int 
 
 /* One decode step of grouped-query attention (see above).  scale <= 0 selects
  * 1/sqrt(D).  Work split: every (sequence, key/value head) pair is cut into
- * up to n_split contiguous ranges of 32-position chunks so that the grid
+ * up to n_split contiguous ranges of 16-position chunks so that the grid
  * covers the SMs; each range's partial (running maximum, sum of weights,
  * weighted sum of values) is merged by a second kernel in fixed range order,
  * so results are deterministic. */
@@ -77,7 +77,7 @@ MOE_API int attn_decode(const moe_bf16* q, const moe_bf16* k_cache, const moe_bf
                         size_t workspace_bytes, moe_stream stream);
 
 /* The work split attn_decode uses for these sizes: n_split ranges per
- * (sequence, key/value head), each of chunks_per_split 32-position chunks. */
+ * (sequence, key/value head), each of chunks_per_split 16-position chunks. */
 MOE_API int attn_decode_plan(int B, int Hkv, int block, int max_blocks, int* n_split, int* chunks_per_split);
 
 #ifdef __cplusplus

@@ -36,7 +36,7 @@ def test_plan_covers_every_chunk(lib):
     for B, Hkv, block, mb in [(1, 2, 64, 64), (1, 2, 64, 512), (1, 2, 64, 2048), (3, 2, 32, 7), (96, 2, 64, 5),
                               (1, 8, 128, 1), (200, 1, 64, 100)]:
         ns, cps = attn.plan(B, Hkv, block, mb)
-        chunks = mb * block // 32
+        chunks = mb * block // 16
         assert ns >= 1 and cps >= 1
         assert (ns - 1) * cps < chunks <= ns * cps          # no empty trailing range, every chunk owned
         if B * Hkv >= 148:
@@ -48,7 +48,7 @@ def test_workspace_size(lib):
     ns, _ = attn.plan(1, 2, 64, 2048)
     assert attn.workspace_size(1, 2, 256, 64, 2048) >= 256 + ns * 2 * 8 * 256 * 4
     assert attn.workspace_size(1, 2, 192, 64, 8) == 0       # unsupported D
-    assert attn.workspace_size(1, 2, 256, 48, 8) == 0       # block not a multiple of 32
+    assert attn.workspace_size(1, 2, 256, 40, 8) == 0       # block not a multiple of 16
 
 
 def _call(lib, B=1, Hq=16, Hkv=2, D=256, block=64, max_blocks=4, n_blocks=4, ws=FAKE, ws_bytes=1 << 30,
@@ -64,7 +64,7 @@ def test_host_rejections(lib):
     assert _call(lib, D=192) == moe.MOE_ERR_UNSUPPORTED
     assert _call(lib, Hq=18, Hkv=2) == moe.MOE_ERR_UNSUPPORTED      # group of 9 heads
     assert _call(lib, Hq=15, Hkv=2) == moe.MOE_ERR_UNSUPPORTED      # not a multiple
-    assert _call(lib, block=48) == moe.MOE_ERR_UNSUPPORTED
+    assert _call(lib, block=40) == moe.MOE_ERR_UNSUPPORTED
     assert _call(lib, B=0) == moe.MOE_ERR_UNSUPPORTED
     assert _call(lib, n_blocks=1 << 20, block=1024, Hkv=8, Hq=8) == moe.MOE_ERR_UNSUPPORTED   # rows >= 2^31
     assert _call(lib, ws=None) == moe.MOE_ERR_WORKSPACE

@@ -141,7 +141,7 @@ def test_bad_block_index_is_reported_and_the_next_call_is_correct():
 
 
 def test_waits_run_out_and_the_next_call_is_correct():
-    """Every CTA streams ~28 chunks through its 6-stage ring, so its waits are for copies just
+    """Every CTA streams ~56 chunks through its 12-stage ring, so its waits are for copies just
     issued; with a one-cycle limit they give up, the copies in flight are drained, the CTA leaves."""
     c = synth.make_attention_case(59, [65536], D=256, block=64)
     q, k, v, table, ctx = _to_dev(c)
