@@ -13,13 +13,16 @@
 //
 // Design.
 //   * Grid (n_split, Hkv, B): CTA (s, g, b) takes a contiguous range of
-//     16-position chunks of sequence b's key/value head g.  One producer
-//     thread streams each chunk's keys and values with TMA tiled copies
-//     (D / 64 boxes of 16 rows x 128 B per cache, 128-byte swizzle) into a
-//     ring of shared-memory stages (12 for D = 256: three per consumer warp,
-//     so a warp computes on one chunk while its next two are in flight);
-//     four consumer warps take the chunks in turn, each keeping its own
-//     running maximum, weight sum and output.
+//     16-position chunks of sequence b's key/value head g.  Each chunk's keys
+//     and values arrive by TMA tiled copies (D / 64 boxes of 16 rows x 128 B
+//     per cache, 128-byte swizzle) in a ring of shared-memory stages (12 for
+//     D = 256).  The four warps take the chunks in turn and each owns the
+//     stages of its chunks (three): it computes on one while the next two
+//     are in flight, and its lane 0 refills a stage as soon as the warp has
+//     read it.  (A single producer thread feeding all stages through
+//     empty/full barriers streamed at under 2.5 TB/s with the arithmetic
+//     removed.)  Each warp keeps its own running maximum, weight sum and
+//     output.
 //   * Per chunk a warp computes S^T = K Q^T on mma.sync m16n8k16 with the 16
 //     positions as M and the group's heads as the 8 columns, so
 //     no tensor-core row is padding; the keys come from shared memory by
@@ -52,7 +55,7 @@ constexpr int kAMT = kAChunk / 16;              // m16 tiles per stage
 constexpr int kABoxCols = 64;                   // elements per swizzled box row (128 B)
 constexpr int kABoxBytes = kAChunk * 128;       // one box: 16 rows x 128 B
 constexpr int kAWarps = 4;                      // consumer warps
-constexpr int kAThreads = (kAWarps + 1) * 32;   // + the producer warp
+constexpr int kAThreads = kAWarps * 32;         // every warp consumes and refills its own stages
 constexpr int kAMaxGroup = 8;                   // query heads per key/value head: the n8 columns
 constexpr int kARingMax = 24;
 constexpr int kACombThreads = 256;              // combine CTA: 32 dims x 8 warps over the ranges
@@ -138,8 +141,7 @@ __global__ void __launch_bounds__(kAThreads, 1) attn_decode_kernel(const __grid_
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + a.ring * STAGE);
-  uint64_t* empty = full + kARingMax;
-  int* bad = reinterpret_cast<int*>(empty + kARingMax);     // [ring] stage skipped: block index out of range
+  int* bad = reinterpret_cast<int*>(full + kARingMax);      // [ring] stage skipped: block index out of range
   float* wml = reinterpret_cast<float*>(bad + kARingMax);   // [warps][8 heads][2]
   int* abort_i = reinterpret_cast<int*>(wml + kAWarps * kAMaxGroup * 2);
   volatile int* abort_flag = abort_i;
@@ -149,14 +151,9 @@ __global__ void __launch_bounds__(kAThreads, 1) attn_decode_kernel(const __grid_
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int group = a.Hq / a.Hkv;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < a.ring; ++i) {
-      tc::mbar_init(&full[i], 1);
-      tc::mbar_init(&empty[i], 1);
-    }
+    for (int i = 0; i < a.ring; ++i) tc::mbar_init(&full[i], 1);
     *abort_i = 0;
     tc::fence_barrier_init();
-  }
-  if (warp == kAWarps && lane == 0) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(&a.tk) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(&a.tv) : "memory");
   }
@@ -172,49 +169,40 @@ __global__ void __launch_bounds__(kAThreads, 1) attn_decode_kernel(const __grid_
   const int c0 = sp * a.cps;
   const int nc = max(min(c0 + a.cps, n_chunks) - c0, 0);
   pdl_launch_dependents();
+  // the range's block-table entries, all loads in flight together
+  const int blk0 = c0 * kAChunk / a.block;
+  const int nblk = nc > 0 ? ((c0 + nc) * kAChunk - 1) / a.block - blk0 + 1 : 0;
+  const int32_t* trow = a.table + static_cast<size_t>(b) * a.max_blocks;
+  for (int j = threadIdx.x; j < min(nblk, kATabCache); j += kAThreads) s_tab[j] = __ldg(trow + blk0 + j);
+  __syncthreads();
 
-  if (warp == kAWarps) {
-    // ------------------------------------------------------- producer
-    // the range's block-table entries, one load per lane, all in flight
-    // together (a load per chunk would put a memory round trip before
-    // every copy)
-    const int blk0 = c0 * kAChunk / a.block;
-    const int nblk = nc > 0 ? ((c0 + nc) * kAChunk - 1) / a.block - blk0 + 1 : 0;
-    const int32_t* trow = a.table + static_cast<size_t>(b) * a.max_blocks;
-    for (int j = lane; j < min(nblk, kATabCache); j += 32) s_tab[j] = __ldg(trow + blk0 + j);
-    __syncwarp();
-    if (lane == 0) {
-      int issued = 0;
-      for (int i = 0; i < nc; ++i) {
-        const int sl = i % a.ring;
-        if (!tc::mbar_wait(&empty[sl], ((i / a.ring) & 1) ^ 1, abort_flag, a.status, a.wait_limit)) break;
-        const int pos = (c0 + i) * kAChunk;
-        const int jb = pos / a.block - blk0;
-        const int phys = jb < kATabCache ? s_tab[jb] : __ldg(trow + blk0 + jb);
-        if (phys < 0 || phys >= a.n_blocks) {
-          bad[sl] = 1;                      // published by the arrival's release
-          atomicExch(a.status, kStatusBadIndex);
-          tc::mbar_arrive(&full[sl]);
-        } else {
-          bad[sl] = 0;
-          const int y = (phys * a.Hkv + g) * a.block + pos % a.block;
-          const uint32_t dst = tc::smem_u32(sm + sl * STAGE);
-          tc::mbar_arrive_expect_tx(&full[sl], STAGE);
+  // Chunk i goes to stage i % ring, and ring is a multiple of the warps, so
+  // every stage belongs to one warp: the warp that consumes a stage also
+  // refills it (lane 0 issues the copies right after the warp's reads), no
+  // other warp touches it, and the warp waits on its phases in order.
+  auto issue = [&](int i) {
+    const int sl = i % a.ring;
+    const int pos = (c0 + i) * kAChunk;
+    const int jb = pos / a.block - blk0;
+    const int phys = jb < kATabCache ? s_tab[jb] : __ldg(trow + blk0 + jb);
+    if (phys < 0 || phys >= a.n_blocks) {
+      bad[sl] = 1;                      // published by the arrival's release
+      atomicExch(a.status, kStatusBadIndex);
+      tc::mbar_arrive(&full[sl]);
+    } else {
+      bad[sl] = 0;
+      const int y = (phys * a.Hkv + g) * a.block + pos % a.block;
+      const uint32_t dst = tc::smem_u32(sm + sl * STAGE);
+      tc::mbar_arrive_expect_tx(&full[sl], STAGE);
 #pragma unroll
-          for (int x = 0; x < NB; ++x) tc::tma_load_2d(dst + x * kABoxBytes, &a.tk, x * kABoxCols, y, &full[sl]);
+      for (int x = 0; x < NB; ++x) tc::tma_load_2d(dst + x * kABoxBytes, &a.tk, x * kABoxCols, y, &full[sl]);
 #pragma unroll
-          for (int x = 0; x < NB; ++x)
-            tc::tma_load_2d(dst + HALF + x * kABoxBytes, &a.tv, x * kABoxCols, y, &full[sl]);
-        }
-        issued = i + 1;
-      }
-      // every copy issued has landed before the CTA may exit
-      tc::drain_ring(full, static_cast<uint32_t>(a.ring), static_cast<uint32_t>(issued), a.status);
+      for (int x = 0; x < NB; ++x) tc::tma_load_2d(dst + HALF + x * kABoxBytes, &a.tv, x * kABoxCols, y, &full[sl]);
     }
-    return;
-  }
+  };
+  if (lane == 0)
+    for (int i = warp; i < min(nc, a.ring); i += kAWarps) issue(i);
 
-  // ------------------------------------------------------ consumer warps
   const int r8 = lane >> 2, t4 = lane & 3;   // fragment row / column pair
   // Q^T as the B operand: lane holds head r8, dims 16 ks + 2 t4 (+1) and +8
   uint32_t qf[KS][2];
@@ -238,9 +226,9 @@ __global__ void __launch_bounds__(kAThreads, 1) attn_decode_kernel(const __grid_
   // ldmatrix lane roles: matrix mi = lane / 8, row mr = lane % 8
   const int mi = lane >> 3, mr = lane & 7;
   bool ok = true;
-  for (int i = warp; i < nc; i += kAWarps) {
+  int i = warp;
+  for (; i < nc; i += kAWarps) {
     const int sl = i % a.ring;
-    // (stage sl is this warp's alone: ring % kAWarps == 0, so its fills arrive in this order)
     ok = __all_sync(0xffffffffu,
                     ok && tc::mbar_wait(&full[sl], (i / a.ring) & 1, abort_flag, a.status, a.wait_limit));
     if (!ok) break;
@@ -326,8 +314,10 @@ __global__ void __launch_bounds__(kAThreads, 1) attn_decode_kernel(const __grid_
     // the stage's generic reads and writes precede its next TMA fill
     tc::fence_proxy_async_smem();
     __syncwarp();
-    if (lane == 0) tc::mbar_arrive(&empty[sl]);
+    if (lane == 0 && i + a.ring < nc) issue(i + a.ring);
   }
+  if (!ok && lane == 0)   // gave up: the copies this warp issued land before the CTA may exit
+    for (int j = i; j < min(nc, i + a.ring); j += kAWarps) tc::mbar_wait_drain(&full[j % a.ring], (j / a.ring) & 1, a.status);
 
   // ---------------------------------------------- merge the four warps
   l0 = sum_over_rows(l0);
@@ -519,7 +509,7 @@ int smem_bytes(int ring) {
   constexpr int stage = 2 * (D / kABoxCols) * kABoxBytes;
   const int red = kAWarps * kAMaxGroup * D * 4;   // the merge reuses the ring
   const int body = (ring * stage > red ? ring * stage : red);
-  return 1024 + body + 2 * kARingMax * 8 + kARingMax * 4 + kAWarps * kAMaxGroup * 2 * 4 + 16 + kATabCache * 4;
+  return 1024 + body + kARingMax * 8 + kARingMax * 4 + kAWarps * kAMaxGroup * 2 * 4 + 16 + kATabCache * 4;
 }
 
 template <int D>

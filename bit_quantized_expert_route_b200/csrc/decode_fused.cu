@@ -749,58 +749,76 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
     const Sched s = make_sched(a, rt.n_act);
 
     // -------------------------------------------------------------- phase C
-    // gate/up, one unit at a time (its compute overlaps the next unit's
-    // arrival): warp w owns the 16-row tile w % 2 (gate or up) for the K
-    // eighth w / 2; per group of 64 inputs four mma.sync, then the group's
-    // scale and bias for the lane's two token columns.
-    float* red = lg;   // [2 tiles][8 K eighths][16 rows][NT] partial sums (logits are no longer needed)
+    // gate/up, two units at a time (their dot products are independent, so
+    // their tensor-core chains overlap, and the pair shares one round of CTA
+    // barriers): warp w owns the 16-row tile w % 2 (gate or up) for the K
+    // eighth w / 2 of both units; per group of 64 inputs four mma.sync, then
+    // the group's scale and bias for the lane's two token columns.
+    float* red = lg;   // [2 units][2 tiles][8 K eighths][16 rows][NT] partial sums (logits are no longer needed)
     {
       const int m = warp & 1, ke = warp >> 1;
       const int ge = ngrp / 8;                       // groups per K eighth
-      for (int i = 0; i < s.my_gu; ++i, ++fill) {
-        const int sl = static_cast<int>(fill % a.ring);
-        const bool got =
-            __all_sync(0xffffffffu, tc::mbar_wait(&full[sl], (fill / a.ring) & 1u, abort_flag, a.status, a.wait_limit));
-        int slot, f0;
-        gu_unit(s, blockIdx.x + i * G, slot, f0);
-        unsigned tmask = 0;                            // tokens of this unit's expert
-        if (slot == 0)
-          tmask = (1u << T) - 1u;
-        else
-          for (int r = 0; r < rt.slot_cnt[slot]; ++r) tmask |= 1u << (rt.perm[rt.slot_off[slot] + r] / k);
-        const uint8_t* ub = fsm + sl * a.slot_bytes;
-        const uint8_t* qrow = ub + (m * kFFeat + lg4) * a.rs_gu + lt * 8;     // rows lg4, lg4 + 8
-        const uint16_t* srow = reinterpret_cast<const uint16_t*>(ub + 2 * kFFeat * a.rs_gu + m * 2 * sb);
-        const uint16_t* brow = srow + sb / 2;
-        const bool tok_live = lg4 < T && ((tmask >> lg4) & 1u);
-        const uint4* xrow = reinterpret_cast<const uint4*>(xs + (tok_live ? lg4 : 0) * g.H) + lt * 2;
-        float y[2][2] = {{0.f, 0.f}, {0.f, 0.f}};     // [row lg4 / lg4 + 8][token 2 lt / 2 lt + 1]
-        tile_groups<4>(y, qrow, a.rs_gu, srow, brow, ngrp, ke * ge, got ? ge : 0, xrow, tok_live, xsum, ngrp, T, lg4,
-                       lt);
-        // every read of the unit's slot is done: release it (a slot that never
-        // filled is not handed back: the producer is stopping as well)
-        tc::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0 && got) tc::mbar_arrive(&empty[sl]);
+      constexpr int kRedUnit = 2 * 8 * 16 * NT;
+      for (int i = 0; i < s.my_gu; i += 2) {
+        const int nu = min(2, s.my_gu - i);
+        int slot[2], f0[2];
+        float y[2][2][2] = {};                         // [unit][row lg4 / lg4 + 8][token 2 lt / 2 lt + 1]
 #pragma unroll
-        for (int c = 0; c < 2; ++c)
-          if (2 * lt + c < T)
+        for (int u = 0; u < 2; ++u) {
+          if (u < nu) {
+            const uint32_t f = fill + u;
+            const int sl = static_cast<int>(f % a.ring);
+            const bool got = __all_sync(
+                0xffffffffu, tc::mbar_wait(&full[sl], (f / a.ring) & 1u, abort_flag, a.status, a.wait_limit));
+            gu_unit(s, blockIdx.x + (i + u) * G, slot[u], f0[u]);
+            unsigned tmask = 0;                        // tokens of this unit's expert
+            if (slot[u] == 0)
+              tmask = (1u << T) - 1u;
+            else
+              for (int r = 0; r < rt.slot_cnt[slot[u]]; ++r) tmask |= 1u << (rt.perm[rt.slot_off[slot[u]] + r] / k);
+            const uint8_t* ub = fsm + sl * a.slot_bytes;
+            const uint8_t* qrow = ub + (m * kFFeat + lg4) * a.rs_gu + lt * 8;     // rows lg4, lg4 + 8
+            const uint16_t* srow = reinterpret_cast<const uint16_t*>(ub + 2 * kFFeat * a.rs_gu + m * 2 * sb);
+            const uint16_t* brow = srow + sb / 2;
+            const bool tok_live = lg4 < T && ((tmask >> lg4) & 1u);
+            const uint4* xrow = reinterpret_cast<const uint4*>(xs + (tok_live ? lg4 : 0) * g.H) + lt * 2;
+            tile_groups<4>(y[u], qrow, a.rs_gu, srow, brow, ngrp, ke * ge, got ? ge : 0, xrow, tok_live, xsum, ngrp,
+                           T, lg4, lt);
+            // every read of the unit's slot is done: release it (a slot that
+            // never filled is not handed back: the producer is stopping as well)
+            tc::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && got) tc::mbar_arrive(&empty[sl]);
+          }
+        }
+        fill += nu;
 #pragma unroll
-            for (int r = 0; r < 2; ++r) red[((m * 8 + ke) * 16 + lg4 + 8 * r) * NT + 2 * lt + c] = y[r][c];
+        for (int u = 0; u < 2; ++u)
+          if (u < nu)
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+              if (2 * lt + c < T)
+#pragma unroll
+                for (int r = 0; r < 2; ++r)
+                  red[u * kRedUnit + ((m * 8 + ke) * 16 + lg4 + 8 * r) * NT + 2 * lt + c] = y[u][r][c];
         consumers_sync();
-        // h = bf16(silu(g) * u) for (feature pair, token); K eighths summed in
-        // order; each pair goes out as one exchange word of h row `pos`
-        // (routed rows in expert order, then the shared expert's rows)
-        if (tid < (kFFeat / 2) * T && !rt.abort) {
-          const int fp = tid / T, t = tid % T;
-          bool member = slot == 0;
+        // h = bf16(silu(g) * u) for (unit, feature pair, token); K eighths
+        // summed in order; each pair goes out as one exchange word of h row
+        // `pos` (routed rows in expert order, then the shared expert's rows)
+        if (tid < nu * (kFFeat / 2) * T && !rt.abort) {
+          const int u = tid / ((kFFeat / 2) * T), rem = tid % ((kFFeat / 2) * T);
+          const int fp = rem / T, t = rem % T;
+          const int sl_u = u == 0 ? slot[0] : slot[1];
+          const int f0_u = u == 0 ? f0[0] : f0[1];
+          bool member = sl_u == 0;
           int pos = Tk + t;
-          for (int r = 0; r < (slot == 0 ? 0 : rt.slot_cnt[slot]); ++r)
-            if (rt.perm[rt.slot_off[slot] + r] / k == t) {
+          for (int r = 0; r < (sl_u == 0 ? 0 : rt.slot_cnt[sl_u]); ++r)
+            if (rt.perm[rt.slot_off[sl_u] + r] / k == t) {
               member = true;
-              pos = rt.slot_off[slot] + r;
+              pos = rt.slot_off[sl_u] + r;
             }
           if (member) {
+            const float* ru = red + u * kRedUnit;
             uint32_t hv[2];
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
@@ -808,15 +826,15 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
               float gs = 0.f, us = 0.f;
 #pragma unroll
               for (int e8 = 0; e8 < 8; ++e8) {
-                gs += red[((0 * 8 + e8) * 16 + f) * NT + t];
-                us += red[((1 * 8 + e8) * 16 + f) * NT + t];
+                gs += ru[((0 * 8 + e8) * 16 + f) * NT + t];
+                us += ru[((1 * 8 + e8) * 16 + f) * NT + t];
               }
               hv[q] = float_to_bf16_bits(silu(gs) * us);
             }
-            st_word(a.hx + static_cast<size_t>(pos) * (Kmax / 2) + (f0 / 2 + fp), tag, hv[0] | (hv[1] << 16));
+            st_word(a.hx + static_cast<size_t>(pos) * (Kmax / 2) + (f0_u / 2 + fp), tag, hv[0] | (hv[1] << 16));
           }
         }
-        consumers_sync();   // red is reused by the next unit
+        consumers_sync();   // red is reused by the next pair
       }
     }
     consumers_sync();
@@ -860,54 +878,74 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
       }
       consumers_sync();
     }
-    // down units: warp w owns expert slot w % 8 of the unit (16 dims x K) for
-    // the K half w / 8; lanes hold rows (dims) lg4, lg4 + 8 and token columns
-    // 2 lt, 2 lt + 1
+    // down units, two at a time as the gate/up units: warp w owns expert slot
+    // w % 8 of each unit (16 dims x K) for the K half w / 8; lanes hold rows
+    // (dims) lg4, lg4 + 8 and token columns 2 lt, 2 lt + 1
     {
       const int jj = warp & 7, kh = warp >> 3;
       const int kg = Kmax / kGroup;
-      float* redd = lg;   // [8 slots][2 K halves][16 dims][NT]
-      for (int di = 0; di < s.my_blocks * s.n_down_parts; ++di, ++fill) {
-        const int sl = static_cast<int>(fill % a.ring);
-        const bool got =
-            __all_sync(0xffffffffu, tc::mbar_wait(&full[sl], (fill / a.ring) & 1u, abort_flag, a.status, a.wait_limit));
-        const int bl = di / s.n_down_parts;
-        const int j0 = (di % s.n_down_parts) * s.spd, nj = min(s.spd, s.n_slots - j0);
-        const bool jlive = got && jj < nj;
-        const int j = j0 + jj;
-        const int K = j == 0 ? g.Is : g.I;
-        const int ng = K / kGroup, gh = ng / 2;       // groups, groups per K half
-        const int nt = jlive ? rt.slot_cnt[j] : 0;
-        const int pos0 = jlive ? rt.slot_off[j] : 0;
-        float y[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-        if (jlive) {
-          const uint8_t* ub = fsm + sl * a.slot_bytes + jj * a.dslot;
-          const uint8_t* qrow = ub + lg4 * a.rs_dn + lt * 8;
-          const uint16_t* srow = reinterpret_cast<const uint16_t*>(ub + kFDims * a.rs_dn);
-          const uint16_t* brow = reinterpret_cast<const uint16_t*>(ub + kFDims * a.rs_dn + Kmax / 2);
-          const bool tok_live = lg4 < nt;
-          const int hr = pos0 + (tok_live ? lg4 : 0);
-          const uint4* hrow = reinterpret_cast<const uint4*>(hs + static_cast<size_t>(hr) * Kmax) + lt * 2;
-          for (int gb = 0; gb < gh; gb += 4)
-            tile_groups<4>(y, qrow, a.rs_dn, srow, brow, ng, kh * gh + gb, min(4, gh - gb), hrow, tok_live,
-                           hsum + pos0 * kg, kg, nt, lg4, lt);
+      float* redd = lg;   // [2 units][8 slots][2 K halves][16 dims][NT]
+      constexpr int kRedUnit = 8 * 2 * 16 * NT;
+      const int n_du = s.my_blocks * s.n_down_parts;
+      for (int di = 0; di < n_du; di += 2) {
+        const int nu = min(2, n_du - di);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          if (u < nu) {
+            const uint32_t f = fill + u;
+            const int sl = static_cast<int>(f % a.ring);
+            const bool got = __all_sync(
+                0xffffffffu, tc::mbar_wait(&full[sl], (f / a.ring) & 1u, abort_flag, a.status, a.wait_limit));
+            const int dd = di + u;
+            const int j0 = (dd % s.n_down_parts) * s.spd, nj = min(s.spd, s.n_slots - j0);
+            const bool jlive = got && jj < nj;
+            const int j = j0 + jj;
+            const int K = j == 0 ? g.Is : g.I;
+            const int ng = K / kGroup, gh = ng / 2;       // groups, groups per K half
+            const int nt = jlive ? rt.slot_cnt[j] : 0;
+            const int pos0 = jlive ? rt.slot_off[j] : 0;
+            float y[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+            if (jlive) {
+              const uint8_t* ub = fsm + sl * a.slot_bytes + jj * a.dslot;
+              const uint8_t* qrow = ub + lg4 * a.rs_dn + lt * 8;
+              const uint16_t* srow = reinterpret_cast<const uint16_t*>(ub + kFDims * a.rs_dn);
+              const uint16_t* brow = reinterpret_cast<const uint16_t*>(ub + kFDims * a.rs_dn + Kmax / 2);
+              const bool tok_live = lg4 < nt;
+              const int hr = pos0 + (tok_live ? lg4 : 0);
+              const uint4* hrow = reinterpret_cast<const uint4*>(hs + static_cast<size_t>(hr) * Kmax) + lt * 2;
+              for (int gb = 0; gb < gh; gb += 4)
+                tile_groups<4>(y, qrow, a.rs_dn, srow, brow, ng, kh * gh + gb, min(4, gh - gb), hrow, tok_live,
+                               hsum + pos0 * kg, kg, nt, lg4, lt);
+            }
+            tc::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && got) tc::mbar_arrive(&empty[sl]);
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+              if (2 * lt + c < nt)
+#pragma unroll
+                for (int r = 0; r < 2; ++r)
+                  redd[u * kRedUnit + ((jj * 2 + kh) * 16 + lg4 + 8 * r) * NT + 2 * lt + c] = y[r][c];
+          }
         }
-        tc::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0 && got) tc::mbar_arrive(&empty[sl]);
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-          if (2 * lt + c < nt)
-#pragma unroll
-            for (int r = 0; r < 2; ++r) redd[((jj * 2 + kh) * 16 + lg4 + 8 * r) * NT + 2 * lt + c] = y[r][c];
+        fill += nu;
         consumers_sync();
-        // y rows of this unit's slots: both K halves summed in order
-        for (int q = tid; q < nj * kFDims * NT; q += nthr) {
-          const int js = q / (kFDims * NT), d = (q / NT) % kFDims, t = q % NT;
-          const int jx = j0 + js;
-          if (t < rt.slot_cnt[jx])
-            ys[((rt.slot_off[jx] + t) * s.my_blocks + bl) * kFDims + d] =
-                redd[((js * 2 + 0) * 16 + d) * NT + t] + redd[((js * 2 + 1) * 16 + d) * NT + t];
+        // y rows of these units' slots: both K halves summed in order
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          if (u < nu) {
+            const int dd = di + u;
+            const int bl = dd / s.n_down_parts;
+            const int j0 = (dd % s.n_down_parts) * s.spd, nj = min(s.spd, s.n_slots - j0);
+            const float* ru = redd + u * kRedUnit;
+            for (int q = tid; q < nj * kFDims * NT; q += nthr) {
+              const int js = q / (kFDims * NT), d = (q / NT) % kFDims, t = q % NT;
+              const int jx = j0 + js;
+              if (t < rt.slot_cnt[jx])
+                ys[((rt.slot_off[jx] + t) * s.my_blocks + bl) * kFDims + d] =
+                    ru[((js * 2 + 0) * 16 + d) * NT + t] + ru[((js * 2 + 1) * 16 + d) * NT + t];
+            }
+          }
         }
         consumers_sync();
       }
@@ -1012,7 +1050,7 @@ FusedLayout fused_layout(const Geometry& g, int G) {
   const int blocks_per_cta = (g.H / kFDims + G - 1) / G;
   auto al = [](int v) { return (v + 127) / 128 * 128; };
   const int lg_floats = max(max(g.T * (g.E + 1), f.rows_per_cta * kFWarps * kFMaxT),
-                            max(16 * 16 * kFMaxT, g.T * blocks_per_cta * kFDims));
+                            max(2 * 16 * 16 * kFMaxT, g.T * blocks_per_cta * kFDims));   // pairs of units
   const int stage_bytes = max(g.T * g.H * 2, rows * Kmax * 2);
   const int sums_bytes = max(g.T * (g.H / kGroup) * 4, rows * (Kmax / kGroup) * 4);
   const int fixed = al((2 * kFRingMax + 3) * 8) + al(f.rows_per_cta * g.H * 2) + al(stage_bytes) + al(sums_bytes) +

@@ -41,10 +41,15 @@
  * Ownership.  The caller owns every buffer (weights, x, out, routing,
  * workspace).  The library allocates no device memory and keeps no state
  * between calls except cached kernel attributes.  Two calls must not share a
- * workspace concurrently.  The first 256 bytes of a workspace are a control
- * block (status word, a CTA counter) that must be zero before the workspace
- * is first used (e.g. cudaMemset); the library leaves them zero after every
- * call except for a recorded error status, which moe_get_status clears.
+ * workspace concurrently.  A workspace must be zero-filled once before its
+ * first use (e.g. cudaMemset of the whole buffer).  Its first 256 bytes are a
+ * control block (status word, a CTA counter, the fused decode kernel's exit
+ * counter and launch epoch); the library leaves the status word zero after
+ * every call except for a recorded error status, which moe_get_status
+ * clears.  The fused decode kernel's CTAs exchange values through 64-bit
+ * words of the workspace tagged with (launch epoch, layer): a stale word is
+ * never taken for a current one, except one last written exactly a multiple
+ * of 2^26 launches earlier on the same workspace and not rewritten since.
  *
  * Asynchrony.  moe_route, moe_forward, moe_decode and moe_rmsnorm enqueue
  * work on `stream` (a cudaStream_t; NULL = the legacy default stream) and
@@ -175,20 +180,23 @@ MOE_API int moe_route(const moe_layer_desc* layer, const moe_bf16* x, int T, moe
  * bf16 products and FP32 accumulation, and one always-on shared expert.
  * x, out: device bf16 [T, H], 16-byte aligned, not overlapping.
  * r: optional (NULL = keep routing in the workspace).
- * 1 <= T <= 65536.  For T <= 2 with H = 1024 or 2048 and 16-byte aligned
- * scale and bias stacks it runs moe_decode's single-launch fused kernel; for
- * every other T, the tensor-core kernels above (the GEMV kernels of
- * moe_decode spend FP32 work on every weight for every token, which the
- * tensor cores outrun as soon as an expert sees a few tokens). */
+ * 1 <= T <= 65536.  For T <= 8 with H = 1024 or 2048, I and I_shared whole
+ * groups, 16-byte aligned scale and bias stacks and at most E + 1 SMs it
+ * runs moe_decode's single-launch fused kernel; for every other T, the
+ * tensor-core kernels above (the three-launch decode kernels spend work on
+ * every weight for every token, which the grouped GEMMs outrun as soon as an
+ * expert sees a few tokens). */
 MOE_API int moe_forward(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_bf16* out,
                 moe_routing* r, void* workspace, size_t workspace_bytes, moe_stream stream);
 
 /* The same function for 1 <= T <= 64 through the bandwidth-bound decode
  * kernels (batch-1 decoding streams the active experts' weights: "How It
  * Works: Prefill and Decode Strategies").  T > 64 is MOE_ERR_INVALID_ARG.
- * For T <= 2 with H = 1024 or 2048 and 16-byte aligned scale and bias stacks
- * the whole layer is ONE cooperative launch of one CTA per SM (grid-wide
- * barriers in the workspace control block); otherwise three launches. */
+ * Under the same conditions as moe_forward's fused path (T <= 8, ...) the
+ * whole layer is ONE cooperative launch of one CTA per SM whose CTAs exchange
+ * the router logits, the SwiGLU activations and the outputs through tagged
+ * workspace words (no grid-wide barrier); otherwise three launches (routing,
+ * gate/up, down + combine). */
 MOE_API int moe_decode(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_bf16* out,
                moe_routing* r, void* workspace, size_t workspace_bytes, moe_stream stream);
 
@@ -199,10 +207,13 @@ MOE_API int moe_decode(const moe_layer_desc* layer, const moe_bf16* x, int T, mo
  * can also be captured once as a CUDA graph and replayed:
  *   a_0 = x;  y_l = layer_l(a_l);  a_{l+1} = bf16(y_l / sqrt(mean(y_l^2) + eps))
  * (RMSNorm with weight 1 and no residual, over the bf16 values of y_l);
- * out = y_{n_layers-1}.  Each layer runs what moe_forward runs for T; on the
+ * out = y_{n_layers-1}.  Each layer runs what moe_forward runs for T.  On the
  * tensor-core path the RMSNorm is computed inside the layer's combine kernel
- * (the row's sum of squares is formed while its output is written), after
- * the fused decode kernel it is a separate small kernel.
+ * (the row's sum of squares is formed while its output is written).  On the
+ * fused decode path up to 40 layers run in ONE launch, the RMSNorm between
+ * them inside it (each CTA publishes the sum of squares of its outputs);
+ * longer stacks are cut into launches of 40 layers joined by a small
+ * RMSNorm kernel.
  *   layers: host array of n_layers (1..1024) descriptors with equal H, I,
  *           I_shared, E and k.
  *   x, out: device bf16 [T, H], 16-byte aligned, not overlapping.
