@@ -61,6 +61,7 @@ DECODE_KERNEL_SRC = "bit_quantized_expert_route_b200/csrc/decode.cu"
 DECODE_KERNEL = "decode_gateup_kernel"
 FUSED_DECODE_KERNEL_SRC = "bit_quantized_expert_route_b200/csrc/decode_fused.cu"
 FUSED_DECODE_KERNEL = "decode_fused_kernel<1>"
+ATTN_SRC = "bit_quantized_expert_route_b200/csrc/attn.cu"
 EPS = 1e-6
 
 
@@ -581,12 +582,13 @@ def attention_phase(a, world, rank, dev, peaks, peak_src):
         del graph
         assert moe.moe_get_status(ws) == 0
         n_split, cps = attn.plan(1, 2, 64, mb)
+        trd = committed_traffic("attn_decode_kernel<256>", ATTN_SRC, f"attn_L{L}")   # main kernel, per launch
         overhead = (n_split * 2 * 8 * (256 + 2) * 4 * 2) if n_split > 1 else 0   # partials written + read
         pts[str(L)] = {"us": round(ms * 1e3, 3), "steps_per_s": round(whole_job_rate(1, world, ms), 1),
                        "kv_bytes": kv, "split_partial_bytes": overhead, "n_split": n_split, "chunks_per_split": cps,
                        "launches_per_step": 2 if n_split > 1 else 1, "distinct_caches_cycled": n_cases,
                        "roofline": hbm_roofline("attn_decode_kernel<256> + attn_combine_kernel<256>", kv, ms, peaks,
-                                                peak_src)}
+                                                peak_src, traffic=trd[0] if trd else None)}
         del cases, outs, ws
         torch.cuda.empty_cache()
     return {"workload": "decode attention, 1 sequence, 16 Q heads / 2 KV heads (GQA groups of 8), D=256, "

@@ -245,20 +245,21 @@ __global__ void __launch_bounds__(kAThreads, 1) attn_decode_kernel(const __grid_
       }
       const uint32_t kb = sbase + sl * STAGE, vb = kb + HALF;
       // S^T = K Q^T for the two 16-row tiles
-      float s[kAMT][4], s2[kAMT][4];   // even and odd k-steps accumulate apart (two dependency chains)
+      float s[kAMT][4];
 #pragma unroll
       for (int mt = 0; mt < kAMT; ++mt) {
-        s[mt][0] = s[mt][1] = s[mt][2] = s[mt][3] = 0.f;
-        s2[mt][0] = s2[mt][1] = s2[mt][2] = s2[mt][3] = 0.f;
+        float c4[4][4];   // k-steps mod 4 accumulate apart: four short dependency chains instead of one
+#pragma unroll
+        for (int c = 0; c < 4; ++c) c4[c][0] = c4[c][1] = c4[c][2] = c4[c][3] = 0.f;
         const int row = mt * 16 + mr + 8 * (mi & 1);
 #pragma unroll
         for (int ks = 0; ks < KS; ++ks) {
           uint32_t a0, a1, a2, a3;
           ldsm_x4(kb + tile_off(row, 2 * ks + (mi >> 1)), a0, a1, a2, a3);
-          mma16816((ks & 1) ? s2[mt] : s[mt], a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
+          mma16816(c4[ks & 3], a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
         }
 #pragma unroll
-        for (int e = 0; e < 4; ++e) s[mt][e] += s2[mt][e];
+        for (int e = 0; e < 4; ++e) s[mt][e] = (c4[0][e] + c4[1][e]) + (c4[2][e] + c4[3][e]);
       }
       // scale, mask, running maximum per head column
       float mx0 = -INFINITY, mx1 = -INFINITY;

@@ -16,7 +16,7 @@
 // Each layer has three all-to-all exchanges between the CTAs (all CTAs are
 // co-resident: cooperative launch).  None is a grid barrier: the values
 // travel in tagged 64-bit words that a reader polls until they are current
-// (see wait_word), so a CTA goes on the moment the data it needs is there.
+// (see wait_words), so a CTA goes on the moment the data it needs is there.
 //
 //   A  input: layer 0 reads x; layer l > 0 reads the previous layer's output
 //      y (bf16) and the CTAs' partial sums of its squares and applies
@@ -53,6 +53,8 @@
 // operands use the order (0,4,1,5,2,6,3,7) in which the AND-OR yields code
 // pairs; the activations are staged in that order, so no permutes are
 // needed.
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
@@ -204,6 +206,7 @@ __device__ __forceinline__ void tile_groups(float (&y)[2][2], const uint8_t* qro
   }
 }
 
+
 // Order-preserving 32-bit key of a float (larger float -> larger key; every
 // non-NaN float maps above 0).
 __device__ __forceinline__ uint32_t order_key(float f) {
@@ -294,13 +297,25 @@ __device__ __forceinline__ void st_word(unsigned long long* p, uint32_t tag, uin
   asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
-// The payload of *p once it carries `tag`.  Bounded: gives up (ok = false,
+// The payloads of up to N words once each carries `tag`: all N loads are in
+// flight together, and only the words still stale are loaded again, so a
+// thread pays one round trip through L2 for the batch rather than one per
+// word (one at a time, staging h took 12 us at T = 8).  A NULL pointer is a
+// slot with nothing to wait for (payload 0).  Bounded: gives up (ok = false,
 // status recorded, the CTA's abort flag raised) after the deadline or as
 // soon as another thread of the CTA has given up.
-__device__ __forceinline__ uint32_t wait_word(const unsigned long long* p, uint32_t tag, long long deadline,
-                                              volatile int* abort, int* status, bool& ok) {
-  unsigned long long v = ld_word(p);
-  for (uint32_t n = 0; ok && static_cast<uint32_t>(v >> 32) != tag; ++n) {
+template <int N>
+__device__ __forceinline__ void wait_words(const unsigned long long* const (&p)[N], uint32_t tag,
+                                           uint32_t (&out)[N], long long deadline, volatile int* abort,
+                                           int* status, bool& ok) {
+  unsigned long long v[N];
+#pragma unroll
+  for (int i = 0; i < N; ++i) v[i] = p[i] ? ld_word(p[i]) : (static_cast<unsigned long long>(tag) << 32);
+  for (uint32_t n = 0; ok; ++n) {
+    bool all = true;
+#pragma unroll
+    for (int i = 0; i < N; ++i) all = all && static_cast<uint32_t>(v[i] >> 32) == tag;
+    if (all) break;
     if ((n & 15u) == 15u && (*abort || clock64() > deadline)) {
       ok = false;
       if (!*abort) {
@@ -309,9 +324,12 @@ __device__ __forceinline__ uint32_t wait_word(const unsigned long long* p, uint3
       }
       break;
     }
-    v = ld_word(p);
+#pragma unroll
+    for (int i = 0; i < N; ++i)
+      if (static_cast<uint32_t>(v[i] >> 32) != tag) v[i] = ld_word(p[i]);
   }
-  return static_cast<uint32_t>(v);
+#pragma unroll
+  for (int i = 0; i < N; ++i) out[i] = static_cast<uint32_t>(v[i]);
 }
 
 // Called once per CTA at its end: the last CTA to leave advances the epoch
@@ -584,29 +602,32 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
     } else {
       const long long deadline = clock64() + a.wait_limit;
       const unsigned long long* yrow = a.yx + tid * 2;
+      const unsigned long long* yp[2 * NT];
+      uint32_t yv[2 * NT];
 #pragma unroll
       for (int t = 0; t < NT; ++t) {
-        xv[t] = make_uint2(0u, 0u);
-        if (live && t < T) {
-          xv[t].x = wait_word(yrow + t * (g.H / 2), tag - 1u, deadline, abort_flag, a.status, ok);
-          xv[t].y = wait_word(yrow + t * (g.H / 2) + 1, tag - 1u, deadline, abort_flag, a.status, ok);
-        }
+        const bool need = live && t < T;
+        yp[2 * t] = need ? yrow + t * (g.H / 2) : nullptr;
+        yp[2 * t + 1] = need ? yrow + t * (g.H / 2) + 1 : nullptr;
       }
+      wait_words<2 * NT>(yp, tag - 1u, yv, deadline, abort_flag, a.status, ok);
+#pragma unroll
+      for (int t = 0; t < NT; ++t) xv[t] = make_uint2(yv[2 * t], yv[2 * t + 1]);
       // warp t sums the CTAs' partial sums of squares of token t: lane i
       // takes CTAs i, i+32, ..., then a fixed shuffle tree; the same order in
       // every CTA
       if (warp < T) {
-        float part[kFMaxGrid / 32];
+        const unsigned long long* sp_[kFMaxGrid / 32];
+        uint32_t part[kFMaxGrid / 32];
 #pragma unroll
         for (int j = 0; j < kFMaxGrid / 32; ++j) {
           const int c = lane + 32 * j;
-          part[j] = c < G ? __uint_as_float(wait_word(a.ssx + c * kFMaxT + warp, tag - 1u, deadline, abort_flag,
-                                                      a.status, ok))
-                          : 0.f;
+          sp_[j] = c < G ? a.ssx + c * kFMaxT + warp : nullptr;
         }
+        wait_words<kFMaxGrid / 32>(sp_, tag - 1u, part, deadline, abort_flag, a.status, ok);
         float ss = 0.f;
 #pragma unroll
-        for (int j = 0; j < kFMaxGrid / 32; ++j) ss += part[j];
+        for (int j = 0; j < kFMaxGrid / 32; ++j) ss += __uint_as_float(part[j]);
         ss = warp_sum(ss);
         if (lane == 0) nrm[warp] = 1.0f / sqrtf(ss / static_cast<float>(g.H) + a.eps);
       }
@@ -694,8 +715,16 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
     // further exchange is needed before the expert weights can be requested.
     {
       const long long deadline = clock64() + a.wait_limit;
-      for (int i = tid; i < T * E1; i += nthr)
-        lg[i] = __uint_as_float(wait_word(a.lgx + i, tag, deadline, abort_flag, a.status, ok));
+      for (int i0 = tid; i0 < T * E1; i0 += 8 * nthr) {
+        const unsigned long long* lp[8];
+        uint32_t lv[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) lp[j] = i0 + j * nthr < T * E1 ? a.lgx + i0 + j * nthr : nullptr;
+        wait_words<8>(lp, tag, lv, deadline, abort_flag, a.status, ok);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (i0 + j * nthr < T * E1) lg[i0 + j * nthr] = __uint_as_float(lv[j]);
+      }
     }
     consumers_sync();
     if (rt.abort) break;
@@ -847,17 +876,28 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
       // sums over groups of 64
       const long long deadline = clock64() + a.wait_limit;
       const int vmax = Kmax / 8;
-      for (int i = tid; i < (Tk + T) * vmax; i += nthr) {
-        const int r = i / vmax, u = i - r * vmax;
-        const bool shr = r >= Tk;
-        if (u * 8 >= (shr ? g.Is : g.I)) continue;
-        const unsigned long long* w4 = a.hx + static_cast<size_t>(r) * (Kmax / 2) + u * 4;
-        uint4 v;
-        v.x = wait_word(w4, tag, deadline, abort_flag, a.status, ok);
-        v.y = wait_word(w4 + 1, tag, deadline, abort_flag, a.status, ok);
-        v.z = wait_word(w4 + 2, tag, deadline, abort_flag, a.status, ok);
-        v.w = wait_word(w4 + 3, tag, deadline, abort_flag, a.status, ok);
-        reinterpret_cast<uint4*>(hs + static_cast<size_t>(r) * Kmax)[u] = interleave8(v);
+      const int ng4 = (Tk + T) * vmax;
+      for (int i0 = tid; i0 < ng4; i0 += 4 * nthr) {   // four 8-value groups (16 words) per batch
+        const unsigned long long* hp[16];
+        uint32_t hv16[16];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int i = i0 + q * nthr;
+          const int r = i / vmax, u = i - r * vmax;
+          const bool need = i < ng4 && u * 8 < (r >= Tk ? g.Is : g.I);
+          const unsigned long long* w4 = a.hx + static_cast<size_t>(r) * (Kmax / 2) + u * 4;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) hp[4 * q + e] = need ? w4 + e : nullptr;
+        }
+        wait_words<16>(hp, tag, hv16, deadline, abort_flag, a.status, ok);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int i = i0 + q * nthr;
+          const int r = i / vmax, u = i - r * vmax;
+          if (i < ng4 && u * 8 < (r >= Tk ? g.Is : g.I))
+            reinterpret_cast<uint4*>(hs + static_cast<size_t>(r) * Kmax)[u] =
+                interleave8(make_uint4(hv16[4 * q], hv16[4 * q + 1], hv16[4 * q + 2], hv16[4 * q + 3]));
+        }
       }
       consumers_sync();
       const int kg = Kmax / kGroup;
@@ -1020,6 +1060,13 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
   if (tid == 0) launch_exit(a.bar, gridDim.x);
 }
 
+const void* fused_kernel_fn(int T) {
+  return T == 1   ? reinterpret_cast<const void*>(decode_fused_kernel<1>)
+         : T == 2 ? reinterpret_cast<const void*>(decode_fused_kernel<2>)
+         : T <= 4 ? reinterpret_cast<const void*>(decode_fused_kernel<4>)
+                  : reinterpret_cast<const void*>(decode_fused_kernel<8>);
+}
+
 int fused_grid() {
   static int n = 0;
   if (n == 0) {
@@ -1092,7 +1139,27 @@ bool decode_fused_supported(const Geometry& g) {
   if (G > g.E + 1) return false;
   if ((g.E + 1 + G - 1) / G > kFMaxRouterRows) return false;
   const FusedLayout f = fused_layout(g, G);
-  return f.spd >= 1 && f.ring >= 2 && f.total <= 227 * 1024;   // spd: at least one expert slot per down unit
+  if (f.spd < 1 || f.ring < 2 || f.total > 227 * 1024) return false;   // spd: at least one expert slot per down unit
+  // the cooperative launch needs one resident CTA per SM (registers, shared
+  // memory); checked once per kernel instance and shared-memory size
+  struct Fit {
+    int total = -1;
+    bool ok = false;
+  };
+  static Fit fit[4];
+  static std::mutex mu;
+  const int slot = g.T == 1 ? 0 : g.T == 2 ? 1 : g.T <= 4 ? 2 : 3;
+  std::lock_guard<std::mutex> lock(mu);
+  if (fit[slot].total != f.total) {
+    const void* fn = fused_kernel_fn(g.T);
+    int per_sm = 0;
+    fit[slot].ok = ensure_smem(fn, f.total) == cudaSuccess &&
+                   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kFThreads, f.total) == cudaSuccess &&
+                   per_sm >= 1;
+    (void)cudaGetLastError();   // a failed query leaves no sticky error for the caller's next check
+    fit[slot].total = f.total;
+  }
+  return fit[slot].ok;
 }
 
 int decode_fused_max_layers() { return kFMaxLayers; }
@@ -1137,10 +1204,7 @@ cudaError_t launch_decode_fused(const Geometry& g, const LayerPtr* layers, int n
   a.off_rt = f.off_rt;
   a.off_y = f.off_y;
   a.off_nrm = f.off_nrm;
-  const void* fn = g.T == 1   ? reinterpret_cast<const void*>(decode_fused_kernel<1>)
-                   : g.T == 2 ? reinterpret_cast<const void*>(decode_fused_kernel<2>)
-                   : g.T <= 4 ? reinterpret_cast<const void*>(decode_fused_kernel<4>)
-                              : reinterpret_cast<const void*>(decode_fused_kernel<8>);
+  const void* fn = fused_kernel_fn(g.T);
   cudaError_t e = ensure_smem(fn, f.total);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
