@@ -73,7 +73,6 @@ constexpr int kFRouterRows = 2;                 // router rows per CTA with load
 constexpr int kFMaxRouterRows = 4;              // router rows per CTA held in shared memory
 constexpr int kFMaxLayers = 40;                 // layers per launch (kernel-parameter space)
 constexpr int kFMaxGrid = 160;                  // CTAs (SMs) the RMSNorm partial sums are read for in one pass
-constexpr int kFRowPad = 32;                    // bytes after each staged row of codes (bank spread)
 
 struct FusedArgs {
   Geometry g;
@@ -380,14 +379,16 @@ __device__ __forceinline__ void gu_unit(const Sched& s, int u, int& slot, int& f
   f0 = (sh ? u : (u - s.n_sh_units) % s.units_per_exp) * kFFeat;
 }
 
-// Staged tiles.  Every row of 4-bit codes is copied to its own shared-memory
-// row of stride (row bytes + 32): the 8 rows that one mma fragment reads then
-// start in 8 different bank groups, so a warp's code load is conflict-free.
-// The producer warp's 32 lanes issue the row copies together (lane 0 first
-// raised the slot's transaction count; the caller's __syncwarp orders it).
+// Staged tiles: a few large contiguous copies per tile, issued by the
+// producer warp's lanes together (lane 0 first raised the slot's transaction
+// count; the caller's __syncwarp orders it).  One copy per code row into a
+// padded row (so that the 8 rows one mma fragment reads start in different
+// bank groups) made ~36 copies per gate/up unit and ~90 per down unit; the
+// copies then reached the memory system so late that the tiles' arrival, not
+// the bank conflicts, bound the layer.
 //
 // gate/up unit (expert e, features f0..f0+15):
-//   [16 gate rows][16 up rows] (stride rs_gu = H/2 + 32), then
+//   [16 gate rows][16 up rows] (H/2 bytes each), then
 //   [s gate][b gate][s up][b up] (16 x H/64 bf16 each).
 __device__ __forceinline__ uint32_t gateup_bytes(const Geometry& g) {
   return 2 * kFFeat * (g.H / 2) + 4 * (kFFeat * g.H / 32);
@@ -397,20 +398,24 @@ __device__ void issue_gateup(const FusedArgs& a, const LayerPtr& L, int e, int f
   const Geometry& g = a.g;
   const bool sh = e >= g.E;
   const size_t row0 = static_cast<size_t>(sh ? 0 : e * g.I) + f0;
-  const QMatPtr& W = lane < 16 ? (sh ? L.sh_gate : L.gate) : (sh ? L.sh_up : L.up);
-  const int r = lane & 15;
-  tc::bulk_load(dst + (lane >> 4) * kFFeat * a.rs_gu + r * a.rs_gu, W.q + (row0 + r) * (g.H / 8), g.H / 2, full);
-  if (lane < 4) {
-    const QMatPtr& V = lane < 2 ? (sh ? L.sh_gate : L.gate) : (sh ? L.sh_up : L.up);
-    const uint32_t sb = kFFeat * g.H / 32;
-    tc::bulk_load(dst + 2 * kFFeat * a.rs_gu + lane * sb, ((lane & 1) ? V.b : V.s) + row0 * (g.H / kGroup), sb,
-                  full);
+  const uint32_t qb = kFFeat * g.H / 2, sb = kFFeat * g.H / 32;
+  if (lane < 2) {
+    const QMatPtr& W = lane == 0 ? (sh ? L.sh_gate : L.gate) : (sh ? L.sh_up : L.up);
+    tc::bulk_load(dst + lane * qb, W.q + row0 * (g.H / 8), qb, full);
+  } else if (lane < 6) {
+    const int j = lane - 2;
+    const QMatPtr& V = j < 2 ? (sh ? L.sh_gate : L.gate) : (sh ? L.sh_up : L.up);
+    tc::bulk_load(dst + 2 * qb + j * sb, ((j & 1) ? V.b : V.s) + row0 * (g.H / kGroup), sb, full);
   }
 }
 
 // down unit (16 output dims of dim block blk, expert slots j0..j0+nj-1): per
-// slot jj at jj * dslot: [16 code rows, stride rs_dn = Kmax/2 + 32][s: 16 x
-// K/64][b at + Kmax/2].  Returns the bytes to expect.
+// slot jj at jj * dslot (dslot = 9 Kmax): [16 code rows of K/2 bytes,
+// contiguous][s: 16 x K/64 at + 8 Kmax][b at + 8 Kmax + Kmax / 2], three
+// copies per slot, lane jj issuing slot jj's.  (One copy per 256-byte row
+// spread the rows over the banks but made ~90 copies per unit, and the
+// producer then finished issuing a layer's tiles ~12 us after its routing
+// was known.)  Returns the bytes to expect.
 __device__ __forceinline__ uint32_t down_bytes(const Geometry& g, int j0, int nj) {
   uint32_t bytes = 0;
   for (int jj = 0; jj < nj; ++jj) {
@@ -423,18 +428,17 @@ __device__ void issue_down(const FusedArgs& a, const LayerPtr& L, const RouteSme
                            uint32_t dst, uint64_t* full, int lane) {
   const Geometry& g = a.g;
   const int Kmax = max(g.I, g.Is);
-  for (int c = lane; c < nj * (kFDims + 2); c += 32) {
-    const int jj = c / (kFDims + 2), r = c % (kFDims + 2);
+  if (lane < nj) {
+    const int jj = lane;
     const bool sh = j0 + jj == 0;
     const int K = sh ? g.Is : g.I;
     const QMatPtr& W = sh ? L.sh_down : L.down;
     const size_t row0 = static_cast<size_t>(sh ? 0 : rt.slot_e[j0 + jj] * g.H) + blk * kFDims;
     const uint32_t base = dst + jj * a.dslot;
-    if (r < kFDims)
-      tc::bulk_load(base + r * a.rs_dn, W.q + (row0 + r) * (K / 8), K / 2, full);
-    else
-      tc::bulk_load(base + kFDims * a.rs_dn + (r - kFDims) * (Kmax / 2), (r == kFDims ? W.s : W.b) +
-                    row0 * (K / kGroup), kFDims * K / 32, full);
+    const uint32_t qb = kFDims * K / 2, sb = kFDims * K / 32;
+    tc::bulk_load(base, W.q + row0 * (K / 8), qb, full);
+    tc::bulk_load(base + 8 * Kmax, W.s + row0 * (K / kGroup), sb, full);
+    tc::bulk_load(base + 8 * Kmax + Kmax / 2, W.b + row0 * (K / kGroup), sb, full);
   }
 }
 
@@ -591,6 +595,13 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
     // the layer input: x, or RMSNorm of the previous layer's output, read
     // from the exchange words as soon as every CTA has published its part
     const uint32_t tag = (rt.epoch + 1u) * 64u + static_cast<uint32_t>(l);
+    // the router bias of the logit this thread will publish, fetched now so
+    // that its memory latency overlaps the input exchange
+    float my_bias = 0.f;
+    if (tid < nrows * T && L.router_bias) {
+      const int row = static_cast<int>(blockIdx.x) + (tid / T) * G;
+      if (row < E) my_bias = __ldg(L.router_bias + row);
+    }
     const int c4 = 4 * tid;
     const bool live = c4 < g.H;
     uint2 xv[NT];
@@ -692,8 +703,9 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
       const int rr = tid / T, t = tid % T;
       const int row = blockIdx.x + rr * G;
       float v = 0.f;
+#pragma unroll
       for (int w = 0; w < kFWarps; ++w) v += part[(rr * kFWarps + w) * NT + t];
-      if (row < E && L.router_bias) v += L.router_bias[row];
+      v += my_bias;
       st_word(a.lgx + static_cast<size_t>(t) * E1 + row, tag, __float_as_uint(v));
     }
     for (int i = tid; i < T * ngrp; i += nthr) {     // sums over groups of 64 (fixed order)
@@ -732,7 +744,11 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
       topk_redux(lg + warp * E1, E, k, lane, rt.idx + warp * k, rt.w + warp * k);
       if (lane == 0) rt.sigma[warp] = sigmoid(lg[warp * E1 + E]);
     }
-    consumers_sync();
+    // one token: warp 0 selected and now groups, so a warp barrier suffices
+    if (T > 1)
+      consumers_sync();
+    else
+      __syncwarp();
     if (warp == 0) {
       // grouping by one warp, O(n) per entry: first occurrences, then each
       // entry's stable rank (entries with a smaller expert, then earlier
@@ -772,9 +788,12 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
         rt.slot_cnt[0] = T;
         rt.slot_off[0] = Tk;
       }
+      // the producer may now schedule this layer's units: the warp's writes
+      // are ordered before lane 0's arrival (release) by the warp barrier
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(ready);
     }
     consumers_sync();
-    if (tid == 0) tc::mbar_arrive(ready);   // the producer may now schedule this layer's units
     const Sched s = make_sched(a, rt.n_act);
 
     // -------------------------------------------------------------- phase C
@@ -947,14 +966,14 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
             float y[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
             if (jlive) {
               const uint8_t* ub = fsm + sl * a.slot_bytes + jj * a.dslot;
-              const uint8_t* qrow = ub + lg4 * a.rs_dn + lt * 8;
-              const uint16_t* srow = reinterpret_cast<const uint16_t*>(ub + kFDims * a.rs_dn);
-              const uint16_t* brow = reinterpret_cast<const uint16_t*>(ub + kFDims * a.rs_dn + Kmax / 2);
+              const uint8_t* qrow = ub + lg4 * (K / 2) + lt * 8;
+              const uint16_t* srow = reinterpret_cast<const uint16_t*>(ub + 8 * Kmax);
+              const uint16_t* brow = reinterpret_cast<const uint16_t*>(ub + 8 * Kmax + Kmax / 2);
               const bool tok_live = lg4 < nt;
               const int hr = pos0 + (tok_live ? lg4 : 0);
               const uint4* hrow = reinterpret_cast<const uint4*>(hs + static_cast<size_t>(hr) * Kmax) + lt * 2;
               for (int gb = 0; gb < gh; gb += 4)
-                tile_groups<4>(y, qrow, a.rs_dn, srow, brow, ng, kh * gh + gb, min(4, gh - gb), hrow, tok_live,
+                tile_groups<4>(y, qrow, K / 2, srow, brow, ng, kh * gh + gb, min(4, gh - gb), hrow, tok_live,
                                hsum + pos0 * kg, kg, nt, lg4, lt);
             }
             tc::fence_proxy_async_smem();
@@ -1086,9 +1105,9 @@ struct FusedLayout {
 FusedLayout fused_layout(const Geometry& g, int G) {
   FusedLayout f{};
   const int Kmax = g.I > g.Is ? g.I : g.Is;
-  f.rs_gu = g.H / 2 + kFRowPad;
-  f.rs_dn = Kmax / 2 + kFRowPad;
-  f.dslot = kFDims * f.rs_dn + Kmax;                        // codes, then scales and biases
+  f.rs_gu = g.H / 2;
+  f.rs_dn = Kmax / 2;                                       // down code rows are copied contiguously
+  f.dslot = 9 * Kmax;                                        // codes (8 Kmax), then scales and biases
   f.slot_bytes = 2 * kFFeat * f.rs_gu + 4 * (kFFeat * g.H / 32);   // one gate/up unit
   f.spd = f.slot_bytes / f.dslot;
   if (f.spd > kFMaxSpd) f.spd = kFMaxSpd;
