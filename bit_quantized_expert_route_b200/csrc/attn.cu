@@ -169,9 +169,10 @@ __global__ void __launch_bounds__(kAThreads, 1) attn_decode_kernel(const __grid_
   const int c0 = sp * a.cps;
   const int nc = max(min(c0 + a.cps, n_chunks) - c0, 0);
   pdl_launch_dependents();
-  // the range's block-table entries, all loads in flight together
+  // the block-table entries of the CTA's whole range, fetched together and
+  // without waiting for ctx_len (entries past the sequence are never used)
   const int blk0 = c0 * kAChunk / a.block;
-  const int nblk = nc > 0 ? ((c0 + nc) * kAChunk - 1) / a.block - blk0 + 1 : 0;
+  const int nblk = min((c0 + a.cps) * kAChunk - 1, cap - 1) / a.block - blk0 + 1;
   const int32_t* trow = a.table + static_cast<size_t>(b) * a.max_blocks;
   for (int j = threadIdx.x; j < min(nblk, kATabCache); j += kAThreads) s_tab[j] = __ldg(trow + blk0 + j);
   __syncthreads();
