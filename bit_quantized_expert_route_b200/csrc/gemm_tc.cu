@@ -63,11 +63,15 @@ constexpr int kThreads = (kMmaWarp + 1) * 32;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxCtaUnits = 256;   // chunk descriptors cached in shared memory per CTA
 
-template <bool kGateUp>
+// kNA: 128-row weight tiles per stage.  gate/up: 2 (the gate and up
+// matrices, same rows); down: 2 (two consecutive 128-row blocks of the same
+// matrix, which share every token tile: half the token-tile traffic per
+// FLOP) or 1 (H not a multiple of 256).
+template <bool kGateUp, int kNA>
 struct Cfg {
-  static constexpr int NA = kGateUp ? 2 : 1;                 // weight matrices per stage
+  static constexpr int NA = kNA;                              // weight tiles per stage
   static constexpr int ACC_COLS = NA * BN;                    // one accumulator set
-  static constexpr int ACC_BUFS = kGateUp ? 1 : 2;
+  static constexpr int ACC_BUFS = kNA == 2 ? 1 : 2;
   static constexpr int A_COLS = NA * BK / 2;                  // TMEM columns per A stage
   static constexpr int A_BASE = ACC_BUFS * ACC_COLS;
   static constexpr int A_STAGES = (static_cast<int>(kTmemCols) - A_BASE) / A_COLS;
@@ -83,7 +87,7 @@ struct Cfg {
   static constexpr int BAR_OFF = OFF_OUT + OUT_BYTES;
   static constexpr int OFF_UNITS = BAR_OFF + 512;             // this CTA's chunk descriptors
   static constexpr int SMEM = OFF_UNITS + kMaxCtaUnits * 16 + 1024;   // + alignment slack
-  static constexpr int DQ_PER_STAGE = kGateUp ? 256 : 128;    // dequant threads consuming one stage
+  static constexpr int DQ_PER_STAGE = kNA * 128;             // dequant threads consuming one stage
 };
 
 struct alignas(64) TcArgs {
@@ -110,7 +114,7 @@ struct UnitInfo {
   int e, row0, rows, f0, K, nks, wrow;   // wrow: first weight row of the tile in its matrix stack
 };
 
-template <bool kGateUp>
+template <bool kGateUp, int kNA>
 __device__ __forceinline__ UnitInfo unit_info(const TcArgs& a, int u, int nfb, const Chunk* cache) {
   // this CTA's units are u = blockIdx.x + i * gridDim.x; their chunks were
   // copied to shared memory at the start, so the per-stage bookkeeping of
@@ -122,7 +126,7 @@ __device__ __forceinline__ UnitInfo unit_info(const TcArgs& a, int u, int nfb, c
   ui.e = ch.e;
   ui.row0 = ch.row0;
   ui.rows = ch.rows;
-  ui.f0 = (u % nfb) * BM;
+  ui.f0 = (u % nfb) * BM * (kGateUp ? 1 : kNA);   // first weight row (down: of the unit's kNA blocks)
   const int Ie = ui.shared ? a.g.Is : a.g.I;
   const int R = kGateUp ? Ie : a.g.H;          // weight rows of this expert's matrix
   ui.skip = ui.f0 >= R || ui.rows <= 0;
@@ -134,7 +138,7 @@ __device__ __forceinline__ UnitInfo unit_info(const TcArgs& a, int u, int nfb, c
 
 // Walks this CTA's stages in order: (unit, k-step) with global stage and
 // scale-block counts (a scale block starts at every k-step multiple of 8).
-template <bool kGateUp>
+template <bool kGateUp, int kNA>
 struct StageCursor {
   int u, ks;
   uint32_t it, blk;
@@ -144,7 +148,7 @@ struct StageCursor {
   const Chunk* cache;
   __device__ __forceinline__ void seek_unit(const TcArgs& a, int from, int n_units, int nfb) {
     for (u = from; u < n_units; u += gridDim.x) {
-      ui = unit_info<kGateUp>(a, u, nfb, cache);
+      ui = unit_info<kGateUp, kNA>(a, u, nfb, cache);
       if (!ui.skip) {
         ks = 0;
         done = false;
@@ -166,9 +170,9 @@ struct StageCursor {
   }
 };
 
-template <bool kGateUp>
+template <bool kGateUp, int kNA>
 __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __grid_constant__ TcArgs a) {
-  using C = Cfg<kGateUp>;
+  using C = Cfg<kGateUp, kNA>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = tc::smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);   // 1024-B aligned swizzle atoms
@@ -224,7 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
   // router, or of an earlier call, gave up) means the chunk list may not
   // describe this call's tokens: do nothing (uniform over the CTA)
   if (*reinterpret_cast<volatile const int*>(a.status) != 0) return;
-  const int nfb = (kGateUp ? max(a.g.I, a.g.Is) : a.g.H) / BM;
+  const int nfb = (kGateUp ? max(a.g.I, a.g.Is) / BM : a.g.H / (BM * kNA));
   const int n_units = *a.n_chunks * nfb;
   const int Tk = a.g.T * a.g.k;
   Chunk* units = reinterpret_cast<Chunk*>(smem + C::OFF_UNITS);
@@ -247,13 +251,13 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
     // latency of one stage's loads, dequantisation and TMEM store overlaps the
     // other sets' work.
     const int set = warp >> 2;
-    const int m = kGateUp ? (set & 1) : 0;
+    const int m = kNA == 2 ? (set & 1) : 0;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const int psw = (r >> 2) & 1;                    // 32-byte swizzle of the packed tile rows
     auto mine = [&](uint32_t it) {
-      return kGateUp ? static_cast<int>(it & 1u) == (set >> 1) : static_cast<int>(it & 3u) == set;
+      return kNA == 2 ? static_cast<int>(it & 1u) == (set >> 1) : static_cast<int>(it & 3u) == set;
     };
-    StageCursor<kGateUp> cur;
+    StageCursor<kGateUp, kNA> cur;
     cur.begin(a, n_units, nfb, units);
     while (!cur.done && !mine(cur.it)) cur.next(a, n_units, nfb);
     bool ok = true;
@@ -281,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
         bv = sb[C::S_BYTES / 2 + ks % kSBlock];
       } else {
         const QMatPtr& W = cur.ui.shared ? (m == 0 ? a.S0 : a.S1) : (m == 0 ? a.W0 : a.W1);
-        const size_t row = static_cast<size_t>(cur.ui.wrow + r);
+        const size_t row = static_cast<size_t>(cur.ui.wrow + (kGateUp ? 0 : m * BM) + r);
         sv = __ldg(W.s + row * (cur.ui.K / kGroup) + ks);
         bv = __ldg(W.b + row * (cur.ui.K / kGroup) + ks);
       }
@@ -339,49 +343,64 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
     uint16_t* stage = reinterpret_cast<uint16_t*>(smem + C::OFF_OUT);   // [BN tokens][BM features]
     uint32_t tt = 0;
     for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
-      const UnitInfo ui = unit_info<kGateUp>(a, u, nfb, units);
+      const UnitInfo ui = unit_info<kGateUp, kNA>(a, u, nfb, units);
       if (ui.skip) continue;
       const int buf = static_cast<int>(tt % C::ACC_BUFS);
       if (!tc::mbar_wait(&acc_full[buf], (tt / C::ACC_BUFS) & 1u, abort_flag, a.status, a.wait_limit)) break;
       tc::tc_fence_after();
       const uint32_t acc = lane_base + buf * C::ACC_COLS;
-      for (int n0 = 0; n0 < ui.rows; n0 += 16) {
-        float v0[16];
-        tc::tmem_ld16(acc + n0, v0);
-        if (kGateUp) {
-          float v1[16];
-          tc::tmem_ld16(acc + BN + n0, v1);
-          tc::tmem_wait_ld();
+      // gate/up: one output tile (SwiGLU of the two accumulators); down: one
+      // tile per 128-row block, staged and written out in turn
+      constexpr int kRounds = kGateUp ? 1 : kNA;
+      bool ok = true;
+      for (int mm = 0; mm < kRounds && ok; ++mm) {
+        const uint32_t rr = tt * kRounds + mm;         // staging rounds so far: the epi_sync phases
+        for (int n0 = 0; n0 < ui.rows; n0 += 16) {
+          float v0[16];
+          tc::tmem_ld16(acc + mm * BN + n0, v0);
+          if (kGateUp) {
+            float v1[16];
+            tc::tmem_ld16(acc + BN + n0, v1);
+            tc::tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float g = v0[j];
-            stage[(n0 + j) * BM + rpos] = float_to_bf16_bits(__fdividef(g * v1[j], 1.0f + __expf(-g)));
+            for (int j = 0; j < 16; ++j) {
+              const float g = v0[j];
+              stage[(n0 + j) * BM + rpos] = float_to_bf16_bits(__fdividef(g * v1[j], 1.0f + __expf(-g)));
+            }
+          } else {
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) stage[(n0 + j) * BM + r] = float_to_bf16_bits(v0[j]);
           }
-        } else {
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 16; ++j) stage[(n0 + j) * BM + r] = float_to_bf16_bits(v0[j]);
         }
+        if (mm == kRounds - 1) {
+          // accumulator drained: hand it back to the MMA before writing the tile out
+          tc::tc_fence_before();
+          tc::mbar_arrive(&acc_empty[buf]);
+        }
+        tc::mbar_arrive(&epi_sync[0]);
+        if (!tc::mbar_wait(&epi_sync[0], rr & 1u, abort_flag, a.status, a.wait_limit)) {
+          ok = false;
+          break;
+        }
+        // coalesced copy-out: each token row of the tile is BM contiguous outputs (256 B)
+        const int chunks = ui.rows * (BM / 8);
+        for (int i = et; i < chunks; i += 128) {
+          const int n = i / (BM / 8), c = i % (BM / 8);
+          const int R = ui.row0 + n;
+          uint16_t* dst;
+          if (kGateUp)
+            dst = ui.shared ? a.hs_out + static_cast<size_t>(R - Tk) * a.g.Is
+                            : a.h_out + static_cast<size_t>(R) * a.g.I;
+          else
+            dst = a.Y + static_cast<size_t>(R) * a.g.H;
+          *reinterpret_cast<uint4*>(dst + ui.f0 + mm * BM + c * 8) =
+              *reinterpret_cast<const uint4*>(stage + n * BM + c * 8);
+        }
+        tc::mbar_arrive(&epi_sync[1]);                     // the staging tile is free again
+        if (!tc::mbar_wait(&epi_sync[1], rr & 1u, abort_flag, a.status, a.wait_limit)) ok = false;
       }
-      // accumulator drained: hand it back to the MMA before writing the tile out
-      tc::tc_fence_before();
-      tc::mbar_arrive(&acc_empty[buf]);
-      tc::mbar_arrive(&epi_sync[0]);
-      if (!tc::mbar_wait(&epi_sync[0], tt & 1u, abort_flag, a.status, a.wait_limit)) break;
-      // coalesced copy-out: each token row of the tile is BM contiguous outputs (256 B)
-      const int chunks = ui.rows * (BM / 8);
-      for (int i = et; i < chunks; i += 128) {
-        const int n = i / (BM / 8), c = i % (BM / 8);
-        const int R = ui.row0 + n;
-        uint16_t* dst;
-        if (kGateUp)
-          dst = ui.shared ? a.hs_out + static_cast<size_t>(R - Tk) * a.g.Is : a.h_out + static_cast<size_t>(R) * a.g.I;
-        else
-          dst = a.Y + static_cast<size_t>(R) * a.g.H;
-        *reinterpret_cast<uint4*>(dst + ui.f0 + c * 8) = *reinterpret_cast<const uint4*>(stage + n * BM + c * 8);
-      }
-      tc::mbar_arrive(&epi_sync[1]);                     // the staging tile is free again
-      if (!tc::mbar_wait(&epi_sync[1], tt & 1u, abort_flag, a.status, a.wait_limit)) break;
+      if (!ok) break;
       ++tt;
     }
   } else if (warp == kLoadWarp) {
@@ -390,7 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
       uint32_t it = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-        const UnitInfo ui = unit_info<kGateUp>(a, u, nfb, units);
+        const UnitInfo ui = unit_info<kGateUp, kNA>(a, u, nfb, units);
         if (ui.skip) continue;
         // gate/up: rows of the grouped x (shared-expert rows follow the routed
         // ones); down: routed h or shared h
@@ -413,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
   } else if (warp == kTmaWarp) {
     // ----------------------------------------- packed tiles and scales (TMA)
     if (lane == 0) {
-      StageCursor<kGateUp> cur;
+      StageCursor<kGateUp, kNA> cur;
       cur.begin(a, n_units, nfb, units);
       uint32_t last_blk = 0xffffffffu;
       uint32_t p_fills = 0, s_fills = 0;   // packed-tile and scale-block fills issued
@@ -429,8 +448,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
           const uint32_t sdst = sbase + C::OFF_S + ss * C::S_SLOT;
 #pragma unroll
           for (int mm = 0; mm < C::NA; ++mm) {
-            tc::tma_load_2d(sdst + mm * 2 * C::S_BYTES, &a.tm_s[side][mm], cur.ks, cur.ui.wrow, &full_s[ss]);
-            tc::tma_load_2d(sdst + mm * 2 * C::S_BYTES + C::S_BYTES, &a.tm_b[side][mm], cur.ks, cur.ui.wrow,
+            tc::tma_load_2d(sdst + mm * 2 * C::S_BYTES, &a.tm_s[side][kGateUp ? mm : 0], cur.ks,
+                            cur.ui.wrow + (kGateUp ? 0 : mm * BM), &full_s[ss]);
+            tc::tma_load_2d(sdst + mm * 2 * C::S_BYTES + C::S_BYTES, &a.tm_b[side][kGateUp ? mm : 0], cur.ks,
+                            cur.ui.wrow + (kGateUp ? 0 : mm * BM),
                             &full_s[ss]);
           }
         }
@@ -441,8 +462,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
         tc::mbar_arrive_expect_tx(&full_p[sp], C::NA * C::P_BYTES);
 #pragma unroll
         for (int mm = 0; mm < C::NA; ++mm)
-          tc::tma_load_2d(sbase + C::OFF_P + (sp * C::NA + mm) * C::P_BYTES, &a.tm_q[side][mm], cur.ks * 8,
-                          cur.ui.wrow, &full_p[sp]);
+          tc::tma_load_2d(sbase + C::OFF_P + (sp * C::NA + mm) * C::P_BYTES, &a.tm_q[side][kGateUp ? mm : 0],
+                          cur.ks * 8, cur.ui.wrow + (kGateUp ? 0 : mm * BM), &full_p[sp]);
         cur.next(a, n_units, nfb);
       }
       // every copy this thread requested has landed before the CTA may exit
@@ -460,7 +481,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
     uint32_t it = 0, tt = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const UnitInfo ui = unit_info<kGateUp>(a, u, nfb, units);
+      const UnitInfo ui = unit_info<kGateUp, kNA>(a, u, nfb, units);
       if (ui.skip) continue;
       const int n_mma = max(16, (ui.rows + 15) & ~15);
       const uint32_t idesc = tc::idesc_bf16(BM, n_mma);
@@ -577,12 +598,12 @@ cudaError_t launch_gateup(const Geometry& g, const LayerPtr& L, const uint16_t* 
       !make_map(&a.tm_h[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, xg, g.H, rows, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   a.tm_h[1] = a.tm_h[0];
-  using C = Cfg<true>;
-  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(grouped_gemm_tc_kernel<true>), C::SMEM);
+  using C = Cfg<true, 2>;
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(grouped_gemm_tc_kernel<true, 2>), C::SMEM);
   if (e != cudaSuccess) return e;
   const int nfb = max(g.I, g.Is) / BM;
   const int grid = max(1, min(max_chunks * nfb, num_sms()));
-  return launch_pdl(grouped_gemm_tc_kernel<true>, dim3(grid), dim3(kThreads), C::SMEM, s, a);
+  return launch_pdl(grouped_gemm_tc_kernel<true, 2>, dim3(grid), dim3(kThreads), C::SMEM, s, a);
 }
 
 cudaError_t launch_down(const Geometry& g, const LayerPtr& L, const uint16_t* h, const uint16_t* h_s,
@@ -605,12 +626,20 @@ cudaError_t launch_down(const Geometry& g, const LayerPtr& L, const uint16_t* h,
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map(&a.tm_h[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h_s, g.Is, g.T, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  using C = Cfg<false>;
-  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(grouped_gemm_tc_kernel<false>), C::SMEM);
+  if (g.H % (2 * BM) == 0) {   // two 128-row blocks per unit share each token tile
+    using C = Cfg<false, 2>;
+    cudaError_t e = ensure_smem(reinterpret_cast<const void*>(grouped_gemm_tc_kernel<false, 2>), C::SMEM);
+    if (e != cudaSuccess) return e;
+    const int nfb = g.H / (2 * BM);
+    const int grid = max(1, min(max_chunks * nfb, num_sms()));
+    return launch_pdl(grouped_gemm_tc_kernel<false, 2>, dim3(grid), dim3(kThreads), C::SMEM, s, a);
+  }
+  using C = Cfg<false, 1>;
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(grouped_gemm_tc_kernel<false, 1>), C::SMEM);
   if (e != cudaSuccess) return e;
   const int nfb = g.H / BM;
   const int grid = max(1, min(max_chunks * nfb, num_sms()));
-  return launch_pdl(grouped_gemm_tc_kernel<false>, dim3(grid), dim3(kThreads), C::SMEM, s, a);
+  return launch_pdl(grouped_gemm_tc_kernel<false, 1>, dim3(grid), dim3(kThreads), C::SMEM, s, a);
 }
 
 }  // namespace moe
