@@ -51,8 +51,8 @@ namespace {
 constexpr int BM = 128;          // weight rows per tile = TMEM lanes (MMA M)
 constexpr int BN = 128;          // rows (tokens) per chunk: MMA N <= 128
 constexpr int BK = 64;           // inputs per stage: one quantisation group
-constexpr int kBStages = 6;      // token-tile ring
-constexpr int kPStages = 8;      // packed-tile ring
+constexpr int kBStagesMax = 6;   // token-tile ring
+constexpr int kPStagesMax = 8;   // packed-tile ring
 constexpr int kSBlock = 8;       // quantisation groups per scale block (16 B per row)
 constexpr int kDqWarps = 16;     // dequantiser warps (4 sets of 4: one per TMEM lane quadrant)
 constexpr int kEpiWarp0 = kDqWarps;
@@ -79,10 +79,17 @@ struct Cfg {
   static constexpr int P_BYTES = BM * 32;                     // 4 KB packed tile of one matrix
   static constexpr int S_BYTES = BM * kSBlock * 2;            // 2 KB: 8 groups of scales (or biases)
   static constexpr int S_SLOT = NA * 2 * S_BYTES;             // scales + biases of every matrix
-  static constexpr int OUT_BYTES = BN * BM * 2;               // epilogue staging tile (bf16)
+  // Down with two blocks stages both output tiles at once, so the single
+  // accumulator goes back to the MMA as soon as it is drained; the rings
+  // give up one token stage and two packed stages to make room.
+  static constexpr bool STAGE_ALL = !kGateUp && kNA == 2;
+  static constexpr int OUT_TILES = STAGE_ALL ? kNA : 1;
+  static constexpr int BST = STAGE_ALL ? kBStagesMax - 1 : kBStagesMax;
+  static constexpr int PST = STAGE_ALL ? kPStagesMax - 2 : kPStagesMax;
+  static constexpr int OUT_BYTES = OUT_TILES * BN * BM * 2;   // epilogue staging tiles (bf16)
   static constexpr int OFF_B = 0;
-  static constexpr int OFF_P = OFF_B + kBStages * B_BYTES;
-  static constexpr int OFF_S = OFF_P + kPStages * NA * P_BYTES;
+  static constexpr int OFF_P = OFF_B + BST * B_BYTES;
+  static constexpr int OFF_S = OFF_P + PST * NA * P_BYTES;
   static constexpr int OFF_OUT = OFF_S + 2 * S_SLOT;
   static constexpr int BAR_OFF = OFF_OUT + OUT_BYTES;
   static constexpr int OFF_UNITS = BAR_OFF + 512;             // this CTA's chunk descriptors
@@ -178,11 +185,11 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
   uint8_t* smem = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);   // 1024-B aligned swizzle atoms
   const uint32_t sbase = tc::smem_u32(smem);
 
-  uint64_t* full_b = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);   // [kBStages]
-  uint64_t* empty_b = full_b + kBStages;                                // [kBStages]
-  uint64_t* full_p = empty_b + kBStages;                                // [kPStages]
-  uint64_t* empty_p = full_p + kPStages;                                // [kPStages]
-  uint64_t* full_s = empty_p + kPStages;                                // [2]
+  uint64_t* full_b = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);   // [C::BST]
+  uint64_t* empty_b = full_b + C::BST;                                // [C::BST]
+  uint64_t* full_p = empty_b + C::BST;                                // [C::PST]
+  uint64_t* empty_p = full_p + C::PST;                                // [C::PST]
+  uint64_t* full_s = empty_p + C::PST;                                // [2]
   uint64_t* empty_s = full_s + 2;                                       // [2]
   uint64_t* full_a = empty_s + 2;                                       // [A_STAGES]
   uint64_t* empty_a = full_a + C::A_STAGES;                             // [A_STAGES]
@@ -195,11 +202,11 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kBStages; ++s) {
+    for (int s = 0; s < C::BST; ++s) {
       tc::mbar_init(&full_b[s], 1);
       tc::mbar_init(&empty_b[s], 1);
     }
-    for (int s = 0; s < kPStages; ++s) {
+    for (int s = 0; s < C::PST; ++s) {
       tc::mbar_init(&full_p[s], 1);
       tc::mbar_init(&empty_p[s], C::DQ_PER_STAGE);
     }
@@ -290,8 +297,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
         bv = __ldg(W.b + row * (cur.ui.K / kGroup) + ks);
       }
       // packed words of this stage's tile row
-      const int sp = static_cast<int>(it % kPStages);
-      if (!tc::mbar_wait(&full_p[sp], (it / kPStages) & 1u, abort_flag, a.status, a.wait_limit)) {
+      const int sp = static_cast<int>(it % C::PST);
+      if (!tc::mbar_wait(&full_p[sp], (it / C::PST) & 1u, abort_flag, a.status, a.wait_limit)) {
         ok = false;
         break;
       }
@@ -350,11 +357,14 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
       tc::tc_fence_after();
       const uint32_t acc = lane_base + buf * C::ACC_COLS;
       // gate/up: one output tile (SwiGLU of the two accumulators); down: one
-      // tile per 128-row block, staged and written out in turn
+      // tile per 128-row block, staged and written out in turn, or (two
+      // blocks) both staged before either is written, so that the single
+      // accumulator is handed back as early as possible
       constexpr int kRounds = kGateUp ? 1 : kNA;
+      constexpr bool kAll = C::STAGE_ALL;
       bool ok = true;
       for (int mm = 0; mm < kRounds && ok; ++mm) {
-        const uint32_t rr = tt * kRounds + mm;         // staging rounds so far: the epi_sync phases
+        uint16_t* st = stage + (kAll ? mm * BN * BM : 0);
         for (int n0 = 0; n0 < ui.rows; n0 += 16) {
           float v0[16];
           tc::tmem_ld16(acc + mm * BN + n0, v0);
@@ -365,12 +375,12 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
               const float g = v0[j];
-              stage[(n0 + j) * BM + rpos] = float_to_bf16_bits(__fdividef(g * v1[j], 1.0f + __expf(-g)));
+              st[(n0 + j) * BM + rpos] = float_to_bf16_bits(__fdividef(g * v1[j], 1.0f + __expf(-g)));
             }
           } else {
             tc::tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 16; ++j) stage[(n0 + j) * BM + r] = float_to_bf16_bits(v0[j]);
+            for (int j = 0; j < 16; ++j) st[(n0 + j) * BM + r] = float_to_bf16_bits(v0[j]);
           }
         }
         if (mm == kRounds - 1) {
@@ -378,26 +388,31 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
           tc::tc_fence_before();
           tc::mbar_arrive(&acc_empty[buf]);
         }
+        if (kAll && mm != kRounds - 1) continue;
+        const uint32_t rr = kAll ? tt : tt * kRounds + mm;   // staging rounds so far: the epi_sync phases
         tc::mbar_arrive(&epi_sync[0]);
         if (!tc::mbar_wait(&epi_sync[0], rr & 1u, abort_flag, a.status, a.wait_limit)) {
           ok = false;
           break;
         }
-        // coalesced copy-out: each token row of the tile is BM contiguous outputs (256 B)
+        // coalesced copy-out: each token row of a tile is BM contiguous outputs (256 B)
         const int chunks = ui.rows * (BM / 8);
-        for (int i = et; i < chunks; i += 128) {
-          const int n = i / (BM / 8), c = i % (BM / 8);
-          const int R = ui.row0 + n;
-          uint16_t* dst;
-          if (kGateUp)
-            dst = ui.shared ? a.hs_out + static_cast<size_t>(R - Tk) * a.g.Is
-                            : a.h_out + static_cast<size_t>(R) * a.g.I;
-          else
-            dst = a.Y + static_cast<size_t>(R) * a.g.H;
-          *reinterpret_cast<uint4*>(dst + ui.f0 + mm * BM + c * 8) =
-              *reinterpret_cast<const uint4*>(stage + n * BM + c * 8);
+        for (int mo = kAll ? 0 : mm; mo <= mm; ++mo) {
+          const uint16_t* so = stage + (kAll ? mo * BN * BM : 0);
+          for (int i = et; i < chunks; i += 128) {
+            const int n = i / (BM / 8), c = i % (BM / 8);
+            const int R = ui.row0 + n;
+            uint16_t* dst;
+            if (kGateUp)
+              dst = ui.shared ? a.hs_out + static_cast<size_t>(R - Tk) * a.g.Is
+                              : a.h_out + static_cast<size_t>(R) * a.g.I;
+            else
+              dst = a.Y + static_cast<size_t>(R) * a.g.H;
+            *reinterpret_cast<uint4*>(dst + ui.f0 + mo * BM + c * 8) =
+                *reinterpret_cast<const uint4*>(so + n * BM + c * 8);
+          }
         }
-        tc::mbar_arrive(&epi_sync[1]);                     // the staging tile is free again
+        tc::mbar_arrive(&epi_sync[1]);                     // the staging tiles are free again
         if (!tc::mbar_wait(&epi_sync[1], rr & 1u, abort_flag, a.status, a.wait_limit)) ok = false;
       }
       if (!ok) break;
@@ -416,8 +431,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
         const void* tm = &a.tm_h[(!kGateUp && ui.shared) ? 1 : 0];
         const int y = (!kGateUp && ui.shared) ? ui.row0 - Tk : ui.row0;
         for (int ks = 0; ks < ui.nks; ++ks, ++it) {
-          const int s = static_cast<int>(it % kBStages);
-          if (!tc::mbar_wait(&empty_b[s], ((it / kBStages) & 1u) ^ 1u, abort_flag, a.status, a.wait_limit)) {
+          const int s = static_cast<int>(it % C::BST);
+          if (!tc::mbar_wait(&empty_b[s], ((it / C::BST) & 1u) ^ 1u, abort_flag, a.status, a.wait_limit)) {
             ok = false;
             break;
           }
@@ -426,7 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
         }
       }
       // every tile this thread requested has landed before the CTA may exit
-      tc::drain_ring(full_b, kBStages, it, a.status);
+      tc::drain_ring(full_b, C::BST, it, a.status);
     }
     __syncwarp();
   } else if (warp == kTmaWarp) {
@@ -455,8 +470,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
                             &full_s[ss]);
           }
         }
-        const int sp = static_cast<int>(cur.it % kPStages);
-        if (!tc::mbar_wait(&empty_p[sp], ((cur.it / kPStages) & 1u) ^ 1u, abort_flag, a.status, a.wait_limit)) break;
+        const int sp = static_cast<int>(cur.it % C::PST);
+        if (!tc::mbar_wait(&empty_p[sp], ((cur.it / C::PST) & 1u) ^ 1u, abort_flag, a.status, a.wait_limit)) break;
         tc::fence_proxy_async_smem();   // consumers' generic reads of the slot precede this async-proxy refill
         ++p_fills;
         tc::mbar_arrive_expect_tx(&full_p[sp], C::NA * C::P_BYTES);
@@ -467,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
         cur.next(a, n_units, nfb);
       }
       // every copy this thread requested has landed before the CTA may exit
-      tc::drain_ring(full_p, kPStages, p_fills, a.status);
+      tc::drain_ring(full_p, C::PST, p_fills, a.status);
       tc::drain_ring(full_s, 2, s_fills, a.status);
     }
     __syncwarp();
@@ -493,9 +508,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
       tc::tc_fence_after();
       const uint32_t acc = tmem + buf * C::ACC_COLS;
       for (int ks = 0; ks < ui.nks; ++ks, ++it) {
-        const int sb = static_cast<int>(it % kBStages);
+        const int sb = static_cast<int>(it % C::BST);
         const int sa = static_cast<int>(it % C::A_STAGES);
-        const bool got = tc::mbar_wait(&full_b[sb], (it / kBStages) & 1u, abort_flag, a.status, a.wait_limit) &&
+        const bool got = tc::mbar_wait(&full_b[sb], (it / C::BST) & 1u, abort_flag, a.status, a.wait_limit) &&
                          tc::mbar_wait(&full_a[sa], (it / C::A_STAGES) & 1u, abort_flag, a.status, a.wait_limit);
         if (!__all_sync(0xffffffffu, got)) {
           ok = false;
