@@ -101,7 +101,10 @@ struct alignas(64) TcArgs {
   CUtensorMap tm_q[2][2];  // packed words: [routed, shared][matrix]
   CUtensorMap tm_s[2][2];  // scales:       [routed, shared][matrix] (valid when scales_tma)
   CUtensorMap tm_b[2][2];  // biases
-  CUtensorMap tm_h[2];     // token tiles: gate/up [grouped x rows, -], down [routed h, shared h]
+  // token tiles: [gate/up: grouped x rows, - | down: routed h, shared h] x
+  // box height [16, 32, 64, 128 rows]: a chunk loads the smallest box that
+  // covers its rows (a 3-row expert group needs 2 KB per stage, not 16 KB)
+  CUtensorMap tm_h[2][4];
   Geometry g;
   QMatPtr W0, W1;          // routed stacks: {gate, up} or {down, -}
   QMatPtr S0, S1;          // shared expert: {sh_gate, sh_up} or {sh_down, -}
@@ -428,7 +431,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
         if (ui.skip) continue;
         // gate/up: rows of the grouped x (shared-expert rows follow the routed
         // ones); down: routed h or shared h
-        const void* tm = &a.tm_h[(!kGateUp && ui.shared) ? 1 : 0];
+        const int bsz = ui.rows <= 16 ? 0 : ui.rows <= 32 ? 1 : ui.rows <= 64 ? 2 : 3;
+        const void* tm = &a.tm_h[(!kGateUp && ui.shared) ? 1 : 0][bsz];
+        const uint32_t bbytes = static_cast<uint32_t>(16 << bsz) * BK * 2;   // rows x 64 inputs x bf16
         const int y = (!kGateUp && ui.shared) ? ui.row0 - Tk : ui.row0;
         for (int ks = 0; ks < ui.nks; ++ks, ++it) {
           const int s = static_cast<int>(it % C::BST);
@@ -436,7 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
             ok = false;
             break;
           }
-          tc::mbar_arrive_expect_tx(&full_b[s], C::B_BYTES);
+          tc::mbar_arrive_expect_tx(&full_b[s], bbytes);
           tc::tma_load_2d(sbase + C::OFF_B + s * C::B_BYTES, tm, ks * BK, y, &full_b[s]);
         }
       }
@@ -569,6 +574,15 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* bas
   return make_tmap_2d(m, dt, esize, base, cols, rows, box_cols, box_rows, sw);
 }
 
+// Token-tile maps of a bf16 [rows, K] matrix: 64-input boxes of 16, 32, 64
+// and 128 rows, 128-byte swizzle (K-major, the UMMA B layout).
+bool make_token_maps(CUtensorMap (&m)[4], const void* base, int K, uint64_t rows) {
+  for (int i = 0; i < 4; ++i)
+    if (!make_map(&m[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, K, rows, BK, 16u << i, CU_TENSOR_MAP_SWIZZLE_128B))
+      return false;
+  return true;
+}
+
 // Maps of one affine 4-bit matrix stack [rows, K]: packed words (box 128 rows
 // x 8 words, 32-B swizzle) and, when the scale rows are 16-B strided, scales
 // and biases (box 128 rows x 8 groups).
@@ -610,9 +624,9 @@ cudaError_t launch_gateup(const Geometry& g, const LayerPtr& L, const uint16_t* 
   const uint64_t rows = static_cast<uint64_t>(g.T) * g.k + g.T;
   if (!make_qmat_maps(a, 0, 0, L.gate, g.E * g.I, g.H) || !make_qmat_maps(a, 0, 1, L.up, g.E * g.I, g.H) ||
       !make_qmat_maps(a, 1, 0, L.sh_gate, g.Is, g.H) || !make_qmat_maps(a, 1, 1, L.sh_up, g.Is, g.H) ||
-      !make_map(&a.tm_h[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, xg, g.H, rows, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+      !make_token_maps(a.tm_h[0], xg, g.H, rows))
     return cudaErrorInvalidValue;
-  a.tm_h[1] = a.tm_h[0];
+  for (int i = 0; i < 4; ++i) a.tm_h[1][i] = a.tm_h[0][i];
   using C = Cfg<true, 2>;
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(grouped_gemm_tc_kernel<true, 2>), C::SMEM);
   if (e != cudaSuccess) return e;
@@ -637,9 +651,8 @@ cudaError_t launch_down(const Geometry& g, const LayerPtr& L, const uint16_t* h,
   a.wait_limit = wait_limit_cycles();
   a.scales_tma = (g.I % (kGroup * kSBlock)) == 0 && (g.Is % (kGroup * kSBlock)) == 0;
   if (!make_qmat_maps(a, 0, 0, L.down, g.E * g.H, g.I) || !make_qmat_maps(a, 1, 0, L.sh_down, g.H, g.Is) ||
-      !make_map(&a.tm_h[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, g.I, static_cast<uint64_t>(g.T) * g.k, BK, BN,
-                CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&a.tm_h[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h_s, g.Is, g.T, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+      !make_token_maps(a.tm_h[0], h, g.I, static_cast<uint64_t>(g.T) * g.k) ||
+      !make_token_maps(a.tm_h[1], h_s, g.Is, g.T))
     return cudaErrorInvalidValue;
   if (g.H % (2 * BM) == 0) {   // two 128-row blocks per unit share each token tile
     using C = Cfg<false, 2>;
