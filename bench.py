@@ -49,7 +49,7 @@ ATTN_L = (4096, 32768, 131072)    # decode-attention context lengths (one sequen
 GDN_B = (1, 8, 64)                # recurrence batch sizes (16 key heads, 32 value heads, 128 x 128 FP32 state)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PREFILL_LAUNCHES_PER_STEP = 7     # router (+ segment counts), scan, scatter, gather, gate/up, down, combine
-UNFUSED_DECODE_LAUNCHES = 3       # routing (router+top-k+sort), gate/up GEMV, down GEMV+combine
+UNFUSED_DECODE_LAUNCHES = 4       # routing (router+top-k+sort), gate/up GEMV, down GEMV, combine
 FUSED_DECODE_LAUNCHES = 1         # T <= 2: the whole layer in one cooperative launch
 NOMINAL_BF16_TFLOPS = 2250.0      # B200 dense bf16 datasheet figure (context)
 NOMINAL_HBM_GBS = 8000.0          # B200 HBM3e nominal bandwidth (context)
@@ -58,7 +58,7 @@ GEMM_SRC = "bit_quantized_expert_route_b200/csrc/gemm_tc.cu"
 GATEUP_KERNEL = "grouped_gemm_tc_kernel<true>"
 DOWN_KERNEL = "grouped_gemm_tc_kernel<false>"
 DECODE_KERNEL_SRC = "bit_quantized_expert_route_b200/csrc/decode.cu"
-DECODE_KERNEL = "decode_gateup_kernel"
+DECODE_KERNEL = "mid_gateup_kernel"
 FUSED_DECODE_KERNEL_SRC = "bit_quantized_expert_route_b200/csrc/decode_fused.cu"
 FUSED_DECODE_KERNEL = "decode_fused_kernel<1>"
 ATTN_SRC = "bit_quantized_expert_route_b200/csrc/attn.cu"

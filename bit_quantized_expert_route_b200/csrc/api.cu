@@ -64,6 +64,7 @@ using namespace moe;
 
 constexpr int kDecodeMaxT = 64;
 constexpr int kFusedMaxT = 8;       // tokens the fused decode kernel takes
+constexpr int kMidMaxT = 64;        // tokens the mid-size decode path takes
 constexpr int kMaxT = 65536;
 constexpr int kMaxStackLayers = 1024;
 constexpr size_t kAlign = 256;
@@ -252,38 +253,62 @@ bool fused_decode_ok(const moe_layer_desc* d, const Geometry& g) {
   return decode_fused_supported(g);
 }
 
-// moe_forward's choice for T tokens: the single-launch fused decode kernel
-// where it applies, else the tensor-core path.  (The GEMV kernels of
-// moe_decode do FP32 work per weight and token, which the tensor cores
-// outrun as soon as an expert sees more than a couple of tokens.)
-bool forward_uses_fused_decode(const moe_layer_desc* d, int T) {
-  const Geometry g{T, d->H, d->I, d->I_shared, d->E, d->k};
-  return T <= kFusedMaxT && fused_decode_ok(d, g);
+// The mid-size decode kernels load 4 groups' scales (or biases) of a row as
+// one 8-byte word.
+bool mid_decode_ok(const moe_layer_desc* d, const Geometry& g) {
+  const moe_qmat* m[6] = {&d->gate, &d->up, &d->down, &d->sh_gate, &d->sh_up, &d->sh_down};
+  for (const moe_qmat* q : m)
+    if ((reinterpret_cast<uintptr_t>(q->scales) & 7u) || (reinterpret_cast<uintptr_t>(q->biases) & 7u)) return false;
+  return mid_decode_supported(g);
 }
 
-int enqueue_decode(const moe_layer_desc* d, const uint16_t* x, int T, uint16_t* out, const Bufs& b,
-                   cudaStream_t s, Tracer* tr = nullptr) {
-  {
-    const Geometry g{T, d->H, d->I, d->I_shared, d->E, d->k};
-    if (fused_decode_ok(d, g)) {
-      mark(tr, s);
-      const LayerPtr L = layer_ptrs(d);
-      const cudaError_t e = launch_fused_layers(g, &L, 1, x, out, nullptr, 0.f, b, true, s);
-      mark(tr, s);
-      return cuda_status(e);
-    }
-  }
+// The kernels one layer of T tokens runs on: the single-launch fused decode
+// kernel where it applies (T <= 8), else for T <= kMidMaxT the mid-size
+// decode path (small-T router, mma.sync GEMVs over the active experts,
+// combine), else the tensor-core (tcgen05) grouped-GEMM path.
+enum class Path { kFused, kMid, kPrefill };
+
+Path layer_path(const moe_layer_desc* d, int T) {
+  const Geometry g{T, d->H, d->I, d->I_shared, d->E, d->k};
+  if (T <= kFusedMaxT && fused_decode_ok(d, g)) return Path::kFused;
+  if (T <= kMidMaxT && mid_decode_ok(d, g)) return Path::kMid;
+  return Path::kPrefill;
+}
+
+bool forward_uses_fused_decode(const moe_layer_desc* d, int T) { return layer_path(d, T) == Path::kFused; }
+
+// The fused decode kernel for one layer (routing outputs included).
+int enqueue_fused(const moe_layer_desc* d, const uint16_t* x, int T, uint16_t* out, const Bufs& b,
+                  cudaStream_t s, Tracer* tr = nullptr) {
+  const Geometry g{T, d->H, d->I, d->I_shared, d->E, d->k};
+  mark(tr, s);
+  const LayerPtr L = layer_ptrs(d);
+  const cudaError_t e = launch_fused_layers(g, &L, 1, x, out, nullptr, 0.f, b, true, s);
+  mark(tr, s);
+  return cuda_status(e);
+}
+
+// The mid-size decode path: router (one launch), gate/up, down, combine
+// (which also writes RMSNorm(out) to norm_out when given; out may then be
+// NULL).
+int enqueue_mid(const moe_layer_desc* d, const uint16_t* x, int T, uint16_t* out, const Bufs& b, cudaStream_t s,
+                Tracer* tr = nullptr, uint16_t* norm_out = nullptr, float eps = 0.f) {
   int st = enqueue_route(d, x, T, b, s, tr);
   if (st != MOE_OK) return st;
   const Geometry g{T, d->H, d->I, d->I_shared, d->E, d->k};
   const LayerPtr L = layer_ptrs(d);
   uint16_t* h = b.at<uint16_t>(b.w.h);
   uint16_t* h_s = b.at<uint16_t>(b.w.h_s);
-  cudaError_t e = launch_decode_gateup(g, L, x, b.offsets, b.perm, b.at<int32_t>(b.w.active),
-                                       b.at<int32_t>(b.w.n_active), h, h_s, s);
+  uint16_t* Y = b.at<uint16_t>(b.w.Y);
+  const int32_t* active = b.at<int32_t>(b.w.active);
+  const int32_t* n_active = b.at<int32_t>(b.w.n_active);
+  cudaError_t e = launch_mid_gateup(g, L, x, b.offsets, b.perm, active, n_active, h, h_s, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   mark(tr, s);
-  e = launch_decode_down_combine(g, L, h, h_s, b.topk_idx, b.topk_w, b.inv_perm, b.sigma, out, s);
+  e = launch_mid_down(g, L, h, h_s, b.offsets, active, n_active, Y, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  mark(tr, s);
+  e = launch_combine(Y, b.inv_perm, b.topk_w, b.sigma, T, d->k, d->H, out, norm_out, eps, b.at<int>(b.w.status), s);
   mark(tr, s);
   return cuda_status(e);
 }
@@ -321,11 +346,25 @@ int enqueue_prefill(const moe_layer_desc* d, const uint16_t* x, int T, uint16_t*
 // norm_out (may be NULL) its RMSNorm, the next layer's input.
 int enqueue_layer(const moe_layer_desc* d, const uint16_t* x, int T, uint16_t* out, uint16_t* norm_out, float eps,
                   const Bufs& b, cudaStream_t s) {
-  if (!forward_uses_fused_decode(d, T)) return enqueue_prefill(d, x, T, out, b, s, nullptr, norm_out, eps);
+  switch (layer_path(d, T)) {
+    case Path::kPrefill: return enqueue_prefill(d, x, T, out, b, s, nullptr, norm_out, eps);
+    case Path::kMid: return enqueue_mid(d, x, T, out, b, s, nullptr, norm_out, eps);
+    default: break;
+  }
   uint16_t* y = out ? out : norm_out;
-  const int st = enqueue_decode(d, x, T, y, b, s);
+  const int st = enqueue_fused(d, x, T, y, b, s);
   if (st != MOE_OK || !norm_out) return st;
   return cuda_status(launch_rmsnorm(y, norm_out, T, d->H, eps, s));   // in place when out is NULL
+}
+
+// One layer, output to out (the path layer_path picks).
+int enqueue_forward(const moe_layer_desc* d, const uint16_t* x, int T, uint16_t* out, const Bufs& b, cudaStream_t s,
+                    Tracer* tr = nullptr) {
+  switch (layer_path(d, T)) {
+    case Path::kFused: return enqueue_fused(d, x, T, out, b, s, tr);
+    case Path::kMid: return enqueue_mid(d, x, T, out, b, s, tr);
+    default: return enqueue_prefill(d, x, T, out, b, s, tr);
+  }
 }
 
 int check_call(const moe_layer_desc* d, const void* x, int T, int T_limit, const void* out, const moe_routing* r,
@@ -434,16 +473,14 @@ int moe_forward(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_bf16*
   const int st = check_call(layer, x, T, kMaxT, out, r, ws, ws_bytes, true);
   if (st != MOE_OK) return st;
   const Bufs b = resolve(layer, T, ws, r);
-  const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (forward_uses_fused_decode(layer, T)) return enqueue_decode(layer, x, T, out, b, s);
-  return enqueue_prefill(layer, x, T, out, b, s);
+  return enqueue_forward(layer, x, T, out, b, static_cast<cudaStream_t>(stream));
 }
 
 int moe_decode(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_bf16* out, moe_routing* r, void* ws,
                size_t ws_bytes, moe_stream stream) {
   const int st = check_call(layer, x, T, kDecodeMaxT, out, r, ws, ws_bytes, true);
   if (st != MOE_OK) return st;
-  return enqueue_decode(layer, x, T, out, resolve(layer, T, ws, r), static_cast<cudaStream_t>(stream));
+  return enqueue_forward(layer, x, T, out, resolve(layer, T, ws, r), static_cast<cudaStream_t>(stream));
 }
 
 int moe_forward_stack(const moe_layer_desc* layers, int n_layers, const moe_bf16* x, int T, moe_bf16* out,
@@ -548,7 +585,7 @@ static int forward_host_enqueue(const moe_layer_desc* layer, const moe_bf16* x_h
   uint16_t* od = b.at<uint16_t>(b.w.out_stage);
   const size_t bytes = static_cast<size_t>(T) * layer->H * sizeof(uint16_t);
   if (cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return MOE_ERR_CUDA;
-  st = forward_uses_fused_decode(layer, T) ? enqueue_decode(layer, xd, T, od, b, s) : enqueue_prefill(layer, xd, T, od, b, s);
+  st = enqueue_forward(layer, xd, T, od, b, s);
   if (st != MOE_OK) return st;
   if (cudaMemcpyAsync(out_host, od, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
@@ -589,7 +626,7 @@ int moe_forward_profiled(const moe_layer_desc* layer, const moe_bf16* x, int T, 
       for (int j = 0; j < i; ++j) cudaEventDestroy(tr.ev[j]);
       return MOE_ERR_CUDA;
     }
-  st = forward_uses_fused_decode(layer, T) ? enqueue_decode(layer, x, T, out, b, s, &tr) : enqueue_prefill(layer, x, T, out, b, s, &tr);
+  st = enqueue_forward(layer, x, T, out, b, s, &tr);
   if (st == MOE_OK && cudaEventSynchronize(tr.ev[tr.n - 1]) != cudaSuccess) st = MOE_ERR_CUDA;
   *n_stages = 0;
   if (st == MOE_OK) {
@@ -611,8 +648,14 @@ int moe_get_status(void* ws, moe_stream stream) {
   int host = 0;
   if (cudaMemcpyAsync(&host, ws, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
-  // a device timeout can leave the control block's counters mid-count: clear it whole
+  // a device timeout can leave the control block's counters mid-count: clear
+  // them (the status word, the routing and exit counters, the small-T
+  // router's token-group counters; not the fused kernel's epoch)
   if (host != MOE_OK && cudaMemsetAsync(ws, 0, 16, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (host != MOE_OK &&
+      cudaMemsetAsync(static_cast<char*>(ws) + 4 * (1 + kSmallGroupCounter), 0, 4 * kSmallMaxGroups, s) !=
+          cudaSuccess)
+    return MOE_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
   return host;
 }

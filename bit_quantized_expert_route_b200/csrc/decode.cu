@@ -1,33 +1,48 @@
-// Decode path (T <= 64): the layer as bandwidth-bound GEMVs over the active
-// experts only.  Batch-1 decoding barely reuses a weight, so every packed
-// weight byte is read once with 128-bit coalesced loads and rebuilt in
-// registers in FP32 ("Perplexity's Lily: ...", section "How It Works: Prefill
-// and Decode Strategies", decode paragraph; "Frequently Asked Questions":
-// decode is bound by moving weights, not by arithmetic).
+// Decode path for steps of up to 64 tokens that the fused kernel does not
+// take: the tokens of the step spread over many experts with a few tokens
+// each, so the layer is bound by streaming the active experts' packed weights
+// ("Perplexity's Lily: ...", section "How It Works: Prefill and Decode
+// Strategies", decode paragraph; "Frequently Asked Questions": decode moves
+// weights, not arithmetic).  Two persistent kernels do the expert GEMVs on
+// the tensor cores through warp-level mma.sync, the (up to) 8 tokens of an
+// expert being the 8 columns of the n8 tile; the fixed-order combine kernel
+// of the prefill path then adds each token's k + 1 terms.
 //
-// Dequantisation in FP32 without per-weight multiplies: for the 32 codes q_i
-// of one 128-bit load (half a quantisation group: one scale s, one bias b)
-//   sum_i (s q_i + b) x_i = 128 s * sum_i f_i x_i + (b - 128 s) * sum_i x_i,
-//   f_i = 1 + q_i / 128,
-// where f_i is built exactly by OR-ing the code into the mantissa of 1.0f
-// (one shift + one LOP3), and sum_i x_i is computed once per token per
-// segment when the activations are staged.  So a code costs about three
-// instructions per token instead of a convert, a dequant FMA and a dot FMA.
+// Work items.  An active expert slot with n tokens is cut into ceil(n/8)
+// token tiles; an item is one token tile of one slot times one block of rows
+// (gate/up: 128 features; down: 256 output dims).  A CTA of 8 warps takes
+// items blockIdx.x, blockIdx.x + gridDim.x, ...; the items of one (slot, row
+// block) are numbered consecutively over their token tiles, so the CTAs that
+// read the same weights run side by side and all but the first read them
+// from L2.  Per item the CTA stages the tile's activations in shared memory
+// (bf16, in the interleaved order of mma_dq.cuh, plus per-group sums); each
+// warp computes two 16-row tiles against it (gate/up: the gate and the up
+// tile of the same 16 features, so SwiGLU needs no exchange; down: 32
+// consecutive dims), so every activation fragment read from shared memory
+// feeds two MMAs.
+//
+// Weight streaming.  The packed codes go from global memory straight into
+// the MMA operand registers (8 bytes per lane per row and group): a warp
+// holds the next 4 groups of both tiles in flight (group j of the next block
+// of 4 is loaded right after group j of the current block has been used),
+// running on into the CTA's next item, whose weights do not depend on the
+// activations; the scales and biases of the next block (one 8-byte load per
+// row) are loaded a block ahead.  Shared memory carries only the
+// activations, read conflict-free: token rows are padded by 16 bytes and the
+// group sums are stored token-minor, so a lane's two sums are one 8-byte
+// read.
 #include "common.cuh"
 #include "kernels.h"
+#include "mma_dq.cuh"
 
 namespace moe {
 
-constexpr int kDecWarps = 8;
-constexpr int kRowsPerWarp = 4;                        // features per warp (each: gate row and up row)
-constexpr int kDecFeat = kDecWarps * kRowsPerWarp;     // features per CTA
-constexpr int kDownDims = 16;                          // output dims per CTA (8 warps x 2 half-warps)
-constexpr int kDecTokMaxDecode = 8;                    // tokens per pass over an expert's weights
-
-// Staged row strides (floats): whole interleave windows of 32 (gate/up) or
-// 16 (down) lanes x 32 codes.
-__host__ __device__ __forceinline__ int xstride_of(int H) { return (H + 1023) / 1024 * 1024; }
-__host__ __device__ __forceinline__ int hstride_of(int I) { return (I + 511) / 512 * 512; }
+constexpr int kMWarps = 8;
+constexpr int kMThreads = kMWarps * 32;
+constexpr int kMGateUpRows = 16 * kMWarps;   // features of a gate/up item
+constexpr int kMDownRows = 32 * kMWarps;     // output dims of a down item
+constexpr int kMTok = 8;                     // tokens of an item: the n8 column tile
+constexpr int kMBlock = 4;                   // groups of 64 inputs per pipeline block
 
 __device__ __forceinline__ QMatPtr expert_qmat(const QMatPtr& stack, int e, size_t rows, size_t cols) {
   return QMatPtr{stack.q + static_cast<size_t>(e) * rows * (cols / 8),
@@ -35,327 +50,401 @@ __device__ __forceinline__ QMatPtr expert_qmat(const QMatPtr& stack, int e, size
                  stack.b + static_cast<size_t>(e) * rows * (cols / kGroup)};
 }
 
-// f_i = 1 + q_i/128 for the eight codes of a word (code i in bits 4i..4i+3).
-__device__ __forceinline__ void codes_plus_one(uint32_t w, float (&f)[8]) {
-  const uint32_t M = 0x000F0000u, ONE = 0x3F800000u;
-  f[0] = __uint_as_float(((w << 16) & M) | ONE);
-  f[1] = __uint_as_float(((w << 12) & M) | ONE);
-  f[2] = __uint_as_float(((w << 8) & M) | ONE);
-  f[3] = __uint_as_float(((w << 4) & M) | ONE);
-  f[4] = __uint_as_float((w & M) | ONE);
-  f[5] = __uint_as_float(((w >> 4) & M) | ONE);
-  f[6] = __uint_as_float(((w >> 8) & M) | ONE);
-  f[7] = __uint_as_float(((w >> 12) & M) | ONE);
-}
-
-// sum_i f_i * x_i over the 32 codes of one 128-bit load; x comes from the
-// lane-interleaved staging buffer: float4 j (codes 4j..4j+3) of this lane's
-// segment at xl[j * stride4] (stride4 in float4 units).
-__device__ __forceinline__ float dot32(const uint4& qv, const float4* __restrict__ xl, int stride4) {
-  const uint32_t words[4] = {qv.x, qv.y, qv.z, qv.w};
-  float a = 0.f;
+// Items of every active slot, as an exclusive prefix in shared memory:
+// start[s] = first item of slot s, start[n_act] = the total.  Slot s is
+// expert active[s] (E: the shared expert, which sees all T tokens) with
+// ceil(n/8) token tiles times `blocks_routed` (or `blocks_shared`) row blocks.
+// Two slots per thread, so up to 2 * kMThreads slots.
+__device__ int build_items(const Geometry& g, const int32_t* offsets, const int32_t* active, int n_act,
+                           int blocks_routed, int blocks_shared, int* start, int* warp_tot) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int c[2];
 #pragma unroll
-  for (int wd = 0; wd < 4; ++wd) {
-    float f[8];
-    codes_plus_one(words[wd], f);
-    const float4 x0 = xl[(2 * wd) * stride4];
-    const float4 x1 = xl[(2 * wd + 1) * stride4];
-    a = fmaf(f[0], x0.x, a); a = fmaf(f[1], x0.y, a); a = fmaf(f[2], x0.z, a); a = fmaf(f[3], x0.w, a);
-    a = fmaf(f[4], x1.x, a); a = fmaf(f[5], x1.y, a); a = fmaf(f[6], x1.z, a); a = fmaf(f[7], x1.w, a);
+  for (int j = 0; j < 2; ++j) {
+    const int s = 2 * threadIdx.x + j;
+    c[j] = 0;
+    if (s < n_act) {
+      const int e = active[s];
+      const int n = e >= g.E ? g.T : offsets[e + 1] - offsets[e];
+      c[j] = (n + kMTok - 1) / kMTok * (e >= g.E ? blocks_shared : blocks_routed);
+    }
   }
-  return a;
+  const int v = c[0] + c[1];
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  int before = 0, total = 0;
+#pragma unroll
+  for (int w = 0; w < kMWarps; ++w) {
+    const int t = warp_tot[w];
+    before += w < warp ? t : 0;
+    total += t;
+  }
+  const int excl = before + incl - v;
+  if (2 * threadIdx.x < n_act) start[2 * threadIdx.x] = excl;
+  if (2 * threadIdx.x + 1 < n_act) start[2 * threadIdx.x + 1] = excl + c[0];
+  if (threadIdx.x == 0) start[n_act] = total;
+  __syncthreads();
+  return total;
 }
 
-// ---------------------------------------------------------------------------
-// gate/up: CTA (active expert slot, block of 32 features).  Warp w owns
-// features f0 + 4w .. +3; lane l owns the 128-bit load positions c = 32 v + l
-// (v = 0 .. H/1024 - 1) of every row.  Activations of up to `kb` tokens at a
-// time are staged as FP32 in a lane-interleaved layout:
-//   element c*32 + i of token r at float index ((v*8 + i/4) * 32 + l) * 4 + i%4
-// so that lane l's eight float4 reads are conflict-free, plus per-segment sums.
-// ---------------------------------------------------------------------------
-template <int NT>
-__device__ __forceinline__ void gateup_warp(const QMatPtr& Wg, const QMatPtr& Wu, int H, int frow, int nf,
-                                            const float* __restrict__ xs, const float* __restrict__ xsum,
-                                            int nt, int lane, float (&res)[2][kRowsPerWarp][NT]) {
-  const int xst = xstride_of(H);
-  float acc[2][kRowsPerWarp][NT];
+// Item `it` decoded: slot s = the last with start[s] <= it, its expert, the
+// token tile (first grouped position pos0, tn tokens) and the row block.
+struct Item {
+  int e;        // expert (E: shared)
+  bool sh;
+  int blk;      // row block
+  int tn;       // tokens in the tile (1..8)
+  int pos0;     // routed: first grouped position; shared: first token
+};
+
+__device__ __forceinline__ Item decode_item(const Geometry& g, const int* start, int n_act, const int32_t* offsets,
+                                            const int32_t* active, int it) {
+  int lo = 0, hi = n_act - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (start[mid] <= it) lo = mid;
+    else hi = mid - 1;
+  }
+  Item r;
+  r.e = active[lo];
+  r.sh = r.e >= g.E;
+  const int nt = r.sh ? g.T : offsets[r.e + 1] - offsets[r.e];
+  const int ntt = (nt + kMTok - 1) / kMTok;
+  const int local = it - start[lo];
+  r.blk = local / ntt;
+  const int tt = local - r.blk * ntt;
+  r.tn = min(kMTok, nt - tt * kMTok);
+  r.pos0 = (r.sh ? 0 : offsets[r.e]) + tt * kMTok;
+  return r;
+}
+
+// Stage `tn` activation rows of `cols` bf16 values (row r at row_of(r)) as
+// xs[r][cols/8 + 1] uint4 in the interleaved order, and their sums per group
+// of 64 (FP32) as xsum[group][8 tokens].  Each group's 8 uint4 are handled by
+// 8 consecutive lanes, which add their partial sums with shuffles; each
+// thread has kStageLoads loads in flight.
+constexpr int kStageLoads = 4;
+template <class RowOf>
+__device__ __forceinline__ void stage_tile(RowOf row_of, int tn, int cols, uint4* xs, float* xsum) {
+  const int cpr = cols / 8;
+  const int n = tn * cpr;
+  // the loop bound is the warp's first index, so whole warps take part in the shuffles
+  for (int base = threadIdx.x & ~31; base < n; base += kMThreads * kStageLoads) {
+    const int i0 = base + (threadIdx.x & 31);
+    uint4 v[kStageLoads];
+#pragma unroll
+    for (int j = 0; j < kStageLoads; ++j) {
+      const int i = i0 + j * kMThreads;
+      const int r = i / cpr, u = i - r * cpr;
+      v[j] = i < n ? __ldg(reinterpret_cast<const uint4*>(row_of(r)) + u) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int j = 0; j < kStageLoads; ++j) {
+      const int i = i0 + j * kMThreads;
+      const int r = i / cpr, u = i - r * cpr;
+      float sm = ((bf16_lo(v[j].x) + bf16_hi(v[j].x)) + (bf16_lo(v[j].y) + bf16_hi(v[j].y))) +
+                 ((bf16_lo(v[j].z) + bf16_hi(v[j].z)) + (bf16_lo(v[j].w) + bf16_hi(v[j].w)));
+      sm += __shfl_xor_sync(0xffffffffu, sm, 1);
+      sm += __shfl_xor_sync(0xffffffffu, sm, 2);
+      sm += __shfl_xor_sync(0xffffffffu, sm, 4);
+      if (i < n) {
+        xs[r * (cpr + 1) + u] = interleave8(v[j]);
+        if ((u & 7) == 0) xsum[(u >> 3) * kMTok + r] = sm;
+      }
+    }
+  }
+}
+
+// The two 16-row tiles one warp computes for an item, as this lane's
+// pointers: the codes of rows lg4 and lg4 + 8 of tile m start at q[m] and
+// q[m] + 8 rs (rs = 32 ngr bytes per row; already offset by the lane's 8
+// bytes of a group), the scales and biases of row lg4 at s[m] and b[m]
+// (row lg4 + 8: + 8 ngr).
+struct WTile {
+  const uint8_t* q[2];
+  const uint16_t* s[2];
+  const uint16_t* b[2];
+};
+
+__device__ __forceinline__ WTile make_wtile(const QMatPtr& W0, size_t row0, const QMatPtr& W1, size_t row1, int ngr,
+                                            int lg4, int lt) {
+  const size_t rs = static_cast<size_t>(ngr) * 32;
+  WTile w;
+  w.q[0] = reinterpret_cast<const uint8_t*>(W0.q) + (row0 + lg4) * rs + lt * 8;
+  w.q[1] = reinterpret_cast<const uint8_t*>(W1.q) + (row1 + lg4) * rs + lt * 8;
+  w.s[0] = W0.s + (row0 + lg4) * ngr;
+  w.b[0] = W0.b + (row0 + lg4) * ngr;
+  w.s[1] = W1.s + (row1 + lg4) * ngr;
+  w.b[1] = W1.b + (row1 + lg4) * ngr;
+  return w;
+}
+
+// Codes of group G of both tiles (rows lg4 and lg4 + 8) into registers.
+__device__ __forceinline__ void load_group(uint2 (&a)[2][2], const WTile& w, int ngr, int G) {
 #pragma unroll
   for (int m = 0; m < 2; ++m)
 #pragma unroll
-    for (int f = 0; f < kRowsPerWarp; ++f)
+    for (int r = 0; r < 2; ++r)
+      a[m][r] = __ldg(reinterpret_cast<const uint2*>(w.q[m] + static_cast<size_t>(r) * 8 * ngr * 32 + G * 32));
+}
+
+// Scales and biases of groups G0 .. G0 + 3 (4 bf16 per row and tile).
+struct BlockS {
+  uint2 s[2][2], b[2][2];   // [tile][row]
+};
+__device__ __forceinline__ void load_scales(BlockS& S, const WTile& w, int ngr, int G0) {
 #pragma unroll
-      for (int r = 0; r < NT; ++r) acc[m][f][r] = 0.f;
-  const int nv = xst / 1024;               // 128-bit positions per lane per row
-  const int wpr = H / 8, gpr = H / kGroup;
-  const int seg_per_tok = xst / 32;
-  for (int v = 0; v < nv; ++v) {
-    const int c = v * 32 + lane;
-    if (c >= H / 32) break;
-    uint4 q[2][kRowsPerWarp];
-    float s[2][kRowsPerWarp], b[2][kRowsPerWarp];
+  for (int m = 0; m < 2; ++m)
 #pragma unroll
-    for (int m = 0; m < 2; ++m) {
-      const QMatPtr& W = m == 0 ? Wg : Wu;
-#pragma unroll
-      for (int f = 0; f < kRowsPerWarp; ++f) {
-        const size_t row = static_cast<size_t>(frow + min(f, nf - 1));
-        q[m][f] = __ldg(reinterpret_cast<const uint4*>(W.q + row * wpr) + c);
-        s[m][f] = bf16_bits_to_float(__ldg(W.s + row * gpr + (c >> 1)));
-        b[m][f] = bf16_bits_to_float(__ldg(W.b + row * gpr + (c >> 1)));
-      }
+    for (int r = 0; r < 2; ++r) {
+      S.s[m][r] = __ldg(reinterpret_cast<const uint2*>(w.s[m] + r * 8 * ngr + G0));
+      S.b[m][r] = __ldg(reinterpret_cast<const uint2*>(w.b[m] + r * 8 * ngr + G0));
     }
-    const float4* xl = reinterpret_cast<const float4*>(xs) + (v * 8) * 32 + lane;
+}
+
+// Group G (position j of its block) of both tiles against the staged token
+// tile: y[m][r][c] += s * sum (128 + q) x + (b - 128 s) X for row lg4 + 8r
+// of tile m and token column 2lt + c.
+__device__ __forceinline__ void group_step(float (&y)[2][2][2], const uint2 (&a)[2][2], const BlockS& S, int j,
+                                           const uint4* xr, const float* xsum, int G, int lt) {
+  const uint4 xb0 = xr[G * 8], xb1 = xr[G * 8 + 1];
+  const float2 X = *reinterpret_cast<const float2*>(xsum + G * kMTok + 2 * lt);
 #pragma unroll
-    for (int r = 0; r < NT; ++r) {
-      if (r < nt) {
-        const float4* xr = xl + static_cast<size_t>(r) * (xst / 4);
-        const float X = xsum[r * seg_per_tok + c];
+  for (int m = 0; m < 2; ++m) {
+    float d[4];
+    group_dot(d, a[m][0], a[m][1], xb0, xb1);
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const uint32_t sp = (j < 2) ? S.s[m][r].x : S.s[m][r].y;
+      const uint32_t bp = (j < 2) ? S.b[m][r].x : S.b[m][r].y;
+      const float sc = (j & 1) ? bf16_hi(sp) : bf16_lo(sp);
+      const float cb = fmaf(-128.f, sc, (j & 1) ? bf16_hi(bp) : bf16_lo(bp));
+      y[m][r][0] = fmaf(cb, X.x, fmaf(sc, d[2 * r], y[m][r][0]));
+      y[m][r][1] = fmaf(cb, X.y, fmaf(sc, d[2 * r + 1], y[m][r][1]));
+    }
+  }
+}
+
+// The body both kernels share.  tile_of(item, warp, lg4, lt) -> WTile: the
+// warp's two tiles; k_of(item): inputs per row (a multiple of 256);
+// row_of(item) -> a function r -> activation row r of the token tile;
+// store(item, warp, y, lg4, lt): the epilogue.  Shared memory: the staged
+// token tile.
+template <class TileOf, class KOf, class RowOf, class Store>
+__device__ __forceinline__ void mid_body(const Geometry& g, const int32_t* offsets, const int32_t* active,
+                                         const int32_t* n_active, int blocks_routed, int blocks_shared, int kmax,
+                                         uint8_t* msm, TileOf tile_of, KOf k_of, RowOf row_of, Store store) {
+  __shared__ int s_start[2 * kMThreads + 1];
+  __shared__ int s_wt[kMWarps];
+  const int n_act = *n_active;
+  const int total = build_items(g, offsets, active, n_act, blocks_routed, blocks_shared, s_start, s_wt);
+  if (static_cast<int>(blockIdx.x) >= total) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, lg4 = lane >> 2, lt = lane & 3;
+  uint4* xs = reinterpret_cast<uint4*>(msm);
+  float* xsum = reinterpret_cast<float*>(xs + kMTok * (kmax / 8 + 1));
+
+  Item I = decode_item(g, s_start, n_act, offsets, active, blockIdx.x);
+  WTile cur = tile_of(I, warp, lg4, lt);
+  int ngr = k_of(I) / kGroup;
+  uint2 A[kMBlock][2][2];
+  BlockS S;
+#pragma unroll
+  for (int j = 0; j < kMBlock; ++j) load_group(A[j], cur, ngr, j);
+  load_scales(S, cur, ngr, 0);
+  for (int k = 0;; ++k) {
+    const int K = k_of(I);
+    if (k > 0) __syncthreads();   // every warp is done with the previous item's staged tile
+    stage_tile(row_of(I), I.tn, K, xs, xsum);
+    __syncthreads();
+    const int nit = blockIdx.x + (k + 1) * gridDim.x;
+    const bool has_next = nit < total;
+    Item NI = I;
+    WTile nxt = cur;
+    int nngr = ngr;
+    if (has_next) {
+      NI = decode_item(g, s_start, n_act, offsets, active, nit);
+      nxt = tile_of(NI, warp, lg4, lt);
+      nngr = k_of(NI) / kGroup;
+    }
+    float y[2][2][2] = {{{0.f, 0.f}, {0.f, 0.f}}, {{0.f, 0.f}, {0.f, 0.f}}};
+    const uint4* xr = xs + lg4 * (K / 8 + 1) + lt * 2;
+    const int nbat = ngr / kMBlock;
+    for (int b = 0; b < nbat; ++b) {
+      const bool last = b + 1 == nbat;
+      const bool nvalid = !last || has_next;       // a next block to prefetch
+      const WTile& nw = last ? nxt : cur;
+      const int nG0 = last ? 0 : (b + 1) * kMBlock;
+      const int ng = last ? nngr : ngr;
+      BlockS NS = S;
+      if (nvalid) load_scales(NS, nw, ng, nG0);
+#pragma unroll
+      for (int j = 0; j < kMBlock; ++j) {
+        group_step(y, A[j], S, j, xr, xsum, b * kMBlock + j, lt);
+        if (nvalid) load_group(A[j], nw, ng, nG0 + j);
+      }
+      S = NS;
+    }
+    store(I, warp, y, lg4, lt);
+    if (!has_next) break;
+    I = NI;
+    cur = nxt;
+    ngr = nngr;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// gate/up + SwiGLU: h[pos] = bf16(silu(W_g x_t) * (W_u x_t)) for every routed
+// entry pos (token t = perm[pos] / k) and h_s[t] for the shared expert.
+// Warp w: the gate and up rows of features blk * 128 + 16 w .. + 15.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kMThreads, 2) mid_gateup_kernel(
+    Geometry g, LayerPtr L, const uint16_t* __restrict__ x, const int32_t* __restrict__ offsets,
+    const int32_t* __restrict__ perm, const int32_t* __restrict__ active, const int32_t* __restrict__ n_active,
+    uint16_t* __restrict__ h, uint16_t* __restrict__ h_s) {
+  extern __shared__ __align__(16) uint8_t msm[];
+  pdl_wait();
+  pdl_launch_dependents();
+  const int ngr = g.H / kGroup;
+  auto tile_of = [&](const Item& I, int warp, int lg4, int lt) {
+    const size_t f0 = static_cast<size_t>(I.blk) * kMGateUpRows + warp * 16;
+    const QMatPtr Wg = I.sh ? L.sh_gate : expert_qmat(L.gate, I.e, g.I, g.H);
+    const QMatPtr Wu = I.sh ? L.sh_up : expert_qmat(L.up, I.e, g.I, g.H);
+    return make_wtile(Wg, f0, Wu, f0, ngr, lg4, lt);
+  };
+  auto k_of = [&](const Item&) { return g.H; };
+  auto row_of = [&](const Item& I) {
+    return [&, I](int r) { return x + static_cast<size_t>(I.sh ? I.pos0 + r : perm[I.pos0 + r] / g.k) * g.H; };
+  };
+  auto store = [&](const Item& I, int warp, float (&y)[2][2][2], int lg4, int lt) {
+    const int Ie = I.sh ? g.Is : g.I;
+    const int f0 = I.blk * kMGateUpRows + warp * 16;
+    uint16_t* dst = I.sh ? h_s : h;
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const int col = 2 * lt + c;
+      if (col < I.tn)
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+          dst[static_cast<size_t>(I.pos0 + col) * Ie + f0 + lg4 + 8 * r] =
+              float_to_bf16_bits(silu(y[0][r][c]) * y[1][r][c]);
+    }
+  };
+  mid_body(g, offsets, active, n_active, g.I / kMGateUpRows, g.Is / kMGateUpRows, g.H, msm, tile_of, k_of, row_of,
+           store);
+}
+
+// ---------------------------------------------------------------------------
+// down: Y[pos] = bf16(W_d[e] h[pos]) for every routed entry (rows in the
+// grouped order, as the prefill path's down GEMM writes them) and
+// Y[T*k + t] = bf16(W_sd h_s[t]); the combine kernel then forms
+// out_t = sum_j w[t,j] Y[inv_perm[t*k+j]] + sigma_t Y[T*k+t] in that order.
+// Warp w: dims blk * 256 + 32 w .. + 31 (two tiles of 16).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kMThreads, 2) mid_down_kernel(
+    Geometry g, LayerPtr L, const uint16_t* __restrict__ h, const uint16_t* __restrict__ h_s,
+    const int32_t* __restrict__ offsets, const int32_t* __restrict__ active, const int32_t* __restrict__ n_active,
+    uint16_t* __restrict__ Y) {
+  extern __shared__ __align__(16) uint8_t msm[];
+  pdl_wait();
+  pdl_launch_dependents();
+  const int blocks = g.H / kMDownRows;
+  auto tile_of = [&](const Item& I, int warp, int lg4, int lt) {
+    const size_t d0 = static_cast<size_t>(I.blk) * kMDownRows + warp * 32;
+    const QMatPtr W = I.sh ? L.sh_down : expert_qmat(L.down, I.e, g.H, g.I);
+    return make_wtile(W, d0, W, d0 + 16, (I.sh ? g.Is : g.I) / kGroup, lg4, lt);
+  };
+  auto k_of = [&](const Item& I) { return I.sh ? g.Is : g.I; };
+  auto row_of = [&](const Item& I) {
+    return [&, I](int r) { return (I.sh ? h_s : h) + static_cast<size_t>(I.pos0 + r) * (I.sh ? g.Is : g.I); };
+  };
+  auto store = [&](const Item& I, int warp, float (&y)[2][2][2], int lg4, int lt) {
+    const int d0 = I.blk * kMDownRows + warp * 32;
+    const size_t row0 = I.sh ? static_cast<size_t>(g.T) * g.k + I.pos0 : static_cast<size_t>(I.pos0);
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const int col = 2 * lt + c;
+      if (col < I.tn)
 #pragma unroll
         for (int m = 0; m < 2; ++m)
 #pragma unroll
-          for (int f = 0; f < kRowsPerWarp; ++f) {
-            const float A = dot32(q[m][f], xr, 32);
-            const float s128 = 128.f * s[m][f];
-            acc[m][f][r] = fmaf(s128, A, fmaf(b[m][f] - s128, X, acc[m][f][r]));
-          }
-      }
+          for (int r = 0; r < 2; ++r)
+            Y[(row0 + col) * g.H + d0 + 16 * m + lg4 + 8 * r] = float_to_bf16_bits(y[m][r][c]);
     }
-  }
-#pragma unroll
-  for (int m = 0; m < 2; ++m)
-#pragma unroll
-    for (int f = 0; f < kRowsPerWarp; ++f)
-#pragma unroll
-      for (int r = 0; r < NT; ++r) res[m][f][r] = warp_sum(acc[m][f][r]);
+  };
+  mid_body(g, offsets, active, n_active, blocks, blocks, max(g.I, g.Is), msm, tile_of, k_of, row_of, store);
 }
 
-template <int NT>
-__device__ __forceinline__ void gateup_store(const QMatPtr& Wg, const QMatPtr& Wu, int H, int frow, int nf,
-                                             const float* xs, const float* xsum, int nt, int lane,
-                                             uint16_t* const* dst) {
-  float res[2][kRowsPerWarp][NT];
-  gateup_warp<NT>(Wg, Wu, H, frow, nf, xs, xsum, nt, lane, res);
-#pragma unroll
-  for (int f = 0; f < kRowsPerWarp; ++f)
-#pragma unroll
-    for (int r = 0; r < NT; ++r)
-      if (lane == ((f * NT + r) & 31) && f < nf && r < nt)
-        dst[r][frow + f] = float_to_bf16_bits(silu(res[0][f][r]) * res[1][f][r]);
+namespace {
+
+// Resident CTAs of a mid-size kernel on this device (cached per kernel,
+// device and shared-memory size).
+int resident_ctas(int which, const void* func, int smem) {
+  static int cache[2][16] = {};
+  static int cache_smem[2][16] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16) return 0;
+  if (cache[which][dev] > 0 && cache_smem[which][dev] == smem) return cache[which][dev];
+  int sms = 0, per_sm = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, func, kMThreads, smem) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  if (per_sm < 1) return 0;
+  cache[which][dev] = sms * per_sm;
+  cache_smem[which][dev] = smem;
+  return cache[which][dev];
 }
 
-// Stage `nt` activation rows (bf16) as FP32 in the lane-interleaved layout
-// and their 32-element segment sums.
-__device__ __forceinline__ void stage_rows(const uint16_t* const* rows, int nt, int H, int lanes, int stride,
-                                           float* xs, float* xsum) {
-  const int vec = H / 8;
-  for (int i = threadIdx.x; i < nt * vec; i += blockDim.x) {
-    const int r = i / vec, u = i - r * vec;           // u: 8-element chunk index
-    const uint4 v = reinterpret_cast<const uint4*>(rows[r])[u];
-    const int e0 = u * 8;                             // first element
-    const int c = e0 >> 5, ii = e0 & 31;              // segment, offset in segment
-    const int win = c / lanes, ln = c - win * lanes;
-    float4* base = reinterpret_cast<float4*>(xs + static_cast<size_t>(r) * stride);
-    base[((win * 8 + (ii >> 2)) * lanes) + ln] = make_float4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y));
-    base[((win * 8 + (ii >> 2) + 1) * lanes) + ln] =
-        make_float4(bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w));
-  }
-  __syncthreads();
-  const int segs = H / 32, sstride = stride / 32;
-  for (int i = threadIdx.x; i < nt * segs; i += blockDim.x) {
-    const int r = i / segs, c = i - r * segs;
-    const int win = c / lanes, ln = c - win * lanes;
-    const float4* base = reinterpret_cast<const float4*>(xs + static_cast<size_t>(r) * stride);
-    float sum = 0.f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float4 q = base[(win * 8 + j) * lanes + ln];
-      sum += (q.x + q.y) + (q.z + q.w);
-    }
-    xsum[r * sstride + c] = sum;
-  }
-  __syncthreads();
+// An upper bound of the items of a call: every routed entry may open its own
+// token tile, and the active slots add at most one partial tile each.
+int max_items(const Geometry& g, int blocks_routed, int blocks_shared) {
+  const int n = g.T * g.k;
+  const int slots = min(g.E, n);
+  return (n / kMTok + slots) * blocks_routed + (g.T + kMTok - 1) / kMTok * blocks_shared;
 }
 
-__global__ void __launch_bounds__(256) decode_gateup_kernel(
-    Geometry g, LayerPtr L, const uint16_t* __restrict__ x, const int32_t* __restrict__ offsets,
-    const int32_t* __restrict__ perm, const int32_t* __restrict__ active, const int32_t* __restrict__ n_active,
-    uint16_t* __restrict__ h, uint16_t* __restrict__ h_s, int kb) {
-  extern __shared__ float sm[];
-  const int slot = blockIdx.x;
-  if (slot >= *n_active) return;
-  const int e = active[slot];
-  const bool shared = e >= g.E;
-  const int Ie = shared ? g.Is : g.I;
-  const int i0 = blockIdx.y * kDecFeat;
-  if (i0 >= Ie) return;
-  const QMatPtr Wg = shared ? L.sh_gate : expert_qmat(L.gate, e, g.I, g.H);
-  const QMatPtr Wu = shared ? L.sh_up : expert_qmat(L.up, e, g.I, g.H);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int frow = i0 + warp * kRowsPerWarp;
-  const int nf = max(0, min(kRowsPerWarp, Ie - frow));
-  // warm this warp's first weight bytes before the token-list dependency chain
-  if (nf > 0) {
-    const int wpr = g.H / 8;
-#pragma unroll
-    for (int f = 0; f < kRowsPerWarp; ++f) {
-      const size_t row = static_cast<size_t>(frow + min(f, nf - 1));
-      asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<const uint4*>(Wg.q + row * wpr) + lane));
-      asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<const uint4*>(Wu.q + row * wpr) + lane));
-    }
-  }
-  const int pos0 = shared ? 0 : offsets[e];
-  const int ntok = shared ? g.T : offsets[e + 1] - pos0;
-  const int xst = xstride_of(g.H);
-  float* xs = sm;                                        // [kb][xst]
-  float* xsum = sm + static_cast<size_t>(kb) * xst;      // [kb][xst/32]
-  for (int tb = 0; tb < ntok; tb += kb) {
-    const int nt = min(kb, ntok - tb);
-    const uint16_t* rows[kDecTokMaxDecode];
-    uint16_t* dst[kDecTokMaxDecode];
-#pragma unroll
-    for (int r = 0; r < kDecTokMaxDecode; ++r) {
-      const int rr = min(r, nt - 1);
-      const int tok = shared ? (tb + rr) : perm[pos0 + tb + rr] / g.k;
-      rows[r] = x + static_cast<size_t>(tok) * g.H;
-      dst[r] = shared ? h_s + static_cast<size_t>(tb + rr) * g.Is : h + static_cast<size_t>(pos0 + tb + rr) * g.I;
-    }
-    __syncthreads();
-    stage_rows(rows, nt, g.H, 32, xst, xs, xsum);
-    if (nf > 0) {
-      if (nt == 1)
-        gateup_store<1>(Wg, Wu, g.H, frow, nf, xs, xsum, nt, lane, dst);
-      else if (nt == 2)
-        gateup_store<2>(Wg, Wu, g.H, frow, nf, xs, xsum, nt, lane, dst);
-      else if (nt <= 4)
-        gateup_store<4>(Wg, Wu, g.H, frow, nf, xs, xsum, nt, lane, dst);
-      else
-        gateup_store<8>(Wg, Wu, g.H, frow, nf, xs, xsum, nt, lane, dst);
-    }
-  }
+// Shared memory: the staged token tile for rows of up to kmax inputs.
+int mid_smem(int kmax) { return kMTok * (kmax / 8 + 1) * 16 + kMTok * (kmax / kGroup) * 4; }
+
+}  // namespace
+
+bool mid_decode_supported(const Geometry& g) {
+  return g.T >= 1 && g.T <= 64 && g.H % 256 == 0 && g.I % 256 == 0 && g.Is % 256 == 0 && g.H <= 8192 &&
+         g.I <= 2048 && g.Is <= 2048;
 }
 
-__device__ __forceinline__ float halfwarp_sum(float v) {
-#pragma unroll
-  for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
-// ---------------------------------------------------------------------------
-// down + combine: CTA (token t, block of 16 output dims); half-warp per dim.
-//   out[t, d] = bf16( sum_j w[t,j] * (W_d[idx_j][d,:] . h_{t,j})  +  sigma_t * (W_sd[d,:] . hs_t) )
-// The k + 1 terms are added in slot order, then the shared term.  The h rows
-// are staged as FP32 with 16-lane interleaving (both half-warps read the same
-// addresses) plus segment sums.
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) decode_down_combine_kernel(
-    Geometry g, LayerPtr L, const uint16_t* __restrict__ h, const uint16_t* __restrict__ h_s,
-    const int32_t* __restrict__ topk_idx, const float* __restrict__ topk_w, const int32_t* __restrict__ inv_perm,
-    const float* __restrict__ sigma, uint16_t* __restrict__ out) {
-  extern __shared__ float sm[];
-  const int t = blockIdx.x;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int hl = lane & 15;
-  const int d = blockIdx.y * kDownDims + warp * 2 + (lane >> 4);
-  const bool live = d < g.H;
-  const int dd = min(d, g.H - 1);
-  const int Imax = max(g.I, g.Is);
-  const int hst = hstride_of(Imax);
-  const int nterm = g.k + 1;
-  float* hs = sm;                                          // [k+1][hst]
-  float* hsum = sm + static_cast<size_t>(nterm) * hst;     // [k+1][hst/32]
-  const uint16_t* rows[kMaxK + 1];
-  for (int j = 0; j < nterm; ++j)
-    rows[j] = j < g.k ? h + static_cast<size_t>(inv_perm[t * g.k + j]) * g.I : h_s + static_cast<size_t>(t) * g.Is;
-  // stage h rows (routed rows have I columns, the shared row Is; Imax stride)
-  {
-    const int vec = Imax / 8;
-    for (int i = threadIdx.x; i < nterm * vec; i += blockDim.x) {
-      const int j = i / vec, u = i - j * vec;
-      const int Ij = j < g.k ? g.I : g.Is;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (u * 8 < Ij) v = reinterpret_cast<const uint4*>(rows[j])[u];
-      const int e0 = u * 8, c = e0 >> 5, ii = e0 & 31;
-      const int win = c >> 4, ln = c & 15;
-      float4* base = reinterpret_cast<float4*>(hs + static_cast<size_t>(j) * hst);
-      base[(win * 8 + (ii >> 2)) * 16 + ln] = make_float4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y));
-      base[(win * 8 + (ii >> 2) + 1) * 16 + ln] = make_float4(bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w));
-    }
-    __syncthreads();
-    const int segs = Imax / 32;
-    for (int i = threadIdx.x; i < nterm * segs; i += blockDim.x) {
-      const int j = i / segs, c = i - j * segs;
-      const int win = c >> 4, ln = c & 15;
-      const float4* base = reinterpret_cast<const float4*>(hs + static_cast<size_t>(j) * hst);
-      float sum = 0.f;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const float4 f4 = base[(win * 8 + q) * 16 + ln];
-        sum += (f4.x + f4.y) + (f4.z + f4.w);
-      }
-      hsum[j * (hst / 32) + c] = sum;
-    }
-    __syncthreads();
-  }
-  float acc = 0.f;
-  for (int j = 0; j < nterm; ++j) {
-    const bool sh = j == g.k;
-    const int Ie = sh ? g.Is : g.I;
-    const QMatPtr W = sh ? L.sh_down : expert_qmat(L.down, topk_idx[t * g.k + j], g.H, g.I);
-    const int nv = hst / 512;
-    float p = 0.f;
-    for (int v = 0; v < nv; ++v) {
-      const int c = v * 16 + hl;
-      if (c < Ie / 32) {
-        const size_t row = static_cast<size_t>(dd);
-        const uint4 qv = __ldg(reinterpret_cast<const uint4*>(W.q + row * (Ie / 8)) + c);
-        const float s = bf16_bits_to_float(__ldg(W.s + row * (Ie / kGroup) + (c >> 1)));
-        const float b = bf16_bits_to_float(__ldg(W.b + row * (Ie / kGroup) + (c >> 1)));
-        const float4* hl4 = reinterpret_cast<const float4*>(hs + static_cast<size_t>(j) * hst) + (v * 8) * 16 + hl;
-        const float A = dot32(qv, hl4, 16);
-        const float X = hsum[j * (hst / 32) + c];
-        const float s128 = 128.f * s;
-        p = fmaf(s128, A, fmaf(b - s128, X, p));
-      }
-    }
-    p = halfwarp_sum(p);
-    const float coef = sh ? sigma[t] : topk_w[t * g.k + j];
-    acc = fmaf(coef, p, acc);
-  }
-  if (live && hl == 0) out[static_cast<size_t>(t) * g.H + d] = float_to_bf16_bits(acc);
-}
-
-int decode_tokens_per_pass(int H) {
-  const int per_tok = xstride_of(H) * 4 + xstride_of(H) / 8;
-  return max(1, min(kDecTokMaxDecode, 98304 / per_tok));
-}
-
-cudaError_t launch_decode_gateup(const Geometry& g, const LayerPtr& L, const uint16_t* x,
-                                 const int32_t* offsets, const int32_t* perm,
-                                 const int32_t* active, const int32_t* n_active,
-                                 uint16_t* h, uint16_t* h_s, cudaStream_t s) {
-  const int slots = min(g.E, g.T * g.k) + 1;
-  const int fblocks = (max(g.I, g.Is) + kDecFeat - 1) / kDecFeat;
-  const int kb = min(decode_tokens_per_pass(g.H), g.T);
-  const int smem = kb * (xstride_of(g.H) * 4 + (xstride_of(g.H) / 32) * 4);
-  const cudaError_t e = ensure_smem(reinterpret_cast<const void*>(decode_gateup_kernel), smem);
+cudaError_t launch_mid_gateup(const Geometry& g, const LayerPtr& L, const uint16_t* x, const int32_t* offsets,
+                              const int32_t* perm, const int32_t* active, const int32_t* n_active, uint16_t* h,
+                              uint16_t* h_s, cudaStream_t s) {
+  const int smem = mid_smem(g.H);
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(mid_gateup_kernel), smem);
   if (e != cudaSuccess) return e;
-  decode_gateup_kernel<<<dim3(slots, fblocks), 256, smem, s>>>(g, L, x, offsets, perm, active, n_active, h, h_s,
-                                                               kb);
-  return cudaGetLastError();
+  const int res = resident_ctas(0, reinterpret_cast<const void*>(mid_gateup_kernel), smem);
+  if (res <= 0) return cudaErrorInvalidConfiguration;
+  const int grid = max(1, min(res, max_items(g, g.I / kMGateUpRows, g.Is / kMGateUpRows)));
+  return launch_pdl(mid_gateup_kernel, dim3(grid), dim3(kMThreads), smem, s, g, L, x, offsets, perm, active,
+                    n_active, h, h_s);
 }
 
-cudaError_t launch_decode_down_combine(const Geometry& g, const LayerPtr& L, const uint16_t* h,
-                                       const uint16_t* h_s, const int32_t* topk_idx, const float* topk_w,
-                                       const int32_t* inv_perm, const float* sigma, uint16_t* out,
-                                       cudaStream_t s) {
-  const int hst = hstride_of(max(g.I, g.Is));
-  const int smem = (g.k + 1) * (hst * 4 + (hst / 32) * 4);
-  const cudaError_t e = ensure_smem(reinterpret_cast<const void*>(decode_down_combine_kernel), smem);
+cudaError_t launch_mid_down(const Geometry& g, const LayerPtr& L, const uint16_t* h, const uint16_t* h_s,
+                            const int32_t* offsets, const int32_t* active, const int32_t* n_active, uint16_t* Y,
+                            cudaStream_t s) {
+  const int smem = mid_smem(max(g.I, g.Is));
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(mid_down_kernel), smem);
   if (e != cudaSuccess) return e;
-  decode_down_combine_kernel<<<dim3(g.T, (g.H + kDownDims - 1) / kDownDims), 256, smem, s>>>(
-      g, L, h, h_s, topk_idx, topk_w, inv_perm, sigma, out);
-  return cudaGetLastError();
+  const int res = resident_ctas(1, reinterpret_cast<const void*>(mid_down_kernel), smem);
+  if (res <= 0) return cudaErrorInvalidConfiguration;
+  const int blocks = g.H / kMDownRows;
+  const int grid = max(1, min(res, max_items(g, blocks, blocks)));
+  return launch_pdl(mid_down_kernel, dim3(grid), dim3(kMThreads), smem, s, g, L, h, h_s, offsets, active,
+                    n_active, Y);
 }
 
 }  // namespace moe

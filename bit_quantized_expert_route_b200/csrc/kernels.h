@@ -82,10 +82,18 @@ cudaError_t launch_router(const uint16_t* x, const uint16_t* w_router, const flo
                           int32_t* topk_idx, float* topk_w, float* sigma, int32_t* seg_counts, int* status,
                           cudaStream_t s);
 
+// route.cu: small-T router (T <= kSmallTB * kSmallMaxGroups).  `counter`
+// points at a zeroed control area of at least (kSmallGroupCounter +
+// kSmallMaxGroups) words: word 0 counts finished token groups, word
+// kSmallGroupCounter + y the finished CTAs of token group y.
+constexpr int kSmallTB = 8;
+constexpr int kSmallMaxGroups = 8;
+constexpr int kSmallGroupCounter = 16;
+
 // route.cu
 int num_segments(int T);   // 128-token segments of the counting sort
 // T <= 64: router + top-k + shared gate + counting sort + active list in one launch.
-// logits: workspace [T, E+1] FP32; counter: workspace word that must be zero.
+// logits: workspace [T, E+1] FP32; counter: the control area described above.
 cudaError_t launch_route_small(const uint16_t* x, const LayerPtr& L, int T, int H, int I, int Is, int E, int k,
                                float* logits, unsigned* counter, const RoutingPtrs& r, int32_t* active,
                                int32_t* n_active, cudaStream_t s);
@@ -125,15 +133,17 @@ cudaError_t launch_combine(const uint16_t* Y, const int32_t* inv_perm, const flo
                            cudaStream_t s);
 cudaError_t launch_rmsnorm(const uint16_t* y, uint16_t* out, int T, int H, float eps, cudaStream_t s);
 
-// decode.cu: T <= 64
-cudaError_t launch_decode_gateup(const Geometry& g, const LayerPtr& L, const uint16_t* x,
-                                 const int32_t* offsets, const int32_t* perm,
-                                 const int32_t* active, const int32_t* n_active,
-                                 uint16_t* h, uint16_t* h_s, cudaStream_t s);
-cudaError_t launch_decode_down_combine(const Geometry& g, const LayerPtr& L, const uint16_t* h,
-                                       const uint16_t* h_s, const int32_t* topk_idx, const float* topk_w,
-                                       const int32_t* inv_perm, const float* sigma, uint16_t* out,
-                                       cudaStream_t s);
+// decode.cu: steps of up to 64 tokens outside the fused kernel's range.
+// Persistent mma.sync GEMVs over the active experts; gate/up writes h (rows
+// in the grouped order) and h_s, down writes Y in the layout combine_kernel
+// reads (routed rows in the grouped order, then the T shared rows).
+bool mid_decode_supported(const Geometry& g);
+cudaError_t launch_mid_gateup(const Geometry& g, const LayerPtr& L, const uint16_t* x, const int32_t* offsets,
+                              const int32_t* perm, const int32_t* active, const int32_t* n_active, uint16_t* h,
+                              uint16_t* h_s, cudaStream_t s);
+cudaError_t launch_mid_down(const Geometry& g, const LayerPtr& L, const uint16_t* h, const uint16_t* h_s,
+                            const int32_t* offsets, const int32_t* active, const int32_t* n_active, uint16_t* Y,
+                            cudaStream_t s);
 
 // decode_fused.cu: a stack of 1..decode_fused_max_layers() decode layers
 // (T <= 8, H = 1024 or 2048) in one cooperative launch; layer l > 0 takes

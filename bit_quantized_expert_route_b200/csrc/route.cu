@@ -183,13 +183,17 @@ __global__ void __launch_bounds__(32 * kSegWarps) scatter_kernel(
 
 // ---------------------------------------------------------------------------
 // Small-T routing (T <= 64): one launch does the router GEMV, top-k, shared
-// gate and the whole counting sort.  Warp w of CTA b scores row e = 8b + w
-// (e == E: the shared-gate vector) for every token, so the 1 MB router matrix
-// is streamed by ~33 CTAs at once.  The last CTA to finish (a counter in the
-// workspace, reset by that CTA) selects the experts, sorts the T*k entries
-// stably by expert and builds the active-expert list.
+// gate and the whole counting sort.  CTA (b, y) scores rows e = 8b + w (warp
+// w; e == E: the shared-gate vector) for the TB tokens of token group y, so
+// the 1 MB router matrix is streamed by ~33 CTAs per group, all groups at
+// once.  The last CTA of a token group to finish (a counter per group in the
+// workspace's control block) selects the experts of the group's tokens, one
+// token per warp; the last group to finish (one more counter) sorts the T*k
+// entries stably by expert and builds the active-expert list.  Each counter
+// is reset by the CTA that saw it complete.
 // ---------------------------------------------------------------------------
 constexpr int kSmallWarps = 8;
+constexpr int kSmallLoads = 8;          // loads per thread in flight together
 
 template <int TB>
 __global__ void __launch_bounds__(256) router_small_kernel(
@@ -207,34 +211,52 @@ __global__ void __launch_bounds__(256) router_small_kernel(
   const int e = blockIdx.x * kSmallWarps + warp;
   const bool live = e <= E;
   const uint4* wrow = reinterpret_cast<const uint4*>(e < E ? L.w_router + static_cast<size_t>(e) * H : L.w_sg);
+  const int t0 = blockIdx.y * TB;
+  const int nt = min(TB, T - t0);
 
   uint4* xs = smem_u4;   // [TB][vec]
-  for (int t0 = 0; t0 < T; t0 += TB) {
-    const int nt = min(TB, T - t0);
-    __syncthreads();
-    for (int i = threadIdx.x; i < TB * vec; i += blockDim.x) {
+  for (int i0 = threadIdx.x; i0 < TB * vec; i0 += blockDim.x * kSmallLoads) {
+    uint4 v[kSmallLoads];   // all loads in flight before the first store
+#pragma unroll
+    for (int j = 0; j < kSmallLoads; ++j) {
+      const int i = i0 + j * blockDim.x;
       const int r = i / vec, c = i - r * vec;
-      xs[i] = r < nt ? reinterpret_cast<const uint4*>(x + static_cast<size_t>(t0 + r) * H)[c]
-                     : make_uint4(0u, 0u, 0u, 0u);
+      v[j] = (i < TB * vec && r < nt) ? reinterpret_cast<const uint4*>(x + static_cast<size_t>(t0 + r) * H)[c]
+                                      : make_uint4(0u, 0u, 0u, 0u);
     }
-    __syncthreads();
-    if (!live) continue;
+#pragma unroll
+    for (int j = 0; j < kSmallLoads; ++j)
+      if (i0 + j * blockDim.x < TB * vec) xs[i0 + j * blockDim.x] = v[j];
+  }
+  __syncthreads();
+  if (live) {
     float acc[TB];
 #pragma unroll
     for (int r = 0; r < TB; ++r) acc[r] = 0.f;
-    for (int c = lane; c < vec; c += 32) {
-      const uint4 wv = __ldg(wrow + c);
-      const float w0 = bf16_lo(wv.x), w1 = bf16_hi(wv.x), w2 = bf16_lo(wv.y), w3 = bf16_hi(wv.y);
-      const float w4 = bf16_lo(wv.z), w5 = bf16_hi(wv.z), w6 = bf16_lo(wv.w), w7 = bf16_hi(wv.w);
+    for (int c0 = lane; c0 < vec; c0 += 32 * kSmallLoads) {
+      uint4 wv[kSmallLoads];
 #pragma unroll
-      for (int r = 0; r < TB; ++r) {
-        const uint4 xv = xs[r * vec + c];
-        float a = acc[r];
-        a = fmaf(bf16_lo(xv.x), w0, a); a = fmaf(bf16_hi(xv.x), w1, a);
-        a = fmaf(bf16_lo(xv.y), w2, a); a = fmaf(bf16_hi(xv.y), w3, a);
-        a = fmaf(bf16_lo(xv.z), w4, a); a = fmaf(bf16_hi(xv.z), w5, a);
-        a = fmaf(bf16_lo(xv.w), w6, a); a = fmaf(bf16_hi(xv.w), w7, a);
-        acc[r] = a;
+      for (int u = 0; u < kSmallLoads; ++u) {
+        const int c = c0 + 32 * u;
+        wv[u] = c < vec ? __ldg(wrow + c) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < kSmallLoads; ++u) {
+        const int c = c0 + 32 * u;
+        if (c < vec) {
+          const float w0 = bf16_lo(wv[u].x), w1 = bf16_hi(wv[u].x), w2 = bf16_lo(wv[u].y), w3 = bf16_hi(wv[u].y);
+          const float w4 = bf16_lo(wv[u].z), w5 = bf16_hi(wv[u].z), w6 = bf16_lo(wv[u].w), w7 = bf16_hi(wv[u].w);
+#pragma unroll
+          for (int r = 0; r < TB; ++r) {
+            const uint4 xv = xs[r * vec + c];
+            float a = acc[r];
+            a = fmaf(bf16_lo(xv.x), w0, a); a = fmaf(bf16_hi(xv.x), w1, a);
+            a = fmaf(bf16_lo(xv.y), w2, a); a = fmaf(bf16_hi(xv.y), w3, a);
+            a = fmaf(bf16_lo(xv.z), w4, a); a = fmaf(bf16_hi(xv.z), w5, a);
+            a = fmaf(bf16_lo(xv.w), w6, a); a = fmaf(bf16_hi(xv.w), w7, a);
+            acc[r] = a;
+          }
+        }
       }
     }
     const float b = (e < E && L.router_bias) ? L.router_bias[e] : 0.f;
@@ -245,31 +267,52 @@ __global__ void __launch_bounds__(256) router_small_kernel(
     }
   }
 
-  // ---- the last CTA to finish does selection and grouping ----
+  // ---- the last CTA of this token group selects its tokens' experts ----
+  unsigned* group_counter = counter + kSmallGroupCounter + blockIdx.y;
   __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) s_last = (atomicAdd(counter, 1u) == gridDim.x - 1) ? 1 : 0;
+  if (threadIdx.x == 0) s_last = (atomicAdd(group_counter, 1u) == gridDim.x - 1) ? 1 : 0;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  if (threadIdx.x == 0) *group_counter = 0u;
+  float* lg = reinterpret_cast<float*>(smem_u4);   // [TB][E1], reuses the x tile
+  for (int i0 = threadIdx.x; i0 < nt * E1; i0 += blockDim.x * kSmallLoads) {
+    float v[kSmallLoads];
+#pragma unroll
+    for (int j = 0; j < kSmallLoads; ++j) {
+      const int i = i0 + j * blockDim.x;
+      v[j] = i < nt * E1 ? __ldcg(logits + static_cast<size_t>(t0) * E1 + i) : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < kSmallLoads; ++j)
+      if (i0 + j * blockDim.x < nt * E1) lg[i0 + j * blockDim.x] = v[j];
+  }
+  __syncthreads();
+  for (int r = warp; r < nt; r += kSmallWarps) {
+    const int t = t0 + r;
+    select_topk_warp(lg + r * E1, E, k, lane, topk_idx + t * k, topk_w + t * k);
+    if (lane == 0) sigma[t] = sigmoid(lg[r * E1 + E]);
+  }
+
+  // ---- the last token group to finish groups the T*k entries ----
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = (atomicAdd(counter, 1u) == gridDim.y - 1) ? 1 : 0;
   __syncthreads();
   if (!s_last) return;
   __threadfence();
   if (threadIdx.x == 0) *counter = 0u;
 
-  float* lg = reinterpret_cast<float*>(smem_u4);   // [T][E1], reuses the x tile
-  for (int i = threadIdx.x; i < T * E1; i += blockDim.x) lg[i] = __ldcg(logits + i);
-  __syncthreads();
-  for (int t = warp; t < T; t += kSmallWarps) {
-    select_topk_warp(lg + t * E1, E, k, lane, topk_idx + t * k, topk_w + t * k);
-    if (lane == 0) sigma[t] = sigmoid(lg[t * E1 + E]);
-  }
-  __syncthreads();
-
   // histogram, exclusive scan and stable scatter of the n = T*k entries
-  int* hist = reinterpret_cast<int*>(smem_u4);       // [256] (logits no longer needed)
+  int* hist = reinterpret_cast<int*>(smem_u4);       // [256]
   int* cursor = hist + 256;                          // [256]
+  int* sel = cursor + 256;                           // [T*k] the selected experts
   const int n = T * k;
   hist[threadIdx.x] = 0;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) sel[i] = __ldcg(topk_idx + i);
   __syncthreads();
-  for (int i = threadIdx.x; i < n; i += blockDim.x) atomicAdd(&hist[topk_idx[i]], 1);
+  for (int i = threadIdx.x; i < n; i += blockDim.x) atomicAdd(&hist[sel[i]], 1);
   __syncthreads();
   const int c = threadIdx.x < E ? hist[threadIdx.x] : 0;
   int off = 0;
@@ -291,7 +334,7 @@ __global__ void __launch_bounds__(256) router_small_kernel(
   if (warp == 0) {
     for (int base = 0; base < n; base += 32) {
       const int i = base + lane;
-      const int ex = i < n ? topk_idx[i] : -1;
+      const int ex = i < n ? sel[i] : -1;
       const unsigned peers = __match_any_sync(0xffffffffu, ex);
       const int rank = __popc(peers & lanemask_lt());
       const int start = ex >= 0 ? cursor[ex] : 0;
@@ -315,8 +358,8 @@ template <int TB>
 static cudaError_t launch_small_tb(const uint16_t* x, const LayerPtr& L, int T, int H, int I, int Is, int E, int k,
                                    float* logits, unsigned* counter, const RoutingPtrs& r, int32_t* active,
                                    int32_t* n_active, cudaStream_t s) {
-  const int grid = (E + 1 + kSmallWarps - 1) / kSmallWarps;
-  const int smem = max(TB * H * 2, max(T * (E + 1) * 4, 2048));
+  const dim3 grid((E + 1 + kSmallWarps - 1) / kSmallWarps, (T + TB - 1) / TB);
+  const int smem = max(TB * H * 2, max(TB * (E + 1) * 4, (512 + T * k) * 4));
   const cudaError_t e = ensure_smem(reinterpret_cast<const void*>(router_small_kernel<TB>), smem);
   if (e != cudaSuccess) return e;
   router_small_kernel<TB><<<grid, 256, smem, s>>>(x, L, T, H, I, Is, E, k, logits, counter, r.topk_idx, r.topk_w,
@@ -328,11 +371,13 @@ static cudaError_t launch_small_tb(const uint16_t* x, const LayerPtr& L, int T, 
 cudaError_t launch_route_small(const uint16_t* x, const LayerPtr& L, int T, int H, int I, int Is, int E, int k,
                                float* logits, unsigned* counter, const RoutingPtrs& r, int32_t* active,
                                int32_t* n_active, cudaStream_t s) {
-  // tokens per pass over the router matrix: x tile of TB rows (bf16) in smem
+  // tokens per CTA: x tile of TB rows (bf16) in smem; at most
+  // kSmallMaxGroups token groups (one counter each)
+  if (T > kSmallTB * kSmallMaxGroups) return cudaErrorInvalidValue;
   if (T == 1) return launch_small_tb<1>(x, L, T, H, I, Is, E, k, logits, counter, r, active, n_active, s);
   if (T <= 2) return launch_small_tb<2>(x, L, T, H, I, Is, E, k, logits, counter, r, active, n_active, s);
-  if (T <= 4 || H > 4096) return launch_small_tb<4>(x, L, T, H, I, Is, E, k, logits, counter, r, active, n_active, s);
-  return launch_small_tb<8>(x, L, T, H, I, Is, E, k, logits, counter, r, active, n_active, s);
+  if (T <= 4) return launch_small_tb<4>(x, L, T, H, I, Is, E, k, logits, counter, r, active, n_active, s);
+  return launch_small_tb<kSmallTB>(x, L, T, H, I, Is, E, k, logits, counter, r, active, n_active, s);
 }
 
 cudaError_t launch_group(const int32_t* topk_idx, int T, int k, int E, int chunk_rows,

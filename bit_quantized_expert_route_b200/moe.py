@@ -264,7 +264,7 @@ def moe_rmsnorm(y: torch.Tensor, y_out: torch.Tensor, eps: float = 1e-6, stream=
 
 
 PREFILL_STAGES = ("router", "group", "gather", "gateup", "down", "combine")
-DECODE_STAGES = ("route", "gateup", "down_combine")
+MID_DECODE_STAGES = ("route", "gateup", "down", "combine")
 FUSED_DECODE_STAGES = ("decode_fused",)
 
 
@@ -277,7 +277,7 @@ def moe_forward_profiled(layer: MoELayer, x: torch.Tensor, out: torch.Tensor, wo
     _check(library().moe_forward_profiled(ctypes.byref(layer.desc), x.data_ptr(), T, out.data_ptr(),
                                           workspace.data_ptr(), workspace.numel(), _stream(stream), ms,
                                           ctypes.byref(n)), "moe_forward_profiled")
-    names = {1: FUSED_DECODE_STAGES, len(DECODE_STAGES): DECODE_STAGES, len(PREFILL_STAGES): PREFILL_STAGES}[n.value]
+    names = {1: FUSED_DECODE_STAGES, len(MID_DECODE_STAGES): MID_DECODE_STAGES, len(PREFILL_STAGES): PREFILL_STAGES}[n.value]
     return {names[i]: float(ms[i]) for i in range(n.value)}
 
 

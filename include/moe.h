@@ -180,23 +180,27 @@ MOE_API int moe_route(const moe_layer_desc* layer, const moe_bf16* x, int T, moe
  * bf16 products and FP32 accumulation, and one always-on shared expert.
  * x, out: device bf16 [T, H], 16-byte aligned, not overlapping.
  * r: optional (NULL = keep routing in the workspace).
- * 1 <= T <= 65536.  For T <= 8 with H = 1024 or 2048, I and I_shared whole
- * groups, 16-byte aligned scale and bias stacks and at most E + 1 SMs it
- * runs moe_decode's single-launch fused kernel; for every other T, the
- * tensor-core kernels above (the three-launch decode kernels spend work on
- * every weight for every token, which the grouped GEMMs outrun as soon as an
- * expert sees a few tokens). */
+ * 1 <= T <= 65536.  Three kernel sets, chosen by T:
+ *   T <= 8 with H = 1024 or 2048, I and I_shared whole groups, 16-byte
+ *     aligned scale and bias stacks and at most E + 1 SMs: the single-launch
+ *     fused decode kernel (see moe_decode);
+ *   T <= 64 with H, I and I_shared multiples of 256 and 8-byte aligned scale
+ *     and bias stacks (the mid-size decode path): the one-launch small-T
+ *     router, then gate/up + SwiGLU and down as GEMVs over the active experts
+ *     only (warp-level mma.sync on 8-token tiles, codes streamed from global
+ *     memory into the operand registers), then the fixed-order combine;
+ *   every other T: the tensor-core (tcgen05) kernels above. */
 MOE_API int moe_forward(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_bf16* out,
                 moe_routing* r, void* workspace, size_t workspace_bytes, moe_stream stream);
 
-/* The same function for 1 <= T <= 64 through the bandwidth-bound decode
- * kernels (batch-1 decoding streams the active experts' weights: "How It
- * Works: Prefill and Decode Strategies").  T > 64 is MOE_ERR_INVALID_ARG.
- * Under the same conditions as moe_forward's fused path (T <= 8, ...) the
- * whole layer is ONE cooperative launch of one CTA per SM whose CTAs exchange
- * the router logits, the SwiGLU activations and the outputs through tagged
- * workspace words (no grid-wide barrier); otherwise three launches (routing,
- * gate/up, down + combine). */
+/* The same function for 1 <= T <= 64 (batch decoding streams the active
+ * experts' weights: "How It Works: Prefill and Decode Strategies"); it runs
+ * what moe_forward runs for T.  T > 64 is MOE_ERR_INVALID_ARG.  Under the
+ * fused conditions above the whole layer is ONE cooperative launch of one CTA
+ * per SM whose CTAs exchange the router logits, the SwiGLU activations and
+ * the outputs through tagged workspace words (no grid-wide barrier);
+ * otherwise the mid-size decode path's four launches (routing, gate/up, down,
+ * combine), or the tensor-core kernels where that path does not apply. */
 MOE_API int moe_decode(const moe_layer_desc* layer, const moe_bf16* x, int T, moe_bf16* out,
                moe_routing* r, void* workspace, size_t workspace_bytes, moe_stream stream);
 
@@ -208,10 +212,10 @@ MOE_API int moe_decode(const moe_layer_desc* layer, const moe_bf16* x, int T, mo
  *   a_0 = x;  y_l = layer_l(a_l);  a_{l+1} = bf16(y_l / sqrt(mean(y_l^2) + eps))
  * (RMSNorm with weight 1 and no residual, over the bf16 values of y_l);
  * out = y_{n_layers-1}.  Each layer runs what moe_forward runs for T.  On the
- * tensor-core path the RMSNorm is computed inside the layer's combine kernel
- * (the row's sum of squares is formed while its output is written).  On the
- * fused decode path up to 40 layers run in ONE launch, the RMSNorm between
- * them inside it (each CTA publishes the sum of squares of its outputs);
+ * tensor-core and mid-size paths the RMSNorm is computed inside the layer's
+ * combine kernel (the row's sum of squares is formed while its output is
+ * written).  On the fused decode path up to 40 layers run in ONE launch,
+ * the RMSNorm between them inside it (each CTA publishes the sum of squares of its outputs);
  * longer stacks are cut into launches of 40 layers joined by a small
  * RMSNorm kernel.
  *   layers: host array of n_layers (1..1024) descriptors with equal H, I,
@@ -287,6 +291,7 @@ MOE_API int moe_rmsnorm(const moe_bf16* y, moe_bf16* y_out, int T, int H, float 
  * writes each stage's device time in milliseconds to stage_ms[0..n-1]:
  *   tensor-core path: router, group (histogram+scan+scatter), gather of the
  *            grouped token rows, gate/up GEMM, down GEMM, combine (6 stages)
+ *   mid-size decode path: routing, gate/up, down, combine (4 stages)
  *   fused decode kernel (when moe_forward uses it): one stage
  * stage_ms: host array of at least 6 floats; *n_stages receives the count.
  * The events are created and destroyed inside the call. */

@@ -166,7 +166,7 @@ def test_decode_entry_rejects_large_T():
 
 @pytest.mark.parametrize("dims,T", [(TINY, 40), (FULL, 12)])
 def test_decode_entry_and_forward_both_match_oracle(dims, T):
-    # moe_decode runs the GEMV kernels; moe_forward runs the tensor-core path at these T
+    # both entries run the mid-size decode path (mma.sync GEMVs over the active experts) at these T
     lay, x, _ = workload(8, T, dims)
     L = moe.MoELayer.from_synth(lay)
     ref = moe_ref.moe_layer(x, lay, dims.k)
@@ -197,12 +197,12 @@ def test_rmsnorm_matches_oracle():
 # ------------------------------------------------------------- full layer --
 
 @pytest.mark.parametrize("T,entry", [(1, "forward"), (2, "forward"), (3, "forward"), (5, "forward"),
-                                     (8, "forward"), (9, "forward"), (64, "forward"),
-                                     (3, "decode"), (8, "decode"), (9, "decode"), (64, "decode")])
+                                     (8, "forward"), (9, "forward"), (16, "forward"), (33, "forward"),
+                                     (64, "forward"), (3, "decode"), (8, "decode"), (9, "decode"), (64, "decode")])
 def test_full_decode(T, entry):
-    # T <= 8 runs the single-launch fused decode kernel (both entries); larger
-    # T runs the tensor-core path through moe_forward and the GEMV kernels
-    # through moe_decode
+    # T <= 8 runs the single-launch fused decode kernel (both entries); 9 <= T
+    # <= 64 the mid-size decode path (small-T router, mma.sync GEMVs over the
+    # active experts in 8-token tiles, fixed-order combine)
     lay, x, _ = workload(10 + T, T, FULL)
     ref = moe_ref.moe_layer(x, lay, FULL.k)
     gpu = run_layer(lay, x, entry=entry)
@@ -211,11 +211,14 @@ def test_full_decode(T, entry):
     assert_output_close(gpu["out"], ref["out"])
 
 
-@pytest.mark.parametrize("T", [1, 2, 8])
+@pytest.mark.parametrize("T", [1, 2, 8, 24, 64])
 def test_full_decode_zipf(T):
+    # at T = 24 and 64 the hot experts see more than 8 tokens: several token tiles per expert
     lay, x, _ = workload(30 + T, T, FULL, zipf=True)
     ref = moe_ref.moe_layer(x, lay, FULL.k)
     gpu = run_layer(lay, x, entry="decode")
+    if T > 8:
+        assert int(np.max(ref["counts"])) > 8
     assert gpu["status"] == 0
     assert_routing_exact(gpu, ref)
     assert_output_close(gpu["out"], ref["out"])
