@@ -231,11 +231,30 @@ __device__ __forceinline__ void group_step(float (&y)[2][2][2], const uint2 (&a)
   }
 }
 
-// The body both kernels share.  tile_of(item, warp, lg4, lt) -> WTile: the
-// warp's two tiles; k_of(item): inputs per row (a multiple of 256);
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+// A position in the CTA's sequence of weight blocks (4 groups of its items'
+// tiles, item after item): item k (index blockIdx.x + k gridDim.x), block b.
+struct Cursor {
+  int k, b, nbat;
+  bool valid;
+};
+
+// The body both kernels share.  tile_of(item, warp, row, lt) -> WTile: the
+// warp's two tiles as seen by a lane that reads row `row` (and row + 8) at
+// byte 8 lt of each group; k_of(item): inputs per row (a multiple of 256);
 // row_of(item) -> a function r -> activation row r of the token tile;
 // store(item, warp, y, lg4, lt): the epilogue.  Shared memory: the staged
 // token tile.
+//
+// Three walks over the same block sequence: the computation; the register
+// loads one block ahead of it (group j of block n + 1 right after group j of
+// block n has been used); and L2 prefetches kPrefetchBlocks ahead, one
+// 128-byte line per lane and block (lane = tile * 16 + row), so the register
+// loads find their lines in L2.
+constexpr int kPrefetchBlocks = 4;
 template <class TileOf, class KOf, class RowOf, class Store>
 __device__ __forceinline__ void mid_body(const Geometry& g, const int32_t* offsets, const int32_t* active,
                                          const int32_t* n_active, int blocks_routed, int blocks_shared, int kmax,
@@ -249,52 +268,84 @@ __device__ __forceinline__ void mid_body(const Geometry& g, const int32_t* offse
   uint4* xs = reinterpret_cast<uint4*>(msm);
   float* xsum = reinterpret_cast<float*>(xs + kMTok * (kmax / 8 + 1));
 
-  Item I = decode_item(g, s_start, n_act, offsets, active, blockIdx.x);
-  WTile cur = tile_of(I, warp, lg4, lt);
-  int ngr = k_of(I) / kGroup;
+  // open item k of a cursor (false past the CTA's last item)
+  auto open = [&](int k, Item& I) -> bool {
+    const int it = blockIdx.x + k * gridDim.x;
+    if (it >= total) return false;
+    I = decode_item(g, s_start, n_act, offsets, active, it);
+    return true;
+  };
+  // the load walk: this lane's operand pointers for the cursor's item
+  Cursor lc{0, 0, 0, true};
+  WTile lw;
+  int lngr;
+  auto load_open = [&](const Item& I) {
+    lw = tile_of(I, warp, lg4, lt);
+    lngr = k_of(I) / kGroup;
+    lc.nbat = lngr / kMBlock;
+  };
+  // the prefetch walk: the line of row (lane % 16) of tile (lane / 16)
+  Cursor pc{0, 0, 0, true};
+  const uint8_t* pq;
+  auto pf_open = [&](const Item& I) {
+    const WTile w = tile_of(I, warp, lane & 15, 0);
+    pq = w.q[lane >> 4];
+    pc.nbat = k_of(I) / kGroup / kMBlock;
+  };
+  auto advance = [&](Cursor& c, bool is_load) {
+    if (!c.valid) return;
+    if (++c.b < c.nbat) return;
+    c.b = 0;
+    Item N;
+    c.valid = open(++c.k, N);
+    if (c.valid) {
+      if (is_load) load_open(N);
+      else pf_open(N);
+    }
+  };
+
+  Item I;
+  open(0, I);
+  load_open(I);
+  pf_open(I);
   uint2 A[kMBlock][2][2];
   BlockS S;
 #pragma unroll
-  for (int j = 0; j < kMBlock; ++j) load_group(A[j], cur, ngr, j);
-  load_scales(S, cur, ngr, 0);
+  for (int j = 0; j < kMBlock; ++j) load_group(A[j], lw, lngr, j);
+  load_scales(S, lw, lngr, 0);
+  advance(lc, true);
+  for (int i = 0; i < kPrefetchBlocks; ++i) {
+    advance(pc, false);
+    if (pc.valid) prefetch_l2(pq + pc.b * 128);
+  }
+
   for (int k = 0;; ++k) {
     const int K = k_of(I);
+    const int ngr = K / kGroup, nbat = ngr / kMBlock;
     if (k > 0) __syncthreads();   // every warp is done with the previous item's staged tile
     stage_tile(row_of(I), I.tn, K, xs, xsum);
     __syncthreads();
-    const int nit = blockIdx.x + (k + 1) * gridDim.x;
-    const bool has_next = nit < total;
-    Item NI = I;
-    WTile nxt = cur;
-    int nngr = ngr;
-    if (has_next) {
-      NI = decode_item(g, s_start, n_act, offsets, active, nit);
-      nxt = tile_of(NI, warp, lg4, lt);
-      nngr = k_of(NI) / kGroup;
-    }
     float y[2][2][2] = {{{0.f, 0.f}, {0.f, 0.f}}, {{0.f, 0.f}, {0.f, 0.f}}};
     const uint4* xr = xs + lg4 * (K / 8 + 1) + lt * 2;
-    const int nbat = ngr / kMBlock;
     for (int b = 0; b < nbat; ++b) {
-      const bool last = b + 1 == nbat;
-      const bool nvalid = !last || has_next;       // a next block to prefetch
-      const WTile& nw = last ? nxt : cur;
-      const int nG0 = last ? 0 : (b + 1) * kMBlock;
-      const int ng = last ? nngr : ngr;
+      advance(pc, false);
+      if (pc.valid) prefetch_l2(pq + pc.b * 128);
+      const bool lv = lc.valid;
+      const int lG0 = lc.b * kMBlock;
       BlockS NS = S;
-      if (nvalid) load_scales(NS, nw, ng, nG0);
+      if (lv) load_scales(NS, lw, lngr, lG0);
 #pragma unroll
       for (int j = 0; j < kMBlock; ++j) {
         group_step(y, A[j], S, j, xr, xsum, b * kMBlock + j, lt);
-        if (nvalid) load_group(A[j], nw, ng, nG0 + j);
+        if (lv) load_group(A[j], lw, lngr, lG0 + j);
       }
       S = NS;
+      advance(lc, true);
     }
     store(I, warp, y, lg4, lt);
-    if (!has_next) break;
-    I = NI;
-    cur = nxt;
-    ngr = nngr;
+    Item N;
+    if (!open(k + 1, N)) break;
+    I = N;
   }
 }
 

@@ -163,75 +163,6 @@ __device__ __forceinline__ void tile_groups(float (&y)[2][2], const uint8_t* qro
 }
 
 
-// Order-preserving 32-bit key of a float (larger float -> larger key; every
-// non-NaN float maps above 0).
-__device__ __forceinline__ uint32_t order_key(float f) {
-  const uint32_t u = f == 0.f ? 0u : __float_as_uint(f);   // -0 and +0 are one value
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-// Warp top-k over E <= 256 logits in shared memory with the same order as
-// the other routing kernels (larger logit first, equal logits -> lower expert
-// index).  Lane i holds the keys of experts i, i + 32, ..., sorted once by a
-// 19-comparator network on (key, expert) pairs, so its best candidate is
-// always its head.  A pick is one redux.sync max over the heads and one min
-// over the experts of the lanes holding that key; the winning lane pops its
-// head.  Lanes j < k then form exp(l_j - l_0) in parallel and divide by their
-// sum (a fixed shuffle tree).
-__device__ __forceinline__ bool key_before(uint32_t ka, int ia, uint32_t kb, int ib) {
-  return ka > kb || (ka == kb && ia < ib);
-}
-__device__ __forceinline__ void cas(uint32_t (&key)[8], int (&ix)[8], int i, int j) {
-  const bool keep = key_before(key[i], ix[i], key[j], ix[j]);
-  const uint32_t ki = keep ? key[i] : key[j], kj = keep ? key[j] : key[i];
-  const int ii = keep ? ix[i] : ix[j], ij = keep ? ix[j] : ix[i];
-  key[i] = ki;
-  key[j] = kj;
-  ix[i] = ii;
-  ix[j] = ij;
-}
-__device__ __forceinline__ void topk_redux(const float* lg, int E, int k, int lane, int32_t* idx_out,
-                                           float* w_out) {
-  uint32_t key[8];
-  int ix[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    ix[i] = lane + 32 * i;
-    key[i] = ix[i] < E ? order_key(lg[ix[i]]) : 0u;
-  }
-  cas(key, ix, 0, 1); cas(key, ix, 2, 3); cas(key, ix, 4, 5); cas(key, ix, 6, 7);
-  cas(key, ix, 0, 2); cas(key, ix, 1, 3); cas(key, ix, 4, 6); cas(key, ix, 5, 7);
-  cas(key, ix, 1, 2); cas(key, ix, 5, 6);
-  cas(key, ix, 0, 4); cas(key, ix, 1, 5); cas(key, ix, 2, 6); cas(key, ix, 3, 7);
-  cas(key, ix, 2, 4); cas(key, ix, 3, 5);
-  cas(key, ix, 1, 2); cas(key, ix, 3, 4); cas(key, ix, 5, 6);
-  int mine = 0, first = 0;
-#pragma unroll
-  for (int j = 0; j < kMaxK; ++j) {
-    if (j < k) {
-      const uint32_t m = __reduce_max_sync(0xffffffffu, key[0]);
-      const uint32_t win = __reduce_min_sync(0xffffffffu, key[0] == m ? static_cast<uint32_t>(ix[0]) : 0xffffffffu);
-      if (static_cast<uint32_t>(ix[0]) == win) {   // pop the head
-#pragma unroll
-        for (int i = 0; i < 7; ++i) {
-          key[i] = key[i + 1];
-          ix[i] = ix[i + 1];
-        }
-        key[7] = 0u;
-        ix[7] = 0x7fffffff;
-      }
-      if (lane == j) mine = static_cast<int>(win);
-      if (j == 0) first = static_cast<int>(win);
-    }
-  }
-  const float z = lane < k ? expf(lg[mine] - lg[first]) : 0.f;
-  const float sum = warp_sum(z);
-  if (lane < k) {
-    idx_out[lane] = mine;
-    w_out[lane] = z / sum;
-  }
-}
-
 __device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kFWarps * 32) : "memory"); }
 
 // Exchanges between CTAs carry their own readiness: every value travels in a

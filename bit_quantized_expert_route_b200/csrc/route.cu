@@ -291,7 +291,7 @@ __global__ void __launch_bounds__(256) router_small_kernel(
   __syncthreads();
   for (int r = warp; r < nt; r += kSmallWarps) {
     const int t = t0 + r;
-    select_topk_warp(lg + r * E1, E, k, lane, topk_idx + t * k, topk_w + t * k);
+    topk_redux(lg + r * E1, E, k, lane, topk_idx + t * k, topk_w + t * k);
     if (lane == 0) sigma[t] = sigmoid(lg[r * E1 + E]);
   }
 
@@ -304,48 +304,63 @@ __global__ void __launch_bounds__(256) router_small_kernel(
   __threadfence();
   if (threadIdx.x == 0) *counter = 0u;
 
-  // histogram, exclusive scan and stable scatter of the n = T*k entries
-  int* hist = reinterpret_cast<int*>(smem_u4);       // [256]
-  int* cursor = hist + 256;                          // [256]
-  int* sel = cursor + 256;                           // [T*k] the selected experts
+  // Stable counting sort of the n = T*k entries by expert.  Warp w owns the
+  // entries [w*chunk, (w+1)*chunk): it counts them per expert (wcnt[w][e]),
+  // one exclusive scan over the experts gives the offsets (and, packed in the
+  // high half, the active-list positions), each expert's per-warp bases
+  // follow in warp order, and every warp scatters its entries in order.
+  int* wcnt = reinterpret_cast<int*>(smem_u4);       // [kSmallWarps][256]
+  int* sel = wcnt + kSmallWarps * 256;               // [T*k] the selected experts
   const int n = T * k;
-  hist[threadIdx.x] = 0;
+  const int chunk = (n + kSmallWarps - 1) / kSmallWarps;
+  for (int i = threadIdx.x; i < kSmallWarps * 256; i += blockDim.x) wcnt[i] = 0;
   for (int i = threadIdx.x; i < n; i += blockDim.x) sel[i] = __ldcg(topk_idx + i);
   __syncthreads();
-  for (int i = threadIdx.x; i < n; i += blockDim.x) atomicAdd(&hist[sel[i]], 1);
+  const int lo = warp * chunk, hi = min(n, lo + chunk);
+  for (int base = lo; base < hi; base += 32) {
+    const int i = base + lane;
+    const int ex = i < hi ? sel[i] : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, ex);
+    if (ex >= 0 && (peers >> lane) == 1u) wcnt[warp * 256 + ex] += __popc(peers);   // one writer per expert
+    __syncwarp();
+  }
   __syncthreads();
-  const int c = threadIdx.x < E ? hist[threadIdx.x] : 0;
-  int off = 0;
-  const int total = block_exclusive_scan(c, s_scan, &off);
+  int c = 0;
+  if (threadIdx.x < E)
+    for (int w = 0; w < kSmallWarps; ++w) c += wcnt[w * 256 + threadIdx.x];
+  int excl = 0;   // low 16 bits: entries before this expert; high 16 bits: active experts before it
+  const int tot = block_exclusive_scan(c + ((c > 0) << 16), s_scan, &excl);
+  const int off = excl & 0xFFFF, apos = excl >> 16, nact = tot >> 16;
   if (threadIdx.x < E) {
     counts[threadIdx.x] = c;
     offsets[threadIdx.x] = off;
-    cursor[threadIdx.x] = off;
+    if (c > 0) active[apos] = threadIdx.x;
+    int run = off;
+    for (int w = 0; w < kSmallWarps; ++w) {
+      const int t = wcnt[w * 256 + threadIdx.x];
+      wcnt[w * 256 + threadIdx.x] = run;
+      run += t;
+    }
   }
-  if (threadIdx.x == 0) offsets[E] = total;
-  int apos = 0;
-  const int nact = block_exclusive_scan((threadIdx.x < E && c > 0) ? 1 : 0, s_scan, &apos);
-  if (threadIdx.x < E && c > 0) active[apos] = threadIdx.x;
   if (threadIdx.x == 0) {
+    offsets[E] = tot & 0xFFFF;
     active[nact] = E;
     *n_active = nact + 1;
   }
   __syncthreads();
-  if (warp == 0) {
-    for (int base = 0; base < n; base += 32) {
-      const int i = base + lane;
-      const int ex = i < n ? sel[i] : -1;
-      const unsigned peers = __match_any_sync(0xffffffffu, ex);
-      const int rank = __popc(peers & lanemask_lt());
-      const int start = ex >= 0 ? cursor[ex] : 0;
-      __syncwarp();
-      if (ex >= 0) {
-        perm[start + rank] = i;
-        inv_perm[i] = start + rank;
-        if ((peers >> lane) == 1u) cursor[ex] = start + __popc(peers);
-      }
-      __syncwarp();
+  for (int base = lo; base < hi; base += 32) {
+    const int i = base + lane;
+    const int ex = i < hi ? sel[i] : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, ex);
+    const int rank = __popc(peers & lanemask_lt());
+    const int start = ex >= 0 ? wcnt[warp * 256 + ex] : 0;
+    __syncwarp();
+    if (ex >= 0) {
+      perm[start + rank] = i;
+      inv_perm[i] = start + rank;
+      if ((peers >> lane) == 1u) wcnt[warp * 256 + ex] = start + __popc(peers);
     }
+    __syncwarp();
   }
 }
 
@@ -359,7 +374,7 @@ static cudaError_t launch_small_tb(const uint16_t* x, const LayerPtr& L, int T, 
                                    float* logits, unsigned* counter, const RoutingPtrs& r, int32_t* active,
                                    int32_t* n_active, cudaStream_t s) {
   const dim3 grid((E + 1 + kSmallWarps - 1) / kSmallWarps, (T + TB - 1) / TB);
-  const int smem = max(TB * H * 2, max(TB * (E + 1) * 4, (512 + T * k) * 4));
+  const int smem = max(TB * H * 2, max(TB * (E + 1) * 4, (kSmallWarps * 256 + T * k) * 4));
   const cudaError_t e = ensure_smem(reinterpret_cast<const void*>(router_small_kernel<TB>), smem);
   if (e != cudaSuccess) return e;
   router_small_kernel<TB><<<grid, 256, smem, s>>>(x, L, T, H, I, Is, E, k, logits, counter, r.topk_idx, r.topk_w,
