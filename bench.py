@@ -95,6 +95,10 @@ def parse_args(argv=None):
     ap.add_argument("--sweep-reps", type=int, default=3, help="timed stack calls per sweep point")
     ap.add_argument("--oracle-sweep-T", type=str, default=",".join(str(t) for t in SWEEP_T),
                     help="sweep points at which the CPU oracle is timed (layer 0)")
+    ap.add_argument("--probe-T", type=int, default=0,
+                    help="profiling probe: only `--probe-calls` moe_forward calls of T tokens on two resident "
+                         "layers (~0.9 GB), no timing, no JSON line")
+    ap.add_argument("--probe-calls", type=int, default=4)
     return ap.parse_args(argv)
 
 
@@ -858,8 +862,29 @@ def run_reference(a):
     print(json.dumps(line), flush=True)
 
 
+def run_probe(a):
+    """A small, fixed sequence of layer calls for ncu captures (one GPU)."""
+    import torch
+    from bit_quantized_expert_route_b200 import moe, synth
+    dev = torch.device("cuda", 0)
+    dims = synth.Dims()
+    layers = [moe.MoELayer.from_tensors(dims, synth.make_layer_on_device(300 + l, l, dims, dev, False))
+              for l in range(2)]
+    x = synth.make_x_on_device(7, a.probe_T, dims.H, dev)
+    out = torch.empty_like(x)
+    ws = moe.alloc_workspace(layers[0], a.probe_T, dev)
+    for i in range(a.probe_calls):
+        moe.moe_forward(layers[i % 2], x, out, ws)
+    torch.cuda.synchronize()
+    st = moe.moe_get_status(ws)
+    print(f"probe T={a.probe_T} calls={a.probe_calls} status={st}")
+    return 0 if st == 0 else 1
+
+
 def main(argv=None):
     a = parse_args(argv)
+    if a.probe_T:
+        return run_probe(a)
     if a.impl == "reference":
         run_reference(a)
     else:

@@ -235,13 +235,6 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
-// A position in the CTA's sequence of weight blocks (4 groups of its items'
-// tiles, item after item): item k (index blockIdx.x + k gridDim.x), block b.
-struct Cursor {
-  int k, b, nbat;
-  bool valid;
-};
-
 // The body both kernels share.  tile_of(item, warp, row, lt) -> WTile: the
 // warp's two tiles as seen by a lane that reads row `row` (and row + 8) at
 // byte 8 lt of each group; k_of(item): inputs per row (a multiple of 256);
@@ -268,56 +261,58 @@ __device__ __forceinline__ void mid_body(const Geometry& g, const int32_t* offse
   uint4* xs = reinterpret_cast<uint4*>(msm);
   float* xsum = reinterpret_cast<float*>(xs + kMTok * (kmax / 8 + 1));
 
-  // open item k of a cursor (false past the CTA's last item)
-  auto open = [&](int k, Item& I) -> bool {
-    const int it = blockIdx.x + k * gridDim.x;
-    if (it >= total) return false;
-    I = decode_item(g, s_start, n_act, offsets, active, it);
-    return true;
-  };
-  // the load walk: this lane's operand pointers for the cursor's item
-  Cursor lc{0, 0, 0, true};
-  WTile lw;
-  int lngr;
-  auto load_open = [&](const Item& I) {
-    lw = tile_of(I, warp, lg4, lt);
-    lngr = k_of(I) / kGroup;
-    lc.nbat = lngr / kMBlock;
-  };
-  // the prefetch walk: the line of row (lane % 16) of tile (lane / 16)
-  Cursor pc{0, 0, 0, true};
+  // The load walk (this lane's operand pointers lw for item lk, block lb)
+  // and the prefetch walk (the line of row lane % 16 of tile lane / 16 at
+  // pq, for item pk, block pb).  Both step through the same sequence.
+  Item I = decode_item(g, s_start, n_act, offsets, active, blockIdx.x);
+  WTile lw = tile_of(I, warp, lg4, lt);
+  int lngr = k_of(I) / kGroup;
+  int lk = 0, lb = 0, lnbat = lngr / kMBlock;
+  bool lvalid = true;
   const uint8_t* pq;
-  auto pf_open = [&](const Item& I) {
+  {
     const WTile w = tile_of(I, warp, lane & 15, 0);
-    pq = w.q[lane >> 4];
-    pc.nbat = k_of(I) / kGroup / kMBlock;
-  };
-  auto advance = [&](Cursor& c, bool is_load) {
-    if (!c.valid) return;
-    if (++c.b < c.nbat) return;
-    c.b = 0;
-    Item N;
-    c.valid = open(++c.k, N);
-    if (c.valid) {
-      if (is_load) load_open(N);
-      else pf_open(N);
-    }
-  };
+    pq = (lane >> 4) ? w.q[1] : w.q[0];
+  }
+  int pk = 0, pb = 0, pnbat = lnbat;
+  bool pvalid = true;
 
-  Item I;
-  open(0, I);
-  load_open(I);
-  pf_open(I);
   uint2 A[kMBlock][2][2];
   BlockS S;
 #pragma unroll
   for (int j = 0; j < kMBlock; ++j) load_group(A[j], lw, lngr, j);
   load_scales(S, lw, lngr, 0);
-  advance(lc, true);
-  for (int i = 0; i < kPrefetchBlocks; ++i) {
-    advance(pc, false);
-    if (pc.valid) prefetch_l2(pq + pc.b * 128);
-  }
+#define MID_STEP_LOAD()                                                             \
+  do {                                                                              \
+    if (lvalid && ++lb == lnbat) {                                                  \
+      lb = 0;                                                                       \
+      const int it_ = blockIdx.x + (++lk) * gridDim.x;                              \
+      lvalid = it_ < total;                                                         \
+      if (lvalid) {                                                                 \
+        const Item n_ = decode_item(g, s_start, n_act, offsets, active, it_);       \
+        lw = tile_of(n_, warp, lg4, lt);                                            \
+        lngr = k_of(n_) / kGroup;                                                   \
+        lnbat = lngr / kMBlock;                                                     \
+      }                                                                             \
+    }                                                                               \
+  } while (0)
+#define MID_STEP_PREFETCH()                                                         \
+  do {                                                                              \
+    if (pvalid && ++pb == pnbat) {                                                  \
+      pb = 0;                                                                       \
+      const int it_ = blockIdx.x + (++pk) * gridDim.x;                              \
+      pvalid = it_ < total;                                                         \
+      if (pvalid) {                                                                 \
+        const Item n_ = decode_item(g, s_start, n_act, offsets, active, it_);       \
+        const WTile w_ = tile_of(n_, warp, lane & 15, 0);                           \
+        pq = (lane >> 4) ? w_.q[1] : w_.q[0];                                       \
+        pnbat = k_of(n_) / kGroup / kMBlock;                                        \
+      }                                                                             \
+    }                                                                               \
+    if (pvalid) prefetch_l2(pq + pb * 128);                                         \
+  } while (0)
+  MID_STEP_LOAD();
+  for (int i = 0; i < kPrefetchBlocks; ++i) MID_STEP_PREFETCH();
 
   for (int k = 0;; ++k) {
     const int K = k_of(I);
@@ -328,10 +323,9 @@ __device__ __forceinline__ void mid_body(const Geometry& g, const int32_t* offse
     float y[2][2][2] = {{{0.f, 0.f}, {0.f, 0.f}}, {{0.f, 0.f}, {0.f, 0.f}}};
     const uint4* xr = xs + lg4 * (K / 8 + 1) + lt * 2;
     for (int b = 0; b < nbat; ++b) {
-      advance(pc, false);
-      if (pc.valid) prefetch_l2(pq + pc.b * 128);
-      const bool lv = lc.valid;
-      const int lG0 = lc.b * kMBlock;
+      MID_STEP_PREFETCH();
+      const bool lv = lvalid;
+      const int lG0 = lb * kMBlock;
       BlockS NS = S;
       if (lv) load_scales(NS, lw, lngr, lG0);
 #pragma unroll
@@ -340,13 +334,15 @@ __device__ __forceinline__ void mid_body(const Geometry& g, const int32_t* offse
         if (lv) load_group(A[j], lw, lngr, lG0 + j);
       }
       S = NS;
-      advance(lc, true);
+      MID_STEP_LOAD();
     }
     store(I, warp, y, lg4, lt);
-    Item N;
-    if (!open(k + 1, N)) break;
-    I = N;
+    const int nit = blockIdx.x + (k + 1) * gridDim.x;
+    if (nit >= total) break;
+    I = decode_item(g, s_start, n_act, offsets, active, nit);
   }
+#undef MID_STEP_LOAD
+#undef MID_STEP_PREFETCH
 }
 
 // ---------------------------------------------------------------------------
