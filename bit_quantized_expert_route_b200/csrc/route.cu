@@ -183,21 +183,32 @@ __global__ void __launch_bounds__(32 * kSegWarps) scatter_kernel(
 
 // ---------------------------------------------------------------------------
 // Small-T routing (T <= 64): one launch does the router GEMV, top-k, shared
-// gate and the whole counting sort.  CTA (b, y) scores rows e = 8b + w (warp
-// w; e == E: the shared-gate vector) for the TB tokens of token group y, so
-// the 1 MB router matrix is streamed by ~33 CTAs per group, all groups at
-// once.  The last CTA of a token group to finish (a counter per group in the
-// workspace's control block) selects the experts of the group's tokens, one
-// token per warp; the last group to finish (one more counter) sorts the T*k
-// entries stably by expert and builds the active-expert list.  Each counter
-// is reset by the CTA that saw it complete.
+// gate and the whole counting sort.  CTA (b, y) scores the 16 rows e = 16b ..
+// 16b + 15 of [W_r; w_sg] (row E: the shared-gate vector) for the 8 tokens of
+// token group y on the tensor cores (mma.sync m16n8k16, bf16 operands, FP32
+// accumulation); its 8 warps split K and add their partial tiles in shared
+// memory in warp order.  The last CTA of a token group to finish (a counter
+// per group in the workspace's control block) selects the experts of the
+// group's tokens, one token per warp; the last group to finish (one more
+// counter) sorts the T*k entries stably by expert and builds the
+// active-expert list.  Each counter is reset by the CTA that saw it complete.
 // ---------------------------------------------------------------------------
 constexpr int kSmallWarps = 8;
+constexpr int kSmallRows = 16;          // router rows per CTA (the MMA's M)
 constexpr int kSmallLoads = 8;          // loads per thread in flight together
+constexpr int kSmallKSteps = 4;         // 16-wide K steps whose loads are in flight together
 
-template <int TB>
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 __global__ void __launch_bounds__(256) router_small_kernel(
-    const uint16_t* __restrict__ x, LayerPtr L, int T, int H, int I, int Is, int E, int k,
+    const uint16_t* __restrict__ x, LayerPtr L, int T, int H, int E, int k,
     float* __restrict__ logits, unsigned* __restrict__ counter,
     int32_t* __restrict__ topk_idx, float* __restrict__ topk_w, float* __restrict__ sigma,
     int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
@@ -205,66 +216,53 @@ __global__ void __launch_bounds__(256) router_small_kernel(
   extern __shared__ uint4 smem_u4[];
   __shared__ int s_last;
   __shared__ int s_scan[33];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int vec = H / 8;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int E1 = E + 1;
-  const int e = blockIdx.x * kSmallWarps + warp;
-  const bool live = e <= E;
-  const uint4* wrow = reinterpret_cast<const uint4*>(e < E ? L.w_router + static_cast<size_t>(e) * H : L.w_sg);
-  const int t0 = blockIdx.y * TB;
-  const int nt = min(TB, T - t0);
+  const int e0 = blockIdx.x * kSmallRows;
+  const int t0 = blockIdx.y * kSmallTB;
+  const int nt = min(kSmallTB, T - t0);
 
-  uint4* xs = smem_u4;   // [TB][vec]
-  for (int i0 = threadIdx.x; i0 < TB * vec; i0 += blockDim.x * kSmallLoads) {
-    uint4 v[kSmallLoads];   // all loads in flight before the first store
+  // Lane (g, t) of the MMA holds rows e0 + g and e0 + g + 8 and token t0 + g.
+  // Within each 16-wide K step the lane's logical K pairs (2t, 2t+1) and
+  // (2t+8, 2t+9) are the four consecutive inputs 4t .. 4t+3 of the step, for
+  // both operands, so each operand is one 8-byte load per step.
+  auto row_of = [&](int e) -> const uint16_t* {
+    return e < E ? L.w_router + static_cast<size_t>(e) * H : (e == E ? L.w_sg : nullptr);
+  };
+  const uint16_t* ra = row_of(e0 + g);
+  const uint16_t* rb = row_of(e0 + g + 8);
+  const uint16_t* xr = g < nt ? x + static_cast<size_t>(t0 + g) * H : nullptr;
+  const int kw = H / kSmallWarps;              // inputs per warp (a multiple of 16)
+  const int kbeg = warp * kw + 4 * t;
+  float d[4] = {0.f, 0.f, 0.f, 0.f};
+  const uint2 z = make_uint2(0u, 0u);
+  for (int ks0 = 0; ks0 < kw; ks0 += 16 * kSmallKSteps) {
+    uint2 a[kSmallKSteps], b[kSmallKSteps], xb[kSmallKSteps];
 #pragma unroll
-    for (int j = 0; j < kSmallLoads; ++j) {
-      const int i = i0 + j * blockDim.x;
-      const int r = i / vec, c = i - r * vec;
-      v[j] = (i < TB * vec && r < nt) ? reinterpret_cast<const uint4*>(x + static_cast<size_t>(t0 + r) * H)[c]
-                                      : make_uint4(0u, 0u, 0u, 0u);
+    for (int j = 0; j < kSmallKSteps; ++j) {
+      const int kk = kbeg + ks0 + 16 * j;
+      const bool in = ks0 + 16 * j < kw;
+      a[j] = (in && ra) ? __ldg(reinterpret_cast<const uint2*>(ra + kk)) : z;
+      b[j] = (in && rb) ? __ldg(reinterpret_cast<const uint2*>(rb + kk)) : z;
+      xb[j] = (in && xr) ? __ldg(reinterpret_cast<const uint2*>(xr + kk)) : z;
     }
 #pragma unroll
-    for (int j = 0; j < kSmallLoads; ++j)
-      if (i0 + j * blockDim.x < TB * vec) xs[i0 + j * blockDim.x] = v[j];
+    for (int j = 0; j < kSmallKSteps; ++j) mma_bf16_16816(d, a[j].x, b[j].x, a[j].y, b[j].y, xb[j].x, xb[j].y);
   }
+  // partial tiles of the 8 K slices: part[warp][row][token], added in warp order
+  float* part = reinterpret_cast<float*>(smem_u4);
+  part[(warp * kSmallRows + g) * kSmallTB + 2 * t] = d[0];
+  part[(warp * kSmallRows + g) * kSmallTB + 2 * t + 1] = d[1];
+  part[(warp * kSmallRows + g + 8) * kSmallTB + 2 * t] = d[2];
+  part[(warp * kSmallRows + g + 8) * kSmallTB + 2 * t + 1] = d[3];
   __syncthreads();
-  if (live) {
-    float acc[TB];
+  if (threadIdx.x < kSmallRows * kSmallTB) {
+    const int r = threadIdx.x / kSmallTB, c = threadIdx.x % kSmallTB;
+    const int e = e0 + r;
+    float sum = 0.f;
 #pragma unroll
-    for (int r = 0; r < TB; ++r) acc[r] = 0.f;
-    for (int c0 = lane; c0 < vec; c0 += 32 * kSmallLoads) {
-      uint4 wv[kSmallLoads];
-#pragma unroll
-      for (int u = 0; u < kSmallLoads; ++u) {
-        const int c = c0 + 32 * u;
-        wv[u] = c < vec ? __ldg(wrow + c) : make_uint4(0u, 0u, 0u, 0u);
-      }
-#pragma unroll
-      for (int u = 0; u < kSmallLoads; ++u) {
-        const int c = c0 + 32 * u;
-        if (c < vec) {
-          const float w0 = bf16_lo(wv[u].x), w1 = bf16_hi(wv[u].x), w2 = bf16_lo(wv[u].y), w3 = bf16_hi(wv[u].y);
-          const float w4 = bf16_lo(wv[u].z), w5 = bf16_hi(wv[u].z), w6 = bf16_lo(wv[u].w), w7 = bf16_hi(wv[u].w);
-#pragma unroll
-          for (int r = 0; r < TB; ++r) {
-            const uint4 xv = xs[r * vec + c];
-            float a = acc[r];
-            a = fmaf(bf16_lo(xv.x), w0, a); a = fmaf(bf16_hi(xv.x), w1, a);
-            a = fmaf(bf16_lo(xv.y), w2, a); a = fmaf(bf16_hi(xv.y), w3, a);
-            a = fmaf(bf16_lo(xv.z), w4, a); a = fmaf(bf16_hi(xv.z), w5, a);
-            a = fmaf(bf16_lo(xv.w), w6, a); a = fmaf(bf16_hi(xv.w), w7, a);
-            acc[r] = a;
-          }
-        }
-      }
-    }
-    const float b = (e < E && L.router_bias) ? L.router_bias[e] : 0.f;
-#pragma unroll
-    for (int r = 0; r < TB; ++r) {
-      const float sum = warp_sum(acc[r]);
-      if (lane == 0 && r < nt) logits[static_cast<size_t>(t0 + r) * E1 + e] = sum + b;
-    }
+    for (int w = 0; w < kSmallWarps; ++w) sum += part[(w * kSmallRows + r) * kSmallTB + c];
+    if (e <= E && c < nt) logits[static_cast<size_t>(t0 + c) * E1 + e] = sum + ((e < E && L.router_bias) ? L.router_bias[e] : 0.f);
   }
 
   // ---- the last CTA of this token group selects its tokens' experts ----
@@ -276,7 +274,7 @@ __global__ void __launch_bounds__(256) router_small_kernel(
   if (!s_last) return;
   __threadfence();
   if (threadIdx.x == 0) *group_counter = 0u;
-  float* lg = reinterpret_cast<float*>(smem_u4);   // [TB][E1], reuses the x tile
+  float* lg = reinterpret_cast<float*>(smem_u4);   // [8 tokens][E1], reuses the partial tiles
   for (int i0 = threadIdx.x; i0 < nt * E1; i0 += blockDim.x * kSmallLoads) {
     float v[kSmallLoads];
 #pragma unroll
@@ -369,30 +367,20 @@ __global__ void __launch_bounds__(256) router_small_kernel(
 // ---------------------------------------------------------------------------
 int num_segments(int T) { return (T + kRouteSegTokens - 1) / kRouteSegTokens; }
 
-template <int TB>
-static cudaError_t launch_small_tb(const uint16_t* x, const LayerPtr& L, int T, int H, int I, int Is, int E, int k,
-                                   float* logits, unsigned* counter, const RoutingPtrs& r, int32_t* active,
-                                   int32_t* n_active, cudaStream_t s) {
-  const dim3 grid((E + 1 + kSmallWarps - 1) / kSmallWarps, (T + TB - 1) / TB);
-  const int smem = max(TB * H * 2, max(TB * (E + 1) * 4, (kSmallWarps * 256 + T * k) * 4));
-  const cudaError_t e = ensure_smem(reinterpret_cast<const void*>(router_small_kernel<TB>), smem);
-  if (e != cudaSuccess) return e;
-  router_small_kernel<TB><<<grid, 256, smem, s>>>(x, L, T, H, I, Is, E, k, logits, counter, r.topk_idx, r.topk_w,
-                                                  r.sigma, r.counts, r.offsets, r.perm, r.inv_perm, active,
-                                                  n_active);
-  return cudaGetLastError();
-}
-
 cudaError_t launch_route_small(const uint16_t* x, const LayerPtr& L, int T, int H, int I, int Is, int E, int k,
                                float* logits, unsigned* counter, const RoutingPtrs& r, int32_t* active,
                                int32_t* n_active, cudaStream_t s) {
-  // tokens per CTA: x tile of TB rows (bf16) in smem; at most
-  // kSmallMaxGroups token groups (one counter each)
-  if (T > kSmallTB * kSmallMaxGroups) return cudaErrorInvalidValue;
-  if (T == 1) return launch_small_tb<1>(x, L, T, H, I, Is, E, k, logits, counter, r, active, n_active, s);
-  if (T <= 2) return launch_small_tb<2>(x, L, T, H, I, Is, E, k, logits, counter, r, active, n_active, s);
-  if (T <= 4) return launch_small_tb<4>(x, L, T, H, I, Is, E, k, logits, counter, r, active, n_active, s);
-  return launch_small_tb<kSmallTB>(x, L, T, H, I, Is, E, k, logits, counter, r, active, n_active, s);
+  (void)I;
+  (void)Is;
+  // one token group (one counter) per 8 tokens
+  if (T > kSmallTB * kSmallMaxGroups || H % (16 * kSmallWarps)) return cudaErrorInvalidValue;
+  const dim3 grid((E + 1 + kSmallRows - 1) / kSmallRows, (T + kSmallTB - 1) / kSmallTB);
+  const int smem = max(kSmallWarps * kSmallRows * kSmallTB * 4, max(kSmallTB * (E + 1) * 4, (kSmallWarps * 256 + T * k) * 4));
+  const cudaError_t e = ensure_smem(reinterpret_cast<const void*>(router_small_kernel), smem);
+  if (e != cudaSuccess) return e;
+  router_small_kernel<<<grid, 256, smem, s>>>(x, L, T, H, E, k, logits, counter, r.topk_idx, r.topk_w, r.sigma,
+                                              r.counts, r.offsets, r.perm, r.inv_perm, active, n_active);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_group(const int32_t* topk_idx, int T, int k, int E, int chunk_rows,
