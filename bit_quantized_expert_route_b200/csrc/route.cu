@@ -236,15 +236,33 @@ __global__ void __launch_bounds__(256) router_small_kernel(
   const int kbeg = warp * kw + 4 * t;
   float d[4] = {0.f, 0.f, 0.f, 0.f};
   const uint2 z = make_uint2(0u, 0u);
+  // The router rows do not depend on the previous kernel of the stream: the
+  // first K steps' rows are requested before waiting for it (programmatic
+  // dependent launch), x and every output after.
+  uint2 a[kSmallKSteps], b[kSmallKSteps], xb[kSmallKSteps];
+#pragma unroll
+  for (int j = 0; j < kSmallKSteps; ++j) {
+    const int kk = kbeg + 16 * j;
+    const bool in = 16 * j < kw;
+    a[j] = (in && ra) ? __ldg(reinterpret_cast<const uint2*>(ra + kk)) : z;
+    b[j] = (in && rb) ? __ldg(reinterpret_cast<const uint2*>(rb + kk)) : z;
+  }
+  pdl_wait();
+  pdl_launch_dependents();
   for (int ks0 = 0; ks0 < kw; ks0 += 16 * kSmallKSteps) {
-    uint2 a[kSmallKSteps], b[kSmallKSteps], xb[kSmallKSteps];
+    if (ks0 > 0) {
+#pragma unroll
+      for (int j = 0; j < kSmallKSteps; ++j) {
+        const int kk = kbeg + ks0 + 16 * j;
+        const bool in = ks0 + 16 * j < kw;
+        a[j] = (in && ra) ? __ldg(reinterpret_cast<const uint2*>(ra + kk)) : z;
+        b[j] = (in && rb) ? __ldg(reinterpret_cast<const uint2*>(rb + kk)) : z;
+      }
+    }
 #pragma unroll
     for (int j = 0; j < kSmallKSteps; ++j) {
       const int kk = kbeg + ks0 + 16 * j;
-      const bool in = ks0 + 16 * j < kw;
-      a[j] = (in && ra) ? __ldg(reinterpret_cast<const uint2*>(ra + kk)) : z;
-      b[j] = (in && rb) ? __ldg(reinterpret_cast<const uint2*>(rb + kk)) : z;
-      xb[j] = (in && xr) ? __ldg(reinterpret_cast<const uint2*>(xr + kk)) : z;
+      xb[j] = (ks0 + 16 * j < kw && xr) ? __ldg(reinterpret_cast<const uint2*>(xr + kk)) : z;
     }
 #pragma unroll
     for (int j = 0; j < kSmallKSteps; ++j) mma_bf16_16816(d, a[j].x, b[j].x, a[j].y, b[j].y, xb[j].x, xb[j].y);
@@ -378,9 +396,8 @@ cudaError_t launch_route_small(const uint16_t* x, const LayerPtr& L, int T, int 
   const int smem = max(kSmallWarps * kSmallRows * kSmallTB * 4, max(kSmallTB * (E + 1) * 4, (kSmallWarps * 256 + T * k) * 4));
   const cudaError_t e = ensure_smem(reinterpret_cast<const void*>(router_small_kernel), smem);
   if (e != cudaSuccess) return e;
-  router_small_kernel<<<grid, 256, smem, s>>>(x, L, T, H, E, k, logits, counter, r.topk_idx, r.topk_w, r.sigma,
-                                              r.counts, r.offsets, r.perm, r.inv_perm, active, n_active);
-  return cudaGetLastError();
+  return launch_pdl(router_small_kernel, grid, dim3(256), smem, s, x, L, T, H, E, k, logits, counter, r.topk_idx,
+                    r.topk_w, r.sigma, r.counts, r.offsets, r.perm, r.inv_perm, active, n_active);
 }
 
 cudaError_t launch_group(const int32_t* topk_idx, int T, int k, int E, int chunk_rows,
