@@ -177,6 +177,30 @@ def test_decode_entry_and_forward_both_match_oracle(dims, T):
         assert_output_close(gpu["out"], ref["out"])
 
 
+# A second geometry for the mid-size decode path (H, I, I_shared multiples of
+# 256): 8 groups per gate/up row and 4 per down row, and with 16 experts of
+# which 4 are chosen every expert sees 16+ tokens at T >= 64 (several 8-token
+# tiles per expert, the last one ragged).
+MID = dataclasses.replace(TINY, H=512, E=16, k=4, I=256, I_s=256)
+
+
+@pytest.mark.parametrize("T,zipf", [(9, False), (40, True), (64, False), (64, True)])
+def test_mid_size_path_second_geometry(T, zipf):
+    lay, x, _ = workload(70 + T, T, MID, zipf=zipf)
+    ref = moe_ref.moe_layer(x, lay, MID.k)
+    L = moe.MoELayer.from_synth(lay)
+    assert len(moe.moe_forward_profiled(L, to_dev_bits(x), torch.empty((T, MID.H), dtype=torch.bfloat16,
+                                                                         device="cuda"),
+                                        moe.alloc_workspace(L, T))) == len(moe.MID_DECODE_STAGES)
+    if T == 64:
+        assert int(np.max(ref["counts"])) > 8
+    for entry in ("forward", "decode"):
+        gpu = run_layer(lay, x, entry=entry, dev_layer=L)
+        assert gpu["status"] == 0
+        assert_routing_exact(gpu, ref)
+        assert_output_close(gpu["out"], ref["out"])
+
+
 def test_rmsnorm_matches_oracle():
     rng = np.random.default_rng(9)
     y_bits = synth.to_bf16_bits(rng.normal(0, 0.05, size=(37, 2048)))
