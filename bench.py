@@ -50,7 +50,7 @@ GDN_B = (1, 8, 64)                # recurrence batch sizes (16 key heads, 32 val
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PREFILL_LAUNCHES_PER_STEP = 7     # router (+ segment counts), scan, scatter, gather, gate/up, down, combine
 UNFUSED_DECODE_LAUNCHES = 4       # routing (router+top-k+sort), gate/up GEMV, down GEMV, combine
-FUSED_DECODE_LAUNCHES = 1         # T <= 2: the whole layer in one cooperative launch
+FUSED_DECODE_LAUNCHES = 1         # T <= 3 (single layer): the whole layer in one cooperative launch
 NOMINAL_BF16_TFLOPS = 2250.0      # B200 dense bf16 datasheet figure (context)
 NOMINAL_HBM_GBS = 8000.0          # B200 HBM3e nominal bandwidth (context)
 COMPUTE_DTYPE = "bf16"            # grouped GEMM operands (FP32 accumulation in tensor memory)

@@ -63,7 +63,13 @@ namespace {
 using namespace moe;
 
 constexpr int kDecodeMaxT = 64;
-constexpr int kFusedMaxT = 8;       // tokens the fused decode kernel takes
+// Tokens the fused decode kernel takes: a stack of layers runs up to 40 of
+// them per cooperative launch and wins up to T = 8; a single layer pays the
+// cooperative launch and the kernel's fixed phases every call, and the
+// mid-size path is faster from T = 4 (measured per layer, 40 distinct
+// layers: T=3 38.9 vs 39.8 us, T=4 46.6 vs 40.9, T=8 81.1 vs 59.1).
+constexpr int kFusedMaxT = 3;       // single-layer calls
+constexpr int kFusedMaxTStack = 8;  // moe_forward_stack
 constexpr int kMidMaxT = 64;        // tokens the mid-size decode path takes
 constexpr int kMaxT = 65536;
 constexpr int kMaxStackLayers = 1024;
@@ -115,7 +121,7 @@ WsLayout ws_layout(const moe_layer_desc* d, int T) {
   // the fused decode kernel's exchange words: logits, h, outputs between
   // stacked layers and the CTAs' sums of squares of them
   for (int i = 0; i < 4; ++i)
-    w.xch[i] = take(T <= kFusedMaxT ? fused_exchange_words(T, d->H, d->I, d->I_shared, d->E, d->k, i) * 8 : 0);
+    w.xch[i] = take(T <= kFusedMaxTStack ? fused_exchange_words(T, d->H, d->I, d->I_shared, d->E, d->k, i) * 8 : 0);
   w.total = off;
   return w;
 }
@@ -268,14 +274,16 @@ bool mid_decode_ok(const moe_layer_desc* d, const Geometry& g) {
 // combine), else the tensor-core (tcgen05) grouped-GEMM path.
 enum class Path { kFused, kMid, kPrefill };
 
-Path layer_path(const moe_layer_desc* d, int T) {
+Path layer_path(const moe_layer_desc* d, int T, bool stacked = false) {
   const Geometry g{T, d->H, d->I, d->I_shared, d->E, d->k};
-  if (T <= kFusedMaxT && fused_decode_ok(d, g)) return Path::kFused;
+  if (T <= (stacked ? kFusedMaxTStack : kFusedMaxT) && fused_decode_ok(d, g)) return Path::kFused;
   if (T <= kMidMaxT && mid_decode_ok(d, g)) return Path::kMid;
   return Path::kPrefill;
 }
 
-bool forward_uses_fused_decode(const moe_layer_desc* d, int T) { return layer_path(d, T) == Path::kFused; }
+bool forward_uses_fused_decode(const moe_layer_desc* d, int T, bool stacked = false) {
+  return layer_path(d, T, stacked) == Path::kFused;
+}
 
 // The fused decode kernel for one layer (routing outputs included).
 int enqueue_fused(const moe_layer_desc* d, const uint16_t* x, int T, uint16_t* out, const Bufs& b,
@@ -346,7 +354,7 @@ int enqueue_prefill(const moe_layer_desc* d, const uint16_t* x, int T, uint16_t*
 // norm_out (may be NULL) its RMSNorm, the next layer's input.
 int enqueue_layer(const moe_layer_desc* d, const uint16_t* x, int T, uint16_t* out, uint16_t* norm_out, float eps,
                   const Bufs& b, cudaStream_t s) {
-  switch (layer_path(d, T)) {
+  switch (layer_path(d, T, /*stacked=*/true)) {
     case Path::kPrefill: return enqueue_prefill(d, x, T, out, b, s, nullptr, norm_out, eps);
     case Path::kMid: return enqueue_mid(d, x, T, out, b, s, nullptr, norm_out, eps);
     default: break;
@@ -501,7 +509,7 @@ int moe_forward_stack(const moe_layer_desc* layers, int n_layers, const moe_bf16
   uint16_t* pingpong[2] = {b0.at<uint16_t>(b0.w.x_stage), b0.at<uint16_t>(b0.w.out_stage)};
   uint16_t* tr = reinterpret_cast<uint16_t*>(trace);
   bool fused = true;
-  for (int l = 0; l < n_layers; ++l) fused = fused && forward_uses_fused_decode(&layers[l], T);
+  for (int l = 0; l < n_layers; ++l) fused = fused && forward_uses_fused_decode(&layers[l], T, /*stacked=*/true);
   if (fused) {
     // whole chunks of layers per launch of the fused decode kernel, which
     // applies the RMSNorm between its layers itself and writes the trace

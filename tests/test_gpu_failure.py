@@ -94,26 +94,35 @@ def test_router_wait_runs_out_and_the_next_call_is_correct():
     _assert_next_call_correct(lay, x, L, xd, out, ws)
 
 
-@pytest.mark.parametrize("T", [1, 8])
-def test_fused_decode_waits_run_out_and_the_next_call_is_correct(T):
+@pytest.mark.parametrize("T,entry", [(1, "forward"), (3, "forward"), (8, "stack")])
+def test_fused_decode_waits_run_out_and_the_next_call_is_correct(T, entry):
     """The single-launch decode kernel's producer, consumers and grid barriers all give up
     after one cycle; every CTA leaves (its copies landed), the grid-barrier words are reset
-    for the next launch, and the next call on the same workspace is correct."""
+    for the next launch, and the next call on the same workspace is correct.  A single
+    layer runs the fused kernel up to T = 3, a stack (here of one layer) up to T = 8."""
     lay, x, _ = workload(82 + T, T, FULL)
     L = moe.MoELayer.from_synth(lay)
     xd = to_dev_bits(x)
     out = torch.empty_like(xd)
     ws = moe.alloc_workspace(L, T)
+
+    def call():
+        if entry == "stack":
+            moe.moe_forward_stack(moe.LayerStack([L]), xd, out, ws, eps=1e-6)
+        else:
+            moe.moe_forward(L, xd, out, ws)
+
+    assert len(moe.moe_forward_profiled(L, xd, out, ws)) == (1 if entry == "forward" else 4)
     moe.moe_set_wait_limit(1)
     try:
-        moe.moe_forward(L, xd, out, ws)
+        call()
         torch.cuda.synchronize()
     finally:
         moe.moe_set_wait_limit(0)
     assert moe.moe_get_status(ws) == moe.MOE_ERR_DEVICE_TIMEOUT
     assert int(ws[:16].count_nonzero()) == 0
     for _ in range(2):
-        moe.moe_forward(L, xd, out, ws)
+        call()
         torch.cuda.synchronize()
         assert moe.moe_get_status(ws) == moe.MOE_OK
         m = moe_ref.compare(moe_ref.bf16_to_f64(bits_of(out)), moe_ref.moe_layer(x, lay, FULL.k)["out"])

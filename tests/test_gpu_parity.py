@@ -224,7 +224,7 @@ def test_rmsnorm_matches_oracle():
                                      (8, "forward"), (9, "forward"), (16, "forward"), (33, "forward"),
                                      (64, "forward"), (3, "decode"), (8, "decode"), (9, "decode"), (64, "decode")])
 def test_full_decode(T, entry):
-    # T <= 8 runs the single-launch fused decode kernel (both entries); 9 <= T
+    # T <= 3 runs the single-launch fused decode kernel (both entries); 4 <= T
     # <= 64 the mid-size decode path (small-T router, mma.sync GEMVs over the
     # active experts in 8-token tiles, fixed-order combine)
     lay, x, _ = workload(10 + T, T, FULL)

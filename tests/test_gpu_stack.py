@@ -157,13 +157,15 @@ def _ulp_distance(a: np.ndarray, b: np.ndarray) -> np.ndarray:
 # T <= 8: the fused decode kernel runs the stack in launches of up to 40
 # layers (42 layers: two launches and a stand-alone RMSNorm between them);
 # larger T: the tensor-core path with the RMSNorm fused into the combine.
-@pytest.mark.parametrize("T,n_layers", [(1, 4), (2, 42), (8, 3), (64, 3), (65, 2), (512, 3)])
+@pytest.mark.parametrize("T,n_layers", [(1, 4), (2, 42), (5, 2), (8, 3), (64, 3), (65, 2), (512, 3)])
 def test_forward_stack_matches_single_layer_calls(T, n_layers):
-    """moe_forward_stack vs the per-layer entry points on the stack's own activations: every
-    layer's output is bit-identical to moe_forward on the same input (same kernels), and every
-    next input is the RMSNorm of that output (float64 identity within one bf16 ulp, and within
-    one ulp of the stand-alone moe_rmsnorm).  The per-layer path itself is held to the oracle by
-    test_stack_layer_by_layer."""
+    """moe_forward_stack vs per-layer calls on the stack's own activations: every layer's output
+    is bit-identical to a one-layer stack call on the same input (same kernels) and, where a
+    single moe_forward call runs the same kernel set (T <= 3 or T >= 9), to moe_forward as well;
+    for 4 <= T <= 8 a stack keeps the fused kernel while a single call takes the mid-size path,
+    and the two agree within the layer tolerance.  Every next input is the RMSNorm of the
+    previous output (float64 identity within one bf16 ulp, and within one ulp of the stand-alone
+    moe_rmsnorm).  The per-layer path itself is held to the oracle by test_stack_layer_by_layer."""
     dev = torch.device("cuda", 0)
     layers = [moe.MoELayer.from_tensors(FULL, synth.make_layer_on_device(300 + T, l, FULL, dev, l % 2 == 1))
               for l in range(n_layers)]
@@ -180,9 +182,16 @@ def test_forward_stack_matches_single_layer_calls(T, n_layers):
     ws1 = moe.alloc_workspace(layers[0], T, dev)
     for l, L in enumerate(layers):
         y = torch.empty_like(x)
+        moe.moe_forward_stack(moe.LayerStack([L]), trace[l, 0].contiguous(), y, ws1)
+        torch.cuda.synchronize()
+        assert torch.equal(y, trace[l, 1]), f"layer {l}: stack output differs from a one-layer stack call"
         moe.moe_forward(L, trace[l, 0].contiguous(), y, ws1)
         torch.cuda.synchronize()
-        assert torch.equal(y, trace[l, 1]), f"layer {l}: stack output differs from moe_forward"
+        if T <= 3 or T >= 9:
+            assert torch.equal(y, trace[l, 1]), f"layer {l}: stack output differs from moe_forward"
+        else:
+            m = moe_ref.compare(moe_ref.bf16_to_f64(bits_of(y)), moe_ref.bf16_to_f64(bits_of(trace[l, 1])))
+            assert m["rel_l2"] <= moe_ref.REL_L2_TOL and m["max_err_rel"] <= moe_ref.MAX_ERR_TOL, m
         if l + 1 < n_layers:
             got = bits_of(trace[l + 1, 0])
             assert int(_ulp_distance(got, _rmsnorm_f64_bits(bits_of(trace[l, 1]))).max()) <= 1
