@@ -182,6 +182,143 @@ __global__ void __launch_bounds__(32 * kSegWarps) scatter_kernel(
 }
 
 // ---------------------------------------------------------------------------
+// Passes 2 and 3 in one launch when the segments are few (T <= 64 * 128): CTA
+// s recomputes, from the router's per-segment counts, every expert's total
+// and the counts of the segments before s (nseg loads per thread, a few KB
+// from L2), scans the totals into the offsets, and scatters its own segment
+// as scatter_kernel does (8 warps of 16 tokens here).  CTA 0 also writes the
+// counts, offsets, chunk list and active list exactly as scan_kernel does.
+// One launch less, and no single-CTA pass on the critical path.
+// ---------------------------------------------------------------------------
+constexpr int kGroupThreads = 256;          // one routed expert per thread (E <= 256)
+constexpr int kGroupWarps = kGroupThreads / 32;
+constexpr int kGroupFuseSegs = 64;          // fused for up to 64 segments
+constexpr int kGroupLoads = 16;             // segment counts per thread in flight together
+
+__global__ void __launch_bounds__(kGroupThreads) group_fused_kernel(
+    const int32_t* __restrict__ seg_counts, int nseg, int E, int T, int k, int chunk_rows,
+    const int32_t* __restrict__ topk_idx, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+    Chunk* __restrict__ chunks, int32_t* __restrict__ n_chunks, int32_t* __restrict__ active,
+    int32_t* __restrict__ n_active, int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm) {
+  pdl_wait();
+  pdl_launch_dependents();
+  extern __shared__ int sh_cnt[];   // [kGroupWarps][E]: slice counts, then each slice's first positions
+  __shared__ int scratch[33];
+  __shared__ int seg_first[kMaxE];  // this segment's first position per expert
+  const int e = threadIdx.x;
+  const int seg = blockIdx.x;
+  int c = 0, before = 0;
+  if (e < E)
+    for (int s0 = 0; s0 < nseg; s0 += kGroupLoads) {
+      int v[kGroupLoads];
+#pragma unroll
+      for (int j = 0; j < kGroupLoads; ++j)
+        v[j] = (s0 + j < nseg) ? seg_counts[static_cast<size_t>(s0 + j) * E + e] : 0;
+#pragma unroll
+      for (int j = 0; j < kGroupLoads; ++j) {
+        c += v[j];
+        if (s0 + j < seg) before += v[j];
+      }
+    }
+  int off = 0;
+  const int total = block_exclusive_scan(e < E ? c : 0, scratch, &off);
+  if (e < E) seg_first[e] = off + before;
+
+  if (seg == 0) {
+    // counts, offsets, chunk list (routed experts in order, then the shared
+    // expert's rows T*k + t) and active list, as scan_kernel writes them
+    if (e < E) {
+      counts[e] = c;
+      offsets[e] = off;
+    }
+    if (e == 0) offsets[E] = total;
+    const int rows = e < E ? c : 0;
+    const int nch = (rows + chunk_rows - 1) / chunk_rows;
+    int first = 0;
+    const int routed_chunks = block_exclusive_scan(nch, scratch, &first);
+    {
+      const int base = nch > 0 ? rows / nch : 0, rem = nch > 0 ? rows % nch : 0;
+      int r0 = 0;
+      for (int q = 0; q < nch; ++q) {
+        const int r1 = (q + 1) * base + ((q + 1) * rem) / nch;
+        Chunk ch;
+        ch.e = e; ch.row0 = off + r0; ch.rows = r1 - r0; ch.pad = 0;
+        chunks[first + q] = ch;
+        r0 = r1;
+      }
+    }
+    if (e == 0) {
+      const int srows = T, snch = (T + chunk_rows - 1) / chunk_rows;
+      const int base = srows / snch, rem = srows % snch;
+      int r0 = 0;
+      for (int q = 0; q < snch; ++q) {
+        const int r1 = (q + 1) * base + ((q + 1) * rem) / snch;
+        Chunk ch;
+        ch.e = E; ch.row0 = T * k + r0; ch.rows = r1 - r0; ch.pad = 0;
+        chunks[routed_chunks + q] = ch;
+        r0 = r1;
+      }
+      *n_chunks = routed_chunks + snch;
+    }
+    int apos = 0;
+    const int nact = block_exclusive_scan((e < E && c > 0) ? 1 : 0, scratch, &apos);
+    if (e < E && c > 0) active[apos] = e;
+    if (e == 0) {
+      active[nact] = E;
+      *n_active = nact + 1;
+    }
+  }
+
+  // scatter this segment: warp w ranks the entries of tokens [16 w, 16 w + 16)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n = T * k;
+  const int seg_len = kRouteSegTokens * k;
+  const int slice_len = seg_len / kGroupWarps;
+  const int b = seg * seg_len + warp * slice_len, end = min(b + slice_len, n);
+  int* cnt = sh_cnt + warp * E;
+  for (int x = lane; x < E; x += 32) cnt[x] = 0;
+  constexpr int kRounds = kRouteSegTokens * kMaxK / 32 / kGroupWarps;   // 4 rounds of 32 entries at most
+  int ex[kRounds];
+#pragma unroll
+  for (int j = 0; j < kRounds; ++j) {
+    const int i = b + j * 32 + lane;
+    const int x = (i < end) ? topk_idx[i] : -1;
+    ex[j] = (x >= 0 && x < E) ? x : -1;
+  }
+  __syncwarp();
+#pragma unroll
+  for (int j = 0; j < kRounds; ++j)
+    if (ex[j] >= 0) atomicAdd(&cnt[ex[j]], 1);   // counting is order-independent
+  __syncthreads();
+  if (e < E) {
+    int run = seg_first[e];
+    for (int w = 0; w < kGroupWarps; ++w) {
+      const int t = sh_cnt[w * E + e];
+      sh_cnt[w * E + e] = run;
+      run += t;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < kRounds; ++j) {
+    if (b + j * 32 >= end) break;
+    const int i = b + j * 32 + lane;
+    const int x = ex[j];
+    const unsigned peers = __match_any_sync(0xffffffffu, x);
+    const int rank = __popc(peers & lanemask_lt());
+    const int start = (x >= 0) ? cnt[x] : 0;
+    __syncwarp();
+    if (x >= 0) {
+      const int pos = start + rank;
+      perm[pos] = i;
+      inv_perm[i] = pos;
+      if ((peers >> lane) == 1u) cnt[x] = start + __popc(peers);   // highest lane of the group
+    }
+    __syncwarp();
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Small-T routing (T <= 64): one launch does the router GEMV, top-k, shared
 // gate and the whole counting sort.  CTA (b, y) scores the 16 rows e = 16b ..
 // 16b + 15 of [W_r; w_sg] (row E: the shared-gate vector) for the 8 tokens of
@@ -406,6 +543,12 @@ cudaError_t launch_group(const int32_t* topk_idx, int T, int k, int E, int chunk
                          int32_t* active, int32_t* n_active, cudaStream_t s) {
   const int n = T * k;
   const int nseg = num_segments(T);
+  if (nseg <= kGroupFuseSegs && E <= kGroupThreads) {
+    const int fsmem = kGroupWarps * E * static_cast<int>(sizeof(int));
+    return launch_pdl(group_fused_kernel, dim3(nseg), dim3(kGroupThreads), static_cast<size_t>(fsmem), s,
+                      static_cast<const int32_t*>(seg_scratch), nseg, E, T, k, chunk_rows, topk_idx, counts, offsets,
+                      chunks, n_chunks, active, n_active, perm, inv_perm);
+  }
   const int grid = nseg;
   const int smem = kSegWarps * E * static_cast<int>(sizeof(int));
   cudaError_t e = launch_pdl(scan_kernel, dim3(1), dim3(kScanThreads), 0, s, seg_scratch, nseg, E, T, k, chunk_rows,
