@@ -544,10 +544,10 @@ def tiny_phase(a, world, dev):
     s_ms = timed_loop(lambda i: moe.moe_forward(L, x, out, ws), 200, world) / 200
     del graph
     assert moe.moe_get_status(ws) == 0
-    return {"workload": "tiny layer T=16, H=256, E=16, k=2, I=I_s=128 (decode kernels: T <= 64)",
+    return {"workload": "tiny layer T=16, H=256, E=16, k=2, I=I_s=128 (mid-size decode path)",
             "layer_us": round(g_ms * 1e3, 3), "layer_us_stream_launched": round(s_ms * 1e3, 3),
             "tokens_per_s": round(whole_job_rate(T, world, g_ms), 1),
-            "bound": "launch latency (3 dependent launches of ~1 KB of work each)"}
+            "bound": "launch latency (4 dependent launches: router, gate/up, down, combine; ~1 MB of weights)"}
 
 
 # --------------------------------------------------- decode attention ---

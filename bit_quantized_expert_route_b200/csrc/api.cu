@@ -259,12 +259,8 @@ bool fused_decode_ok(const moe_layer_desc* d, const Geometry& g) {
   return decode_fused_supported(g);
 }
 
-// The mid-size decode kernels load 4 groups' scales (or biases) of a row as
-// one 8-byte word.
 bool mid_decode_ok(const moe_layer_desc* d, const Geometry& g) {
-  const moe_qmat* m[6] = {&d->gate, &d->up, &d->down, &d->sh_gate, &d->sh_up, &d->sh_down};
-  for (const moe_qmat* q : m)
-    if ((reinterpret_cast<uintptr_t>(q->scales) & 7u) || (reinterpret_cast<uintptr_t>(q->biases) & 7u)) return false;
+  (void)d;
   return mid_decode_supported(g);
 }
 

@@ -31,6 +31,8 @@
 // activations, read conflict-free: token rows are padded by 16 bytes and the
 // group sums are stored token-minor, so a lane's two sums are one 8-byte
 // read.
+#include <initializer_list>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "mma_dq.cuh"
@@ -42,7 +44,9 @@ constexpr int kMThreads = kMWarps * 32;
 constexpr int kMGateUpRows = 16 * kMWarps;   // features of a gate/up item
 constexpr int kMDownRows = 32 * kMWarps;     // output dims of a down item
 constexpr int kMTok = 8;                     // tokens of an item: the n8 column tile
-constexpr int kMBlock = 4;                   // groups of 64 inputs per pipeline block
+// Groups of 64 inputs per pipeline block: 4 when every row has a multiple of
+// 4 groups and the scale/bias stacks are 8-byte aligned (one 8-byte load per
+// row and block), else 2 (one 4-byte load).
 
 __device__ __forceinline__ QMatPtr expert_qmat(const QMatPtr& stack, int e, size_t rows, size_t cols) {
   return QMatPtr{stack.q + static_cast<size_t>(e) * rows * (cols / 8),
@@ -194,24 +198,36 @@ __device__ __forceinline__ void load_group(uint2 (&a)[2][2], const WTile& w, int
       a[m][r] = __ldg(reinterpret_cast<const uint2*>(w.q[m] + static_cast<size_t>(r) * 8 * ngr * 32 + G * 32));
 }
 
-// Scales and biases of groups G0 .. G0 + 3 (4 bf16 per row and tile).
+// Scales and biases of groups G0 .. G0 + B - 1 (B bf16 per row and tile,
+// two per word).
+template <int B>
 struct BlockS {
-  uint2 s[2][2], b[2][2];   // [tile][row]
+  uint32_t s[2][2][B / 2], b[2][2][B / 2];   // [tile][row][word]
 };
-__device__ __forceinline__ void load_scales(BlockS& S, const WTile& w, int ngr, int G0) {
+template <int B>
+__device__ __forceinline__ void load_scales(BlockS<B>& S, const WTile& w, int ngr, int G0) {
 #pragma unroll
   for (int m = 0; m < 2; ++m)
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
-      S.s[m][r] = __ldg(reinterpret_cast<const uint2*>(w.s[m] + r * 8 * ngr + G0));
-      S.b[m][r] = __ldg(reinterpret_cast<const uint2*>(w.b[m] + r * 8 * ngr + G0));
+      const uint16_t* sp = w.s[m] + r * 8 * ngr + G0;
+      const uint16_t* bp = w.b[m] + r * 8 * ngr + G0;
+      if constexpr (B == 4) {
+        const uint2 sv = __ldg(reinterpret_cast<const uint2*>(sp)), bv = __ldg(reinterpret_cast<const uint2*>(bp));
+        S.s[m][r][0] = sv.x; S.s[m][r][1] = sv.y;
+        S.b[m][r][0] = bv.x; S.b[m][r][1] = bv.y;
+      } else {
+        S.s[m][r][0] = __ldg(reinterpret_cast<const uint32_t*>(sp));
+        S.b[m][r][0] = __ldg(reinterpret_cast<const uint32_t*>(bp));
+      }
     }
 }
 
 // Group G (position j of its block) of both tiles against the staged token
 // tile: y[m][r][c] += s * sum (128 + q) x + (b - 128 s) X for row lg4 + 8r
 // of tile m and token column 2lt + c.
-__device__ __forceinline__ void group_step(float (&y)[2][2][2], const uint2 (&a)[2][2], const BlockS& S, int j,
+template <int B>
+__device__ __forceinline__ void group_step(float (&y)[2][2][2], const uint2 (&a)[2][2], const BlockS<B>& S, int j,
                                            const uint4* xr, const float* xsum, int G, int lt) {
   const uint4 xb0 = xr[G * 8], xb1 = xr[G * 8 + 1];
   const float2 X = *reinterpret_cast<const float2*>(xsum + G * kMTok + 2 * lt);
@@ -221,8 +237,8 @@ __device__ __forceinline__ void group_step(float (&y)[2][2][2], const uint2 (&a)
     group_dot(d, a[m][0], a[m][1], xb0, xb1);
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
-      const uint32_t sp = (j < 2) ? S.s[m][r].x : S.s[m][r].y;
-      const uint32_t bp = (j < 2) ? S.b[m][r].x : S.b[m][r].y;
+      const uint32_t sp = S.s[m][r][j >> 1];
+      const uint32_t bp = S.b[m][r][j >> 1];
       const float sc = (j & 1) ? bf16_hi(sp) : bf16_lo(sp);
       const float cb = fmaf(-128.f, sc, (j & 1) ? bf16_hi(bp) : bf16_lo(bp));
       y[m][r][0] = fmaf(cb, X.x, fmaf(sc, d[2 * r], y[m][r][0]));
@@ -237,18 +253,18 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
 
 // The body both kernels share.  tile_of(item, warp, row, lt) -> WTile: the
 // warp's two tiles as seen by a lane that reads row `row` (and row + 8) at
-// byte 8 lt of each group; k_of(item): inputs per row (a multiple of 256);
+// byte 8 lt of each group; k_of(item): inputs per row (a multiple of 64 B);
 // row_of(item) -> a function r -> activation row r of the token tile;
 // store(item, warp, y, lg4, lt): the epilogue.  Shared memory: the staged
 // token tile.
 //
 // Three walks over the same block sequence: the computation; the register
 // loads one block ahead of it (group j of block n + 1 right after group j of
-// block n has been used); and L2 prefetches kPrefetchBlocks ahead, one
-// 128-byte line per lane and block (lane = tile * 16 + row), so the register
-// loads find their lines in L2.
+// block n has been used); and L2 prefetches kPrefetchBlocks ahead, the
+// line of one row per lane and block (lane = tile * 16 + row), so the
+// register loads find their lines in L2.
 constexpr int kPrefetchBlocks = 4;
-template <class TileOf, class KOf, class RowOf, class Store>
+template <int B, class TileOf, class KOf, class RowOf, class Store>
 __device__ __forceinline__ void mid_body(const Geometry& g, const int32_t* offsets, const int32_t* active,
                                          const int32_t* n_active, int blocks_routed, int blocks_shared, int kmax,
                                          uint8_t* msm, TileOf tile_of, KOf k_of, RowOf row_of, Store store) {
@@ -267,7 +283,7 @@ __device__ __forceinline__ void mid_body(const Geometry& g, const int32_t* offse
   Item I = decode_item(g, s_start, n_act, offsets, active, blockIdx.x);
   WTile lw = tile_of(I, warp, lg4, lt);
   int lngr = k_of(I) / kGroup;
-  int lk = 0, lb = 0, lnbat = lngr / kMBlock;
+  int lk = 0, lb = 0, lnbat = lngr / B;
   bool lvalid = true;
   const uint8_t* pq;
   {
@@ -277,11 +293,11 @@ __device__ __forceinline__ void mid_body(const Geometry& g, const int32_t* offse
   int pk = 0, pb = 0, pnbat = lnbat;
   bool pvalid = true;
 
-  uint2 A[kMBlock][2][2];
-  BlockS S;
+  uint2 A[B][2][2];
+  BlockS<B> S;
 #pragma unroll
-  for (int j = 0; j < kMBlock; ++j) load_group(A[j], lw, lngr, j);
-  load_scales(S, lw, lngr, 0);
+  for (int j = 0; j < B; ++j) load_group(A[j], lw, lngr, j);
+  load_scales<B>(S, lw, lngr, 0);
 #define MID_STEP_LOAD()                                                             \
   do {                                                                              \
     if (lvalid && ++lb == lnbat) {                                                  \
@@ -292,7 +308,7 @@ __device__ __forceinline__ void mid_body(const Geometry& g, const int32_t* offse
         const Item n_ = decode_item(g, s_start, n_act, offsets, active, it_);       \
         lw = tile_of(n_, warp, lg4, lt);                                            \
         lngr = k_of(n_) / kGroup;                                                   \
-        lnbat = lngr / kMBlock;                                                     \
+        lnbat = lngr / B;                                                           \
       }                                                                             \
     }                                                                               \
   } while (0)
@@ -306,17 +322,17 @@ __device__ __forceinline__ void mid_body(const Geometry& g, const int32_t* offse
         const Item n_ = decode_item(g, s_start, n_act, offsets, active, it_);       \
         const WTile w_ = tile_of(n_, warp, lane & 15, 0);                           \
         pq = (lane >> 4) ? w_.q[1] : w_.q[0];                                       \
-        pnbat = k_of(n_) / kGroup / kMBlock;                                        \
+        pnbat = k_of(n_) / kGroup / B;                                              \
       }                                                                             \
     }                                                                               \
-    if (pvalid) prefetch_l2(pq + pb * 128);                                         \
+    if (pvalid) prefetch_l2(pq + pb * (B * 32));                                    \
   } while (0)
   MID_STEP_LOAD();
   for (int i = 0; i < kPrefetchBlocks; ++i) MID_STEP_PREFETCH();
 
   for (int k = 0;; ++k) {
     const int K = k_of(I);
-    const int ngr = K / kGroup, nbat = ngr / kMBlock;
+    const int ngr = K / kGroup, nbat = ngr / B;
     if (k > 0) __syncthreads();   // every warp is done with the previous item's staged tile
     stage_tile(row_of(I), I.tn, K, xs, xsum);
     __syncthreads();
@@ -325,12 +341,12 @@ __device__ __forceinline__ void mid_body(const Geometry& g, const int32_t* offse
     for (int b = 0; b < nbat; ++b) {
       MID_STEP_PREFETCH();
       const bool lv = lvalid;
-      const int lG0 = lb * kMBlock;
-      BlockS NS = S;
-      if (lv) load_scales(NS, lw, lngr, lG0);
+      const int lG0 = lb * B;
+      BlockS<B> NS = S;
+      if (lv) load_scales<B>(NS, lw, lngr, lG0);
 #pragma unroll
-      for (int j = 0; j < kMBlock; ++j) {
-        group_step(y, A[j], S, j, xr, xsum, b * kMBlock + j, lt);
+      for (int j = 0; j < B; ++j) {
+        group_step<B>(y, A[j], S, j, xr, xsum, b * B + j, lt);
         if (lv) load_group(A[j], lw, lngr, lG0 + j);
       }
       S = NS;
@@ -350,6 +366,7 @@ __device__ __forceinline__ void mid_body(const Geometry& g, const int32_t* offse
 // entry pos (token t = perm[pos] / k) and h_s[t] for the shared expert.
 // Warp w: the gate and up rows of features blk * 128 + 16 w .. + 15.
 // ---------------------------------------------------------------------------
+template <int B>
 __global__ void __launch_bounds__(kMThreads, 2) mid_gateup_kernel(
     Geometry g, LayerPtr L, const uint16_t* __restrict__ x, const int32_t* __restrict__ offsets,
     const int32_t* __restrict__ perm, const int32_t* __restrict__ active, const int32_t* __restrict__ n_active,
@@ -382,7 +399,7 @@ __global__ void __launch_bounds__(kMThreads, 2) mid_gateup_kernel(
               float_to_bf16_bits(silu(y[0][r][c]) * y[1][r][c]);
     }
   };
-  mid_body(g, offsets, active, n_active, g.I / kMGateUpRows, g.Is / kMGateUpRows, g.H, msm, tile_of, k_of, row_of,
+  mid_body<B>(g, offsets, active, n_active, g.I / kMGateUpRows, g.Is / kMGateUpRows, g.H, msm, tile_of, k_of, row_of,
            store);
 }
 
@@ -393,6 +410,7 @@ __global__ void __launch_bounds__(kMThreads, 2) mid_gateup_kernel(
 // out_t = sum_j w[t,j] Y[inv_perm[t*k+j]] + sigma_t Y[T*k+t] in that order.
 // Warp w: dims blk * 256 + 32 w .. + 31 (two tiles of 16).
 // ---------------------------------------------------------------------------
+template <int B>
 __global__ void __launch_bounds__(kMThreads, 2) mid_down_kernel(
     Geometry g, LayerPtr L, const uint16_t* __restrict__ h, const uint16_t* __restrict__ h_s,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ active, const int32_t* __restrict__ n_active,
@@ -424,16 +442,16 @@ __global__ void __launch_bounds__(kMThreads, 2) mid_down_kernel(
             Y[(row0 + col) * g.H + d0 + 16 * m + lg4 + 8 * r] = float_to_bf16_bits(y[m][r][c]);
     }
   };
-  mid_body(g, offsets, active, n_active, blocks, blocks, max(g.I, g.Is), msm, tile_of, k_of, row_of, store);
+  mid_body<B>(g, offsets, active, n_active, blocks, blocks, max(g.I, g.Is), msm, tile_of, k_of, row_of, store);
 }
 
 namespace {
 
-// Resident CTAs of a mid-size kernel on this device (cached per kernel,
-// device and shared-memory size).
+// Resident CTAs of a mid-size kernel on this device (cached per kernel
+// instance, device and shared-memory size).
 int resident_ctas(int which, const void* func, int smem) {
-  static int cache[2][16] = {};
-  static int cache_smem[2][16] = {};
+  static int cache[4][16] = {};
+  static int cache_smem[4][16] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16) return 0;
   if (cache[which][dev] > 0 && cache_smem[which][dev] == smem) return cache[which][dev];
@@ -460,38 +478,71 @@ int max_items(const Geometry& g, int blocks_routed, int blocks_shared) {
 // Shared memory: the staged token tile for rows of up to kmax inputs.
 int mid_smem(int kmax) { return kMTok * (kmax / 8 + 1) * 16 + kMTok * (kmax / kGroup) * 4; }
 
+bool aligned8(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 7u) == 0; }
+
+// Blocks of 4 groups when every row of the launch has a multiple of 4 groups
+// and the scale/bias stacks allow 8-byte loads (rows and expert strides are
+// then multiples of 8 bytes too), else blocks of 2.
+bool blocks_of_4(std::initializer_list<int> ngrs, std::initializer_list<const QMatPtr*> mats) {
+  for (int n : ngrs)
+    if (n % 4) return false;
+  for (const QMatPtr* m : mats)
+    if (!aligned8(m->s) || !aligned8(m->b)) return false;
+  return true;
+}
+
+template <int B>
+cudaError_t launch_gateup_b(int which, const Geometry& g, const LayerPtr& L, const uint16_t* x,
+                            const int32_t* offsets, const int32_t* perm, const int32_t* active,
+                            const int32_t* n_active, uint16_t* h, uint16_t* h_s, cudaStream_t s) {
+  const int smem = mid_smem(g.H);
+  const void* fn = reinterpret_cast<const void*>(mid_gateup_kernel<B>);
+  cudaError_t e = ensure_smem(fn, smem);
+  if (e != cudaSuccess) return e;
+  const int res = resident_ctas(which, fn, smem);
+  if (res <= 0) return cudaErrorInvalidConfiguration;
+  const int grid = max(1, min(res, max_items(g, g.I / kMGateUpRows, g.Is / kMGateUpRows)));
+  return launch_pdl(mid_gateup_kernel<B>, dim3(grid), dim3(kMThreads), smem, s, g, L, x, offsets, perm, active,
+                    n_active, h, h_s);
+}
+
+template <int B>
+cudaError_t launch_down_b(int which, const Geometry& g, const LayerPtr& L, const uint16_t* h, const uint16_t* h_s,
+                          const int32_t* offsets, const int32_t* active, const int32_t* n_active, uint16_t* Y,
+                          cudaStream_t s) {
+  const int smem = mid_smem(max(g.I, g.Is));
+  const void* fn = reinterpret_cast<const void*>(mid_down_kernel<B>);
+  cudaError_t e = ensure_smem(fn, smem);
+  if (e != cudaSuccess) return e;
+  const int res = resident_ctas(which, fn, smem);
+  if (res <= 0) return cudaErrorInvalidConfiguration;
+  const int blocks = g.H / kMDownRows;
+  const int grid = max(1, min(res, max_items(g, blocks, blocks)));
+  return launch_pdl(mid_down_kernel<B>, dim3(grid), dim3(kMThreads), smem, s, g, L, h, h_s, offsets, active,
+                    n_active, Y);
+}
+
 }  // namespace
 
 bool mid_decode_supported(const Geometry& g) {
-  return g.T >= 1 && g.T <= 64 && g.H % 256 == 0 && g.I % 256 == 0 && g.Is % 256 == 0 && g.H <= 8192 &&
-         g.I <= 2048 && g.Is <= 2048;
+  return g.T >= 1 && g.T <= 64 && g.H % kMDownRows == 0 && g.I % kMGateUpRows == 0 && g.Is % kMGateUpRows == 0 &&
+         g.H <= 8192 && g.I <= 2048 && g.Is <= 2048;
 }
 
 cudaError_t launch_mid_gateup(const Geometry& g, const LayerPtr& L, const uint16_t* x, const int32_t* offsets,
                               const int32_t* perm, const int32_t* active, const int32_t* n_active, uint16_t* h,
                               uint16_t* h_s, cudaStream_t s) {
-  const int smem = mid_smem(g.H);
-  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(mid_gateup_kernel), smem);
-  if (e != cudaSuccess) return e;
-  const int res = resident_ctas(0, reinterpret_cast<const void*>(mid_gateup_kernel), smem);
-  if (res <= 0) return cudaErrorInvalidConfiguration;
-  const int grid = max(1, min(res, max_items(g, g.I / kMGateUpRows, g.Is / kMGateUpRows)));
-  return launch_pdl(mid_gateup_kernel, dim3(grid), dim3(kMThreads), smem, s, g, L, x, offsets, perm, active,
-                    n_active, h, h_s);
+  if (blocks_of_4({g.H / kGroup}, {&L.gate, &L.up, &L.sh_gate, &L.sh_up}))
+    return launch_gateup_b<4>(0, g, L, x, offsets, perm, active, n_active, h, h_s, s);
+  return launch_gateup_b<2>(1, g, L, x, offsets, perm, active, n_active, h, h_s, s);
 }
 
 cudaError_t launch_mid_down(const Geometry& g, const LayerPtr& L, const uint16_t* h, const uint16_t* h_s,
                             const int32_t* offsets, const int32_t* active, const int32_t* n_active, uint16_t* Y,
                             cudaStream_t s) {
-  const int smem = mid_smem(max(g.I, g.Is));
-  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(mid_down_kernel), smem);
-  if (e != cudaSuccess) return e;
-  const int res = resident_ctas(1, reinterpret_cast<const void*>(mid_down_kernel), smem);
-  if (res <= 0) return cudaErrorInvalidConfiguration;
-  const int blocks = g.H / kMDownRows;
-  const int grid = max(1, min(res, max_items(g, blocks, blocks)));
-  return launch_pdl(mid_down_kernel, dim3(grid), dim3(kMThreads), smem, s, g, L, h, h_s, offsets, active,
-                    n_active, Y);
+  if (blocks_of_4({g.I / kGroup, g.Is / kGroup}, {&L.down, &L.sh_down}))
+    return launch_down_b<4>(2, g, L, h, h_s, offsets, active, n_active, Y, s);
+  return launch_down_b<2>(3, g, L, h, h_s, offsets, active, n_active, Y, s);
 }
 
 }  // namespace moe
