@@ -23,14 +23,17 @@
 //
 // Weight streaming.  The packed codes go from global memory straight into
 // the MMA operand registers (8 bytes per lane per row and group): a warp
-// holds the next 4 groups of both tiles in flight (group j of the next block
-// of 4 is loaded right after group j of the current block has been used),
-// running on into the CTA's next item, whose weights do not depend on the
-// activations; the scales and biases of the next block (one 8-byte load per
-// row) are loaded a block ahead.  Shared memory carries only the
-// activations, read conflict-free: token rows are padded by 16 bytes and the
-// group sums are stored token-minor, so a lane's two sums are one 8-byte
-// read.
+// holds the next block of B groups (B = 4, or 2 where a row has 2 mod 4
+// groups or the scale stacks are only 4-byte aligned) of both tiles in
+// flight (group j of the next block is loaded right after group j of the
+// current block has been used), running on into the CTA's next item, whose
+// weights do not depend on the activations; the scales and biases of the
+// next block (one load per row) are loaded a block ahead, and L2 prefetches
+// run 4 blocks ahead.  Shared memory carries only the activations, read
+// conflict-free: token rows are padded by 16 bytes and the group sums are
+// stored token-minor, so a lane's two sums are one 8-byte read.  The kernels
+// are issue-bound rather than memory-bound: the dequantising AND-OR/shift
+// work and the MMA -> scale -> accumulate chains dominate.
 #include <initializer_list>
 
 #include "common.cuh"
@@ -44,9 +47,6 @@ constexpr int kMThreads = kMWarps * 32;
 constexpr int kMGateUpRows = 16 * kMWarps;   // features of a gate/up item
 constexpr int kMDownRows = 32 * kMWarps;     // output dims of a down item
 constexpr int kMTok = 8;                     // tokens of an item: the n8 column tile
-// Groups of 64 inputs per pipeline block: 4 when every row has a multiple of
-// 4 groups and the scale/bias stacks are 8-byte aligned (one 8-byte load per
-// row and block), else 2 (one 4-byte load).
 
 __device__ __forceinline__ QMatPtr expert_qmat(const QMatPtr& stack, int e, size_t rows, size_t cols) {
   return QMatPtr{stack.q + static_cast<size_t>(e) * rows * (cols / 8),
