@@ -53,8 +53,11 @@ def run_layer(layer_np, x_bits: np.ndarray, entry: str = "forward", dev_layer=No
     return res
 
 
-def assert_routing_exact(gpu: dict, ref: dict, tokens=None):
-    """Routing must match the oracle bit for bit on screened inputs."""
+def assert_routing_exact(gpu: dict, ref: dict, tokens=None, w_atol: float = 2e-6):
+    """Routing must match the oracle bit for bit on screened inputs.
+
+    w_atol bounds the FP32 weights and gates; the default is set for H = 2048,
+    and the error of an FP32 dot product grows with its length H."""
     idx = ref["topk_idx"]
     np.testing.assert_array_equal(gpu["topk_idx"], idx)
     np.testing.assert_array_equal(gpu["counts"], ref["counts"])
@@ -62,8 +65,8 @@ def assert_routing_exact(gpu: dict, ref: dict, tokens=None):
     np.testing.assert_array_equal(gpu["perm"], ref["perm"])
     np.testing.assert_array_equal(gpu["inv_perm"], ref["inv_perm"])
     # weights: FP32 softmax over the chosen FP32 logits vs float64
-    np.testing.assert_allclose(gpu["topk_w"], ref["topk_w"], rtol=0, atol=2e-6)
-    np.testing.assert_allclose(gpu["sigma"], ref["sigma"], rtol=0, atol=2e-6)
+    np.testing.assert_allclose(gpu["topk_w"], ref["topk_w"], rtol=0, atol=w_atol)
+    np.testing.assert_allclose(gpu["sigma"], ref["sigma"], rtol=0, atol=w_atol)
     assert np.all(np.abs(gpu["topk_w"].sum(axis=1) - 1.0) < 1e-6)
 
 

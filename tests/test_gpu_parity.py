@@ -201,6 +201,24 @@ def test_mid_size_path_second_geometry(T, zipf):
         assert_output_close(gpu["out"], ref["out"])
 
 
+# The widest layer the ABI takes (H = 8192: a 131 KB staged token tile, one
+# CTA per SM on the mid-size path) with I != I_shared and 2 groups per down
+# row (pipeline blocks of 2); T = 65 runs the tensor-core path on it.
+WIDE = dataclasses.replace(TINY, H=8192, E=16, k=4, I=128, I_s=256)
+
+
+@pytest.mark.parametrize("T", [7, 64, 65])
+def test_widest_layer(T):
+    lay, x, _ = workload(90 + T, T, WIDE)
+    ref = moe_ref.moe_layer(x, lay, WIDE.k)
+    gpu = run_layer(lay, x)
+    assert gpu["status"] == 0
+    # the logits are FP32 sums of 8192 products, 4x the default's length: the
+    # weight tolerance scales with H (worst-case linear growth), times 2
+    assert_routing_exact(gpu, ref, w_atol=2e-6 * (WIDE.H / 2048) * 2)
+    assert_output_close(gpu["out"], ref["out"])
+
+
 def test_rmsnorm_matches_oracle():
     rng = np.random.default_rng(9)
     y_bits = synth.to_bf16_bits(rng.normal(0, 0.05, size=(37, 2048)))
