@@ -99,6 +99,8 @@ def parse_args(argv=None):
                     help="profiling probe: only `--probe-calls` moe_forward calls of T tokens on two resident "
                          "layers (~0.9 GB), no timing, no JSON line")
     ap.add_argument("--probe-calls", type=int, default=4)
+    ap.add_argument("--probe-stack", type=int, default=0,
+                    help="with --probe-T: call moe_forward_stack on this many resident layers instead")
     return ap.parse_args(argv)
 
 
@@ -868,13 +870,18 @@ def run_probe(a):
     from bit_quantized_expert_route_b200 import moe, synth
     dev = torch.device("cuda", 0)
     dims = synth.Dims()
+    n_layers = a.probe_stack if a.probe_stack else 2
     layers = [moe.MoELayer.from_tensors(dims, synth.make_layer_on_device(300 + l, l, dims, dev, False))
-              for l in range(2)]
+              for l in range(n_layers)]
     x = synth.make_x_on_device(7, a.probe_T, dims.H, dev)
     out = torch.empty_like(x)
     ws = moe.alloc_workspace(layers[0], a.probe_T, dev)
+    stack = moe.LayerStack(layers)
     for i in range(a.probe_calls):
-        moe.moe_forward(layers[i % 2], x, out, ws)
+        if a.probe_stack:
+            moe.moe_forward_stack(stack, x, out, ws, eps=EPS)
+        else:
+            moe.moe_forward(layers[i % 2], x, out, ws)
     torch.cuda.synchronize()
     st = moe.moe_get_status(ws)
     print(f"probe T={a.probe_T} calls={a.probe_calls} status={st}")
