@@ -57,10 +57,11 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(
     uint16_t* __restrict__ norm_out, float eps, const int* status) {
   pdl_wait();
   pdl_launch_dependents();
-  // a recorded error means inv_perm may hold entries no kernel wrote: skip
-  if (*reinterpret_cast<volatile const int*>(status) != 0) return;
   __shared__ float part[kCombThreads / 32];
   const int t = blockIdx.x;
+  // the status word is read together with the routing of the token; a
+  // recorded error means inv_perm may hold entries no kernel wrote: skip
+  const int st = *reinterpret_cast<volatile const int*>(status);
   int pos[kMaxK];
   float w[kMaxK];
 #pragma unroll
@@ -69,6 +70,7 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(
     w[j] = j < k ? __ldg(topk_w + static_cast<size_t>(t) * k + j) : 0.f;
   }
   const float sg = __ldg(sigma + t);
+  if (st != 0) return;
   const size_t shared_row = static_cast<size_t>(T) * k + t;
   uint4 keep[2 * kCombMaxIters];      // this thread's bf16 outputs, kept for the normalisation
   float ss = 0.f;
@@ -187,12 +189,14 @@ __global__ void __launch_bounds__(kGatherWarps * 32) gather_k8_kernel(const uint
                                                                     uint4* __restrict__ xg, const int* status) {
   pdl_wait();
   pdl_launch_dependents();
-  // a recorded error means perm may hold entries no kernel wrote: skip
-  if (*reinterpret_cast<volatile const int*>(status) != 0) return;
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * kGatherWarps + (threadIdx.x >> 5);
   if (row >= rows) return;
+  // the status word is read together with the row's token; a recorded error
+  // means perm may hold entries no kernel wrote: skip
+  const int st = *reinterpret_cast<volatile const int*>(status);
   const int t = row < Tk ? __ldg(perm + row) / k : row - Tk;
+  if (st != 0) return;
   const uint4* src = x + static_cast<size_t>(t) * h8;
   uint4* dst = xg + static_cast<size_t>(row) * h8;
   for (int c0 = 0; c0 < h8; c0 += 32 * kGatherPieces) {
