@@ -3,6 +3,7 @@
 // except in moe_get_status and moe_forward_host.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdint>
 #include <cstring>
@@ -460,7 +461,13 @@ int moe_workspace_size(const moe_layer_desc* layer, int T_max, size_t* bytes) {
   const int st = validate_layer(layer);
   if (st != MOE_OK) return st;
   if (T_max < 1 || T_max > kMaxT) return MOE_ERR_INVALID_ARG;
-  *bytes = ws_layout(layer, T_max).total;
+  // The layout grows with T inside each regime, but a smaller T can need
+  // more: T <= 8 adds the fused kernel's exchange words and T <= 64 the small
+  // router's logits.  A workspace must serve every T <= T_max.
+  size_t need = ws_layout(layer, T_max).total;
+  for (int t : {kFusedMaxTStack, kDecodeMaxT})
+    if (t < T_max) need = std::max(need, ws_layout(layer, t).total);
+  *bytes = need;
   return MOE_OK;
 }
 

@@ -68,6 +68,23 @@ def test_workspace_size_monotone(lib):
     assert sizes[4] >= 9 * 4096 * 2048 * 2
 
 
+@pytest.mark.parametrize("over", [dict(), dict(H=256, E=16, k=2, I=128, I_shared=128),
+                                  dict(H=1024, I=256, I_shared=256)])
+def test_workspace_for_t_max_serves_every_smaller_t(lib, over):
+    """The header promises a workspace for any T <= T_max.  The layout of a
+    call grows with T within each kernel set, but T <= 8 also holds the fused
+    decode kernel's exchange words and T <= 64 the small router's logits, so
+    the size for T_max = 9 must still cover a call with T = 8: the reported
+    sizes never decrease with T."""
+    L = fake_layer(**over)
+    prev = 0
+    for T in list(range(1, 140)) + [255, 256, 257, 4095, 4096, 4097]:
+        st, n = ws_size(lib, L, T)
+        assert st == 0
+        assert n >= prev, (T, n, prev)
+        prev = n
+
+
 @pytest.mark.parametrize("over,code", [
     (dict(bits=8), moe.MOE_ERR_UNSUPPORTED),
     (dict(group_size=128), moe.MOE_ERR_UNSUPPORTED),
