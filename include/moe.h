@@ -43,10 +43,11 @@
  * between calls except cached kernel attributes.  Two calls must not share a
  * workspace concurrently.  A workspace must be zero-filled once before its
  * first use (e.g. cudaMemset of the whole buffer).  Its first 256 bytes are a
- * control block (status word, a CTA counter, the fused decode kernel's exit
- * counter and launch epoch); the library leaves the status word zero after
- * every call except for a recorded error status, which moe_get_status
- * clears.  The fused decode kernel's CTAs exchange values through 64-bit
+ * control block (status word, the small-T router's completion counters, the
+ * fused decode kernel's exit counter and launch epoch); the library leaves
+ * the counters and the status word zero after every call except for a
+ * recorded error status, which moe_get_status clears together with the
+ * counters.  The fused decode kernel's CTAs exchange values through 64-bit
  * words of the workspace tagged with (launch epoch, layer): a stale word is
  * never taken for a current one, except one last written exactly a multiple
  * of 2^26 launches earlier on the same workspace and not rewritten since.
