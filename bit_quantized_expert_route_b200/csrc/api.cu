@@ -71,7 +71,7 @@ constexpr int kDecodeMaxT = 64;
 // layers: T=3 38.9 vs 39.8 us, T=4 46.6 vs 40.9, T=8 81.1 vs 59.1).
 constexpr int kFusedMaxT = 3;       // single-layer calls
 constexpr int kFusedMaxTStack = 8;  // moe_forward_stack
-constexpr int kMidMaxT = 64;        // tokens the mid-size decode path takes
+constexpr int kMidMaxT = 128;       // tokens the mid-size decode path takes (moe_forward)
 constexpr int kMaxT = 65536;
 constexpr int kMaxStackLayers = 1024;
 constexpr size_t kAlign = 256;
@@ -113,7 +113,7 @@ WsLayout ws_layout(const moe_layer_desc* d, int T) {
   w.n_chunks = take(4);
   w.active = take(static_cast<size_t>(d->E + 1) * 4);
   w.n_active = take(4);
-  w.logits = take(static_cast<size_t>(T <= kDecodeMaxT ? T : 0) * (d->E + 1) * 4);
+  w.logits = take(static_cast<size_t>(T <= kMidMaxT ? T : 0) * (d->E + 1) * 4);
   w.h = take(n * d->I * 2);
   w.h_s = take(static_cast<size_t>(T) * d->I_shared * 2);
   w.Y = take((n + T) * d->H * 2);   // also holds the gate/up GEMM's grouped token rows before the down GEMM
@@ -211,14 +211,15 @@ inline void mark(Tracer* tr, cudaStream_t s) {
   if (tr) tr->mark(s);
 }
 
-// Routing of T tokens.  T <= 64 without `grouped`: one launch of the small-T
-// router (routing outputs and active list only).  Otherwise the tensor-core
-// router and the counting-sort passes, which also build the chunk list the
-// grouped GEMMs walk.
+// Routing of T tokens.  T <= 64 without `grouped` (T <= 128 for the
+// mid-size decode path): one launch of the small-T router (routing outputs
+// and active list only).  Otherwise the tensor-core router and the
+// counting-sort passes, which also build the chunk list the grouped GEMMs
+// walk.
 int enqueue_route(const moe_layer_desc* d, const uint16_t* x, int T, const Bufs& b, cudaStream_t s,
-                  Tracer* tr = nullptr, bool grouped = false) {
+                  Tracer* tr = nullptr, bool grouped = false, int small_max_t = kDecodeMaxT) {
   mark(tr, s);
-  if (T <= kDecodeMaxT && !grouped) {
+  if (T <= small_max_t && !grouped) {
     const RoutingPtrs rp{b.topk_idx, b.topk_w, b.sigma, b.counts, b.offsets, b.perm, b.inv_perm};
     const cudaError_t e = launch_route_small(x, layer_ptrs(d), T, d->H, d->I, d->I_shared, d->E, d->k,
                                              b.at<float>(b.w.logits), b.at<unsigned>(b.w.counter), rp,
@@ -298,7 +299,7 @@ int enqueue_fused(const moe_layer_desc* d, const uint16_t* x, int T, uint16_t* o
 // NULL).
 int enqueue_mid(const moe_layer_desc* d, const uint16_t* x, int T, uint16_t* out, const Bufs& b, cudaStream_t s,
                 Tracer* tr = nullptr, uint16_t* norm_out = nullptr, float eps = 0.f) {
-  int st = enqueue_route(d, x, T, b, s, tr);
+  int st = enqueue_route(d, x, T, b, s, tr, /*grouped=*/false, kMidMaxT);
   if (st != MOE_OK) return st;
   const Geometry g{T, d->H, d->I, d->I_shared, d->E, d->k};
   const LayerPtr L = layer_ptrs(d);
@@ -465,7 +466,7 @@ int moe_workspace_size(const moe_layer_desc* layer, int T_max, size_t* bytes) {
   // more: T <= 8 adds the fused kernel's exchange words and T <= 64 the small
   // router's logits.  A workspace must serve every T <= T_max.
   size_t need = ws_layout(layer, T_max).total;
-  for (int t : {kFusedMaxTStack, kDecodeMaxT})
+  for (int t : {kFusedMaxTStack, kMidMaxT})
     if (t < T_max) need = std::max(need, ws_layout(layer, t).total);
   *bytes = need;
   return MOE_OK;

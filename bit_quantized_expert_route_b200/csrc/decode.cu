@@ -1,4 +1,4 @@
-// Decode path for steps of up to 64 tokens that the fused kernel does not
+// Decode path for steps of up to 128 tokens that the fused kernel does not
 // take: the tokens of the step spread over many experts with a few tokens
 // each, so the layer is bound by streaming the active experts' packed weights
 // ("Perplexity's Lily: ...", section "How It Works: Prefill and Decode
@@ -525,7 +525,7 @@ cudaError_t launch_down_b(int which, const Geometry& g, const LayerPtr& L, const
 }  // namespace
 
 bool mid_decode_supported(const Geometry& g) {
-  return g.T >= 1 && g.T <= 64 && g.H % kMDownRows == 0 && g.I % kMGateUpRows == 0 && g.Is % kMGateUpRows == 0 &&
+  return g.T >= 1 && g.T <= 128 && g.H % kMDownRows == 0 && g.I % kMGateUpRows == 0 && g.Is % kMGateUpRows == 0 &&
          g.H <= 8192 && g.I <= 2048 && g.Is <= 2048;
 }
 

@@ -87,7 +87,7 @@ cudaError_t launch_router(const uint16_t* x, const uint16_t* w_router, const flo
 // kSmallMaxGroups) words: word 0 counts finished token groups, word
 // kSmallGroupCounter + y the finished CTAs of token group y.
 constexpr int kSmallTB = 8;
-constexpr int kSmallMaxGroups = 8;
+constexpr int kSmallMaxGroups = 16;
 constexpr int kSmallGroupCounter = 16;
 
 // route.cu

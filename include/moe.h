@@ -185,7 +185,7 @@ MOE_API int moe_route(const moe_layer_desc* layer, const moe_bf16* x, int T, moe
  *   T <= 3 (T <= 8 inside moe_forward_stack) with H = 1024 or 2048, I and
  *     I_shared whole groups, 16-byte aligned scale and bias stacks and at
  *     most E + 1 SMs: the single-launch fused decode kernel (see moe_decode);
- *   T <= 64 with H a multiple of 256 and I, I_shared multiples of 128 (the
+ *   T <= 128 with H a multiple of 256 and I, I_shared multiples of 128 (the
  *     mid-size decode path): the one-launch small-T router, then gate/up +
  *     SwiGLU and down as GEMVs over the active experts only (warp-level
  *     mma.sync on 8-token tiles, codes streamed from global memory into the

@@ -240,11 +240,13 @@ def test_rmsnorm_matches_oracle():
 
 @pytest.mark.parametrize("T,entry", [(1, "forward"), (2, "forward"), (3, "forward"), (5, "forward"),
                                      (8, "forward"), (9, "forward"), (16, "forward"), (33, "forward"),
-                                     (64, "forward"), (3, "decode"), (8, "decode"), (9, "decode"), (64, "decode")])
+                                     (64, "forward"), (65, "forward"), (128, "forward"), (3, "decode"),
+                                     (8, "decode"), (9, "decode"), (64, "decode")])
 def test_full_decode(T, entry):
     # T <= 3 runs the single-launch fused decode kernel (both entries); 4 <= T
-    # <= 64 the mid-size decode path (small-T router, mma.sync GEMVs over the
-    # active experts in 8-token tiles, fixed-order combine)
+    # <= 128 the mid-size decode path (small-T router, mma.sync GEMVs over the
+    # active experts in 8-token tiles, fixed-order combine); moe_decode takes
+    # T <= 64
     lay, x, _ = workload(10 + T, T, FULL)
     ref = moe_ref.moe_layer(x, lay, FULL.k)
     gpu = run_layer(lay, x, entry=entry)
