@@ -93,6 +93,8 @@ def parse_args(argv=None):
     ap.add_argument("--decode-layers", type=int, default=40, help="resident layers of the decode and sweep stacks")
     ap.add_argument("--sweep-T", type=str, default=",".join(str(t) for t in SWEEP_T))
     ap.add_argument("--sweep-reps", type=int, default=3, help="timed stack calls per sweep point")
+    ap.add_argument("--no-mid", action="store_true", help="skip the single-layer mid-size decode workload")
+    ap.add_argument("--mid-T", type=str, default="16,64", help="token counts of the mid-size decode workload")
     ap.add_argument("--oracle-sweep-T", type=str, default=",".join(str(t) for t in SWEEP_T),
                     help="sweep points at which the CPU oracle is timed (layer 0)")
     ap.add_argument("--probe-T", type=int, default=0,
@@ -461,6 +463,50 @@ def decode_phase(a, world, rank, dev, dims, peaks, peak_src, dl):
     return res
 
 
+# ------------------------------------------------- mid-size decode (single layers) ---
+
+def decode_mid_phase(a, world, rank, dev, dims, peaks, peak_src, dl):
+    """Single-layer calls at 4 <= T <= 128 (the mid-size decode path) through the resident layers, as a CUDA
+    graph of one call per layer; HBM roofline over the distinct experts each call's routing touches."""
+    import torch
+    from bit_quantized_expert_route_b200 import moe, synth
+    NL = len(dl)
+    out_rows = {}
+    for T in [int(t) for t in a.mid_T.split(",") if t]:
+        x = synth.make_x_on_device(9000 + 10 * T + rank, T, dims.H, dev)
+        out = torch.empty_like(x)
+        ws = moe.alloc_workspace(dl[0], T, dev)
+        stages = moe.moe_forward_profiled(dl[0], x, out, ws)
+        graph = capture_graph(lambda: [moe.moe_forward(dl[l], x, out, ws) for l in range(NL)])
+        graph.replay()
+        reps = max(1, a.sweep_reps)
+        g_ms = timed_loop(lambda i: graph.replay(), reps, world) / reps
+        del graph
+        # the distinct experts of each layer's routing of x (+ the shared expert)
+        r = moe.Routing(T, dims.E, dims.k, dev)
+        distinct = 0
+        for l in range(NL):
+            moe.moe_route(dl[l], x, r, ws)
+            distinct += int((r.counts > 0).sum().item()) + 1
+        assert moe.moe_get_status(ws) == 0
+        layer_ms = g_ms / NL
+        out_rows[str(T)] = {
+            "layer_us": round(layer_ms * 1e3, 3), "us_per_token": round(layer_ms * 1e3 / T, 4),
+            "tokens_per_s": round(whole_job_rate(T, world, layer_ms), 1),
+            "kernel_set": "mid-size decode" if len(stages) == len(moe.MID_DECODE_STAGES) else
+                          ("fused decode" if len(stages) == 1 else "tensor-core"),
+            "distinct_experts_per_layer": round(distinct / NL, 2),
+            "roofline": hbm_roofline("whole layer (router, gate/up, down, combine)", distinct * expert_bytes(dims),
+                                     g_ms, peaks, peak_src)}
+    torch.cuda.empty_cache()
+    return {"workload": f"single-layer calls (moe_forward), {NL} distinct resident layers, random inputs "
+                        f"(uniform routing), H={dims.H}, E={dims.E}, k={dims.k}, I={dims.I}",
+            "timing": "one call per layer captured as one CUDA graph and replayed; per-layer time = graph time / layers",
+            "roofline_note": "HBM bytes = the distinct experts each call's routing touches (routed + shared) x "
+                             "1,769,472 B, over the whole layer's time",
+            "points": out_rows}
+
+
 # ------------------------------------------------------------ sweep (CFG4) ---
 
 def sweep_phase(a, world, rank, dev, dims, peaks, peak_src, dl):
@@ -780,6 +826,8 @@ def run_ours(a):
         workloads["decode"] = decode_phase(a, world, rank, dev, dims, peaks, peak_src, dl)
     if not a.no_sweep and not a.decode_only:
         workloads["sweep"] = sweep_phase(a, world, rank, dev, dims, peaks, peak_src, dl)
+    if not a.no_mid and not a.decode_only and dl is not None:
+        workloads["decode_mid"] = decode_mid_phase(a, world, rank, dev, dims, peaks, peak_src, dl)
     del dl
     torch.cuda.empty_cache()
     if not a.no_tiny and not a.decode_only:
