@@ -29,7 +29,8 @@
 // current block has been used), running on into the CTA's next item, whose
 // weights do not depend on the activations; the scales and biases of the
 // next block (one load per row) are loaded a block ahead, and L2 prefetches
-// run 4 blocks ahead.  Shared memory carries only the activations, read
+// run a block further (deeper prefetches brought lines that were evicted
+// before use: 309 MB read for 263 MB of weights at T=64, 3.5% slower).  Shared memory carries only the activations, read
 // conflict-free: token rows are padded by 16 bytes and the group sums are
 // stored token-minor, so a lane's two sums are one 8-byte read.  The kernels
 // are issue-bound rather than memory-bound: the dequantising AND-OR/shift
@@ -263,7 +264,7 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
 // block n has been used); and L2 prefetches kPrefetchBlocks ahead, the
 // line of one row per lane and block (lane = tile * 16 + row), so the
 // register loads find their lines in L2.
-constexpr int kPrefetchBlocks = 4;
+constexpr int kPrefetchBlocks = 1;
 template <int B, class TileOf, class KOf, class RowOf, class Store>
 __device__ __forceinline__ void mid_body(const Geometry& g, const int32_t* offsets, const int32_t* active,
                                          const int32_t* n_active, int blocks_routed, int blocks_shared, int kmax,
