@@ -333,7 +333,7 @@ __global__ void __launch_bounds__(kGroupThreads) group_fused_kernel(
 constexpr int kSmallWarps = 8;
 constexpr int kSmallRows = 16;          // router rows per CTA (the MMA's M)
 constexpr int kSmallLoads = 8;          // loads per thread in flight together
-constexpr int kSmallKSteps = 4;         // 16-wide K steps whose loads are in flight together
+constexpr int kSmallKSteps = 8;         // 16-wide K steps whose loads are in flight together
 
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                                uint32_t b0, uint32_t b1) {
