@@ -65,12 +65,13 @@ using namespace moe;
 
 constexpr int kDecodeMaxT = 64;
 // Tokens the fused decode kernel takes: a stack of layers runs up to 40 of
-// them per cooperative launch and wins up to T = 8; a single layer pays the
-// cooperative launch and the kernel's fixed phases every call, and the
-// mid-size path is faster from T = 4 (measured per layer, 40 distinct
-// layers: T=3 38.9 vs 39.8 us, T=4 46.6 vs 40.9, T=8 81.1 vs 59.1).
+// them per cooperative launch and wins up to T = 7 (T=4 28.4 vs 37.3 us per
+// layer, T=6 35.7 vs 39.5, T=8 42.2 vs 40.6 on the mid-size path); a single
+// layer pays the cooperative launch and the kernel's fixed phases every call,
+// and the mid-size path is faster from T = 4 (T=3 38.9 vs 39.8 us, T=4 46.6
+// vs 40.9, T=8 81.1 vs 59.1).
 constexpr int kFusedMaxT = 3;       // single-layer calls
-constexpr int kFusedMaxTStack = 8;  // moe_forward_stack
+constexpr int kFusedMaxTStack = 7;  // moe_forward_stack
 constexpr int kMidMaxT = 128;       // tokens the mid-size decode path takes (moe_forward)
 constexpr int kMaxT = 65536;
 constexpr int kMaxStackLayers = 1024;

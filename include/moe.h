@@ -182,7 +182,7 @@ MOE_API int moe_route(const moe_layer_desc* layer, const moe_bf16* x, int T, moe
  * x, out: device bf16 [T, H], 16-byte aligned, not overlapping.
  * r: optional (NULL = keep routing in the workspace).
  * 1 <= T <= 65536.  Three kernel sets, chosen by T:
- *   T <= 3 (T <= 8 inside moe_forward_stack) with H = 1024 or 2048, I and
+ *   T <= 3 (T <= 7 inside moe_forward_stack) with H = 1024 or 2048, I and
  *     I_shared whole groups, 16-byte aligned scale and bias stacks and at
  *     most E + 1 SMs: the single-launch fused decode kernel (see moe_decode);
  *   T <= 128 with H a multiple of 256 and I, I_shared multiples of 128 (the

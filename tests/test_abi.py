@@ -72,9 +72,9 @@ def test_workspace_size_monotone(lib):
                                   dict(H=1024, I=256, I_shared=256)])
 def test_workspace_for_t_max_serves_every_smaller_t(lib, over):
     """The header promises a workspace for any T <= T_max.  The layout of a
-    call grows with T within each kernel set, but T <= 8 also holds the fused
-    decode kernel's exchange words and T <= 64 the small router's logits, so
-    the size for T_max = 9 must still cover a call with T = 8: the reported
+    call grows with T within each kernel set, but T <= 7 also holds the fused
+    decode kernel's exchange words and T <= 128 the small router's logits, so
+    the size for T_max = 8 must still cover a call with T = 7: the reported
     sizes never decrease with T."""
     L = fake_layer(**over)
     prev = 0

@@ -94,12 +94,12 @@ def test_router_wait_runs_out_and_the_next_call_is_correct():
     _assert_next_call_correct(lay, x, L, xd, out, ws)
 
 
-@pytest.mark.parametrize("T,entry", [(1, "forward"), (3, "forward"), (8, "stack")])
+@pytest.mark.parametrize("T,entry", [(1, "forward"), (3, "forward"), (7, "stack")])
 def test_fused_decode_waits_run_out_and_the_next_call_is_correct(T, entry):
     """The single-launch decode kernel's producer, consumers and grid barriers all give up
     after one cycle; every CTA leaves (its copies landed), the grid-barrier words are reset
     for the next launch, and the next call on the same workspace is correct.  A single
-    layer runs the fused kernel up to T = 3, a stack (here of one layer) up to T = 8."""
+    layer runs the fused kernel up to T = 3, a stack (here of one layer) up to T = 7."""
     lay, x, _ = workload(82 + T, T, FULL)
     L = moe.MoELayer.from_synth(lay)
     xd = to_dev_bits(x)
