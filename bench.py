@@ -88,6 +88,9 @@ def parse_args(argv=None):
     ap.add_argument("--gdn-only", action="store_true", help="only the recurrence measurement (profiling)")
     ap.add_argument("--gdn-B", type=str, default=",".join(str(n) for n in GDN_B))
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass (profiling)")
+    ap.add_argument("--e2e-streams", type=int, default=4,
+                    help="streams (each with its own workspace and output buffer) that consecutive "
+                         "host-buffer calls rotate over")
     ap.add_argument("--no-stages", action="store_true", help="skip the per-stage traced pass (profiling)")
     ap.add_argument("--layers", type=int, default=4, help="prefill layers cycled")
     ap.add_argument("--decode-layers", type=int, default=40, help="resident layers of the decode and sweep stacks")
@@ -364,13 +367,18 @@ def prefill_phase(a, world, rank, dev, dims, zipf, peaks, peak_src, e2e: bool):
         for i in range(2):
             step_host(i)
         sync_ms = timed_loop(step_host, a.steps, world)
-        # streaming use: consecutive calls alternate two streams (each with its
+        # streaming use: consecutive calls rotate over S streams (each with its
         # own workspace and output buffer), so one call's host<->device copies
-        # overlap the other's kernels; every step still copies its x in and
-        # its result out inside the timed region
-        ws2 = [ws, moe.alloc_workspace(layers[0], T_PREFILL, dev)]
-        oh2 = [oh, torch.empty_like(oh).pin_memory()]
-        streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+        # overlap the others' kernels; every step still copies its x in and
+        # its result out inside the timed region.  One stream runs its call's
+        # copy in, layer and copy out in order (~0.33 + 0.43 + 0.33 ms at
+        # T=4096), so S = 2 holds a step to about half of that chain; from
+        # S = 3 the copies hide behind the kernels (S = 1, 2, 3, 4, 6: 1.06,
+        # 0.578, 0.459, 0.450, 0.459 ms per step against 0.425 device-only).
+        S = max(1, a.e2e_streams)
+        ws2 = [ws] + [moe.alloc_workspace(layers[0], T_PREFILL, dev) for _ in range(S - 1)]
+        oh2 = [oh] + [torch.empty_like(oh).pin_memory() for _ in range(S - 1)]
+        streams = [torch.cuda.Stream() for _ in range(S)]
 
         def run_pipelined(n):
             cur = torch.cuda.current_stream()
@@ -380,7 +388,7 @@ def prefill_phase(a, world, rank, dev, dims, zipf, peaks, peak_src, e2e: bool):
             for st in streams:
                 st.wait_stream(cur)
             for i in range(n):
-                moe.moe_forward_host_async(layers[i % NL], xh[i % NL], oh2[i % 2], ws2[i % 2], stream=streams[i % 2])
+                moe.moe_forward_host_async(layers[i % NL], xh[i % NL], oh2[i % S], ws2[i % S], stream=streams[i % S])
             for st in streams:
                 cur.wait_stream(st)
             stop.record(cur)
@@ -393,7 +401,7 @@ def prefill_phase(a, world, rank, dev, dims, zipf, peaks, peak_src, e2e: bool):
             assert moe.moe_get_status(w_) == 0
         res["e2e"] = {"value": round(whole_job_rate(T_PREFILL * a.steps, world, e2e_ms), 1), "unit": "tokens/s",
                       "h2d_bytes_per_step": T_PREFILL * dims.H * 2, "d2h_bytes_per_step": T_PREFILL * dims.H * 2,
-                      "how": "moe_forward_host_async, two streams alternating (copies overlap kernels)",
+                      "how": f"moe_forward_host_async, {S} streams in rotation (copies overlap kernels)",
                       "blocking_call_value": round(whole_job_rate(T_PREFILL * a.steps, world, sync_ms), 1)}
     del layers, xs
     torch.cuda.empty_cache()

@@ -277,8 +277,10 @@ MOE_API int moe_forward_host(const moe_layer_desc* layer, const moe_bf16* x_host
  * workspace, the layer and the copy of the result to out_host on `stream` and
  * returns.  out_host is valid once the stream reaches that point; x_host must
  * stay unchanged until then.  With page-locked buffers the copies are
- * asynchronous, so a caller that alternates two streams (each with its own
- * workspace) overlaps one call's copies with another call's kernels. */
+ * asynchronous, so a caller that rotates over a few streams (each with its
+ * own workspace and output buffer) overlaps one call's copies with the other
+ * calls' kernels: one stream runs its copy in, layer and copy out in order,
+ * so with large T three streams are needed to hide both copies. */
 MOE_API int moe_forward_host_async(const moe_layer_desc* layer, const moe_bf16* x_host, int T, moe_bf16* out_host,
                                    void* workspace, size_t workspace_bytes, moe_stream stream);
 
