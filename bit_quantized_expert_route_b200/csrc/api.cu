@@ -392,8 +392,8 @@ int check_call(const moe_layer_desc* d, const void* x, int T, int T_limit, const
 // the library (a CUDA __device__ variable exists on every device of the
 // context), so callers that cannot allocate need not pass a workspace.
 constexpr size_t kRouteStaticBytes = 512u * 1024u;
-// moe.h states the scratch limit with 128-token segments and 128-row chunks.
-static_assert(moe::kGemmChunkRows == 128 && moe::kRouteSegTokens == 128,
+// moe.h states the scratch limit with 128-token segments and 160-row chunks.
+static_assert(moe::kGemmChunkRows == 160 && moe::kRouteSegTokens == 128,
               "update moe_route_static's documented limit");
 static __device__ __align__(256) unsigned char g_route_static_scratch[kRouteStaticBytes];
 

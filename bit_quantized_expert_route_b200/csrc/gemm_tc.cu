@@ -49,10 +49,10 @@ namespace moe {
 namespace {
 
 constexpr int BM = 128;          // weight rows per tile = TMEM lanes (MMA M)
-constexpr int BN = 128;          // rows (tokens) per chunk: MMA N <= 128
+constexpr int BN = 160;          // rows (tokens) per chunk: MMA N <= 160
 constexpr int BK = 64;           // inputs per stage: one quantisation group
-constexpr int kBStagesMax = 6;   // token-tile ring
-constexpr int kPStagesMax = 8;   // packed-tile ring
+constexpr int kBStagesMax = 5;   // token-tile ring
+constexpr int kPStagesMax = 7;   // packed-tile ring
 constexpr int kSBlock = 8;       // quantisation groups per scale block (16 B per row)
 constexpr int kDqWarps = 16;     // dequantiser warps (4 sets of 4: one per TMEM lane quadrant)
 constexpr int kEpiWarp0 = kDqWarps;
@@ -62,6 +62,9 @@ constexpr int kMmaWarp = kTmaWarp + 1;
 constexpr int kThreads = (kMmaWarp + 1) * 32;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxCtaUnits = 256;   // chunk descriptors cached in shared memory per CTA
+// token-tile box heights: a chunk loads the smallest box that covers its rows
+constexpr int kTokenBoxes = 5;
+__device__ __host__ constexpr int token_box(int i) { return i == 4 ? BN : 16 << i; }
 
 // kNA: 128-row weight tiles per stage.  gate/up: 2 (the gate and up
 // matrices, same rows); down: 2 (two consecutive 128-row blocks of the same
@@ -75,7 +78,7 @@ struct Cfg {
   static constexpr int A_COLS = NA * BK / 2;                  // TMEM columns per A stage
   static constexpr int A_BASE = ACC_BUFS * ACC_COLS;
   static constexpr int A_STAGES = (static_cast<int>(kTmemCols) - A_BASE) / A_COLS;
-  static constexpr int B_BYTES = BN * BK * 2;                 // 16 KB swizzled token tile
+  static constexpr int B_BYTES = BN * BK * 2;                 // 20 KB swizzled token tile
   static constexpr int P_BYTES = BM * 32;                     // 4 KB packed tile of one matrix
   static constexpr int S_BYTES = BM * kSBlock * 2;            // 2 KB: 8 groups of scales (or biases)
   static constexpr int S_SLOT = NA * 2 * S_BYTES;             // scales + biases of every matrix
@@ -94,6 +97,7 @@ struct Cfg {
   static constexpr int BAR_OFF = OFF_OUT + OUT_BYTES;
   static constexpr int OFF_UNITS = BAR_OFF + 512;             // this CTA's chunk descriptors
   static constexpr int SMEM = OFF_UNITS + kMaxCtaUnits * 16 + 1024;   // + alignment slack
+  static_assert(SMEM <= 227 * 1024, "dynamic shared memory of one CTA");
   static constexpr int DQ_PER_STAGE = kNA * 128;             // dequant threads consuming one stage
 };
 
@@ -104,7 +108,7 @@ struct alignas(64) TcArgs {
   // token tiles: [gate/up: grouped x rows, - | down: routed h, shared h] x
   // box height [16, 32, 64, 128 rows]: a chunk loads the smallest box that
   // covers its rows (a 3-row expert group needs 2 KB per stage, not 16 KB)
-  CUtensorMap tm_h[2][4];
+  CUtensorMap tm_h[2][kTokenBoxes];
   Geometry g;
   QMatPtr W0, W1;          // routed stacks: {gate, up} or {down, -}
   QMatPtr S0, S1;          // shared expert: {sh_gate, sh_up} or {sh_down, -}
@@ -431,9 +435,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
         if (ui.skip) continue;
         // gate/up: rows of the grouped x (shared-expert rows follow the routed
         // ones); down: routed h or shared h
-        const int bsz = ui.rows <= 16 ? 0 : ui.rows <= 32 ? 1 : ui.rows <= 64 ? 2 : 3;
+        int bsz = 0;
+        while (bsz < kTokenBoxes - 1 && token_box(bsz) < ui.rows) ++bsz;
         const void* tm = &a.tm_h[(!kGateUp && ui.shared) ? 1 : 0][bsz];
-        const uint32_t bbytes = static_cast<uint32_t>(16 << bsz) * BK * 2;   // rows x 64 inputs x bf16
+        const uint32_t bbytes = static_cast<uint32_t>(token_box(bsz)) * BK * 2;   // rows x 64 inputs x bf16
         const int y = (!kGateUp && ui.shared) ? ui.row0 - Tk : ui.row0;
         for (int ks = 0; ks < ui.nks; ++ks, ++it) {
           const int s = static_cast<int>(it % C::BST);
@@ -574,11 +579,12 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* bas
   return make_tmap_2d(m, dt, esize, base, cols, rows, box_cols, box_rows, sw);
 }
 
-// Token-tile maps of a bf16 [rows, K] matrix: 64-input boxes of 16, 32, 64
-// and 128 rows, 128-byte swizzle (K-major, the UMMA B layout).
-bool make_token_maps(CUtensorMap (&m)[4], const void* base, int K, uint64_t rows) {
-  for (int i = 0; i < 4; ++i)
-    if (!make_map(&m[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, K, rows, BK, 16u << i, CU_TENSOR_MAP_SWIZZLE_128B))
+// Token-tile maps of a bf16 [rows, K] matrix: 64-input boxes of 16, 32, 64,
+// 128 and 160 rows, 128-byte swizzle (K-major, the UMMA B layout).
+bool make_token_maps(CUtensorMap (&m)[kTokenBoxes], const void* base, int K, uint64_t rows) {
+  for (int i = 0; i < kTokenBoxes; ++i)
+    if (!make_map(&m[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, K, rows, BK, static_cast<uint32_t>(token_box(i)),
+                  CU_TENSOR_MAP_SWIZZLE_128B))
       return false;
   return true;
 }
@@ -626,7 +632,7 @@ cudaError_t launch_gateup(const Geometry& g, const LayerPtr& L, const uint16_t* 
       !make_qmat_maps(a, 1, 0, L.sh_gate, g.Is, g.H) || !make_qmat_maps(a, 1, 1, L.sh_up, g.Is, g.H) ||
       !make_token_maps(a.tm_h[0], xg, g.H, rows))
     return cudaErrorInvalidValue;
-  for (int i = 0; i < 4; ++i) a.tm_h[1][i] = a.tm_h[0][i];
+  for (int i = 0; i < kTokenBoxes; ++i) a.tm_h[1][i] = a.tm_h[0][i];
   using C = Cfg<true, 2>;
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(grouped_gemm_tc_kernel<true, 2>), C::SMEM);
   if (e != cudaSuccess) return e;

@@ -107,7 +107,7 @@ cudaError_t launch_group(const int32_t* topk_idx, int T, int k, int E, int chunk
 // gemm_tc.cu: tcgen05 grouped expert GEMMs over the device chunk list.
 // Rows per chunk of the chunk list (the GEMM tile's token count); moe.h states
 // moe_route_static's scratch limit with this value.
-constexpr int kGemmChunkRows = 128;
+constexpr int kGemmChunkRows = 160;
 int gemm_chunk_rows();
 // xg: the grouped token rows [T*k + T, H] (routed rows in expert order, then
 // the shared expert's T rows), each group of 8 in the interleaved K order.

@@ -246,11 +246,11 @@ MOE_API int moe_forward_stack(const moe_layer_desc* layers, int n_layers, const 
  * which every GPU that loads the library holds until the process exits.
  *   Limit: the call needs 256 bytes of control block, plus for T <= 64
  *   T*(E+1)*4 bytes of logits, or for T > 64 ceil(T/128)*E*4 bytes of counts
- *   and (T*k/128 + T/128 + E + 2)*16 + 4 bytes of chunk list, plus
+ *   and (T*k/160 + T/160 + E + 2)*16 + 4 bytes of chunk list, plus
  *   (E+1)*4 + 4 bytes of active list, plus T*4 bytes if r->sigma is NULL,
  *   each piece rounded up to 256 bytes; a call whose need exceeds 512 KiB
  *   returns MOE_ERR_WORKSPACE and enqueues nothing (for E=256, k=8 this
- *   admits T <= 56704 when r->sigma is given, T <= 39424 when it is NULL).
+ *   admits T <= 58112 when r->sigma is given, T <= 40099 when it is NULL).
  *   Set-up: the first call on each device looks up the array's device
  *   address with cudaGetSymbolAddress while that device is current, so make
  *   that first call before any stream capture on that device.

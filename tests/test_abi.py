@@ -167,24 +167,25 @@ def test_library_is_built_for_sm100a():
     assert os.path.exists(moe_build.LIB)
 
 
-def _static_route_need(T, E, k, sigma_given, chunk=128):
-    """Scratch bytes of moe_route_static as moe.h states them (each piece rounded to 256 B)."""
+def _static_route_need(T, E, k, sigma_given, seg=128, chunk=160):
+    """Scratch bytes of moe_route_static as moe.h states them (each piece rounded to 256 B):
+    per-segment counts of 128-token segments, a chunk list of <= 160-row chunks."""
     r = lambda b: (b + 255) // 256 * 256
     n = 256
     if T <= 64:
         n += r(T * (E + 1) * 4)
     else:
-        n += r(-(-T // chunk) * E * 4) + r((T * k // chunk + T // chunk + E + 2) * 16) + r(4)
+        n += r(-(-T // seg) * E * 4) + r((T * k // chunk + T // chunk + E + 2) * 16) + r(4)
     n += r((E + 1) * 4) + r(4)
     return n + (0 if sigma_given else r(T * 4))
 
 
 def test_static_route_limits(lib):
-    """moe_route_static admits T <= 56704 (sigma given) / 39424 (sigma NULL) for E=256, k=8,
+    """moe_route_static admits T <= 58112 (sigma given) / 40099 (sigma NULL) for E=256, k=8,
     and rejects the next T on the host with MOE_ERR_WORKSPACE before any CUDA call.
     (Only the rejecting side is called: an accepted call would launch kernels.)"""
     L = fake_layer()
-    for sigma, limit in ((FAKE, 56704), (None, 39424)):
+    for sigma, limit in ((FAKE, 58112), (None, 40099)):
         assert _static_route_need(limit, 256, 8, sigma is not None) <= 512 * 1024
         assert _static_route_need(limit + 1, 256, 8, sigma is not None) > 512 * 1024
         r = moe.RoutingC(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, sigma)
