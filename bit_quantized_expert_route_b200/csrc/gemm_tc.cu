@@ -12,7 +12,7 @@
 //   warps rebuild bf16(scale * q + bias) and store the tile into tensor
 //   memory, where the MMA reads it as its A operand.  The dense tile never
 //   touches shared memory.
-// * The expert's tokens are the MMA's N dimension (16..128 per chunk), staged
+// * The expert's tokens are the MMA's N dimension (16..160 per chunk), staged
 //   in shared memory in the 128-byte swizzled K-major layout by one 2-D TMA
 //   per stage: the chunk's rows are contiguous (gate/up: a gather pass has
 //   written x's rows in grouped order; down: h is produced in that order).
@@ -27,18 +27,29 @@
 //   the tile out with coalesced 16-byte stores, overlapping the next unit.
 //
 // One persistent CTA per SM walks the device-built unit list
-//   unit = (chunk of <= 128 rows of one expert) x (block of 128 weight rows).
-// Warp roles (736 threads):
+//   unit = (chunk of <= 160 rows of one expert) x (block of 128 weight rows).
+// Warp roles (864 threads):
 //   warps 0-15  dequantisers in 4 sets of 4 (gate/up: set = stage parity x
 //               matrix; down: set = stage mod 4); TMEM lane quadrant =
 //               warp % 4 = row / 32
-//   warps 16-19 epilogue (lane quadrant = warp % 4)
-//   warp 20     token tiles: one lane issues a 2-D TMA per stage
-//   warp 21     one lane issues the TMA loads of packed tiles and scales
-//   warp 22     tensor-memory allocation; one lane issues tcgen05.mma
+//   warps 16-23 epilogue, two per lane quadrant (warp % 4), taking alternate
+//               16-column blocks of the accumulators
+//   warp 24     token tiles: one lane issues a 2-D TMA per stage
+//   warp 25     one lane issues the TMA loads of packed tiles and scales
+//   warp 26     tensor-memory allocation; one lane issues tcgen05.mma
 // Tensor memory (512 columns): gate/up = one accumulator pair (gate, up:
-// 2 x 128 columns) + 4 A stages of 64 columns; down = two accumulators of 128
-// columns (double-buffered) + 8 A stages of 32 columns.
+// 2 x 160 columns) + 3 A stages of 64 columns; down with two weight blocks
+// per unit = two accumulators of 160 columns + 3 A stages of 64 columns;
+// down with one block = a double-buffered 160-column accumulator + 6 A
+// stages of 32 columns.
+//
+// Why chunks of up to 160 rows: a unit costs about the same whatever its N
+// (the per-stage hand-offs between the roles, not the MMAs, set its length),
+// so the number of units sets the kernel time.  With 128-row chunks an
+// expert that receives a few more than 128 tokens (about half of them with
+// uniform routing at T = 4096) paid for a second, nearly empty unit; 160 is
+// the most tensor memory allows while keeping three A stages beside the
+// gate/up accumulators.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -56,7 +67,8 @@ constexpr int kPStagesMax = 7;   // packed-tile ring
 constexpr int kSBlock = 8;       // quantisation groups per scale block (16 B per row)
 constexpr int kDqWarps = 16;     // dequantiser warps (4 sets of 4: one per TMEM lane quadrant)
 constexpr int kEpiWarp0 = kDqWarps;
-constexpr int kLoadWarp = kEpiWarp0 + 4;   // token tiles
+constexpr int kEpiWarps = 8;      // two per TMEM lane quadrant, alternate 16-column blocks
+constexpr int kLoadWarp = kEpiWarp0 + kEpiWarps;   // token tiles
 constexpr int kTmaWarp = kLoadWarp + 1;
 constexpr int kMmaWarp = kTmaWarp + 1;
 constexpr int kThreads = (kMmaWarp + 1) * 32;
@@ -106,7 +118,7 @@ struct alignas(64) TcArgs {
   CUtensorMap tm_s[2][2];  // scales:       [routed, shared][matrix] (valid when scales_tma)
   CUtensorMap tm_b[2][2];  // biases
   // token tiles: [gate/up: grouped x rows, - | down: routed h, shared h] x
-  // box height [16, 32, 64, 128 rows]: a chunk loads the smallest box that
+  // box height [16, 32, 64, 128, 160 rows]: a chunk loads the smallest box that
   // covers its rows (a 3-row expert group needs 2 KB per stage, not 16 KB)
   CUtensorMap tm_h[2][kTokenBoxes];
   Geometry g;
@@ -227,11 +239,11 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
     }
     for (int b = 0; b < C::ACC_BUFS; ++b) {
       tc::mbar_init(&acc_full[b], 1);
-      tc::mbar_init(&acc_empty[b], 128);
+      tc::mbar_init(&acc_empty[b], kEpiWarps * 32);
     }
     tc::mbar_init(drain, 1);
-    tc::mbar_init(&epi_sync[0], 128);
-    tc::mbar_init(&epi_sync[1], 128);
+    tc::mbar_init(&epi_sync[0], kEpiWarps * 32);
+    tc::mbar_init(&epi_sync[1], kEpiWarps * 32);
     *abort_flag = 0;
     tc::fence_barrier_init();
   }
@@ -352,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
     const int q = warp & 3;
     const int r = q * 32 + lane;                     // weight row == TMEM lane == output feature in tile
     const int rpos = kGateUp ? tc::k8_pos(r) : r;    // h is stored in the K order of the down GEMM
-    const int et = threadIdx.x - kEpiWarp0 * 32;     // 0..127
+    const int et = threadIdx.x - kEpiWarp0 * 32;     // 0 .. kEpiWarps * 32 - 1
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
     uint16_t* stage = reinterpret_cast<uint16_t*>(smem + C::OFF_OUT);   // [BN tokens][BM features]
     uint32_t tt = 0;
@@ -372,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
       bool ok = true;
       for (int mm = 0; mm < kRounds && ok; ++mm) {
         uint16_t* st = stage + (kAll ? mm * BN * BM : 0);
-        for (int n0 = 0; n0 < ui.rows; n0 += 16) {
+        for (int n0 = 16 * ((warp - kEpiWarp0) >> 2); n0 < ui.rows; n0 += 32) {
           float v0[16];
           tc::tmem_ld16(acc + mm * BN + n0, v0);
           if (kGateUp) {
@@ -406,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc_kernel(const __gr
         const int chunks = ui.rows * (BM / 8);
         for (int mo = kAll ? 0 : mm; mo <= mm; ++mo) {
           const uint16_t* so = stage + (kAll ? mo * BN * BM : 0);
-          for (int i = et; i < chunks; i += 128) {
+          for (int i = et; i < chunks; i += kEpiWarps * 32) {
             const int n = i / (BM / 8), c = i % (BM / 8);
             const int R = ui.row0 + n;
             uint16_t* dst;

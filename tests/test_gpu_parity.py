@@ -73,6 +73,20 @@ def test_degenerate_expert_counts(E, k, T):
     assert_output_close(gpu["out"], ref["out"])
 
 
+# Expert groups at the edges of the expert GEMMs' chunks of at most 160 rows:
+# with E = k = 8 every expert, and the shared expert, receives exactly T rows
+# (one full chunk, one full chunk plus a 1-row chunk, two full chunks, ...).
+@pytest.mark.parametrize("T", [159, 160, 161, 320, 321])
+def test_gemm_chunk_boundaries(T):
+    dims = dataclasses.replace(TINY, E=8, k=8)
+    lay, x, _ = workload(80 + T, T, dims)
+    ref = moe_ref.moe_layer(x, lay, 8)
+    gpu = run_layer(lay, x)
+    assert gpu["status"] == 0
+    assert_routing_exact(gpu, ref)
+    assert_output_close(gpu["out"], ref["out"])
+
+
 # Token counts at the edges of the router's 128-token tiles (one cluster each).
 @pytest.mark.parametrize("T", [127, 128, 129, 256])
 def test_router_tile_boundaries(T):
