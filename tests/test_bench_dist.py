@@ -69,3 +69,24 @@ def test_reference_arm_prints_once_under_two_ranks():
     line = json.loads(lines[0])
     assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_committed_traffic_needs_the_same_source_and_workload(tmp_path, monkeypatch):
+    """The roofline's `traffic` comes from a committed ncu summary only while the kernel's source
+    file is byte-identical to the one profiled, and only for the workload it was captured on."""
+    sys.path.insert(0, ROOT)
+    import hashlib
+    import bench
+    src = tmp_path / "k.cu"
+    src.write_text("__global__ void k() {}\n")
+    sha = hashlib.sha256(src.read_bytes()).hexdigest()[:16]
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "k.md").write_text(
+        f"traffic_bytes_per_launch: k<true> 1234 src_sha={sha} workload=wl_a\n"
+        f"traffic_bytes_per_launch: k<true> 999 src_sha=0000000000000000 workload=wl_b\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.committed_traffic("k<true>", "k.cu", "wl_a") == (1234, "wl_a")
+    assert bench.committed_traffic("k<true>", "k.cu", "wl_b") is None       # captured on an older source
+    assert bench.committed_traffic("k<false>", "k.cu", "wl_a") is None      # another kernel
+    src.write_text("__global__ void k() { /* changed */ }\n")
+    assert bench.committed_traffic("k<true>", "k.cu", "wl_a") is None       # source changed since
